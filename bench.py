@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA2 decode hot path on B200.
+
+One step = one call of the 20-layer decoder stack (csa2_layer_stack) over one
+batch of seeded synthetic inputs of the `stack20_128k` workload: 16 sequences x
+131072 cached positions, layers [Full, Reuse, Reuse, Reindex] x 5, pool 8192,
+top-k 2048, SWA 512, 16 heads x 128, indexer 8 x 64 int8. Inputs are resident in
+HBM; L2 is flushed (a 256 MB write) before every timed step, outside its events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own replica (its own sequences; the path
+shards by sequence with no collective) and rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode queries/s at 128K ctx (1 B200); achieved HBM GB/s vs peak"
+UNIT = "queries/s"
+DEFAULT_WORKLOAD = "stack20_128k"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--kernel-launches", type=int, default=50)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ accounting
+def unit_bytes(spec):
+    """Algorithmic bytes one query moves through the whole stack (each distinct row
+    once per kernel call): index keys scanned or gathered, pool/list indices, FP4
+    rows gathered (D/2 + D/16 bytes), local K+V rows, queries and outputs."""
+    D, Di, Hi, Hq = spec.D, spec.Di, spec.Hi, spec.Hq
+    t = spec.N - 1
+    total = 0
+    k_cur, pool_P = 0, 0
+    for L in spec.layers:
+        if L.mode == "FULL":
+            total += (t + 1) * Di + Hi * Di + (L.P + L.k) * 4
+            k_cur = L.k
+            pool_P = L.P or pool_P
+        elif L.mode == "REINDEX":
+            total += pool_P * (Di + 4) + Hi * Di + L.k * 4
+            k_cur = L.k
+        total += k_cur * (D // 2 + D // 16 + 4) + min(spec.W, t + 1) * 2 * D * 2 + 2 * Hq * D * 2
+    return total
+
+
+def full_launch_bytes(spec, units):
+    L = spec.layers[0]
+    return units * (spec.N * spec.Di + spec.Hi * spec.Di + (L.P + L.k) * 4)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:  # noqa: BLE001
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:  # noqa: BLE001
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ our arm
+def build_device_stack(wl, torch, ops, np):
+    s = wl.spec
+
+    def dev(a, dtype=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(dtype) if dtype is not None else t).cuda()
+
+    q_pos, base = dev(wl.q_pos()), dev(wl.local_base_arr())
+    kv = dev(wl.kv_f32())
+    codes, scales = ops.fp4_quantize(kv.view(-1, s.D))
+    del kv
+    wl.drop("kv")
+    codes, scales = codes.view(s.B, s.N, -1), scales.view(s.B, s.N, -1)
+    keys = {}
+    layers = []
+    for li, L in enumerate(s.layers):
+        d = {"mode": L.mode, "q": dev(wl.q(li).view(np.int16), torch.bfloat16),
+             "kl": dev(wl.kl(li).view(np.int16), torch.bfloat16),
+             "vl": dev(wl.vl(li).view(np.int16), torch.bfloat16), "W": s.W}
+        if L.mode != "REUSE":
+            if L.key_set not in keys:
+                keys[L.key_set] = dev(wl.ki(L.key_set))
+                wl.drop(("ki", L.key_set))
+            d.update(qi=dev(wl.qi(li)), w=wl.w(li), ki=keys[L.key_set], k=L.k, P=L.P)
+        layers.append(d)
+    stack = ops.LayerStack(layers, q_pos, codes, scales, base)
+    return stack, layers, q_pos, codes, scales, base
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import synth
+    from sparse_attention_shared_b200 import capi, ops
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    wl = synth.make_workload(args.workload, seed=rank)
+    s = wl.spec
+    units = s.B * s.Tq
+    stack, layers, q_pos, codes, scales, base = build_device_stack(wl, torch, ops, np)
+    ws, st = ops.Workspace(), ops.Status()
+    buf = ws.get(stack.ws_bytes)
+    stream = torch.cuda.current_stream()
+    sptr = int(stream.cuda_stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        return stack.run_raw(int(buf.data_ptr()), buf.numel(), st.ptr, sptr)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        capi.check(step(), "warmup")
+    st.check("warmup")
+
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(local_rank)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(K):
+        flush.zero_()
+        ev0[i].record(stream)
+        rc = step()
+        ev1[i].record(stream)
+        if rc:
+            capi.check(rc, "timed step")
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    st.check("timed region")
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    total_ms = sum(step_ms)
+    tmax = torch.tensor([total_ms], device="cuda")
+    if dist:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    total_ms = float(tmax.item())
+    ms_per_step = total_ms / K
+    value = units * world * K / (total_ms / 1e3)
+    n_idx = sum(1 for L in s.layers if L.mode != "REUSE")
+    launches_per_step = n_idx + len(s.layers)
+
+    # dominant kernel: the Full-mode indexer of layer 0, alone, same stream, L2 flushed
+    d0 = layers[0]
+    import numpy as _np
+    w_host = _np.ascontiguousarray(_np.asarray(d0["w"], dtype=_np.int32))
+    pool_t = torch.empty((s.B, s.Tq, s.layers[0].P), dtype=torch.int32, device="cuda")
+    topk_t = torch.empty((s.B, s.Tq, s.layers[0].k), dtype=torch.int32, device="cuda")
+    ia = ops.make_index_args(capi.CSA2_FULL, q_pos, d0["qi"], w_host, d0["ki"], s.layers[0].k, s.layers[0].P,
+                             None, pool_t, topk_t)
+    ibuf = ws.get(max(stack.ws_bytes, capi.csa2_workspace_bytes(0, ia)))
+    kl_ms = []
+    for i in range(args.kernel_launches + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        capi.check(capi.csa2_index_topk(ia, int(ibuf.data_ptr()), ibuf.numel(), st.ptr, sptr), "kernel timing")
+        b.record(stream)
+        if i >= 3:
+            kl_ms.append((a, b))
+    torch.cuda.synchronize()
+    st.check("kernel timing")
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kl_ms)
+    kbytes = full_launch_bytes(s, units)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:  # noqa: BLE001
+        pass
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    achieved = kbytes / (kern_ms * 1e-3) / 1e9
+    traffic = None
+    try:
+        prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        traffic = prof.get(args.workload, {}).get("index_full_bytes_per_launch")
+    except Exception:  # noqa: BLE001
+        pass
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                "kernel": "index_select_kernel<8,64> (Full mode, layer 0)",
+                "kernel_ms": round(kern_ms, 4), "algorithmic_bytes": kbytes,
+                "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback 6650 GB/s"}
+    step_bytes = unit_bytes(s) * units
+    step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, args.cpu_seconds)
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8+bf16", "data": "synthetic",
+        "config": {"workload": s.name, "B": s.B, "N": s.N, "layers": s.L, "schedule": "[F,U,U,RI]x5",
+                   "Hq": s.Hq, "D": s.D, "Hi": s.Hi, "Di": s.Di, "pool": s.layers[0].P, "k": s.layers[0].k,
+                   "W": s.W, "per_gpu_queries": units, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (256 MB write) before every timed step, outside its events"},
+        "step_hbm_gbs": round(step_gbs, 1), "step_frac_of_peak": round(step_gbs / hbm_peak, 4),
+        "algorithmic_bytes_per_step": step_bytes,
+        "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * K, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st):
+    """Per step: copy the step's per-query inputs (main queries of every layer, index
+    queries of Full/Reindex layers, query positions) from pinned host memory, run the
+    stack, and copy every layer's output and lse back to pinned host memory."""
+    dev_in = [q_pos] + [d["q"] for d in layers] + [d["qi"] for d in layers if d["mode"] != "REUSE"]
+    host_in = [t.cpu().pin_memory() for t in dev_in]
+    dev_out = list(stack.outs) + [x for x in stack.lses if x is not None]
+    host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in dev_out]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    ws = ops.Workspace()
+    buf = ws.get(stack.ws_bytes)
+    sptr = int(stream.cuda_stream)
+    K = max(10, args.steps // 5)
+    evs = []
+    for i in range(K + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        capi.check(stack.run_raw(int(buf.data_ptr()), buf.numel(), st.ptr, sptr), "e2e step")
+        for h, d in zip(host_out, dev_out):
+            h.copy_(d, non_blocking=True)
+        b.record(stream)
+        if i >= 3:
+            evs.append((a, b))
+    torch.cuda.synchronize()
+    st.check("e2e")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    units = s.B * s.Tq
+    return {"value": round(units / (ms * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 5), "steps": K}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def cpu_baseline(workload: str, seconds: float):
+    """The oracle, as it stands, on whole queries (all 20 layers) of the same workload
+    until `seconds` of CPU work have run (at least one query)."""
+    import synth
+    from oracle.workload import OracleCache, layer_inputs, run_units
+    from oracle import csa2_oracle as O
+
+    wl = synth.make_workload(workload)
+    s = wl.spec
+    cache = OracleCache(wl)
+    cache.seq(0)                           # quantising the cache is setup, not a decode step
+    done, t0 = 0, time.perf_counter()
+    while True:
+        run_units(wl, [(0, done % s.Tq)], cache)
+        done += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    return {"value": round(done / el, 4), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done} queries of sequence 0 through all {s.L} layers ({el:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is one layer of one query (cycling
+    through the schedule), reported as whole-stack queries/s."""
+    if rank != 0:
+        return
+    import synth
+    from oracle import csa2_oracle as O
+    from oracle.workload import OracleCache, layer_inputs
+
+    wl = synth.make_workload(args.workload)
+    s = wl.spec
+    cache = OracleCache(wl)
+    codes, scales = cache.seq(0)
+    layers = layer_inputs(wl, 0, 0)
+    t = int(wl.q_pos()[0, 0])
+    base = int(wl.local_base_arr()[0])
+    state = {"cur": None, "pool": None}
+
+    def layer_step(li):
+        L = layers[li]
+        if L["mode"] == "FULL":
+            pool, state["cur"] = O.index_full(L["qi"], L["w"], L["keys"], t, L["k"], L["P"])
+            if pool is not None:
+                state["pool"] = pool
+        elif L["mode"] == "REINDEX":
+            state["cur"] = O.index_reindex(L["qi"], L["w"], L["keys"], state["pool"], L["k"])
+        O.attention_unit(L["q"], codes, scales, state["cur"], L["kl"], L["vl"], base, t, L["W"])
+
+    for i in range(args.warmup):
+        layer_step(i % s.L)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        layer_step((args.warmup + i) % s.L)
+    el = time.perf_counter() - t0
+    value = args.steps / s.L / el
+    res = {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": s.name, "B": s.B, "N": s.N, "layers": s.L},
+           "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                            "sample": f"{args.steps} layer-steps of query (0,0), one layer per step"},
+           "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,105 @@
+"""The C-ABI library without a GPU: it builds for sm_100a, loads, exports every
+entry point that include/csa2.h declares, and rejects bad arguments on the host
+before launching anything."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from sparse_attention_shared_b200 import capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(csa2_\w+)\s*\(", txt))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = capi.lib()
+    declared = _declared()
+    assert {"csa2_index_topk", "csa2_sparse_attn", "csa2_layer_stack", "csa2_fp4_quantize",
+            "csa2_workspace_bytes", "csa2_status_string"} <= declared
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for code in range(10):
+        assert capi.csa2_status_string(code)
+
+
+def _index_args(**kw):
+    a = capi.IndexArgs()
+    a.B, a.Tq, a.N, a.Hi, a.Di, a.k, a.P, a.mode = 1, 1, 1024, 8, 64, 16, 64, capi.CSA2_FULL
+    fake = 1 << 20       # aligned, never dereferenced: validation fails or no workspace is given
+    w = np.ones(8, np.int32)
+    a.q_pos = a.qi = a.ki = a.topk_out = a.pool_out = fake
+    a.w = w.ctypes.data
+    a.ki_seq_stride = 1024 * 64
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a, w
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("q_pos", 0, 1), ("Hi", 17, 2), ("Di", 24, 2), ("k", 0, 2), ("k", 65, 2), ("N", 1 << 27, 2),
+    ("ki_seq_stride", 1000, 3), ("qi", (1 << 20) + 4, 3), ("mode", 2, 4), ("pool_out", 0, 1),
+])
+def test_index_validation(field, value, code):
+    a, _w = _index_args(**{field: value})
+    assert capi.csa2_index_topk(a, 0, 0, 0, 0) == code
+
+
+def test_index_weight_bound_and_workspace():
+    a, w = _index_args()
+    w[:] = 300                                   # 8 * 300 * 64 * 16384 >= 2^31
+    assert capi.csa2_index_topk(a, 0, 0, 0, 0) == 5
+    a, w = _index_args()
+    assert capi.csa2_workspace_bytes(0, a) > 0
+    assert capi.csa2_index_topk(a, 0, 0, 0, 0) == 9          # no workspace
+
+
+def test_attn_validation():
+    a = capi.AttnArgs()
+    a.B, a.Tq, a.N, a.Hq, a.D, a.k, a.W, a.Lloc = 1, 1, 1024, 16, 128, 64, 128, 128
+    fake = 1 << 20
+    a.q_pos = a.q = a.kv_fp4 = a.kv_scale = a.topk = a.kl = a.vl = a.local_base = a.out = fake
+    assert capi.csa2_workspace_bytes(1, a) > 0
+    assert capi.csa2_sparse_attn(a, 0, 0, 0, 0) == 9
+    a.D = 96
+    assert capi.csa2_sparse_attn(a, 0, 0, 0, 0) == 6
+    a.D, a.Hq = 128, 33
+    assert capi.csa2_sparse_attn(a, 0, 0, 0, 0) == 6
+    a.Hq, a.kl = 16, 0
+    assert capi.csa2_sparse_attn(a, 0, 0, 0, 0) == 1
+
+
+def test_stack_mode_order():
+    ia, _w = _index_args()
+    aa = capi.AttnArgs()
+    aa.B, aa.Tq, aa.N, aa.Hq, aa.D, aa.W = 1, 1, 1024, 16, 128, 0
+    aa.q_pos = aa.q = aa.kv_fp4 = aa.kv_scale = aa.out = 1 << 20
+    reuse = capi.IndexArgs()
+    reuse.mode = capi.CSA2_REUSE
+    idx = (capi.IndexArgs * 2)(reuse, ia)
+    att = (capi.AttnArgs * 2)(aa, aa)
+    assert capi.csa2_layer_stack(capi.StackArgs(2, idx, att), 0, 0, 0, 0) == 4
+    idx = (capi.IndexArgs * 2)(ia, reuse)
+    s = capi.StackArgs(2, idx, att)
+    assert capi.csa2_workspace_bytes(2, s) > 0
+    assert capi.csa2_layer_stack(s, 0, 0, 0, 0) == 9
+    ri = capi.IndexArgs.from_buffer_copy(ia)
+    ri.mode = capi.CSA2_REINDEX
+    ia0 = capi.IndexArgs.from_buffer_copy(ia)
+    ia0.P = 0
+    idx = (capi.IndexArgs * 2)(ia0, ri)          # REINDEX without a pool
+    assert capi.csa2_layer_stack(capi.StackArgs(2, idx, att), 0, 0, 0, 0) == 4

@@ -1,0 +1,291 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Index lists must be bit-exact; attention outputs within 3e-3 (max abs) of the
+fp64 oracle and lse within 1e-3. Sizes span several tiles, ragged tails,
+adversarial ties and the degenerate cases (W = 0, k = 1, early positions)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import csa2_oracle as O
+from oracle.workload import OracleCache, run_units
+from sparse_attention_shared_b200 import ops
+
+from gpu_util import DeviceWorkload, assert_attn_close, assert_lists_equal, bf16_dev, dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ws():
+    return ops.Workspace()
+
+
+@pytest.fixture
+def status():
+    s = ops.Status()
+    yield s
+    s.check("after test")
+
+
+# ---------------------------------------------------------------- FP4 codec
+def test_fp4_quantize_bit_exact():
+    x = synth.normal_f32(0, 77, (4096, 128))
+    rng = np.random.default_rng(0)
+    special = np.zeros((8, 128), np.float32)
+    special[1] = 1e-6                                      # scale rounds to zero
+    special[2] = rng.standard_normal(128) * 1000           # saturating scale
+    e4 = torch.arange(1, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    for r in range(3, 8):                                   # grid values and exact E2M1 midpoints
+        s = e4[rng.integers(0, len(e4), 8)].repeat(16)
+        m = np.array([0, .25, .5, .75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6, -6], np.float32)
+        special[r] = (m[rng.integers(0, 16, 128)] * s * rng.choice([-1, 1], 128)).astype(np.float32)
+        special[r, ::16] = 6 * s[::16]
+    x = np.concatenate([x, special])
+    codes, scales = ops.fp4_quantize(dev(x))
+    rc, rs = O.fp4_quantize(x)
+    assert_lists_equal(scales, rs, "scales")
+    assert_lists_equal(codes, rc, "codes")
+
+
+# ---------------------------------------------------------------- indexer
+def _oracle_full(qi, w, ki, q_pos, k, P):
+    B, Tq = q_pos.shape
+    pools = np.full((B, Tq, max(P, 1)), -1, np.int32)
+    topk = np.full((B, Tq, k), -1, np.int32)
+    for b in range(B):
+        for j in range(Tq):
+            p, t = O.index_full(qi[b, j], w, ki[b], int(q_pos[b, j]), k, P)
+            topk[b, j] = t
+            if P:
+                pools[b, j] = p
+    return (pools if P else None), topk
+
+
+def _check_full(qi, w, ki, q_pos, k, P, ws, status):
+    pool, topk = ops.index_topk("FULL", dev(q_pos), dev(qi), w, dev(ki), k, P, ws=ws, status=status)
+    rpool, rtopk = _oracle_full(qi, w, ki, q_pos, k, P)
+    assert_lists_equal(topk, rtopk, "topk")
+    if P:
+        assert_lists_equal(pool, rpool, "pool")
+    return pool, topk
+
+
+def test_index_full_tiny(ws, status):
+    wl = synth.make_workload("tiny")
+    for P in (0, 512):
+        _check_full(wl.qi(0), wl.w(0), wl.ki(0), wl.q_pos(), 256, P, ws, status)
+
+
+@pytest.mark.parametrize("B,N,Tq,k,P", [(4, 8192, 1, 2048, 4096), (3, 5000, 2, 300, 1000), (2, 20000, 1, 2048, 8192),
+                                        (1, 70001, 1, 2048, 8192), (40, 3000, 1, 100, 0)])
+def test_index_full_shapes(B, N, Tq, k, P, ws, status):
+    qi = synth.randint_i8(1, 10 + B, (B, Tq, 8, 64))
+    ki = synth.randint_i8(1, 20 + N, (B, N, 64))
+    w = synth.randint_i32(1, 30, (8,), 1, 8)
+    q_pos = np.broadcast_to(np.arange(N - Tq, N, dtype=np.int32), (B, Tq)).copy()
+    _check_full(qi, w, ki, q_pos, k, P, ws, status)
+
+
+def test_index_full_early_positions_and_padding(ws, status):
+    B, N = 2, 4096
+    qi = synth.randint_i8(2, 1, (B, 6, 8, 64))
+    ki = synth.randint_i8(2, 2, (B, N, 64))
+    w = synth.randint_i32(2, 3, (8,), 1, 8)
+    q_pos = np.array([[0, 1, 100, 300, 2047, 4095], [5, 255, 256, 257, 1000, 3000]], np.int32)
+    _check_full(qi, w, ki, q_pos, 300, 600, ws, status)
+
+
+@pytest.mark.parametrize("kind", ["all_equal", "relu_zero", "half_equal", "negative_w", "few_values"])
+def test_index_ties(kind, ws, status):
+    B, N, Tq = 2, 30000, 1
+    rng = np.random.default_rng(5)
+    qi = synth.randint_i8(3, 1, (B, Tq, 8, 64))
+    ki = synth.randint_i8(3, 2, (B, N, 64))
+    w = synth.randint_i32(3, 3, (8,), 1, 8)
+    if kind == "all_equal":
+        ki[:] = 5
+    elif kind == "relu_zero":
+        qi[:] = 100
+        ki[:] = -127
+    elif kind == "half_equal":
+        ki[:, ::2] = 7
+    elif kind == "negative_w":
+        w = -w
+    elif kind == "few_values":
+        ki[:] = rng.integers(-2, 3, ki.shape).astype(np.int8)
+        qi[:] = 1
+    q_pos = np.full((B, Tq), N - 1, np.int32)
+    _check_full(qi, w, ki, q_pos, 2048, 8192, ws, status)
+
+
+def test_index_reindex(ws, status):
+    B, N = 3, 12000
+    qi = synth.randint_i8(4, 1, (B, 1, 8, 64))
+    ki = synth.randint_i8(4, 2, (B, N, 64))
+    w = synth.randint_i32(4, 3, (8,), 1, 8)
+    q_pos = np.array([[N - 1], [N - 1], [3000]], np.int32)
+    pool, _ = _check_full(qi, w, ki, q_pos, 1024, 4096, ws, status)
+    qi2 = synth.randint_i8(4, 4, (B, 1, 8, 64))
+    ki2 = synth.randint_i8(4, 5, (B, N, 64))
+    w2 = synth.randint_i32(4, 6, (8,), 1, 8)
+    _, topk2 = ops.index_topk("REINDEX", dev(q_pos), dev(qi2), w2, dev(ki2), 1024, pool_in=pool, ws=ws, status=status)
+    rpool = pool.cpu().numpy()
+    ref = np.stack([[O.index_reindex(qi2[b, 0], w2, ki2[b], rpool[b, 0], 1024)] for b in range(B)])
+    assert_lists_equal(topk2, ref, "reindex topk")
+    for b in range(B):
+        got = set(topk2[b, 0].cpu().numpy().tolist()) - {-1}
+        assert got <= set(rpool[b, 0].tolist())
+
+
+def test_index_reindex_ties_small_pool(ws, status):
+    B, N = 2, 5000
+    qi = synth.randint_i8(6, 1, (B, 1, 4, 32))
+    ki = np.full((B, N, 32), 3, np.int8)
+    w = np.array([1, 2, 3, 4], np.int32)
+    q_pos = np.array([[N - 1], [200]], np.int32)
+    pool, _ = _check_full(qi, w, ki, q_pos, 100, 500, ws, status)
+    _, t2 = ops.index_topk("REINDEX", dev(q_pos), dev(qi), w, dev(ki), 100, pool_in=pool, ws=ws, status=status)
+    rp = pool.cpu().numpy()
+    ref = np.stack([[O.index_reindex(qi[b, 0], w, ki[b], rp[b, 0], 100)] for b in range(B)])
+    assert_lists_equal(t2, ref, "reindex ties")
+
+
+# ---------------------------------------------------------------- attention
+def _attn_case(B, N, Tq, Hq, D, k, W, seed, topk_fn=None, ws=None, status=None):
+    kv = synth.normal_f32(seed, 1, (B, N, D))
+    codes, scales = O.fp4_quantize(kv)
+    q = synth.normal_bf16(seed, 2, (B, Tq, Hq, D))
+    base = max(0, N - Tq - W + 1)
+    Lloc = N - base
+    kl = synth.normal_bf16(seed, 3, (B, max(Lloc, 1), D))
+    vl = synth.normal_bf16(seed, 4, (B, max(Lloc, 1), D))
+    q_pos = np.broadcast_to(np.arange(N - Tq, N, dtype=np.int32), (B, Tq)).copy()
+    rng = np.random.default_rng(seed)
+    topk = np.full((B, Tq, k), -1, np.int32)
+    for b in range(B):
+        for j in range(Tq):
+            t = q_pos[b, j]
+            sel = topk_fn(t, rng) if topk_fn else np.sort(rng.choice(t + 1, min(k, t + 1), replace=False))
+            topk[b, j, :len(sel)] = sel
+    gcodes, gscales = ops.fp4_quantize(dev(kv.reshape(-1, D)))
+    out, lse = ops.sparse_attn(dev(q_pos), bf16_dev(q), gcodes.view(B, N, D // 2), gscales.view(B, N, D // 16),
+                               dev(topk), bf16_dev(kl) if W else None, bf16_dev(vl) if W else None,
+                               dev(np.full((B,), base, np.int32)) if W else None, W, ws=ws, status=status)
+    ref_o = np.zeros((B, Tq, Hq, D))
+    ref_l = np.zeros((B, Tq, Hq))
+    for b in range(B):
+        klf, vlf = O.bf16_to_f64(kl[b]), O.bf16_to_f64(vl[b])
+        for j in range(Tq):
+            ref_o[b, j], ref_l[b, j] = O.attention_unit(O.bf16_to_f64(q[b, j]), codes[b], scales[b], topk[b, j],
+                                                       klf, vlf, base, int(q_pos[b, j]), W)
+    return assert_attn_close(out, lse, ref_o, ref_l, f"attn B{B} N{N} Tq{Tq} Hq{Hq} D{D} k{k} W{W}")
+
+
+def test_attention_tiny(ws, status):
+    wl = synth.make_workload("tiny")
+    dw = DeviceWorkload(wl)
+    s = wl.spec
+    _, topk = O.index_full(wl.qi(0)[0, 0], wl.w(0), wl.ki(0)[0], 2047, 256)
+    topks = np.stack([[O.index_full(wl.qi(0)[0, j], wl.w(0), wl.ki(0)[0], int(wl.q_pos()[0, j]), 256)[1]
+                       for j in range(s.Tq)]])
+    out, lse = ops.sparse_attn(dw.q_pos, bf16_dev(wl.q(0)), dw.kv_fp4, dw.kv_scale, dev(topks), bf16_dev(wl.kl(0)),
+                               bf16_dev(wl.vl(0)), dw.local_base, s.W, ws=ws, status=status)
+    res = run_units(wl, [(0, j) for j in range(s.Tq)])
+    ro = np.stack([[res[(0, j)][0]["out"] for j in range(s.Tq)]])
+    rl = np.stack([[res[(0, j)][0]["lse"] for j in range(s.Tq)]])
+    assert_lists_equal(dev(topks), np.stack([[res[(0, j)][0]["topk"] for j in range(s.Tq)]]), "oracle topk")
+    assert_attn_close(out, lse, ro, rl, "tiny attention")
+
+
+@pytest.mark.parametrize("B,N,Tq,Hq,D,k,W", [
+    (2, 4096, 1, 16, 128, 2048, 512),
+    (3, 3000, 2, 16, 128, 300, 200),     # ragged tiles on both branches
+    (2, 2500, 3, 32, 128, 256, 128),     # 32 heads (prefill shape)
+    (2, 2048, 2, 8, 64, 256, 128),       # D = 64, padded heads
+    (2, 4096, 1, 16, 128, 1, 0),         # single global entry, no window
+    (2, 4096, 1, 16, 128, 2048, 0),      # no local branch
+    (1, 300, 1, 16, 128, 512, 64),       # fewer positions than k: -1 padding
+])
+def test_attention_shapes(B, N, Tq, Hq, D, k, W, ws, status):
+    _attn_case(B, N, Tq, Hq, D, k, W, seed=B * 7 + N, ws=ws, status=status)
+
+
+def test_attention_overlap_window_and_global(ws, status):
+    """Positions in both the list and the window are counted twice."""
+    def sel(t, rng):
+        return np.arange(t - 63, t + 1)           # the last 64 positions, all inside the window
+    _attn_case(2, 2048, 1, 16, 128, 64, 128, seed=9, topk_fn=sel, ws=ws, status=status)
+
+
+def test_attention_reports_bad_positions(ws):
+    st = ops.Status()
+    B, N, D = 1, 512, 128
+    kv = synth.normal_f32(1, 1, (B * N, D))
+    c, s = ops.fp4_quantize(dev(kv))
+    topk = dev(np.array([[[0, 5, 700, -1]]], np.int32))      # 700 >= N
+    ops.sparse_attn(dev(np.array([[N - 1]], np.int32)), bf16_dev(synth.normal_bf16(1, 2, (B, 1, 16, D))),
+                    c.view(B, N, D // 2), s.view(B, N, D // 16), topk, None, None, None, 0, ws=ws, status=st)
+    code, _ = st.read()
+    assert code == 5   # CSA2_ERR_RANGE
+
+
+# ---------------------------------------------------------------- layer stack
+def _check_stack(wl, units, ws, status, keep_reuse=True):
+    dw = DeviceWorkload(wl)
+    st = ops.LayerStack(dw.layer_dicts(), dw.q_pos, dw.kv_fp4, dw.kv_scale, dw.local_base, keep_reuse_lists=keep_reuse)
+    st.run(ws, status)
+    torch.cuda.synchronize()
+    res = run_units(wl, units)
+    worst = 0.0
+    for (b, j), layers in res.items():
+        last_src = None
+        for li, r in enumerate(layers):
+            if st.topks[li] is not None:
+                assert_lists_equal(st.topks[li][b, j], r["topk"], f"layer {li} ({r['mode']}) topk unit {(b, j)}")
+            if st.pools[li] is not None:
+                assert_lists_equal(st.pools[li][b, j], r["pool"], f"layer {li} pool unit {(b, j)}")
+            if r["mode"] == "REUSE" and st.topks[li] is not None:
+                assert torch.equal(st.topks[li][b, j], st.topks[last_src][b, j])
+            if r["mode"] != "REUSE":
+                last_src = li
+            worst = max(worst, assert_attn_close(st.outs[li][b, j], st.lses[li][b, j], r["out"], r["lse"],
+                                                 f"layer {li} unit {(b, j)}"))
+    return worst
+
+
+def test_layer_stack_stack20_schedule_small(ws, status):
+    wl = synth.make_workload("stack20_128k", B=2, N=16384)
+    _check_stack(wl, [(0, 0), (1, 0)], ws, status)
+
+
+def test_layer_stack_long_schedule_small(ws, status):
+    wl = synth.make_workload("long_1m", N=40000, Tq=8)
+    _check_stack(wl, [(0, j) for j in range(8)], ws, status)
+
+
+def test_layer_stack_paper_schedule_small(ws, status):
+    wl = synth.make_workload("paper_schedule", B=3, N=9000)
+    _check_stack(wl, [(b, 0) for b in range(3)], ws, status)
+
+
+def test_layer_stack_rejects_bad_mode_order(ws):
+    wl = synth.make_workload("stack20_128k", B=1, N=4096)
+    dw = DeviceWorkload(wl)
+    layers = dw.layer_dicts()
+    with pytest.raises(ValueError):
+        ops.LayerStack([layers[1]] + layers[1:], dw.q_pos, dw.kv_fp4, dw.kv_scale, dw.local_base)   # REUSE first
+    with pytest.raises(ValueError):
+        ops.LayerStack([layers[3]], dw.q_pos, dw.kv_fp4, dw.kv_scale, dw.local_base)                # REINDEX first
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled
+def test_decode_full_sampled(ws, status):
+    wl = synth.make_workload("decode_full")
+    _check_stack(wl, [(0, 0), (17, 0), (31, 0)], ws, status, keep_reuse=False)
+
+
+def test_stack20_128k_sampled(ws, status):
+    wl = synth.make_workload("stack20_128k")
+    _check_stack(wl, [(0, 0), (15, 0)], ws, status, keep_reuse=False)
