@@ -29,7 +29,7 @@
  *     their 16-bit patterns (uint16_t).
  *   - The caller owns every buffer, including the workspace. The library never
  *     allocates device memory and keeps no per-call state outside the
- *     workspace. Calls are asynchronous on `stream` (a cudaStream_t; NULL =
+ *     workspace (csa2_sparse_attn_noalloc, at the end, uses a static array). Calls are asynchronous on `stream` (a cudaStream_t; NULL =
  *     the legacy default stream).
  *   - Arguments are validated on the host before anything is launched; on an
  *     error the call returns a status and launches nothing.
@@ -170,6 +170,20 @@ csa2_status csa2_layer_stack(const csa2_stack_args* args, void* workspace, size_
  *   x [rows, D] fp32, D % 16 == 0 -> fp4 [rows, D/2], scale [rows, D/16]. */
 csa2_status csa2_fp4_quantize(const float* x, int64_t rows, int32_t D, uint8_t* fp4,
                               uint8_t* scale, void* stream);
+
+/* Attention without a caller workspace, for callers that cannot allocate device
+ * memory: code running inside a host framework that owns every device allocation
+ * and forbids others, or a latency-critical decode loop that must not risk the
+ * device-wide synchronisation a cudaMalloc or cudaFree can cause. The pages have
+ * no counterpart: this is a deployment variant of csa2_sparse_attn, with the same
+ * arguments, results and errors, and no workspace.
+ * Scratch: a static 8 MiB device array per GPU (64 KiB of merge tickets, the rest
+ * for per-tile partials of 4 * (Hq<=16 ? 16 : 32) * (D + 2) bytes per 128-key
+ * tile and query). Calls needing more return CSA2_ERR_WORKSPACE and launch
+ * nothing. The first call on a device looks up that array's address (make it
+ * before any stream capture). Every call clears the tickets on `stream`; calls
+ * that overlap on the GPU share the array and race. */
+csa2_status csa2_sparse_attn_noalloc(const csa2_attn_args* args, int32_t* d_status, void* stream);
 
 /* Static text for a status code. */
 const char* csa2_status_string(csa2_status s);

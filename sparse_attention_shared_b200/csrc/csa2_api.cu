@@ -260,3 +260,63 @@ csa2_status csa2_fp4_quantize(const float* x, int64_t rows, int32_t D, uint8_t* 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// csa2_sparse_attn_noalloc: the attention call for callers that cannot allocate
+// device memory. Its scratch (merge tickets, then per-tile partials) lives in the
+// file-scope array below, which every GPU that loads this library holds until
+// the process exits. Host code must not use the array's name as an address: on
+// the host it is only a stand-in. The device address is looked up once per
+// device with cudaGetSymbolAddress, on the first call made with that device
+// current (so make that first call before any stream capture), and cached.
+// All calls share the array and it keeps the last call's contents: the tickets
+// are cleared on the stream before every launch, and two calls that overlap on
+// the GPU (other streams, other host threads) race on it.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace csa2 {
+constexpr size_t kStaticScratchBytes = (size_t)8 << 20;   // 8 MiB in total
+constexpr size_t kStaticTicketBytes = (size_t)64 << 10;   // tickets for up to 16384 queries
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+static std::mutex g_static_mu;
+static void* g_static_addr[kMaxDevices] = {nullptr};
+
+static csa2_status static_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return CSA2_ERR_CUDA;
+        g_static_addr[dev] = p;
+    }
+    *out = g_static_addr[dev];
+    return CSA2_OK;
+}
+}  // namespace csa2
+
+extern "C" csa2_status csa2_sparse_attn_noalloc(const csa2_attn_args* args, int32_t* d_status, void* stream) {
+    csa2_status st = check_attn(args, false);
+    if (st != CSA2_OK) return st;
+    const int units = args->B * args->Tq;
+    const size_t ticket_bytes = (size_t)units * sizeof(int);
+    if (ticket_bytes > kStaticTicketBytes || attn_scratch_bytes(*args) > kStaticScratchBytes - kStaticTicketBytes)
+        return CSA2_ERR_WORKSPACE;
+    void* base = nullptr;
+    st = static_scratch(&base);
+    if (st != CSA2_OK) return st;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    int* tickets = static_cast<int*>(base);
+    void* partials = static_cast<uint8_t*>(base) + kStaticTicketBytes;
+    if (cudaMemsetAsync(tickets, 0, ticket_bytes, strm) != cudaSuccess) return CSA2_ERR_CUDA;
+    csa2_attn_args a = *args;
+    if (a.W == 0) {
+        a.local_base = a.q_pos;
+        a.Lloc = 0;
+    }
+    return launch_attn(a, a.topk, tickets, partials, d_status, strm);
+}
