@@ -42,6 +42,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--kernel-launches", type=int, default=50)
+    ap.add_argument("--eager", action="store_true", help="launch directly instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -123,6 +124,30 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
+def capture_graph(torch, fn):
+    """Capture fn(stream_ptr) into a CUDA graph; None if capture is not possible."""
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            rc = fn(int(side.cuda_stream))            # one eager call to settle lazy init
+            if rc:
+                return None
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            rc = fn(int(torch.cuda.current_stream().cuda_stream))
+        if rc:
+            return None
+        torch.cuda.synchronize()
+        return g
+    except Exception as e:  # noqa: BLE001
+        print(f"graph capture failed, timing eager launches: {e}", file=sys.stderr)
+        torch.cuda.synchronize()
+        return None
+
+
 def build_device_stack(wl, torch, ops, np):
     s = wl.spec
 
@@ -176,8 +201,16 @@ def run_ours(args, rank, world, local_rank):
     sptr = int(stream.cuda_stream)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
+    def call(stream_ptr):
+        return stack.run_raw(int(buf.data_ptr()), buf.numel(), st.ptr, stream_ptr)
+
+    graph = None if args.eager else capture_graph(torch, call)
+
     def step():
-        return stack.run_raw(int(buf.data_ptr()), buf.numel(), st.ptr, sptr)
+        if graph is not None:
+            graph.replay()
+            return 0
+        return call(sptr)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -225,12 +258,20 @@ def run_ours(args, rank, world, local_rank):
     ia = ops.make_index_args(capi.CSA2_FULL, q_pos, d0["qi"], w_host, d0["ki"], s.layers[0].k, s.layers[0].P,
                              None, pool_t, topk_t)
     ibuf = ws.get(max(stack.ws_bytes, capi.csa2_workspace_bytes(0, ia)))
+
+    def kcall(stream_ptr):
+        return capi.csa2_index_topk(ia, int(ibuf.data_ptr()), ibuf.numel(), st.ptr, stream_ptr)
+
+    kgraph = None if args.eager else capture_graph(torch, kcall)
     kl_ms = []
     for i in range(args.kernel_launches + 3):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        capi.check(capi.csa2_index_topk(ia, int(ibuf.data_ptr()), ibuf.numel(), st.ptr, sptr), "kernel timing")
+        if kgraph is not None:
+            kgraph.replay()
+        else:
+            capi.check(kcall(sptr), "kernel timing")
         b.record(stream)
         if i >= 3:
             kl_ms.append((a, b))
@@ -262,7 +303,7 @@ def run_ours(args, rank, world, local_rank):
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st)
+        e2e = run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st, graph)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -275,7 +316,8 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": s.name, "B": s.B, "N": s.N, "layers": s.L, "schedule": "[F,U,U,RI]x5",
                    "Hq": s.Hq, "D": s.D, "Hi": s.Hi, "Di": s.Di, "pool": s.layers[0].P, "k": s.layers[0].k,
                    "W": s.W, "per_gpu_queries": units, "parallelism": f"replicas x{world}",
-                   "l2": "flushed (256 MB write) before every timed step, outside its events"},
+                   "l2": "flushed (256 MB write) before every timed step, outside its events",
+                   "launch": "CUDA graph of one csa2_layer_stack call" if graph is not None else "eager"},
         "step_hbm_gbs": round(step_gbs, 1), "step_frac_of_peak": round(step_gbs / hbm_peak, 4),
         "algorithmic_bytes_per_step": step_bytes,
         "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
@@ -288,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
-def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st):
+def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st, graph):
     """Per step: copy the step's per-query inputs (main queries of every layer, index
     queries of Full/Reindex layers, query positions) from pinned host memory, run the
     stack, and copy every layer's output and lse back to pinned host memory."""
@@ -301,6 +343,11 @@ def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, 
     ws = ops.Workspace()
     buf = ws.get(stack.ws_bytes)
     sptr = int(stream.cuda_stream)
+
+    def call(stream_ptr):
+        return stack.run_raw(int(buf.data_ptr()), buf.numel(), st.ptr, stream_ptr)
+
+    g2 = None if graph is None else capture_graph(torch, call)
     K = max(10, args.steps // 5)
     evs = []
     for i in range(K + 3):
@@ -309,7 +356,10 @@ def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, 
         a.record(stream)
         for d, h in zip(dev_in, host_in):
             d.copy_(h, non_blocking=True)
-        capi.check(stack.run_raw(int(buf.data_ptr()), buf.numel(), st.ptr, sptr), "e2e step")
+        if g2 is not None:
+            g2.replay()
+        else:
+            capi.check(call(sptr), "e2e step")
         for h, d in zip(host_out, dev_out):
             h.copy_(d, non_blocking=True)
         b.record(stream)

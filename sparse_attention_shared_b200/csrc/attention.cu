@@ -181,21 +181,35 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
         }
         const uint4* kls = reinterpret_cast<const uint4*>(p.kl);
         const uint4* vls = reinterpret_cast<const uint4*>(p.vl);
-        constexpr int CPR = D / 8;   // 16-byte chunks per row
-        for (int i = tid; i < kTileKeys * CPR; i += kAttnThreads) {
-            const int rr = i / CPR, c = i % CPR;
-            const int pr = p0 + rr;
-            const int lrow = pr - base;
-            const bool ok = (t >= 0) && (p.W > 0) && (pr <= t) && lrow >= 0 && lrow < p.Lloc;
-            uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-            if (ok) {
-                const size_t off = ((size_t)b * p.Lloc + lrow) * CPR + c;
-                kv = __ldg(kls + off);
-                vv = __ldg(vls + off);
+        constexpr int CPR = D / 8;                              // 16-byte chunks per row
+        constexpr int ITERS = kTileKeys * CPR / kAttnThreads;   // chunks per thread per tensor
+        constexpr int BATCH = ITERS < 8 ? ITERS : 8;            // loads in flight per tensor
+#pragma unroll
+        for (int i0 = 0; i0 < ITERS; i0 += BATCH) {
+            uint4 kv[BATCH], vv[BATCH];
+#pragma unroll
+            for (int j = 0; j < BATCH; ++j) {
+                const int i = tid + (i0 + j) * kAttnThreads;
+                const int rr = i / CPR, c = i % CPR;
+                const int pr = p0 + rr;
+                const int lrow = pr - base;
+                const bool ok = (t >= 0) && (p.W > 0) && (pr <= t) && lrow >= 0 && lrow < p.Lloc;
+                kv[j] = make_uint4(0, 0, 0, 0);
+                vv[j] = make_uint4(0, 0, 0, 0);
+                if (ok) {
+                    const size_t off = ((size_t)b * p.Lloc + lrow) * CPR + c;
+                    kv[j] = __ldg(kls + off);
+                    vv[j] = __ldg(vls + off);
+                }
             }
-            const uint32_t dst = (c >> 3) * kPanelBytes + sw128(rr, c & 7);
-            *reinterpret_cast<uint4*>(S.kbuf + dst) = kv;
-            *reinterpret_cast<uint4*>(S.vbuf + dst) = vv;
+#pragma unroll
+            for (int j = 0; j < BATCH; ++j) {
+                const int i = tid + (i0 + j) * kAttnThreads;
+                const int rr = i / CPR, c = i % CPR;
+                const uint32_t dst = (c >> 3) * kPanelBytes + sw128(rr, c & 7);
+                *reinterpret_cast<uint4*>(S.kbuf + dst) = kv[j];
+                *reinterpret_cast<uint4*>(S.vbuf + dst) = vv[j];
+            }
         }
     }
     fence_proxy_async_smem();
@@ -313,35 +327,70 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
         part[HQP * D + tid] = mv;
         part[HQP * D + HQP + tid] = lv;
     }
-    __threadfence();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) S.is_last = (atomicAdd(p.tickets + u, 1) == p.ntiles - 1);
+    if (tid == 0) {
+        __threadfence();
+        S.is_last = (atomicAdd(p.tickets + u, 1) == p.ntiles - 1);
+    }
     __syncthreads();
 
     if (S.is_last) {
+        // Merge the query's tile partials: weights exp2(m_s - M) / L per (tile, head)
+        // into shared memory, then every thread accumulates float4 slices of o.
         __threadfence();
         const float* pu = p.part + (size_t)u * p.ntiles * (HQP * (D + 2));
         const size_t stride = HQP * (D + 2);
-        for (int h = 0; h < p.Hq; ++h) {
+        const int nt = p.ntiles;
+        float* wgt = reinterpret_cast<float*>(S.kbuf);             // [nt][HQP]
+        float* Mh = reinterpret_cast<float*>(S.vbuf);              // [HQP]
+        float* Lh = Mh + HQP;                                      // [HQP]
+        float* lsum = reinterpret_cast<float*>(S.kbuf + kPanelBytes);   // [nt][HQP] tile sums
+        for (int i = tid; i < nt * HQP; i += kAttnThreads) {
+            const int s2 = i / HQP, h = i % HQP;
+            wgt[i] = __ldcg(pu + s2 * stride + HQP * D + h);
+            lsum[i] = __ldcg(pu + s2 * stride + HQP * D + HQP + h);
+        }
+        __syncthreads();
+        if (tid < HQP) {
             float M = -INFINITY;
-            for (int s = 0; s < p.ntiles; ++s) M = fmaxf(M, __ldcg(pu + s * stride + HQP * D + h));
-            float L = 0.f, acc = 0.f;
-            if (M != -INFINITY) {
-                for (int s = 0; s < p.ntiles; ++s) {
-                    const float ms = __ldcg(pu + s * stride + HQP * D + h);
-                    if (ms == -INFINITY) continue;
-                    const float wgt = exp2f(ms - M);
-                    L += wgt * __ldcg(pu + s * stride + HQP * D + HQP + h);
-                    if (tid < D) acc += wgt * __ldcg(pu + s * stride + h * D + tid);
+            for (int s2 = 0; s2 < nt; ++s2) M = fmaxf(M, wgt[s2 * HQP + tid]);
+            float L = 0.f;
+            if (M != -INFINITY)
+                for (int s2 = 0; s2 < nt; ++s2) {
+                    const float ms = wgt[s2 * HQP + tid];
+                    if (ms != -INFINITY) L += exp2f(ms - M) * lsum[s2 * HQP + tid];
                 }
+            Mh[tid] = M;
+            Lh[tid] = L;
+        }
+        __syncthreads();
+        for (int i = tid; i < nt * HQP; i += kAttnThreads) {
+            const int h = i % HQP;
+            const float ms = wgt[i];
+            wgt[i] = (ms == -INFINITY || !(Lh[h] > 0.f)) ? 0.f : exp2f(ms - Mh[h]) / Lh[h];
+        }
+        __syncthreads();
+        constexpr int D4 = D / 4;
+        for (int it = tid; it < p.Hq * D4; it += kAttnThreads) {
+            const int h = it / D4, d4 = it % D4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4* src = reinterpret_cast<const float4*>(pu + h * D) + d4;
+#pragma unroll 8
+            for (int s2 = 0; s2 < nt; ++s2) {
+                const float4 v = __ldcg(src + s2 * (stride / 4));
+                const float w = wgt[s2 * HQP + h];
+                acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
             }
-            if (tid < D) {
-                const float o = (L > 0.f) ? acc / L : 0.f;
-                p.out[((size_t)u * p.Hq + h) * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-            }
-            if (tid == 0 && p.lse != nullptr)
-                p.lse[(size_t)u * p.Hq + h] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(p.out + ((size_t)u * p.Hq + h) * D + 4 * d4) = pk;
+        }
+        if (tid < p.Hq && p.lse != nullptr) {
+            const float L = Lh[tid];
+            p.lse[(size_t)u * p.Hq + tid] = (L > 0.f) ? (Mh[tid] + log2f(L)) * 0.69314718055994530942f : -INFINITY;
         }
         if (tid == 0) p.tickets[u] = 0;
     }
@@ -374,7 +423,7 @@ template <int HQP, int D>
 static cudaError_t launch_attn_variant(const AttnParams& p, int units, cudaStream_t stream) {
     auto kern = sparse_attn_kernel<HQP, D>;
     const size_t smem = sizeof(AttnSmem<HQP>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.ntiles, units);
     kern<<<grid, kAttnThreads, smem, stream>>>(p);

@@ -70,6 +70,7 @@ static csa2_status check_attn(const csa2_attn_args* a, bool in_stack) {
     if (a->Hq < 1 || a->Hq > 32) return CSA2_ERR_UNSUPPORTED;
     if (a->D != 64 && a->D != 128) return CSA2_ERR_UNSUPPORTED;
     if ((!in_stack && a->k < 1) || a->W < 0 || a->Lloc < 0) return CSA2_ERR_SHAPE;
+    if ((int64_t)a->k + a->W > 16384) return CSA2_ERR_UNSUPPORTED;   // the merge keeps <= 128 tile weights
     if (!a->q_pos || !a->q || !a->kv_fp4 || !a->kv_scale || !a->out) return CSA2_ERR_NULL;
     if (!in_stack && !a->topk) return CSA2_ERR_NULL;
     if (a->W > 0 && (!a->kl || !a->vl || !a->local_base || a->Lloc < 1)) return CSA2_ERR_NULL;

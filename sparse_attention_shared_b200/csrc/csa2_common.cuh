@@ -5,6 +5,8 @@
 #pragma once
 
 #include <cstdint>
+#include <mutex>
+
 #include <cuda_runtime.h>
 
 #include "../../include/csa2.h"
@@ -69,17 +71,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     return true;
 }
 
-// ------------------------------------------------------------ bulk copies
-// 1-D bulk copy global -> shared memory of this CTA, completing on `bar`.
-// src and dst 16-byte aligned, bytes a multiple of 16. No cluster multicast.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -114,6 +105,17 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// D[tmem] (+)= A x B with signed int8 operands and int32 accumulation (kind::i8).
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on `bar` once all tcgen05.mma issued so far by this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -133,6 +135,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 32 bits, 8 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, int (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -140,14 +149,15 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 format):
 // start address >> 4 in bits [0,14), leading byte offset >> 4 in [16,30),
 // stride byte offset >> 4 in [32,46), version 1 in [46,48), base offset 0,
-// swizzle mode in [61,64) (2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+// swizzle mode in [61,64): 2 = 128-byte, 4 = 64-byte, 6 = 32-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t swizzle = 2) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFF);
     d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
     d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
     d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
+    d |= (uint64_t)(swizzle & 7u) << 61;
     return d;
 }
 
@@ -163,10 +173,39 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major) 
            | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 
+// Instruction descriptor, kind::i8 with signed int8 A/B (both K-major) and int32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+    return (2u << 4)                          // D format: s32
+           | (1u << 7)                        // A format: signed 8-bit
+           | (1u << 10)                       // B format: signed 8-bit
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
 // Byte offset of the 16-byte chunk `chunk` of row `row` inside a 128-byte-swizzled
 // panel whose rows are 128 bytes long (panel base 1024-byte aligned).
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+inline cudaError_t set_smem_once(const void* kern, int bytes) {
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    constexpr int kSlots = 64;
+    static const void* kerns[kSlots] = {nullptr};
+    static unsigned long long done[kSlots] = {0};   // bit per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    int slot = -1;
+    for (int i = 0; i < kSlots; ++i) {
+        if (kerns[i] == kern) { slot = i; break; }
+        if (kerns[i] == nullptr) { kerns[i] = kern; slot = i; break; }
+    }
+    if (slot >= 0 && dev < 64 && (done[slot] >> dev) & 1ull) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && slot >= 0 && dev < 64) done[slot] |= 1ull << dev;
+    return e;
 }
 
 }  // namespace csa2

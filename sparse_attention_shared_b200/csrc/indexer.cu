@@ -13,30 +13,40 @@
 // Design (B200): one cooperative launch. A "unit" is one query; a group of G
 // co-resident CTAs handles one unit at a time (persistent loop when there are
 // more units than groups). Each CTA scores a contiguous chunk of the unit's
-// candidates into shared memory (Full: key tiles arrive by TMA into a 4-stage
-// ring; Reindex: pool rows are gathered with 16-byte loads), then the group
-// finds the exact k-th best with a distributed radix select on a 36-bit
-// order-preserving key of the score: a 12-bit log-scale digit first, then two
-// 12-bit digits of the remaining bits. Each round costs one group barrier
-// (an atomic counter with a bounded spin). Once the threshold digit holds at
-// most kCandCap elements, they are gathered and every CTA sorts them (score,
-// position) in shared memory and knows the exact cut; exact ties at the last
-// digit are cut by position through per-CTA counts. Every CTA then writes its
+// candidates into shared memory:
+//   * Full mode with 32/64/128-byte keys: warp-specialised tensor-core scan.
+//     A TMA warp streams 256-row key tiles into a 6-stage ring, an MMA warp
+//     issues tcgen05.mma kind::i8 (keys as M = 128 rows, the index query's
+//     heads as N = 16) into 4 TMEM buffers, and 8 epilogue warps apply the
+//     ReLU and head weights to the int32 accumulators. mbarriers link the
+//     roles, so the scan runs at the rate of its slowest role.
+//   * Reindex mode and other key widths: rows are gathered (or TMA-staged)
+//     and scored with dp4a.
+// Then the group finds the exact cut with a distributed radix select on a
+// 36-bit order-preserving key of the score: a 12-bit log-scale digit first,
+// then two 12-bit digits of the remaining bits. Each round costs one group
+// barrier (an atomic counter with a bounded spin). Once the threshold digit
+// holds at most kCandCap elements, they are gathered and every CTA finds the
+// exact threshold score T among them with a local radix select; exact ties at
+// T are cut by position through per-CTA counts. Every CTA then writes its
 // selected positions at its offset, in ascending order, with no further sync.
 #include <cuda.h>
 
 #include <algorithm>
+#include <climits>
 #include <cstring>
 
 #include "csa2_common.cuh"
 
 namespace csa2 {
 
-constexpr int kIdxThreads = 256;
+constexpr int kSel = 256;                    // threads that run the select phase
+constexpr int kTcThreads = kSel + 64;        // + one TMA warp and one MMA warp
 constexpr int kBins = 4096;
 constexpr int kCandCap = 4096;
 constexpr int kStageBytes = 16384;
-constexpr int kStages = 4;
+constexpr int kStages = 6;
+constexpr int kTmemBufs = 4;
 constexpr int kSmemScores = 16384;                  // scores kept in shared memory
 constexpr int kSkewLen = kSmemScores / 64 * 65;     // padded: one spare word per 64
 constexpr int kCtrlInts = 32;
@@ -59,25 +69,50 @@ struct IdxParams {
     int P_in;
     int units, G, groups, chunk;
     int32_t* spill;      // [groups*G][skewed chunk] when chunk > kSmemScores
-    int* ctrl;           // [groups][kCtrlInts]
-    int* g0;             // [groups][3][kBins]
-    int* gl;             // [groups][2 tracks][2 levels][kBins]
-    int2* cand;          // [groups][2 tracks][kCandCap]
-    int* pub;            // [groups][2 tracks][2][kMaxG]
+    int* ctrl;           // [slots][kCtrlInts]
+    int* g0;             // [slots][3][kBins]
+    int* gl;             // [slots][2 tracks][2 levels][kBins]
+    int2* cand;          // [slots][2 tracks][kCandCap]
+    int* pub;            // [slots][2 tracks][3][kMaxG]
     int32_t* status;
 };
 
-struct __align__(16) IdxSmem {
-    uint8_t stage[kStages][kStageBytes];   // key tiles; later the candidate sort buffer
+struct __align__(1024) IdxSmem {
+    uint8_t stage[kStages][kStageBytes];   // key tiles; later the candidate buffers
+    uint8_t qtc[16 * 128];                 // index query as a tensor-core operand (16 rows)
     int sc[kSkewLen];                      // scores of this CTA's chunk (skewed index)
     int hist0[kBins];
     int histl[2][kBins];
     int8_t q[16 * 128];
     uint64_t full_bar[kStages];
+    uint64_t empty_bar[kStages];
+    uint64_t tfull_bar[kTmemBufs];
+    uint64_t tempty_bar[kTmemBufs];
+    uint32_t tmem_base;
+    int abort;
     int red[64];
     int info[64];
 };
-static_assert(sizeof(uint64_t) * kCandCap <= sizeof(((IdxSmem*)0)->stage), "candidate buffer");
+static_assert(2 * sizeof(int2) * kCandCap <= sizeof(((IdxSmem*)0)->stage), "candidate buffers");
+static_assert(kStages * kStageBytes % 1024 == 0, "tensor-core operand alignment");
+
+struct Slot {
+    int* ctrl;
+    int* g0;
+    int* gl;
+    int2* cand;
+    int* pub;
+};
+
+__device__ __forceinline__ Slot slot_of(const IdxParams& p, int group) {
+    Slot s;
+    s.ctrl = p.ctrl + (size_t)group * kCtrlInts;
+    s.g0 = p.g0 + (size_t)group * 3 * kBins;
+    s.gl = p.gl + (size_t)group * 4 * kBins;
+    s.cand = p.cand + (size_t)group * 2 * kCandCap;
+    s.pub = p.pub + (size_t)group * 6 * kMaxG;
+    return s;
+}
 
 __device__ __forceinline__ int skew(int e) { return (e >> 6) * 65 + (e & 63); }
 
@@ -112,14 +147,48 @@ __device__ __forceinline__ uint32_t digit_at(uint64_t ext, int level) {
     return (uint32_t)(ext >> (24 - 12 * level)) & 4095u;
 }
 
-// composite key: larger = ranked earlier (higher score, then lower index)
-__device__ __forceinline__ uint64_t comp_key(int32_t x, int idx) {
-    return (ext_key(x) << 27) | (uint64_t)(0x7FFFFFF - idx);
+// Level-0 digit only (the 12-bit log-scale bin of the score).
+__device__ __forceinline__ uint32_t bin0(int32_t x) {
+    return x >= 0 ? 2048u + mag_bin((uint32_t)x) : 2047u - mag_bin((uint32_t)(-1 - x));
 }
 
-// ------------------------------------------------------------ block helpers
-// Exclusive scan over the block (256 threads); returns the block total in `total`.
-__device__ __forceinline__ int block_scan_excl(int v, int* red, int& total) {
+// The score interval [lo, hi] that maps to level-0 bin d.
+__device__ __forceinline__ void bin0_interval(uint32_t d, int& lo, int& hi) {
+    const bool pos = d >= 2048u;
+    const uint32_t f = pos ? d - 2048u : 2047u - d;
+    long long ylo, yhi;
+    if (f < 64u) {
+        ylo = yhi = f;
+    } else {
+        const int e = (int)((f - 64u) / 64u) + 6;
+        const long long m = (f - 64u) % 64u;
+        ylo = (64 + m) << (e - 6);
+        yhi = ((64 + m + 1) << (e - 6)) - 1;
+    }
+    if (pos) { lo = (int)ylo; hi = (int)yhi; }
+    else     { lo = (int)(-1 - yhi); hi = (int)(-1 - ylo); }
+}
+
+// ------------------------------------------------------------ select-group sync
+// The select phase runs on threads [0, kSel) and synchronises on named barrier 1,
+// so extra warps of the CTA (the TMA and MMA warps) need not take part.
+__device__ __forceinline__ void sel_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ int sel_and(int v) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.s32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, 256, q;\n\t"
+        "selp.s32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(v)
+        : "memory");
+    return r;
+}
+
+// Exclusive scan over the select threads; returns the total in `total`.
+__device__ __forceinline__ int sel_scan_excl(int v, int* red, int& total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
 #pragma unroll
@@ -127,33 +196,43 @@ __device__ __forceinline__ int block_scan_excl(int v, int* red, int& total) {
         int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    __syncthreads();
+    sel_sync();
     if (lane == 31) red[warp] = x;
-    __syncthreads();
+    sel_sync();
     if (warp == 0) {
-        int s = lane < (kIdxThreads / 32) ? red[lane] : 0;
+        int s = lane < (kSel / 32) ? red[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             int y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        if (lane < kIdxThreads / 32) red[32 + lane] = s;
+        if (lane < kSel / 32) red[32 + lane] = s;
     }
-    __syncthreads();
+    sel_sync();
     const int warp_excl = warp ? red[32 + warp - 1] : 0;
-    total = red[32 + kIdxThreads / 32 - 1];
+    total = red[32 + kSel / 32 - 1];
     return warp_excl + x - v;
 }
 
-__device__ __forceinline__ int block_sum(int v, int* red) {
+__device__ __forceinline__ int sel_sum(int v, int* red) {
     int total;
-    block_scan_excl(v, red, total);
+    sel_scan_excl(v, red, total);
     return total;
 }
 
-// Group barrier over the G CTAs of a slot: counter increments once per CTA.
+__device__ __forceinline__ int sel_min(int v, int* red) {
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    sel_sync();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    sel_sync();
+    int m = red[0];
+    for (int w = 1; w < kSel / 32; ++w) m = min(m, red[w]);
+    return m;
+}
+
+// Group barrier over the G CTAs of a slot: the counter grows by one per CTA.
 __device__ bool group_barrier(int* counter, int target, int32_t* st) {
-    __syncthreads();
+    sel_sync();
     int ok = 1;
     if (threadIdx.x == 0) {
         __threadfence();
@@ -171,25 +250,31 @@ __device__ bool group_barrier(int* counter, int target, int32_t* st) {
         }
         __threadfence();
     }
-    return __syncthreads_and(ok) != 0;
+    return sel_and(ok) != 0;
 }
 
-// In a global 4096-bin histogram, find the bin holding the r-th largest element
-// (1-based). Writes {bin, count above the bin, count in the bin} to out[0..2].
+// In a 4096-bin histogram (global or shared), find the bin holding the r-th
+// largest element (1-based). Writes {bin, count above the bin, count in it}.
+template <bool kGlobal>
 __device__ void find_rank_bin(const int* hist, int r, int* red, int* out) {
     const int t = threadIdx.x;
     int h[16];
-    const int4* src = reinterpret_cast<const int4*>(hist + 16 * t);
+    if (kGlobal) {
+        const int4* src = reinterpret_cast<const int4*>(hist + 16 * t);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        int4 v = __ldcg(src + i);
-        h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
+        for (int i = 0; i < 4; ++i) {
+            int4 v = __ldcg(src + i);
+            h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) h[i] = hist[16 * t + i];
     }
     int s = 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) s += h[i];
     int total;
-    const int excl = block_scan_excl(s, red, total);
+    const int excl = sel_scan_excl(s, red, total);
     int above = total - excl - s;    // elements in bins above this thread's range
     if (above < r && r <= above + s) {
 #pragma unroll
@@ -202,12 +287,12 @@ __device__ void find_rank_bin(const int* hist, int r, int* red, int* out) {
             above += h[i];
         }
     }
-    __syncthreads();
+    sel_sync();
 }
 
 // Push the non-zero bins of a shared histogram into a global one.
 __device__ __forceinline__ void push_hist(const int* sh, int* gh) {
-    for (int i = threadIdx.x; i < kBins; i += kIdxThreads) {
+    for (int i = threadIdx.x; i < kBins; i += kSel) {
         const int v = sh[i];
         if (v) atomicAdd(gh + i, v);
     }
@@ -215,28 +300,284 @@ __device__ __forceinline__ void push_hist(const int* sh, int* gh) {
 
 __device__ __forceinline__ int sum_above(const int* sh, int bin) {
     int s = 0;
-    for (int i = threadIdx.x; i < kBins; i += kIdxThreads) s += (i > bin) ? sh[i] : 0;
+    for (int i = threadIdx.x; i < kBins; i += kSel) s += (i > bin) ? sh[i] : 0;
     return s;
 }
 
-// Bitonic sort of n (power of two) 64-bit keys in shared memory, descending.
-__device__ void bitonic_desc(uint64_t* a, int n) {
-    for (int k = 2; k <= n; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < n; i += kIdxThreads) {
-                const int l = i ^ j;
-                if (l > i) {
-                    const uint64_t x = a[i], y = a[l];
-                    const bool desc = (i & k) == 0;
-                    if (desc ? (x < y) : (x > y)) { a[i] = y; a[l] = x; }
-                }
-            }
-            __syncthreads();
-        }
-    }
+// Sum of the first `n` entries (n <= kSel) of a global array, loaded in parallel.
+__device__ __forceinline__ int prefix_total(const int* arr, int n, int* red) {
+    const int v = (threadIdx.x < n) ? __ldcg(arr + threadIdx.x) : 0;
+    return sel_sum(v, red);
 }
 
-// ------------------------------------------------------------ scoring
+// The r-th largest value (1-based, with multiplicity) of cx[0..C) in shared
+// memory, by 12-bit radix passes over x - min. Returns T; need_eq = how many of
+// the elements equal to T are ranked within the first r.
+__device__ int local_select(const int* cx, int C, int r, int* hist, int* red, int* info, int& need_eq) {
+    int mn = INT_MAX, mx = INT_MIN;
+    for (int i = threadIdx.x; i < C; i += kSel) { mn = min(mn, cx[i]); mx = max(mx, cx[i]); }
+    mn = sel_min(mn, red);
+    mx = -sel_min(-mx, red);
+    const uint32_t w = (uint32_t)((long long)mx - (long long)mn);
+    int rem = (w == 0u) ? 0 : 32 - __clz(w);
+    uint32_t prefix = 0;
+    while (rem > 0) {
+        const int take = rem < 12 ? rem : 12;
+        const int sh = rem - take;
+        for (int i = threadIdx.x; i < kBins; i += kSel) hist[i] = 0;
+        sel_sync();
+        for (int i = threadIdx.x; i < C; i += kSel) {
+            const uint32_t v = (uint32_t)((long long)cx[i] - (long long)mn);
+            if ((uint32_t)(((uint64_t)v) >> (sh + take)) == prefix) atomicAdd(&hist[(v >> sh) & ((1u << take) - 1u)], 1);
+        }
+        sel_sync();
+        find_rank_bin<false>(hist, r, red, info);
+        r -= info[1];
+        prefix = (prefix << take) | (uint32_t)info[0];
+        rem = sh;
+    }
+    need_eq = r;
+    return (int)((long long)mn + (long long)prefix);
+}
+
+// ------------------------------------------------------------ select + write
+// Track states (identical in every CTA of a group).
+enum { TS_OFF = 0, TS_ALL = 1, TS_RADIX = 2, TS_CAND = 3, TS_EQ = 4, TS_FIN_CAND = 5, TS_FIN_EQ = 6 };
+
+struct UnitCtx {
+    int u, t, lo, my_n, n_all, cta, j, epoch;
+    const int32_t* pool;   // Reindex: the unit's pool (positions of the elements)
+};
+
+// Exact pool/top-k cut for one unit and the write of this CTA's selected
+// positions. Runs on threads [0, kSel). The chunk's scores are in sc (skewed
+// index) and their level-0 histogram in S.hist0. Returns false on a timeout.
+__device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c, int& bar_target,
+                            const int* sc) {
+    const int tid = threadIdx.x;
+    const bool full = p.mode == CSA2_FULL;
+    const int lo = c.lo, my_n = c.my_n;
+
+    // ---- round 0: histogram of level 0; zero the buffers the next steps use
+    int* g0cur = sl.g0 + ((c.epoch + c.j) % 3) * kBins;
+    int* g0nxt = sl.g0 + ((c.epoch + c.j + 1) % 3) * kBins;
+    push_hist(S.hist0, g0cur);
+    {
+        const int per = (kBins + p.G - 1) / p.G;
+        const int zlo = c.cta * per, zhi = min(kBins, zlo + per);
+        for (int i = zlo + tid; i < zhi; i += kSel) {
+            g0nxt[i] = 0;
+            sl.gl[i] = 0; sl.gl[kBins + i] = 0; sl.gl[2 * kBins + i] = 0; sl.gl[3 * kBins + i] = 0;
+        }
+        if (c.cta == 0 && tid == 0) { sl.ctrl[CTRL_CAND0] = 0; sl.ctrl[CTRL_CAND1] = 0; }
+    }
+    bar_target += p.G;
+    if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
+
+    int n_total;
+    if (full) {
+        n_total = c.n_all;
+    } else {
+        int s2 = 0;
+        for (int i = tid; i < kBins; i += kSel) s2 += __ldcg(g0cur + i);
+        n_total = sel_sum(s2, S.red);
+    }
+    int state[2], rrem[2], C[2], level[2], above_loc[2], clo[2], chi[2];
+    uint64_t prefix[2];
+    for (int tr = 0; tr < 2; ++tr) {
+        state[tr] = TS_OFF; rrem[tr] = 0; C[tr] = 0; level[tr] = 0; above_loc[tr] = 0; prefix[tr] = 0;
+        clo[tr] = 0; chi[tr] = -1;
+        const int r = p.r[tr];
+        if (r <= 0) continue;
+        if (n_total <= r) { state[tr] = TS_ALL; continue; }
+        find_rank_bin<true>(g0cur, r, S.red, S.info + 8 * tr);
+        const int d = S.info[8 * tr + 0];
+        rrem[tr] = r - S.info[8 * tr + 1];
+        C[tr] = S.info[8 * tr + 2];
+        prefix[tr] = (uint64_t)d;
+        above_loc[tr] = sel_sum(sum_above(S.hist0, d), S.red);
+        bin0_interval((uint32_t)d, clo[tr], chi[tr]);
+        state[tr] = (C[tr] <= kCandCap) ? TS_CAND : TS_RADIX;
+    }
+
+    // ---- rounds until every track knows its cut (usually one)
+    while (true) {
+        bool any = false;
+        for (int tr = 0; tr < 2; ++tr) {
+            if (state[tr] == TS_RADIX) {
+                // histogram of the next digit over own elements matching the prefix
+                any = true;
+                int* hl = S.histl[tr];
+                for (int i = tid; i < kBins; i += kSel) hl[i] = 0;
+                sel_sync();
+                const int lv = level[tr] + 1;
+                for (int e = tid; e < my_n; e += kSel) {
+                    const int x = sc[skew(e)];
+                    if (x < clo[tr] || x > chi[tr]) continue;
+                    const uint64_t ek = ext_key(x);
+                    if ((ek >> (36 - 12 * lv)) == prefix[tr]) atomicAdd(&hl[digit_at(ek, lv)], 1);
+                }
+                sel_sync();
+                push_hist(hl, sl.gl + (2 * tr + (lv - 1)) * kBins);
+            } else if (state[tr] == TS_CAND) {
+                // gather own elements of the threshold digit: compact them in shared
+                // memory, reserve a range of the group's buffer with one atomic, copy
+                any = true;
+                const int lv = level[tr] + 1;
+                int2* lbuf = reinterpret_cast<int2*>(&S.stage[0][0]) + tr * kCandCap;
+                if (tid == 0) S.info[40 + tr] = 0;
+                sel_sync();
+                for (int e0 = 0; e0 < my_n; e0 += kSel) {
+                    const int e = e0 + tid;
+                    int x = 0;
+                    bool m = false;
+                    if (e < my_n) {
+                        x = sc[skew(e)];
+                        m = x >= clo[tr] && x <= chi[tr];
+                        if (m && lv > 1) m = (ext_key(x) >> (36 - 12 * lv)) == prefix[tr];
+                    }
+                    const unsigned bal = __ballot_sync(0xffffffffu, m);
+                    if (bal) {
+                        int basei = 0;
+                        if ((tid & 31) == 0) basei = atomicAdd(&S.info[40 + tr], __popc(bal));
+                        basei = __shfl_sync(0xffffffffu, basei, 0);
+                        if (m) {
+                            const int slot = basei + __popc(bal & ((1u << (tid & 31)) - 1u));
+                            if (slot < kCandCap) lbuf[slot] = make_int2(x, lo + e);
+                        }
+                    }
+                }
+                sel_sync();
+                const int n_mine = min(S.info[40 + tr], kCandCap);
+                if (tid == 0) S.info[44 + tr] = n_mine ? atomicAdd(sl.ctrl + CTRL_CAND0 + tr, n_mine) : 0;
+                sel_sync();
+                const int gbase = S.info[44 + tr];
+                for (int i = tid; i < n_mine; i += kSel)
+                    if (gbase + i < kCandCap) sl.cand[tr * kCandCap + gbase + i] = lbuf[i];
+                if (tid == 0) sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = above_loc[tr];
+            } else if (state[tr] == TS_EQ) {
+                // the value is exact: count own ties and publish it
+                any = true;
+                int eq = 0, val = 0;
+                bool have = false;
+                for (int e = tid; e < my_n; e += kSel) {
+                    const int x = sc[skew(e)];
+                    if (x >= clo[tr] && x <= chi[tr] && ext_key(x) == prefix[tr]) { eq++; val = x; have = true; }
+                }
+                if (have) sl.pub[(tr * 3 + 2) * kMaxG + 0] = val;   // every writer stores the same value
+                eq = sel_sum(eq, S.red);
+                if (tid == 0) {
+                    sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = above_loc[tr];
+                    sl.pub[(tr * 3 + 1) * kMaxG + c.cta] = eq;
+                }
+            }
+        }
+        if (!any) break;
+        bar_target += p.G;
+        if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
+        bool pending = false;
+        for (int tr = 0; tr < 2; ++tr) {
+            if (state[tr] == TS_RADIX) {
+                const int lv = level[tr] + 1;
+                find_rank_bin<true>(sl.gl + (2 * tr + (lv - 1)) * kBins, rrem[tr], S.red, S.info + 8 * tr);
+                const int d = S.info[8 * tr + 0];
+                rrem[tr] -= S.info[8 * tr + 1];
+                C[tr] = S.info[8 * tr + 2];
+                prefix[tr] = (prefix[tr] << 12) | (uint64_t)d;
+                level[tr] = lv;
+                above_loc[tr] += sel_sum(sum_above(S.histl[tr], d), S.red);
+                state[tr] = (C[tr] <= kCandCap) ? TS_CAND : (lv < 2 ? TS_RADIX : TS_EQ);
+                pending = true;
+            } else if (state[tr] == TS_CAND) {
+                state[tr] = TS_FIN_CAND;
+            } else if (state[tr] == TS_EQ) {
+                state[tr] = TS_FIN_EQ;
+            }
+        }
+        if (!pending) break;
+    }
+
+    // ---- write each track's list
+    for (int tr = 0; tr < 2; ++tr) {
+        const int r = p.r[tr];
+        if (r <= 0) continue;
+        int32_t* outp = p.out[tr] + (size_t)c.u * r;
+        const int st = state[tr];
+        int T = INT_MAX, base_off = lo, quota = 0;
+        if (st == TS_FIN_CAND || st == TS_FIN_EQ) {
+            const int prev = prefix_total(sl.pub + (tr * 3 + 0) * kMaxG, c.cta, S.red);
+            int need_eq = 0, gt_before = 0, eq_before = 0, my_eq = 0;
+            if (st == TS_FIN_CAND) {
+                // exact threshold among the gathered candidates
+                int* cx = reinterpret_cast<int*>(&S.stage[0][0]);
+                int* ci = cx + kCandCap;
+                const int Cn = C[tr];
+                for (int i = tid; i < Cn; i += kSel) {
+                    const int2 cv = __ldcg(sl.cand + tr * kCandCap + i);
+                    cx[i] = cv.x;
+                    ci[i] = cv.y;
+                }
+                sel_sync();
+                T = local_select(cx, Cn, rrem[tr], S.histl[tr], S.red, S.info + 8 * tr, need_eq);
+                for (int i = tid; i < Cn; i += kSel) {
+                    const int x = cx[i], idx = ci[i];
+                    gt_before += (x > T && idx < lo);
+                    eq_before += (x == T && idx < lo);
+                    my_eq += (x == T && idx >= lo && idx < lo + my_n);
+                }
+                gt_before = sel_sum(gt_before, S.red);
+                eq_before = sel_sum(eq_before, S.red);
+                my_eq = sel_sum(my_eq, S.red);
+            } else {
+                T = __ldcg(sl.pub + (tr * 3 + 2) * kMaxG + 0);
+                need_eq = rrem[tr];
+                eq_before = prefix_total(sl.pub + (tr * 3 + 1) * kMaxG, c.cta, S.red);
+                my_eq = __ldcg(sl.pub + (tr * 3 + 1) * kMaxG + c.cta);
+            }
+            quota = max(0, min(need_eq - eq_before, my_eq));
+            base_off = prev + gt_before + min(need_eq, eq_before);
+        }
+        // ordered compaction: thread tid owns elements [tid*R, tid*R+R)
+        const int R = (my_n + kSel - 1) / kSel;
+        const int e0 = min(tid * R, my_n), e1 = min(e0 + R, my_n);
+        const bool all = (st == TS_ALL);
+        int cnt = 0, ceq = 0;
+        if (all) {
+            cnt = e1 - e0;
+        } else {
+            for (int e = e0; e < e1; ++e) {
+                const int x = sc[skew(e)];
+                cnt += x > T;
+                ceq += x == T;
+            }
+        }
+        int tot;
+        const int eq_excl = sel_scan_excl(ceq, S.red, tot);
+        const int eq_take = max(0, min(quota - eq_excl, ceq));
+        const int off = base_off + sel_scan_excl(cnt + eq_take, S.red, tot);
+        int k2 = off, eq_seen = 0;
+        for (int e = e0; e < e1; ++e) {
+            bool sel = all;
+            if (!all) {
+                const int x = sc[skew(e)];
+                sel = x > T;
+                if (x == T) { sel = eq_seen < eq_take; eq_seen++; }
+            }
+            if (sel) {
+                if (k2 < r) outp[k2] = full ? (lo + e) : c.pool[lo + e];
+                k2++;
+            }
+        }
+        // padding: entries [min(r, n_total), r) = -1
+        if (c.cta == p.G - 1) {
+            for (int i = min(r, n_total) + tid; i < r; i += kSel) outp[i] = -1;
+        }
+        sel_sync();
+    }
+    return true;
+}
+
+// ------------------------------------------------------------ scoring helpers
 template <int HI, int DI>
 struct RegQ {
     int q[HI][DI / 4];
@@ -305,354 +646,293 @@ __device__ __forceinline__ void tma_load_keys(void* dst, const CUtensorMap* map,
         : "memory");
 }
 
-// ------------------------------------------------------------ the kernel
-template <int HI, int DI>
-__global__ void __launch_bounds__(kIdxThreads, 1)
-    index_select_kernel(const __grid_constant__ IdxParams p, const __grid_constant__ CUtensorMap kmap) {
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ IdxSmem& idx_smem() {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    IdxSmem& S = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    return *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+}
+
+// ------------------------------------------------------------ Full mode on the tensor cores
+// Warps 0-7: epilogue and select; warp 8: TMA producer; warp 9: MMA issuer.
+template <int DI>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    index_full_tc_kernel(const __grid_constant__ IdxParams p, const __grid_constant__ CUtensorMap kmap) {
+    static_assert(DI == 32 || DI == 64 || DI == 128, "tensor-core key widths");
+    IdxSmem& S = idx_smem();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int group = blockIdx.x / p.G;
+    const int cta = blockIdx.x % p.G;
+    const Slot sl = slot_of(p, group);
+    int* sc = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * ((p.chunk + 63) / 64 * 65) : S.sc;
+    constexpr int kRows = (kStageBytes / DI) < 256 ? (kStageBytes / DI) : 256;   // rows per tile
+    constexpr int kBlocks = kRows / 128;                                          // MMA row blocks per tile
+    constexpr uint32_t kSwz = DI == 32 ? 6u : DI == 64 ? 4u : 2u;
+    constexpr uint32_t kSbo = 8 * DI;                                             // bytes per 8-row group
+    constexpr uint32_t kIdesc = idesc_i8(128, 16);
+
+    const int epoch = __ldcg(sl.ctrl + CTRL_EPOCH);
+    int bar_target = __ldcg(sl.ctrl + CTRL_BAR_BASE);
+    if (warp == 0) tmem_alloc(&S.tmem_base, 32 * kTmemBufs);
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) { mbar_init(&S.full_bar[i], 1); mbar_init(&S.empty_bar[i], 1); }
+        for (int i = 0; i < kTmemBufs; ++i) { mbar_init(&S.tfull_bar[i], 1); mbar_init(&S.tempty_bar[i], kSel); }
+        S.abort = 0;
+        mbar_fence_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    uint32_t seq = 0;   // tiles processed by this CTA so far (same count in every role)
+
+    int j = 0;
+    for (int u = group; u < p.units; u += p.groups, ++j) {
+        const int b = u / p.Tq;
+        int t = p.q_pos[u];
+        if (t < 0 || t >= p.N) {
+            if (tid == 0 && cta == 0) report(p.status, CSA2_ERR_RANGE, u);
+            t = -1;
+        }
+        const int n_all = t + 1;
+        const int lo = min(cta * p.chunk, n_all);
+        const int my_n = min(lo + p.chunk, n_all) - lo;
+        const int nst = (my_n + kRows - 1) / kRows;
+
+        // index query -> B operand (16 rows: heads, zero past Hi); zero the histogram
+        fence_proxy_async_smem();
+        for (int i = tid; i < p.Hi * DI / 16; i += kTcThreads)
+            reinterpret_cast<int4*>(S.q)[i] = reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * DI)[i];
+        for (int i = tid; i < kBins; i += kTcThreads) S.hist0[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < DI; i += kTcThreads) {
+            const int h = i / (DI / 16), c2 = i % (DI / 16);
+            int4 v = make_int4(0, 0, 0, 0);
+            if (h < p.Hi) v = reinterpret_cast<const int4*>(S.q + h * DI)[c2];
+            *reinterpret_cast<int4*>(S.qtc + tile_off(h, c2, DI)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        if (warp == kSel / 32) {
+            // ---- TMA producer
+            if (lane == 0) {
+                for (int s2 = 0; s2 < nst; ++s2) {
+                    const uint32_t i = seq + s2, slot = i % kStages;
+                    if (i >= (uint32_t)kStages &&
+                        !mbar_wait(&S.empty_bar[slot], ((i / kStages) - 1) & 1u, p.status, 5)) { S.abort = 1; break; }
+                    mbar_arrive_expect_tx(&S.full_bar[slot], (uint32_t)(kRows * DI));
+                    tma_load_keys(S.stage[slot], &kmap, 0, lo + s2 * kRows, b, &S.full_bar[slot]);
+                }
+            }
+        } else if (warp == kSel / 32 + 1) {
+            // ---- MMA issuer
+            if (lane == 0) {
+                const uint32_t b0 = smem_u32(S.qtc);
+                for (int s2 = 0; s2 < nst; ++s2) {
+                    const uint32_t i = seq + s2, slot = i % kStages, buf = i % kTmemBufs;
+                    if (!mbar_wait(&S.full_bar[slot], (i / kStages) & 1u, p.status, 3)) { S.abort = 1; break; }
+                    if (i >= (uint32_t)kTmemBufs &&
+                        !mbar_wait(&S.tempty_bar[buf], ((i / kTmemBufs) - 1) & 1u, p.status, 6)) { S.abort = 1; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(S.stage[slot]);
+                    const uint32_t d0 = tmem + buf * 32u;
+#pragma unroll
+                    for (int blk = 0; blk < kBlocks; ++blk) {
+#pragma unroll
+                        for (int kk = 0; kk < DI / 32; ++kk)
+                            mma_i8(d0 + blk * 16, smem_desc(a0 + blk * 128 * DI + kk * 32, 16, kSbo, kSwz),
+                                   smem_desc(b0 + kk * 32, 16, kSbo, kSwz), kIdesc, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&S.empty_bar[slot]);
+                    mma_commit(&S.tfull_bar[buf]);
+                }
+            }
+        } else {
+            // ---- epilogue: ReLU and head weights on the int32 accumulators
+            const bool in_block = (warp >> 2) < kBlocks;              // warp-uniform
+            const uint32_t lane_base = tmem + (uint32_t)(warp >> 2) * 16u + ((uint32_t)(warp & 3) * 32u << 16);
+            for (int s2 = 0; s2 < nst; ++s2) {
+                const uint32_t i = seq + s2, buf = i % kTmemBufs;
+                if (!mbar_wait(&S.tfull_bar[buf], (i / kTmemBufs) & 1u, p.status, 4)) { S.abort = 1; break; }
+                tc_fence_after();
+                int x = 0;
+                if (in_block) {
+                    int acc[8];
+                    const uint32_t ta = lane_base + buf * 32u;
+                    tmem_ld8(ta, acc);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) x += p.w[h] * max(acc[h], 0);
+                    if (p.Hi > 8) {
+                        tmem_ld8(ta + 8, acc);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) x += p.w[8 + h] * max(acc[h], 0);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&S.tempty_bar[buf]);
+                const int e = s2 * kRows + tid;
+                if (in_block && e < my_n) {
+                    sc[skew(e)] = x;
+                    atomicAdd(&S.hist0[bin0(x)], 1);
+                }
+            }
+        }
+        seq += nst;
+        __syncthreads();
+        if (S.abort) break;
+
+        if (tid < kSel) {
+            UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, nullptr};
+            if (!select_unit(p, S, sl, c, bar_target, sc) && tid == 0) S.abort = 1;
+        }
+        __syncthreads();
+        if (S.abort) break;
+    }
+    if (!S.abort && cta == 0 && tid == 0) {
+        sl.ctrl[CTRL_EPOCH] = epoch + j;
+        sl.ctrl[CTRL_BAR_BASE] = bar_target;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 32 * kTmemBufs);
+}
+
+// ------------------------------------------------------------ Reindex, and Full for other key widths
+template <int HI, int DI>
+__global__ void __launch_bounds__(kSel, 1)
+    index_dp4a_kernel(const __grid_constant__ IdxParams p, const __grid_constant__ CUtensorMap kmap) {
+    IdxSmem& S = idx_smem();
     const int tid = threadIdx.x;
     const int group = blockIdx.x / p.G;
     const int cta = blockIdx.x % p.G;
+    const Slot sl = slot_of(p, group);
     const bool full = p.mode == CSA2_FULL;
-    const bool generic = (HI == 0);
-
-    int* ctrl = p.ctrl + (size_t)group * kCtrlInts;
-    int* g0 = p.g0 + (size_t)group * 3 * kBins;
-    int* gl = p.gl + (size_t)group * 4 * kBins;
-    int2* cand = p.cand + (size_t)group * 2 * kCandCap;
-    int* pub = p.pub + (size_t)group * 4 * kMaxG;
+    constexpr bool generic = (HI == 0);
     int* sc = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * ((p.chunk + 63) / 64 * 65) : S.sc;
 
-    const int epoch = __ldcg(ctrl + CTRL_EPOCH);
-    int bar_target = __ldcg(ctrl + CTRL_BAR_BASE);
+    const int epoch = __ldcg(sl.ctrl + CTRL_EPOCH);
+    int bar_target = __ldcg(sl.ctrl + CTRL_BAR_BASE);
     const int rows_per_stage = (full ? min(256, kStageBytes / p.Di) : 0);
     const int nchunk = p.Di / 16;
 
     if (tid < kStages) mbar_init(&S.full_bar[tid], 1);
     mbar_fence_init();
     __syncthreads();
-    uint32_t stage_seq = 0;   // stages issued by this CTA so far
+    uint32_t stage_seq = 0;   // key tiles issued by this CTA so far
     bool alive = true;
 
     int j = 0;
     for (int u = group; u < p.units && alive; u += p.groups, ++j) {
         const int b = u / p.Tq;
         int t = p.q_pos[u];
-        bool bad_t = (t < 0 || t >= p.N);
+        const bool bad_t = (t < 0 || t >= p.N);
         if (bad_t) {
             if (tid == 0 && cta == 0) report(p.status, CSA2_ERR_RANGE, u);
             t = -1;
         }
-        // candidates of this unit: Full -> positions 0..t; Reindex -> pool entries
         const int n_all = full ? (t + 1) : (bad_t ? 0 : p.P_in);
         const int lo = min(cta * p.chunk, n_all);
         const int hi = min(lo + p.chunk, n_all);
         const int32_t* pool = full ? nullptr : p.pool_in + (size_t)u * p.P_in;
 
-        // ---- indexer query and local histogram
-        for (int i = tid; i < p.Hi * p.Di / 16; i += kIdxThreads)
+        fence_proxy_async_smem();
+        for (int i = tid; i < p.Hi * p.Di / 16; i += kSel)
             reinterpret_cast<int4*>(S.q)[i] = reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * p.Di)[i];
-        for (int i = tid; i < kBins; i += kIdxThreads) S.hist0[i] = 0;
+        for (int i = tid; i < kBins; i += kSel) S.hist0[i] = 0;
         __syncthreads();
         RegQ<(HI > 0 ? HI : 1), (DI > 0 ? DI : 16)> rq;
         if (!generic) rq.load(S.q);
 
-        // ---- score own chunk
         int my_n = hi - lo;
         if (full) {
             const int nst = (my_n + rows_per_stage - 1) / rows_per_stage;
             if (tid == 0) {
-                for (int s = 0; s < min(kStages, nst); ++s) {
-                    const uint32_t k = stage_seq + s;
+                for (int s2 = 0; s2 < min(kStages, nst); ++s2) {
+                    const uint32_t k = stage_seq + s2;
                     mbar_arrive_expect_tx(&S.full_bar[k % kStages], (uint32_t)(rows_per_stage * p.Di));
-                    tma_load_keys(S.stage[k % kStages], &kmap, 0, lo + s * rows_per_stage, b,
+                    tma_load_keys(S.stage[k % kStages], &kmap, 0, lo + s2 * rows_per_stage, b,
                                   &S.full_bar[k % kStages]);
                 }
             }
-            for (int s = 0; s < nst; ++s) {
-                const uint32_t k = stage_seq + s;
-                if (!mbar_wait(&S.full_bar[k % kStages], (k / kStages) & 1u, p.status, 2)) { alive = false; }
+            for (int s2 = 0; s2 < nst; ++s2) {
+                const uint32_t k = stage_seq + s2;
+                if (!mbar_wait(&S.full_bar[k % kStages], (k / kStages) & 1u, p.status, 2)) alive = false;
                 if (__syncthreads_or(!alive)) { alive = false; break; }
-                const int e = s * rows_per_stage + tid;
+                const int e = s2 * rows_per_stage + tid;
                 if (tid < rows_per_stage && e < my_n) {
                     const uint8_t* tile = S.stage[k % kStages];
                     int4 rowc[8];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        if (c < nchunk) rowc[c] = *reinterpret_cast<const int4*>(tile + tile_off(tid, c, p.Di));
-                    const int x = generic ? score_generic(rowc, nchunk, S.q, p.Hi, p.Di, p.w)
-                                          : rq.score(rowc, p.w);
+                    for (int c2 = 0; c2 < 8; ++c2)
+                        if (c2 < nchunk) rowc[c2] = *reinterpret_cast<const int4*>(tile + tile_off(tid, c2, p.Di));
+                    const int x = generic ? score_generic(rowc, nchunk, S.q, p.Hi, p.Di, p.w) : rq.score(rowc, p.w);
                     sc[skew(e)] = x;
-                    atomicAdd(&S.hist0[digit_at(ext_key(x), 0)], 1);
+                    atomicAdd(&S.hist0[bin0(x)], 1);
                 }
                 __syncthreads();
-                if (tid == 0 && s + kStages < nst) {
+                if (tid == 0 && s2 + kStages < nst) {
                     const uint32_t k2 = k + kStages;
                     mbar_arrive_expect_tx(&S.full_bar[k2 % kStages], (uint32_t)(rows_per_stage * p.Di));
-                    tma_load_keys(S.stage[k2 % kStages], &kmap, 0, lo + (s + kStages) * rows_per_stage, b,
+                    tma_load_keys(S.stage[k2 % kStages], &kmap, 0, lo + (s2 + kStages) * rows_per_stage, b,
                                   &S.full_bar[k2 % kStages]);
                 }
             }
             stage_seq += nst;
             if (!alive) break;
         } else {
-            // Reindex: valid pool entries form a prefix (ascending, -1 padded at the end)
+            // valid pool entries (0 <= s <= t) form a prefix, -1 padding after
             int first_bad = my_n;
-            for (int e = tid; e < my_n; e += kIdxThreads) {
-                const int s = pool[lo + e];
-                if (s < 0 || s > t) first_bad = min(first_bad, e);
+            for (int e = tid; e < my_n; e += kSel) {
+                const int s2 = pool[lo + e];
+                if (s2 < 0 || s2 > t) first_bad = min(first_bad, e);
             }
-            int fb = first_bad;
-            {
-                // block min
-                for (int o = 16; o > 0; o >>= 1) fb = min(fb, __shfl_xor_sync(0xffffffffu, fb, o));
-                if ((tid & 31) == 0) S.red[tid >> 5] = fb;
-                __syncthreads();
-                fb = S.red[0];
-                for (int w2 = 1; w2 < kIdxThreads / 32; ++w2) fb = min(fb, S.red[w2]);
-                __syncthreads();
-            }
+            const int fb = sel_min(first_bad, S.red);
             if (fb < my_n) {
                 // an entry past the first invalid one must be padding, never a position
-                for (int e = fb + tid; e < my_n; e += kIdxThreads)
+                for (int e = fb + tid; e < my_n; e += kSel)
                     if (pool[lo + e] >= 0) report(p.status, CSA2_ERR_RANGE, u);
                 my_n = fb;
             }
             if (my_n > 0 && lo > 0 && tid == 0 && pool[lo - 1] < 0) report(p.status, CSA2_ERR_RANGE, u);
             const int8_t* kb = p.ki + (size_t)b * p.ki_seq_stride;
-            for (int e = tid; e < my_n; e += kIdxThreads) {
-                const int s = pool[lo + e];
-                const int4* row = reinterpret_cast<const int4*>(kb + (size_t)s * p.Di);
-                int4 rowc[8];
+            constexpr int RB = 4;   // rows per thread in flight
+            for (int e0 = 0; e0 < my_n; e0 += RB * kSel) {
+                int4 rows[RB][8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    if (c < nchunk) rowc[c] = __ldg(row + c);
-                const int x = generic ? score_generic(rowc, nchunk, S.q, p.Hi, p.Di, p.w) : rq.score(rowc, p.w);
-                sc[skew(e)] = x;
-                atomicAdd(&S.hist0[digit_at(ext_key(x), 0)], 1);
+                for (int q2 = 0; q2 < RB; ++q2) {
+                    const int e = e0 + q2 * kSel + tid;
+                    if (e < my_n) {
+                        const int4* row = reinterpret_cast<const int4*>(kb + (size_t)pool[lo + e] * p.Di);
+#pragma unroll
+                        for (int c2 = 0; c2 < 8; ++c2)
+                            if (c2 < nchunk) rows[q2][c2] = __ldg(row + c2);
+                    }
+                }
+#pragma unroll
+                for (int q2 = 0; q2 < RB; ++q2) {
+                    const int e = e0 + q2 * kSel + tid;
+                    if (e < my_n) {
+                        const int x = generic ? score_generic(rows[q2], nchunk, S.q, p.Hi, p.Di, p.w)
+                                              : rq.score(rows[q2], p.w);
+                        sc[skew(e)] = x;
+                        atomicAdd(&S.hist0[bin0(x)], 1);
+                    }
+                }
             }
         }
         __syncthreads();
-
-        // ---- round 0: histogram of level 0, zero the buffers the next steps use
-        int* g0cur = g0 + ((epoch + j) % 3) * kBins;
-        int* g0nxt = g0 + ((epoch + j + 1) % 3) * kBins;
-        push_hist(S.hist0, g0cur);
-        {
-            const int per = (kBins + p.G - 1) / p.G;
-            const int zlo = cta * per, zhi = min(kBins, zlo + per);
-            for (int i = zlo + tid; i < zhi; i += kIdxThreads) {
-                g0nxt[i] = 0;
-                gl[i] = 0; gl[kBins + i] = 0; gl[2 * kBins + i] = 0; gl[3 * kBins + i] = 0;
-            }
-            if (cta == 0 && tid == 0) { ctrl[CTRL_CAND0] = 0; ctrl[CTRL_CAND1] = 0; }
-        }
-        bar_target += p.G;
-        if (!group_barrier(ctrl + CTRL_BAR, bar_target, p.status)) { alive = false; break; }
-
-        // ---- per-track state (identical in every CTA of the group)
-        // info layout per track: [0]=state [1]=r_rem [2]=C [3]=level [4..5]=prefix lo/hi [6]=above_local
-        // state: 0 off, 1 all, 2 radix in progress, 3 cand gather, 4 eq counts, 9 finished
-        int n_total;
-        if (full) n_total = n_all;
-        else {
-            int s = 0;
-            for (int i = tid; i < kBins; i += kIdxThreads) s += __ldcg(g0cur + i);
-            n_total = block_sum(s, S.red);
-        }
-        int state[2], rrem[2], C[2], level[2], above_loc[2];
-        uint64_t prefix[2];
-        for (int tr = 0; tr < 2; ++tr) {
-            state[tr] = 0; rrem[tr] = 0; C[tr] = 0; level[tr] = 0; above_loc[tr] = 0; prefix[tr] = 0;
-            const int r = p.r[tr];
-            if (r <= 0) continue;
-            if (n_total <= r) { state[tr] = 1; continue; }
-            find_rank_bin(g0cur, r, S.red, S.info + 8 * tr);
-            const int d = S.info[8 * tr + 0];
-            rrem[tr] = r - S.info[8 * tr + 1];
-            C[tr] = S.info[8 * tr + 2];
-            prefix[tr] = (uint64_t)d;
-            level[tr] = 0;
-            above_loc[tr] = block_sum(sum_above(S.hist0, d), S.red);
-            state[tr] = (C[tr] <= kCandCap) ? 3 : 2;
-        }
-
-        // ---- rounds until every track knows its cut
-        while (alive) {
-            bool any = false;
-            for (int tr = 0; tr < 2; ++tr) {
-                if (state[tr] == 2) {
-                    // histogram of the next digit over elements matching the prefix
-                    any = true;
-                    int* hl = S.histl[tr];
-                    for (int i = tid; i < kBins; i += kIdxThreads) hl[i] = 0;
-                    __syncthreads();
-                    const int lv = level[tr] + 1;
-                    for (int e = tid; e < my_n; e += kIdxThreads) {
-                        const uint64_t ek = ext_key(sc[skew(e)]);
-                        if ((ek >> (36 - 12 * lv)) == prefix[tr]) atomicAdd(&hl[digit_at(ek, lv)], 1);
-                    }
-                    __syncthreads();
-                    push_hist(hl, gl + (2 * tr + (lv - 1)) * kBins);
-                } else if (state[tr] == 3) {
-                    // gather the elements of the threshold bin
-                    any = true;
-                    const int lv = level[tr] + 1;
-                    for (int e0 = 0; e0 < my_n; e0 += kIdxThreads) {
-                        const int e = e0 + tid;
-                        int x = 0;
-                        bool m = false;
-                        if (e < my_n) {
-                            x = sc[skew(e)];
-                            m = (ext_key(x) >> (36 - 12 * lv)) == prefix[tr];
-                        }
-                        const unsigned bal = __ballot_sync(0xffffffffu, m);
-                        if (bal) {
-                            int basei = 0;
-                            if ((tid & 31) == 0) basei = atomicAdd(ctrl + CTRL_CAND0 + tr, __popc(bal));
-                            basei = __shfl_sync(0xffffffffu, basei, 0);
-                            if (m) {
-                                const int slot = basei + __popc(bal & ((1u << (tid & 31)) - 1u));
-                                if (slot < kCandCap) cand[tr * kCandCap + slot] = make_int2(x, lo + e);
-                            }
-                        }
-                    }
-                    if (tid == 0) pub[(tr * 2 + 0) * kMaxG + cta] = above_loc[tr];
-                } else if (state[tr] == 4) {
-                    any = true;
-                    int eq = 0;
-                    for (int e = tid; e < my_n; e += kIdxThreads) eq += (ext_key(sc[skew(e)]) == prefix[tr]);
-                    eq = block_sum(eq, S.red);
-                    if (tid == 0) {
-                        pub[(tr * 2 + 0) * kMaxG + cta] = above_loc[tr];
-                        pub[(tr * 2 + 1) * kMaxG + cta] = eq;
-                    }
-                }
-            }
-            if (!any) break;
-            bar_target += p.G;
-            if (!group_barrier(ctrl + CTRL_BAR, bar_target, p.status)) { alive = false; break; }
-            for (int tr = 0; tr < 2; ++tr) {
-                if (state[tr] == 2) {
-                    const int lv = level[tr] + 1;
-                    const int* gh = gl + (2 * tr + (lv - 1)) * kBins;
-                    find_rank_bin(gh, rrem[tr], S.red, S.info + 8 * tr);
-                    const int d = S.info[8 * tr + 0];
-                    rrem[tr] -= S.info[8 * tr + 1];
-                    C[tr] = S.info[8 * tr + 2];
-                    prefix[tr] = (prefix[tr] << 12) | (uint64_t)d;
-                    level[tr] = lv;
-                    above_loc[tr] += block_sum(sum_above(S.histl[tr], d), S.red);
-                    state[tr] = (C[tr] <= kCandCap) ? 3 : (lv < 2 ? 2 : 4);
-                } else if (state[tr] == 3) {
-                    state[tr] = 5;   // finalize from candidates
-                } else if (state[tr] == 4) {
-                    state[tr] = 6;   // finalize from equal counts
-                }
-            }
-            bool pending = false;
-            for (int tr = 0; tr < 2; ++tr) pending |= (state[tr] == 2 || state[tr] == 3 || state[tr] == 4);
-            if (!pending) break;
-        }
-        if (!alive) break;
-
-        // ---- write each track's list
-        for (int tr = 0; tr < 2; ++tr) {
-            const int r = p.r[tr];
-            if (r <= 0) continue;
-            int32_t* outp = p.out[tr] + (size_t)u * r;
-            int base_off = 0;
-            uint64_t kcut = 0;         // cand: select comp_key >= kcut
-            uint64_t ecut = 0;         // eq: select ext > ecut, or == with quota
-            int quota = 0;
-            const int st = state[tr];
-            if (st == 1) {
-                base_off = lo;   // every candidate is taken; valid entries are a prefix
-            } else if (st == 5) {
-                // exact cut among the candidates
-                uint64_t* keys = reinterpret_cast<uint64_t*>(&S.stage[0][0]);
-                const int Cn = C[tr];
-                int np2 = 1;
-                while (np2 < Cn) np2 <<= 1;
-                for (int i = tid; i < np2; i += kIdxThreads) {
-                    if (i < Cn) {
-                        const int2 cv = __ldcg(cand + tr * kCandCap + i);
-                        keys[i] = comp_key(cv.x, cv.y);
-                    } else {
-                        keys[i] = 0;
-                    }
-                }
-                __syncthreads();
-                bitonic_desc(keys, np2);
-                kcut = keys[rrem[tr] - 1];
-                int before = 0;
-                for (int i = tid; i < Cn; i += kIdxThreads) {
-                    const int idx = 0x7FFFFFF - (int)(keys[i] & 0x7FFFFFFull);
-                    before += (keys[i] >= kcut && idx < lo);
-                }
-                before = block_sum(before, S.red);
-                int prev = 0;
-                for (int c2 = 0; c2 < cta; ++c2) prev += __ldcg(pub + (tr * 2 + 0) * kMaxG + c2);
-                base_off = prev + before;
-            } else if (st == 6) {
-                ecut = prefix[tr];
-                int prev = 0, eqb = 0;
-                for (int c2 = 0; c2 < cta; ++c2) {
-                    prev += __ldcg(pub + (tr * 2 + 0) * kMaxG + c2);
-                    eqb += __ldcg(pub + (tr * 2 + 1) * kMaxG + c2);
-                }
-                const int my_eq = __ldcg(pub + (tr * 2 + 1) * kMaxG + cta);
-                quota = max(0, min(rrem[tr] - eqb, my_eq));
-                base_off = prev + min(rrem[tr], eqb);
-            }
-            // ordered compaction: thread tid owns elements [tid*R, tid*R+R)
-            const int R = (my_n + kIdxThreads - 1) / kIdxThreads;
-            const int e0 = min(tid * R, my_n), e1 = min(e0 + R, my_n);
-            int cnt = 0, ceq = 0;
-            for (int e = e0; e < e1; ++e) {
-                const int x = sc[skew(e)];
-                if (st == 1) cnt++;
-                else if (st == 5) cnt += comp_key(x, lo + e) >= kcut;
-                else {
-                    const uint64_t ek = ext_key(x);
-                    cnt += ek > ecut;
-                    ceq += ek == ecut;
-                }
-            }
-            int tot;
-            int eq_excl = 0;
-            if (st == 6) eq_excl = block_scan_excl(ceq, S.red, tot);
-            const int eq_take = (st == 6) ? max(0, min(quota - eq_excl, ceq)) : 0;
-            const int off = base_off + block_scan_excl(cnt + eq_take, S.red, tot);
-            int k2 = off, eq_seen = 0;
-            for (int e = e0; e < e1; ++e) {
-                const int x = sc[skew(e)];
-                bool sel;
-                if (st == 1) sel = true;
-                else if (st == 5) sel = comp_key(x, lo + e) >= kcut;
-                else {
-                    const uint64_t ek = ext_key(x);
-                    sel = ek > ecut;
-                    if (ek == ecut) { sel = eq_seen < eq_take; eq_seen++; }
-                }
-                if (sel) {
-                    const int pos = full ? (lo + e) : pool[lo + e];
-                    if (k2 < r) outp[k2] = pos;
-                    k2++;
-                }
-            }
-            // padding: entries [min(r, n_total), r) = -1
-            if (cta == p.G - 1) {
-                for (int i = min(r, n_total) + tid; i < r; i += kIdxThreads) outp[i] = -1;
-            }
-            __syncthreads();
-        }
+        UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
+        alive = select_unit(p, S, sl, c, bar_target, sc);
+        __syncthreads();
     }
-    // persist the slot state for the next launch
     if (alive && cta == 0 && tid == 0) {
-        ctrl[CTRL_EPOCH] = epoch + j;
-        ctrl[CTRL_BAR_BASE] = bar_target;
+        sl.ctrl[CTRL_EPOCH] = epoch + j;
+        sl.ctrl[CTRL_BAR_BASE] = bar_target;
     }
 }
 
@@ -705,7 +985,7 @@ IdxRegion idx_region(int slots) {
     r.off_g0 = off;   off += align_up((size_t)slots * 3 * kBins * 4, 256);
     r.off_gl = off;   off += align_up((size_t)slots * 4 * kBins * 4, 256);
     r.off_cand = off; off += align_up((size_t)slots * 2 * kCandCap * 8, 256);
-    r.off_pub = off;  off += align_up((size_t)slots * 4 * kMaxG * 4, 256);
+    r.off_pub = off;  off += align_up((size_t)slots * 6 * kMaxG * 4, 256);
     r.bytes = off;
     return r;
 }
@@ -734,15 +1014,15 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
 
 size_t index_smem_bytes() { return sizeof(IdxSmem) + 1024; }
 
-template <int HI, int DI>
-static cudaError_t launch_variant(const IdxParams& p, const CUtensorMap& map, int grid, cudaStream_t stream) {
-    auto kern = index_select_kernel<HI, DI>;
+template <typename Kern>
+static cudaError_t launch_coop(Kern kern, int threads, const IdxParams& p, const CUtensorMap& map, int grid,
+                               cudaStream_t stream) {
     const size_t smem = index_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kIdxThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -803,9 +1083,12 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
     }
     const int grid = pl.groups * pl.G;
     cudaError_t e;
-    if (a.Hi <= 8 && a.Di == 64) e = launch_variant<8, 64>(p, map, grid, stream);
-    else if (a.Hi <= 4 && a.Di == 32) e = launch_variant<4, 32>(p, map, grid, stream);
-    else e = launch_variant<0, 0>(p, map, grid, stream);
+    if (a.mode == CSA2_FULL && a.Di == 64) e = launch_coop(index_full_tc_kernel<64>, kTcThreads, p, map, grid, stream);
+    else if (a.mode == CSA2_FULL && a.Di == 32) e = launch_coop(index_full_tc_kernel<32>, kTcThreads, p, map, grid, stream);
+    else if (a.mode == CSA2_FULL && a.Di == 128) e = launch_coop(index_full_tc_kernel<128>, kTcThreads, p, map, grid, stream);
+    else if (a.Hi <= 8 && a.Di == 64) e = launch_coop(index_dp4a_kernel<8, 64>, kSel, p, map, grid, stream);
+    else if (a.Hi <= 4 && a.Di == 32) e = launch_coop(index_dp4a_kernel<4, 32>, kSel, p, map, grid, stream);
+    else e = launch_coop(index_dp4a_kernel<0, 0>, kSel, p, map, grid, stream);
     return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }
 
