@@ -294,7 +294,7 @@ def run_ours(args, rank, world, local_rank):
         pass
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                "kernel": "index_select_kernel<8,64> (Full mode, layer 0)",
+                "kernel": "index_full_tc_kernel<64> (Full mode, layer 0: scan + exact pool/top-k select)",
                 "kernel_ms": round(kern_ms, 4), "algorithmic_bytes": kbytes,
                 "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback 6650 GB/s"}
     step_bytes = unit_bytes(s) * units

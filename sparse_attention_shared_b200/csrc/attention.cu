@@ -18,7 +18,10 @@
 // as an M-major operand. Partials go to the workspace; the last CTA of the
 // query (atomic ticket, no waiting) merges them by log-sum-exp and writes the
 // bf16 output and the fp32 log-sum-exp.
+#include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <cstring>
 
 #include "csa2_common.cuh"
 
@@ -83,7 +86,7 @@ template <int HQP, int D>
 __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_constant__ AttnParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     AttnSmem<HQP>& S =
-        *reinterpret_cast<AttnSmem<HQP>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+        *reinterpret_cast<AttnSmem<HQP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     constexpr uint32_t kCols = (2 * HQP < 32) ? 32 : 2 * HQP;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int tau = blockIdx.x;
@@ -400,6 +403,312 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
     if (warp == 0) tmem_dealloc(tmem, kCols);
 }
 
+// ------------------------------------------------------------ clustered variant
+// One thread-block cluster per query: CTA r < ngt2 takes 256 entries of the
+// global list (two 128-row MMA blocks), the others one 128-row tile of the
+// window each. Every CTA issues all of its loads at once (the list entries,
+// then its FP4 rows; local tiles by TMA), computes its softmax partial on the
+// tensor cores, parks it in shared memory, and the cluster merges the
+// partials through distributed shared memory: CTA r writes the heads
+// h = r, r + CS, ... . No partial goes through global memory.
+constexpr int kCLBuf = 4 * kPanelBytes;   // 64 KB: a 256-row global tile or a local K+V tile
+
+template <int HQP>
+struct __align__(1024) AttnClSmem {
+    uint8_t tbuf[kCLBuf];
+    uint8_t qbuf[2 * HQP * 128];
+    uint8_t pbuf[4 * HQP * 128];          // P as [HQP rows x 256 keys] in 64-key panels
+    uint32_t lut[256];
+    float red[4][HQP];
+    float part_m[HQP], part_l[HQP];
+    uint64_t bar_tma, bar_s, bar_o;
+    uint32_t tmem_base;
+};
+
+template <int HQP, int D>
+__global__ void __launch_bounds__(kAttnThreads)
+    sparse_attn_cl_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap kl_map,
+                          const __grid_constant__ CUtensorMap vl_map) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    AttnClSmem<HQP>& S =
+        *reinterpret_cast<AttnClSmem<HQP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    constexpr uint32_t kCols = (3 * HQP <= 32) ? 32 : (3 * HQP <= 64 ? 64 : 128);
+    constexpr int kPanels = D / 64;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int CS = gridDim.x;
+    const int rank = (int)cluster_ctarank();
+    const int u = blockIdx.y;
+    const int b = u / p.Tq;
+    const int ngt2 = (p.k + 2 * kTileKeys - 1) / (2 * kTileKeys);
+    const bool glob = rank < ngt2;
+    float* part_o = reinterpret_cast<float*>(S.tbuf);      // [HQP][D] once the MMAs are done
+
+    // ---- 1. loads that depend on nothing
+    int t = p.q_pos[u];
+    const int base = p.local_base[b];
+    int s0 = -1, s1 = -1;
+    if (glob) {
+        const int j0 = rank * 2 * kTileKeys + tid, j1 = j0 + kTileKeys;
+        s0 = (j0 < p.k) ? p.topk[(size_t)u * p.k + j0] : -1;
+        s1 = (j1 < p.k) ? p.topk[(size_t)u * p.k + j1] : -1;
+    }
+    uint4 qv[(HQP * D / 8 + kAttnThreads - 1) / kAttnThreads];
+#pragma unroll
+    for (int q = 0; q < (int)(sizeof(qv) / sizeof(qv[0])); ++q) {
+        const int i = tid + q * kAttnThreads;
+        const int h = i / (D / 8), c = i % (D / 8);
+        qv[q] = make_uint4(0, 0, 0, 0);
+        if (i < HQP * (D / 8) && h < p.Hq) qv[q] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
+    }
+    if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
+    if (tid == 0) {
+        mbar_init(&S.bar_tma, 1);
+        mbar_init(&S.bar_s, 1);
+        mbar_init(&S.bar_o, 1);
+        mbar_fence_init();
+    }
+    if (t < 0 || t >= p.N) {
+        if (tid == 0 && rank == 0) report(p.status, CSA2_ERR_RANGE, u);
+        t = -1;
+    }
+    const int lo_w = max(max(base, t - p.W + 1), 0);
+
+    // ---- 2. the tile's rows
+    bool v0 = false, v1 = false;
+    uint4 c0[D / 32], c1[D / 32];
+    uint32_t sc0[D / 64], sc1[D / 64];
+    if (glob) {
+        if (s0 >= 0 && (s0 > t || s0 >= p.N)) { report(p.status, CSA2_ERR_RANGE, u); s0 = -1; }
+        if (s1 >= 0 && (s1 > t || s1 >= p.N)) { report(p.status, CSA2_ERR_RANGE, u); s1 = -1; }
+        v0 = s0 >= 0;
+        v1 = s1 >= 0;
+        auto ldrow = [&](int s, uint4 (&cw)[D / 32], uint32_t (&sw)[D / 64]) {
+            const size_t row = (size_t)b * p.N + s;
+            const uint4* cp = reinterpret_cast<const uint4*>(p.kv_fp4 + row * (D / 2));
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) cw[q] = __ldg(cp + q);
+            if (D == 128) {
+                const uint2 s2 = __ldg(reinterpret_cast<const uint2*>(p.kv_scale + row * 8));
+                sw[0] = s2.x;
+                sw[(D / 64) - 1] = s2.y;
+            } else {
+                sw[0] = __ldg(reinterpret_cast<const uint32_t*>(p.kv_scale + row * 4));
+            }
+        };
+        if (v0) ldrow(s0, c0, sc0);
+        if (v1) ldrow(s1, c1, sc1);
+    } else {
+        const int lt = rank - ngt2;
+        const int pos = lo_w + lt * kTileKeys + tid;
+        v0 = (t >= 0) && (p.W > 0) && (pos <= t) && (pos - base) < p.Lloc;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&S.bar_tma, 2u * kPanels * kPanelBytes);
+            const int y = lo_w - base + lt * kTileKeys;
+#pragma unroll
+            for (int pn = 0; pn < kPanels; ++pn) {
+                tma_load_3d(S.tbuf + pn * kPanelBytes, &kl_map, pn * 64, y, b, &S.bar_tma);
+                tma_load_3d(S.tbuf + 2 * kPanelBytes + pn * kPanelBytes, &vl_map, pn * 64, y, b, &S.bar_tma);
+            }
+        }
+    }
+    for (int i = tid; i < 256; i += kAttnThreads)
+        S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
+#pragma unroll
+    for (int q = 0; q < (int)(sizeof(qv) / sizeof(qv[0])); ++q) {
+        const int i = tid + q * kAttnThreads;
+        const int h = i / (D / 8), c = i % (D / 8);
+        if (i < HQP * (D / 8)) *reinterpret_cast<uint4*>(S.qbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = qv[q];
+    }
+    if (glob && D == 64) {   // the value operand's second M-half stays zero
+        for (int i = tid; i < 2 * kPanelBytes / 16; i += kAttnThreads)
+            reinterpret_cast<uint4*>(S.tbuf + 2 * kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
+    }
+    if (!glob && D == 64) {
+        for (int i = tid; i < kPanelBytes / 16; i += kAttnThreads) {
+            reinterpret_cast<uint4*>(S.tbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(S.tbuf + 3 * kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    __syncthreads();   // the table is ready
+    bool ok = true;
+    if (glob) {
+        // global tile panels hold 256 rows: panel p at p * 2 * kPanelBytes
+        auto dequant = [&](int r, bool v, const uint4 (&cw)[D / 32], const uint32_t (&sw)[D / 64]) {
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+                uint4 o = make_uint4(0, 0, 0, 0);
+                if (v) {
+                    const uint4 w4 = cw[c >> 2];
+                    const uint32_t w = (c & 3) == 0 ? w4.x : (c & 3) == 1 ? w4.y : (c & 3) == 2 ? w4.z : w4.w;
+                    const uint32_t g = c >> 1;
+                    const uint32_t s16 = e4m3_bf16_bits((sw[g >> 2] >> (8 * (g & 3))) & 0xFFu);
+                    const uint32_t s2x = s16 | (s16 << 16);
+                    o.x = bf16x2_mul(S.lut[w & 0xFFu], s2x);
+                    o.y = bf16x2_mul(S.lut[(w >> 8) & 0xFFu], s2x);
+                    o.z = bf16x2_mul(S.lut[(w >> 16) & 0xFFu], s2x);
+                    o.w = bf16x2_mul(S.lut[w >> 24], s2x);
+                }
+                *reinterpret_cast<uint4*>(S.tbuf + (c >> 3) * (2 * kPanelBytes) + sw128(r, c & 7)) = o;
+            }
+        };
+        dequant(tid, v0, c0, sc0);
+        dequant(tid + kTileKeys, v1, c1, sc1);
+    } else {
+        ok = mbar_wait(&S.bar_tma, 0, p.status, 12);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int nblk = glob ? 2 : 1;
+    const uint32_t panel_stride = glob ? 2 * kPanelBytes : kPanelBytes;
+
+    // ---- 3. S = K Q^T per 128-row block
+    if (tid == 0) {
+        const uint32_t ka = smem_u32(S.tbuf), qa = smem_u32(S.qbuf);
+        constexpr uint32_t idesc = idesc_bf16(128, HQP, 0);
+        for (int blk = 0; blk < nblk; ++blk) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t ad = smem_desc(ka + (kk >> 2) * panel_stride + blk * kPanelBytes + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = smem_desc(qa + (kk >> 2) * (HQP * 128) + (kk & 3) * 32, 16, 1024);
+                mma_bf16(tmem + blk * HQP, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+        }
+        mma_commit(&S.bar_s);
+    }
+    ok = mbar_wait(&S.bar_s, 0, p.status, 10) && ok;
+    tc_fence_after();
+
+    // ---- 4. softmax partial over the tile's rows (two rows per thread on a global tile)
+    float a0[HQP], a1[HQP];
+    {
+        float tmp[16];
+#pragma unroll
+        for (int c0i = 0; c0i < HQP; c0i += 16) {
+            tmem_ld16(tmem + lane_off + c0i, tmp);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) a0[c0i + q] = tmp[q];
+            if (glob) {
+                tmem_ld16(tmem + HQP + lane_off + c0i, tmp);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) a1[c0i + q] = tmp[q];
+            }
+        }
+    }
+    const bool r0 = v0 && ok, r1 = glob && v1 && ok;
+#pragma unroll
+    for (int h = 0; h < HQP; ++h) {
+        a0[h] = r0 ? a0[h] * p.scale_log2 : -INFINITY;
+        a1[h] = r1 ? a1[h] * p.scale_log2 : -INFINITY;
+    }
+    float mh[HQP];
+#pragma unroll
+    for (int h = 0; h < HQP; ++h) {
+        float m = fmaxf(a0[h], a1[h]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        mh[h] = m;
+    }
+    if ((tid & 31) == 0) {
+#pragma unroll
+        for (int h = 0; h < HQP; ++h) S.red[warp][h] = mh[h];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < HQP; ++h) mh[h] = fmaxf(fmaxf(S.red[0][h], S.red[1][h]), fmaxf(S.red[2][h], S.red[3][h]));
+    __syncthreads();
+    float lh[HQP];
+#pragma unroll
+    for (int h = 0; h < HQP; ++h) {
+        const bool live = mh[h] != -INFINITY;
+        const float p0 = (r0 && live) ? exp2f(a0[h] - mh[h]) : 0.f;
+        const float p1 = (r1 && live) ? exp2f(a1[h] - mh[h]) : 0.f;
+        // key k -> panel k / 64, column k % 64
+        *reinterpret_cast<__nv_bfloat16*>(S.pbuf + (tid >> 6) * (HQP * 128) + sw128(h, (tid & 63) >> 3) + (tid & 7) * 2) =
+            __float2bfloat16_rn(p0);
+        *reinterpret_cast<__nv_bfloat16*>(S.pbuf + (2 + (tid >> 6)) * (HQP * 128) + sw128(h, (tid & 63) >> 3) +
+                                          (tid & 7) * 2) = __float2bfloat16_rn(p1);
+        float l = p0 + p1;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        lh[h] = l;
+    }
+    if ((tid & 31) == 0) {
+#pragma unroll
+        for (int h = 0; h < HQP; ++h) S.red[warp][h] = lh[h];
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+#pragma unroll
+    for (int h = 0; h < HQP; ++h) lh[h] = S.red[0][h] + S.red[1][h] + S.red[2][h] + S.red[3][h];
+
+    // ---- 5. O^T = V^T P (keys as the reduction; the head dim as M)
+    if (tid == 0) {
+        const uint32_t va = smem_u32(glob ? S.tbuf : S.tbuf + 2 * kPanelBytes), pa = smem_u32(S.pbuf);
+        constexpr uint32_t idesc = idesc_bf16(128, HQP, 1);
+        const int nk = nblk * (kTileKeys / 16);
+        for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t ad = smem_desc(va + kk * 2048, panel_stride, 1024);
+            const uint64_t bd = smem_desc(pa + (kk >> 2) * (HQP * 128) + (kk & 3) * 32, 16, 1024);
+            mma_bf16(tmem + 2 * HQP, ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&S.bar_o);
+    }
+    ok = mbar_wait(&S.bar_o, 0, p.status, 11) && ok;
+    tc_fence_after();
+    float ov[HQP];
+    {
+        float tmp[16];
+#pragma unroll
+        for (int c0i = 0; c0i < HQP; c0i += 16) {
+            tmem_ld16(tmem + 2 * HQP + lane_off + c0i, tmp);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) ov[c0i + q] = tmp[q];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();    // every MMA operand read is done: the tile buffer holds the partial now
+    if (tid < D) {
+#pragma unroll
+        for (int h = 0; h < HQP; ++h) part_o[h * D + tid] = ok ? ov[h] : 0.f;
+    }
+    if (tid == 0) {
+#pragma unroll
+        for (int h = 0; h < HQP; ++h) { S.part_m[h] = ok ? mh[h] : -INFINITY; S.part_l[h] = ok ? lh[h] : 0.f; }
+    }
+
+    // ---- 6. merge the cluster's partials through distributed shared memory
+    cluster_sync_all();
+    for (int h = rank; h < p.Hq; h += CS) {
+        float M = -INFINITY;
+        for (int c = 0; c < CS; ++c) M = fmaxf(M, ld_dsmem(dsmem_addr(&S.part_m[h], c)));
+        float L = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+            for (int c = 0; c < CS; ++c) {
+                const float mc = ld_dsmem(dsmem_addr(&S.part_m[h], c));
+                if (mc == -INFINITY) continue;
+                const float wgt = exp2f(mc - M);
+                L += wgt * ld_dsmem(dsmem_addr(&S.part_l[h], c));
+                if (tid < D) acc += wgt * ld_dsmem(dsmem_addr(&part_o[h * D + tid], c));
+            }
+        }
+        if (tid < D)
+            p.out[((size_t)u * p.Hq + h) * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(L > 0.f ? acc / L : 0.f));
+        if (tid == 0 && p.lse != nullptr)
+            p.lse[(size_t)u * p.Hq + h] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+    }
+    cluster_sync_all();   // no CTA leaves while others read its shared memory
+    if (warp == 0) tmem_dealloc(tmem, kCols);
+}
+
 // ------------------------------------------------------------ host side
 struct AttnPlan {
     int units, ngt, nlt, ntiles, HQP;
@@ -453,5 +762,105 @@ csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* ticke
 }
 
 size_t attn_scratch_bytes(const csa2_attn_args& a) { return plan_attn(a).part_bytes; }
+
+}  // namespace csa2
+
+namespace csa2 {
+
+typedef CUresult (*EncodeTiledFnA)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFnA encode_fn() {
+    static EncodeTiledFnA fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFnA>(ptr);
+    }
+    return fn;
+}
+
+// [B, Lloc, D] bf16 local K or V as a 3-D map with 128-row x 64-element boxes,
+// 128-byte swizzle (the tcgen05 operand layout).
+static bool encode_local_map(CUtensorMap* m, const uint16_t* ptr, int B, int Lloc, int D) {
+    EncodeTiledFnA enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Lloc, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Lloc * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int HQP, int D>
+static cudaError_t launch_cl_variant(const AttnParams& p, const CUtensorMap& km, const CUtensorMap& vm, int cs,
+                                     int units, cudaStream_t stream) {
+    auto kern = sparse_attn_cl_kernel<HQP, D>;
+    const size_t smem = sizeof(AttnClSmem<HQP>) + 1024;
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
+    if (e != cudaSuccess) return e;
+    if (cs > 8) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(cs, units);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p, km, vm);
+}
+
+// Clustered attention: one cluster of ceil(k/256) + ceil(W/128) <= 16 CTAs per
+// query; false when the call needs more CTAs than a cluster holds.
+bool attn_cluster_fits(const csa2_attn_args& a) {
+    const int cs = (a.k + 2 * kTileKeys - 1) / (2 * kTileKeys) + (a.W + kTileKeys - 1) / kTileKeys;
+    return cs >= 1 && cs <= 16 && (int64_t)a.B * a.Tq <= 65535;
+}
+
+csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int32_t* d_status,
+                                cudaStream_t stream) {
+    const int units = a.B * a.Tq;
+    if (units == 0) return CSA2_OK;
+    AttnParams p{};
+    p.B = a.B; p.Tq = a.Tq; p.N = a.N; p.Hq = a.Hq; p.D = a.D; p.k = a.k; p.W = a.W; p.Lloc = a.Lloc;
+    const int ngt2 = (a.k + 2 * kTileKeys - 1) / (2 * kTileKeys);
+    p.nlt = (a.W + kTileKeys - 1) / kTileKeys;
+    p.ngt = ngt2;
+    p.ntiles = ngt2 + p.nlt;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)a.D));
+    p.q_pos = a.q_pos; p.q = a.q; p.kv_fp4 = a.kv_fp4; p.kv_scale = a.kv_scale; p.topk = topk;
+    p.kl = a.kl; p.vl = a.vl; p.local_base = a.local_base; p.out = a.out; p.lse = a.lse;
+    p.part = nullptr;
+    p.tickets = nullptr;
+    p.status = d_status;
+    CUtensorMap km, vm;
+    memset(&km, 0, sizeof(km));
+    memset(&vm, 0, sizeof(vm));
+    if (a.W > 0) {
+        if (!encode_local_map(&km, a.kl, a.B, a.Lloc, a.D) || !encode_local_map(&vm, a.vl, a.B, a.Lloc, a.D))
+            return CSA2_ERR_CUDA;
+    }
+    const int HQP = a.Hq <= 16 ? 16 : 32;
+    const int cs = p.ntiles;
+    cudaError_t e;
+    if (HQP == 16 && a.D == 128) e = launch_cl_variant<16, 128>(p, km, vm, cs, units, stream);
+    else if (HQP == 16 && a.D == 64) e = launch_cl_variant<16, 64>(p, km, vm, cs, units, stream);
+    else if (HQP == 32 && a.D == 128) e = launch_cl_variant<32, 128>(p, km, vm, cs, units, stream);
+    else e = launch_cl_variant<32, 64>(p, km, vm, cs, units, stream);
+    return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
 
 }  // namespace csa2

@@ -32,6 +32,8 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
 size_t attn_scratch_bytes(const csa2_attn_args& a);
 csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* tickets, void* scratch,
                         int32_t* d_status, cudaStream_t stream);
+bool attn_cluster_fits(const csa2_attn_args& a);
+csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int32_t* d_status, cudaStream_t stream);
 // fp4_quant.cu
 cudaError_t launch_fp4_quantize(const float* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales,
                                 cudaStream_t stream);
@@ -198,6 +200,7 @@ csa2_status csa2_sparse_attn(const csa2_attn_args* args, void* workspace, size_t
         a.local_base = a.q_pos;
         a.Lloc = 0;
     }
+    if (attn_cluster_fits(a)) return launch_attn_cluster(a, a.topk, d_status, static_cast<cudaStream_t>(stream));
     return launch_attn(a, a.topk, tickets, scratch, d_status, static_cast<cudaStream_t>(stream));
 }
 
@@ -245,7 +248,8 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
             a.local_base = a.q_pos;
             a.Lloc = 0;
         }
-        st = launch_attn(a, cur, tickets, scratch, d_status, strm);
+        st = attn_cluster_fits(a) ? launch_attn_cluster(a, cur, d_status, strm)
+                                  : launch_attn(a, cur, tickets, scratch, d_status, strm);
         if (st != CSA2_OK) return st;
     }
     return CSA2_OK;

@@ -90,8 +90,8 @@ struct __align__(1024) IdxSmem {
     uint64_t tempty_bar[kTmemBufs];
     uint32_t tmem_base;
     int abort;
-    int red[64];
-    int info[64];
+    alignas(16) int red[64];
+    alignas(16) int info[64];
 };
 static_assert(2 * sizeof(int2) * kCandCap <= sizeof(((IdxSmem*)0)->stage), "candidate buffers");
 static_assert(kStages * kStageBytes % 1024 == 0, "tensor-core operand alignment");
@@ -145,6 +145,11 @@ __device__ __forceinline__ uint64_t ext_key(int32_t x) {
 
 __device__ __forceinline__ uint32_t digit_at(uint64_t ext, int level) {
     return (uint32_t)(ext >> (24 - 12 * level)) & 4095u;
+}
+
+// Rare path, kept out of line: does x match a deeper (level >= 1) digit prefix?
+__device__ __noinline__ bool deep_prefix_match(int x, int shift, uint64_t prefix) {
+    return (ext_key(x) >> shift) == prefix;
 }
 
 // Level-0 digit only (the 12-bit log-scale bin of the score).
@@ -231,12 +236,13 @@ __device__ __forceinline__ int sel_min(int v, int* red) {
 }
 
 // Group barrier over the G CTAs of a slot: the counter grows by one per CTA.
+// The arrival is a release add (it publishes this CTA's earlier writes, which the
+// named barrier has ordered before it) and the poll an acquire load.
 __device__ bool group_barrier(int* counter, int target, int32_t* st) {
     sel_sync();
     int ok = 1;
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(counter, 1);
+        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter) : "memory");
         if (ld_acquire_gpu(counter) < target) {
             const long long t0 = clock64();
             while (ld_acquire_gpu(counter) < target) {
@@ -245,12 +251,40 @@ __device__ bool group_barrier(int* counter, int target, int32_t* st) {
                     ok = 0;
                     break;
                 }
-                __nanosleep(32);
+                __nanosleep(20);
             }
         }
-        __threadfence();
     }
     return sel_and(ok) != 0;
+}
+
+// Four exclusive scans at once over the select threads (totals in `total`).
+__device__ __forceinline__ int4 sel_scan4(int4 v, int* red, int4& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int4 x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, x.x, o), b = __shfl_up_sync(0xffffffffu, x.y, o);
+        const int c = __shfl_up_sync(0xffffffffu, x.z, o), d = __shfl_up_sync(0xffffffffu, x.w, o);
+        if (lane >= o) { x.x += a; x.y += b; x.z += c; x.w += d; }
+    }
+    sel_sync();
+    if (lane == 31) reinterpret_cast<int4*>(red)[warp] = x;
+    sel_sync();
+    if (warp == 0) {
+        int4 s = lane < (kSel / 32) ? reinterpret_cast<int4*>(red)[lane] : make_int4(0, 0, 0, 0);
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, s.x, o), b = __shfl_up_sync(0xffffffffu, s.y, o);
+            const int c = __shfl_up_sync(0xffffffffu, s.z, o), d = __shfl_up_sync(0xffffffffu, s.w, o);
+            if (lane >= o) { s.x += a; s.y += b; s.z += c; s.w += d; }
+        }
+        if (lane < kSel / 32) reinterpret_cast<int4*>(red)[8 + lane] = s;
+    }
+    sel_sync();
+    const int4 we = warp ? reinterpret_cast<int4*>(red)[8 + warp - 1] : make_int4(0, 0, 0, 0);
+    total = reinterpret_cast<int4*>(red)[8 + kSel / 32 - 1];
+    return make_int4(we.x + x.x - v.x, we.y + x.y - v.y, we.z + x.z - v.z, we.w + x.w - v.w);
 }
 
 // In a 4096-bin histogram (global or shared), find the bin holding the r-th
@@ -290,6 +324,41 @@ __device__ void find_rank_bin(const int* hist, int r, int* red, int* out) {
     sel_sync();
 }
 
+// Both tracks' rank bins in one pass over a global 4096-bin histogram: for rank
+// r[k] > 0 writes {bin, count above, count in bin} to out[8k..8k+2].
+__device__ void find_rank_bins2(const int* hist, const int* r, int* red, int* out) {
+    const int t = threadIdx.x;
+    int h[16];
+    const int4* src = reinterpret_cast<const int4*>(hist + 16 * t);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int4 v = __ldcg(src + i);
+        h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
+    }
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s += h[i];
+    int total;
+    const int excl = sel_scan_excl(s, red, total);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int rk = r[k];
+        int above = total - excl - s;
+        if (rk > 0 && above < rk && rk <= above + s) {
+#pragma unroll
+            for (int i = 15; i >= 0; --i) {
+                if (above < rk && rk <= above + h[i]) {
+                    out[8 * k + 0] = 16 * t + i;
+                    out[8 * k + 1] = above;
+                    out[8 * k + 2] = h[i];
+                }
+                above += h[i];
+            }
+        }
+    }
+    sel_sync();
+}
+
 // Push the non-zero bins of a shared histogram into a global one.
 __device__ __forceinline__ void push_hist(const int* sh, int* gh) {
     for (int i = threadIdx.x; i < kBins; i += kSel) {
@@ -311,14 +380,19 @@ __device__ __forceinline__ int prefix_total(const int* arr, int n, int* red) {
 }
 
 // The r-th largest value (1-based, with multiplicity) of cx[0..C) in shared
-// memory, by 12-bit radix passes over x - min. Returns T; need_eq = how many of
-// the elements equal to T are ranked within the first r.
-__device__ int local_select(const int* cx, int C, int r, int* hist, int* red, int* info, int& need_eq) {
-    int mn = INT_MAX, mx = INT_MIN;
-    for (int i = threadIdx.x; i < C; i += kSel) { mn = min(mn, cx[i]); mx = max(mx, cx[i]); }
-    mn = sel_min(mn, red);
-    mx = -sel_min(-mx, red);
-    const uint32_t w = (uint32_t)((long long)mx - (long long)mn);
+// memory, by 12-bit radix passes over x - lo. [lo, hi] bounds the values (pass
+// hi < lo to compute the bounds here). Returns T; need_eq = how many of the
+// elements equal to T are ranked within the first r.
+__device__ int local_select(const int* cx, int C, int r, int lo, int hi, int* hist, int* red, int* info,
+                            int& need_eq) {
+    if (hi < lo) {
+        int mn = INT_MAX, mx = INT_MIN;
+        for (int i = threadIdx.x; i < C; i += kSel) { mn = min(mn, cx[i]); mx = max(mx, cx[i]); }
+        lo = sel_min(mn, red);
+        hi = -sel_min(-mx, red);
+    }
+    const int mn = lo;
+    const uint32_t w = (uint32_t)((long long)hi - (long long)lo);
     int rem = (w == 0u) ? 0 : 32 - __clz(w);
     uint32_t prefix = 0;
     while (rem > 0) {
@@ -350,10 +424,13 @@ struct UnitCtx {
 };
 
 // Exact pool/top-k cut for one unit and the write of this CTA's selected
-// positions. Runs on threads [0, kSel). The chunk's scores are in sc (skewed
-// index) and their level-0 histogram in S.hist0. Returns false on a timeout.
+// positions. Runs on threads [0, kSel). The chunk's scores are in S.sc or spill (skewed
+// index) and their level-0 histogram in S.hist0. The two tracks (pool P and
+// top-k) share every pass and every group barrier. Returns false on a timeout.
 __device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c, int& bar_target,
-                            const int* sc) {
+                            const int* spill) {
+    // a chunk's scores live in shared memory unless they were spilled to the workspace
+    auto sc_at = [&](int e) -> int { return spill ? spill[skew(e)] : S.sc[skew(e)]; };
     const int tid = threadIdx.x;
     const bool full = p.mode == CSA2_FULL;
     const int lo = c.lo, my_n = c.my_n;
@@ -384,25 +461,96 @@ __device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, cons
     }
     int state[2], rrem[2], C[2], level[2], above_loc[2], clo[2], chi[2];
     uint64_t prefix[2];
+    int rq[2];
     for (int tr = 0; tr < 2; ++tr) {
         state[tr] = TS_OFF; rrem[tr] = 0; C[tr] = 0; level[tr] = 0; above_loc[tr] = 0; prefix[tr] = 0;
         clo[tr] = 0; chi[tr] = -1;
         const int r = p.r[tr];
+        rq[tr] = 0;
         if (r <= 0) continue;
         if (n_total <= r) { state[tr] = TS_ALL; continue; }
-        find_rank_bin<true>(g0cur, r, S.red, S.info + 8 * tr);
-        const int d = S.info[8 * tr + 0];
-        rrem[tr] = r - S.info[8 * tr + 1];
-        C[tr] = S.info[8 * tr + 2];
-        prefix[tr] = (uint64_t)d;
-        above_loc[tr] = sel_sum(sum_above(S.hist0, d), S.red);
-        bin0_interval((uint32_t)d, clo[tr], chi[tr]);
-        state[tr] = (C[tr] <= kCandCap) ? TS_CAND : TS_RADIX;
+        rq[tr] = r;
+    }
+    if (rq[0] > 0 || rq[1] > 0) {
+        find_rank_bins2(g0cur, rq, S.red, S.info);
+        int a0 = 0, a1 = 0;
+        const int d0 = S.info[0], d1 = S.info[8];
+        for (int i = tid; i < kBins; i += kSel) {
+            const int v = S.hist0[i];
+            a0 += (rq[0] > 0 && i > d0) ? v : 0;
+            a1 += (rq[1] > 0 && i > d1) ? v : 0;
+        }
+        int4 tot;
+        sel_scan4(make_int4(a0, a1, 0, 0), S.red, tot);
+        for (int tr = 0; tr < 2; ++tr) {
+            if (rq[tr] <= 0) continue;
+            const int d = S.info[8 * tr + 0];
+            rrem[tr] = rq[tr] - S.info[8 * tr + 1];
+            C[tr] = S.info[8 * tr + 2];
+            prefix[tr] = (uint64_t)d;
+            above_loc[tr] = tr == 0 ? tot.x : tot.y;
+            bin0_interval((uint32_t)d, clo[tr], chi[tr]);
+            state[tr] = (C[tr] <= kCandCap) ? TS_CAND : TS_RADIX;
+        }
     }
 
     // ---- rounds until every track knows its cut (usually one)
     while (true) {
         bool any = false;
+        // fused candidate gather for every track in TS_CAND: compact in shared
+        // memory, reserve a range of the group buffer with one atomic, copy out
+        const bool g0on = state[0] == TS_CAND, g1on = state[1] == TS_CAND;
+        if (g0on || g1on) {
+            any = true;
+            int2* lbuf = reinterpret_cast<int2*>(&S.stage[0][0]);
+            // per-track bounds as scalars (no indexed arrays in the loops)
+            const int lo0 = clo[0], hi0 = chi[0], lo1 = clo[1], hi1 = chi[1];
+            const bool deep0 = level[0] > 0, deep1 = level[1] > 0;
+            const int sh0 = 24 - 12 * level[0], sh1 = 24 - 12 * level[1];
+            const uint64_t pf0 = prefix[0], pf1 = prefix[1];
+            auto is_cand = [&](int x, bool& m0, bool& m1) {
+                m0 = g0on && x >= lo0 && x <= hi0;
+                m1 = g1on && x >= lo1 && x <= hi1;
+                if (deep0 && m0) m0 = deep_prefix_match(x, sh0, pf0);
+                if (deep1 && m1) m1 = deep_prefix_match(x, sh1, pf1);
+            };
+            // pass 1 counts, pass 2 writes at the scanned offsets (candidate order is free)
+            int c0 = 0, c1 = 0;
+#pragma unroll 4
+            for (int e = tid; e < my_n; e += kSel) {
+                bool m0, m1;
+                is_cand(sc_at(e), m0, m1);
+                c0 += m0;
+                c1 += m1;
+            }
+            int4 ctot;
+            const int4 cex = sel_scan4(make_int4(c0, c1, 0, 0), S.red, ctot);
+            int w0 = cex.x, w1 = cex.y;
+#pragma unroll 4
+            for (int e = tid; e < my_n; e += kSel) {
+                const int x = sc_at(e);
+                bool m0, m1;
+                is_cand(x, m0, m1);
+                if (m0) { if (w0 < kCandCap) lbuf[w0] = make_int2(x, lo + e); w0++; }
+                if (m1) { if (w1 < kCandCap) lbuf[kCandCap + w1] = make_int2(x, lo + e); w1++; }
+            }
+            if (tid == 0) { S.info[40] = ctot.x; S.info[41] = ctot.y; }
+            sel_sync();
+            if (tid == 0 || tid == 32) {
+                const int tr = tid >> 5;
+                const int n_mine = min(S.info[40 + tr], kCandCap);
+                S.info[44 + tr] = ((tr == 0 ? g0on : g1on) && n_mine) ? atomicAdd(sl.ctrl + CTRL_CAND0 + tr, n_mine) : 0;
+                if (tr == 0 ? g0on : g1on) sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = above_loc[tr];
+            }
+            sel_sync();
+#pragma unroll
+            for (int tr = 0; tr < 2; ++tr) {
+                if (!(tr == 0 ? g0on : g1on)) continue;
+                const int n_mine = min(S.info[40 + tr], kCandCap), gbase = S.info[44 + tr];
+                for (int i = tid; i < n_mine; i += kSel)
+                    if (gbase + i < kCandCap) sl.cand[tr * kCandCap + gbase + i] = lbuf[tr * kCandCap + i];
+            }
+        }
         for (int tr = 0; tr < 2; ++tr) {
             if (state[tr] == TS_RADIX) {
                 // histogram of the next digit over own elements matching the prefix
@@ -412,56 +560,20 @@ __device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, cons
                 sel_sync();
                 const int lv = level[tr] + 1;
                 for (int e = tid; e < my_n; e += kSel) {
-                    const int x = sc[skew(e)];
+                    const int x = sc_at(e);
                     if (x < clo[tr] || x > chi[tr]) continue;
                     const uint64_t ek = ext_key(x);
                     if ((ek >> (36 - 12 * lv)) == prefix[tr]) atomicAdd(&hl[digit_at(ek, lv)], 1);
                 }
                 sel_sync();
                 push_hist(hl, sl.gl + (2 * tr + (lv - 1)) * kBins);
-            } else if (state[tr] == TS_CAND) {
-                // gather own elements of the threshold digit: compact them in shared
-                // memory, reserve a range of the group's buffer with one atomic, copy
-                any = true;
-                const int lv = level[tr] + 1;
-                int2* lbuf = reinterpret_cast<int2*>(&S.stage[0][0]) + tr * kCandCap;
-                if (tid == 0) S.info[40 + tr] = 0;
-                sel_sync();
-                for (int e0 = 0; e0 < my_n; e0 += kSel) {
-                    const int e = e0 + tid;
-                    int x = 0;
-                    bool m = false;
-                    if (e < my_n) {
-                        x = sc[skew(e)];
-                        m = x >= clo[tr] && x <= chi[tr];
-                        if (m && lv > 1) m = (ext_key(x) >> (36 - 12 * lv)) == prefix[tr];
-                    }
-                    const unsigned bal = __ballot_sync(0xffffffffu, m);
-                    if (bal) {
-                        int basei = 0;
-                        if ((tid & 31) == 0) basei = atomicAdd(&S.info[40 + tr], __popc(bal));
-                        basei = __shfl_sync(0xffffffffu, basei, 0);
-                        if (m) {
-                            const int slot = basei + __popc(bal & ((1u << (tid & 31)) - 1u));
-                            if (slot < kCandCap) lbuf[slot] = make_int2(x, lo + e);
-                        }
-                    }
-                }
-                sel_sync();
-                const int n_mine = min(S.info[40 + tr], kCandCap);
-                if (tid == 0) S.info[44 + tr] = n_mine ? atomicAdd(sl.ctrl + CTRL_CAND0 + tr, n_mine) : 0;
-                sel_sync();
-                const int gbase = S.info[44 + tr];
-                for (int i = tid; i < n_mine; i += kSel)
-                    if (gbase + i < kCandCap) sl.cand[tr * kCandCap + gbase + i] = lbuf[i];
-                if (tid == 0) sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = above_loc[tr];
             } else if (state[tr] == TS_EQ) {
                 // the value is exact: count own ties and publish it
                 any = true;
                 int eq = 0, val = 0;
                 bool have = false;
                 for (int e = tid; e < my_n; e += kSel) {
-                    const int x = sc[skew(e)];
+                    const int x = sc_at(e);
                     if (x >= clo[tr] && x <= chi[tr] && ext_key(x) == prefix[tr]) { eq++; val = x; have = true; }
                 }
                 if (have) sl.pub[(tr * 3 + 2) * kMaxG + 0] = val;   // every writer stores the same value
@@ -497,83 +609,122 @@ __device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, cons
         if (!pending) break;
     }
 
-    // ---- write each track's list
-    for (int tr = 0; tr < 2; ++tr) {
-        const int r = p.r[tr];
-        if (r <= 0) continue;
-        int32_t* outp = p.out[tr] + (size_t)c.u * r;
-        const int st = state[tr];
-        int T = INT_MAX, base_off = lo, quota = 0;
-        if (st == TS_FIN_CAND || st == TS_FIN_EQ) {
-            const int prev = prefix_total(sl.pub + (tr * 3 + 0) * kMaxG, c.cta, S.red);
-            int need_eq = 0, gt_before = 0, eq_before = 0, my_eq = 0;
-            if (st == TS_FIN_CAND) {
-                // exact threshold among the gathered candidates
-                int* cx = reinterpret_cast<int*>(&S.stage[0][0]);
-                int* ci = cx + kCandCap;
-                const int Cn = C[tr];
-                for (int i = tid; i < Cn; i += kSel) {
-                    const int2 cv = __ldcg(sl.cand + tr * kCandCap + i);
-                    cx[i] = cv.x;
-                    ci[i] = cv.y;
-                }
-                sel_sync();
-                T = local_select(cx, Cn, rrem[tr], S.histl[tr], S.red, S.info + 8 * tr, need_eq);
-                for (int i = tid; i < Cn; i += kSel) {
-                    const int x = cx[i], idx = ci[i];
-                    gt_before += (x > T && idx < lo);
-                    eq_before += (x == T && idx < lo);
-                    my_eq += (x == T && idx >= lo && idx < lo + my_n);
-                }
-                gt_before = sel_sum(gt_before, S.red);
-                eq_before = sel_sum(eq_before, S.red);
-                my_eq = sel_sum(my_eq, S.red);
-            } else {
-                T = __ldcg(sl.pub + (tr * 3 + 2) * kMaxG + 0);
-                need_eq = rrem[tr];
-                eq_before = prefix_total(sl.pub + (tr * 3 + 1) * kMaxG, c.cta, S.red);
-                my_eq = __ldcg(sl.pub + (tr * 3 + 1) * kMaxG + c.cta);
-            }
-            quota = max(0, min(need_eq - eq_before, my_eq));
-            base_off = prev + gt_before + min(need_eq, eq_before);
-        }
-        // ordered compaction: thread tid owns elements [tid*R, tid*R+R)
-        const int R = (my_n + kSel - 1) / kSel;
-        const int e0 = min(tid * R, my_n), e1 = min(e0 + R, my_n);
-        const bool all = (st == TS_ALL);
-        int cnt = 0, ceq = 0;
-        if (all) {
-            cnt = e1 - e0;
-        } else {
-            for (int e = e0; e < e1; ++e) {
-                const int x = sc[skew(e)];
-                cnt += x > T;
-                ceq += x == T;
-            }
-        }
-        int tot;
-        const int eq_excl = sel_scan_excl(ceq, S.red, tot);
-        const int eq_take = max(0, min(quota - eq_excl, ceq));
-        const int off = base_off + sel_scan_excl(cnt + eq_take, S.red, tot);
-        int k2 = off, eq_seen = 0;
-        for (int e = e0; e < e1; ++e) {
-            bool sel = all;
-            if (!all) {
-                const int x = sc[skew(e)];
-                sel = x > T;
-                if (x == T) { sel = eq_seen < eq_take; eq_seen++; }
-            }
-            if (sel) {
-                if (k2 < r) outp[k2] = full ? (lo + e) : c.pool[lo + e];
-                k2++;
-            }
-        }
-        // padding: entries [min(r, n_total), r) = -1
-        if (c.cta == p.G - 1) {
-            for (int i = min(r, n_total) + tid; i < r; i += kSel) outp[i] = -1;
+    // ---- finalize both tracks: threshold T, tie quota and this CTA's output offset
+    int T[2] = {INT_MAX, INT_MAX}, base_off[2] = {lo, lo}, quota[2] = {0, 0};
+    {
+        // published counts of the earlier CTAs, one parallel load round
+        const int grp = tid >> 6, ci = tid & 63;     // grp: 0 above0, 1 above1, 2 eq0, 3 eq1
+        const int tr_g = grp & 1;
+        const int fin = (state[tr_g] == TS_FIN_CAND || state[tr_g] == TS_FIN_EQ);
+        int v = 0;
+        if (fin && ci < c.cta && (grp < 2 || state[tr_g] == TS_FIN_EQ))
+            v = __ldcg(sl.pub + (tr_g * 3 + (grp >> 1)) * kMaxG + ci);
+        int4 tot;
+        sel_scan4(make_int4(grp == 0 ? v : 0, grp == 1 ? v : 0, grp == 2 ? v : 0, grp == 3 ? v : 0), S.red, tot);
+        const int prev[2] = {tot.x, tot.y}, eqb[2] = {tot.z, tot.w};
+        // candidates of both tracks, one load round
+        int* cx[2] = {reinterpret_cast<int*>(&S.stage[0][0]), reinterpret_cast<int*>(&S.stage[0][0]) + 2 * kCandCap};
+        const int n0 = state[0] == TS_FIN_CAND ? C[0] : 0, n1 = state[1] == TS_FIN_CAND ? C[1] : 0;
+        for (int i = tid; i < n0 + n1; i += kSel) {
+            const int tr = i < n0 ? 0 : 1, k = i < n0 ? i : i - n0;
+            const int2 cv = __ldcg(sl.cand + tr * kCandCap + k);
+            cx[tr][k] = cv.x;
+            cx[tr][kCandCap + k] = cv.y;
         }
         sel_sync();
+        for (int tr = 0; tr < 2; ++tr) {
+            const int st = state[tr];
+            if (st != TS_FIN_CAND && st != TS_FIN_EQ) continue;
+            int need_eq = 0, gt_before = 0, eq_before = 0, my_eq = 0;
+            if (st == TS_FIN_CAND) {
+                const bool lvl0 = level[tr] == 0;   // level-0 candidates lie in the bin's score interval
+                T[tr] = local_select(cx[tr], C[tr], rrem[tr], lvl0 ? clo[tr] : 1, lvl0 ? chi[tr] : 0, S.histl[tr],
+                                     S.red, S.info + 8 * tr, need_eq);
+                const int Tt = T[tr];
+                for (int i = tid; i < C[tr]; i += kSel) {
+                    const int x = cx[tr][i], idx = cx[tr][kCandCap + i];
+                    gt_before += (x > Tt && idx < lo);
+                    eq_before += (x == Tt && idx < lo);
+                    my_eq += (x == Tt && idx >= lo && idx < lo + my_n);
+                }
+                int4 t3;
+                sel_scan4(make_int4(gt_before, eq_before, my_eq, 0), S.red, t3);
+                gt_before = t3.x; eq_before = t3.y; my_eq = t3.z;
+            } else {
+                T[tr] = __ldcg(sl.pub + (tr * 3 + 2) * kMaxG + 0);
+                need_eq = rrem[tr];
+                eq_before = eqb[tr];
+                my_eq = __ldcg(sl.pub + (tr * 3 + 1) * kMaxG + c.cta);
+            }
+            quota[tr] = max(0, min(need_eq - eq_before, my_eq));
+            base_off[tr] = prev[tr] + gt_before + min(need_eq, eq_before);
+        }
     }
+
+    // ---- ordered compaction of both tracks, 256 elements at a time: warp ballots
+    // give each element its rank among the tile's ties and its output slot
+    const bool all0 = state[0] == TS_ALL, all1 = state[1] == TS_ALL;
+    const int T0 = T[0], T1 = T[1];
+    const bool on0 = p.r[0] > 0, on1 = p.r[1] > 0;
+    int32_t* out0 = on0 ? p.out[0] + (size_t)c.u * p.r[0] : nullptr;
+    int32_t* out1 = on1 ? p.out[1] + (size_t)c.u * p.r[1] : nullptr;
+    const int lane = tid & 31, wp = tid >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    int* wsum = S.info + 48;   // [8 warps][2] counts of one tile
+    int run0 = base_off[0], run1 = base_off[1], eqs0 = 0, eqs1 = 0;
+#pragma unroll 1
+    for (int e0 = 0; e0 < my_n; e0 += kSel) {
+        const int e = e0 + tid;
+        const bool in = e < my_n;
+        const int x = in ? sc_at(e) : INT_MIN;
+        const bool gt0 = in && (all0 || x > T0), eq0 = in && !all0 && x == T0;
+        const bool gt1 = in && (all1 || x > T1), eq1 = in && !all1 && x == T1;
+        // ties: rank among the tile's equal elements, in position order
+        const unsigned be0 = __ballot_sync(0xffffffffu, eq0), be1 = __ballot_sync(0xffffffffu, eq1);
+        if (lane == 0) { wsum[2 * wp] = __popc(be0); wsum[2 * wp + 1] = __popc(be1); }
+        sel_sync();
+        int pe0 = 0, pe1 = 0, te0 = 0, te1 = 0;
+#pragma unroll
+        for (int w = 0; w < kSel / 32; ++w) {
+            const int a = wsum[2 * w], bq = wsum[2 * w + 1];
+            pe0 += w < wp ? a : 0;
+            pe1 += w < wp ? bq : 0;
+            te0 += a;
+            te1 += bq;
+        }
+        const bool s0 = gt0 || (eq0 && eqs0 + pe0 + __popc(be0 & below) < quota[0]);
+        const bool s1 = gt1 || (eq1 && eqs1 + pe1 + __popc(be1 & below) < quota[1]);
+        eqs0 += te0;
+        eqs1 += te1;
+        sel_sync();
+        // output slots
+        const unsigned bs0 = __ballot_sync(0xffffffffu, s0), bs1 = __ballot_sync(0xffffffffu, s1);
+        if (lane == 0) { wsum[2 * wp] = __popc(bs0); wsum[2 * wp + 1] = __popc(bs1); }
+        sel_sync();
+        int ps0 = 0, ps1 = 0, ts0 = 0, ts1 = 0;
+#pragma unroll
+        for (int w = 0; w < kSel / 32; ++w) {
+            const int a = wsum[2 * w], bq = wsum[2 * w + 1];
+            ps0 += w < wp ? a : 0;
+            ps1 += w < wp ? bq : 0;
+            ts0 += a;
+            ts1 += bq;
+        }
+        if (s0 || s1) {
+            const int pos = full ? (lo + e) : c.pool[lo + e];
+            if (on0 && s0) { const int k2 = run0 + ps0 + __popc(bs0 & below); if (k2 < p.r[0]) out0[k2] = pos; }
+            if (on1 && s1) { const int k2 = run1 + ps1 + __popc(bs1 & below); if (k2 < p.r[1]) out1[k2] = pos; }
+        }
+        run0 += ts0;
+        run1 += ts1;
+        sel_sync();
+    }
+    // padding: entries [min(r, n_total), r) = -1
+    if (c.cta == p.G - 1) {
+        if (on0) for (int i = min(p.r[0], n_total) + tid; i < p.r[0]; i += kSel) out0[i] = -1;
+        if (on1) for (int i = min(p.r[1], n_total) + tid; i < p.r[1]; i += kSel) out1[i] = -1;
+    }
+    sel_sync();
     return true;
 }
 
@@ -652,7 +803,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 __device__ __forceinline__ IdxSmem& idx_smem() {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    return *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    return *reinterpret_cast<IdxSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
 }
 
 // ------------------------------------------------------------ Full mode on the tensor cores
@@ -666,7 +817,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int group = blockIdx.x / p.G;
     const int cta = blockIdx.x % p.G;
     const Slot sl = slot_of(p, group);
-    int* sc = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * ((p.chunk + 63) / 64 * 65) : S.sc;
+    int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * ((p.chunk + 63) / 64 * 65) : nullptr;
     constexpr int kRows = (kStageBytes / DI) < 256 ? (kStageBytes / DI) : 256;   // rows per tile
     constexpr int kBlocks = kRows / 128;                                          // MMA row blocks per tile
     constexpr uint32_t kSwz = DI == 32 ? 6u : DI == 64 ? 4u : 2u;
@@ -777,7 +928,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_arrive(&S.tempty_bar[buf]);
                 const int e = s2 * kRows + tid;
                 if (in_block && e < my_n) {
-                    sc[skew(e)] = x;
+                    if (spill) spill[skew(e)] = x; else S.sc[skew(e)] = x;
                     atomicAdd(&S.hist0[bin0(x)], 1);
                 }
             }
@@ -788,7 +939,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
         if (tid < kSel) {
             UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, nullptr};
-            if (!select_unit(p, S, sl, c, bar_target, sc) && tid == 0) S.abort = 1;
+            if (!select_unit(p, S, sl, c, bar_target, spill) && tid == 0) S.abort = 1;
         }
         __syncthreads();
         if (S.abort) break;
@@ -813,7 +964,7 @@ __global__ void __launch_bounds__(kSel, 1)
     const Slot sl = slot_of(p, group);
     const bool full = p.mode == CSA2_FULL;
     constexpr bool generic = (HI == 0);
-    int* sc = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * ((p.chunk + 63) / 64 * 65) : S.sc;
+    int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * ((p.chunk + 63) / 64 * 65) : nullptr;
 
     const int epoch = __ldcg(sl.ctrl + CTRL_EPOCH);
     int bar_target = __ldcg(sl.ctrl + CTRL_BAR_BASE);
@@ -871,7 +1022,7 @@ __global__ void __launch_bounds__(kSel, 1)
                     for (int c2 = 0; c2 < 8; ++c2)
                         if (c2 < nchunk) rowc[c2] = *reinterpret_cast<const int4*>(tile + tile_off(tid, c2, p.Di));
                     const int x = generic ? score_generic(rowc, nchunk, S.q, p.Hi, p.Di, p.w) : rq.score(rowc, p.w);
-                    sc[skew(e)] = x;
+                    if (spill) spill[skew(e)] = x; else S.sc[skew(e)] = x;
                     atomicAdd(&S.hist0[bin0(x)], 1);
                 }
                 __syncthreads();
@@ -919,7 +1070,7 @@ __global__ void __launch_bounds__(kSel, 1)
                     if (e < my_n) {
                         const int x = generic ? score_generic(rows[q2], nchunk, S.q, p.Hi, p.Di, p.w)
                                               : rq.score(rows[q2], p.w);
-                        sc[skew(e)] = x;
+                        if (spill) spill[skew(e)] = x; else S.sc[skew(e)] = x;
                         atomicAdd(&S.hist0[bin0(x)], 1);
                     }
                 }
@@ -927,7 +1078,7 @@ __global__ void __launch_bounds__(kSel, 1)
         }
         __syncthreads();
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
-        alive = select_unit(p, S, sl, c, bar_target, sc);
+        alive = select_unit(p, S, sl, c, bar_target, spill);
         __syncthreads();
     }
     if (alive && cta == 0 && tid == 0) {
