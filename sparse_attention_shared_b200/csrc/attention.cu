@@ -443,7 +443,20 @@ __global__ void __launch_bounds__(kAttnThreads)
     const bool glob = rank < ngt2;
     float* part_o = reinterpret_cast<float*>(S.tbuf);      // [HQP][D] once the MMAs are done
 
-    // ---- 1. loads that depend on nothing
+    // ---- 0. set-up that reads no input; it may overlap the previous kernel
+    if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
+    if (tid == 0) {
+        mbar_init(&S.bar_tma, 1);
+        mbar_init(&S.bar_s, 1);
+        mbar_init(&S.bar_o, 1);
+        mbar_fence_init();
+    }
+    for (int i = tid; i < 256; i += kAttnThreads)
+        S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
+    pdl_wait();
+    pdl_launch_dependents();
+
+    // ---- 1. loads that depend on nothing else
     int t = p.q_pos[u];
     const int base = p.local_base[b];
     int s0 = -1, s1 = -1;
@@ -459,13 +472,6 @@ __global__ void __launch_bounds__(kAttnThreads)
         const int h = i / (D / 8), c = i % (D / 8);
         qv[q] = make_uint4(0, 0, 0, 0);
         if (i < HQP * (D / 8) && h < p.Hq) qv[q] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
-    }
-    if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
-    if (tid == 0) {
-        mbar_init(&S.bar_tma, 1);
-        mbar_init(&S.bar_s, 1);
-        mbar_init(&S.bar_o, 1);
-        mbar_fence_init();
     }
     if (t < 0 || t >= p.N) {
         if (tid == 0 && rank == 0) report(p.status, CSA2_ERR_RANGE, u);
@@ -511,8 +517,6 @@ __global__ void __launch_bounds__(kAttnThreads)
             }
         }
     }
-    for (int i = tid; i < 256; i += kAttnThreads)
-        S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
 #pragma unroll
     for (int q = 0; q < (int)(sizeof(qv) / sizeof(qv[0])); ++q) {
         const int i = tid + q * kAttnThreads;
@@ -685,19 +689,30 @@ __global__ void __launch_bounds__(kAttnThreads)
         for (int h = 0; h < HQP; ++h) { S.part_m[h] = ok ? mh[h] : -INFINITY; S.part_l[h] = ok ? lh[h] : 0.f; }
     }
 
-    // ---- 6. merge the cluster's partials through distributed shared memory
+    // ---- 6. merge the cluster's partials through distributed shared memory: every
+    // load of a head is issued before any is used (one remote round trip per head)
     cluster_sync_all();
     for (int h = rank; h < p.Hq; h += CS) {
+        float mc[16], lc[16], oc[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            mc[c] = -INFINITY; lc[c] = 0.f; oc[c] = 0.f;
+            if (c < CS) {
+                mc[c] = ld_dsmem(dsmem_addr(&S.part_m[h], c));
+                lc[c] = ld_dsmem(dsmem_addr(&S.part_l[h], c));
+                if (tid < D) oc[c] = ld_dsmem(dsmem_addr(&part_o[h * D + tid], c));
+            }
+        }
         float M = -INFINITY;
-        for (int c = 0; c < CS; ++c) M = fmaxf(M, ld_dsmem(dsmem_addr(&S.part_m[h], c)));
+#pragma unroll
+        for (int c = 0; c < 16; ++c) M = fmaxf(M, mc[c]);
         float L = 0.f, acc = 0.f;
         if (M != -INFINITY) {
-            for (int c = 0; c < CS; ++c) {
-                const float mc = ld_dsmem(dsmem_addr(&S.part_m[h], c));
-                if (mc == -INFINITY) continue;
-                const float wgt = exp2f(mc - M);
-                L += wgt * ld_dsmem(dsmem_addr(&S.part_l[h], c));
-                if (tid < D) acc += wgt * ld_dsmem(dsmem_addr(&part_o[h * D + tid], c));
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const float wgt = (mc[c] == -INFINITY) ? 0.f : exp2f(mc[c] - M);
+                L += wgt * lc[c];
+                acc += wgt * oc[c];
             }
         }
         if (tid < D)
@@ -813,13 +828,17 @@ static cudaError_t launch_cl_variant(const AttnParams& p, const CUtensorMap& km,
     cfg.blockDim = dim3(kAttnThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // the kernel reads no input before pdl_wait(), so it may start while the
+    // previous kernel of the stream is still running
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, p, km, vm);
 }
 

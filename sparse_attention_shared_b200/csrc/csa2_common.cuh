@@ -105,6 +105,14 @@ __device__ __forceinline__ float ld_dsmem(uint32_t addr) {
     return v;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start before the previous kernel in the stream has finished;
+// pdl_wait() blocks until that kernel has completed and its writes are visible
+// (it returns at once when there is no such dependency). pdl_launch_dependents()
+// lets the next kernel start early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

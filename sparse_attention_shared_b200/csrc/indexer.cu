@@ -40,15 +40,16 @@
 
 namespace csa2 {
 
-constexpr int kSel = 256;                    // threads that run the select phase
+constexpr int kSel = 512;                    // threads that run the scan epilogue and the select phase
+constexpr int kSelWarps = kSel / 32;
+constexpr int kBpt = 4096 / kSel;            // level-0 bins per select thread
 constexpr int kTcThreads = kSel + 64;        // + one TMA warp and one MMA warp
 constexpr int kBins = 4096;
 constexpr int kCandCap = 4096;
 constexpr int kStageBytes = 16384;
-constexpr int kStages = 6;
+constexpr int kStages = 8;
 constexpr int kTmemBufs = 4;
 constexpr int kSmemScores = 16384;                  // scores kept in shared memory
-constexpr int kSkewLen = kSmemScores / 64 * 65;     // padded: one spare word per 64
 constexpr int kCtrlInts = 32;
 constexpr int kMaxG = 64;
 
@@ -68,7 +69,7 @@ struct IdxParams {
     const int32_t* pool_in;
     int P_in;
     int units, G, groups, chunk;
-    int32_t* spill;      // [groups*G][skewed chunk] when chunk > kSmemScores
+    int32_t* spill;      // [groups*G][chunk] scores when chunk > kSmemScores
     int* ctrl;           // [slots][kCtrlInts]
     int* g0;             // [slots][3][kBins]
     int* gl;             // [slots][2 tracks][2 levels][kBins]
@@ -78,11 +79,11 @@ struct IdxParams {
 };
 
 struct __align__(1024) IdxSmem {
-    uint8_t stage[kStages][kStageBytes];   // key tiles; later the candidate buffers
+    // key tiles; after a unit's scan: candidate buffers [0, 64 KB), radix histograms [64 KB, 96 KB)
+    uint8_t stage[kStages][kStageBytes];
     uint8_t qtc[16 * 128];                 // index query as a tensor-core operand (16 rows)
-    int sc[kSkewLen];                      // scores of this CTA's chunk (skewed index)
+    int sc[kSmemScores];                   // scores of this CTA's chunk, by element index
     int hist0[kBins];
-    int histl[2][kBins];
     int8_t q[16 * 128];
     uint64_t full_bar[kStages];
     uint64_t empty_bar[kStages];
@@ -90,11 +91,14 @@ struct __align__(1024) IdxSmem {
     uint64_t tempty_bar[kTmemBufs];
     uint32_t tmem_base;
     int abort;
-    alignas(16) int red[64];
+    alignas(16) int red[8 * kSelWarps];
     alignas(16) int info[64];
+    alignas(16) int wsum[4 * kSelWarps];
 };
-static_assert(2 * sizeof(int2) * kCandCap <= sizeof(((IdxSmem*)0)->stage), "candidate buffers");
+constexpr int kHistlOff = 2 * (int)sizeof(int2) * kCandCap;   // byte offset of the radix histograms
+static_assert(kHistlOff + 2 * kBins * 4 <= (int)sizeof(((IdxSmem*)0)->stage), "select buffers");
 static_assert(kStages * kStageBytes % 1024 == 0, "tensor-core operand alignment");
+static_assert(sizeof(IdxSmem) + 1024 <= 232448, "shared memory per block");
 
 struct Slot {
     int* ctrl;
@@ -103,6 +107,11 @@ struct Slot {
     int2* cand;
     int* pub;
 };
+
+// Radix histogram of track tr (select phase only: it overlays the key stages).
+__device__ __forceinline__ int* histl(IdxSmem& S, int tr) {
+    return reinterpret_cast<int*>(&S.stage[0][0] + kHistlOff) + tr * kBins;
+}
 
 __device__ __forceinline__ Slot slot_of(const IdxParams& p, int group) {
     Slot s;
@@ -113,8 +122,6 @@ __device__ __forceinline__ Slot slot_of(const IdxParams& p, int group) {
     s.pub = p.pub + (size_t)group * 6 * kMaxG;
     return s;
 }
-
-__device__ __forceinline__ int skew(int e) { return (e >> 6) * 65 + (e & 63); }
 
 // ------------------------------------------------------------ order key
 // 12-bit log-scale bin of a non-negative magnitude: exact below 64, then 64 bins
@@ -147,11 +154,6 @@ __device__ __forceinline__ uint32_t digit_at(uint64_t ext, int level) {
     return (uint32_t)(ext >> (24 - 12 * level)) & 4095u;
 }
 
-// Rare path, kept out of line: does x match a deeper (level >= 1) digit prefix?
-__device__ __noinline__ bool deep_prefix_match(int x, int shift, uint64_t prefix) {
-    return (ext_key(x) >> shift) == prefix;
-}
-
 // Level-0 digit only (the 12-bit log-scale bin of the score).
 __device__ __forceinline__ uint32_t bin0(int32_t x) {
     return x >= 0 ? 2048u + mag_bin((uint32_t)x) : 2047u - mag_bin((uint32_t)(-1 - x));
@@ -177,14 +179,18 @@ __device__ __forceinline__ void bin0_interval(uint32_t d, int& lo, int& hi) {
 // ------------------------------------------------------------ select-group sync
 // The select phase runs on threads [0, kSel) and synchronises on named barrier 1,
 // so extra warps of the CTA (the TMA and MMA warps) need not take part.
-__device__ __forceinline__ void sel_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+#define CSA2_STR2(x) #x
+#define CSA2_STR(x) CSA2_STR2(x)
+#define CSA2_SEL_THREADS 512
+static_assert(CSA2_SEL_THREADS == kSel, "named-barrier thread count");
+__device__ __forceinline__ void sel_sync() { asm volatile("bar.sync 1, " CSA2_STR(CSA2_SEL_THREADS) ";" ::: "memory"); }
 
 __device__ __forceinline__ int sel_and(int v) {
     int r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.s32 q, %1, 0;\n\t"
-        "bar.red.and.pred p, 1, 256, q;\n\t"
+        "bar.red.and.pred p, 1, " CSA2_STR(CSA2_SEL_THREADS) ", q;\n\t"
         "selp.s32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
         : "r"(v)
@@ -274,47 +280,41 @@ __device__ __forceinline__ int4 sel_scan4(int4 v, int* red, int4& total) {
     if (warp == 0) {
         int4 s = lane < (kSel / 32) ? reinterpret_cast<int4*>(red)[lane] : make_int4(0, 0, 0, 0);
 #pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
+        for (int o = 1; o < kSelWarps; o <<= 1) {
             const int a = __shfl_up_sync(0xffffffffu, s.x, o), b = __shfl_up_sync(0xffffffffu, s.y, o);
             const int c = __shfl_up_sync(0xffffffffu, s.z, o), d = __shfl_up_sync(0xffffffffu, s.w, o);
             if (lane >= o) { s.x += a; s.y += b; s.z += c; s.w += d; }
         }
-        if (lane < kSel / 32) reinterpret_cast<int4*>(red)[8 + lane] = s;
+        if (lane < kSel / 32) reinterpret_cast<int4*>(red)[kSelWarps + lane] = s;
     }
     sel_sync();
-    const int4 we = warp ? reinterpret_cast<int4*>(red)[8 + warp - 1] : make_int4(0, 0, 0, 0);
-    total = reinterpret_cast<int4*>(red)[8 + kSel / 32 - 1];
+    const int4 we = warp ? reinterpret_cast<int4*>(red)[kSelWarps + warp - 1] : make_int4(0, 0, 0, 0);
+    total = reinterpret_cast<int4*>(red)[2 * kSelWarps - 1];
     return make_int4(we.x + x.x - v.x, we.y + x.y - v.y, we.z + x.z - v.z, we.w + x.w - v.w);
 }
 
-// In a 4096-bin histogram (global or shared), find the bin holding the r-th
+// In a global 4096-bin histogram, find the bin holding the r-th
 // largest element (1-based). Writes {bin, count above the bin, count in it}.
-template <bool kGlobal>
-__device__ void find_rank_bin(const int* hist, int r, int* red, int* out) {
+__device__ void find_rank_bin_global(const int* hist, int r, int* red, int* out) {
     const int t = threadIdx.x;
-    int h[16];
-    if (kGlobal) {
-        const int4* src = reinterpret_cast<const int4*>(hist + 16 * t);
+    int h[kBpt];
+    const int4* src = reinterpret_cast<const int4*>(hist + kBpt * t);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            int4 v = __ldcg(src + i);
-            h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) h[i] = hist[16 * t + i];
+    for (int i = 0; i < kBpt / 4; ++i) {
+        int4 v = __ldcg(src + i);
+        h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
     }
     int s = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s += h[i];
+    for (int i = 0; i < kBpt; ++i) s += h[i];
     int total;
     const int excl = sel_scan_excl(s, red, total);
     int above = total - excl - s;    // elements in bins above this thread's range
     if (above < r && r <= above + s) {
 #pragma unroll
-        for (int i = 15; i >= 0; --i) {
+        for (int i = kBpt - 1; i >= 0; --i) {
             if (above < r && r <= above + h[i]) {
-                out[0] = 16 * t + i;
+                out[0] = kBpt * t + i;
                 out[1] = above;
                 out[2] = h[i];
             }
@@ -328,16 +328,16 @@ __device__ void find_rank_bin(const int* hist, int r, int* red, int* out) {
 // r[k] > 0 writes {bin, count above, count in bin} to out[8k..8k+2].
 __device__ void find_rank_bins2(const int* hist, const int* r, int* red, int* out) {
     const int t = threadIdx.x;
-    int h[16];
-    const int4* src = reinterpret_cast<const int4*>(hist + 16 * t);
+    int h[kBpt];
+    const int4* src = reinterpret_cast<const int4*>(hist + kBpt * t);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kBpt / 4; ++i) {
         int4 v = __ldcg(src + i);
         h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
     }
     int s = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s += h[i];
+    for (int i = 0; i < kBpt; ++i) s += h[i];
     int total;
     const int excl = sel_scan_excl(s, red, total);
 #pragma unroll
@@ -346,9 +346,9 @@ __device__ void find_rank_bins2(const int* hist, const int* r, int* red, int* ou
         int above = total - excl - s;
         if (rk > 0 && above < rk && rk <= above + s) {
 #pragma unroll
-            for (int i = 15; i >= 0; --i) {
+            for (int i = kBpt - 1; i >= 0; --i) {
                 if (above < rk && rk <= above + h[i]) {
-                    out[8 * k + 0] = 16 * t + i;
+                    out[8 * k + 0] = kBpt * t + i;
                     out[8 * k + 1] = above;
                     out[8 * k + 2] = h[i];
                 }
@@ -379,18 +379,40 @@ __device__ __forceinline__ int prefix_total(const int* arr, int n, int* red) {
     return sel_sum(v, red);
 }
 
-// The r-th largest value (1-based, with multiplicity) of cx[0..C) in shared
-// memory, by 12-bit radix passes over x - lo. [lo, hi] bounds the values (pass
-// hi < lo to compute the bounds here). Returns T; need_eq = how many of the
-// elements equal to T are ranked within the first r.
-__device__ int local_select(const int* cx, int C, int r, int lo, int hi, int* hist, int* red, int* info,
-                            int& need_eq) {
-    if (hi < lo) {
-        int mn = INT_MAX, mx = INT_MIN;
-        for (int i = threadIdx.x; i < C; i += kSel) { mn = min(mn, cx[i]); mx = max(mx, cx[i]); }
-        lo = sel_min(mn, red);
-        hi = -sel_min(-mx, red);
+// In a shared histogram of kSel * per bins (per <= 8), find the bin holding the
+// r-th largest element (1-based). Writes {bin, count above the bin, count in it}.
+__device__ void find_rank_bin_smem(const int* hist, int per, int r, int* red, int* out) {
+    const int t = threadIdx.x;
+    int h[kBpt];
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < kBpt; ++i) {
+        h[i] = i < per ? hist[per * t + i] : 0;
+        s += h[i];
     }
+    int total;
+    const int excl = sel_scan_excl(s, red, total);
+    int above = total - excl - s;    // elements in bins above this thread's range
+    if (above < r && r <= above + s) {
+#pragma unroll
+        for (int i = kBpt - 1; i >= 0; --i) {
+            if (above < r && r <= above + h[i]) {
+                out[0] = per * t + i;
+                out[1] = above;
+                out[2] = h[i];
+            }
+            above += h[i];
+        }
+    }
+    sel_sync();
+}
+
+// The r-th largest value (1-based, with multiplicity) of cx[0..C) in shared
+// memory, by radix passes of up to 12 bits over x - lo (a pass of b bits uses
+// max(kSel, 2^b) bins); every value lies in [lo, hi]. Returns T; need_eq = how
+// many of the elements equal to T are ranked within the first r.
+__device__ __noinline__ int local_select(const int* cx, int C, int r, int lo, int hi, int* hist, int* red,
+                                         int* info, int& need_eq) {
     const int mn = lo;
     const uint32_t w = (uint32_t)((long long)hi - (long long)lo);
     int rem = (w == 0u) ? 0 : 32 - __clz(w);
@@ -398,14 +420,15 @@ __device__ int local_select(const int* cx, int C, int r, int lo, int hi, int* hi
     while (rem > 0) {
         const int take = rem < 12 ? rem : 12;
         const int sh = rem - take;
-        for (int i = threadIdx.x; i < kBins; i += kSel) hist[i] = 0;
+        const int per = max(kSel, 1 << take) / kSel;
+        for (int i = threadIdx.x; i < kSel * per; i += kSel) hist[i] = 0;
         sel_sync();
         for (int i = threadIdx.x; i < C; i += kSel) {
             const uint32_t v = (uint32_t)((long long)cx[i] - (long long)mn);
             if ((uint32_t)(((uint64_t)v) >> (sh + take)) == prefix) atomicAdd(&hist[(v >> sh) & ((1u << take) - 1u)], 1);
         }
         sel_sync();
-        find_rank_bin<false>(hist, r, red, info);
+        find_rank_bin_smem(hist, per, r, red, info);
         r -= info[1];
         prefix = (prefix << take) | (uint32_t)info[0];
         rem = sh;
@@ -415,6 +438,12 @@ __device__ int local_select(const int* cx, int C, int r, int lo, int hi, int* hi
 }
 
 // ------------------------------------------------------------ select + write
+// The select code runs once per unit, straight after a scan that has streamed the
+// keys through L2, so its instructions are fetched cold: it is kept small. Each
+// pass over the chunk's scores is one out-of-line loop, the per-track bookkeeping
+// runs in plain loops, and every digit prefix is turned into the interval of
+// scores it covers, so the common passes only compare scores with bounds.
+
 // Track states (identical in every CTA of a group).
 enum { TS_OFF = 0, TS_ALL = 1, TS_RADIX = 2, TS_CAND = 3, TS_EQ = 4, TS_FIN_CAND = 5, TS_FIN_EQ = 6 };
 
@@ -423,14 +452,251 @@ struct UnitCtx {
     const int32_t* pool;   // Reindex: the unit's pool (positions of the elements)
 };
 
+// Select state of one track (pool or top-k); the same in every CTA of a group.
+struct Track {
+    int state;        // TS_*
+    int rrem;         // rank still to find inside the current prefix
+    int C;            // elements of the whole group inside the current prefix
+    int level;        // index of the last fixed digit (0: the level-0 bin)
+    int above;        // this CTA's elements above the current prefix
+    int lo, hi;       // interval of scores whose key starts with the prefix
+    uint64_t prefix;  // the fixed digits
+};
+
+// Scores whose order key starts with `prefix` (digits 0..level) form an interval,
+// since the key is strictly increasing in the score. Bisection inside [lo, hi],
+// the interval of the enclosing prefix.
+__device__ void prefix_interval(int level, uint64_t prefix, int& lo, int& hi) {
+    const int sh = 24 - 12 * level;
+    long long a = lo, b = (long long)hi + 1;   // first score with key prefix >= prefix
+    while (a < b) {
+        const long long m = (a + b) >> 1;
+        if ((ext_key((int)m) >> sh) >= prefix) b = m; else a = m + 1;
+    }
+    const long long first = a;
+    b = (long long)hi + 1;                     // first score with key prefix > prefix
+    while (a < b) {
+        const long long m = (a + b) >> 1;
+        if ((ext_key((int)m) >> sh) > prefix) b = m; else a = m + 1;
+    }
+    lo = (int)first;
+    hi = (int)(a - 1);
+}
+
+// The chunk's scores as int4 vectors: element e sits at index e, in shared memory
+// or, for chunks longer than kSmemScores, in this CTA's spill area.
+__device__ __forceinline__ int4 ld_scores4(const int* sc, int v) { return reinterpret_cast<const int4*>(sc)[v]; }
+
+// Steps of 32 vectors (128 elements) owned by this warp: one contiguous range per
+// warp, so each warp meets its elements in position order.
+__device__ __forceinline__ void warp_steps(int n, int& s0, int& s1) {
+    const int nstep = (n + 127) >> 7;
+    const int spw = (nstep + kSel / 32 - 1) / (kSel / 32);
+    s0 = min(nstep, (threadIdx.x >> 5) * spw);
+    s1 = min(nstep, s0 + spw);
+}
+
+__device__ __forceinline__ int4 warp_sum4(int4 v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+        v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+        v.z += __shfl_xor_sync(0xffffffffu, v.z, o);
+        v.w += __shfl_xor_sync(0xffffffffu, v.w, o);
+    }
+    return v;
+}
+
+// Totals of two int4 over the select threads (two barriers).
+__device__ __noinline__ void sel_total8(int4& a, int4& b, int* red) {
+    a = warp_sum4(a);
+    b = warp_sum4(b);
+    sel_sync();
+    int4* r4 = reinterpret_cast<int4*>(red);
+    if ((threadIdx.x & 31) == 0) { r4[2 * (threadIdx.x >> 5)] = a; r4[2 * (threadIdx.x >> 5) + 1] = b; }
+    sel_sync();
+    a = make_int4(0, 0, 0, 0);
+    b = a;
+#pragma unroll 1
+    for (int w = 0; w < kSel / 32; ++w) {
+        const int4 x = r4[2 * w], y = r4[2 * w + 1];
+        a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+        b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+    }
+}
+
+// Candidates of both tracks (scores in [lo0, hi0] / [lo1, hi1]; lo > hi = off)
+// into lbuf[0..) and lbuf[kCandCap..) as (score, element index + base). A warp
+// reserves room once per step that holds candidates; the order is free.
+__device__ __noinline__ void gather_cands(const int* sc, int n, int base, int lo0, int hi0, int lo1, int hi1,
+                                          int2* lbuf, int* lcnt) {
+    const int lane = threadIdx.x & 31;
+    int s0, s1;
+    warp_steps(n, s0, s1);
+#pragma unroll 1
+    for (int st = s0; st < s1; ++st) {
+        const int v = st * 32 + lane;
+        const int4 x4 = ld_scores4(sc, v);
+        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
+        unsigned m0 = 0, m1 = 0;   // bit q: sub-element q is a candidate
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const bool ok = 4 * v + q < n;
+            m0 |= (ok && xs[q] >= lo0 && xs[q] <= hi0) ? 1u << q : 0u;
+            m1 |= (ok && xs[q] >= lo1 && xs[q] <= hi1) ? 1u << q : 0u;
+        }
+        if (!__any_sync(0xffffffffu, (m0 | m1) != 0)) continue;
+        const int c0 = __popc(m0), c1 = __popc(m1);
+        // lanes' counts -> exclusive prefix within the warp
+        int p0 = c0, p1 = c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y0 = __shfl_up_sync(0xffffffffu, p0, o), y1 = __shfl_up_sync(0xffffffffu, p1, o);
+            if (lane >= o) { p0 += y0; p1 += y1; }
+        }
+        int w0 = 0, w1 = 0;
+        if (lane == 31) {
+            w0 = p0 ? atomicAdd(lcnt, p0) : 0;
+            w1 = p1 ? atomicAdd(lcnt + 1, p1) : 0;
+        }
+        w0 = __shfl_sync(0xffffffffu, w0, 31) + p0 - c0;
+        w1 = __shfl_sync(0xffffffffu, w1, 31) + p1 - c1;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int2 cv = make_int2(xs[q], base + 4 * v + q);
+            if (m0 & (1u << q)) { if (w0 < kCandCap) lbuf[w0] = cv; w0++; }
+            if (m1 & (1u << q)) { if (w1 < kCandCap) lbuf[kCandCap + w1] = cv; w1++; }
+        }
+    }
+}
+
+// Histogram of digit `lv` over the elements in [lo_t, hi_t] (they share digits 0..lv-1).
+__device__ __noinline__ void radix_hist(const int* sc, int n, int lo_t, int hi_t, int lv, int* hist) {
+    const int lane = threadIdx.x & 31;
+    int s0, s1;
+    warp_steps(n, s0, s1);
+#pragma unroll 1
+    for (int st = s0; st < s1; ++st) {
+        const int v = st * 32 + lane;
+        const int4 x4 = ld_scores4(sc, v);
+        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+            const int x = xs[q];
+            if (4 * v + q < n && x >= lo_t && x <= hi_t) atomicAdd(&hist[digit_at(ext_key(x), lv)], 1);
+        }
+    }
+}
+
+// Number of this thread's elements in [lo_t, hi_t].
+__device__ __noinline__ int count_range(const int* sc, int n, int lo_t, int hi_t) {
+    const int lane = threadIdx.x & 31;
+    int s0, s1, cnt = 0;
+    warp_steps(n, s0, s1);
+#pragma unroll 1
+    for (int st = s0; st < s1; ++st) {
+        const int v = st * 32 + lane;
+        const int4 x4 = ld_scores4(sc, v);
+        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cnt += (4 * v + q < n && xs[q] >= lo_t && xs[q] <= hi_t);
+    }
+    return cnt;
+}
+
+// Where one track's cut leaves this CTA: elements above T are taken, and so are the
+// first `quota` elements equal to T in position order (all = take every element).
+// The taken elements go to out[base ..] in position order.
+struct ListCut {
+    int T, all, quota, base, r;
+    int32_t* out;   // nullptr: track off
+};
+
+__device__ __forceinline__ void take_flags(int x, bool ok, const ListCut& c, bool& g, bool& e) {
+    g = ok && c.out != nullptr && (c.all || x > c.T);
+    e = ok && c.out != nullptr && !c.all && x == c.T;
+}
+
+// Ordered write of both tracks: pass 1 counts per warp, pass 2 walks the same
+// ranges with running counts and ballots for the ranks inside a step.
+__device__ __noinline__ void write_lists(const int* sc, int n, int base, const int32_t* pool, ListCut c0,
+                                         ListCut c1, int* wsum) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    int s0, s1;
+    warp_steps(n, s0, s1);
+    int4 cnt = make_int4(0, 0, 0, 0);   // gt0, eq0, gt1, eq1
+#pragma unroll 1
+    for (int st = s0; st < s1; ++st) {
+        const int v = st * 32 + lane;
+        const int4 x4 = ld_scores4(sc, v);
+        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            bool g, e;
+            take_flags(xs[q], 4 * v + q < n, c0, g, e);
+            cnt.x += g; cnt.y += e;
+            take_flags(xs[q], 4 * v + q < n, c1, g, e);
+            cnt.z += g; cnt.w += e;
+        }
+    }
+    cnt = warp_sum4(cnt);
+    int4* w4 = reinterpret_cast<int4*>(wsum);
+    if (lane == 0) w4[wp] = cnt;
+    sel_sync();
+    int rg0 = 0, re0 = 0, rg1 = 0, re1 = 0;
+#pragma unroll 1
+    for (int w = 0; w < wp; ++w) {
+        const int4 a = w4[w];
+        rg0 += a.x; re0 += a.y; rg1 += a.z; re1 += a.w;
+    }
+#pragma unroll 1
+    for (int st = s0; st < s1; ++st) {
+        const int v = st * 32 + lane;
+        const int4 x4 = ld_scores4(sc, v);
+        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
+        unsigned fg0 = 0, fe0 = 0, fg1 = 0, fe1 = 0;   // bit q: sub-element q's flags
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            bool g, e;
+            take_flags(xs[q], 4 * v + q < n, c0, g, e);
+            fg0 |= g ? 1u << q : 0u; fe0 |= e ? 1u << q : 0u;
+            take_flags(xs[q], 4 * v + q < n, c1, g, e);
+            fg1 |= g ? 1u << q : 0u; fe1 |= e ? 1u << q : 0u;
+        }
+        if (!__any_sync(0xffffffffu, (fg0 | fe0 | fg1 | fe1) != 0)) continue;
+        // exclusive prefix of the four counts over the lanes
+        int4 mine = make_int4(__popc(fg0), __popc(fe0), __popc(fg1), __popc(fe1)), pre = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, pre.x, o), b = __shfl_up_sync(0xffffffffu, pre.y, o);
+            const int cc = __shfl_up_sync(0xffffffffu, pre.z, o), d = __shfl_up_sync(0xffffffffu, pre.w, o);
+            if (lane >= o) { pre.x += a; pre.y += b; pre.z += cc; pre.w += d; }
+        }
+        int og0 = rg0 + pre.x - mine.x, oe0 = re0 + pre.y - mine.y;
+        int og1 = rg1 + pre.z - mine.z, oe1 = re1 + pre.w - mine.w;
+        rg0 += __shfl_sync(0xffffffffu, pre.x, 31); re0 += __shfl_sync(0xffffffffu, pre.y, 31);
+        rg1 += __shfl_sync(0xffffffffu, pre.z, 31); re1 += __shfl_sync(0xffffffffu, pre.w, 31);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const bool g0 = fg0 >> q & 1u, e0 = fe0 >> q & 1u, g1 = fg1 >> q & 1u, e1 = fe1 >> q & 1u;
+            const bool t0 = g0 || (e0 && oe0 < c0.quota), t1 = g1 || (e1 && oe1 < c1.quota);
+            if (t0 || t1) {
+                const int e = base + 4 * v + q;
+                const int pos = pool ? pool[e] : e;
+                if (t0) { const int k = c0.base + og0 + min(oe0, c0.quota); if (k < c0.r) c0.out[k] = pos; }
+                if (t1) { const int k = c1.base + og1 + min(oe1, c1.quota); if (k < c1.r) c1.out[k] = pos; }
+            }
+            og0 += g0; oe0 += e0; og1 += g1; oe1 += e1;
+        }
+    }
+}
+
 // Exact pool/top-k cut for one unit and the write of this CTA's selected
-// positions. Runs on threads [0, kSel). The chunk's scores are in S.sc or spill (skewed
-// index) and their level-0 histogram in S.hist0. The two tracks (pool P and
+// positions. Runs on threads [0, kSel). `sc` holds the chunk's scores (element
+// index order) and S.hist0 their level-0 histogram. The two tracks (pool P and
 // top-k) share every pass and every group barrier. Returns false on a timeout.
-__device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c, int& bar_target,
-                            const int* spill) {
-    // a chunk's scores live in shared memory unless they were spilled to the workspace
-    auto sc_at = [&](int e) -> int { return spill ? spill[skew(e)] : S.sc[skew(e)]; };
+__device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c,
+                                         int& bar_target, const int* sc) {
     const int tid = threadIdx.x;
     const bool full = p.mode == CSA2_FULL;
     const int lo = c.lo, my_n = c.my_n;
@@ -442,6 +708,7 @@ __device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, cons
     {
         const int per = (kBins + p.G - 1) / p.G;
         const int zlo = c.cta * per, zhi = min(kBins, zlo + per);
+#pragma unroll 1
         for (int i = zlo + tid; i < zhi; i += kSel) {
             g0nxt[i] = 0;
             sl.gl[i] = 0; sl.gl[kBins + i] = 0; sl.gl[2 * kBins + i] = 0; sl.gl[3 * kBins + i] = 0;
@@ -456,130 +723,97 @@ __device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, cons
         n_total = c.n_all;
     } else {
         int s2 = 0;
+#pragma unroll 1
         for (int i = tid; i < kBins; i += kSel) s2 += __ldcg(g0cur + i);
         n_total = sel_sum(s2, S.red);
     }
-    int state[2], rrem[2], C[2], level[2], above_loc[2], clo[2], chi[2];
-    uint64_t prefix[2];
+    Track tk[2];
     int rq[2];
+#pragma unroll 1
     for (int tr = 0; tr < 2; ++tr) {
-        state[tr] = TS_OFF; rrem[tr] = 0; C[tr] = 0; level[tr] = 0; above_loc[tr] = 0; prefix[tr] = 0;
-        clo[tr] = 0; chi[tr] = -1;
+        tk[tr] = Track{TS_OFF, 0, 0, 0, 0, 1, 0, 0};
         const int r = p.r[tr];
         rq[tr] = 0;
         if (r <= 0) continue;
-        if (n_total <= r) { state[tr] = TS_ALL; continue; }
+        if (n_total <= r) { tk[tr].state = TS_ALL; continue; }
         rq[tr] = r;
     }
     if (rq[0] > 0 || rq[1] > 0) {
         find_rank_bins2(g0cur, rq, S.red, S.info);
         int a0 = 0, a1 = 0;
         const int d0 = S.info[0], d1 = S.info[8];
+#pragma unroll 1
         for (int i = tid; i < kBins; i += kSel) {
             const int v = S.hist0[i];
             a0 += (rq[0] > 0 && i > d0) ? v : 0;
             a1 += (rq[1] > 0 && i > d1) ? v : 0;
         }
-        int4 tot;
-        sel_scan4(make_int4(a0, a1, 0, 0), S.red, tot);
+        int4 ta = make_int4(a0, a1, 0, 0), tb = make_int4(0, 0, 0, 0);
+        sel_total8(ta, tb, S.red);
+#pragma unroll 1
         for (int tr = 0; tr < 2; ++tr) {
             if (rq[tr] <= 0) continue;
+            Track& k = tk[tr];
             const int d = S.info[8 * tr + 0];
-            rrem[tr] = rq[tr] - S.info[8 * tr + 1];
-            C[tr] = S.info[8 * tr + 2];
-            prefix[tr] = (uint64_t)d;
-            above_loc[tr] = tr == 0 ? tot.x : tot.y;
-            bin0_interval((uint32_t)d, clo[tr], chi[tr]);
-            state[tr] = (C[tr] <= kCandCap) ? TS_CAND : TS_RADIX;
+            k.rrem = rq[tr] - S.info[8 * tr + 1];
+            k.C = S.info[8 * tr + 2];
+            k.prefix = (uint64_t)d;
+            k.above = tr == 0 ? ta.x : ta.y;
+            bin0_interval((uint32_t)d, k.lo, k.hi);
+            k.state = (k.C <= kCandCap) ? TS_CAND : TS_RADIX;
         }
     }
 
     // ---- rounds until every track knows its cut (usually one)
+#pragma unroll 1
     while (true) {
         bool any = false;
-        // fused candidate gather for every track in TS_CAND: compact in shared
-        // memory, reserve a range of the group buffer with one atomic, copy out
-        const bool g0on = state[0] == TS_CAND, g1on = state[1] == TS_CAND;
+        const bool g0on = tk[0].state == TS_CAND, g1on = tk[1].state == TS_CAND;
         if (g0on || g1on) {
             any = true;
             int2* lbuf = reinterpret_cast<int2*>(&S.stage[0][0]);
-            // per-track bounds as scalars (no indexed arrays in the loops)
-            const int lo0 = clo[0], hi0 = chi[0], lo1 = clo[1], hi1 = chi[1];
-            const bool deep0 = level[0] > 0, deep1 = level[1] > 0;
-            const int sh0 = 24 - 12 * level[0], sh1 = 24 - 12 * level[1];
-            const uint64_t pf0 = prefix[0], pf1 = prefix[1];
-            auto is_cand = [&](int x, bool& m0, bool& m1) {
-                m0 = g0on && x >= lo0 && x <= hi0;
-                m1 = g1on && x >= lo1 && x <= hi1;
-                if (deep0 && m0) m0 = deep_prefix_match(x, sh0, pf0);
-                if (deep1 && m1) m1 = deep_prefix_match(x, sh1, pf1);
-            };
-            // pass 1 counts, pass 2 writes at the scanned offsets (candidate order is free)
-            int c0 = 0, c1 = 0;
-#pragma unroll 4
-            for (int e = tid; e < my_n; e += kSel) {
-                bool m0, m1;
-                is_cand(sc_at(e), m0, m1);
-                c0 += m0;
-                c1 += m1;
-            }
-            int4 ctot;
-            const int4 cex = sel_scan4(make_int4(c0, c1, 0, 0), S.red, ctot);
-            int w0 = cex.x, w1 = cex.y;
-#pragma unroll 4
-            for (int e = tid; e < my_n; e += kSel) {
-                const int x = sc_at(e);
-                bool m0, m1;
-                is_cand(x, m0, m1);
-                if (m0) { if (w0 < kCandCap) lbuf[w0] = make_int2(x, lo + e); w0++; }
-                if (m1) { if (w1 < kCandCap) lbuf[kCandCap + w1] = make_int2(x, lo + e); w1++; }
-            }
-            if (tid == 0) { S.info[40] = ctot.x; S.info[41] = ctot.y; }
+            int* lcnt = S.info + 40;
+            if (tid == 0) { lcnt[0] = 0; lcnt[1] = 0; }
+            sel_sync();
+            gather_cands(sc, my_n, lo, g0on ? tk[0].lo : 1, g0on ? tk[0].hi : 0, g1on ? tk[1].lo : 1,
+                         g1on ? tk[1].hi : 0, lbuf, lcnt);
             sel_sync();
             if (tid == 0 || tid == 32) {
                 const int tr = tid >> 5;
-                const int n_mine = min(S.info[40 + tr], kCandCap);
-                S.info[44 + tr] = ((tr == 0 ? g0on : g1on) && n_mine) ? atomicAdd(sl.ctrl + CTRL_CAND0 + tr, n_mine) : 0;
-                if (tr == 0 ? g0on : g1on) sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = above_loc[tr];
+                const bool on = tr == 0 ? g0on : g1on;
+                const int n_mine = min(lcnt[tr], kCandCap);
+                S.info[44 + tr] = (on && n_mine) ? atomicAdd(sl.ctrl + CTRL_CAND0 + tr, n_mine) : 0;
+                S.info[46 + tr] = on ? n_mine : 0;
+                if (on) sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = tk[tr].above;
             }
             sel_sync();
-#pragma unroll
+#pragma unroll 1
             for (int tr = 0; tr < 2; ++tr) {
-                if (!(tr == 0 ? g0on : g1on)) continue;
-                const int n_mine = min(S.info[40 + tr], kCandCap), gbase = S.info[44 + tr];
+                const int n_mine = S.info[46 + tr], gbase = S.info[44 + tr];
+#pragma unroll 1
                 for (int i = tid; i < n_mine; i += kSel)
                     if (gbase + i < kCandCap) sl.cand[tr * kCandCap + gbase + i] = lbuf[tr * kCandCap + i];
             }
         }
+#pragma unroll 1
         for (int tr = 0; tr < 2; ++tr) {
-            if (state[tr] == TS_RADIX) {
-                // histogram of the next digit over own elements matching the prefix
+            Track& k = tk[tr];
+            if (k.state == TS_RADIX) {
+                // histogram of the next digit over own elements inside the prefix
                 any = true;
-                int* hl = S.histl[tr];
+                int* hl = histl(S, tr);
+#pragma unroll 1
                 for (int i = tid; i < kBins; i += kSel) hl[i] = 0;
                 sel_sync();
-                const int lv = level[tr] + 1;
-                for (int e = tid; e < my_n; e += kSel) {
-                    const int x = sc_at(e);
-                    if (x < clo[tr] || x > chi[tr]) continue;
-                    const uint64_t ek = ext_key(x);
-                    if ((ek >> (36 - 12 * lv)) == prefix[tr]) atomicAdd(&hl[digit_at(ek, lv)], 1);
-                }
+                radix_hist(sc, my_n, k.lo, k.hi, k.level + 1, hl);
                 sel_sync();
-                push_hist(hl, sl.gl + (2 * tr + (lv - 1)) * kBins);
-            } else if (state[tr] == TS_EQ) {
-                // the value is exact: count own ties and publish it
+                push_hist(hl, sl.gl + (2 * tr + k.level) * kBins);
+            } else if (k.state == TS_EQ) {
+                // the prefix is the whole key: the score is exact; count own ties
                 any = true;
-                int eq = 0, val = 0;
-                bool have = false;
-                for (int e = tid; e < my_n; e += kSel) {
-                    const int x = sc_at(e);
-                    if (x >= clo[tr] && x <= chi[tr] && ext_key(x) == prefix[tr]) { eq++; val = x; have = true; }
-                }
-                if (have) sl.pub[(tr * 3 + 2) * kMaxG + 0] = val;   // every writer stores the same value
-                eq = sel_sum(eq, S.red);
+                const int eq = sel_sum(count_range(sc, my_n, k.lo, k.hi), S.red);
                 if (tid == 0) {
-                    sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = above_loc[tr];
+                    sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = k.above;
                     sl.pub[(tr * 3 + 1) * kMaxG + c.cta] = eq;
                 }
             }
@@ -588,178 +822,138 @@ __device__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, cons
         bar_target += p.G;
         if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
         bool pending = false;
+#pragma unroll 1
         for (int tr = 0; tr < 2; ++tr) {
-            if (state[tr] == TS_RADIX) {
-                const int lv = level[tr] + 1;
-                find_rank_bin<true>(sl.gl + (2 * tr + (lv - 1)) * kBins, rrem[tr], S.red, S.info + 8 * tr);
+            Track& k = tk[tr];
+            if (k.state == TS_RADIX) {
+                const int lv = k.level + 1;
+                find_rank_bin_global(sl.gl + (2 * tr + (lv - 1)) * kBins, k.rrem, S.red, S.info + 8 * tr);
                 const int d = S.info[8 * tr + 0];
-                rrem[tr] -= S.info[8 * tr + 1];
-                C[tr] = S.info[8 * tr + 2];
-                prefix[tr] = (prefix[tr] << 12) | (uint64_t)d;
-                level[tr] = lv;
-                above_loc[tr] += sel_sum(sum_above(S.histl[tr], d), S.red);
-                state[tr] = (C[tr] <= kCandCap) ? TS_CAND : (lv < 2 ? TS_RADIX : TS_EQ);
+                k.rrem -= S.info[8 * tr + 1];
+                k.C = S.info[8 * tr + 2];
+                k.prefix = (k.prefix << 12) | (uint64_t)d;
+                k.level = lv;
+                k.above += sel_sum(sum_above(histl(S, tr), d), S.red);
+                prefix_interval(lv, k.prefix, k.lo, k.hi);
+                k.state = (k.C <= kCandCap) ? TS_CAND : (lv < 2 ? TS_RADIX : TS_EQ);
                 pending = true;
-            } else if (state[tr] == TS_CAND) {
-                state[tr] = TS_FIN_CAND;
-            } else if (state[tr] == TS_EQ) {
-                state[tr] = TS_FIN_EQ;
+            } else if (k.state == TS_CAND) {
+                k.state = TS_FIN_CAND;
+            } else if (k.state == TS_EQ) {
+                k.state = TS_FIN_EQ;
             }
         }
         if (!pending) break;
     }
 
     // ---- finalize both tracks: threshold T, tie quota and this CTA's output offset
-    int T[2] = {INT_MAX, INT_MAX}, base_off[2] = {lo, lo}, quota[2] = {0, 0};
+    ListCut cut[2];
     {
         // published counts of the earlier CTAs, one parallel load round
         const int grp = tid >> 6, ci = tid & 63;     // grp: 0 above0, 1 above1, 2 eq0, 3 eq1
         const int tr_g = grp & 1;
-        const int fin = (state[tr_g] == TS_FIN_CAND || state[tr_g] == TS_FIN_EQ);
+        const int st_g = tk[tr_g].state;
+        const bool fin = st_g == TS_FIN_CAND || st_g == TS_FIN_EQ;
         int v = 0;
-        if (fin && ci < c.cta && (grp < 2 || state[tr_g] == TS_FIN_EQ))
+        if (grp < 4 && fin && ci < c.cta && (grp < 2 || st_g == TS_FIN_EQ))
             v = __ldcg(sl.pub + (tr_g * 3 + (grp >> 1)) * kMaxG + ci);
         int4 tot;
         sel_scan4(make_int4(grp == 0 ? v : 0, grp == 1 ? v : 0, grp == 2 ? v : 0, grp == 3 ? v : 0), S.red, tot);
         const int prev[2] = {tot.x, tot.y}, eqb[2] = {tot.z, tot.w};
         // candidates of both tracks, one load round
-        int* cx[2] = {reinterpret_cast<int*>(&S.stage[0][0]), reinterpret_cast<int*>(&S.stage[0][0]) + 2 * kCandCap};
-        const int n0 = state[0] == TS_FIN_CAND ? C[0] : 0, n1 = state[1] == TS_FIN_CAND ? C[1] : 0;
+        int* cx0 = reinterpret_cast<int*>(&S.stage[0][0]);
+        const int n0 = tk[0].state == TS_FIN_CAND ? tk[0].C : 0, n1 = tk[1].state == TS_FIN_CAND ? tk[1].C : 0;
+#pragma unroll 1
         for (int i = tid; i < n0 + n1; i += kSel) {
             const int tr = i < n0 ? 0 : 1, k = i < n0 ? i : i - n0;
             const int2 cv = __ldcg(sl.cand + tr * kCandCap + k);
-            cx[tr][k] = cv.x;
-            cx[tr][kCandCap + k] = cv.y;
+            cx0[tr * 2 * kCandCap + k] = cv.x;
+            cx0[tr * 2 * kCandCap + kCandCap + k] = cv.y;
         }
         sel_sync();
+        int T[2] = {INT_MAX, INT_MAX}, need[2] = {0, 0};
+#pragma unroll 1
         for (int tr = 0; tr < 2; ++tr) {
-            const int st = state[tr];
-            if (st != TS_FIN_CAND && st != TS_FIN_EQ) continue;
-            int need_eq = 0, gt_before = 0, eq_before = 0, my_eq = 0;
-            if (st == TS_FIN_CAND) {
-                const bool lvl0 = level[tr] == 0;   // level-0 candidates lie in the bin's score interval
-                T[tr] = local_select(cx[tr], C[tr], rrem[tr], lvl0 ? clo[tr] : 1, lvl0 ? chi[tr] : 0, S.histl[tr],
-                                     S.red, S.info + 8 * tr, need_eq);
-                const int Tt = T[tr];
-                for (int i = tid; i < C[tr]; i += kSel) {
-                    const int x = cx[tr][i], idx = cx[tr][kCandCap + i];
-                    gt_before += (x > Tt && idx < lo);
-                    eq_before += (x == Tt && idx < lo);
-                    my_eq += (x == Tt && idx >= lo && idx < lo + my_n);
-                }
-                int4 t3;
-                sel_scan4(make_int4(gt_before, eq_before, my_eq, 0), S.red, t3);
-                gt_before = t3.x; eq_before = t3.y; my_eq = t3.z;
-            } else {
-                T[tr] = __ldcg(sl.pub + (tr * 3 + 2) * kMaxG + 0);
-                need_eq = rrem[tr];
-                eq_before = eqb[tr];
-                my_eq = __ldcg(sl.pub + (tr * 3 + 1) * kMaxG + c.cta);
+            const Track& k = tk[tr];
+            if (k.state == TS_FIN_CAND) {
+                T[tr] = local_select(cx0 + tr * 2 * kCandCap, k.C, k.rrem, k.lo, k.hi, histl(S, tr), S.red,
+                                     S.info + 8 * tr, need[tr]);
+            } else if (k.state == TS_FIN_EQ) {
+                T[tr] = k.lo;
+                need[tr] = k.rrem;
             }
-            quota[tr] = max(0, min(need_eq - eq_before, my_eq));
-            base_off[tr] = prev[tr] + gt_before + min(need_eq, eq_before);
+        }
+        // larger candidates and ties before this CTA, and this CTA's ties (both tracks)
+        int4 ca = make_int4(0, 0, 0, 0), cb = make_int4(0, 0, 0, 0);
+        const int e_end = lo + my_n;
+#pragma unroll 1
+        for (int i = tid; i < n0 + n1; i += kSel) {
+            const int tr = i < n0 ? 0 : 1, k = i < n0 ? i : i - n0;
+            const int x = cx0[tr * 2 * kCandCap + k], idx = cx0[tr * 2 * kCandCap + kCandCap + k];
+            const int gtb = x > T[tr] && idx < lo, eqb2 = x == T[tr] && idx < lo;
+            const int mine = x == T[tr] && idx >= lo && idx < e_end;
+            if (tr == 0) { ca.x += gtb; ca.y += eqb2; cb.x += mine; }
+            else         { ca.z += gtb; ca.w += eqb2; cb.y += mine; }
+        }
+        sel_total8(ca, cb, S.red);
+        const int gtb[2] = {ca.x, ca.z}, eqc[2] = {ca.y, ca.w}, mye[2] = {cb.x, cb.y};
+#pragma unroll 1
+        for (int tr = 0; tr < 2; ++tr) {
+            const int st = tk[tr].state;
+            ListCut& lc = cut[tr];
+            lc.r = p.r[tr];
+            lc.out = lc.r > 0 ? p.out[tr] + (size_t)c.u * lc.r : nullptr;
+            lc.all = st == TS_ALL;
+            lc.T = T[tr];
+            lc.quota = 0;
+            lc.base = lo;
+            if (st != TS_FIN_CAND && st != TS_FIN_EQ) continue;
+            const bool cand = st == TS_FIN_CAND;
+            const int gt_before = cand ? gtb[tr] : 0;
+            const int eq_before = cand ? eqc[tr] : eqb[tr];
+            const int my_eq = cand ? mye[tr] : __ldcg(sl.pub + (tr * 3 + 1) * kMaxG + c.cta);
+            lc.quota = max(0, min(need[tr] - eq_before, my_eq));
+            lc.base = prev[tr] + gt_before + min(need[tr], eq_before);
         }
     }
 
-    // ---- ordered compaction of both tracks, 256 elements at a time: warp ballots
-    // give each element its rank among the tile's ties and its output slot
-    const bool all0 = state[0] == TS_ALL, all1 = state[1] == TS_ALL;
-    const int T0 = T[0], T1 = T[1];
-    const bool on0 = p.r[0] > 0, on1 = p.r[1] > 0;
-    int32_t* out0 = on0 ? p.out[0] + (size_t)c.u * p.r[0] : nullptr;
-    int32_t* out1 = on1 ? p.out[1] + (size_t)c.u * p.r[1] : nullptr;
-    const int lane = tid & 31, wp = tid >> 5;
-    const unsigned below = (1u << lane) - 1u;
-    int* wsum = S.info + 48;   // [8 warps][2] counts of one tile
-    int run0 = base_off[0], run1 = base_off[1], eqs0 = 0, eqs1 = 0;
-#pragma unroll 1
-    for (int e0 = 0; e0 < my_n; e0 += kSel) {
-        const int e = e0 + tid;
-        const bool in = e < my_n;
-        const int x = in ? sc_at(e) : INT_MIN;
-        const bool gt0 = in && (all0 || x > T0), eq0 = in && !all0 && x == T0;
-        const bool gt1 = in && (all1 || x > T1), eq1 = in && !all1 && x == T1;
-        // ties: rank among the tile's equal elements, in position order
-        const unsigned be0 = __ballot_sync(0xffffffffu, eq0), be1 = __ballot_sync(0xffffffffu, eq1);
-        if (lane == 0) { wsum[2 * wp] = __popc(be0); wsum[2 * wp + 1] = __popc(be1); }
-        sel_sync();
-        int pe0 = 0, pe1 = 0, te0 = 0, te1 = 0;
-#pragma unroll
-        for (int w = 0; w < kSel / 32; ++w) {
-            const int a = wsum[2 * w], bq = wsum[2 * w + 1];
-            pe0 += w < wp ? a : 0;
-            pe1 += w < wp ? bq : 0;
-            te0 += a;
-            te1 += bq;
-        }
-        const bool s0 = gt0 || (eq0 && eqs0 + pe0 + __popc(be0 & below) < quota[0]);
-        const bool s1 = gt1 || (eq1 && eqs1 + pe1 + __popc(be1 & below) < quota[1]);
-        eqs0 += te0;
-        eqs1 += te1;
-        sel_sync();
-        // output slots
-        const unsigned bs0 = __ballot_sync(0xffffffffu, s0), bs1 = __ballot_sync(0xffffffffu, s1);
-        if (lane == 0) { wsum[2 * wp] = __popc(bs0); wsum[2 * wp + 1] = __popc(bs1); }
-        sel_sync();
-        int ps0 = 0, ps1 = 0, ts0 = 0, ts1 = 0;
-#pragma unroll
-        for (int w = 0; w < kSel / 32; ++w) {
-            const int a = wsum[2 * w], bq = wsum[2 * w + 1];
-            ps0 += w < wp ? a : 0;
-            ps1 += w < wp ? bq : 0;
-            ts0 += a;
-            ts1 += bq;
-        }
-        if (s0 || s1) {
-            const int pos = full ? (lo + e) : c.pool[lo + e];
-            if (on0 && s0) { const int k2 = run0 + ps0 + __popc(bs0 & below); if (k2 < p.r[0]) out0[k2] = pos; }
-            if (on1 && s1) { const int k2 = run1 + ps1 + __popc(bs1 & below); if (k2 < p.r[1]) out1[k2] = pos; }
-        }
-        run0 += ts0;
-        run1 += ts1;
-        sel_sync();
-    }
+    // ---- ordered write of both tracks
+    write_lists(sc, my_n, lo, full ? nullptr : c.pool, cut[0], cut[1], S.wsum);
     // padding: entries [min(r, n_total), r) = -1
     if (c.cta == p.G - 1) {
-        if (on0) for (int i = min(p.r[0], n_total) + tid; i < p.r[0]; i += kSel) out0[i] = -1;
-        if (on1) for (int i = min(p.r[1], n_total) + tid; i < p.r[1]; i += kSel) out1[i] = -1;
+#pragma unroll 1
+        for (int tr = 0; tr < 2; ++tr)
+            if (cut[tr].out)
+#pragma unroll 1
+                for (int i = min(cut[tr].r, n_total) + tid; i < cut[tr].r; i += kSel) cut[tr].out[i] = -1;
     }
     sel_sync();
     return true;
 }
 
 // ------------------------------------------------------------ scoring helpers
+// Score of one key row (DI/16 int4 chunks) against the index query held in
+// shared memory (HI heads of DI bytes, read as broadcasts). Heads at or past
+// the call's Hi have weight 0.
 template <int HI, int DI>
-struct RegQ {
-    int q[HI][DI / 4];
-    __device__ void load(const int8_t* qs) {
+__device__ __forceinline__ int score_smem(const int4* rowc, const int8_t* qs, const int32_t* w) {
+    int s = 0;
 #pragma unroll
-        for (int h = 0; h < HI; ++h)
-#pragma unroll
-            for (int d = 0; d < DI / 4; ++d) q[h][d] = reinterpret_cast<const int*>(qs + h * DI)[d];
-    }
-    // score of one key row given as DI/16 int4 chunks (chunk c = bytes 16c..16c+15)
-    __device__ __forceinline__ int score(const int4* rowc, const int32_t* w) const {
-        int acc[HI];
-#pragma unroll
-        for (int h = 0; h < HI; ++h) acc[h] = 0;
+    for (int h = 0; h < HI; ++h) {
+        int acc = 0;
+        const int4* qh = reinterpret_cast<const int4*>(qs + h * DI);
 #pragma unroll
         for (int c = 0; c < DI / 16; ++c) {
-            const int4 k = rowc[c];
-#pragma unroll
-            for (int h = 0; h < HI; ++h) {
-                acc[h] = __dp4a(k.x, q[h][4 * c + 0], acc[h]);
-                acc[h] = __dp4a(k.y, q[h][4 * c + 1], acc[h]);
-                acc[h] = __dp4a(k.z, q[h][4 * c + 2], acc[h]);
-                acc[h] = __dp4a(k.w, q[h][4 * c + 3], acc[h]);
-            }
+            const int4 k = rowc[c], qq = qh[c];
+            acc = __dp4a(k.x, qq.x, acc);
+            acc = __dp4a(k.y, qq.y, acc);
+            acc = __dp4a(k.z, qq.z, acc);
+            acc = __dp4a(k.w, qq.w, acc);
         }
-        int s = 0;
-#pragma unroll
-        for (int h = 0; h < HI; ++h) s += w[h] * max(acc[h], 0);
-        return s;
+        s += w[h] * max(acc, 0);
     }
-};
+    return s;
+}
 
 // Generic shapes: Hi <= 16, Di <= 128, queries read from shared memory.
 __device__ __forceinline__ int score_generic(const int4* rowc, int nchunk, const int8_t* qs, int Hi, int Di,
@@ -788,12 +982,21 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c, int di) {
     return off ^ (((off >> 7) & ((1u << b) - 1u)) << 4);
 }
 
+// Key tiles are read once per launch: they are loaded with an L2 evict-first
+// policy, so the stream does not push the kernel's own instructions and the
+// select state out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 __device__ __forceinline__ void tma_load_keys(void* dst, const CUtensorMap* map, int x, int y, int z,
-                                              uint64_t* bar) {
+                                              uint64_t* bar, uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
-        "%4}], [%5];" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+        "{%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
 
@@ -807,7 +1010,7 @@ __device__ __forceinline__ IdxSmem& idx_smem() {
 }
 
 // ------------------------------------------------------------ Full mode on the tensor cores
-// Warps 0-7: epilogue and select; warp 8: TMA producer; warp 9: MMA issuer.
+// Warps 0-15: epilogue and select; warp 16: TMA producer; warp 17: MMA issuer.
 template <int DI>
 __global__ void __launch_bounds__(kTcThreads, 1)
     index_full_tc_kernel(const __grid_constant__ IdxParams p, const __grid_constant__ CUtensorMap kmap) {
@@ -817,7 +1020,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int group = blockIdx.x / p.G;
     const int cta = blockIdx.x % p.G;
     const Slot sl = slot_of(p, group);
-    int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * ((p.chunk + 63) / 64 * 65) : nullptr;
+    int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * p.chunk : nullptr;
     constexpr int kRows = (kStageBytes / DI) < 256 ? (kStageBytes / DI) : 256;   // rows per tile
     constexpr int kBlocks = kRows / 128;                                          // MMA row blocks per tile
     constexpr uint32_t kSwz = DI == 32 ? 6u : DI == 64 ? 4u : 2u;
@@ -829,13 +1032,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) tmem_alloc(&S.tmem_base, 32 * kTmemBufs);
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) { mbar_init(&S.full_bar[i], 1); mbar_init(&S.empty_bar[i], 1); }
-        for (int i = 0; i < kTmemBufs; ++i) { mbar_init(&S.tfull_bar[i], 1); mbar_init(&S.tempty_bar[i], kSel); }
+        for (int i = 0; i < kTmemBufs; ++i) { mbar_init(&S.tfull_bar[i], 1); mbar_init(&S.tempty_bar[i], kSel / 2); }
         S.abort = 0;
         mbar_fence_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_launch_dependents();   // the next kernel may start its own set-up
     const uint32_t tmem = S.tmem_base;
     uint32_t seq = 0;   // tiles processed by this CTA so far (same count in every role)
 
@@ -870,12 +1074,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (warp == kSel / 32) {
             // ---- TMA producer
             if (lane == 0) {
+                const uint64_t pol = l2_evict_first_policy();
                 for (int s2 = 0; s2 < nst; ++s2) {
                     const uint32_t i = seq + s2, slot = i % kStages;
                     if (i >= (uint32_t)kStages &&
                         !mbar_wait(&S.empty_bar[slot], ((i / kStages) - 1) & 1u, p.status, 5)) { S.abort = 1; break; }
                     mbar_arrive_expect_tx(&S.full_bar[slot], (uint32_t)(kRows * DI));
-                    tma_load_keys(S.stage[slot], &kmap, 0, lo + s2 * kRows, b, &S.full_bar[slot]);
+                    tma_load_keys(S.stage[slot], &kmap, 0, lo + s2 * kRows, b, &S.full_bar[slot], pol);
                 }
             }
         } else if (warp == kSel / 32 + 1) {
@@ -902,10 +1107,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
         } else {
-            // ---- epilogue: ReLU and head weights on the int32 accumulators
-            const bool in_block = (warp >> 2) < kBlocks;              // warp-uniform
-            const uint32_t lane_base = tmem + (uint32_t)(warp >> 2) * 16u + ((uint32_t)(warp & 3) * 32u << 16);
-            for (int s2 = 0; s2 < nst; ++s2) {
+            // ---- epilogue: ReLU and head weights on the int32 accumulators. Two
+            // groups of 8 warps take alternate tiles; in a group, warp wl reads
+            // TMEM lane quarter wl % 4 of row block wl / 4.
+            const int egrp = warp >> 3, wl = warp & 7, tl = tid & 255;
+            const bool in_block = (wl >> 2) < kBlocks;                // warp-uniform
+            const uint32_t lane_base = tmem + (uint32_t)(wl >> 2) * 16u + ((uint32_t)(wl & 3) * 32u << 16);
+            for (int s2 = egrp; s2 < nst; s2 += 2) {
                 const uint32_t i = seq + s2, buf = i % kTmemBufs;
                 if (!mbar_wait(&S.tfull_bar[buf], (i / kTmemBufs) & 1u, p.status, 4)) { S.abort = 1; break; }
                 tc_fence_after();
@@ -926,9 +1134,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 tc_fence_before();
                 mbar_arrive(&S.tempty_bar[buf]);
-                const int e = s2 * kRows + tid;
+                const int e = s2 * kRows + tl;
                 if (in_block && e < my_n) {
-                    if (spill) spill[skew(e)] = x; else S.sc[skew(e)] = x;
+                    if (spill) spill[e] = x; else S.sc[e] = x;
                     atomicAdd(&S.hist0[bin0(x)], 1);
                 }
             }
@@ -939,7 +1147,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
         if (tid < kSel) {
             UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, nullptr};
-            if (!select_unit(p, S, sl, c, bar_target, spill) && tid == 0) S.abort = 1;
+            const bool ok = select_unit(p, S, sl, c, bar_target, spill ? spill : S.sc);
+            if (!ok && tid == 0) S.abort = 1;
         }
         __syncthreads();
         if (S.abort) break;
@@ -964,7 +1173,7 @@ __global__ void __launch_bounds__(kSel, 1)
     const Slot sl = slot_of(p, group);
     const bool full = p.mode == CSA2_FULL;
     constexpr bool generic = (HI == 0);
-    int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * ((p.chunk + 63) / 64 * 65) : nullptr;
+    int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * p.chunk : nullptr;
 
     const int epoch = __ldcg(sl.ctrl + CTRL_EPOCH);
     int bar_target = __ldcg(sl.ctrl + CTRL_BAR_BASE);
@@ -974,6 +1183,7 @@ __global__ void __launch_bounds__(kSel, 1)
     if (tid < kStages) mbar_init(&S.full_bar[tid], 1);
     mbar_fence_init();
     __syncthreads();
+    pdl_launch_dependents();   // the next kernel may start its own set-up
     uint32_t stage_seq = 0;   // key tiles issued by this CTA so far
     bool alive = true;
 
@@ -996,18 +1206,17 @@ __global__ void __launch_bounds__(kSel, 1)
             reinterpret_cast<int4*>(S.q)[i] = reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * p.Di)[i];
         for (int i = tid; i < kBins; i += kSel) S.hist0[i] = 0;
         __syncthreads();
-        RegQ<(HI > 0 ? HI : 1), (DI > 0 ? DI : 16)> rq;
-        if (!generic) rq.load(S.q);
 
         int my_n = hi - lo;
         if (full) {
             const int nst = (my_n + rows_per_stage - 1) / rows_per_stage;
+            const uint64_t pol = l2_evict_first_policy();
             if (tid == 0) {
                 for (int s2 = 0; s2 < min(kStages, nst); ++s2) {
                     const uint32_t k = stage_seq + s2;
                     mbar_arrive_expect_tx(&S.full_bar[k % kStages], (uint32_t)(rows_per_stage * p.Di));
                     tma_load_keys(S.stage[k % kStages], &kmap, 0, lo + s2 * rows_per_stage, b,
-                                  &S.full_bar[k % kStages]);
+                                  &S.full_bar[k % kStages], pol);
                 }
             }
             for (int s2 = 0; s2 < nst; ++s2) {
@@ -1021,8 +1230,9 @@ __global__ void __launch_bounds__(kSel, 1)
 #pragma unroll
                     for (int c2 = 0; c2 < 8; ++c2)
                         if (c2 < nchunk) rowc[c2] = *reinterpret_cast<const int4*>(tile + tile_off(tid, c2, p.Di));
-                    const int x = generic ? score_generic(rowc, nchunk, S.q, p.Hi, p.Di, p.w) : rq.score(rowc, p.w);
-                    if (spill) spill[skew(e)] = x; else S.sc[skew(e)] = x;
+                    const int x = generic ? score_generic(rowc, nchunk, S.q, p.Hi, p.Di, p.w)
+                                          : score_smem<(HI > 0 ? HI : 1), (DI > 0 ? DI : 16)>(rowc, S.q, p.w);
+                    if (spill) spill[e] = x; else S.sc[e] = x;
                     atomicAdd(&S.hist0[bin0(x)], 1);
                 }
                 __syncthreads();
@@ -1030,7 +1240,7 @@ __global__ void __launch_bounds__(kSel, 1)
                     const uint32_t k2 = k + kStages;
                     mbar_arrive_expect_tx(&S.full_bar[k2 % kStages], (uint32_t)(rows_per_stage * p.Di));
                     tma_load_keys(S.stage[k2 % kStages], &kmap, 0, lo + (s2 + kStages) * rows_per_stage, b,
-                                  &S.full_bar[k2 % kStages]);
+                                  &S.full_bar[k2 % kStages], pol);
                 }
             }
             stage_seq += nst;
@@ -1069,8 +1279,8 @@ __global__ void __launch_bounds__(kSel, 1)
                     const int e = e0 + q2 * kSel + tid;
                     if (e < my_n) {
                         const int x = generic ? score_generic(rows[q2], nchunk, S.q, p.Hi, p.Di, p.w)
-                                              : rq.score(rows[q2], p.w);
-                        if (spill) spill[skew(e)] = x; else S.sc[skew(e)] = x;
+                                              : score_smem<(HI > 0 ? HI : 1), (DI > 0 ? DI : 16)>(rows[q2], S.q, p.w);
+                        if (spill) spill[e] = x; else S.sc[e] = x;
                         atomicAdd(&S.hist0[bin0(x)], 1);
                     }
                 }
@@ -1078,7 +1288,7 @@ __global__ void __launch_bounds__(kSel, 1)
         }
         __syncthreads();
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
-        alive = select_unit(p, S, sl, c, bar_target, spill);
+        alive = select_unit(p, S, sl, c, bar_target, spill ? spill : S.sc);
         __syncthreads();
     }
     if (alive && cta == 0 && tid == 0) {
@@ -1159,7 +1369,7 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
     chunk = (int)align_up((size_t)std::max(chunk, 1), 256);
     pl.chunk = chunk;
     pl.spill_bytes = 0;
-    if (chunk > kSmemScores) pl.spill_bytes = align_up((size_t)pl.groups * pl.G * ((chunk + 63) / 64 * 65) * 4, 256);
+    if (chunk > kSmemScores) pl.spill_bytes = align_up((size_t)pl.groups * pl.G * chunk * 4, 256);
     return pl;
 }
 
