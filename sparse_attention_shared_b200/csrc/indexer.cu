@@ -264,35 +264,6 @@ __device__ bool group_barrier(int* counter, int target, int32_t* st) {
     return sel_and(ok) != 0;
 }
 
-// Four exclusive scans at once over the select threads (totals in `total`).
-__device__ __forceinline__ int4 sel_scan4(int4 v, int* red, int4& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int4 x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int a = __shfl_up_sync(0xffffffffu, x.x, o), b = __shfl_up_sync(0xffffffffu, x.y, o);
-        const int c = __shfl_up_sync(0xffffffffu, x.z, o), d = __shfl_up_sync(0xffffffffu, x.w, o);
-        if (lane >= o) { x.x += a; x.y += b; x.z += c; x.w += d; }
-    }
-    sel_sync();
-    if (lane == 31) reinterpret_cast<int4*>(red)[warp] = x;
-    sel_sync();
-    if (warp == 0) {
-        int4 s = lane < (kSel / 32) ? reinterpret_cast<int4*>(red)[lane] : make_int4(0, 0, 0, 0);
-#pragma unroll
-        for (int o = 1; o < kSelWarps; o <<= 1) {
-            const int a = __shfl_up_sync(0xffffffffu, s.x, o), b = __shfl_up_sync(0xffffffffu, s.y, o);
-            const int c = __shfl_up_sync(0xffffffffu, s.z, o), d = __shfl_up_sync(0xffffffffu, s.w, o);
-            if (lane >= o) { s.x += a; s.y += b; s.z += c; s.w += d; }
-        }
-        if (lane < kSel / 32) reinterpret_cast<int4*>(red)[kSelWarps + lane] = s;
-    }
-    sel_sync();
-    const int4 we = warp ? reinterpret_cast<int4*>(red)[kSelWarps + warp - 1] : make_int4(0, 0, 0, 0);
-    total = reinterpret_cast<int4*>(red)[2 * kSelWarps - 1];
-    return make_int4(we.x + x.x - v.x, we.y + x.y - v.y, we.z + x.z - v.z, we.w + x.w - v.w);
-}
-
 // In a global 4096-bin histogram, find the bin holding the r-th
 // largest element (1-based). Writes {bin, count above the bin, count in it}.
 __device__ void find_rank_bin_global(const int* hist, int r, int* red, int* out) {
@@ -379,62 +350,56 @@ __device__ __forceinline__ int prefix_total(const int* arr, int n, int* red) {
     return sel_sum(v, red);
 }
 
-// In a shared histogram of kSel * per bins (per <= 8), find the bin holding the
-// r-th largest element (1-based). Writes {bin, count above the bin, count in it}.
-__device__ void find_rank_bin_smem(const int* hist, int per, int r, int* red, int* out) {
-    const int t = threadIdx.x;
-    int h[kBpt];
-    int s = 0;
-#pragma unroll
-    for (int i = 0; i < kBpt; ++i) {
-        h[i] = i < per ? hist[per * t + i] : 0;
-        s += h[i];
-    }
-    int total;
-    const int excl = sel_scan_excl(s, red, total);
-    int above = total - excl - s;    // elements in bins above this thread's range
-    if (above < r && r <= above + s) {
-#pragma unroll
-        for (int i = kBpt - 1; i >= 0; --i) {
-            if (above < r && r <= above + h[i]) {
-                out[0] = per * t + i;
-                out[1] = above;
-                out[2] = h[i];
-            }
-            above += h[i];
-        }
-    }
-    sel_sync();
-}
-
 // The r-th largest value (1-based, with multiplicity) of cx[0..C) in shared
 // memory, by radix passes of up to 12 bits over x - lo (a pass of b bits uses
-// max(kSel, 2^b) bins); every value lies in [lo, hi]. Returns T; need_eq = how
-// many of the elements equal to T are ranked within the first r.
+// max(kSel, 2^b) bins, thread t owning bins [per*t, per*t + per)); every value
+// lies in [lo, hi]. Returns T; need_eq = how many of the elements equal to T are
+// ranked within the first r.
 __device__ __noinline__ int local_select(const int* cx, int C, int r, int lo, int hi, int* hist, int* red,
                                          int* info, int& need_eq) {
-    const int mn = lo;
+    const int t = threadIdx.x;
     const uint32_t w = (uint32_t)((long long)hi - (long long)lo);
     int rem = (w == 0u) ? 0 : 32 - __clz(w);
     uint32_t prefix = 0;
+#pragma unroll 1
     while (rem > 0) {
         const int take = rem < 12 ? rem : 12;
         const int sh = rem - take;
         const int per = max(kSel, 1 << take) / kSel;
-        for (int i = threadIdx.x; i < kSel * per; i += kSel) hist[i] = 0;
+#pragma unroll 1
+        for (int i = t; i < kSel * per; i += kSel) hist[i] = 0;
         sel_sync();
-        for (int i = threadIdx.x; i < C; i += kSel) {
-            const uint32_t v = (uint32_t)((long long)cx[i] - (long long)mn);
+#pragma unroll 1
+        for (int i = t; i < C; i += kSel) {
+            const uint32_t v = (uint32_t)((long long)cx[i] - (long long)lo);
             if ((uint32_t)(((uint64_t)v) >> (sh + take)) == prefix) atomicAdd(&hist[(v >> sh) & ((1u << take) - 1u)], 1);
         }
         sel_sync();
-        find_rank_bin_smem(hist, per, r, red, info);
+        int s = 0;
+#pragma unroll 1
+        for (int i = 0; i < per; ++i) s += hist[per * t + i];
+        int total;
+        const int excl = sel_scan_excl(s, red, total);
+        int above = total - excl - s;    // elements in bins above this thread's range
+        if (above < r && r <= above + s) {
+#pragma unroll 1
+            for (int i = per - 1; i >= 0; --i) {
+                const int h = hist[per * t + i];
+                if (r <= above + h) {
+                    info[0] = per * t + i;
+                    info[1] = above;
+                    break;
+                }
+                above += h;
+            }
+        }
+        sel_sync();
         r -= info[1];
         prefix = (prefix << take) | (uint32_t)info[0];
         rem = sh;
     }
     need_eq = r;
-    return (int)((long long)mn + (long long)prefix);
+    return (int)((long long)lo + (long long)prefix);
 }
 
 // ------------------------------------------------------------ select + write
@@ -483,32 +448,31 @@ __device__ void prefix_interval(int level, uint64_t prefix, int& lo, int& hi) {
     hi = (int)(a - 1);
 }
 
-// The chunk's scores as int4 vectors: element e sits at index e, in shared memory
-// or, for chunks longer than kSmemScores, in this CTA's spill area.
-__device__ __forceinline__ int4 ld_scores4(const int* sc, int v) { return reinterpret_cast<const int4*>(sc)[v]; }
+// The chunk's scores: element e sits at sc[e], in shared memory or, for chunks
+// longer than kSmemScores, in this CTA's spill area (padding past n is ignored).
+// Each warp walks one contiguous range of 32-element steps (lane = element in
+// the step), so a warp meets its elements in position order and the warps'
+// ranges follow each other.
+template <bool kSpill>
+__device__ __forceinline__ int ld_score(const int* sc, int e) {
+    if constexpr (kSpill) return __ldcg(sc + e);
+    else return sc[e];
+}
 
-// Steps of 32 vectors (128 elements) owned by this warp: one contiguous range per
-// warp, so each warp meets its elements in position order.
 __device__ __forceinline__ void warp_steps(int n, int& s0, int& s1) {
-    const int nstep = (n + 127) >> 7;
-    const int spw = (nstep + kSel / 32 - 1) / (kSel / 32);
+    const int nstep = (n + 31) >> 5;
+    const int spw = (nstep + kSelWarps - 1) / kSelWarps;
     s0 = min(nstep, (threadIdx.x >> 5) * spw);
     s1 = min(nstep, s0 + spw);
 }
 
 __device__ __forceinline__ int4 warp_sum4(int4 v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
-        v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
-        v.z += __shfl_xor_sync(0xffffffffu, v.z, o);
-        v.w += __shfl_xor_sync(0xffffffffu, v.w, o);
-    }
-    return v;
+    return make_int4(__reduce_add_sync(0xffffffffu, v.x), __reduce_add_sync(0xffffffffu, v.y),
+                     __reduce_add_sync(0xffffffffu, v.z), __reduce_add_sync(0xffffffffu, v.w));
 }
 
 // Totals of two int4 over the select threads (two barriers).
-__device__ __noinline__ void sel_total8(int4& a, int4& b, int* red) {
+__device__ __forceinline__ void sel_total8(int4& a, int4& b, int* red) {
     a = warp_sum4(a);
     b = warp_sum4(b);
     sel_sync();
@@ -518,7 +482,7 @@ __device__ __noinline__ void sel_total8(int4& a, int4& b, int* red) {
     a = make_int4(0, 0, 0, 0);
     b = a;
 #pragma unroll 1
-    for (int w = 0; w < kSel / 32; ++w) {
+    for (int w = 0; w < kSelWarps; ++w) {
         const int4 x = r4[2 * w], y = r4[2 * w + 1];
         a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
         b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
@@ -528,78 +492,56 @@ __device__ __noinline__ void sel_total8(int4& a, int4& b, int* red) {
 // Candidates of both tracks (scores in [lo0, hi0] / [lo1, hi1]; lo > hi = off)
 // into lbuf[0..) and lbuf[kCandCap..) as (score, element index + base). A warp
 // reserves room once per step that holds candidates; the order is free.
-__device__ __noinline__ void gather_cands(const int* sc, int n, int base, int lo0, int hi0, int lo1, int hi1,
+template <bool kSpill>
+__device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int lo0, int hi0, int lo1, int hi1,
                                           int2* lbuf, int* lcnt) {
     const int lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
     int s0, s1;
     warp_steps(n, s0, s1);
 #pragma unroll 1
     for (int st = s0; st < s1; ++st) {
-        const int v = st * 32 + lane;
-        const int4 x4 = ld_scores4(sc, v);
-        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
-        unsigned m0 = 0, m1 = 0;   // bit q: sub-element q is a candidate
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const bool ok = 4 * v + q < n;
-            m0 |= (ok && xs[q] >= lo0 && xs[q] <= hi0) ? 1u << q : 0u;
-            m1 |= (ok && xs[q] >= lo1 && xs[q] <= hi1) ? 1u << q : 0u;
-        }
-        if (!__any_sync(0xffffffffu, (m0 | m1) != 0)) continue;
-        const int c0 = __popc(m0), c1 = __popc(m1);
-        // lanes' counts -> exclusive prefix within the warp
-        int p0 = c0, p1 = c1;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y0 = __shfl_up_sync(0xffffffffu, p0, o), y1 = __shfl_up_sync(0xffffffffu, p1, o);
-            if (lane >= o) { p0 += y0; p1 += y1; }
-        }
+        const int e = st * 32 + lane;
+        const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
+        const bool m0 = e < n && x >= lo0 && x <= hi0, m1 = e < n && x >= lo1 && x <= hi1;
+        const unsigned b0 = __ballot_sync(0xffffffffu, m0), b1 = __ballot_sync(0xffffffffu, m1);
+        if ((b0 | b1) == 0u) continue;
         int w0 = 0, w1 = 0;
-        if (lane == 31) {
-            w0 = p0 ? atomicAdd(lcnt, p0) : 0;
-            w1 = p1 ? atomicAdd(lcnt + 1, p1) : 0;
+        if (lane == 0) {
+            w0 = b0 ? atomicAdd(lcnt, __popc(b0)) : 0;
+            w1 = b1 ? atomicAdd(lcnt + 1, __popc(b1)) : 0;
         }
-        w0 = __shfl_sync(0xffffffffu, w0, 31) + p0 - c0;
-        w1 = __shfl_sync(0xffffffffu, w1, 31) + p1 - c1;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int2 cv = make_int2(xs[q], base + 4 * v + q);
-            if (m0 & (1u << q)) { if (w0 < kCandCap) lbuf[w0] = cv; w0++; }
-            if (m1 & (1u << q)) { if (w1 < kCandCap) lbuf[kCandCap + w1] = cv; w1++; }
-        }
+        w0 = __shfl_sync(0xffffffffu, w0, 0) + __popc(b0 & below);
+        w1 = __shfl_sync(0xffffffffu, w1, 0) + __popc(b1 & below);
+        const int2 cv = make_int2(x, base + e);
+        if (m0 && w0 < kCandCap) lbuf[w0] = cv;
+        if (m1 && w1 < kCandCap) lbuf[kCandCap + w1] = cv;
     }
 }
 
 // Histogram of digit `lv` over the elements in [lo_t, hi_t] (they share digits 0..lv-1).
+template <bool kSpill>
 __device__ __noinline__ void radix_hist(const int* sc, int n, int lo_t, int hi_t, int lv, int* hist) {
-    const int lane = threadIdx.x & 31;
     int s0, s1;
     warp_steps(n, s0, s1);
 #pragma unroll 1
     for (int st = s0; st < s1; ++st) {
-        const int v = st * 32 + lane;
-        const int4 x4 = ld_scores4(sc, v);
-        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-            const int x = xs[q];
-            if (4 * v + q < n && x >= lo_t && x <= hi_t) atomicAdd(&hist[digit_at(ext_key(x), lv)], 1);
-        }
+        const int e = st * 32 + (threadIdx.x & 31);
+        const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
+        if (e < n && x >= lo_t && x <= hi_t) atomicAdd(&hist[digit_at(ext_key(x), lv)], 1);
     }
 }
 
 // Number of this thread's elements in [lo_t, hi_t].
+template <bool kSpill>
 __device__ __noinline__ int count_range(const int* sc, int n, int lo_t, int hi_t) {
-    const int lane = threadIdx.x & 31;
     int s0, s1, cnt = 0;
     warp_steps(n, s0, s1);
 #pragma unroll 1
     for (int st = s0; st < s1; ++st) {
-        const int v = st * 32 + lane;
-        const int4 x4 = ld_scores4(sc, v);
-        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) cnt += (4 * v + q < n && xs[q] >= lo_t && xs[q] <= hi_t);
+        const int e = st * 32 + (threadIdx.x & 31);
+        const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
+        cnt += (e < n && x >= lo_t && x <= hi_t);
     }
     return cnt;
 }
@@ -619,25 +561,23 @@ __device__ __forceinline__ void take_flags(int x, bool ok, const ListCut& c, boo
 
 // Ordered write of both tracks: pass 1 counts per warp, pass 2 walks the same
 // ranges with running counts and ballots for the ranks inside a step.
-__device__ __noinline__ void write_lists(const int* sc, int n, int base, const int32_t* pool, ListCut c0,
+template <bool kSpill>
+__device__ __forceinline__ void write_lists(const int* sc, int n, int base, const int32_t* pool, ListCut c0,
                                          ListCut c1, int* wsum) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const unsigned below = (1u << lane) - 1u;
     int s0, s1;
     warp_steps(n, s0, s1);
     int4 cnt = make_int4(0, 0, 0, 0);   // gt0, eq0, gt1, eq1
 #pragma unroll 1
     for (int st = s0; st < s1; ++st) {
-        const int v = st * 32 + lane;
-        const int4 x4 = ld_scores4(sc, v);
-        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            bool g, e;
-            take_flags(xs[q], 4 * v + q < n, c0, g, e);
-            cnt.x += g; cnt.y += e;
-            take_flags(xs[q], 4 * v + q < n, c1, g, e);
-            cnt.z += g; cnt.w += e;
-        }
+        const int e = st * 32 + lane;
+        const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
+        bool g, q;
+        take_flags(x, e < n, c0, g, q);
+        cnt.x += g; cnt.y += q;
+        take_flags(x, e < n, c1, g, q);
+        cnt.z += g; cnt.w += q;
     }
     cnt = warp_sum4(cnt);
     int4* w4 = reinterpret_cast<int4*>(wsum);
@@ -651,43 +591,23 @@ __device__ __noinline__ void write_lists(const int* sc, int n, int base, const i
     }
 #pragma unroll 1
     for (int st = s0; st < s1; ++st) {
-        const int v = st * 32 + lane;
-        const int4 x4 = ld_scores4(sc, v);
-        const int xs[4] = {x4.x, x4.y, x4.z, x4.w};
-        unsigned fg0 = 0, fe0 = 0, fg1 = 0, fe1 = 0;   // bit q: sub-element q's flags
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            bool g, e;
-            take_flags(xs[q], 4 * v + q < n, c0, g, e);
-            fg0 |= g ? 1u << q : 0u; fe0 |= e ? 1u << q : 0u;
-            take_flags(xs[q], 4 * v + q < n, c1, g, e);
-            fg1 |= g ? 1u << q : 0u; fe1 |= e ? 1u << q : 0u;
+        const int e = st * 32 + lane;
+        const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
+        bool g0, q0, g1, q1;
+        take_flags(x, e < n, c0, g0, q0);
+        take_flags(x, e < n, c1, g1, q1);
+        const unsigned bg0 = __ballot_sync(0xffffffffu, g0), bq0 = __ballot_sync(0xffffffffu, q0);
+        const unsigned bg1 = __ballot_sync(0xffffffffu, g1), bq1 = __ballot_sync(0xffffffffu, q1);
+        if ((bg0 | bq0 | bg1 | bq1) == 0u) continue;
+        const int og0 = rg0 + __popc(bg0 & below), oq0 = re0 + __popc(bq0 & below);
+        const int og1 = rg1 + __popc(bg1 & below), oq1 = re1 + __popc(bq1 & below);
+        const bool t0 = g0 || (q0 && oq0 < c0.quota), t1 = g1 || (q1 && oq1 < c1.quota);
+        if (t0 || t1) {
+            const int pos = pool ? pool[base + e] : base + e;
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (k < c0.r) c0.out[k] = pos; }
+            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if (k < c1.r) c1.out[k] = pos; }
         }
-        if (!__any_sync(0xffffffffu, (fg0 | fe0 | fg1 | fe1) != 0)) continue;
-        // exclusive prefix of the four counts over the lanes
-        int4 mine = make_int4(__popc(fg0), __popc(fe0), __popc(fg1), __popc(fe1)), pre = mine;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int a = __shfl_up_sync(0xffffffffu, pre.x, o), b = __shfl_up_sync(0xffffffffu, pre.y, o);
-            const int cc = __shfl_up_sync(0xffffffffu, pre.z, o), d = __shfl_up_sync(0xffffffffu, pre.w, o);
-            if (lane >= o) { pre.x += a; pre.y += b; pre.z += cc; pre.w += d; }
-        }
-        int og0 = rg0 + pre.x - mine.x, oe0 = re0 + pre.y - mine.y;
-        int og1 = rg1 + pre.z - mine.z, oe1 = re1 + pre.w - mine.w;
-        rg0 += __shfl_sync(0xffffffffu, pre.x, 31); re0 += __shfl_sync(0xffffffffu, pre.y, 31);
-        rg1 += __shfl_sync(0xffffffffu, pre.z, 31); re1 += __shfl_sync(0xffffffffu, pre.w, 31);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const bool g0 = fg0 >> q & 1u, e0 = fe0 >> q & 1u, g1 = fg1 >> q & 1u, e1 = fe1 >> q & 1u;
-            const bool t0 = g0 || (e0 && oe0 < c0.quota), t1 = g1 || (e1 && oe1 < c1.quota);
-            if (t0 || t1) {
-                const int e = base + 4 * v + q;
-                const int pos = pool ? pool[e] : e;
-                if (t0) { const int k = c0.base + og0 + min(oe0, c0.quota); if (k < c0.r) c0.out[k] = pos; }
-                if (t1) { const int k = c1.base + og1 + min(oe1, c1.quota); if (k < c1.r) c1.out[k] = pos; }
-            }
-            og0 += g0; oe0 += e0; og1 += g1; oe1 += e1;
-        }
+        rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
     }
 }
 
@@ -695,7 +615,8 @@ __device__ __noinline__ void write_lists(const int* sc, int n, int base, const i
 // positions. Runs on threads [0, kSel). `sc` holds the chunk's scores (element
 // index order) and S.hist0 their level-0 histogram. The two tracks (pool P and
 // top-k) share every pass and every group barrier. Returns false on a timeout.
-__device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c,
+template <bool kSpill>
+__device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c,
                                          int& bar_target, const int* sc) {
     const int tid = threadIdx.x;
     const bool full = p.mode == CSA2_FULL;
@@ -729,7 +650,7 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
     }
     Track tk[2];
     int rq[2];
-#pragma unroll 1
+#pragma unroll
     for (int tr = 0; tr < 2; ++tr) {
         tk[tr] = Track{TS_OFF, 0, 0, 0, 0, 1, 0, 0};
         const int r = p.r[tr];
@@ -750,7 +671,7 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
         }
         int4 ta = make_int4(a0, a1, 0, 0), tb = make_int4(0, 0, 0, 0);
         sel_total8(ta, tb, S.red);
-#pragma unroll 1
+#pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
             if (rq[tr] <= 0) continue;
             Track& k = tk[tr];
@@ -775,7 +696,7 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
             int* lcnt = S.info + 40;
             if (tid == 0) { lcnt[0] = 0; lcnt[1] = 0; }
             sel_sync();
-            gather_cands(sc, my_n, lo, g0on ? tk[0].lo : 1, g0on ? tk[0].hi : 0, g1on ? tk[1].lo : 1,
+            gather_cands<kSpill>(sc, my_n, lo, g0on ? tk[0].lo : 1, g0on ? tk[0].hi : 0, g1on ? tk[1].lo : 1,
                          g1on ? tk[1].hi : 0, lbuf, lcnt);
             sel_sync();
             if (tid == 0 || tid == 32) {
@@ -787,7 +708,7 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
                 if (on) sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = tk[tr].above;
             }
             sel_sync();
-#pragma unroll 1
+#pragma unroll
             for (int tr = 0; tr < 2; ++tr) {
                 const int n_mine = S.info[46 + tr], gbase = S.info[44 + tr];
 #pragma unroll 1
@@ -795,7 +716,7 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
                     if (gbase + i < kCandCap) sl.cand[tr * kCandCap + gbase + i] = lbuf[tr * kCandCap + i];
             }
         }
-#pragma unroll 1
+#pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
             Track& k = tk[tr];
             if (k.state == TS_RADIX) {
@@ -805,13 +726,13 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
 #pragma unroll 1
                 for (int i = tid; i < kBins; i += kSel) hl[i] = 0;
                 sel_sync();
-                radix_hist(sc, my_n, k.lo, k.hi, k.level + 1, hl);
+                radix_hist<kSpill>(sc, my_n, k.lo, k.hi, k.level + 1, hl);
                 sel_sync();
                 push_hist(hl, sl.gl + (2 * tr + k.level) * kBins);
             } else if (k.state == TS_EQ) {
                 // the prefix is the whole key: the score is exact; count own ties
                 any = true;
-                const int eq = sel_sum(count_range(sc, my_n, k.lo, k.hi), S.red);
+                const int eq = sel_sum(count_range<kSpill>(sc, my_n, k.lo, k.hi), S.red);
                 if (tid == 0) {
                     sl.pub[(tr * 3 + 0) * kMaxG + c.cta] = k.above;
                     sl.pub[(tr * 3 + 1) * kMaxG + c.cta] = eq;
@@ -822,7 +743,7 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
         bar_target += p.G;
         if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
         bool pending = false;
-#pragma unroll 1
+#pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
             Track& k = tk[tr];
             if (k.state == TS_RADIX) {
@@ -857,9 +778,11 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
         int v = 0;
         if (grp < 4 && fin && ci < c.cta && (grp < 2 || st_g == TS_FIN_EQ))
             v = __ldcg(sl.pub + (tr_g * 3 + (grp >> 1)) * kMaxG + ci);
-        int4 tot;
-        sel_scan4(make_int4(grp == 0 ? v : 0, grp == 1 ? v : 0, grp == 2 ? v : 0, grp == 3 ? v : 0), S.red, tot);
-        const int prev[2] = {tot.x, tot.y}, eqb[2] = {tot.z, tot.w};
+        v = __reduce_add_sync(0xffffffffu, v);
+        if ((tid & 31) == 0 && tid < 256) S.red[tid >> 5] = v;
+        sel_sync();
+        const int prev[2] = {S.red[0] + S.red[1], S.red[2] + S.red[3]};
+        const int eqb[2] = {S.red[4] + S.red[5], S.red[6] + S.red[7]};
         // candidates of both tracks, one load round
         int* cx0 = reinterpret_cast<int*>(&S.stage[0][0]);
         const int n0 = tk[0].state == TS_FIN_CAND ? tk[0].C : 0, n1 = tk[1].state == TS_FIN_CAND ? tk[1].C : 0;
@@ -872,7 +795,7 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
         }
         sel_sync();
         int T[2] = {INT_MAX, INT_MAX}, need[2] = {0, 0};
-#pragma unroll 1
+#pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
             const Track& k = tk[tr];
             if (k.state == TS_FIN_CAND) {
@@ -897,7 +820,7 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
         }
         sel_total8(ca, cb, S.red);
         const int gtb[2] = {ca.x, ca.z}, eqc[2] = {ca.y, ca.w}, mye[2] = {cb.x, cb.y};
-#pragma unroll 1
+#pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
             const int st = tk[tr].state;
             ListCut& lc = cut[tr];
@@ -918,10 +841,10 @@ __device__ __noinline__ bool select_unit(const IdxParams& p, IdxSmem& S, const S
     }
 
     // ---- ordered write of both tracks
-    write_lists(sc, my_n, lo, full ? nullptr : c.pool, cut[0], cut[1], S.wsum);
+    write_lists<kSpill>(sc, my_n, lo, full ? nullptr : c.pool, cut[0], cut[1], S.wsum);
     // padding: entries [min(r, n_total), r) = -1
     if (c.cta == p.G - 1) {
-#pragma unroll 1
+#pragma unroll
         for (int tr = 0; tr < 2; ++tr)
             if (cut[tr].out)
 #pragma unroll 1
@@ -1147,7 +1070,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
         if (tid < kSel) {
             UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, nullptr};
-            const bool ok = select_unit(p, S, sl, c, bar_target, spill ? spill : S.sc);
+            const bool ok = spill ? select_unit<true>(p, S, sl, c, bar_target, spill)
+                                  : select_unit<false>(p, S, sl, c, bar_target, S.sc);
             if (!ok && tid == 0) S.abort = 1;
         }
         __syncthreads();
@@ -1288,7 +1212,8 @@ __global__ void __launch_bounds__(kSel, 1)
         }
         __syncthreads();
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
-        alive = select_unit(p, S, sl, c, bar_target, spill ? spill : S.sc);
+        alive = spill ? select_unit<true>(p, S, sl, c, bar_target, spill)
+                      : select_unit<false>(p, S, sl, c, bar_target, S.sc);
         __syncthreads();
     }
     if (alive && cta == 0 && tid == 0) {
