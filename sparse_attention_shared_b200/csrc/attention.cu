@@ -21,6 +21,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstddef>
 #include <cstring>
 
 #include "csa2_common.cuh"
@@ -48,6 +49,7 @@ struct AttnParams {
     float* part;    // [units][ntiles][HQP * (D + 2)]
     int* tickets;   // [units]
     int32_t* status;
+    int list_ready; // the list and the cache were complete before the previous kernel began
 };
 
 template <int HQP>
@@ -412,29 +414,62 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
 // partials through distributed shared memory: CTA r writes the heads
 // h = r, r + CS, ... . No partial goes through global memory.
 constexpr int kCLBuf = 4 * kPanelBytes;   // 64 KB: a 256-row global tile or a local K+V tile
+constexpr int kClThreads = 256;           // one key row of a global tile per thread
 
 template <int HQP>
-struct __align__(1024) AttnClSmem {
+struct AttnClSmem {   // placed at a 1024-byte-aligned address (operand tiles need it)
     uint8_t tbuf[kCLBuf];
-    uint8_t qbuf[2 * HQP * 128];
-    uint8_t pbuf[4 * HQP * 128];          // P as [HQP rows x 256 keys] in 64-key panels
+    // Q as [HQP rows x D] (two 64-element panels), then, once S = K Q^T has been
+    // computed, P as [HQP rows x 256 keys] in four 64-key panels
+    uint8_t qpbuf[4 * HQP * 128];
     uint32_t lut[256];
-    float red[4][HQP];
+    float red[kClThreads / 32][HQP];      // per-warp head maxima, then sums
+    float mfin[HQP], lfin[HQP];
     float part_m[HQP], part_l[HQP];
     uint64_t bar_tma, bar_s, bar_o;
     uint32_t tmem_base;
 };
 
+static_assert(offsetof(AttnClSmem<16>, qpbuf) % 1024 == 0 && offsetof(AttnClSmem<32>, qpbuf) % 1024 == 0,
+              "operand alignment");
+static_assert(sizeof(AttnClSmem<16>) + 1024 <= 80 * 1024, "two clustered-attention CTAs per SM");
+
+// Reduce V values per lane (V = 16 or 32, one per head) across the 32 lanes of a
+// warp with halving exchanges: after the call, lane l holds in v[0] the result for
+// head (l >> 1) & 15 (V = 16) or l & 31 (V = 32). 31 or 16 shuffles instead of 5*V.
+template <int V, bool kMax>
+__device__ __forceinline__ float warp_transpose_reduce(float (&v)[V]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int half = V / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = up ? v[i] : v[i + half];
+            const float keep = up ? v[i + half] : v[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, bit);
+            v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+    if (V == 16) {   // lanes l and l ^ 1 still hold partials of the same head
+        const float recv = __shfl_xor_sync(0xffffffffu, v[0], 1);
+        v[0] = kMax ? fmaxf(v[0], recv) : v[0] + recv;
+    }
+    return v[0];
+}
+
 template <int HQP, int D>
-__global__ void __launch_bounds__(kAttnThreads)
+__global__ void __launch_bounds__(kClThreads, 2)
     sparse_attn_cl_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap kl_map,
                           const __grid_constant__ CUtensorMap vl_map) {
+    static_assert(HQP == 16 || HQP == 32, "head padding");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     AttnClSmem<HQP>& S =
         *reinterpret_cast<AttnClSmem<HQP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     constexpr uint32_t kCols = (3 * HQP <= 32) ? 32 : (3 * HQP <= 64 ? 64 : 128);
     constexpr int kPanels = D / 64;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    constexpr int kWarps = kClThreads / 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int CS = gridDim.x;
     const int rank = (int)cluster_ctarank();
     const int u = blockIdx.y;
@@ -451,27 +486,24 @@ __global__ void __launch_bounds__(kAttnThreads)
         mbar_init(&S.bar_o, 1);
         mbar_fence_init();
     }
-    for (int i = tid; i < 256; i += kAttnThreads)
+    for (int i = tid; i < 256; i += kClThreads)
         S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
-    pdl_wait();
-    pdl_launch_dependents();
+    // A global CTA of a layer whose list and cache were complete before the previous
+    // kernel began (a Reuse layer of a stack) gathers and dequantises its rows before
+    // waiting for that kernel; everything else (Q, the window) is read after the wait.
+    const bool pre = glob && p.list_ready;
+    if (!pre) {
+        pdl_wait();
+        pdl_launch_dependents();
+    }
 
-    // ---- 1. loads that depend on nothing else
+    // ---- 1. positions and list entries; row tid of the tile is this thread's
     int t = p.q_pos[u];
     const int base = p.local_base[b];
-    int s0 = -1, s1 = -1;
+    int s0 = -1;
     if (glob) {
-        const int j0 = rank * 2 * kTileKeys + tid, j1 = j0 + kTileKeys;
-        s0 = (j0 < p.k) ? p.topk[(size_t)u * p.k + j0] : -1;
-        s1 = (j1 < p.k) ? p.topk[(size_t)u * p.k + j1] : -1;
-    }
-    uint4 qv[(HQP * D / 8 + kAttnThreads - 1) / kAttnThreads];
-#pragma unroll
-    for (int q = 0; q < (int)(sizeof(qv) / sizeof(qv[0])); ++q) {
-        const int i = tid + q * kAttnThreads;
-        const int h = i / (D / 8), c = i % (D / 8);
-        qv[q] = make_uint4(0, 0, 0, 0);
-        if (i < HQP * (D / 8) && h < p.Hq) qv[q] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
+        const int j0 = rank * 2 * kTileKeys + tid;
+        s0 = (j0 < p.k) ? __ldcg(p.topk + (size_t)u * p.k + j0) : -1;
     }
     if (t < 0 || t >= p.N) {
         if (tid == 0 && rank == 0) report(p.status, CSA2_ERR_RANGE, u);
@@ -480,33 +512,29 @@ __global__ void __launch_bounds__(kAttnThreads)
     const int lo_w = max(max(base, t - p.W + 1), 0);
 
     // ---- 2. the tile's rows
-    bool v0 = false, v1 = false;
-    uint4 c0[D / 32], c1[D / 32];
-    uint32_t sc0[D / 64], sc1[D / 64];
+    bool v0 = false;
+    uint4 c0[D / 32];
+    uint32_t sc0[D / 64];
     if (glob) {
         if (s0 >= 0 && (s0 > t || s0 >= p.N)) { report(p.status, CSA2_ERR_RANGE, u); s0 = -1; }
-        if (s1 >= 0 && (s1 > t || s1 >= p.N)) { report(p.status, CSA2_ERR_RANGE, u); s1 = -1; }
         v0 = s0 >= 0;
-        v1 = s1 >= 0;
-        auto ldrow = [&](int s, uint4 (&cw)[D / 32], uint32_t (&sw)[D / 64]) {
-            const size_t row = (size_t)b * p.N + s;
+        if (v0) {
+            const size_t row = (size_t)b * p.N + s0;
             const uint4* cp = reinterpret_cast<const uint4*>(p.kv_fp4 + row * (D / 2));
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) cw[q] = __ldg(cp + q);
+            for (int q = 0; q < D / 32; ++q) c0[q] = __ldg(cp + q);
             if (D == 128) {
                 const uint2 s2 = __ldg(reinterpret_cast<const uint2*>(p.kv_scale + row * 8));
-                sw[0] = s2.x;
-                sw[(D / 64) - 1] = s2.y;
+                sc0[0] = s2.x;
+                sc0[(D / 64) - 1] = s2.y;
             } else {
-                sw[0] = __ldg(reinterpret_cast<const uint32_t*>(p.kv_scale + row * 4));
+                sc0[0] = __ldg(reinterpret_cast<const uint32_t*>(p.kv_scale + row * 4));
             }
-        };
-        if (v0) ldrow(s0, c0, sc0);
-        if (v1) ldrow(s1, c1, sc1);
+        }
     } else {
         const int lt = rank - ngt2;
         const int pos = lo_w + lt * kTileKeys + tid;
-        v0 = (t >= 0) && (p.W > 0) && (pos <= t) && (pos - base) < p.Lloc;
+        v0 = tid < kTileKeys && (t >= 0) && (p.W > 0) && (pos <= t) && (pos - base) < p.Lloc;
         if (tid == 0) {
             mbar_arrive_expect_tx(&S.bar_tma, 2u * kPanels * kPanelBytes);
             const int y = lo_w - base + lt * kTileKeys;
@@ -517,18 +545,12 @@ __global__ void __launch_bounds__(kAttnThreads)
             }
         }
     }
-#pragma unroll
-    for (int q = 0; q < (int)(sizeof(qv) / sizeof(qv[0])); ++q) {
-        const int i = tid + q * kAttnThreads;
-        const int h = i / (D / 8), c = i % (D / 8);
-        if (i < HQP * (D / 8)) *reinterpret_cast<uint4*>(S.qbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = qv[q];
-    }
     if (glob && D == 64) {   // the value operand's second M-half stays zero
-        for (int i = tid; i < 2 * kPanelBytes / 16; i += kAttnThreads)
+        for (int i = tid; i < 2 * kPanelBytes / 16; i += kClThreads)
             reinterpret_cast<uint4*>(S.tbuf + 2 * kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
     }
     if (!glob && D == 64) {
-        for (int i = tid; i < kPanelBytes / 16; i += kAttnThreads) {
+        for (int i = tid; i < kPanelBytes / 16; i += kClThreads) {
             reinterpret_cast<uint4*>(S.tbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
             reinterpret_cast<uint4*>(S.tbuf + 3 * kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
         }
@@ -536,42 +558,49 @@ __global__ void __launch_bounds__(kAttnThreads)
     __syncthreads();   // the table is ready
     bool ok = true;
     if (glob) {
-        // global tile panels hold 256 rows: panel p at p * 2 * kPanelBytes
-        auto dequant = [&](int r, bool v, const uint4 (&cw)[D / 32], const uint32_t (&sw)[D / 64]) {
+        // global tile panels hold 256 rows: panel p at p * 2 * kPanelBytes; row tid
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-                uint4 o = make_uint4(0, 0, 0, 0);
-                if (v) {
-                    const uint4 w4 = cw[c >> 2];
-                    const uint32_t w = (c & 3) == 0 ? w4.x : (c & 3) == 1 ? w4.y : (c & 3) == 2 ? w4.z : w4.w;
-                    const uint32_t g = c >> 1;
-                    const uint32_t s16 = e4m3_bf16_bits((sw[g >> 2] >> (8 * (g & 3))) & 0xFFu);
-                    const uint32_t s2x = s16 | (s16 << 16);
-                    o.x = bf16x2_mul(S.lut[w & 0xFFu], s2x);
-                    o.y = bf16x2_mul(S.lut[(w >> 8) & 0xFFu], s2x);
-                    o.z = bf16x2_mul(S.lut[(w >> 16) & 0xFFu], s2x);
-                    o.w = bf16x2_mul(S.lut[w >> 24], s2x);
-                }
-                *reinterpret_cast<uint4*>(S.tbuf + (c >> 3) * (2 * kPanelBytes) + sw128(r, c & 7)) = o;
+        for (int c = 0; c < D / 8; ++c) {
+            uint4 o = make_uint4(0, 0, 0, 0);
+            if (v0) {
+                const uint4 w4 = c0[c >> 2];
+                const uint32_t w = (c & 3) == 0 ? w4.x : (c & 3) == 1 ? w4.y : (c & 3) == 2 ? w4.z : w4.w;
+                const uint32_t g = c >> 1;
+                const uint32_t s16 = e4m3_bf16_bits((sc0[g >> 2] >> (8 * (g & 3))) & 0xFFu);
+                const uint32_t s2x = s16 | (s16 << 16);
+                o.x = bf16x2_mul(S.lut[w & 0xFFu], s2x);
+                o.y = bf16x2_mul(S.lut[(w >> 8) & 0xFFu], s2x);
+                o.z = bf16x2_mul(S.lut[(w >> 16) & 0xFFu], s2x);
+                o.w = bf16x2_mul(S.lut[w >> 24], s2x);
             }
-        };
-        dequant(tid, v0, c0, sc0);
-        dequant(tid + kTileKeys, v1, c1, sc1);
-    } else {
-        ok = mbar_wait(&S.bar_tma, 0, p.status, 12);
+            *reinterpret_cast<uint4*>(S.tbuf + (c >> 3) * (2 * kPanelBytes) + sw128(tid, c & 7)) = o;
+        }
     }
+    if (pre) {
+        pdl_wait();
+        pdl_launch_dependents();
+    }
+    // the query (it depends on the previous layer)
+#pragma unroll
+    for (int q = 0; q < (HQP * D / 8 + kClThreads - 1) / kClThreads; ++q) {
+        const int i = tid + q * kClThreads;
+        const int h = i / (D / 8), c = i % (D / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (i < HQP * (D / 8) && h < p.Hq) v = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
+        if (i < HQP * (D / 8)) *reinterpret_cast<uint4*>(S.qpbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = v;
+    }
+    if (!glob) ok = mbar_wait(&S.bar_tma, 0, p.status, 12);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int nblk = glob ? 2 : 1;
     const uint32_t panel_stride = glob ? 2 * kPanelBytes : kPanelBytes;
 
     // ---- 3. S = K Q^T per 128-row block
     if (tid == 0) {
-        const uint32_t ka = smem_u32(S.tbuf), qa = smem_u32(S.qbuf);
+        const uint32_t ka = smem_u32(S.tbuf), qa = smem_u32(S.qpbuf);
         constexpr uint32_t idesc = idesc_bf16(128, HQP, 0);
         for (int blk = 0; blk < nblk; ++blk) {
 #pragma unroll
@@ -586,76 +615,66 @@ __global__ void __launch_bounds__(kAttnThreads)
     ok = mbar_wait(&S.bar_s, 0, p.status, 10) && ok;
     tc_fence_after();
 
-    // ---- 4. softmax partial over the tile's rows (two rows per thread on a global tile)
-    float a0[HQP], a1[HQP];
+    // ---- 4. softmax partial over the tile's rows: thread tid holds key tid, which
+    // sits in row block tid / 128, TMEM lane tid % 128 (warp w reads lane quarter w % 4)
+    float a[HQP];
     {
+        const uint32_t ta = tmem + (uint32_t)(tid >> 7) * HQP + ((uint32_t)(warp & 3) * 32u << 16);
         float tmp[16];
 #pragma unroll
         for (int c0i = 0; c0i < HQP; c0i += 16) {
-            tmem_ld16(tmem + lane_off + c0i, tmp);
+            tmem_ld16(ta + c0i, tmp);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) a0[c0i + q] = tmp[q];
-            if (glob) {
-                tmem_ld16(tmem + HQP + lane_off + c0i, tmp);
-                tmem_ld_wait();
-#pragma unroll
-                for (int q = 0; q < 16; ++q) a1[c0i + q] = tmp[q];
-            }
+            for (int q = 0; q < 16; ++q) a[c0i + q] = tmp[q];
         }
     }
-    const bool r0 = v0 && ok, r1 = glob && v1 && ok;
+    const bool r0 = v0 && ok;
 #pragma unroll
-    for (int h = 0; h < HQP; ++h) {
-        a0[h] = r0 ? a0[h] * p.scale_log2 : -INFINITY;
-        a1[h] = r1 ? a1[h] * p.scale_log2 : -INFINITY;
-    }
-    float mh[HQP];
+    for (int h = 0; h < HQP; ++h) a[h] = r0 ? a[h] * p.scale_log2 : -INFINITY;
+    const int hl = (HQP == 16) ? ((lane >> 1) & 15) : lane;   // the head this lane ends up holding
+    {
+        float v[HQP];
 #pragma unroll
-    for (int h = 0; h < HQP; ++h) {
-        float m = fmaxf(a0[h], a1[h]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        mh[h] = m;
-    }
-    if ((tid & 31) == 0) {
-#pragma unroll
-        for (int h = 0; h < HQP; ++h) S.red[warp][h] = mh[h];
+        for (int h = 0; h < HQP; ++h) v[h] = a[h];
+        const float m = warp_transpose_reduce<HQP, true>(v);
+        if (HQP == 32 || (lane & 1) == 0) S.red[warp][hl] = m;
     }
     __syncthreads();
+    if (tid < HQP) {
+        float m = S.red[0][tid];
 #pragma unroll
-    for (int h = 0; h < HQP; ++h) mh[h] = fmaxf(fmaxf(S.red[0][h], S.red[1][h]), fmaxf(S.red[2][h], S.red[3][h]));
+        for (int w = 1; w < kWarps; ++w) m = fmaxf(m, S.red[w][tid]);
+        S.mfin[tid] = m;
+    }
     __syncthreads();
-    float lh[HQP];
+    float pv[HQP];
 #pragma unroll
     for (int h = 0; h < HQP; ++h) {
-        const bool live = mh[h] != -INFINITY;
-        const float p0 = (r0 && live) ? exp2f(a0[h] - mh[h]) : 0.f;
-        const float p1 = (r1 && live) ? exp2f(a1[h] - mh[h]) : 0.f;
-        // key k -> panel k / 64, column k % 64
-        *reinterpret_cast<__nv_bfloat16*>(S.pbuf + (tid >> 6) * (HQP * 128) + sw128(h, (tid & 63) >> 3) + (tid & 7) * 2) =
-            __float2bfloat16_rn(p0);
-        *reinterpret_cast<__nv_bfloat16*>(S.pbuf + (2 + (tid >> 6)) * (HQP * 128) + sw128(h, (tid & 63) >> 3) +
-                                          (tid & 7) * 2) = __float2bfloat16_rn(p1);
-        float l = p0 + p1;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        lh[h] = l;
+        const float mh = S.mfin[h];
+        pv[h] = (r0 && mh != -INFINITY) ? exp2f(a[h] - mh) : 0.f;
+        // key tid -> panel tid / 64, column tid % 64
+        *reinterpret_cast<__nv_bfloat16*>(S.qpbuf + (tid >> 6) * (HQP * 128) + sw128(h, (tid & 63) >> 3) + (tid & 7) * 2) =
+            __float2bfloat16_rn(pv[h]);
     }
-    if ((tid & 31) == 0) {
-#pragma unroll
-        for (int h = 0; h < HQP; ++h) S.red[warp][h] = lh[h];
+    {
+        const float l = warp_transpose_reduce<HQP, false>(pv);
+        if (HQP == 32 || (lane & 1) == 0) S.red[warp][hl] = l;
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (tid < HQP) {
+        float l = 0.f;
 #pragma unroll
-    for (int h = 0; h < HQP; ++h) lh[h] = S.red[0][h] + S.red[1][h] + S.red[2][h] + S.red[3][h];
+        for (int w = 0; w < kWarps; ++w) l += S.red[w][tid];
+        S.lfin[tid] = l;
+    }
 
     // ---- 5. O^T = V^T P (keys as the reduction; the head dim as M)
     if (tid == 0) {
-        const uint32_t va = smem_u32(glob ? S.tbuf : S.tbuf + 2 * kPanelBytes), pa = smem_u32(S.pbuf);
+        const uint32_t va = smem_u32(glob ? S.tbuf : S.tbuf + 2 * kPanelBytes), pa = smem_u32(S.qpbuf);
         constexpr uint32_t idesc = idesc_bf16(128, HQP, 1);
         const int nk = nblk * (kTileKeys / 16);
         for (int kk = 0; kk < nk; ++kk) {
@@ -668,11 +687,11 @@ __global__ void __launch_bounds__(kAttnThreads)
     ok = mbar_wait(&S.bar_o, 0, p.status, 11) && ok;
     tc_fence_after();
     float ov[HQP];
-    {
+    if (warp < 4) {   // O^T rows (the head dim) sit in TMEM lanes 0..127
         float tmp[16];
 #pragma unroll
         for (int c0i = 0; c0i < HQP; c0i += 16) {
-            tmem_ld16(tmem + 2 * HQP + lane_off + c0i, tmp);
+            tmem_ld16(tmem + 2 * HQP + ((uint32_t)(warp * 32) << 16) + c0i, tmp);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 16; ++q) ov[c0i + q] = tmp[q];
@@ -684,15 +703,18 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
         for (int h = 0; h < HQP; ++h) part_o[h * D + tid] = ok ? ov[h] : 0.f;
     }
-    if (tid == 0) {
-#pragma unroll
-        for (int h = 0; h < HQP; ++h) { S.part_m[h] = ok ? mh[h] : -INFINITY; S.part_l[h] = ok ? lh[h] : 0.f; }
+    if (tid < HQP) {
+        S.part_m[tid] = ok ? S.mfin[tid] : -INFINITY;
+        S.part_l[tid] = ok ? S.lfin[tid] : 0.f;
     }
 
-    // ---- 6. merge the cluster's partials through distributed shared memory: every
+    // ---- 6. merge the cluster's partials through distributed shared memory: the
+    // threads split into kClThreads / D slots, each merging one head per round; every
     // load of a head is issued before any is used (one remote round trip per head)
     cluster_sync_all();
-    for (int h = rank; h < p.Hq; h += CS) {
+    constexpr int kSlots = kClThreads / D;
+    const int slot = tid / D, dim = tid % D;
+    for (int h = rank + slot * CS; h < p.Hq; h += kSlots * CS) {
         float mc[16], lc[16], oc[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -700,7 +722,7 @@ __global__ void __launch_bounds__(kAttnThreads)
             if (c < CS) {
                 mc[c] = ld_dsmem(dsmem_addr(&S.part_m[h], c));
                 lc[c] = ld_dsmem(dsmem_addr(&S.part_l[h], c));
-                if (tid < D) oc[c] = ld_dsmem(dsmem_addr(&part_o[h * D + tid], c));
+                oc[c] = ld_dsmem(dsmem_addr(&part_o[h * D + dim], c));
             }
         }
         float M = -INFINITY;
@@ -715,9 +737,8 @@ __global__ void __launch_bounds__(kAttnThreads)
                 acc += wgt * oc[c];
             }
         }
-        if (tid < D)
-            p.out[((size_t)u * p.Hq + h) * D + tid] = __bfloat16_as_ushort(__float2bfloat16_rn(L > 0.f ? acc / L : 0.f));
-        if (tid == 0 && p.lse != nullptr)
+        p.out[((size_t)u * p.Hq + h) * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(L > 0.f ? acc / L : 0.f));
+        if (dim == 0 && p.lse != nullptr)
             p.lse[(size_t)u * p.Hq + h] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
     }
     cluster_sync_all();   // no CTA leaves while others read its shared memory
@@ -812,11 +833,20 @@ static bool encode_local_map(CUtensorMap* m, const uint16_t* ptr, int B, int Llo
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dynamic shared memory of a clustered-attention CTA: at least 80 KB, so that at
+// most two CTAs share an SM. Three fit in the layout, but packing three per SM
+// puts a call's clusters on fewer SMs, and the kernel is latency-bound: measured
+// 22.5 us per launch against 15.3 us with two per SM.
+template <int HQP>
+constexpr size_t attn_cl_smem_bytes() {
+    return sizeof(AttnClSmem<HQP>) + 1024 > 80 * 1024 ? sizeof(AttnClSmem<HQP>) + 1024 : 80 * 1024;
+}
+
 template <int HQP, int D>
 static cudaError_t launch_cl_variant(const AttnParams& p, const CUtensorMap& km, const CUtensorMap& vm, int cs,
                                      int units, cudaStream_t stream) {
     auto kern = sparse_attn_cl_kernel<HQP, D>;
-    const size_t smem = sizeof(AttnClSmem<HQP>) + 1024;
+    const size_t smem = attn_cl_smem_bytes<HQP>();
     cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
     if (e != cudaSuccess) return e;
     if (cs > 8) {
@@ -825,7 +855,7 @@ static cudaError_t launch_cl_variant(const AttnParams& p, const CUtensorMap& km,
     }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(cs, units);
-    cfg.blockDim = dim3(kAttnThreads);
+    cfg.blockDim = dim3(kClThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -849,7 +879,7 @@ bool attn_cluster_fits(const csa2_attn_args& a) {
     return cs >= 1 && cs <= 16 && (int64_t)a.B * a.Tq <= 65535;
 }
 
-csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int32_t* d_status,
+csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
                                 cudaStream_t stream) {
     const int units = a.B * a.Tq;
     if (units == 0) return CSA2_OK;
@@ -865,6 +895,7 @@ csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, in
     p.part = nullptr;
     p.tickets = nullptr;
     p.status = d_status;
+    p.list_ready = list_ready;
     CUtensorMap km, vm;
     memset(&km, 0, sizeof(km));
     memset(&vm, 0, sizeof(vm));

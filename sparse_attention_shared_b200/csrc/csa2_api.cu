@@ -33,7 +33,8 @@ size_t attn_scratch_bytes(const csa2_attn_args& a);
 csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* tickets, void* scratch,
                         int32_t* d_status, cudaStream_t stream);
 bool attn_cluster_fits(const csa2_attn_args& a);
-csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int32_t* d_status, cudaStream_t stream);
+csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
+                                cudaStream_t stream);
 // fp4_quant.cu
 cudaError_t launch_fp4_quantize(const float* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales,
                                 cudaStream_t stream);
@@ -200,7 +201,7 @@ csa2_status csa2_sparse_attn(const csa2_attn_args* args, void* workspace, size_t
         a.local_base = a.q_pos;
         a.Lloc = 0;
     }
-    if (attn_cluster_fits(a)) return launch_attn_cluster(a, a.topk, d_status, static_cast<cudaStream_t>(stream));
+    if (attn_cluster_fits(a)) return launch_attn_cluster(a, a.topk, 0, d_status, static_cast<cudaStream_t>(stream));
     return launch_attn(a, a.topk, tickets, scratch, d_status, static_cast<cudaStream_t>(stream));
 }
 
@@ -222,6 +223,7 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
     int pool_P = 0;
     for (int l = 0; l < s->L; ++l) {
         const csa2_index_args& ix = s->idx[l];
+        bool copied = false;   // a list copy was issued for this layer
         if (ix.mode == CSA2_FULL) {
             st = launch_index(ix, nullptr, 0, workspace, scratch, d_status, strm);
             if (st != CSA2_OK) return st;
@@ -240,6 +242,7 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
             const size_t bytes = (size_t)units * cur_k * sizeof(int32_t);
             if (cudaMemcpyAsync(ix.topk_out, cur, bytes, cudaMemcpyDeviceToDevice, strm) != cudaSuccess)
                 return CSA2_ERR_CUDA;
+            copied = true;
         }
         csa2_attn_args a = s->attn[l];
         a.k = cur_k;
@@ -248,7 +251,11 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
             a.local_base = a.q_pos;
             a.Lloc = 0;
         }
-        st = attn_cluster_fits(a) ? launch_attn_cluster(a, cur, d_status, strm)
+        // A Reuse layer's list was written two or more kernels earlier (the previous
+        // kernel is the previous layer's attention), so its clusters may gather their
+        // global rows before waiting for that kernel; not when a copy came between.
+        const int list_ready = (ix.mode == CSA2_REUSE && !copied) ? 1 : 0;
+        st = attn_cluster_fits(a) ? launch_attn_cluster(a, cur, list_ready, d_status, strm)
                                   : launch_attn(a, cur, tickets, scratch, d_status, strm);
         if (st != CSA2_OK) return st;
     }

@@ -45,6 +45,7 @@ constexpr int kSelWarps = kSel / 32;
 constexpr int kBpt = 4096 / kSel;            // level-0 bins per select thread
 constexpr int kTcThreads = kSel + 64;        // + one TMA warp and one MMA warp
 constexpr int kBins = 4096;
+constexpr int kG0Stride = kBins + 32;        // a level-0 histogram buffer and its element count (word kBins)
 constexpr int kCandCap = 4096;
 constexpr int kStageBytes = 16384;
 constexpr int kStages = 8;
@@ -70,8 +71,11 @@ struct IdxParams {
     int P_in;
     int units, G, groups, chunk;
     int32_t* spill;      // [groups*G][chunk] scores when chunk > kSmemScores
+    int local_sel;       // Reindex: the group leader selects over all of the unit's scores
+    int rstride;         // per-unit stride of rscore
+    int32_t* rscore;     // [units][rstride] published scores (local_sel)
     int* ctrl;           // [slots][kCtrlInts]
-    int* g0;             // [slots][3][kBins]
+    int* g0;             // [slots][3][kG0Stride]: histogram, then the element count
     int* gl;             // [slots][2 tracks][2 levels][kBins]
     int2* cand;          // [slots][2 tracks][kCandCap]
     int* pub;            // [slots][2 tracks][3][kMaxG]
@@ -94,9 +98,13 @@ struct __align__(1024) IdxSmem {
     alignas(16) int red[8 * kSelWarps];
     alignas(16) int info[64];
     alignas(16) int wsum[4 * kSelWarps];
+    int wlist_n[kSelWarps];   // entries in each warp's ordered list
+    int wlist_ovf;            // some warp's list overflowed
 };
 constexpr int kHistlOff = 2 * (int)sizeof(int2) * kCandCap;   // byte offset of the radix histograms
-static_assert(kHistlOff + 2 * kBins * 4 <= (int)sizeof(((IdxSmem*)0)->stage), "select buffers");
+constexpr int kListOff = kHistlOff + 2 * kBins * 4;            // byte offset of the per-warp ordered lists
+constexpr int kListCap = 512;                                  // entries per warp
+static_assert(kListOff + kSelWarps * kListCap * 4 <= (int)sizeof(((IdxSmem*)0)->stage), "select buffers");
 static_assert(kStages * kStageBytes % 1024 == 0, "tensor-core operand alignment");
 static_assert(sizeof(IdxSmem) + 1024 <= 232448, "shared memory per block");
 
@@ -113,10 +121,13 @@ __device__ __forceinline__ int* histl(IdxSmem& S, int tr) {
     return reinterpret_cast<int*>(&S.stage[0][0] + kHistlOff) + tr * kBins;
 }
 
+// Per-warp ordered lists of the write phase (select phase only: they overlay the key stages).
+__device__ __forceinline__ int* wlists(IdxSmem& S) { return reinterpret_cast<int*>(&S.stage[0][0] + kListOff); }
+
 __device__ __forceinline__ Slot slot_of(const IdxParams& p, int group) {
     Slot s;
     s.ctrl = p.ctrl + (size_t)group * kCtrlInts;
-    s.g0 = p.g0 + (size_t)group * 3 * kBins;
+    s.g0 = p.g0 + (size_t)group * 3 * kG0Stride;
     s.gl = p.gl + (size_t)group * 4 * kBins;
     s.cand = p.cand + (size_t)group * 2 * kCandCap;
     s.pub = p.pub + (size_t)group * 6 * kMaxG;
@@ -350,56 +361,108 @@ __device__ __forceinline__ int prefix_total(const int* arr, int n, int* red) {
     return sel_sum(v, red);
 }
 
-// The r-th largest value (1-based, with multiplicity) of cx[0..C) in shared
-// memory, by radix passes of up to 12 bits over x - lo (a pass of b bits uses
-// max(kSel, 2^b) bins, thread t owning bins [per*t, per*t + per)); every value
-// lies in [lo, hi]. Returns T; need_eq = how many of the elements equal to T are
-// ranked within the first r.
-__device__ __noinline__ int local_select(const int* cx, int C, int r, int lo, int hi, int* hist, int* red,
-                                         int* info, int& need_eq) {
-    const int t = threadIdx.x;
-    const uint32_t w = (uint32_t)((long long)hi - (long long)lo);
-    int rem = (w == 0u) ? 0 : 32 - __clz(w);
-    uint32_t prefix = 0;
-#pragma unroll 1
-    while (rem > 0) {
-        const int take = rem < 12 ? rem : 12;
-        const int sh = rem - take;
-        const int per = max(kSel, 1 << take) / kSel;
-#pragma unroll 1
-        for (int i = t; i < kSel * per; i += kSel) hist[i] = 0;
-        sel_sync();
-#pragma unroll 1
-        for (int i = t; i < C; i += kSel) {
-            const uint32_t v = (uint32_t)((long long)cx[i] - (long long)lo);
-            if ((uint32_t)(((uint64_t)v) >> (sh + take)) == prefix) atomicAdd(&hist[(v >> sh) & ((1u << take) - 1u)], 1);
+// Two exclusive scans at once over the select threads; totals in `total`.
+__device__ __forceinline__ int2 sel_scan_excl2(int2 v, int* red, int2& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int2 x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y0 = __shfl_up_sync(0xffffffffu, x.x, o), y1 = __shfl_up_sync(0xffffffffu, x.y, o);
+        if (lane >= o) { x.x += y0; x.y += y1; }
+    }
+    sel_sync();
+    if (lane == 31) { red[2 * warp] = x.x; red[2 * warp + 1] = x.y; }
+    sel_sync();
+    if (warp == 0) {
+        int s0 = lane < kSelWarps ? red[2 * lane] : 0, s1 = lane < kSelWarps ? red[2 * lane + 1] : 0;
+#pragma unroll
+        for (int o = 1; o < kSelWarps; o <<= 1) {
+            const int y0 = __shfl_up_sync(0xffffffffu, s0, o), y1 = __shfl_up_sync(0xffffffffu, s1, o);
+            if (lane >= o) { s0 += y0; s1 += y1; }
         }
+        if (lane < kSelWarps) { red[2 * kSelWarps + 2 * lane] = s0; red[2 * kSelWarps + 2 * lane + 1] = s1; }
+    }
+    sel_sync();
+    const int e0 = warp ? red[2 * kSelWarps + 2 * (warp - 1)] : 0, e1 = warp ? red[2 * kSelWarps + 2 * (warp - 1) + 1] : 0;
+    total = make_int2(red[4 * kSelWarps - 2], red[4 * kSelWarps - 1]);
+    return make_int2(e0 + x.x - v.x, e1 + x.y - v.y);
+}
+
+// The thresholds of both tracks at once. For track k (skipped when Ck = 0): the
+// rk-th largest value (1-based, with multiplicity) among the values xk[0..Ck) in
+// shared memory that lie in [lok, hik] (others are ignored), by radix passes of up
+// to 12 bits over x - lok (a pass of b bits uses max(kSel, 2^b) bins, thread t
+// owning bins [per*t, per*t + per)). The two tracks share every barrier.
+// Returns {T0, need0, T1, need1}: need = how many elements equal to T are ranked
+// within the first r.
+__device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo0, int hi0, const int* x1, int C1,
+                                           int r1, int lo1, int hi1, int* hist, int* red, int* info) {
+    const int t = threadIdx.x;
+    int* h0 = hist;
+    int* h1 = hist + kBins;
+    auto nbits = [](int lo, int hi) {
+        const uint32_t w = (uint32_t)((long long)hi - (long long)lo);
+        return w == 0u ? 0 : 32 - __clz(w);
+    };
+    int rem0 = C0 > 0 ? nbits(lo0, hi0) : 0, rem1 = C1 > 0 ? nbits(lo1, hi1) : 0;
+    uint32_t pf0 = 0, pf1 = 0;
+#pragma unroll 1
+    while (rem0 > 0 || rem1 > 0) {
+        const int tk0 = min(rem0, 12), sh0 = rem0 - tk0, per0 = rem0 > 0 ? max(kSel, 1 << tk0) / kSel : 0;
+        const int tk1 = min(rem1, 12), sh1 = rem1 - tk1, per1 = rem1 > 0 ? max(kSel, 1 << tk1) / kSel : 0;
+#pragma unroll 1
+        for (int i = t; i < kSel * per0; i += kSel) h0[i] = 0;
+#pragma unroll 1
+        for (int i = t; i < kSel * per1; i += kSel) h1[i] = 0;
         sel_sync();
-        int s = 0;
+        if (rem0 > 0) {
 #pragma unroll 1
-        for (int i = 0; i < per; ++i) s += hist[per * t + i];
-        int total;
-        const int excl = sel_scan_excl(s, red, total);
-        int above = total - excl - s;    // elements in bins above this thread's range
-        if (above < r && r <= above + s) {
+            for (int i = t; i < C0; i += kSel) {
+                const int x = x0[i];
+                const uint32_t v = (uint32_t)((long long)x - (long long)lo0);
+                if (x >= lo0 && x <= hi0 && (uint32_t)(((uint64_t)v) >> (sh0 + tk0)) == pf0)
+                    atomicAdd(&h0[(v >> sh0) & ((1u << tk0) - 1u)], 1);
+            }
+        }
+        if (rem1 > 0) {
 #pragma unroll 1
-            for (int i = per - 1; i >= 0; --i) {
-                const int h = hist[per * t + i];
-                if (r <= above + h) {
-                    info[0] = per * t + i;
-                    info[1] = above;
-                    break;
-                }
-                above += h;
+            for (int i = t; i < C1; i += kSel) {
+                const int x = x1[i];
+                const uint32_t v = (uint32_t)((long long)x - (long long)lo1);
+                if (x >= lo1 && x <= hi1 && (uint32_t)(((uint64_t)v) >> (sh1 + tk1)) == pf1)
+                    atomicAdd(&h1[(v >> sh1) & ((1u << tk1) - 1u)], 1);
             }
         }
         sel_sync();
-        r -= info[1];
-        prefix = (prefix << take) | (uint32_t)info[0];
-        rem = sh;
+        int s0 = 0, s1 = 0;
+#pragma unroll 1
+        for (int i = 0; i < per0; ++i) s0 += h0[per0 * t + i];
+#pragma unroll 1
+        for (int i = 0; i < per1; ++i) s1 += h1[per1 * t + i];
+        int2 tot;
+        const int2 ex = sel_scan_excl2(make_int2(s0, s1), red, tot);
+        int ab0 = tot.x - ex.x - s0, ab1 = tot.y - ex.y - s1;   // elements in bins above this thread's range
+        if (rem0 > 0 && ab0 < r0 && r0 <= ab0 + s0) {
+#pragma unroll 1
+            for (int i = per0 - 1; i >= 0; --i) {
+                const int h = h0[per0 * t + i];
+                if (r0 <= ab0 + h) { info[0] = per0 * t + i; info[1] = ab0; break; }
+                ab0 += h;
+            }
+        }
+        if (rem1 > 0 && ab1 < r1 && r1 <= ab1 + s1) {
+#pragma unroll 1
+            for (int i = per1 - 1; i >= 0; --i) {
+                const int h = h1[per1 * t + i];
+                if (r1 <= ab1 + h) { info[2] = per1 * t + i; info[3] = ab1; break; }
+                ab1 += h;
+            }
+        }
+        sel_sync();
+        if (rem0 > 0) { r0 -= info[1]; pf0 = (pf0 << tk0) | (uint32_t)info[0]; rem0 = sh0; }
+        if (rem1 > 0) { r1 -= info[3]; pf1 = (pf1 << tk1) | (uint32_t)info[2]; rem1 = sh1; }
     }
-    need_eq = r;
-    return (int)((long long)lo + (long long)prefix);
+    return make_int4((int)((long long)lo0 + (long long)pf0), r0, (int)((long long)lo1 + (long long)pf1), r1);
 }
 
 // ------------------------------------------------------------ select + write
@@ -492,18 +555,33 @@ __device__ __forceinline__ void sel_total8(int4& a, int4& b, int* red) {
 // Candidates of both tracks (scores in [lo0, hi0] / [lo1, hi1]; lo > hi = off)
 // into lbuf[0..) and lbuf[kCandCap..) as (score, element index + base). A warp
 // reserves room once per step that holds candidates; the order is free.
+// The same pass appends to the warp's ordered list (lists + warp * kListCap)
+// every element that is above a track's interval or inside it, as
+// e | flags << 28 (flag bits: above 0, inside 0, above 1, inside 1), and stores
+// the list lengths in wn; a list longer than kListCap sets *ovf.
 template <bool kSpill>
 __device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int lo0, int hi0, int lo1, int hi1,
-                                          int2* lbuf, int* lcnt) {
-    const int lane = threadIdx.x & 31;
+                                             int2* lbuf, int* lcnt, int* lists, int* wn, int* ovf) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const unsigned below = (1u << lane) - 1u;
+    const bool on0 = lo0 <= hi0, on1 = lo1 <= hi1;
+    int* list = lists + wp * kListCap;
+    int ln = 0;
     int s0, s1;
     warp_steps(n, s0, s1);
-#pragma unroll 1
+#pragma unroll 4
     for (int st = s0; st < s1; ++st) {
         const int e = st * 32 + lane;
         const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
         const bool m0 = e < n && x >= lo0 && x <= hi0, m1 = e < n && x >= lo1 && x <= hi1;
+        const bool a0 = e < n && on0 && x > hi0, a1 = e < n && on1 && x > hi1;
+        const unsigned f = (a0 ? 1u : 0u) | (m0 ? 2u : 0u) | (a1 ? 4u : 0u) | (m1 ? 8u : 0u);
+        const unsigned bk = __ballot_sync(0xffffffffu, f != 0u);
+        if (bk) {
+            const int at = ln + __popc(bk & below);
+            if (f != 0u && at < kListCap) list[at] = e | (int)(f << 28);
+            ln += __popc(bk);
+        }
         const unsigned b0 = __ballot_sync(0xffffffffu, m0), b1 = __ballot_sync(0xffffffffu, m1);
         if ((b0 | b1) == 0u) continue;
         int w0 = 0, w1 = 0;
@@ -516,6 +594,10 @@ __device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int
         const int2 cv = make_int2(x, base + e);
         if (m0 && w0 < kCandCap) lbuf[w0] = cv;
         if (m1 && w1 < kCandCap) lbuf[kCandCap + w1] = cv;
+    }
+    if (lane == 0) {
+        wn[wp] = min(ln, kListCap);
+        if (ln > kListCap) *ovf = 1;
     }
 }
 
@@ -569,7 +651,7 @@ __device__ __forceinline__ void write_lists(const int* sc, int n, int base, cons
     int s0, s1;
     warp_steps(n, s0, s1);
     int4 cnt = make_int4(0, 0, 0, 0);   // gt0, eq0, gt1, eq1
-#pragma unroll 1
+#pragma unroll 4
     for (int st = s0; st < s1; ++st) {
         const int e = st * 32 + lane;
         const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
@@ -589,7 +671,7 @@ __device__ __forceinline__ void write_lists(const int* sc, int n, int base, cons
         const int4 a = w4[w];
         rg0 += a.x; re0 += a.y; rg1 += a.z; re1 += a.w;
     }
-#pragma unroll 1
+#pragma unroll 4
     for (int st = s0; st < s1; ++st) {
         const int e = st * 32 + lane;
         const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
@@ -604,8 +686,66 @@ __device__ __forceinline__ void write_lists(const int* sc, int n, int base, cons
         const bool t0 = g0 || (q0 && oq0 < c0.quota), t1 = g1 || (q1 && oq1 < c1.quota);
         if (t0 || t1) {
             const int pos = pool ? pool[base + e] : base + e;
-            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (k < c0.r) c0.out[k] = pos; }
-            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if (k < c1.r) c1.out[k] = pos; }
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if ((unsigned)k < (unsigned)c0.r) c0.out[k] = pos; }
+            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if ((unsigned)k < (unsigned)c1.r) c1.out[k] = pos; }
+        }
+        rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
+    }
+}
+
+// Ordered write of both tracks from the warps' ordered lists (built by
+// gather_cands with the tracks' final intervals): an entry above a track's
+// interval is taken, one inside it is taken if its score is above T, or equal to
+// T within the quota. Same ranks as write_lists, over ~P/G entries instead of the
+// whole chunk.
+template <bool kSpill>
+__device__ __forceinline__ void write_from_lists(const int* sc, int base, const int32_t* pool, const int* lists,
+                                                 const int* wn, ListCut c0, ListCut c1, int* wsum) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    const int* list = lists + wp * kListCap;
+    const int n = wn[wp];
+    auto flags = [&](int ent, bool ok, bool& g0, bool& q0, bool& g1, bool& q1) {
+        const unsigned f = ok ? ((unsigned)ent >> 28) : 0u;
+        const int x = (f & 10u) ? ld_score<kSpill>(sc, ent & 0x0FFFFFFF) : 0;
+        g0 = c0.out && ((f & 1u) || ((f & 2u) && x > c0.T));
+        q0 = c0.out && (f & 2u) && x == c0.T;
+        g1 = c1.out && ((f & 4u) || ((f & 8u) && x > c1.T));
+        q1 = c1.out && (f & 8u) && x == c1.T;
+    };
+    int4 cnt = make_int4(0, 0, 0, 0);   // gt0, eq0, gt1, eq1
+#pragma unroll 1
+    for (int i = lane; i < n; i += 32) {
+        bool g0, q0, g1, q1;
+        flags(list[i], true, g0, q0, g1, q1);
+        cnt.x += g0; cnt.y += q0; cnt.z += g1; cnt.w += q1;
+    }
+    cnt = warp_sum4(cnt);
+    int4* w4 = reinterpret_cast<int4*>(wsum);
+    if (lane == 0) w4[wp] = cnt;
+    sel_sync();
+    int rg0 = 0, re0 = 0, rg1 = 0, re1 = 0;
+#pragma unroll 1
+    for (int w = 0; w < wp; ++w) {
+        const int4 a = w4[w];
+        rg0 += a.x; re0 += a.y; rg1 += a.z; re1 += a.w;
+    }
+#pragma unroll 1
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const int ent = i < n ? list[i] : 0;
+        bool g0, q0, g1, q1;
+        flags(ent, i < n, g0, q0, g1, q1);
+        const unsigned bg0 = __ballot_sync(0xffffffffu, g0), bq0 = __ballot_sync(0xffffffffu, q0);
+        const unsigned bg1 = __ballot_sync(0xffffffffu, g1), bq1 = __ballot_sync(0xffffffffu, q1);
+        const int og0 = rg0 + __popc(bg0 & below), oq0 = re0 + __popc(bq0 & below);
+        const int og1 = rg1 + __popc(bg1 & below), oq1 = re1 + __popc(bq1 & below);
+        const bool t0 = g0 || (q0 && oq0 < c0.quota), t1 = g1 || (q1 && oq1 < c1.quota);
+        if (t0 || t1) {
+            const int e = base + (ent & 0x0FFFFFFF);
+            const int pos = pool ? pool[e] : e;
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if ((unsigned)k < (unsigned)c0.r) c0.out[k] = pos; }
+            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if ((unsigned)k < (unsigned)c1.r) c1.out[k] = pos; }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
     }
@@ -623,9 +763,10 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
     const int lo = c.lo, my_n = c.my_n;
 
     // ---- round 0: histogram of level 0; zero the buffers the next steps use
-    int* g0cur = sl.g0 + ((c.epoch + c.j) % 3) * kBins;
-    int* g0nxt = sl.g0 + ((c.epoch + c.j + 1) % 3) * kBins;
+    int* g0cur = sl.g0 + ((c.epoch + c.j) % 3) * kG0Stride;
+    int* g0nxt = sl.g0 + ((c.epoch + c.j + 1) % 3) * kG0Stride;
     push_hist(S.hist0, g0cur);
+    if (!full && tid == 0 && my_n > 0) atomicAdd(g0cur + kBins, my_n);   // the group's element count
     {
         const int per = (kBins + p.G - 1) / p.G;
         const int zlo = c.cta * per, zhi = min(kBins, zlo + per);
@@ -634,20 +775,12 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
             g0nxt[i] = 0;
             sl.gl[i] = 0; sl.gl[kBins + i] = 0; sl.gl[2 * kBins + i] = 0; sl.gl[3 * kBins + i] = 0;
         }
-        if (c.cta == 0 && tid == 0) { sl.ctrl[CTRL_CAND0] = 0; sl.ctrl[CTRL_CAND1] = 0; }
+        if (c.cta == 0 && tid == 0) { sl.ctrl[CTRL_CAND0] = 0; sl.ctrl[CTRL_CAND1] = 0; g0nxt[kBins] = 0; }
     }
     bar_target += p.G;
     if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
 
-    int n_total;
-    if (full) {
-        n_total = c.n_all;
-    } else {
-        int s2 = 0;
-#pragma unroll 1
-        for (int i = tid; i < kBins; i += kSel) s2 += __ldcg(g0cur + i);
-        n_total = sel_sum(s2, S.red);
-    }
+    const int n_total = full ? c.n_all : min(max(__ldcg(g0cur + kBins), 0), p.P_in);
     Track tk[2];
     int rq[2];
 #pragma unroll
@@ -685,6 +818,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         }
     }
 
+    int list_tracks = 0;   // tracks whose final intervals the ordered lists hold (bit per track)
     // ---- rounds until every track knows its cut (usually one)
 #pragma unroll 1
     while (true) {
@@ -694,10 +828,11 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
             any = true;
             int2* lbuf = reinterpret_cast<int2*>(&S.stage[0][0]);
             int* lcnt = S.info + 40;
-            if (tid == 0) { lcnt[0] = 0; lcnt[1] = 0; }
+            if (tid == 0) { lcnt[0] = 0; lcnt[1] = 0; S.wlist_ovf = 0; }
             sel_sync();
             gather_cands<kSpill>(sc, my_n, lo, g0on ? tk[0].lo : 1, g0on ? tk[0].hi : 0, g1on ? tk[1].lo : 1,
-                         g1on ? tk[1].hi : 0, lbuf, lcnt);
+                                 g1on ? tk[1].hi : 0, lbuf, lcnt, wlists(S), S.wlist_n, &S.wlist_ovf);
+            list_tracks = (g0on ? 1 : 0) | (g1on ? 2 : 0);   // a gather rebuilds the lists
             sel_sync();
             if (tid == 0 || tid == 32) {
                 const int tr = tid >> 5;
@@ -713,7 +848,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
                 const int n_mine = S.info[46 + tr], gbase = S.info[44 + tr];
 #pragma unroll 1
                 for (int i = tid; i < n_mine; i += kSel)
-                    if (gbase + i < kCandCap) sl.cand[tr * kCandCap + gbase + i] = lbuf[tr * kCandCap + i];
+                    if ((unsigned)(gbase + i) < (unsigned)kCandCap) sl.cand[tr * kCandCap + gbase + i] = lbuf[tr * kCandCap + i];
             }
         }
 #pragma unroll
@@ -795,15 +930,17 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         }
         sel_sync();
         int T[2] = {INT_MAX, INT_MAX}, need[2] = {0, 0};
+        if (n0 > 0 || n1 > 0) {
+            const int4 ls = local_select2(cx0, n0, tk[0].rrem, tk[0].lo, tk[0].hi, cx0 + 2 * kCandCap, n1, tk[1].rrem,
+                                          tk[1].lo, tk[1].hi, histl(S, 0), S.red, S.info);
+            if (n0 > 0) { T[0] = ls.x; need[0] = ls.y; }
+            if (n1 > 0) { T[1] = ls.z; need[1] = ls.w; }
+        }
 #pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
-            const Track& k = tk[tr];
-            if (k.state == TS_FIN_CAND) {
-                T[tr] = local_select(cx0 + tr * 2 * kCandCap, k.C, k.rrem, k.lo, k.hi, histl(S, tr), S.red,
-                                     S.info + 8 * tr, need[tr]);
-            } else if (k.state == TS_FIN_EQ) {
-                T[tr] = k.lo;
-                need[tr] = k.rrem;
+            if (tk[tr].state == TS_FIN_EQ) {
+                T[tr] = tk[tr].lo;
+                need[tr] = tk[tr].rrem;
             }
         }
         // larger candidates and ties before this CTA, and this CTA's ties (both tracks)
@@ -840,8 +977,15 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         }
     }
 
-    // ---- ordered write of both tracks
-    write_lists<kSpill>(sc, my_n, lo, full ? nullptr : c.pool, cut[0], cut[1], S.wsum);
+    // ---- ordered write of both tracks: from the ordered lists when every active
+    // track was cut inside its last gathered interval, else over the whole chunk
+    const bool from_lists = list_tracks != 0 && S.wlist_ovf == 0 &&
+                            (tk[0].state == TS_OFF || (tk[0].state == TS_FIN_CAND && (list_tracks & 1))) &&
+                            (tk[1].state == TS_OFF || (tk[1].state == TS_FIN_CAND && (list_tracks & 2)));
+    if (from_lists)
+        write_from_lists<kSpill>(sc, lo, full ? nullptr : c.pool, wlists(S), S.wlist_n, cut[0], cut[1], S.wsum);
+    else
+        write_lists<kSpill>(sc, my_n, lo, full ? nullptr : c.pool, cut[0], cut[1], S.wsum);
     // padding: entries [min(r, n_total), r) = -1
     if (c.cta == p.G - 1) {
 #pragma unroll
@@ -850,6 +994,85 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
 #pragma unroll 1
                 for (int i = min(cut[tr].r, n_total) + tid; i < cut[tr].r; i += kSel) cut[tr].out[i] = -1;
     }
+    sel_sync();
+    return true;
+}
+
+// ------------------------------------------------------------ Reindex: one select per group
+// A Reindex pool fits in one CTA's shared memory, so the group does not run the
+// distributed select: every CTA publishes its scores (element order) and its
+// element count and meets the group at one barrier; then the group's first CTA
+// loads all of the unit's scores and cuts top-k alone, with the same order key,
+// the same exact threshold search and the same tie rule, while the others go on
+// to their next unit.
+__device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c,
+                                                   int& bar_target) {
+    const int tid = threadIdx.x;
+    int32_t* rs = p.rscore + (size_t)c.u * p.rstride;
+    int* cnt = sl.g0 + ((c.epoch + c.j) % 3) * kG0Stride + kBins;
+    int* cnt_next = sl.g0 + ((c.epoch + c.j + 1) % 3) * kG0Stride + kBins;
+#pragma unroll 1
+    for (int e = tid; e < c.my_n; e += kSel) rs[c.lo + e] = S.sc[e];
+    if (tid == 0 && c.my_n > 0) atomicAdd(cnt, c.my_n);
+    {
+        // the next level-0 buffer (bins and count) must be zero when the next unit,
+        // in this kernel or the next one, starts: each CTA clears its share
+        int* g0nxt = cnt_next - kBins;
+        const int per = (kBins + p.G - 1) / p.G;
+        const int zlo = c.cta * per, zhi = min(kBins, zlo + per);
+#pragma unroll 1
+        for (int i = zlo + tid; i < zhi; i += kSel) g0nxt[i] = 0;
+        if (tid == 0 && c.cta == 0) *cnt_next = 0;
+    }
+    // every CTA waits: the leader's zeroing of the next unit's count (above) is then
+    // ordered before any CTA's add for that unit
+    bar_target += p.G;
+    if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
+    if (c.cta != 0) return true;
+
+    // the leader: all scores of the unit (valid pool entries form a prefix)
+    const int n = min(max(__ldcg(cnt), 0), p.P_in);
+#pragma unroll 1
+    for (int i = tid; i < kBins; i += kSel) S.hist0[i] = 0;
+    sel_sync();
+#pragma unroll 4
+    for (int e = tid; e < n; e += kSel) {
+        const int x = __ldcg(rs + e);
+        S.sc[e] = x;
+        atomicAdd(&S.hist0[bin0(x)], 1);
+    }
+    sel_sync();
+    const int r = p.r[1];
+    ListCut none{INT_MAX, 0, 0, 0, 0, nullptr};
+    ListCut cut{INT_MAX, 0, 0, 0, r, p.out[1] + (size_t)c.u * r};
+    if (n <= r) {
+        cut.all = 1;
+    } else {
+        // level-0 bin holding rank r, from the shared histogram (kBpt bins per thread)
+        int h[kBpt], sum = 0;
+#pragma unroll
+        for (int i = 0; i < kBpt; ++i) { h[i] = S.hist0[kBpt * tid + i]; sum += h[i]; }
+        int total;
+        const int excl = sel_scan_excl(sum, S.red, total);
+        int above = total - excl - sum;
+        if (above < r && r <= above + sum) {
+#pragma unroll
+            for (int i = kBpt - 1; i >= 0; --i) {
+                if (above < r && r <= above + h[i]) { S.info[0] = kBpt * tid + i; S.info[1] = above; }
+                above += h[i];
+            }
+        }
+        sel_sync();
+        int blo, bhi;
+        bin0_interval((uint32_t)S.info[0], blo, bhi);
+        const int rrem = r - S.info[1];
+        const int4 ls = local_select2(S.sc, 0, 0, 1, 0, S.sc, n, rrem, blo, bhi, histl(S, 0), S.red, S.info);
+        cut.T = ls.z;
+        cut.quota = ls.w;   // the ties at T ranked within the first r, all in this CTA
+    }
+    write_lists<false>(S.sc, n, 0, c.pool, none, cut, S.wsum);
+#pragma unroll 1
+    for (int i = min(r, n) + tid; i < r; i += kSel) cut.out[i] = -1;
     sel_sync();
     return true;
 }
@@ -1212,8 +1435,11 @@ __global__ void __launch_bounds__(kSel, 1)
         }
         __syncthreads();
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
-        alive = spill ? select_unit<true>(p, S, sl, c, bar_target, spill)
-                      : select_unit<false>(p, S, sl, c, bar_target, S.sc);
+        if (!full && p.local_sel)
+            alive = reindex_local_unit(p, S, sl, c, bar_target);
+        else
+            alive = spill ? select_unit<true>(p, S, sl, c, bar_target, spill)
+                          : select_unit<false>(p, S, sl, c, bar_target, S.sc);
         __syncthreads();
     }
     if (alive && cta == 0 && tid == 0) {
@@ -1241,6 +1467,7 @@ static EncodeTiledFn get_encode_fn() {
 
 struct IdxPlan {
     int units, G, groups, chunk;
+    int local_sel, rstride;
     size_t spill_bytes;
 };
 
@@ -1268,7 +1495,7 @@ IdxRegion idx_region(int slots) {
     IdxRegion r{};
     size_t off = 0;
     r.off_ctrl = off; off += align_up((size_t)slots * kCtrlInts * 4, 256);
-    r.off_g0 = off;   off += align_up((size_t)slots * 3 * kBins * 4, 256);
+    r.off_g0 = off;   off += align_up((size_t)slots * 3 * kG0Stride * 4, 256);
     r.off_gl = off;   off += align_up((size_t)slots * 4 * kBins * 4, 256);
     r.off_cand = off; off += align_up((size_t)slots * 2 * kCandCap * 8, 256);
     r.off_pub = off;  off += align_up((size_t)slots * 6 * kMaxG * 4, 256);
@@ -1295,6 +1522,10 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
     pl.chunk = chunk;
     pl.spill_bytes = 0;
     if (chunk > kSmemScores) pl.spill_bytes = align_up((size_t)pl.groups * pl.G * chunk * 4, 256);
+    // Reindex with a pool that fits one CTA: published scores, one select per group
+    pl.local_sel = (a.mode == CSA2_REINDEX && pl.G > 1 && a.P_in <= kSmemScores) ? 1 : 0;
+    pl.rstride = (int)align_up((size_t)std::max(a.P_in, 1), 4);
+    if (pl.local_sel) pl.spill_bytes = std::max(pl.spill_bytes, align_up((size_t)pl.units * pl.rstride * 4, 256));
     return pl;
 }
 
@@ -1346,6 +1577,9 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
     p.cand = reinterpret_cast<int2*>(base + rg.off_cand);
     p.pub = reinterpret_cast<int*>(base + rg.off_pub);
     p.spill = (pl.chunk > kSmemScores) ? static_cast<int32_t*>(scratch) : nullptr;
+    p.local_sel = pl.local_sel;
+    p.rstride = pl.rstride;
+    p.rscore = pl.local_sel ? static_cast<int32_t*>(scratch) : nullptr;
     p.status = d_status;
 
     CUtensorMap map;

@@ -120,6 +120,43 @@ def test_index_ties(kind, ws, status):
     _check_full(qi, w, ki, q_pos, 2048, 8192, ws, status)
 
 
+@pytest.mark.parametrize("where", ["front", "back"])
+def test_index_full_concentrated_top(where, ws, status):
+    """Keys aligned with the weighted index query in ~9000 neighbouring positions:
+    one CTA's chunk then holds nearly all of the top-8192, so its warps' ordered
+    lists overflow and the write falls back to the pass over the whole chunk."""
+    B, N, A = 16, 131072, 9000
+    qi = synth.randint_i8(7, 1, (B, 1, 8, 64))
+    ki = synth.randint_i8(7, 2, (B, N, 64))
+    w = synth.randint_i32(7, 3, (8,), 1, 8)
+    noise = synth.randint_i32(7, 4, (B, A, 64), -37, 37)
+    for b in range(B):
+        v = (w[:, None].astype(np.int64) * qi[b, 0].astype(np.int64)).sum(0)
+        rows = slice(0, A) if where == "front" else slice(N - A, N)
+        ki[b, rows] = np.clip(np.sign(v)[None, :] * 90 + noise[b], -127, 127).astype(np.int8)
+    q_pos = np.full((B, 1), N - 1, np.int32)
+    _check_full(qi, w, ki, q_pos, 2048, 8192, ws, status)
+
+
+def test_index_sequence_shares_workspace(ws, status):
+    """Full, Full, Reindex (one select per group), Full on one workspace. The
+    indexer keeps three rotating level-0 histogram buffers per group; every kernel
+    must leave the next one zero whichever select it ran, or the last Full call
+    reads the histogram the first one left behind."""
+    B, N = 16, 65536
+    qs = [synth.randint_i8(8, i, (B, 1, 8, 64)) for i in range(4)]
+    ki = synth.randint_i8(8, 10, (B, N, 64))
+    w = synth.randint_i32(8, 11, (8,), 1, 8)
+    q_pos = np.full((B, 1), N - 1, np.int32)
+    _check_full(qs[0], w, ki, q_pos, 2048, 8192, ws, status)
+    pool, _ = _check_full(qs[1], w, ki, q_pos, 2048, 8192, ws, status)
+    _, t2 = ops.index_topk("REINDEX", dev(q_pos), dev(qs[2]), w, dev(ki), 2048, pool_in=pool, ws=ws, status=status)
+    rp = pool.cpu().numpy()
+    ref = np.stack([[O.index_reindex(qs[2][b, 0], w, ki[b], rp[b, 0], 2048)] for b in range(B)])
+    assert_lists_equal(t2, ref, "reindex topk")
+    _check_full(qs[3], w, ki, q_pos, 2048, 8192, ws, status)
+
+
 def test_index_reindex(ws, status):
     B, N = 3, 12000
     qi = synth.randint_i8(4, 1, (B, 1, 8, 64))
@@ -265,9 +302,11 @@ def test_layer_stack_long_schedule_small(ws, status):
     _check_stack(wl, [(0, j) for j in range(8)], ws, status)
 
 
-def test_layer_stack_paper_schedule_small(ws, status):
+@pytest.mark.parametrize("keep_reuse", [True, False])
+def test_layer_stack_paper_schedule_small(keep_reuse, ws, status):
+    # keep_reuse=False: Reuse layers gather their global rows before the previous kernel ends
     wl = synth.make_workload("paper_schedule", B=3, N=9000)
-    _check_stack(wl, [(b, 0) for b in range(3)], ws, status)
+    _check_stack(wl, [(b, 0) for b in range(3)], ws, status, keep_reuse=keep_reuse)
 
 
 def test_layer_stack_rejects_bad_mode_order(ws):
