@@ -558,8 +558,9 @@ __device__ __forceinline__ void sel_total8(int4& a, int4& b, int* red) {
 // The same pass appends to the warp's ordered list (lists + warp * kListCap)
 // every element that is above a track's interval or inside it, as
 // e | flags << 28 (flag bits: above 0, inside 0, above 1, inside 1), and stores
-// the list lengths in wn; a list longer than kListCap sets *ovf.
-template <bool kSpill>
+// the list lengths in wn; a list longer than kListCap sets *ovf. kCands = false
+// builds the lists only.
+template <bool kSpill, bool kCands = true>
 __device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int lo0, int hi0, int lo1, int hi1,
                                              int2* lbuf, int* lcnt, int* lists, int* wn, int* ovf) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
@@ -582,6 +583,7 @@ __device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int
             if (f != 0u && at < kListCap) list[at] = e | (int)(f << 28);
             ln += __popc(bk);
         }
+        if (!kCands) continue;
         const unsigned b0 = __ballot_sync(0xffffffffu, m0), b1 = __ballot_sync(0xffffffffu, m1);
         if ((b0 | b1) == 0u) continue;
         int w0 = 0, w1 = 0;
@@ -1030,21 +1032,37 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
     if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
     if (c.cta != 0) return true;
 
-    // the leader: all scores of the unit (valid pool entries form a prefix)
+    // the leader: all scores of the unit (valid pool entries form a prefix), as int4
+    // vectors with every load of a thread in flight at once
     const int n = min(max(__ldcg(cnt), 0), p.P_in);
 #pragma unroll 1
     for (int i = tid; i < kBins; i += kSel) S.hist0[i] = 0;
     sel_sync();
-#pragma unroll 4
-    for (int e = tid; e < n; e += kSel) {
-        const int x = __ldcg(rs + e);
-        S.sc[e] = x;
-        atomicAdd(&S.hist0[bin0(x)], 1);
+    {
+        const int nv = (n + 3) >> 2;   // rstride is a multiple of 4: whole vectors stay in the unit's row
+        const int4* rs4 = reinterpret_cast<const int4*>(rs);
+#pragma unroll 1
+        for (int v0 = tid; v0 < nv; v0 += 4 * kSel) {
+            int4 x4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) x4[q] = (v0 + q * kSel < nv) ? __ldcg(rs4 + v0 + q * kSel) : make_int4(0, 0, 0, 0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int v = v0 + q * kSel;
+                if (v >= nv) continue;
+                reinterpret_cast<int4*>(S.sc)[v] = x4[q];
+                const int xs[4] = {x4[q].x, x4[q].y, x4[q].z, x4[q].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (4 * v + k < n) atomicAdd(&S.hist0[bin0(xs[k])], 1);
+            }
+        }
     }
     sel_sync();
     const int r = p.r[1];
     ListCut none{INT_MAX, 0, 0, 0, 0, nullptr};
     ListCut cut{INT_MAX, 0, 0, 0, r, p.out[1] + (size_t)c.u * r};
+    bool lists = false;
     if (n <= r) {
         cut.all = 1;
     } else {
@@ -1062,15 +1080,23 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
                 above += h[i];
             }
         }
+        if (tid == 0) S.wlist_ovf = 0;
         sel_sync();
         int blo, bhi;
         bin0_interval((uint32_t)S.info[0], blo, bhi);
         const int rrem = r - S.info[1];
+        // one pass builds the warps' ordered lists (top-k is track 1); the threshold
+        // comes from a radix select over the scores inside the bin's interval
+        gather_cands<false, false>(S.sc, n, 0, 1, 0, blo, bhi, nullptr, nullptr, wlists(S), S.wlist_n, &S.wlist_ovf);
         const int4 ls = local_select2(S.sc, 0, 0, 1, 0, S.sc, n, rrem, blo, bhi, histl(S, 0), S.red, S.info);
         cut.T = ls.z;
         cut.quota = ls.w;   // the ties at T ranked within the first r, all in this CTA
+        lists = S.wlist_ovf == 0;
     }
-    write_lists<false>(S.sc, n, 0, c.pool, none, cut, S.wsum);
+    if (lists)
+        write_from_lists<false>(S.sc, 0, c.pool, wlists(S), S.wlist_n, none, cut, S.wsum);
+    else
+        write_lists<false>(S.sc, n, 0, c.pool, none, cut, S.wsum);
 #pragma unroll 1
     for (int i = min(r, n) + tid; i < r; i += kSel) cut.out[i] = -1;
     sel_sync();
@@ -1099,6 +1125,29 @@ __device__ __forceinline__ int score_smem(const int4* rowc, const int8_t* qs, co
         s += w[h] * max(acc, 0);
     }
     return s;
+}
+
+// Scores of two key rows at once: each read of the index query from shared memory
+// serves both rows.
+template <int HI, int DI>
+__device__ __forceinline__ void score2_smem(const int4* ra, const int4* rb, const int8_t* qs, const int32_t* w,
+                                            int& xa, int& xb) {
+    int sa = 0, sb = 0;
+#pragma unroll
+    for (int h = 0; h < HI; ++h) {
+        int aa = 0, ab = 0;
+        const int4* qh = reinterpret_cast<const int4*>(qs + h * DI);
+#pragma unroll
+        for (int c = 0; c < DI / 16; ++c) {
+            const int4 qq = qh[c], ka = ra[c], kb = rb[c];
+            aa = __dp4a(ka.x, qq.x, aa); aa = __dp4a(ka.y, qq.y, aa); aa = __dp4a(ka.z, qq.z, aa); aa = __dp4a(ka.w, qq.w, aa);
+            ab = __dp4a(kb.x, qq.x, ab); ab = __dp4a(kb.y, qq.y, ab); ab = __dp4a(kb.z, qq.z, ab); ab = __dp4a(kb.w, qq.w, ab);
+        }
+        sa += w[h] * max(aa, 0);
+        sb += w[h] * max(ab, 0);
+    }
+    xa = sa;
+    xb = sb;
 }
 
 // Generic shapes: Hi <= 16, Di <= 128, queries read from shared memory.
@@ -1347,6 +1396,15 @@ __global__ void __launch_bounds__(kSel, 1)
         const int lo = min(cta * p.chunk, n_all);
         const int hi = min(lo + p.chunk, n_all);
         const int32_t* pool = full ? nullptr : p.pool_in + (size_t)u * p.P_in;
+        constexpr int RB = 2;   // Reindex: rows per thread in flight (one pair)
+        int sidx0[RB];          // the first round's pool entries, loaded while the query is staged
+        if (!full) {
+#pragma unroll
+            for (int q2 = 0; q2 < RB; ++q2) {
+                const int e = q2 * kSel + tid;
+                sidx0[q2] = (e < hi - lo) ? __ldg(pool + lo + e) : -1;
+            }
+        }
 
         fence_proxy_async_smem();
         for (int i = tid; i < p.Hi * p.Di / 16; i += kSel)
@@ -1393,45 +1451,55 @@ __global__ void __launch_bounds__(kSel, 1)
             stage_seq += nst;
             if (!alive) break;
         } else {
-            // valid pool entries (0 <= s <= t) form a prefix, -1 padding after
+            // Reindex: valid pool entries (0 <= s <= t) form a prefix, -1 padding after.
+            // Entries, their check and the key rows come in one dependent chain; the
+            // histogram is built once the valid prefix is known.
+            const int8_t* kb = p.ki + (size_t)b * p.ki_seq_stride;
+            constexpr int kCh = DI > 0 ? DI / 16 : 8;   // 16-byte chunks per key row
             int first_bad = my_n;
-            for (int e = tid; e < my_n; e += kSel) {
-                const int s2 = pool[lo + e];
-                if (s2 < 0 || s2 > t) first_bad = min(first_bad, e);
+#pragma unroll 1
+            for (int e0 = 0; e0 < my_n; e0 += RB * kSel) {
+                int sidx[RB];
+                bool okr[RB];
+                int4 rows[RB][kCh];
+#pragma unroll
+                for (int q2 = 0; q2 < RB; ++q2) {
+                    const int e = e0 + q2 * kSel + tid;
+                    sidx[q2] = (e0 == 0) ? sidx0[q2] : ((e < my_n) ? __ldg(pool + lo + e) : -1);
+                    okr[q2] = e < my_n && sidx[q2] >= 0 && sidx[q2] <= t;
+                    if (e < my_n && !okr[q2]) first_bad = min(first_bad, e);
+                    if (okr[q2]) {
+                        const int4* row = reinterpret_cast<const int4*>(kb + (size_t)sidx[q2] * p.Di);
+#pragma unroll
+                        for (int c2 = 0; c2 < kCh; ++c2)
+                            if (c2 < nchunk) rows[q2][c2] = __ldg(row + c2);
+                    }
+                }
+#pragma unroll
+                for (int q2 = 0; q2 < RB; q2 += 2) {
+                    if (!okr[q2] && !okr[q2 + 1]) continue;
+                    int xa, xb;
+                    if (generic) {
+                        xa = okr[q2] ? score_generic(rows[q2], nchunk, S.q, p.Hi, p.Di, p.w) : 0;
+                        xb = okr[q2 + 1] ? score_generic(rows[q2 + 1], nchunk, S.q, p.Hi, p.Di, p.w) : 0;
+                    } else {
+                        score2_smem<(HI > 0 ? HI : 1), (DI > 0 ? DI : 16)>(rows[q2], rows[q2 + 1], S.q, p.w, xa, xb);
+                    }
+                    const int ea = e0 + q2 * kSel + tid, eb = ea + kSel;
+                    if (okr[q2]) { if (spill) spill[ea] = xa; else S.sc[ea] = xa; }
+                    if (okr[q2 + 1]) { if (spill) spill[eb] = xb; else S.sc[eb] = xb; }
+                }
             }
             const int fb = sel_min(first_bad, S.red);
             if (fb < my_n) {
                 // an entry past the first invalid one must be padding, never a position
                 for (int e = fb + tid; e < my_n; e += kSel)
-                    if (pool[lo + e] >= 0) report(p.status, CSA2_ERR_RANGE, u);
+                    if (__ldg(pool + lo + e) >= 0) report(p.status, CSA2_ERR_RANGE, u);
                 my_n = fb;
             }
-            if (my_n > 0 && lo > 0 && tid == 0 && pool[lo - 1] < 0) report(p.status, CSA2_ERR_RANGE, u);
-            const int8_t* kb = p.ki + (size_t)b * p.ki_seq_stride;
-            constexpr int RB = 4;   // rows per thread in flight
-            for (int e0 = 0; e0 < my_n; e0 += RB * kSel) {
-                int4 rows[RB][8];
-#pragma unroll
-                for (int q2 = 0; q2 < RB; ++q2) {
-                    const int e = e0 + q2 * kSel + tid;
-                    if (e < my_n) {
-                        const int4* row = reinterpret_cast<const int4*>(kb + (size_t)pool[lo + e] * p.Di);
-#pragma unroll
-                        for (int c2 = 0; c2 < 8; ++c2)
-                            if (c2 < nchunk) rows[q2][c2] = __ldg(row + c2);
-                    }
-                }
-#pragma unroll
-                for (int q2 = 0; q2 < RB; ++q2) {
-                    const int e = e0 + q2 * kSel + tid;
-                    if (e < my_n) {
-                        const int x = generic ? score_generic(rows[q2], nchunk, S.q, p.Hi, p.Di, p.w)
-                                              : score_smem<(HI > 0 ? HI : 1), (DI > 0 ? DI : 16)>(rows[q2], S.q, p.w);
-                        if (spill) spill[e] = x; else S.sc[e] = x;
-                        atomicAdd(&S.hist0[bin0(x)], 1);
-                    }
-                }
-            }
+            if (my_n > 0 && lo > 0 && tid == 0 && __ldg(pool + lo - 1) < 0) report(p.status, CSA2_ERR_RANGE, u);
+#pragma unroll 1
+            for (int e = tid; e < my_n; e += kSel) atomicAdd(&S.hist0[bin0(spill ? spill[e] : S.sc[e])], 1);
         }
         __syncthreads();
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
