@@ -177,6 +177,16 @@ def build_device_stack(wl, torch, ops, np):
     return stack, layers, q_pos, codes, scales, base
 
 
+def job_rate(dist, torch, total_ms_local: float, units_per_rank: int, world: int, steps: int, device):
+    """Whole-job queries/s: every rank timed `steps` steps of `units_per_rank` queries;
+    the job's time is the slowest rank's (max over ranks, on the device clock)."""
+    t = torch.tensor([float(total_ms_local)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    return total_ms, units_per_rank * world * steps / (total_ms / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -239,13 +249,8 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     st.check("timed region")
     step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
-    total_ms = sum(step_ms)
-    tmax = torch.tensor([total_ms], device="cuda")
-    if dist:
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    total_ms = float(tmax.item())
+    total_ms, value = job_rate(dist, torch, sum(step_ms), units, world, K, "cuda")
     ms_per_step = total_ms / K
-    value = units * world * K / (total_ms / 1e3)
     n_idx = sum(1 for L in s.layers if L.mode != "REUSE")
     launches_per_step = n_idx + len(s.layers)
 
@@ -303,7 +308,8 @@ def run_ours(args, rank, world, local_rank):
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st, graph)
+        e2e = run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st, graph,
+                      (codes, scales, base))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -330,22 +336,36 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
-def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st, graph):
+def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st, graph, cache):
     """Per step: copy the step's per-query inputs (main queries of every layer, index
     queries of Full/Reindex layers, query positions) from pinned host memory, run the
-    stack, and copy every layer's output and lse back to pinned host memory."""
-    dev_in = [q_pos] + [d["q"] for d in layers] + [d["qi"] for d in layers if d["mode"] != "REUSE"]
-    host_in = [t.cpu().pin_memory() for t in dev_in]
-    dev_out = list(stack.outs) + [x for x in stack.lses if x is not None]
-    host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in dev_out]
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    stack, and copy every layer's output and lse back to pinned host memory. The
+    inputs sit in one device buffer and the outputs in another, as a caller would lay
+    out a decode step, so each direction is one copy."""
+    codes, scales, base = cache
+    src = [q_pos] + [d["q"] for d in layers] + [d["qi"] for d in layers if d["mode"] != "REUSE"]
+    din, views = ops.packed_views([(tuple(t.shape), t.dtype) for t in src], q_pos.device)
+    for v, t in zip(views, src):
+        v.copy_(t)
+    it = iter(views[1:])
+    layers2 = [dict(d) for d in layers]
+    for d in layers2:
+        d["q"] = next(it)
+    for d in layers2:
+        if d["mode"] != "REUSE":
+            d["qi"] = next(it)
+    stack2 = ops.LayerStack(layers2, views[0], codes, scales, base, packed_outputs=True)
+    host_in = din.cpu().pin_memory()
+    host_out = torch.empty_like(stack2.out_buf, device="cpu").pin_memory()
+    h2d = din.numel()                 # bytes of the one input copy (tensors + alignment gaps)
+    d2h = stack2.out_buf.numel()      # bytes of the one output copy
+    dev_in, host_in, dev_out, host_out = [din], [host_in], [stack2.out_buf], [host_out]
     ws = ops.Workspace()
-    buf = ws.get(stack.ws_bytes)
+    buf = ws.get(stack2.ws_bytes)
     sptr = int(stream.cuda_stream)
 
     def call(stream_ptr):
-        return stack.run_raw(int(buf.data_ptr()), buf.numel(), st.ptr, stream_ptr)
+        return stack2.run_raw(int(buf.data_ptr()), buf.numel(), st.ptr, stream_ptr)
 
     g2 = None if graph is None else capture_graph(torch, call)
     K = max(10, args.steps // 5)

@@ -139,6 +139,21 @@ def sparse_attn(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base, W: int, ws
     return out, lse
 
 
+def packed_views(specs, device, align: int = 256):
+    """One uint8 device buffer holding tensors of the given (shape, dtype) back to
+    back, each at an `align`-byte offset, so that a step's inputs or outputs move
+    between host and device in one copy. Returns (buffer, views)."""
+    sizes, offs, off = [], [], 0
+    for shape, dt in specs:
+        n = int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+        sizes.append(n)
+        offs.append(off)
+        off = (off + n + align - 1) // align * align
+    buf = torch.empty(max(off, align), dtype=torch.uint8, device=device)
+    views = [buf[o:o + n].view(dt).view(shape) for (shape, dt), o, n in zip(specs, offs, sizes)]
+    return buf, views
+
+
 class LayerStack:
     """A decoder stack over one shared cache, with its argument structures built once.
 
@@ -148,11 +163,23 @@ class LayerStack:
       every layer:  q [B,Tq,Hq,D] bf16, kl/vl [B,Lloc,D] bf16, W
     Outputs per layer (allocated here): out, lse; topk for FULL/REINDEX (REUSE layers
     get a copy of their list when keep_reuse_lists=True); pool for FULL with P > 0.
+    packed_outputs=True places every out and lse in one device buffer (out_buf).
     """
 
     def __init__(self, layers: Sequence[Dict], q_pos, kv_fp4, kv_scale, local_base,
-                 keep_reuse_lists: bool = False, with_lse: bool = True):
+                 keep_reuse_lists: bool = False, with_lse: bool = True, packed_outputs: bool = False):
         dev = q_pos.device
+        self.out_buf = None
+        packed = None
+        if packed_outputs:
+            specs = []
+            for d in layers:
+                B, Tq, Hq, D = d["q"].shape
+                specs.append(((B, Tq, Hq, D), torch.bfloat16))
+                if with_lse:
+                    specs.append(((B, Tq, Hq), torch.float32))
+            self.out_buf, packed = packed_views(specs, dev)
+            packed = iter(packed)
         self.L = len(layers)
         self.keep = []          # keeps host weight arrays and tensors alive
         self.pools: List[Optional[torch.Tensor]] = []
@@ -183,8 +210,12 @@ class LayerStack:
                 a.mode = mode
                 a.topk_out = _ptr(topk)
                 idx_arr[l] = a
-            out = torch.empty((B, Tq, Hq, D), dtype=torch.bfloat16, device=dev)
-            lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev) if with_lse else None
+            if packed is not None:
+                out = next(packed)
+                lse = next(packed) if with_lse else None
+            else:
+                out = torch.empty((B, Tq, Hq, D), dtype=torch.bfloat16, device=dev)
+                lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev) if with_lse else None
             kl, vl = d.get("kl"), d.get("vl")
             attn_arr[l] = make_attn_args(q_pos, q, kv_fp4, kv_scale, None, kl, vl, local_base, int(d["W"]), out, lse)
             self.keep.extend([d.get("qi"), d.get("ki"), q, kl, vl])
