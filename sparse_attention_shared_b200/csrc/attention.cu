@@ -425,14 +425,17 @@ struct AttnClSmem {   // placed at a 1024-byte-aligned address (operand tiles ne
     uint32_t lut[256];
     float red[kClThreads / 32][HQP];      // per-warp head maxima, then sums
     float mfin[HQP], lfin[HQP];
-    float part_m[HQP], part_l[HQP];
+    // partials pushed by the cluster's CTAs for the heads this CTA merges: head h
+    // (merged by CTA h % CS) from CTA c sits in row (h / CS) * CS + c
+    float recv_o[HQP + 16][128];
+    float recv_m[HQP + 16], recv_l[HQP + 16];
     uint64_t bar_tma, bar_s, bar_o;
     uint32_t tmem_base;
 };
 
 static_assert(offsetof(AttnClSmem<16>, qpbuf) % 1024 == 0 && offsetof(AttnClSmem<32>, qpbuf) % 1024 == 0,
               "operand alignment");
-static_assert(sizeof(AttnClSmem<16>) + 1024 <= 80 * 1024, "two clustered-attention CTAs per SM");
+static_assert(sizeof(AttnClSmem<32>) + 1024 <= 113 * 1024, "two clustered-attention CTAs per SM");
 
 // Reduce V values per lane (V = 16 or 32, one per head) across the 32 lanes of a
 // warp with halving exchanges: after the call, lane l holds in v[0] the result for
@@ -476,7 +479,6 @@ __global__ void __launch_bounds__(kClThreads, 2)
     const int b = u / p.Tq;
     const int ngt2 = (p.k + 2 * kTileKeys - 1) / (2 * kTileKeys);
     const bool glob = rank < ngt2;
-    float* part_o = reinterpret_cast<float*>(S.tbuf);      // [HQP][D] once the MMAs are done
 
     // ---- 0. set-up that reads no input; it may overlap the previous kernel
     if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
@@ -698,50 +700,48 @@ __global__ void __launch_bounds__(kClThreads, 2)
         }
     }
     tc_fence_before();
-    __syncthreads();    // every MMA operand read is done: the tile buffer holds the partial now
+
+    // ---- 6. merge: every CTA pushes its partial of head h into the shared memory of
+    // the CTA that merges h (CTA h % CS); one cluster barrier publishes the pushes,
+    // then each CTA merges its heads from its own shared memory
     if (tid < D) {
 #pragma unroll
-        for (int h = 0; h < HQP; ++h) part_o[h * D + tid] = ok ? ov[h] : 0.f;
+        for (int h = 0; h < HQP; ++h) {
+            if (h >= p.Hq) break;
+            st_dsmem(dsmem_addr(&S.recv_o[(h / CS) * CS + rank][tid], h % CS), ok ? ov[h] : 0.f);
+        }
     }
-    if (tid < HQP) {
-        S.part_m[tid] = ok ? S.mfin[tid] : -INFINITY;
-        S.part_l[tid] = ok ? S.lfin[tid] : 0.f;
+    if (tid < p.Hq) {
+        const int row = (tid / CS) * CS + rank, owner = tid % CS;
+        st_dsmem(dsmem_addr(&S.recv_m[row], owner), ok ? S.mfin[tid] : -INFINITY);
+        st_dsmem(dsmem_addr(&S.recv_l[row], owner), ok ? S.lfin[tid] : 0.f);
     }
-
-    // ---- 6. merge the cluster's partials through distributed shared memory: the
-    // threads split into kClThreads / D slots, each merging one head per round; every
-    // load of a head is issued before any is used (one remote round trip per head)
-    cluster_sync_all();
+    cluster_sync_all();   // after it no CTA touches another's shared memory
     constexpr int kSlots = kClThreads / D;
     const int slot = tid / D, dim = tid % D;
     for (int h = rank + slot * CS; h < p.Hq; h += kSlots * CS) {
-        float mc[16], lc[16], oc[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            mc[c] = -INFINITY; lc[c] = 0.f; oc[c] = 0.f;
-            if (c < CS) {
-                mc[c] = ld_dsmem(dsmem_addr(&S.part_m[h], c));
-                lc[c] = ld_dsmem(dsmem_addr(&S.part_l[h], c));
-                oc[c] = ld_dsmem(dsmem_addr(&part_o[h * D + dim], c));
-            }
-        }
+        const int r0 = (h / CS) * CS;
         float M = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) M = fmaxf(M, mc[c]);
+        for (int c = 0; c < 16; ++c)
+            if (c < CS) M = fmaxf(M, S.recv_m[r0 + c]);
         float L = 0.f, acc = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                const float wgt = (mc[c] == -INFINITY) ? 0.f : exp2f(mc[c] - M);
-                L += wgt * lc[c];
-                acc += wgt * oc[c];
+                if (c >= CS) break;
+                const float mc = S.recv_m[r0 + c];
+                const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+                L += wgt * S.recv_l[r0 + c];
+                acc += wgt * S.recv_o[r0 + c][dim];
             }
         }
         p.out[((size_t)u * p.Hq + h) * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(L > 0.f ? acc / L : 0.f));
         if (dim == 0 && p.lse != nullptr)
             p.lse[(size_t)u * p.Hq + h] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
     }
-    cluster_sync_all();   // no CTA leaves while others read its shared memory
+    tc_fence_before();
+    __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kCols);
 }
 
@@ -834,9 +834,9 @@ static bool encode_local_map(CUtensorMap* m, const uint16_t* ptr, int B, int Llo
 }
 
 // Dynamic shared memory of a clustered-attention CTA: at least 80 KB, so that at
-// most two CTAs share an SM. Three fit in the layout, but packing three per SM
-// puts a call's clusters on fewer SMs, and the kernel is latency-bound: measured
-// 22.5 us per launch against 15.3 us with two per SM.
+// most two CTAs share an SM. Packing three per SM puts a call's clusters on fewer
+// SMs, and the kernel is latency-bound: measured 22.5 us per launch against
+// 15.3 us with two per SM.
 template <int HQP>
 constexpr size_t attn_cl_smem_bytes() {
     return sizeof(AttnClSmem<HQP>) + 1024 > 80 * 1024 ? sizeof(AttnClSmem<HQP>) + 1024 : 80 * 1024;
