@@ -74,6 +74,10 @@ struct IdxParams {
     int local_sel;       // Reindex: the group leader selects over all of the unit's scores
     int rstride;         // per-unit stride of rscore
     int32_t* rscore;     // [units][rstride] published scores (local_sel)
+    // L2 prefetch of the global cache rows each top-k list selects (pf_fp4 nullptr: off)
+    const uint8_t* pf_fp4;
+    const uint8_t* pf_scale;
+    int pf_N, pf_code_bytes, pf_scale_bytes;
     int* ctrl;           // [slots][kCtrlInts]
     int* g0;             // [slots][3][kG0Stride]: histogram, then the element count
     int* gl;             // [slots][2 tracks][2 levels][kBins]
@@ -638,6 +642,33 @@ struct ListCut {
     int32_t* out;   // nullptr: track off
 };
 
+// The global cache rows of one sequence that its top-k list selects are pulled into
+// L2 as the list is written, so that the attention launch after the indexer
+// gathers them from L2 (fp4 nullptr: off).
+struct RowPrefetch {
+    const uint8_t* fp4;     // the sequence's codes [N][code_bytes]
+    const uint8_t* scale;   // the sequence's scales [N][scale_bytes]
+    int code_bytes, scale_bytes;
+};
+
+__device__ __forceinline__ RowPrefetch row_prefetch(const IdxParams& p, int u) {
+    RowPrefetch f{nullptr, nullptr, 0, 0};
+    if (p.pf_fp4 != nullptr) {
+        const size_t b = (size_t)(u / p.Tq);
+        f.fp4 = p.pf_fp4 + b * p.pf_N * p.pf_code_bytes;
+        f.scale = p.pf_scale + b * p.pf_N * p.pf_scale_bytes;
+        f.code_bytes = p.pf_code_bytes;
+        f.scale_bytes = p.pf_scale_bytes;
+    }
+    return f;
+}
+
+__device__ __forceinline__ void prefetch_row(const RowPrefetch& f, int pos) {
+    if (f.fp4 == nullptr || pos < 0) return;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(f.fp4 + (size_t)pos * f.code_bytes));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(f.scale + (size_t)pos * f.scale_bytes));
+}
+
 __device__ __forceinline__ void take_flags(int x, bool ok, const ListCut& c, bool& g, bool& e) {
     g = ok && c.out != nullptr && (c.all || x > c.T);
     e = ok && c.out != nullptr && !c.all && x == c.T;
@@ -647,7 +678,7 @@ __device__ __forceinline__ void take_flags(int x, bool ok, const ListCut& c, boo
 // ranges with running counts and ballots for the ranks inside a step.
 template <bool kSpill>
 __device__ __forceinline__ void write_lists(const int* sc, int n, int base, const int32_t* pool, ListCut c0,
-                                         ListCut c1, int* wsum) {
+                                         ListCut c1, int* wsum, RowPrefetch pf) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const unsigned below = (1u << lane) - 1u;
     int s0, s1;
@@ -689,7 +720,7 @@ __device__ __forceinline__ void write_lists(const int* sc, int n, int base, cons
         if (t0 || t1) {
             const int pos = pool ? pool[base + e] : base + e;
             if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if ((unsigned)k < (unsigned)c0.r) c0.out[k] = pos; }
-            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if ((unsigned)k < (unsigned)c1.r) c1.out[k] = pos; }
+            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if ((unsigned)k < (unsigned)c1.r) { c1.out[k] = pos; prefetch_row(pf, pos); } }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
     }
@@ -702,7 +733,7 @@ __device__ __forceinline__ void write_lists(const int* sc, int n, int base, cons
 // whole chunk.
 template <bool kSpill>
 __device__ __forceinline__ void write_from_lists(const int* sc, int base, const int32_t* pool, const int* lists,
-                                                 const int* wn, ListCut c0, ListCut c1, int* wsum) {
+                                                 const int* wn, ListCut c0, ListCut c1, int* wsum, RowPrefetch pf) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const unsigned below = (1u << lane) - 1u;
     const int* list = lists + wp * kListCap;
@@ -747,7 +778,7 @@ __device__ __forceinline__ void write_from_lists(const int* sc, int base, const 
             const int e = base + (ent & 0x0FFFFFFF);
             const int pos = pool ? pool[e] : e;
             if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if ((unsigned)k < (unsigned)c0.r) c0.out[k] = pos; }
-            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if ((unsigned)k < (unsigned)c1.r) c1.out[k] = pos; }
+            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if ((unsigned)k < (unsigned)c1.r) { c1.out[k] = pos; prefetch_row(pf, pos); } }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
     }
@@ -985,9 +1016,10 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
                             (tk[0].state == TS_OFF || (tk[0].state == TS_FIN_CAND && (list_tracks & 1))) &&
                             (tk[1].state == TS_OFF || (tk[1].state == TS_FIN_CAND && (list_tracks & 2)));
     if (from_lists)
-        write_from_lists<kSpill>(sc, lo, full ? nullptr : c.pool, wlists(S), S.wlist_n, cut[0], cut[1], S.wsum);
+        write_from_lists<kSpill>(sc, lo, full ? nullptr : c.pool, wlists(S), S.wlist_n, cut[0], cut[1], S.wsum,
+                                 row_prefetch(p, c.u));
     else
-        write_lists<kSpill>(sc, my_n, lo, full ? nullptr : c.pool, cut[0], cut[1], S.wsum);
+        write_lists<kSpill>(sc, my_n, lo, full ? nullptr : c.pool, cut[0], cut[1], S.wsum, row_prefetch(p, c.u));
     // padding: entries [min(r, n_total), r) = -1
     if (c.cta == p.G - 1) {
 #pragma unroll
@@ -1094,9 +1126,9 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         lists = S.wlist_ovf == 0;
     }
     if (lists)
-        write_from_lists<false>(S.sc, 0, c.pool, wlists(S), S.wlist_n, none, cut, S.wsum);
+        write_from_lists<false>(S.sc, 0, c.pool, wlists(S), S.wlist_n, none, cut, S.wsum, row_prefetch(p, c.u));
     else
-        write_lists<false>(S.sc, n, 0, c.pool, none, cut, S.wsum);
+        write_lists<false>(S.sc, n, 0, c.pool, none, cut, S.wsum, row_prefetch(p, c.u));
 #pragma unroll 1
     for (int i = min(r, n) + tid; i < r; i += kSel) cut.out[i] = -1;
     sel_sync();
@@ -1620,7 +1652,7 @@ static cudaError_t launch_coop(Kern kern, int threads, const IdxParams& p, const
 
 // Launch one indexer call. `ws` holds plan_index(a).ws_bytes bytes (zero at first use).
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
-                         int32_t* d_status, cudaStream_t stream) {
+                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf) {
     const int sms = num_sms();
     csa2_index_args aa = a;
     aa.P_in = P_in;
@@ -1648,6 +1680,13 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
     p.local_sel = pl.local_sel;
     p.rstride = pl.rstride;
     p.rscore = pl.local_sel ? static_cast<int32_t*>(scratch) : nullptr;
+    if (pf != nullptr && pf->kv_fp4 != nullptr && pf->kv_scale != nullptr && pf->B == a.B) {
+        p.pf_fp4 = pf->kv_fp4;
+        p.pf_scale = pf->kv_scale;
+        p.pf_N = pf->N;
+        p.pf_code_bytes = pf->D / 2;
+        p.pf_scale_bytes = pf->D / 16;
+    }
     p.status = d_status;
 
     CUtensorMap map;
