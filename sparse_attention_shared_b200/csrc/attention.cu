@@ -494,9 +494,21 @@ __global__ void __launch_bounds__(kClThreads, 2)
     // kernel began (a Reuse layer of a stack) gathers and dequantises its rows before
     // waiting for that kernel; everything else (Q, the window) is read after the wait.
     const bool pre = glob && p.list_ready;
+    constexpr int kQv = (HQP * D / 8 + kClThreads - 1) / kClThreads;   // 16-byte chunks of Q per thread
+    uint4 qv[kQv];
+    auto load_q = [&]() {   // the query depends on the previous layer: only after the wait
+#pragma unroll
+        for (int q = 0; q < kQv; ++q) {
+            const int i = tid + q * kClThreads;
+            const int h = i / (D / 8), c = i % (D / 8);
+            qv[q] = make_uint4(0, 0, 0, 0);
+            if (i < HQP * (D / 8) && h < p.Hq) qv[q] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
+        }
+    };
     if (!pre) {
         pdl_wait();
         pdl_launch_dependents();
+        load_q();   // in flight while the list and the rows are fetched
     }
 
     // ---- 1. positions and list entries; row tid of the tile is this thread's
@@ -581,15 +593,13 @@ __global__ void __launch_bounds__(kClThreads, 2)
     if (pre) {
         pdl_wait();
         pdl_launch_dependents();
+        load_q();
     }
-    // the query (it depends on the previous layer)
 #pragma unroll
-    for (int q = 0; q < (HQP * D / 8 + kClThreads - 1) / kClThreads; ++q) {
+    for (int q = 0; q < kQv; ++q) {
         const int i = tid + q * kClThreads;
         const int h = i / (D / 8), c = i % (D / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (i < HQP * (D / 8) && h < p.Hq) v = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
-        if (i < HQP * (D / 8)) *reinterpret_cast<uint4*>(S.qpbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = v;
+        if (i < HQP * (D / 8)) *reinterpret_cast<uint4*>(S.qpbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = qv[q];
     }
     if (!glob) ok = mbar_wait(&S.bar_tma, 0, p.status, 12);
     fence_proxy_async_smem();
