@@ -103,12 +103,6 @@ __device__ __forceinline__ void st_dsmem(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
-__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialisation may start before the previous kernel in the stream has finished;
 // pdl_wait() blocks until that kernel has completed and its writes are visible

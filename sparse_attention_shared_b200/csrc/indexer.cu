@@ -359,12 +359,6 @@ __device__ __forceinline__ int sum_above(const int* sh, int bin) {
     return s;
 }
 
-// Sum of the first `n` entries (n <= kSel) of a global array, loaded in parallel.
-__device__ __forceinline__ int prefix_total(const int* arr, int n, int* red) {
-    const int v = (threadIdx.x < n) ? __ldcg(arr + threadIdx.x) : 0;
-    return sel_sum(v, red);
-}
-
 // Two exclusive scans at once over the select threads; totals in `total`.
 __device__ __forceinline__ int2 sel_scan_excl2(int2 v, int* red, int2& total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -566,12 +560,13 @@ __device__ __forceinline__ void sel_total8(int4& a, int4& b, int* red) {
 // builds the lists only.
 template <bool kSpill, bool kCands = true>
 __device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int lo0, int hi0, int lo1, int hi1,
-                                             int2* lbuf, int* lcnt, int* lists, int* wn, int* ovf) {
+                                             int2* lbuf, int* lcnt, int* lists, int* wn, int* ovf,
+                                             int* above = nullptr) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const unsigned below = (1u << lane) - 1u;
     const bool on0 = lo0 <= hi0, on1 = lo1 <= hi1;
     int* list = lists + wp * kListCap;
-    int ln = 0;
+    int ln = 0, na0 = 0, na1 = 0;
     int s0, s1;
     warp_steps(n, s0, s1);
 #pragma unroll 4
@@ -581,6 +576,8 @@ __device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int
         const bool m0 = e < n && x >= lo0 && x <= hi0, m1 = e < n && x >= lo1 && x <= hi1;
         const bool a0 = e < n && on0 && x > hi0, a1 = e < n && on1 && x > hi1;
         const unsigned f = (a0 ? 1u : 0u) | (m0 ? 2u : 0u) | (a1 ? 4u : 0u) | (m1 ? 8u : 0u);
+        na0 += a0;
+        na1 += a1;
         const unsigned bk = __ballot_sync(0xffffffffu, f != 0u);
         if (bk) {
             const int at = ln + __popc(bk & below);
@@ -601,9 +598,63 @@ __device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int
         if (m0 && w0 < kCandCap) lbuf[w0] = cv;
         if (m1 && w1 < kCandCap) lbuf[kCandCap + w1] = cv;
     }
+    if (above != nullptr) {   // this CTA's elements above each interval (above[] zeroed by the caller)
+        na0 = __reduce_add_sync(0xffffffffu, na0);
+        na1 = __reduce_add_sync(0xffffffffu, na1);
+        if (lane == 0) { atomicAdd(above, na0); atomicAdd(above + 1, na1); }
+    }
     if (lane == 0) {
         wn[wp] = min(ln, kListCap);
         if (ln > kListCap) *ovf = 1;
+    }
+}
+
+// Candidates of both tracks (list entries inside a track's interval) from the warps'
+// ordered lists into lbuf[0..) and lbuf[kCandCap..) as (score, element index + base);
+// counts to lcnt[0..1]. Valid when no list overflowed. wsum: 2 * kSelWarps ints.
+template <bool kSpill>
+__device__ __forceinline__ void cands_from_lists(const int* sc, int base, const int* lists, const int* wn,
+                                                 int2* lbuf, int* lcnt, int* wsum) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    const int* list = lists + wp * kListCap;
+    const int n = wn[wp];
+    int c0 = 0, c1 = 0;
+#pragma unroll 1
+    for (int i = lane; i < n; i += 32) {
+        const unsigned f = (unsigned)list[i] >> 28;
+        c0 += (f & 2u) != 0u;
+        c1 += (f & 8u) != 0u;
+    }
+    c0 = __reduce_add_sync(0xffffffffu, c0);
+    c1 = __reduce_add_sync(0xffffffffu, c1);
+    if (lane == 0) { wsum[2 * wp] = c0; wsum[2 * wp + 1] = c1; }
+    sel_sync();
+    int o0 = 0, o1 = 0, t0 = 0, t1 = 0;
+#pragma unroll 1
+    for (int w = 0; w < kSelWarps; ++w) {
+        const int a = wsum[2 * w], b = wsum[2 * w + 1];
+        o0 += w < wp ? a : 0;
+        o1 += w < wp ? b : 0;
+        t0 += a;
+        t1 += b;
+    }
+    if (threadIdx.x == 0) { lcnt[0] = t0; lcnt[1] = t1; }
+#pragma unroll 1
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const int ent = i < n ? list[i] : 0;
+        const unsigned f = i < n ? ((unsigned)ent >> 28) : 0u;
+        const bool in0 = (f & 2u) != 0u, in1 = (f & 8u) != 0u;
+        const unsigned b0 = __ballot_sync(0xffffffffu, in0), b1 = __ballot_sync(0xffffffffu, in1);
+        if (in0 || in1) {
+            const int e = ent & 0x0FFFFFFF;
+            const int2 cv = make_int2(ld_score<kSpill>(sc, e), base + e);
+            if (in0) { const int k = o0 + __popc(b0 & below); if (k < kCandCap) lbuf[k] = cv; }
+            if (in1) { const int k = o1 + __popc(b1 & below); if (k < kCandCap) lbuf[kCandCap + k] = cv; }
+        }
+        o0 += __popc(b0);
+        o1 += __popc(b1);
     }
 }
 
@@ -827,16 +878,6 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
     }
     if (rq[0] > 0 || rq[1] > 0) {
         find_rank_bins2(g0cur, rq, S.red, S.info);
-        int a0 = 0, a1 = 0;
-        const int d0 = S.info[0], d1 = S.info[8];
-#pragma unroll 1
-        for (int i = tid; i < kBins; i += kSel) {
-            const int v = S.hist0[i];
-            a0 += (rq[0] > 0 && i > d0) ? v : 0;
-            a1 += (rq[1] > 0 && i > d1) ? v : 0;
-        }
-        int4 ta = make_int4(a0, a1, 0, 0), tb = make_int4(0, 0, 0, 0);
-        sel_total8(ta, tb, S.red);
 #pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
             if (rq[tr] <= 0) continue;
@@ -845,9 +886,24 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
             k.rrem = rq[tr] - S.info[8 * tr + 1];
             k.C = S.info[8 * tr + 2];
             k.prefix = (uint64_t)d;
-            k.above = tr == 0 ? ta.x : ta.y;
             bin0_interval((uint32_t)d, k.lo, k.hi);
             k.state = (k.C <= kCandCap) ? TS_CAND : TS_RADIX;
+        }
+        // this CTA's elements above the threshold bin: counted by the candidate gather,
+        // or here from the local histogram for a track that goes to the radix rounds
+        if (tk[0].state == TS_RADIX || tk[1].state == TS_RADIX) {
+            int a0 = 0, a1 = 0;
+            const int d0 = S.info[0], d1 = S.info[8];
+#pragma unroll 1
+            for (int i = tid; i < kBins; i += kSel) {
+                const int v = S.hist0[i];
+                a0 += (rq[0] > 0 && i > d0) ? v : 0;
+                a1 += (rq[1] > 0 && i > d1) ? v : 0;
+            }
+            int4 ta = make_int4(a0, a1, 0, 0), tb = make_int4(0, 0, 0, 0);
+            sel_total8(ta, tb, S.red);
+            if (tk[0].state == TS_RADIX) tk[0].above = ta.x;
+            if (tk[1].state == TS_RADIX) tk[1].above = ta.y;
         }
     }
 
@@ -861,12 +917,26 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
             any = true;
             int2* lbuf = reinterpret_cast<int2*>(&S.stage[0][0]);
             int* lcnt = S.info + 40;
-            if (tid == 0) { lcnt[0] = 0; lcnt[1] = 0; S.wlist_ovf = 0; }
+            const bool lvl0 = tk[0].level == 0 && tk[1].level == 0;   // "above" counts are complete at level 0
+            if (tid == 0) { lcnt[0] = 0; lcnt[1] = 0; S.wlist_ovf = 0; S.info[48] = 0; S.info[49] = 0; }
             sel_sync();
-            gather_cands<kSpill>(sc, my_n, lo, g0on ? tk[0].lo : 1, g0on ? tk[0].hi : 0, g1on ? tk[1].lo : 1,
-                                 g1on ? tk[1].hi : 0, lbuf, lcnt, wlists(S), S.wlist_n, &S.wlist_ovf);
+            const int glo0 = g0on ? tk[0].lo : 1, ghi0 = g0on ? tk[0].hi : 0;
+            const int glo1 = g1on ? tk[1].lo : 1, ghi1 = g1on ? tk[1].hi : 0;
+            gather_cands<kSpill, false>(sc, my_n, lo, glo0, ghi0, glo1, ghi1, nullptr, nullptr, wlists(S), S.wlist_n,
+                                        &S.wlist_ovf, lvl0 ? S.info + 48 : nullptr);
             list_tracks = (g0on ? 1 : 0) | (g1on ? 2 : 0);   // a gather rebuilds the lists
             sel_sync();
+            if (S.wlist_ovf == 0) {
+                cands_from_lists<kSpill>(sc, lo, wlists(S), S.wlist_n, lbuf, lcnt, S.wsum);
+            } else {   // a list overflowed: gather the candidates by reservation
+                gather_cands<kSpill, true>(sc, my_n, lo, glo0, ghi0, glo1, ghi1, lbuf, lcnt, wlists(S), S.wlist_n,
+                                           &S.wlist_ovf);
+            }
+            sel_sync();
+            if (lvl0) {
+                if (g0on) tk[0].above = S.info[48];
+                if (g1on) tk[1].above = S.info[49];
+            }
             if (tid == 0 || tid == 32) {
                 const int tr = tid >> 5;
                 const bool on = tr == 0 ? g0on : g1on;
@@ -943,15 +1013,10 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         const int tr_g = grp & 1;
         const int st_g = tk[tr_g].state;
         const bool fin = st_g == TS_FIN_CAND || st_g == TS_FIN_EQ;
+        // the published counts and the candidates of both tracks: one load round
         int v = 0;
         if (grp < 4 && fin && ci < c.cta && (grp < 2 || st_g == TS_FIN_EQ))
             v = __ldcg(sl.pub + (tr_g * 3 + (grp >> 1)) * kMaxG + ci);
-        v = __reduce_add_sync(0xffffffffu, v);
-        if ((tid & 31) == 0 && tid < 256) S.red[tid >> 5] = v;
-        sel_sync();
-        const int prev[2] = {S.red[0] + S.red[1], S.red[2] + S.red[3]};
-        const int eqb[2] = {S.red[4] + S.red[5], S.red[6] + S.red[7]};
-        // candidates of both tracks, one load round
         int* cx0 = reinterpret_cast<int*>(&S.stage[0][0]);
         const int n0 = tk[0].state == TS_FIN_CAND ? tk[0].C : 0, n1 = tk[1].state == TS_FIN_CAND ? tk[1].C : 0;
 #pragma unroll 1
@@ -961,7 +1026,11 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
             cx0[tr * 2 * kCandCap + k] = cv.x;
             cx0[tr * 2 * kCandCap + kCandCap + k] = cv.y;
         }
+        v = __reduce_add_sync(0xffffffffu, v);
+        if ((tid & 31) == 0 && tid < 256) S.red[tid >> 5] = v;
         sel_sync();
+        const int prev[2] = {S.red[0] + S.red[1], S.red[2] + S.red[3]};
+        const int eqb[2] = {S.red[4] + S.red[5], S.red[6] + S.red[7]};
         int T[2] = {INT_MAX, INT_MAX}, need[2] = {0, 0};
         if (n0 > 0 || n1 > 0) {
             const int4 ls = local_select2(cx0, n0, tk[0].rrem, tk[0].lo, tk[0].hi, cx0 + 2 * kCandCap, n1, tk[1].rrem,
@@ -1283,20 +1352,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int my_n = min(lo + p.chunk, n_all) - lo;
         const int nst = (my_n + kRows - 1) / kRows;
 
-        // index query -> B operand (16 rows: heads, zero past Hi); zero the histogram
-        fence_proxy_async_smem();
-        for (int i = tid; i < p.Hi * DI / 16; i += kTcThreads)
-            reinterpret_cast<int4*>(S.q)[i] = reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * DI)[i];
-        for (int i = tid; i < kBins; i += kTcThreads) S.hist0[i] = 0;
-        __syncthreads();
-        for (int i = tid; i < DI; i += kTcThreads) {
-            const int h = i / (DI / 16), c2 = i % (DI / 16);
-            int4 v = make_int4(0, 0, 0, 0);
-            if (h < p.Hi) v = reinterpret_cast<const int4*>(S.q + h * DI)[c2];
-            *reinterpret_cast<int4*>(S.qtc + tile_off(h, c2, DI)) = v;
+        // index query -> B operand (16 rows: heads, zero past Hi); zero the histogram. The
+        // TMA warp takes no part: it starts streaming keys at once, and the others meet on
+        // named barrier 2 (the previous unit's select ended at a block barrier).
+        if (warp != kSel / 32) {
+            constexpr int kStg = kTcThreads - 32;
+            const int li = tid < kSel ? tid : tid - 32;
+            fence_proxy_async_smem();
+            for (int i = li; i < p.Hi * DI / 16; i += kStg)
+                reinterpret_cast<int4*>(S.q)[i] = reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * DI)[i];
+            for (int i = li; i < kBins; i += kStg) S.hist0[i] = 0;
+            asm volatile("bar.sync 2, %0;" ::"n"(kStg) : "memory");
+            for (int i = li; i < DI; i += kStg) {
+                const int h = i / (DI / 16), c2 = i % (DI / 16);
+                int4 v = make_int4(0, 0, 0, 0);
+                if (h < p.Hi) v = reinterpret_cast<const int4*>(S.q + h * DI)[c2];
+                *reinterpret_cast<int4*>(S.qtc + tile_off(h, c2, DI)) = v;
+            }
+            fence_proxy_async_smem();
+            asm volatile("bar.sync 2, %0;" ::"n"(kStg) : "memory");
         }
-        fence_proxy_async_smem();
-        __syncthreads();
 
         if (warp == kSel / 32) {
             // ---- TMA producer
