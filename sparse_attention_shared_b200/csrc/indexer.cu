@@ -609,6 +609,56 @@ __device__ __forceinline__ void gather_cands(const int* sc, int n, int base, int
     }
 }
 
+// The ordered lists and the counts above each interval, as in gather_cands with
+// kCands = false, two elements per lane per step: lane l holds elements 2l and 2l + 1
+// of a 64-element step, and ballots over both keep the entries in position order.
+template <bool kSpill>
+__device__ __forceinline__ void gather_lists2(const int* sc, int n, int lo0, int hi0, int lo1, int hi1, int* lists,
+                                              int* wn, int* ovf, int* above) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    const bool on0 = lo0 <= hi0, on1 = lo1 <= hi1;
+    int* list = lists + wp * kListCap;
+    int ln = 0, na0 = 0, na1 = 0;
+    const int nstep = (n + 63) >> 6;
+    const int spw = (nstep + kSelWarps - 1) / kSelWarps;
+    const int s0 = min(nstep, wp * spw), s1 = min(nstep, s0 + spw);
+#pragma unroll 2
+    for (int st = s0; st < s1; ++st) {
+        const int e = st * 64 + 2 * lane;
+        int2 x2;
+        if constexpr (kSpill) x2 = __ldcg(reinterpret_cast<const int2*>(sc + e));
+        else x2 = *reinterpret_cast<const int2*>(sc + e);
+        unsigned f[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int x = q == 0 ? x2.x : x2.y;
+            const bool ok = e + q < n;
+            const bool a0 = ok && on0 && x > hi0, m0 = ok && x >= lo0 && x <= hi0;
+            const bool a1 = ok && on1 && x > hi1, m1 = ok && x >= lo1 && x <= hi1;
+            f[q] = (a0 ? 1u : 0u) | (m0 ? 2u : 0u) | (a1 ? 4u : 0u) | (m1 ? 8u : 0u);
+            na0 += a0;
+            na1 += a1;
+        }
+        const unsigned k0 = __ballot_sync(0xffffffffu, f[0] != 0u), k1 = __ballot_sync(0xffffffffu, f[1] != 0u);
+        if ((k0 | k1) == 0u) continue;
+        const int at = ln + __popc(k0 & below) + __popc(k1 & below);
+        if (f[0] != 0u && at < kListCap) list[at] = e | (int)(f[0] << 28);
+        const int at1 = at + (f[0] != 0u ? 1 : 0);
+        if (f[1] != 0u && at1 < kListCap) list[at1] = (e + 1) | (int)(f[1] << 28);
+        ln += __popc(k0) + __popc(k1);
+    }
+    if (above != nullptr) {   // this CTA's elements above each interval (above[] zeroed by the caller)
+        na0 = __reduce_add_sync(0xffffffffu, na0);
+        na1 = __reduce_add_sync(0xffffffffu, na1);
+        if (lane == 0) { atomicAdd(above, na0); atomicAdd(above + 1, na1); }
+    }
+    if (lane == 0) {
+        wn[wp] = min(ln, kListCap);
+        if (ln > kListCap) *ovf = 1;
+    }
+}
+
 // Candidates of both tracks (list entries inside a track's interval) from the warps'
 // ordered lists into lbuf[0..) and lbuf[kCandCap..) as (score, element index + base);
 // counts to lcnt[0..1]. Valid when no list overflowed. wsum: 2 * kSelWarps ints.
@@ -922,8 +972,8 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
             sel_sync();
             const int glo0 = g0on ? tk[0].lo : 1, ghi0 = g0on ? tk[0].hi : 0;
             const int glo1 = g1on ? tk[1].lo : 1, ghi1 = g1on ? tk[1].hi : 0;
-            gather_cands<kSpill, false>(sc, my_n, lo, glo0, ghi0, glo1, ghi1, nullptr, nullptr, wlists(S), S.wlist_n,
-                                        &S.wlist_ovf, lvl0 ? S.info + 48 : nullptr);
+            gather_lists2<kSpill>(sc, my_n, glo0, ghi0, glo1, ghi1, wlists(S), S.wlist_n, &S.wlist_ovf,
+                                  lvl0 ? S.info + 48 : nullptr);
             list_tracks = (g0on ? 1 : 0) | (g1on ? 2 : 0);   // a gather rebuilds the lists
             sel_sync();
             if (S.wlist_ovf == 0) {
@@ -1188,7 +1238,7 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         const int rrem = r - S.info[1];
         // one pass builds the warps' ordered lists (top-k is track 1); the threshold
         // comes from a radix select over the scores inside the bin's interval
-        gather_cands<false, false>(S.sc, n, 0, 1, 0, blo, bhi, nullptr, nullptr, wlists(S), S.wlist_n, &S.wlist_ovf);
+        gather_lists2<false>(S.sc, n, 1, 0, blo, bhi, wlists(S), S.wlist_n, &S.wlist_ovf, nullptr);
         const int4 ls = local_select2(S.sc, 0, 0, 1, 0, S.sc, n, rrem, blo, bhi, histl(S, 0), S.red, S.info);
         cut.T = ls.z;
         cut.quota = ls.w;   // the ties at T ranked within the first r, all in this CTA

@@ -79,7 +79,9 @@ def test_index_full_tiny(ws, status):
 
 
 @pytest.mark.parametrize("B,N,Tq,k,P", [(4, 8192, 1, 2048, 4096), (3, 5000, 2, 300, 1000), (2, 20000, 1, 2048, 8192),
-                                        (1, 70001, 1, 2048, 8192), (40, 3000, 1, 100, 0)])
+                                        (1, 70001, 1, 2048, 8192), (40, 3000, 1, 100, 0),
+                                        # more units than SMs: one CTA per unit, scores spilled past 16384
+                                        (150, 20000, 1, 512, 2048)])
 def test_index_full_shapes(B, N, Tq, k, P, ws, status):
     qi = synth.randint_i8(1, 10 + B, (B, Tq, 8, 64))
     ki = synth.randint_i8(1, 20 + N, (B, N, 64))
@@ -174,6 +176,26 @@ def test_index_reindex(ws, status):
     for b in range(B):
         got = set(topk2[b, 0].cpu().numpy().tolist()) - {-1}
         assert got <= set(rpool[b, 0].tolist())
+
+
+def test_index_reindex_concentrated_top(ws, status):
+    """A 16384-entry pool whose keys are aligned with the weighted index query in one
+    band of positions: the group's single select finds the whole top-k in a few warps'
+    ranges, their ordered lists overflow, and the cut falls back to the passes over
+    all scores."""
+    B, N, P, k = 16, 40000, 16384, 2048
+    qi = synth.randint_i8(9, 1, (B, 1, 8, 64))
+    ki = synth.randint_i8(9, 2, (B, N, 64))
+    w = synth.randint_i32(9, 3, (8,), 1, 8)
+    pool = np.broadcast_to(np.arange(P, dtype=np.int32), (B, 1, P)).copy()
+    noise = synth.randint_i32(9, 4, (B, 3000, 64), -37, 37)
+    for b in range(B):
+        v = (w[:, None].astype(np.int64) * qi[b, 0].astype(np.int64)).sum(0)
+        ki[b, 2000:5000] = np.clip(np.sign(v)[None, :] * 90 + noise[b], -127, 127).astype(np.int8)
+    q_pos = np.full((B, 1), N - 1, np.int32)
+    _, t2 = ops.index_topk("REINDEX", dev(q_pos), dev(qi), w, dev(ki), k, pool_in=dev(pool), ws=ws, status=status)
+    ref = np.stack([[O.index_reindex(qi[b, 0], w, ki[b], pool[b, 0], k)] for b in range(B)])
+    assert_lists_equal(t2, ref, "reindex topk")
 
 
 def test_index_reindex_ties_small_pool(ws, status):
@@ -323,6 +345,12 @@ def test_layer_stack_rejects_bad_mode_order(ws):
 def test_decode_full_sampled(ws, status):
     wl = synth.make_workload("decode_full")
     _check_stack(wl, [(0, 0), (17, 0), (31, 0)], ws, status, keep_reuse=False)
+
+
+def test_prefill_chunk_sampled(ws, status):
+    # 4096 queries of one sequence (one CTA per query, scores spilled), 32 heads
+    wl = synth.make_workload("prefill_chunk")
+    _check_stack(wl, [(0, 0), (0, 1777), (0, 4095)], ws, status, keep_reuse=False)
 
 
 def test_stack20_128k_sampled(ws, status):
