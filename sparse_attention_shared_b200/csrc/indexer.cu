@@ -404,6 +404,8 @@ __device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo
     };
     int rem0 = C0 > 0 ? nbits(lo0, hi0) : 0, rem1 = C1 > 0 ? nbits(lo1, hi1) : 0;
     uint32_t pf0 = 0, pf1 = 0;
+    int T0 = 0, T1 = 0;
+    bool fin0 = false, fin1 = false;   // threshold found by ranking the last few values directly
 #pragma unroll 1
     while (rem0 > 0 || rem1 > 0) {
         const int tk0 = min(rem0, 12), sh0 = rem0 - tk0, per0 = rem0 > 0 ? max(kSel, 1 << tk0) / kSel : 0;
@@ -444,7 +446,7 @@ __device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo
 #pragma unroll 1
             for (int i = per0 - 1; i >= 0; --i) {
                 const int h = h0[per0 * t + i];
-                if (r0 <= ab0 + h) { info[0] = per0 * t + i; info[1] = ab0; break; }
+                if (r0 <= ab0 + h) { info[0] = per0 * t + i; info[1] = ab0; info[4] = h; break; }
                 ab0 += h;
             }
         }
@@ -452,15 +454,58 @@ __device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo
 #pragma unroll 1
             for (int i = per1 - 1; i >= 0; --i) {
                 const int h = h1[per1 * t + i];
-                if (r1 <= ab1 + h) { info[2] = per1 * t + i; info[3] = ab1; break; }
+                if (r1 <= ab1 + h) { info[2] = per1 * t + i; info[3] = ab1; info[5] = h; break; }
                 ab1 += h;
             }
         }
+        if (t == 0) { info[6] = 0; info[7] = 0; }
         sel_sync();
         if (rem0 > 0) { r0 -= info[1]; pf0 = (pf0 << tk0) | (uint32_t)info[0]; rem0 = sh0; }
         if (rem1 > 0) { r1 -= info[3]; pf1 = (pf1 << tk1) | (uint32_t)info[2]; rem1 = sh1; }
+        // a track whose chosen bin holds at most 32 values, with bits still to resolve,
+        // finishes by ranking those values directly instead of another radix pass
+        const bool bf0 = rem0 > 0 && info[4] <= 32, bf1 = rem1 > 0 && info[5] <= 32;
+        if (bf0 || bf1) {
+            if (bf0) {   // this track's histogram is no longer needed: it holds the values
+#pragma unroll 1
+                for (int i = t; i < C0; i += kSel) {
+                    const int x = x0[i];
+                    const uint32_t v = (uint32_t)((long long)x - (long long)lo0);
+                    if (x >= lo0 && x <= hi0 && (uint32_t)(((uint64_t)v) >> rem0) == pf0) h0[atomicAdd(&info[6], 1) & 31] = x;
+                }
+            }
+            if (bf1) {
+#pragma unroll 1
+                for (int i = t; i < C1; i += kSel) {
+                    const int x = x1[i];
+                    const uint32_t v = (uint32_t)((long long)x - (long long)lo1);
+                    if (x >= lo1 && x <= hi1 && (uint32_t)(((uint64_t)v) >> rem1) == pf1) h1[atomicAdd(&info[7], 1) & 31] = x;
+                }
+            }
+            sel_sync();
+            // warp 0 ranks track 0's values, warp 1 track 1's: the value with
+            // (#larger) < r <= (#larger or equal) is the threshold
+            const int wk = t >> 5, ln = t & 31;
+            if ((wk == 0 && bf0) || (wk == 1 && bf1)) {
+                const int m = min(wk == 0 ? info[6] : info[7], 32);
+                const int r = wk == 0 ? r0 : r1;
+                const int vi = ln < m ? (wk == 0 ? h0[ln] : h1[ln]) : 0;
+                int gt = 0, ge = 0;
+#pragma unroll 1
+                for (int j = 0; j < m; ++j) {
+                    const int vj = __shfl_sync(0xffffffffu, vi, j);
+                    gt += vj > vi;
+                    ge += vj >= vi;
+                }
+                if (ln < m && gt < r && r <= ge) { info[8 + 2 * wk] = vi; info[9 + 2 * wk] = r - gt; }
+            }
+            sel_sync();
+            if (bf0) { T0 = info[8]; r0 = info[9]; fin0 = true; rem0 = 0; }
+            if (bf1) { T1 = info[10]; r1 = info[11]; fin1 = true; rem1 = 0; }
+        }
     }
-    return make_int4((int)((long long)lo0 + (long long)pf0), r0, (int)((long long)lo1 + (long long)pf1), r1);
+    return make_int4(fin0 ? T0 : (int)((long long)lo0 + (long long)pf0), r0,
+                     fin1 ? T1 : (int)((long long)lo1 + (long long)pf1), r1);
 }
 
 // ------------------------------------------------------------ select + write
@@ -623,7 +668,7 @@ __device__ __forceinline__ void gather_lists2(const int* sc, int n, int lo0, int
     const int nstep = (n + 63) >> 6;
     const int spw = (nstep + kSelWarps - 1) / kSelWarps;
     const int s0 = min(nstep, wp * spw), s1 = min(nstep, s0 + spw);
-#pragma unroll 2
+#pragma unroll 4
     for (int st = s0; st < s1; ++st) {
         const int e = st * 64 + 2 * lane;
         int2 x2;
@@ -1543,6 +1588,22 @@ __global__ void __launch_bounds__(kSel, 1)
     int j = 0;
     for (int u = group; u < p.units && alive; u += p.groups, ++j) {
         const int b = u / p.Tq;
+        const int32_t* pool = full ? nullptr : p.pool_in + (size_t)u * p.P_in;
+        constexpr int RB = 2;   // Reindex: rows per thread in flight (one pair)
+        // Reindex: this CTA's slice of the pool does not depend on the query position
+        // (the position only validates the entries), so its first entries and the index
+        // query are loaded before the position arrives
+        int sidx0[RB];
+        if (!full) {
+            const int lo_r = min(cta * p.chunk, p.P_in), hi_r = min(lo_r + p.chunk, p.P_in);
+#pragma unroll
+            for (int q2 = 0; q2 < RB; ++q2) {
+                const int e = q2 * kSel + tid;
+                sidx0[q2] = (e < hi_r - lo_r) ? __ldg(pool + lo_r + e) : -1;
+            }
+        }
+        const int nq = p.Hi * p.Di / 16;   // int4 chunks of the index query (<= 128)
+        const int4 qv = tid < nq ? reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * p.Di)[tid] : make_int4(0, 0, 0, 0);
         int t = p.q_pos[u];
         const bool bad_t = (t < 0 || t >= p.N);
         if (bad_t) {
@@ -1552,20 +1613,9 @@ __global__ void __launch_bounds__(kSel, 1)
         const int n_all = full ? (t + 1) : (bad_t ? 0 : p.P_in);
         const int lo = min(cta * p.chunk, n_all);
         const int hi = min(lo + p.chunk, n_all);
-        const int32_t* pool = full ? nullptr : p.pool_in + (size_t)u * p.P_in;
-        constexpr int RB = 2;   // Reindex: rows per thread in flight (one pair)
-        int sidx0[RB];          // the first round's pool entries, loaded while the query is staged
-        if (!full) {
-#pragma unroll
-            for (int q2 = 0; q2 < RB; ++q2) {
-                const int e = q2 * kSel + tid;
-                sidx0[q2] = (e < hi - lo) ? __ldg(pool + lo + e) : -1;
-            }
-        }
 
         fence_proxy_async_smem();
-        for (int i = tid; i < p.Hi * p.Di / 16; i += kSel)
-            reinterpret_cast<int4*>(S.q)[i] = reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * p.Di)[i];
+        if (tid < nq) reinterpret_cast<int4*>(S.q)[tid] = qv;
         for (int i = tid; i < kBins; i += kSel) S.hist0[i] = 0;
         __syncthreads();
 
