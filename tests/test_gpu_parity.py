@@ -266,6 +266,7 @@ def test_attention_tiny(ws, status):
     (2, 4096, 1, 16, 128, 1, 0),         # single global entry, no window
     (2, 4096, 1, 16, 128, 2048, 0),      # no local branch
     (1, 300, 1, 16, 128, 512, 64),       # fewer positions than k: -1 padding
+    (2, 8192, 1, 16, 128, 4096, 1024),   # 16 + 8 tiles: more than one cluster holds, ticket merge
 ])
 def test_attention_shapes(B, N, Tq, Hq, D, k, W, ws, status):
     _attn_case(B, N, Tq, Hq, D, k, W, seed=B * 7 + N, ws=ws, status=status)
