@@ -27,7 +27,7 @@ size_t index_region_bytes();
 size_t index_scratch_bytes(const csa2_index_args& a, int P_in);
 size_t index_smem_bytes();
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
-                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf);
+                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready);
 // attention.cu
 size_t attn_scratch_bytes(const csa2_attn_args& a);
 csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* tickets, void* scratch,
@@ -183,7 +183,7 @@ csa2_status csa2_index_topk(const csa2_index_args* args, void* workspace, size_t
     void* scratch = ws_at(workspace, R + tickets_bytes(args->B * args->Tq));
     const int P_in = args->mode == CSA2_REINDEX ? args->P_in : 0;
     return launch_index(*args, args->pool_in, P_in, workspace, scratch, d_status, static_cast<cudaStream_t>(stream),
-                        nullptr);
+                        nullptr, 0);
 }
 
 csa2_status csa2_sparse_attn(const csa2_attn_args* args, void* workspace, size_t ws_bytes, int32_t* d_status,
@@ -225,8 +225,11 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
     for (int l = 0; l < s->L; ++l) {
         const csa2_index_args& ix = s->idx[l];
         bool copied = false;   // a list copy was issued for this layer
+        // Past the first layer the kernel before an indexer is the previous layer's
+        // attention, which writes no key, position or pool: those were complete when it began.
+        const int keys_ready = l > 0 ? 1 : 0;
         if (ix.mode == CSA2_FULL) {
-            st = launch_index(ix, nullptr, 0, workspace, scratch, d_status, strm, &s->attn[l]);
+            st = launch_index(ix, nullptr, 0, workspace, scratch, d_status, strm, &s->attn[l], keys_ready);
             if (st != CSA2_OK) return st;
             cur = ix.topk_out;
             cur_k = ix.k;
@@ -235,7 +238,7 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
                 pool_P = ix.P;
             }
         } else if (ix.mode == CSA2_REINDEX) {
-            st = launch_index(ix, pool, pool_P, workspace, scratch, d_status, strm, &s->attn[l]);
+            st = launch_index(ix, pool, pool_P, workspace, scratch, d_status, strm, &s->attn[l], keys_ready);
             if (st != CSA2_OK) return st;
             cur = ix.topk_out;
             cur_k = ix.k;

@@ -33,6 +33,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstring>
 
@@ -72,6 +73,7 @@ struct IdxParams {
     int units, G, groups, chunk;
     int32_t* spill;      // [groups*G][chunk] scores when chunk > kSmemScores
     int local_sel;       // Reindex: the group leader selects over all of the unit's scores
+    int keys_ready;      // keys and positions were complete before the previous kernel began
     int rstride;         // per-unit stride of rscore
     int32_t* rscore;     // [units][rstride] published scores (local_sel)
     // L2 prefetch of the global cache rows each top-k list selects (pf_fp4 nullptr: off)
@@ -1418,8 +1420,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr uint32_t kSbo = 8 * DI;                                             // bytes per 8-row group
     constexpr uint32_t kIdesc = idesc_i8(128, 16);
 
-    const int epoch = __ldcg(sl.ctrl + CTRL_EPOCH);
-    int bar_target = __ldcg(sl.ctrl + CTRL_BAR_BASE);
     if (warp == 0) tmem_alloc(&S.tmem_base, 32 * kTmemBufs);
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) { mbar_init(&S.full_bar[i], 1); mbar_init(&S.empty_bar[i], 1); }
@@ -1431,6 +1431,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     pdl_launch_dependents();   // the next kernel may start its own set-up
+    // The workspace and the index query may come from the previous kernel: wait for
+    // it. When the keys and positions were complete before that kernel began, the
+    // TMA producer starts the key stream at once and fills its stages meanwhile.
+    const bool producer = warp == kSel / 32;
+    if (!(producer && p.keys_ready)) pdl_wait();
+    const int epoch = producer ? 0 : __ldcg(sl.ctrl + CTRL_EPOCH);
+    int bar_target = producer ? 0 : __ldcg(sl.ctrl + CTRL_BAR_BASE);
     const uint32_t tmem = S.tmem_base;
     uint32_t seq = 0;   // tiles processed by this CTA so far (same count in every role)
 
@@ -1573,8 +1580,6 @@ __global__ void __launch_bounds__(kSel, 1)
     constexpr bool generic = (HI == 0);
     int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * p.chunk : nullptr;
 
-    const int epoch = __ldcg(sl.ctrl + CTRL_EPOCH);
-    int bar_target = __ldcg(sl.ctrl + CTRL_BAR_BASE);
     const int rows_per_stage = (full ? min(256, kStageBytes / p.Di) : 0);
     const int nchunk = p.Di / 16;
 
@@ -1582,6 +1587,9 @@ __global__ void __launch_bounds__(kSel, 1)
     mbar_fence_init();
     __syncthreads();
     pdl_launch_dependents();   // the next kernel may start its own set-up
+    pdl_wait();                // the workspace, pool and index query may come from the previous kernel
+    const int epoch = __ldcg(sl.ctrl + CTRL_EPOCH);
+    int bar_target = __ldcg(sl.ctrl + CTRL_BAR_BASE);
     uint32_t stage_seq = 0;   // key tiles issued by this CTA so far
     bool alive = true;
 
@@ -1817,17 +1825,32 @@ static cudaError_t launch_coop(Kern kern, int threads, const IdxParams& p, const
     cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    // Programmatic dependent launch on top of the cooperative one: the kernel may be
+    // scheduled while the previous kernel drains (every kernel of this library calls
+    // griddepcontrol.launch_dependents only once all of its own CTAs are resident, so
+    // neither grid can keep the other's CTAs off the device). A runtime that refuses
+    // the pair gets the plain cooperative launch from then on.
+    static std::atomic<int> coop_pdl{1};
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, p, map);
+    cfg.numAttrs = coop_pdl.load() ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, kern, p, map);
+    if (e != cudaSuccess && cfg.numAttrs == 2) {
+        (void)cudaGetLastError();
+        coop_pdl.store(0);
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, p, map);
+    }
+    return e;
 }
 
 // Launch one indexer call. `ws` holds plan_index(a).ws_bytes bytes (zero at first use).
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
-                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf) {
+                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready) {
     const int sms = num_sms();
     csa2_index_args aa = a;
     aa.P_in = P_in;
@@ -1862,6 +1885,7 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
         p.pf_code_bytes = pf->D / 2;
         p.pf_scale_bytes = pf->D / 16;
     }
+    p.keys_ready = keys_ready;
     p.status = d_status;
 
     CUtensorMap map;
