@@ -20,6 +20,7 @@
 // bf16 output and the fp32 log-sum-exp.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <cstddef>
 #include <cstring>
@@ -82,6 +83,50 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
     __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
     __nv_bfloat162 z = __hmul2(x, y);
     return *reinterpret_cast<uint32_t*>(&z);
+}
+
+// Eight E2M1 codes (a 32-bit word, lowest nibble first) as four f16x2 words, lower
+// element in the lower half. The hardware conversion is exact: every E2M1 value is
+// an f16 value.
+__device__ __forceinline__ void e2m1x8_f16(uint32_t w, uint32_t (&d)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(w));
+}
+
+// Two E4M3 scales (lower byte first) as f16x2; exact (E4M3 values are f16 values).
+__device__ __forceinline__ uint32_t e4m3x2_f16(uint32_t two) {
+    uint32_t d;
+    const uint16_t h = (uint16_t)two;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(h));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// bf16x2 -> f16x2 after scaling by a power of two f (exact unless the scaled value
+// falls below f16's normal range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, float f) {
+    const float lo = __uint_as_float(v << 16) * f, hi = __uint_as_float(v & 0xFFFF0000u) * f;
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// largest bf16 exponent field among the eight values of a 16-byte chunk
+__device__ __forceinline__ uint32_t bf16x8_max_exp(const uint4& v) {
+    const uint32_t a = max((v.x >> 7) & 0xFFu, (v.x >> 23) & 0xFFu), b = max((v.y >> 7) & 0xFFu, (v.y >> 23) & 0xFFu);
+    const uint32_t c = max((v.z >> 7) & 0xFFu, (v.z >> 23) & 0xFFu), d = max((v.w >> 7) & 0xFFu, (v.w >> 23) & 0xFFu);
+    return max(max(a, b), max(c, d));
 }
 
 template <int HQP, int D>
@@ -422,7 +467,7 @@ struct AttnClSmem {   // placed at a 1024-byte-aligned address (operand tiles ne
     // Q as [HQP rows x D] (two 64-element panels), then, once S = K Q^T has been
     // computed, P as [HQP rows x 256 keys] in four 64-key panels
     uint8_t qpbuf[4 * HQP * 128];
-    uint32_t lut[256];
+    float qmul[HQP];                      // per head: the softmax scale (log2 units) over the Q scaling
     float red[kClThreads / 32][HQP];      // per-warp head maxima, then sums
     float mfin[HQP], lfin[HQP];
     // partials pushed by the cluster's CTAs for the heads this CTA merges: head h
@@ -488,8 +533,6 @@ __global__ void __launch_bounds__(kClThreads, 2)
         mbar_init(&S.bar_o, 1);
         mbar_fence_init();
     }
-    for (int i = tid; i < 256; i += kClThreads)
-        S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
     // A global CTA of a layer whose list and cache were complete before the previous
     // kernel began (a Reuse layer of a stack) gathers and dequantises its rows before
     // waiting for that kernel; everything else (Q, the window) is read after the wait.
@@ -569,23 +612,30 @@ __global__ void __launch_bounds__(kClThreads, 2)
             reinterpret_cast<uint4*>(S.tbuf + 3 * kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
         }
     }
-    __syncthreads();   // the table is ready
+    __syncthreads();   // the barriers (initialised by thread 0) and TMEM address are set
     bool ok = true;
     if (glob) {
-        // global tile panels hold 256 rows: panel p at p * 2 * kPanelBytes; row tid
+        // A global tile is dequantised to f16 (code times scale is exact in f16) and
+        // multiplied in f16: Q is brought into f16's range by a power of two per head
+        // below. Panels hold 256 rows: panel p at p * 2 * kPanelBytes; row tid.
+        uint32_t sp[D / 32];   // f16x2 scale pairs (groups 2i, 2i + 1)
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) sp[i] = e4m3x2_f16(sc0[i >> 1] >> (16 * (i & 1)));
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
             uint4 o = make_uint4(0, 0, 0, 0);
             if (v0) {
                 const uint4 w4 = c0[c >> 2];
                 const uint32_t w = (c & 3) == 0 ? w4.x : (c & 3) == 1 ? w4.y : (c & 3) == 2 ? w4.z : w4.w;
-                const uint32_t g = c >> 1;
-                const uint32_t s16 = e4m3_bf16_bits((sc0[g >> 2] >> (8 * (g & 3))) & 0xFFu);
-                const uint32_t s2x = s16 | (s16 << 16);
-                o.x = bf16x2_mul(S.lut[w & 0xFFu], s2x);
-                o.y = bf16x2_mul(S.lut[(w >> 8) & 0xFFu], s2x);
-                o.z = bf16x2_mul(S.lut[(w >> 16) & 0xFFu], s2x);
-                o.w = bf16x2_mul(S.lut[w >> 24], s2x);
+                const uint32_t g = c >> 1;   // scale group of 16
+                const uint32_t pr = sp[g >> 1];
+                const uint32_t s2x = (g & 1) ? ((pr >> 16) | (pr & 0xFFFF0000u)) : ((pr & 0xFFFFu) | (pr << 16));
+                uint32_t d[4];
+                e2m1x8_f16(w, d);
+                o.x = f16x2_mul(d[0], s2x);
+                o.y = f16x2_mul(d[1], s2x);
+                o.z = f16x2_mul(d[2], s2x);
+                o.w = f16x2_mul(d[3], s2x);
             }
             *reinterpret_cast<uint4*>(S.tbuf + (c >> 3) * (2 * kPanelBytes) + sw128(tid, c & 7)) = o;
         }
@@ -599,7 +649,26 @@ __global__ void __launch_bounds__(kClThreads, 2)
     for (int q = 0; q < kQv; ++q) {
         const int i = tid + q * kClThreads;
         const int h = i / (D / 8), c = i % (D / 8);
-        if (i < HQP * (D / 8)) *reinterpret_cast<uint4*>(S.qpbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = qv[q];
+        uint4 v = qv[q];
+        float mul = p.scale_log2;
+        if (glob) {
+            // head h's D / 8 chunks sit in D / 8 consecutive lanes: the largest exponent
+            // over the head sets 2^k, which puts the head's largest value in [2^14, 2^15)
+            uint32_t e = bf16x8_max_exp(v);
+#pragma unroll
+            for (int o = 1; o < D / 8; o <<= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+            const int k = (e == 0u) ? 0 : min(141 - (int)e, 126);
+            const float f = __uint_as_float((uint32_t)(127 + k) << 23);
+            v.x = bf16x2_to_f16x2(v.x, f);
+            v.y = bf16x2_to_f16x2(v.y, f);
+            v.z = bf16x2_to_f16x2(v.z, f);
+            v.w = bf16x2_to_f16x2(v.w, f);
+            mul = p.scale_log2 * __uint_as_float((uint32_t)(127 - k) << 23);
+        }
+        if (i < HQP * (D / 8)) {
+            *reinterpret_cast<uint4*>(S.qpbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = v;
+            if (c == 0) S.qmul[h] = mul;
+        }
     }
     if (!glob) ok = mbar_wait(&S.bar_tma, 0, p.status, 12);
     fence_proxy_async_smem();
@@ -613,7 +682,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
     // ---- 3. S = K Q^T per 128-row block
     if (tid == 0) {
         const uint32_t ka = smem_u32(S.tbuf), qa = smem_u32(S.qpbuf);
-        constexpr uint32_t idesc = idesc_bf16(128, HQP, 0);
+        const uint32_t idesc = glob ? idesc_f16(128, HQP, 0) : idesc_bf16(128, HQP, 0);
         for (int blk = 0; blk < nblk; ++blk) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -643,7 +712,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
     }
     const bool r0 = v0 && ok;
 #pragma unroll
-    for (int h = 0; h < HQP; ++h) a[h] = r0 ? a[h] * p.scale_log2 : -INFINITY;
+    for (int h = 0; h < HQP; ++h) a[h] = r0 ? a[h] * S.qmul[h] : -INFINITY;
     const int hl = (HQP == 16) ? ((lane >> 1) & 15) : lane;   // the head this lane ends up holding
     {
         float v[HQP];
@@ -666,8 +735,9 @@ __global__ void __launch_bounds__(kClThreads, 2)
         const float mh = S.mfin[h];
         pv[h] = (r0 && mh != -INFINITY) ? exp2f(a[h] - mh) : 0.f;
         // key tid -> panel tid / 64, column tid % 64
-        *reinterpret_cast<__nv_bfloat16*>(S.qpbuf + (tid >> 6) * (HQP * 128) + sw128(h, (tid & 63) >> 3) + (tid & 7) * 2) =
-            __float2bfloat16_rn(pv[h]);
+        const float pr = pv[h];
+        *reinterpret_cast<uint16_t*>(S.qpbuf + (tid >> 6) * (HQP * 128) + sw128(h, (tid & 63) >> 3) + (tid & 7) * 2) =
+            glob ? __half_as_ushort(__float2half_rn(pr)) : __bfloat16_as_ushort(__float2bfloat16_rn(pr));
     }
     {
         const float l = warp_transpose_reduce<HQP, false>(pv);
@@ -687,7 +757,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
     // ---- 5. O^T = V^T P (keys as the reduction; the head dim as M)
     if (tid == 0) {
         const uint32_t va = smem_u32(glob ? S.tbuf : S.tbuf + 2 * kPanelBytes), pa = smem_u32(S.qpbuf);
-        constexpr uint32_t idesc = idesc_bf16(128, HQP, 1);
+        const uint32_t idesc = glob ? idesc_f16(128, HQP, 1) : idesc_bf16(128, HQP, 1);
         const int nk = nblk * (kTileKeys / 16);
         for (int kk = 0; kk < nk; ++kk) {
             const uint64_t ad = smem_desc(va + kk * 2048, panel_stride, 1024);

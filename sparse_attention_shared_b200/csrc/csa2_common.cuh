@@ -213,6 +213,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major) 
            | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 
+// The same with f16 A and B.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major) {
+    return idesc_bf16(M, N, a_mn_major) & ~((7u << 7) | (7u << 10));
+}
+
 // Instruction descriptor, kind::i8 with signed int8 A/B (both K-major) and int32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
     return (2u << 4)                          // D format: s32
