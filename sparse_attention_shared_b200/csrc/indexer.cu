@@ -755,6 +755,41 @@ __device__ __forceinline__ void cands_from_lists(const int* sc, int base, const 
     }
 }
 
+// Scores of the list entries that carry flag bit `fb` (inside a track's interval),
+// in list order, to out[0..); returns their number. Valid when no list overflowed.
+// wsum: kSelWarps ints.
+__device__ __forceinline__ int vals_from_lists(const int* sc, const int* lists, const int* wn, unsigned fb, int* out,
+                                               int* wsum) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    const int* list = lists + wp * kListCap;
+    const int n = wn[wp];
+    int c = 0;
+#pragma unroll 1
+    for (int i = lane; i < n; i += 32) c += (((unsigned)list[i] >> 28) & fb) != 0u;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (lane == 0) wsum[wp] = c;
+    sel_sync();
+    int o = 0, tot = 0;
+#pragma unroll 1
+    for (int w = 0; w < kSelWarps; ++w) {
+        const int a = wsum[w];
+        o += w < wp ? a : 0;
+        tot += a;
+    }
+#pragma unroll 1
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const int ent = i < n ? list[i] : 0;
+        const bool in = i < n && (((unsigned)ent >> 28) & fb) != 0u;
+        const unsigned b = __ballot_sync(0xffffffffu, in);
+        if (in) out[o + __popc(b & below)] = sc[ent & 0x0FFFFFFF];
+        o += __popc(b);
+    }
+    sel_sync();   // wsum is free again
+    return tot;
+}
+
 // Histogram of digit `lv` over the elements in [lo_t, hi_t] (they share digits 0..lv-1).
 template <bool kSpill>
 __device__ __noinline__ void radix_hist(const int* sc, int n, int lo_t, int hi_t, int lv, int* hist) {
@@ -1286,7 +1321,17 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         // one pass builds the warps' ordered lists (top-k is track 1); the threshold
         // comes from a radix select over the scores inside the bin's interval
         gather_lists2<false>(S.sc, n, 1, 0, blo, bhi, wlists(S), S.wlist_n, &S.wlist_ovf, nullptr);
-        const int4 ls = local_select2(S.sc, 0, 0, 1, 0, S.sc, n, rrem, blo, bhi, histl(S, 0), S.red, S.info);
+        sel_sync();
+        // the radix select runs over the bin's elements only (from the lists), or over
+        // all n scores when a list overflowed; the key stages are free in Reindex mode
+        const int* xs = S.sc;
+        int nx = n;
+        if (S.wlist_ovf == 0) {
+            int* cx = reinterpret_cast<int*>(&S.stage[0][0]);
+            nx = vals_from_lists(S.sc, wlists(S), S.wlist_n, 8u, cx, S.wsum);
+            xs = cx;
+        }
+        const int4 ls = local_select2(S.sc, 0, 0, 1, 0, xs, nx, rrem, blo, bhi, histl(S, 0), S.red, S.info);
         cut.T = ls.z;
         cut.quota = ls.w;   // the ties at T ranked within the first r, all in this CTA
         lists = S.wlist_ovf == 0;
