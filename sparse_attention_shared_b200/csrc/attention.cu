@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         mbar_fence_init();
     }
     // A global CTA of a layer whose list and cache were complete before the previous
-    // kernel began (a Reuse layer of a stack) gathers and dequantises its rows before
+    // kernel began (a Reuse layer of a stack) issues its list and row loads before
     // waiting for that kernel; everything else (Q, the window) is read after the wait.
     const bool pre = glob && p.list_ready;
     constexpr int kQv = (HQP * D / 8 + kClThreads - 1) / kClThreads;   // 16-byte chunks of Q per thread
@@ -612,6 +612,13 @@ __global__ void __launch_bounds__(kClThreads, 2)
             reinterpret_cast<uint4*>(S.tbuf + 3 * kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
         }
     }
+    if (pre) {
+        // the rows are in flight: wait for the previous kernel here, so that a CTA that
+        // starts after it has ended has its query load in flight during the dequantisation
+        pdl_wait();
+        pdl_launch_dependents();
+        load_q();
+    }
     __syncthreads();   // the barriers (initialised by thread 0) and TMEM address are set
     bool ok = true;
     if (glob) {
@@ -639,11 +646,6 @@ __global__ void __launch_bounds__(kClThreads, 2)
             }
             *reinterpret_cast<uint4*>(S.tbuf + (c >> 3) * (2 * kPanelBytes) + sw128(tid, c & 7)) = o;
         }
-    }
-    if (pre) {
-        pdl_wait();
-        pdl_launch_dependents();
-        load_q();
     }
 #pragma unroll
     for (int q = 0; q < kQv; ++q) {
