@@ -67,9 +67,68 @@ def unit_bytes(spec):
     return total
 
 
-def full_launch_bytes(spec, units):
+def full_launch_bytes(spec, q_pos):
+    """Algorithmic bytes of the first layer's Full indexer call: every sequence's keys
+    up to its last query position once, then per query its index query and lists."""
     L = spec.layers[0]
-    return units * (spec.N * spec.Di + spec.Hi * spec.Di + (L.P + L.k) * 4)
+    keys = sum(int(q_pos[b].max()) + 1 for b in range(spec.B)) * spec.Di
+    return keys + spec.B * spec.Tq * (spec.Hi * spec.Di + (L.P + L.k) * 4)
+
+
+def _window_rows(lo, hi):
+    """Rows in the union of the closed intervals [lo_i, hi_i] (empty when hi < lo)."""
+    rows, cur_lo, cur_hi = 0, None, None
+    for a, b in sorted((int(x), int(y)) for x, y in zip(lo, hi) if y >= x):
+        if cur_hi is None or a > cur_hi + 1:
+            if cur_hi is not None:
+                rows += cur_hi - cur_lo + 1
+            cur_lo, cur_hi = a, b
+        else:
+            cur_hi = max(cur_hi, b)
+    if cur_hi is not None:
+        rows += cur_hi - cur_lo + 1
+    return rows
+
+
+def list_bytes(spec, q_pos, local_base, pools, topks):
+    """Algorithmic bytes of one stack call, each distinct row once per kernel call,
+    counted from the index lists the call produced (host arrays): keys scanned by a
+    Full layer (up to the sequence's last query), pool key rows gathered by a Reindex
+    layer, FP4 rows in the union of a sequence's lists, local K+V rows in the union of
+    its windows, and per query its queries, lists and outputs. With one query per
+    sequence this is the per-query sum of unit_bytes."""
+    import numpy as np
+    D, Di, Hi, Hq, W, B, Tq = spec.D, spec.Di, spec.Hi, spec.Hq, spec.W, spec.B, spec.Tq
+    total, cur, pool, P_in = 0, None, None, 0
+    for li, L in enumerate(spec.layers):
+        if L.mode == "FULL":
+            total += sum(int(q_pos[b].max()) + 1 for b in range(B)) * Di
+            total += B * Tq * (Hi * Di + (L.P + L.k) * 4)
+            cur = topks[li]
+            if L.P:
+                pool, P_in = pools[li], L.P
+        elif L.mode == "REINDEX":
+            total += sum(len(np.unique(pool[b][pool[b] >= 0])) for b in range(B)) * Di
+            total += B * Tq * (P_in * 4 + Hi * Di + L.k * 4)
+            cur = topks[li]
+        total += sum(len(np.unique(cur[b][cur[b] >= 0])) for b in range(B)) * (D // 2 + D // 16)
+        if W > 0:
+            for b in range(B):
+                t = q_pos[b].astype(np.int64)
+                lo = np.maximum(np.maximum(t - W + 1, int(local_base[b])), 0)
+                total += _window_rows(lo, t) * 2 * D * 2
+        total += B * Tq * (cur.shape[-1] * 4 + 2 * Hq * D * 2)
+    return total
+
+
+def schedule_str(spec):
+    """The layer modes, with a repeated period written once: [F,U,U,RI]x5."""
+    ab = [{"FULL": "F", "REINDEX": "RI", "REUSE": "U"}[L.mode] for L in spec.layers]
+    n = len(ab)
+    for per in range(1, n // 2 + 1):
+        if n % per == 0 and ab == ab[:per] * (n // per):
+            return "[" + ",".join(ab[:per]) + "]x" + str(n // per)
+    return ",".join(ab)
 
 
 # ------------------------------------------------------------------ clocks
@@ -283,7 +342,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     st.check("kernel timing")
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kl_ms)
-    kbytes = full_launch_bytes(s, units)
+    qp_host = q_pos.cpu().numpy()
+    kbytes = full_launch_bytes(s, qp_host)
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -299,10 +359,13 @@ def run_ours(args, rank, world, local_rank):
         pass
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                "kernel": "index_full_tc_kernel<64> (Full mode, layer 0: scan + exact pool/top-k select)",
+                "kernel": (f"index_full_tc_kernel<{s.Di}>" if s.Di in (32, 64, 128) else "index_dp4a_kernel")
+                + " (Full mode, layer 0: scan + exact pool/top-k select)",
                 "kernel_ms": round(kern_ms, 4), "algorithmic_bytes": kbytes,
                 "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback 6650 GB/s"}
-    step_bytes = unit_bytes(s) * units
+    # the lists of the last timed step (the same inputs every step)
+    host = lambda ts: [t.cpu().numpy() if t is not None else None for t in ts]
+    step_bytes = list_bytes(s, qp_host, base.cpu().numpy(), host(stack.pools), host(stack.topks))
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
 
     # end to end through the public API with host buffers
@@ -316,10 +379,11 @@ def run_ours(args, rank, world, local_rank):
         cpu = cpu_baseline(args.workload, args.cpu_seconds)
 
     res = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "metric": METRIC if s.name == DEFAULT_WORKLOAD else f"CSA2 queries/s, {s.name}; achieved HBM GB/s vs peak",
+        "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8+bf16", "data": "synthetic",
-        "config": {"workload": s.name, "B": s.B, "N": s.N, "layers": s.L, "schedule": "[F,U,U,RI]x5",
+        "config": {"workload": s.name, "B": s.B, "N": s.N, "layers": s.L, "schedule": schedule_str(s),
                    "Hq": s.Hq, "D": s.D, "Hi": s.Hi, "Di": s.Di, "pool": s.layers[0].P, "k": s.layers[0].k,
                    "W": s.W, "per_gpu_queries": units, "parallelism": f"replicas x{world}",
                    "l2": "flushed (256 MB write) before every timed step, outside its events",

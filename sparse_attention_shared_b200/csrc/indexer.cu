@@ -1468,7 +1468,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) tmem_alloc(&S.tmem_base, 32 * kTmemBufs);
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) { mbar_init(&S.full_bar[i], 1); mbar_init(&S.empty_bar[i], 1); }
-        for (int i = 0; i < kTmemBufs; ++i) { mbar_init(&S.tfull_bar[i], 1); mbar_init(&S.tempty_bar[i], kSel / 2); }
+        for (int i = 0; i < kTmemBufs; ++i) { mbar_init(&S.tfull_bar[i], 1); mbar_init(&S.tempty_bar[i], kSel / 64); }
         S.abort = 0;
         mbar_fence_init();
     }
@@ -1564,7 +1564,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t lane_base = tmem + (uint32_t)(wl >> 2) * 16u + ((uint32_t)(wl & 3) * 32u << 16);
             for (int s2 = egrp; s2 < nst; s2 += 2) {
                 const uint32_t i = seq + s2, buf = i % kTmemBufs;
-                if (!mbar_wait(&S.tfull_bar[buf], (i / kTmemBufs) & 1u, p.status, 4)) { S.abort = 1; break; }
+                const bool got = mbar_wait(&S.tfull_bar[buf], (i / kTmemBufs) & 1u, p.status, 4);
+                if (!__all_sync(0xffffffffu, got)) { S.abort = 1; break; }   // warp-uniform exit
                 tc_fence_after();
                 int x = 0;
                 if (in_block) {
@@ -1581,8 +1582,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int h = 0; h < 8; ++h) x += p.w[8 + h] * max(acc[h], 0);
                     }
                 }
+                // one arrival per warp (the buffer's barrier counts the group's 8 warps):
+                // 256 arrivals on one mbarrier per tile were serialised by shared memory
                 tc_fence_before();
-                mbar_arrive(&S.tempty_bar[buf]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.tempty_bar[buf]);
                 const int e = s2 * kRows + tl;
                 if (in_block && e < my_n) {
                     if (spill) spill[e] = x; else S.sc[e] = x;

@@ -354,6 +354,13 @@ def test_prefill_chunk_sampled(ws, status):
     _check_stack(wl, [(0, 0), (0, 1777), (0, 4095)], ws, status, keep_reuse=False)
 
 
+def test_long_1m_sampled(ws, status):
+    # one sequence of 2^20 positions, 64 queries: the Full scan spills its scores (two
+    # CTAs per query), nine Reindex layers select from the pool by the group's single select
+    wl = synth.make_workload("long_1m")
+    _check_stack(wl, [(0, 0), (0, 63)], ws, status, keep_reuse=False)
+
+
 def test_stack20_128k_sampled(ws, status):
     wl = synth.make_workload("stack20_128k")
     _check_stack(wl, [(0, 0), (15, 0)], ws, status, keep_reuse=False)
