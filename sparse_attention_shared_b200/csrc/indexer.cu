@@ -74,6 +74,8 @@ struct IdxParams {
     int32_t* spill;      // [groups*G][chunk] scores when chunk > kSmemScores
     int local_sel;       // Reindex: the group leader selects over all of the unit's scores
     int keys_ready;      // keys and positions were complete before the previous kernel began
+    const int32_t* pre;  // Full, select only: every unit's scores by position ([units][pstride]), else nullptr
+    int64_t pstride;
     int rstride;         // per-unit stride of rscore
     int32_t* rscore;     // [units][rstride] published scores (local_sel)
     // L2 prefetch of the global cache rows each top-k list selects (pf_fp4 nullptr: off)
@@ -791,15 +793,36 @@ __device__ __forceinline__ int vals_from_lists(const int* sc, const int* lists, 
 }
 
 // Histogram of digit `lv` over the elements in [lo_t, hi_t] (they share digits 0..lv-1).
+// Spilled scores are read four steps at a time, all loads in flight before the first
+// use (the histogram's atomics would otherwise keep the next load from issuing).
 template <bool kSpill>
 __device__ __noinline__ void radix_hist(const int* sc, int n, int lo_t, int hi_t, int lv, int* hist) {
     int s0, s1;
     warp_steps(n, s0, s1);
+    const int lane = threadIdx.x & 31;
+    if constexpr (kSpill) {
 #pragma unroll 1
-    for (int st = s0; st < s1; ++st) {
-        const int e = st * 32 + (threadIdx.x & 31);
-        const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
-        if (e < n && x >= lo_t && x <= hi_t) atomicAdd(&hist[digit_at(ext_key(x), lv)], 1);
+        for (int st = s0; st < s1; st += 4) {
+            int xs[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int e = (st + q) * 32 + lane;
+                xs[q] = (st + q < s1 && e < n) ? __ldcg(sc + e) : 0;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int e = (st + q) * 32 + lane;
+                if (st + q < s1 && e < n && xs[q] >= lo_t && xs[q] <= hi_t)
+                    atomicAdd(&hist[digit_at(ext_key(xs[q]), lv)], 1);
+            }
+        }
+    } else {
+#pragma unroll 1
+        for (int st = s0; st < s1; ++st) {
+            const int e = st * 32 + lane;
+            const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
+            if (e < n && x >= lo_t && x <= hi_t) atomicAdd(&hist[digit_at(ext_key(x), lv)], 1);
+        }
     }
 }
 
@@ -808,7 +831,7 @@ template <bool kSpill>
 __device__ __noinline__ int count_range(const int* sc, int n, int lo_t, int hi_t) {
     int s0, s1, cnt = 0;
     warp_steps(n, s0, s1);
-#pragma unroll 1
+#pragma unroll 4
     for (int st = s0; st < s1; ++st) {
         const int e = st * 32 + (threadIdx.x & 31);
         const int x = e < n ? ld_score<kSpill>(sc, e) : 0;
@@ -1458,7 +1481,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int group = blockIdx.x / p.G;
     const int cta = blockIdx.x % p.G;
     const Slot sl = slot_of(p, group);
-    int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * p.chunk : nullptr;
+    int* spill = (p.chunk > kSmemScores && p.pre == nullptr) ? p.spill + (size_t)blockIdx.x * p.chunk : nullptr;
     constexpr int kRows = (kStageBytes / DI) < 256 ? (kStageBytes / DI) : 256;   // rows per tile
     constexpr int kBlocks = kRows / 128;                                          // MMA row blocks per tile
     constexpr uint32_t kSwz = DI == 32 ? 6u : DI == 64 ? 4u : 2u;
@@ -1497,7 +1520,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int n_all = t + 1;
         const int lo = min(cta * p.chunk, n_all);
         const int my_n = min(lo + p.chunk, n_all) - lo;
-        const int nst = (my_n + kRows - 1) / kRows;
+        const int nst = p.pre ? 0 : (my_n + kRows - 1) / kRows;   // select only: no key tiles
 
         // index query -> B operand (16 rows: heads, zero past Hi); zero the histogram. The
         // TMA warp takes no part: it starts streaming keys at once, and the others meet on
@@ -1598,10 +1621,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncthreads();
         if (S.abort) break;
 
+        // select only: the unit's scores come from the multi-query scoring kernel; the
+        // chunk goes to shared memory when it fits, and its histogram is built here
+        const int* src = p.pre ? p.pre + (size_t)u * p.pstride + lo : nullptr;
+        if (src) {
+            // 16-byte loads, four in flight per thread (the unit's row and the chunk
+            // start are multiples of 4 elements)
+            const bool to_smem = p.chunk <= kSmemScores;
+            const int nv = my_n >> 2;
+            const int4* src4 = reinterpret_cast<const int4*>(src);
+#pragma unroll 1
+            for (int v0 = tid; v0 < nv; v0 += 4 * kTcThreads) {
+                int4 x4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int v = v0 + q * kTcThreads;
+                    x4[q] = v < nv ? __ldcg(src4 + v) : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int v = v0 + q * kTcThreads;
+                    if (v >= nv) continue;
+                    if (to_smem) reinterpret_cast<int4*>(S.sc)[v] = x4[q];
+                    atomicAdd(&S.hist0[bin0(x4[q].x)], 1);
+                    atomicAdd(&S.hist0[bin0(x4[q].y)], 1);
+                    atomicAdd(&S.hist0[bin0(x4[q].z)], 1);
+                    atomicAdd(&S.hist0[bin0(x4[q].w)], 1);
+                }
+            }
+            for (int e = 4 * nv + tid; e < my_n; e += kTcThreads) {
+                const int x = __ldcg(src + e);
+                if (to_smem) S.sc[e] = x;
+                atomicAdd(&S.hist0[bin0(x)], 1);
+            }
+            __syncthreads();
+        }
+        const int* sel_src = src ? (p.chunk > kSmemScores ? src : nullptr) : spill;
+
         if (tid < kSel) {
             UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, nullptr};
-            const bool ok = spill ? select_unit<true>(p, S, sl, c, bar_target, spill)
-                                  : select_unit<false>(p, S, sl, c, bar_target, S.sc);
+            const bool ok = sel_src ? select_unit<true>(p, S, sl, c, bar_target, sel_src)
+                                    : select_unit<false>(p, S, sl, c, bar_target, S.sc);
             if (!ok && tid == 0) S.abort = 1;
         }
         __syncthreads();
@@ -1614,6 +1674,181 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 32 * kTmemBufs);
+}
+
+// ------------------------------------------------------------ Full mode, queries that share keys
+// Several queries of one sequence (Tq >= kMqMin) score the same keys. A CTA takes a
+// block of up to kMqQ queries of a sequence and a range of 128-row key tiles. One
+// kind::i8 MMA per 32-byte K step scores a tile against all of the block's queries:
+// B row 8q + h holds query q's head h (zero past Hi or past the block), so N = 8 kMqQ,
+// and each key tile is read once per block instead of once per query. The epilogue
+// writes each query's scores, for the positions up to its own, to a per-unit array
+// that the Full kernel then cuts in its select-only mode.
+constexpr int kMqQ = 16;                                  // queries per block
+constexpr int kMqN = kMqQ * 8;                            // MMA N
+constexpr int kMqRows = 128;                              // key rows per tile (one M = 128 block)
+constexpr int kMqStages = 8;
+constexpr int kMqBufs = 4;                                // TMEM buffers of kMqN columns (512 in all)
+constexpr int kMqGroups = 4;                              // epilogue groups of 4 warps, alternate tiles
+constexpr int kMqThreads = (kMqGroups * 4 + 2) * 32;      // + the TMA and MMA warps
+constexpr int kMqMin = 4;                                 // Tq from which a Full call takes this path
+constexpr int kMqMinN = 8192;                             // ... on a key set of at least this many positions
+
+struct MqParams {
+    int B, Tq, N, Hi, nblk, splits;
+    int32_t w[8];
+    const int32_t* q_pos;
+    const int8_t* qi;
+    int32_t* scores;     // [B*Tq][sstride]
+    int64_t sstride;
+    int32_t* status;
+};
+
+template <int DI>
+struct __align__(1024) MqSmem {
+    uint8_t stage[kMqStages][kMqRows * DI];
+    uint8_t qb[kMqN * DI];               // the block's index queries as the B operand
+    uint64_t full_bar[kMqStages], empty_bar[kMqStages], tfull_bar[kMqBufs], tempty_bar[kMqBufs];
+    int tq[kMqQ];
+    int tile_lo, tile_hi;
+    uint32_t tmem_base;
+};
+
+__device__ __forceinline__ void tmem_ld16i(uint32_t taddr, int (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
+template <int DI>
+__global__ void __launch_bounds__(kMqThreads, 1)
+    index_mq_score_kernel(const __grid_constant__ MqParams p, const __grid_constant__ CUtensorMap kmap) {
+    static_assert(DI == 32 || DI == 64 || DI == 128, "tensor-core key widths");
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    MqSmem<DI>& S = *reinterpret_cast<MqSmem<DI>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    constexpr uint32_t kSwz = DI == 32 ? 6u : DI == 64 ? 4u : 2u;
+    constexpr uint32_t kSbo = 8 * DI;
+    constexpr uint32_t kIdesc = idesc_i8(128, kMqN);
+    constexpr int kEpiWarps = kMqGroups * 4;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int split = blockIdx.x % p.splits;
+    const int bq = blockIdx.x / p.splits;
+    const int b = bq / p.nblk, j0 = (bq % p.nblk) * kMqQ;
+    const int nq = min(kMqQ, p.Tq - j0);
+
+    if (warp == 0) tmem_alloc(&S.tmem_base, kMqBufs * kMqN);
+    if (tid == 0) {
+        for (int i = 0; i < kMqStages; ++i) { mbar_init(&S.full_bar[i], 1); mbar_init(&S.empty_bar[i], 1); }
+        for (int i = 0; i < kMqBufs; ++i) { mbar_init(&S.tfull_bar[i], 1); mbar_init(&S.tempty_bar[i], 4); }
+        mbar_fence_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch_dependents();
+    pdl_wait();   // positions and index queries may come from the previous kernel
+
+    if (tid < kMqQ) {
+        int t = -1;
+        if (tid < nq) {
+            t = p.q_pos[(size_t)b * p.Tq + j0 + tid];
+            if (t < 0 || t >= p.N) t = -1;   // no scores; the select kernel reports the position
+        }
+        S.tq[tid] = t;
+    }
+    fence_proxy_async_smem();
+    for (int i = tid; i < kMqN * (DI / 16); i += kMqThreads) {
+        const int r = i / (DI / 16), c2 = i % (DI / 16);
+        const int q = r >> 3, h = r & 7;
+        int4 v = make_int4(0, 0, 0, 0);
+        if (q < nq && h < p.Hi)
+            v = reinterpret_cast<const int4*>(p.qi + (((size_t)b * p.Tq + j0 + q) * p.Hi + h) * DI)[c2];
+        *reinterpret_cast<int4*>(S.qb + tile_off(r, c2, DI)) = v;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {   // this split's share of the tiles that cover [0, the block's last position]
+        int tmax = -1;
+        for (int q = 0; q < kMqQ; ++q) tmax = max(tmax, S.tq[q]);
+        const int ntile = (tmax + kMqRows) / kMqRows;
+        S.tile_lo = (int)((long long)ntile * split / p.splits);
+        S.tile_hi = (int)((long long)ntile * (split + 1) / p.splits);
+    }
+    __syncthreads();
+    const int tile_lo = S.tile_lo, nt = S.tile_hi - S.tile_lo;
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == kEpiWarps) {
+        if (lane == 0) {   // TMA producer
+            const uint64_t pol = l2_evict_first_policy();
+            for (int i = 0; i < nt; ++i) {
+                const int slot = i % kMqStages;
+                if (i >= kMqStages && !mbar_wait(&S.empty_bar[slot], ((i / kMqStages) - 1) & 1u, p.status, 21)) break;
+                mbar_arrive_expect_tx(&S.full_bar[slot], (uint32_t)(kMqRows * DI));
+                tma_load_keys(S.stage[slot], &kmap, 0, (tile_lo + i) * kMqRows, b, &S.full_bar[slot], pol);
+            }
+        }
+    } else if (warp == kEpiWarps + 1) {
+        if (lane == 0) {   // MMA issuer
+            const uint32_t b0 = smem_u32(S.qb);
+            for (int i = 0; i < nt; ++i) {
+                const int slot = i % kMqStages, buf = i % kMqBufs;
+                if (!mbar_wait(&S.full_bar[slot], (i / kMqStages) & 1u, p.status, 22)) break;
+                if (i >= kMqBufs && !mbar_wait(&S.tempty_bar[buf], ((i / kMqBufs) - 1) & 1u, p.status, 23)) break;
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(S.stage[slot]);
+#pragma unroll
+                for (int kk = 0; kk < DI / 32; ++kk)
+                    mma_i8(tmem + (uint32_t)(buf * kMqN), smem_desc(a0 + kk * 32, 16, kSbo, kSwz),
+                           smem_desc(b0 + kk * 32, 16, kSbo, kSwz), kIdesc, kk > 0 ? 1u : 0u);
+                mma_commit(&S.empty_bar[slot]);
+                mma_commit(&S.tfull_bar[buf]);
+            }
+        }
+    } else {
+        // epilogue: group g takes tiles g, g + 4, ...; warp wl of a group reads TMEM lane
+        // quarter wl, i.e. key rows 32 wl .. 32 wl + 31 of the tile
+        const int g = warp >> 2, wl = warp & 3;
+        int tq[kMqQ], w[8];
+#pragma unroll
+        for (int q = 0; q < kMqQ; ++q) tq[q] = S.tq[q];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) w[h] = p.w[h];
+        for (int i = g; i < nt; i += kMqGroups) {
+            const int buf = i % kMqBufs;
+            const bool got = mbar_wait(&S.tfull_bar[buf], (i / kMqBufs) & 1u, p.status, 24);
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            int x[kMqQ];
+            const uint32_t ta = tmem + (uint32_t)(buf * kMqN) + ((uint32_t)(wl * 32) << 16);
+#pragma unroll
+            for (int q2 = 0; q2 < kMqQ / 2; ++q2) {
+                int acc[16];
+                tmem_ld16i(ta + (uint32_t)(q2 * 16), acc);
+                tmem_ld_wait();
+                int xa = 0, xb = 0;
+#pragma unroll
+                for (int h = 0; h < 8; ++h) {
+                    xa += w[h] * max(acc[h], 0);
+                    xb += w[h] * max(acc[8 + h], 0);
+                }
+                x[2 * q2] = xa;
+                x[2 * q2 + 1] = xb;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.tempty_bar[buf]);
+            const int s = (tile_lo + i) * kMqRows + wl * 32 + lane;
+#pragma unroll
+            for (int q = 0; q < kMqQ; ++q)
+                if (s <= tq[q]) p.scores[((size_t)b * p.Tq + j0 + q) * p.sstride + s] = x[q];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kMqBufs * kMqN);
 }
 
 // ------------------------------------------------------------ Reindex, and Full for other key widths
@@ -1800,6 +2035,8 @@ static EncodeTiledFn get_encode_fn() {
 struct IdxPlan {
     int units, G, groups, chunk;
     int local_sel, rstride;
+    int mq;              // Full with queries sharing keys: multi-query scoring, then select only
+    int64_t pstride;     // per-unit stride of the scores it writes
     size_t spill_bytes;
 };
 
@@ -1858,6 +2095,12 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
     pl.local_sel = (a.mode == CSA2_REINDEX && pl.G > 1 && a.P_in <= kSmemScores) ? 1 : 0;
     pl.rstride = (int)align_up((size_t)std::max(a.P_in, 1), 4);
     if (pl.local_sel) pl.spill_bytes = std::max(pl.spill_bytes, align_up((size_t)pl.units * pl.rstride * 4, 256));
+    // (below kMqMinN keys the second launch costs more than the shared tiles save)
+    pl.mq = (a.mode == CSA2_FULL && a.Tq >= kMqMin && a.N >= kMqMinN && a.Hi <= 8 &&
+             (a.Di == 32 || a.Di == 64 || a.Di == 128)) ? 1 : 0;
+    pl.pstride = (int64_t)align_up((size_t)a.N, 4);
+    // (replaces the spill; the select's paired loads may read one element past a unit's last score)
+    if (pl.mq) pl.spill_bytes = align_up((size_t)pl.units * (size_t)pl.pstride * 4 + 64, 256);
     return pl;
 }
 
@@ -1897,6 +2140,26 @@ static cudaError_t launch_coop(Kern kern, int threads, const IdxParams& p, const
     return e;
 }
 
+template <int DI>
+static cudaError_t launch_mq(const MqParams& mp, const CUtensorMap& map, int grid, cudaStream_t stream) {
+    auto kern = index_mq_score_kernel<DI>;
+    // at least 116 KB, so that one CTA (and its 512 TMEM columns) holds an SM
+    const size_t smem = std::max(sizeof(MqSmem<DI>) + 1024, (size_t)116 * 1024);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kMqThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mp, map);
+}
+
 // Launch one indexer call. `ws` holds plan_index(a).ws_bytes bytes (zero at first use).
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
                          int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready) {
@@ -1923,7 +2186,9 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
     p.gl = reinterpret_cast<int*>(base + rg.off_gl);
     p.cand = reinterpret_cast<int2*>(base + rg.off_cand);
     p.pub = reinterpret_cast<int*>(base + rg.off_pub);
-    p.spill = (pl.chunk > kSmemScores) ? static_cast<int32_t*>(scratch) : nullptr;
+    p.spill = (pl.chunk > kSmemScores && !pl.mq) ? static_cast<int32_t*>(scratch) : nullptr;
+    p.pre = pl.mq ? static_cast<int32_t*>(scratch) : nullptr;
+    p.pstride = pl.pstride;
     p.local_sel = pl.local_sel;
     p.rstride = pl.rstride;
     p.rscore = pl.local_sel ? static_cast<int32_t*>(scratch) : nullptr;
@@ -1958,6 +2223,40 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
     }
     const int grid = pl.groups * pl.G;
     cudaError_t e;
+    if (pl.mq) {
+        // scores of every query first (key tiles shared by blocks of kMqQ queries)
+        EncodeTiledFn enc = get_encode_fn();
+        if (!enc) return CSA2_ERR_CUDA;
+        CUtensorMap mmap;
+        memset(&mmap, 0, sizeof(mmap));
+        cuuint64_t dims[3] = {(cuuint64_t)a.Di, (cuuint64_t)a.N, (cuuint64_t)a.B};
+        cuuint64_t strides[2] = {(cuuint64_t)a.Di, (cuuint64_t)a.ki_seq_stride};
+        cuuint32_t box[3] = {(cuuint32_t)a.Di, (cuuint32_t)kMqRows, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        CUtensorMapSwizzle swz = a.Di == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                 : a.Di == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_128B;
+        CUresult r = enc(&mmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(a.ki), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return CSA2_ERR_CUDA;
+        MqParams mp{};
+        mp.B = a.B; mp.Tq = a.Tq; mp.N = a.N; mp.Hi = a.Hi;
+        mp.nblk = (a.Tq + kMqQ - 1) / kMqQ;
+        const int items = a.B * mp.nblk;
+        // split each block's tiles so that the grid covers the SMs, at least 8 tiles a split
+        mp.splits = std::max(1, std::min(sms / std::max(items, 1), (a.N / kMqRows + 7) / 8));
+        for (int h = 0; h < 8; ++h) mp.w[h] = h < a.Hi ? a.w[h] : 0;
+        mp.q_pos = a.q_pos; mp.qi = a.qi;
+        mp.scores = static_cast<int32_t*>(scratch);
+        mp.sstride = pl.pstride;
+        mp.status = d_status;
+        const int mgrid = items * mp.splits;
+        e = a.Di == 64 ? launch_mq<64>(mp, mmap, mgrid, stream)
+            : a.Di == 32 ? launch_mq<32>(mp, mmap, mgrid, stream)
+                         : launch_mq<128>(mp, mmap, mgrid, stream);
+        if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    }
     if (a.mode == CSA2_FULL && a.Di == 64) e = launch_coop(index_full_tc_kernel<64>, kTcThreads, p, map, grid, stream);
     else if (a.mode == CSA2_FULL && a.Di == 32) e = launch_coop(index_full_tc_kernel<32>, kTcThreads, p, map, grid, stream);
     else if (a.mode == CSA2_FULL && a.Di == 128) e = launch_coop(index_full_tc_kernel<128>, kTcThreads, p, map, grid, stream);

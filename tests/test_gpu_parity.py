@@ -90,6 +90,25 @@ def test_index_full_shapes(B, N, Tq, k, P, ws, status):
     _check_full(qi, w, ki, q_pos, k, P, ws, status)
 
 
+@pytest.mark.parametrize("B,N,Tq,Hi,Di,k,P", [
+    (2, 9000, 20, 8, 64, 300, 1000),     # blocks of 16 + 4 queries, positions spread over the second half
+    (1, 8192, 5, 6, 128, 100, 0),        # 128-byte keys, 6 heads
+    (3, 20000, 40, 8, 64, 2048, 8192),   # scores past 16384 per CTA
+    (1, 12000, 16, 4, 32, 256, 512),     # 32-byte keys, 4 heads
+])
+def test_index_full_shared_keys(B, N, Tq, Hi, Di, k, P, ws, status):
+    """Tq >= 4 queries per sequence: the multi-query scoring kernel scores blocks of
+    queries against shared key tiles, and the Full kernel cuts in its select-only mode."""
+    qi = synth.randint_i8(3, 10 + Tq, (B, Tq, Hi, Di))
+    ki = synth.randint_i8(3, 20 + N, (B, N, Di))
+    w = synth.randint_i32(3, 30, (Hi,), 1, 8)
+    rng = np.random.default_rng(N + Tq)
+    q_pos = np.sort(rng.integers(N // 2, N, size=(B, Tq)), axis=1).astype(np.int32)
+    q_pos[:, -1] = N - 1
+    q_pos[0, 0] = min(q_pos[0, 0], 5)        # a query with fewer positions than k
+    _check_full(qi, w, ki, q_pos, k, P, ws, status)
+
+
 def test_index_full_early_positions_and_padding(ws, status):
     B, N = 2, 4096
     qi = synth.randint_i8(2, 1, (B, 6, 8, 64))
