@@ -103,3 +103,18 @@ def test_stack_mode_order():
     ia0.P = 0
     idx = (capi.IndexArgs * 2)(ia0, ri)          # REINDEX without a pool
     assert capi.csa2_layer_stack(capi.StackArgs(2, idx, att), 0, 0, 0, 0) == 4
+
+
+def test_index_workspace_holds_shared_key_scores():
+    """A Full call with at least 4 queries per sequence on a key set of at least 8192
+    positions scores its queries in blocks first, so its workspace also holds every
+    query's scores (B*Tq*N int32, plus slack, rounded to 256 bytes); smaller calls
+    score one query per unit and need none."""
+    def ws(Tq, N):
+        a, _w = _index_args(Tq=Tq, N=N, ki_seq_stride=N * 64)
+        return capi.csa2_workspace_bytes(0, a)
+    base = ws(1, 8192)
+    for Tq, N in [(64, 1 << 20), (64, 8192), (4, 8192)]:
+        assert ws(Tq, N) - base == (Tq * N * 4 + 64 + 255) // 256 * 256
+    assert ws(64, 4096) == base      # below 8192 keys
+    assert ws(3, 8192) == base       # fewer than 4 queries
