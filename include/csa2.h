@@ -148,7 +148,10 @@ typedef struct {
 
 /* Workspace bytes a call with these arguments needs. which: 0 = csa2_index_topk
  * (args = csa2_index_args*), 1 = csa2_sparse_attn (csa2_attn_args*),
- * 2 = csa2_layer_stack (csa2_stack_args*). Returns 0 for invalid arguments. */
+ * 2 = csa2_layer_stack (csa2_stack_args*). Returns 0 for invalid arguments.
+ * A Full call whose sequences carry Tq >= 4 queries over N >= 8192 positions
+ * (Hi <= 8, Di in {32, 64, 128}) scores its queries in blocks that share key
+ * tiles before it selects; its workspace then also holds B*Tq*N int32 scores. */
 size_t csa2_workspace_bytes(int which, const void* args);
 
 /* Full- or Reindex-mode top-k (and pool) selection ([CED] Fig. 4, Fig. 5). */
