@@ -672,30 +672,43 @@ __device__ __forceinline__ void gather_lists2(const int* sc, int n, int lo0, int
     const int nstep = (n + 63) >> 6;
     const int spw = (nstep + kSelWarps - 1) / kSelWarps;
     const int s0 = min(nstep, wp * spw), s1 = min(nstep, s0 + spw);
-#pragma unroll 4
-    for (int st = s0; st < s1; ++st) {
-        const int e = st * 64 + 2 * lane;
-        int2 x2;
-        if constexpr (kSpill) x2 = __ldcg(reinterpret_cast<const int2*>(sc + e));
-        else x2 = *reinterpret_cast<const int2*>(sc + e);
-        unsigned f[2];
+    // four steps' loads are issued before any of their list stores (which the compiler
+    // cannot tell apart from the scores, so it would not move a later load above them)
+#pragma unroll 1
+    for (int st0 = s0; st0 < s1; st0 += 4) {
+        int2 xv[4];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int x = q == 0 ? x2.x : x2.y;
-            const bool ok = e + q < n;
-            const bool a0 = ok && on0 && x > hi0, m0 = ok && x >= lo0 && x <= hi0;
-            const bool a1 = ok && on1 && x > hi1, m1 = ok && x >= lo1 && x <= hi1;
-            f[q] = (a0 ? 1u : 0u) | (m0 ? 2u : 0u) | (a1 ? 4u : 0u) | (m1 ? 8u : 0u);
-            na0 += a0;
-            na1 += a1;
+        for (int u4 = 0; u4 < 4; ++u4) {
+            const int e = (st0 + u4) * 64 + 2 * lane;
+            xv[u4] = make_int2(0, 0);
+            if (st0 + u4 < s1) {
+                if constexpr (kSpill) xv[u4] = __ldcg(reinterpret_cast<const int2*>(sc + e));
+                else xv[u4] = *reinterpret_cast<const int2*>(sc + e);
+            }
         }
-        const unsigned k0 = __ballot_sync(0xffffffffu, f[0] != 0u), k1 = __ballot_sync(0xffffffffu, f[1] != 0u);
-        if ((k0 | k1) == 0u) continue;
-        const int at = ln + __popc(k0 & below) + __popc(k1 & below);
-        if (f[0] != 0u && at < kListCap) list[at] = e | (int)(f[0] << 28);
-        const int at1 = at + (f[0] != 0u ? 1 : 0);
-        if (f[1] != 0u && at1 < kListCap) list[at1] = (e + 1) | (int)(f[1] << 28);
-        ln += __popc(k0) + __popc(k1);
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+            if (st0 + u4 >= s1) break;   // warp-uniform
+            const int e = (st0 + u4) * 64 + 2 * lane;
+            unsigned f[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int x = q == 0 ? xv[u4].x : xv[u4].y;
+                const bool ok = e + q < n;
+                const bool a0 = ok && on0 && x > hi0, m0 = ok && x >= lo0 && x <= hi0;
+                const bool a1 = ok && on1 && x > hi1, m1 = ok && x >= lo1 && x <= hi1;
+                f[q] = (a0 ? 1u : 0u) | (m0 ? 2u : 0u) | (a1 ? 4u : 0u) | (m1 ? 8u : 0u);
+                na0 += a0;
+                na1 += a1;
+            }
+            const unsigned k0 = __ballot_sync(0xffffffffu, f[0] != 0u), k1 = __ballot_sync(0xffffffffu, f[1] != 0u);
+            if ((k0 | k1) == 0u) continue;
+            const int at = ln + __popc(k0 & below) + __popc(k1 & below);
+            if (f[0] != 0u && at < kListCap) list[at] = e | (int)(f[0] << 28);
+            const int at1 = at + (f[0] != 0u ? 1 : 0);
+            if (f[1] != 0u && at1 < kListCap) list[at1] = (e + 1) | (int)(f[1] << 28);
+            ln += __popc(k0) + __popc(k1);
+        }
     }
     if (above != nullptr) {   // this CTA's elements above each interval (above[] zeroed by the caller)
         na0 = __reduce_add_sync(0xffffffffu, na0);
@@ -2090,7 +2103,8 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
     chunk = (int)align_up((size_t)std::max(chunk, 1), 256);
     pl.chunk = chunk;
     pl.spill_bytes = 0;
-    if (chunk > kSmemScores) pl.spill_bytes = align_up((size_t)pl.groups * pl.G * chunk * 4, 256);
+    // (+ 512 bytes: the select's 64-element steps may read up to 63 elements past a chunk's end)
+    if (chunk > kSmemScores) pl.spill_bytes = align_up((size_t)pl.groups * pl.G * chunk * 4 + 512, 256);
     // Reindex with a pool that fits one CTA: published scores, one select per group
     pl.local_sel = (a.mode == CSA2_REINDEX && pl.G > 1 && a.P_in <= kSmemScores) ? 1 : 0;
     pl.rstride = (int)align_up((size_t)std::max(a.P_in, 1), 4);
@@ -2099,8 +2113,8 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
     pl.mq = (a.mode == CSA2_FULL && a.Tq >= kMqMin && a.N >= kMqMinN && a.Hi <= 8 &&
              (a.Di == 32 || a.Di == 64 || a.Di == 128)) ? 1 : 0;
     pl.pstride = (int64_t)align_up((size_t)a.N, 4);
-    // (replaces the spill; the select's paired loads may read one element past a unit's last score)
-    if (pl.mq) pl.spill_bytes = align_up((size_t)pl.units * (size_t)pl.pstride * 4 + 64, 256);
+    // (replaces the spill; the select's 64-element steps may read up to 63 elements past a unit's last score)
+    if (pl.mq) pl.spill_bytes = align_up((size_t)pl.units * (size_t)pl.pstride * 4 + 512, 256);
     return pl;
 }
 

@@ -115,6 +115,6 @@ def test_index_workspace_holds_shared_key_scores():
         return capi.csa2_workspace_bytes(0, a)
     base = ws(1, 8192)
     for Tq, N in [(64, 1 << 20), (64, 8192), (4, 8192)]:
-        assert ws(Tq, N) - base == (Tq * N * 4 + 64 + 255) // 256 * 256
+        assert ws(Tq, N) - base == (Tq * N * 4 + 512 + 255) // 256 * 256
     assert ws(64, 4096) == base      # below 8192 keys
     assert ws(3, 8192) == base       # fewer than 4 queries
