@@ -1014,7 +1014,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
     const bool full = p.mode == CSA2_FULL;
     const int lo = c.lo, my_n = c.my_n;
 
-    // ---- round 0: histogram of level 0; zero the buffers the next steps use
+    // ---- step 0: histogram of level 0; zero the buffers the next steps use
     int* g0cur = sl.g0 + ((c.epoch + c.j) % 3) * kG0Stride;
     int* g0nxt = sl.g0 + ((c.epoch + c.j + 1) % 3) * kG0Stride;
     push_hist(S.hist0, g0cur);
