@@ -73,3 +73,11 @@ def test_schedule_labels():
     assert label("paper_schedule") == "F,U,U,U," + "RI,U,U,U," * 3 + "RI,U,U,U"
     assert label("long_1m") == "F," + "RI,U," * 9 + "RI"
     assert label("decode_full") == "F"
+
+
+def test_launch_count():
+    count = lambda w: bench.launches_per_step(synth.make_workload(w).spec)
+    assert count("stack20_128k") == 10 + 20          # 5 Full + 5 Reindex indexers, 20 attention launches
+    assert count("long_1m") == 2 + 10 + 20           # the Full layer of 64 queries is scored first
+    assert count("prefill_chunk") == 2 + 1
+    assert count("tiny") == 1 + 1                    # 2048 keys: one indexer launch
