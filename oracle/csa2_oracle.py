@@ -271,13 +271,6 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def bf16_round(x: np.ndarray) -> np.ndarray:
-    """Nearest-even bf16 value of fp64 inputs, as fp64 (for output comparison only)."""
-    f = np.asarray(x, dtype=np.float64).astype(np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << 16
-    return u.astype(np.uint32).view(np.float32).astype(np.float64)
-
 
 # --------------------------------------------------------------------------
 # Layer stack over one shared cache   [CED] "What Full, Reindex, and Reuse Share"

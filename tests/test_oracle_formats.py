@@ -148,3 +148,17 @@ def test_fp4_bytes_per_token():
     x = synth.normal_f32(0, 13, (3, 128))
     c, s = O.fp4_quantize(x)
     assert c.shape[-1] + s.shape[-1] == 72
+
+
+def test_bf16_to_f64_every_pattern():
+    """The oracle's bf16 decoding against torch's bfloat16 -> float64 conversion, for all
+    65536 bit patterns (NaN patterns decode to NaN on both sides)."""
+    import torch
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):      # signalling-NaN patterns
+        ours = O.bf16_to_f64(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))   # -0 stays -0
