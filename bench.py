@@ -405,7 +405,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": metric_of(s),
         "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8+bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8+f16+bf16", "data": "synthetic",
         "config": {**workload_config(s, units), "parallelism": f"replicas x{world}",
                    "l2": "flushed (256 MB write) before every timed step, outside its events",
                    "launch": "CUDA graph of one csa2_layer_stack call" if graph is not None else "eager"},
