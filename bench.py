@@ -336,55 +336,29 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = total_ms / K
     n_launch = launches_per_step(s)
 
-    # dominant kernel: the Full-mode indexer of layer 0, alone, same stream, L2 flushed
-    d0 = layers[0]
-    import numpy as _np
-    w_host = _np.ascontiguousarray(_np.asarray(d0["w"], dtype=_np.int32))
-    pool_t = torch.empty((s.B, s.Tq, s.layers[0].P), dtype=torch.int32, device="cuda")
-    topk_t = torch.empty((s.B, s.Tq, s.layers[0].k), dtype=torch.int32, device="cuda")
-    ia = ops.make_index_args(capi.CSA2_FULL, q_pos, d0["qi"], w_host, d0["ki"], s.layers[0].k, s.layers[0].P,
-                             None, pool_t, topk_t)
-    ibuf = ws.get(max(stack.ws_bytes, capi.csa2_workspace_bytes(0, ia)))
-
-    def kcall(stream_ptr):
-        return capi.csa2_index_topk(ia, int(ibuf.data_ptr()), ibuf.numel(), st.ptr, stream_ptr)
-
-    kgraph = None if args.eager else capture_graph(torch, kcall)
-    kl_ms = []
-    for i in range(args.kernel_launches + 3):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        if kgraph is not None:
-            kgraph.replay()
-        else:
-            capi.check(kcall(sptr), "kernel timing")
-        b.record(stream)
-        if i >= 3:
-            kl_ms.append((a, b))
-    torch.cuda.synchronize()
-    st.check("kernel timing")
-    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kl_ms)
+    # every kernel class of the step, each alone on the same stream with L2 flushed;
+    # the roofline names the class with the largest share of the step
     qp_host = q_pos.cpu().numpy()
-    kbytes = full_launch_bytes(s, qp_host)
+    base_host = base.cpu().numpy()
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
     except Exception:  # noqa: BLE001
         pass
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
-    achieved = kbytes / (kern_ms * 1e-3) / 1e9
-    traffic = None
+    kernels = kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales, base, qp_host, base_host,
+                               ws, st, flush, stream, hbm_peak)
+    traffic_db = {}
     try:
-        prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-        traffic = prof.get(args.workload, {}).get("index_full_bytes_per_launch")
+        traffic_db = json.load(open(os.path.join(ROOT, "profiles", "traffic.json"))).get(args.workload, {})
     except Exception:  # noqa: BLE001
         pass
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                "kernel": (f"index_full_tc_kernel<{s.Di}>" if s.Di in (32, 64, 128) else "index_dp4a_kernel")
-                + " (Full mode, layer 0: scan + exact pool/top-k select)",
-                "kernel_ms": round(kern_ms, 4), "algorithmic_bytes": kbytes,
+    for kc in kernels:
+        kc["traffic"] = traffic_db.get(kc["class"], {}).get("bytes_per_launch")
+    top = max(kernels, key=lambda kc: kc["share"])
+    roofline = {"bound": "hbm", "achieved": top["gbs"], "peak": hbm_peak, "unit": "GB/s", "frac": top["frac"],
+                "traffic": top["traffic"], "kernel": top["kernel"], "class": top["class"],
+                "kernel_ms": top["ms"], "algorithmic_bytes": top["algorithmic_bytes"], "share": top["share"],
                 "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback 6650 GB/s"}
     # the lists of the last timed step (the same inputs every step)
     host = lambda ts: [t.cpu().numpy() if t is not None else None for t in ts]
@@ -411,7 +385,7 @@ def run_ours(args, rank, world, local_rank):
                    "launch": "CUDA graph of one csa2_layer_stack call" if graph is not None else "eager"},
         "step_hbm_gbs": round(step_gbs, 1), "step_frac_of_peak": round(step_gbs / hbm_peak, 4),
         "algorithmic_bytes_per_step": step_bytes,
-        "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
+        "roofline": roofline, "kernels": kernels, "e2e": e2e, "cpu_baseline": cpu,
         "gpu_launches": n_launch * K, "clocks": clk,
     }
     if rank == 0:
@@ -419,6 +393,127 @@ def run_ours(args, rank, world, local_rank):
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def time_alone(args, torch, fn, flush, stream, n):
+    """Mean device time (ms) of fn(stream_ptr) over n calls, each after an L2 flush,
+    timed with CUDA events on `stream` (a CUDA graph of one call unless --eager)."""
+    g = None if args.eager else capture_graph(torch, fn)
+    sptr = int(stream.cuda_stream)
+    evs = []
+    for i in range(n + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        if g is not None:
+            g.replay()
+        else:
+            rc = fn(sptr)
+            if rc:
+                raise RuntimeError(f"kernel timing call failed: {rc}")
+        b.record(stream)
+        if i >= 3:
+            evs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def unique_rows(lists):
+    """Distinct valid entries per sequence of a [B, Tq, n] list array, summed over sequences."""
+    import numpy as np
+    return sum(len(np.unique(l[l >= 0])) for l in lists)
+
+
+def attn_call_bytes(spec, q_pos, local_base, topk):
+    """Algorithmic bytes of one attention call: FP4 rows of the union of each sequence's
+    lists, local K+V rows of the union of its windows, and per query its query, list
+    and output."""
+    import numpy as np
+    D, Hq, W, B, Tq = spec.D, spec.Hq, spec.W, spec.B, spec.Tq
+    total = unique_rows(topk) * (D // 2 + D // 16)
+    if W > 0:
+        for b in range(B):
+            t = q_pos[b].astype(np.int64)
+            lo = np.maximum(np.maximum(t - W + 1, int(local_base[b])), 0)
+            total += _window_rows(lo, t) * 2 * D * 2
+    return total + B * Tq * (topk.shape[-1] * 4 + 2 * Hq * D * 2)
+
+
+def reindex_call_bytes(spec, pool, k):
+    """Algorithmic bytes of one Reindex call: the key rows of each sequence's pool
+    union, and per query its pool, index query and list."""
+    return unique_rows(pool) * spec.Di + spec.B * spec.Tq * (pool.shape[-1] * 4 + spec.Hi * spec.Di + k * 4)
+
+
+def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales, base, qp_host, base_host, ws, st,
+                     flush, stream, hbm_peak):
+    """Each kernel class of one step, timed alone through the public calls on the
+    step's own tensors: the Full-mode indexer, the Reindex indexer, and attention for
+    a Full, a Reuse and a Reindex layer. Per class: ms per launch, launches per step,
+    share of the serial sum, algorithmic bytes per launch and GB/s against peak."""
+    modes = [L.mode for L in s.layers]
+    n_launch = {"FULL": modes.count("FULL"), "REINDEX": modes.count("REINDEX"), "REUSE": modes.count("REUSE")}
+    li_f = modes.index("FULL")
+    Lf = s.layers[li_f]
+    d0 = layers[li_f]
+    n = args.kernel_launches
+    out = []
+
+    def entry(cls, kernel, ms, count, nbytes):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.append({"class": cls, "kernel": kernel, "ms": round(ms, 5), "launches_per_step": count,
+                    "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)})
+
+    w_host = np.ascontiguousarray(np.asarray(d0["w"], dtype=np.int32))
+    pool_t = torch.empty((s.B, s.Tq, max(Lf.P, 1)), dtype=torch.int32, device="cuda")
+    topk_t = torch.empty((s.B, s.Tq, Lf.k), dtype=torch.int32, device="cuda")
+    ia = ops.make_index_args(capi.CSA2_FULL, q_pos, d0["qi"], w_host, d0["ki"], Lf.k, Lf.P, None,
+                             pool_t if Lf.P else None, topk_t)
+    buf = ws.get(capi.csa2_workspace_bytes(0, ia))
+    fcall = lambda sp: capi.csa2_index_topk(ia, int(buf.data_ptr()), buf.numel(), st.ptr, sp)
+    ms = time_alone(args, torch, fcall, flush, stream, n)
+    st.check("Full indexer timing")
+    mq = s.Tq >= 4 and s.N >= 8192 and s.Hi <= 8 and s.Di in (32, 64, 128)
+    kname = (f"index_full_tc_kernel<{s.Di}>" if s.Di in (32, 64, 128) else "index_dp4a_kernel<0,0>")
+    if mq:
+        kname = f"index_mq_score_kernel<{s.Di}> + {kname} (select only)"
+    entry("full_index", kname, ms, n_launch["FULL"], full_launch_bytes(s, qp_host))
+    topk_h = topk_t.cpu().numpy()
+
+    def attn_entry(cls, li, topk_dev, topk_host, count):
+        d = layers[li]
+        o = torch.empty_like(d["q"])
+        lse = torch.empty(d["q"].shape[:-1], dtype=torch.float32, device="cuda")
+        aa = ops.make_attn_args(q_pos, d["q"], codes, scales, topk_dev, d["kl"], d["vl"], base, s.W, o, lse)
+        abuf = ws.get(capi.csa2_workspace_bytes(1, aa))
+        acall = lambda sp: capi.csa2_sparse_attn(aa, int(abuf.data_ptr()), abuf.numel(), st.ptr, sp)
+        t = time_alone(args, torch, acall, flush, stream, n)
+        st.check(f"attention timing ({cls})")
+        HQP = 16 if s.Hq <= 16 else 32
+        entry(cls, f"sparse_attn_cl_kernel<{HQP},{s.D}>", t, count, attn_call_bytes(s, qp_host, base_host, topk_host))
+
+    attn_entry("attn_full", li_f, topk_t, topk_h, n_launch["FULL"])
+    if n_launch["REUSE"]:
+        attn_entry("attn_reuse", modes.index("REUSE"), topk_t, topk_h, n_launch["REUSE"])
+    if n_launch["REINDEX"]:
+        li_r = modes.index("REINDEX")
+        d = layers[li_r]
+        Lr = s.layers[li_r]
+        wr = np.ascontiguousarray(np.asarray(d["w"], dtype=np.int32))
+        topk_r = torch.empty((s.B, s.Tq, Lr.k), dtype=torch.int32, device="cuda")
+        ra = ops.make_index_args(capi.CSA2_REINDEX, q_pos, d["qi"], wr, d["ki"], Lr.k, 0, pool_t, None, topk_r)
+        rbuf = ws.get(capi.csa2_workspace_bytes(0, ra))
+        rcall = lambda sp: capi.csa2_index_topk(ra, int(rbuf.data_ptr()), rbuf.numel(), st.ptr, sp)
+        ms = time_alone(args, torch, rcall, flush, stream, n)
+        st.check("Reindex timing")
+        rk = ("index_dp4a_kernel<8,64>" if (s.Hi <= 8 and s.Di == 64) else
+              "index_dp4a_kernel<4,32>" if (s.Hi <= 4 and s.Di == 32) else "index_dp4a_kernel<0,0>")
+        entry("reindex_index", rk, ms, n_launch["REINDEX"], reindex_call_bytes(s, pool_t.cpu().numpy(), Lr.k))
+        attn_entry("attn_reindex", li_r, topk_r, topk_r.cpu().numpy(), n_launch["REINDEX"])
+    tot = sum(kc["ms"] * kc["launches_per_step"] for kc in out)
+    for kc in out:
+        kc["share"] = round(kc["ms"] * kc["launches_per_step"] / tot, 4) if tot > 0 else 0.0
+    return out
 
 
 def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st, graph, cache):
@@ -506,8 +601,8 @@ def cpu_baseline(workload: str, seconds: float):
         if time.perf_counter() - t0 >= seconds:
             break
     el = time.perf_counter() - t0
-    return {"value": round(done / el, 4), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{done} queries of sequence 0 through all {s.L} layers ({el:.1f} s)"}
+    return {"value": round(done / el, 4), "unit": UNIT, "cores": _blas_threads(), "host_cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"{done} queries of sequence 0 through all {s.L} layers ({el:.1f} s)"}
 
 
 def run_reference(args, rank, world):

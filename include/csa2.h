@@ -185,8 +185,24 @@ csa2_status csa2_fp4_quantize(const float* x, int64_t rows, int32_t D, uint8_t* 
  * tile and query). Calls needing more return CSA2_ERR_WORKSPACE and launch
  * nothing. The first call on a device looks up that array's address (make it
  * before any stream capture). Every call clears the tickets on `stream`; calls
- * that overlap on the GPU share the array and race. */
+ * that overlap on the GPU share the array and race. The looked-up address is
+ * kept for the life of the process: a device reset (cudaDeviceReset) after the
+ * first call on that device is not supported. */
 csa2_status csa2_sparse_attn_noalloc(const csa2_attn_args* args, int32_t* d_status, void* stream);
+
+/* Failure-detection controls, process-wide, read by every later indexer launch.
+ * The indexer's CTAs of one query meet at group barriers (spins on a counter in
+ * the workspace). A CTA that waits there longer than budget_cycles SM clock
+ * cycles writes CSA2_ERR_TIMEOUT to d_status and leaves; the others of its group
+ * leave as soon as they see that status (when d_status is not NULL), so the call
+ * ends after about one budget. budget_cycles = 0 restores the default (4e9
+ * cycles, about 2 s at the boost clock); a negative value returns CSA2_ERR_SHAPE.
+ * skip_arrival != 0 is host-side fault injection for tests and health checks:
+ * the last CTA of every group then leaves before its first group barrier, so the
+ * others' waits run out. Never set it in production. After a call that reported
+ * a timeout, zero the workspace before the next call.
+ * Waits on a CTA's own copies and tensor-core operations keep the fixed budget. */
+csa2_status csa2_set_wait_controls(int64_t budget_cycles, int32_t skip_arrival);
 
 /* Static text for a status code. */
 const char* csa2_status_string(csa2_status s);

@@ -50,7 +50,7 @@ class StackArgs(Structure):
 
 
 EXPORTED = ("csa2_workspace_bytes", "csa2_index_topk", "csa2_sparse_attn", "csa2_layer_stack",
-            "csa2_fp4_quantize", "csa2_status_string")
+            "csa2_fp4_quantize", "csa2_status_string", "csa2_set_wait_controls", "csa2_sparse_attn_noalloc")
 
 
 def library_path() -> str:
@@ -77,6 +77,8 @@ def lib():
                 f.restype = c_int
             L.csa2_fp4_quantize.argtypes = [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]
             L.csa2_fp4_quantize.restype = c_int
+            L.csa2_set_wait_controls.argtypes = [c_int64, c_int32]
+            L.csa2_set_wait_controls.restype = c_int
             L.csa2_status_string.argtypes = [c_int]
             L.csa2_status_string.restype = c_char_p
             _lib = L
@@ -101,6 +103,10 @@ def csa2_layer_stack(args: StackArgs, workspace: int, ws_bytes: int, d_status: i
 
 def csa2_fp4_quantize(x: int, rows: int, D: int, fp4: int, scale: int, stream: int) -> int:
     return lib().csa2_fp4_quantize(x, rows, D, fp4, scale, stream)
+
+
+def csa2_set_wait_controls(budget_cycles: int, skip_arrival: int) -> int:
+    return lib().csa2_set_wait_controls(budget_cycles, skip_arrival)
 
 
 def csa2_status_string(code: int) -> str:

@@ -35,6 +35,7 @@ csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* ticke
 bool attn_cluster_fits(const csa2_attn_args& a);
 csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
                                 cudaStream_t stream);
+void set_wait_controls(long long budget, int skip);
 // fp4_quant.cu
 cudaError_t launch_fp4_quantize(const float* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales,
                                 cudaStream_t stream);
@@ -263,6 +264,12 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
                                   : launch_attn(a, cur, tickets, scratch, d_status, strm);
         if (st != CSA2_OK) return st;
     }
+    return CSA2_OK;
+}
+
+csa2_status csa2_set_wait_controls(int64_t budget_cycles, int32_t skip_arrival) {
+    if (budget_cycles < 0) return CSA2_ERR_SHAPE;
+    set_wait_controls((long long)budget_cycles, skip_arrival);
     return CSA2_OK;
 }
 

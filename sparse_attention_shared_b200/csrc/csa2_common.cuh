@@ -1,7 +1,10 @@
 // Device helpers shared by the CSA2 kernels: status reporting, bounded waits,
 // mbarriers, bulk copies and the tcgen05 (5th-generation tensor core) wrappers.
-// Every wait here is bounded: it gives up after kSpinBudgetCycles SM cycles,
-// records CSA2_ERR_TIMEOUT in the status word and lets the caller return.
+// Every wait here is bounded: a wait on an mbarrier (a copy or an MMA of the
+// CTA itself) gives up after kSpinBudgetCycles SM cycles; a wait on other CTAs
+// (the indexer's group barrier) after a run-time budget that defaults to the
+// same and can be shortened by csa2_set_wait_controls. Either records
+// CSA2_ERR_TIMEOUT in the status word and lets the caller return.
 #pragma once
 
 #include <cstdint>
@@ -24,6 +27,12 @@ __device__ __forceinline__ void report(int32_t* st, int code, int detail) {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {

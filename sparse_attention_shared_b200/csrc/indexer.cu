@@ -15,11 +15,13 @@
 // more units than groups). Each CTA scores a contiguous chunk of the unit's
 // candidates into shared memory:
 //   * Full mode with 32/64/128-byte keys: warp-specialised tensor-core scan.
-//     A TMA warp streams 256-row key tiles into a 6-stage ring, an MMA warp
-//     issues tcgen05.mma kind::i8 (keys as M = 128 rows, the index query's
-//     heads as N = 16) into 4 TMEM buffers, and 8 epilogue warps apply the
-//     ReLU and head weights to the int32 accumulators. mbarriers link the
-//     roles, so the scan runs at the rate of its slowest role.
+//     A TMA warp streams key tiles of up to 256 rows into an 8-stage ring
+//     (kStages), an MMA warp issues tcgen05.mma kind::i8 (keys as M = 128
+//     rows, the index query's heads as N = 16) into 4 TMEM buffers, and 16
+//     epilogue warps (kSel threads, two groups of 8 warps that take alternate
+//     tiles) apply the ReLU and head weights to the int32 accumulators.
+//     mbarriers link the roles, so the scan runs at the rate of its slowest
+//     role.
 //   * Reindex mode and other key widths: rows are gathered (or TMA-staged)
 //     and scored with dp4a.
 // Then the group finds the exact cut with a distributed radix select on a
@@ -82,6 +84,8 @@ struct IdxParams {
     const uint8_t* pf_fp4;
     const uint8_t* pf_scale;
     int pf_N, pf_code_bytes, pf_scale_bytes;
+    long long wait_budget;   // SM cycles a CTA waits at a group barrier before it reports a timeout
+    int skip_arrival;        // fault injection: the last CTA of a group never arrives at its first barrier
     int* ctrl;           // [slots][kCtrlInts]
     int* g0;             // [slots][3][kG0Stride]: histogram, then the element count
     int* gl;             // [slots][2 tracks][2 levels][kBins]
@@ -262,21 +266,33 @@ __device__ __forceinline__ int sel_min(int v, int* red) {
 
 // Group barrier over the G CTAs of a slot: the counter grows by one per CTA.
 // The arrival is a release add (it publishes this CTA's earlier writes, which the
-// named barrier has ordered before it) and the poll an acquire load.
-__device__ bool group_barrier(int* counter, int target, int32_t* st) {
+// named barrier has ordered before it) and the poll an acquire load. The wait
+// ends with a failure after `budget` SM cycles (this CTA reports the timeout) or
+// as soon as the status word shows a timeout another CTA reported, so one
+// missing CTA costs the group one budget, not one per CTA. `skip` (fault
+// injection, set from the host) makes this CTA leave without arriving.
+__device__ bool group_barrier(int* counter, int target, int32_t* st, long long budget, bool skip = false) {
     sel_sync();
     int ok = 1;
     if (threadIdx.x == 0) {
-        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter) : "memory");
-        if (ld_acquire_gpu(counter) < target) {
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(counter) < target) {
-                if (clock64() - t0 > kSpinBudgetCycles) {
-                    report(st, CSA2_ERR_TIMEOUT, 1);
-                    ok = 0;
-                    break;
+        if (skip) {
+            ok = 0;
+        } else {
+            asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter) : "memory");
+            if (ld_acquire_gpu(counter) < target) {
+                const long long t0 = clock64();
+                while (ld_acquire_gpu(counter) < target) {
+                    if (st != nullptr && ld_relaxed_gpu(st) == CSA2_ERR_TIMEOUT) {
+                        ok = 0;
+                        break;
+                    }
+                    if (clock64() - t0 > budget) {
+                        report(st, CSA2_ERR_TIMEOUT, 1);
+                        ok = 0;
+                        break;
+                    }
+                    __nanosleep(20);
                 }
-                __nanosleep(20);
             }
         }
     }
@@ -1030,7 +1046,9 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         if (c.cta == 0 && tid == 0) { sl.ctrl[CTRL_CAND0] = 0; sl.ctrl[CTRL_CAND1] = 0; g0nxt[kBins] = 0; }
     }
     bar_target += p.G;
-    if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
+    if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status, p.wait_budget,
+                       p.skip_arrival && c.cta == p.G - 1))
+        return false;
 
     const int n_total = full ? c.n_all : min(max(__ldcg(g0cur + kBins), 0), p.P_in);
     Track tk[2];
@@ -1147,7 +1165,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         }
         if (!any) break;
         bar_target += p.G;
-        if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
+        if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status, p.wait_budget)) return false;
         bool pending = false;
 #pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
@@ -1298,7 +1316,9 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
     // every CTA waits: the leader's zeroing of the next unit's count (above) is then
     // ordered before any CTA's add for that unit
     bar_target += p.G;
-    if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status)) return false;
+    if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status, p.wait_budget,
+                       p.skip_arrival && c.cta == p.G - 1))
+        return false;
     if (c.cta != 0) return true;
 
     // the leader: all scores of the unit (valid pool entries form a prefix), as int4
@@ -2045,6 +2065,18 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
+// Failure-detection controls (csa2_set_wait_controls): process-wide, read at launch.
+static std::atomic<long long> g_wait_budget{kSpinBudgetCycles};
+static std::atomic<int> g_skip_arrival{0};
+
+long long group_wait_budget() { return g_wait_budget.load(); }
+int group_skip_arrival() { return g_skip_arrival.load(); }
+
+void set_wait_controls(long long budget, int skip) {
+    g_wait_budget.store(budget > 0 ? budget : kSpinBudgetCycles);
+    g_skip_arrival.store(skip ? 1 : 0);
+}
+
 struct IdxPlan {
     int units, G, groups, chunk;
     int local_sel, rstride;
@@ -2215,6 +2247,8 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
     }
     p.keys_ready = keys_ready;
     p.status = d_status;
+    p.wait_budget = group_wait_budget();
+    p.skip_arrival = group_skip_arrival();
 
     CUtensorMap map;
     memset(&map, 0, sizeof(map));

@@ -54,6 +54,19 @@ class DeviceWorkload:
         return out
 
 
+def assert_list_invariants(lists: np.ndarray, q_pos: np.ndarray, what: str):
+    """Every list [..., len] of a query at position t holds distinct positions in
+    [0, t], ascending, with -1 only as padding at the tail ([CED] Fig. 2: causal
+    access; the lists' order and padding are this library's layout)."""
+    g = np.asarray(lists)
+    t = np.asarray(q_pos).reshape(g.shape[:-1] + (1,))
+    valid = g >= 0
+    assert np.all(valid[..., 1:] <= valid[..., :-1]), f"{what}: -1 before a valid entry"
+    assert np.all(g[valid] <= np.broadcast_to(t, g.shape)[valid]), f"{what}: an entry past the query position"
+    inc = (g[..., 1:] > g[..., :-1]) | ~valid[..., 1:]
+    assert np.all(inc), f"{what}: entries not strictly ascending"
+
+
 def assert_lists_equal(gpu: torch.Tensor, ref: np.ndarray, what: str):
     g = gpu.cpu().numpy()
     if not np.array_equal(g, ref):

@@ -32,6 +32,11 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, name), name
 
 
+def test_wait_controls_validation():
+    assert capi.csa2_set_wait_controls(-1, 0) == 2      # CSA2_ERR_SHAPE
+    assert capi.csa2_set_wait_controls(0, 0) == 0       # the default budget, no injection
+
+
 def test_status_strings():
     for code in range(10):
         assert capi.csa2_status_string(code)

@@ -12,7 +12,8 @@ from oracle import csa2_oracle as O
 from oracle.workload import OracleCache, run_units
 from sparse_attention_shared_b200 import ops
 
-from gpu_util import DeviceWorkload, assert_attn_close, assert_lists_equal, bf16_dev, dev
+from gpu_util import (DeviceWorkload, assert_attn_close, assert_list_invariants, assert_lists_equal, bf16_dev,
+                      dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -66,8 +67,10 @@ def _oracle_full(qi, w, ki, q_pos, k, P):
 def _check_full(qi, w, ki, q_pos, k, P, ws, status):
     pool, topk = ops.index_topk("FULL", dev(q_pos), dev(qi), w, dev(ki), k, P, ws=ws, status=status)
     rpool, rtopk = _oracle_full(qi, w, ki, q_pos, k, P)
+    assert_list_invariants(topk.cpu().numpy(), q_pos, "topk")
     assert_lists_equal(topk, rtopk, "topk")
     if P:
+        assert_list_invariants(pool.cpu().numpy(), q_pos, "pool")
         assert_lists_equal(pool, rpool, "pool")
     return pool, topk
 

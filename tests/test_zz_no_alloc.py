@@ -61,6 +61,38 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert d_lse <= LSE_TOL, f"call {call}: lse differs by {d_lse}"
 
 
+def test_noalloc_against_the_oracle_without_window():
+    """Several queries per sequence and no local branch (W = 0), checked directly
+    against the fp64 oracle on two calls in a row."""
+    f = _noalloc()
+    stream = int(torch.cuda.current_stream().cuda_stream)
+    B, N, Tq, Hq, D, k = 2, 3000, 4, 16, 128, 300
+    for call, seed in enumerate((303, 404)):
+        kv = synth.normal_f32(seed, 1, (B, N, D))
+        codes, scales = O.fp4_quantize(kv)
+        q = synth.normal_bf16(seed, 2, (B, Tq, Hq, D))
+        q_pos = np.broadcast_to(np.arange(N - Tq, N, dtype=np.int32), (B, Tq)).copy()
+        rng = np.random.default_rng(seed)
+        topk = np.stack([[np.sort(rng.choice(int(t) + 1, k, replace=False)).astype(np.int32) for t in q_pos[b]]
+                         for b in range(B)])
+        gc, gs = ops.fp4_quantize(dev(kv.reshape(-1, D)))
+        out = torch.empty((B, Tq, Hq, D), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device="cuda")
+        a = ops.make_attn_args(dev(q_pos), bf16_dev(q), gc.view(B, N, D // 2), gs.view(B, N, D // 16), dev(topk),
+                               None, None, None, 0, out, lse)
+        st = ops.Status()
+        assert f(ctypes.byref(a), st.ptr, stream) == 0
+        st.check(f"noalloc call {call}")
+        o, l = out.float().cpu().numpy(), lse.cpu().numpy()
+        for b in range(B):
+            for j in range(Tq):
+                none = np.zeros((1, D))
+                ro, rl = O.attention_unit(O.bf16_to_f64(q[b, j]), codes[b], scales[b], topk[b, j], none, none, 0,
+                                          int(q_pos[b, j]), 0)
+                assert np.abs(o[b, j] - ro).max() <= OUT_TOL, f"call {call}, unit {(b, j)}: out"
+                assert np.abs(l[b, j] - rl).max() <= LSE_TOL, f"call {call}, unit {(b, j)}: lse"
+
+
 def test_noalloc_rejects_sizes_beyond_its_static_scratch():
     f = _noalloc()
     x = _inputs(7, B=2, N=4096)
