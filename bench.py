@@ -574,78 +574,91 @@ def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, 
 
 
 # ------------------------------------------------------------------ CPU oracle
-def _blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:  # noqa: BLE001
-        return 1
-
-
 def cpu_baseline(workload: str, seconds: float):
-    """The oracle, as it stands, on whole queries (all 20 layers) of the same workload
-    until `seconds` of CPU work have run (at least one query)."""
+    """The C++ oracle, as it stands, with std::threads over (sequence, query) units on
+    the host's cores: batches of every sequence's queries through all layers of the
+    workload (index and attention), until `seconds` have run (at least one batch).
+    Also a one-thread figure on one decode_full query (one Full layer)."""
     import synth
-    from oracle.workload import OracleCache, layer_inputs, run_units
-    from oracle import csa2_oracle as O
+    from oracle import cpp as C
 
     wl = synth.make_workload(workload)
     s = wl.spec
-    cache = OracleCache(wl)
-    cache.seq(0)                           # quantising the cache is setup, not a decode step
-    done, t0 = 0, time.perf_counter()
+    threads = C.host_threads()
+    codes, scales = C.fp4_quantize(wl.kv_f32())     # quantising the cache is setup, not a decode step
+    wl.drop("kv")
+    for li in range(s.L):                             # draw every input before the clock starts
+        wl.q(li), wl.kl(li), wl.vl(li)
+        if s.layers[li].mode != "REUSE":
+            wl.qi(li), wl.ki(s.layers[li].key_set)
+    done, batches, t0 = 0, 0, time.perf_counter()
     while True:
-        run_units(wl, [(0, done % s.Tq)], cache)
-        done += 1
+        st = C.StackState(wl)
+        for li in range(s.L):
+            C.run_layer(st, li, codes, scales, threads)
+        done += s.B * s.Tq
+        batches += 1
         if time.perf_counter() - t0 >= seconds:
             break
     el = time.perf_counter() - t0
-    return {"value": round(done / el, 4), "unit": UNIT, "cores": _blas_threads(), "host_cores": os.cpu_count(),
-            "kind": "oracle", "sample": f"{done} queries of sequence 0 through all {s.L} layers ({el:.1f} s)"}
+    # one thread, one decode_full query (B = 1): its Full layer's index and attention
+    w1 = synth.make_workload("decode_full", B=1)
+    c1, s1 = C.fp4_quantize(w1.kv_f32())
+    w1.q(0), w1.kl(0), w1.vl(0), w1.qi(0), w1.ki(0)
+    reps, t1 = 0, time.perf_counter()
+    while True:
+        C.run_layer(C.StackState(w1), 0, c1, s1, threads=1)
+        reps += 1
+        if time.perf_counter() - t1 >= 2.0:
+            break
+    el1 = time.perf_counter() - t1
+    return {"value": round(done / el, 4), "unit": UNIT, "cores": min(threads, s.B * s.Tq), "host_cores": threads,
+            "kind": "oracle",
+            "sample": f"{batches} batch(es) of all {s.B * s.Tq} queries through all {s.L} layers, index and attention "
+                      f"(C++ oracle, {min(threads, s.B * s.Tq)} threads, {el:.1f} s)",
+            "single_thread_decode_full_b1": {"value": round(reps / el1, 4), "unit": "queries/s", "cores": 1,
+                                             "sample": f"{reps} query(ies) of decode_full B=1, one Full layer "
+                                                       f"({el1:.1f} s)"}}
 
 
 def run_reference(args, rank, world):
-    """The oracle as the reference arm: each step is one layer of one query (cycling
-    through the schedule), reported as whole-stack queries/s."""
+    """The oracle as the reference arm: the C++ oracle on the host's cores, each step
+    one layer of the workload for every query (threads over the queries), cycling
+    through the layer schedule; reported as whole-stack queries/s."""
     if rank != 0:
         return
     import synth
-    from oracle import csa2_oracle as O
-    from oracle.workload import OracleCache, layer_inputs
+    from oracle import cpp as C
 
     wl = synth.make_workload(args.workload)
     s = wl.spec
-    cache = OracleCache(wl)
-    codes, scales = cache.seq(0)
-    layers = layer_inputs(wl, 0, 0)
-    t = int(wl.q_pos()[0, 0])
-    base = int(wl.local_base_arr()[0])
-    state = {"cur": None, "pool": None}
+    threads = C.host_threads()
+    codes, scales = C.fp4_quantize(wl.kv_f32())
+    wl.drop("kv")
+    state = {"st": C.StackState(wl)}
 
-    def layer_step(li):
-        L = layers[li]
-        if L["mode"] == "FULL":
-            pool, state["cur"] = O.index_full(L["qi"], L["w"], L["keys"], t, L["k"], L["P"])
-            if pool is not None:
-                state["pool"] = pool
-        elif L["mode"] == "REINDEX":
-            state["cur"] = O.index_reindex(L["qi"], L["w"], L["keys"], state["pool"], L["k"])
-        O.attention_unit(L["q"], codes, scales, state["cur"], L["kl"], L["vl"], base, t, L["W"])
+    def layer_step(i):
+        li = i % s.L
+        if li == 0:
+            state["st"] = C.StackState(wl)
+        C.run_layer(state["st"], li, codes, scales, threads)
 
     for i in range(args.warmup):
-        layer_step(i % s.L)
+        layer_step(i)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        layer_step((args.warmup + i) % s.L)
+        layer_step(args.warmup + i)
     el = time.perf_counter() - t0
-    value = args.steps / s.L / el
+    value = args.steps / s.L * s.B * s.Tq / el
+    cores = min(threads, s.B * s.Tq)
     res = {"metric": metric_of(s), "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64", "data": "synthetic", "impl": "reference",
            "config": {**workload_config(s, s.B * s.Tq), "parallelism": "CPU oracle on rank 0"},
-           "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-                            "sample": f"{args.steps} layer-steps of query (0,0), one layer per step"},
+           "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "host_cores": threads,
+                            "kind": "oracle",
+                            "sample": f"{args.steps} layer-steps, each one layer for all {s.B * s.Tq} queries "
+                                      f"(C++ oracle, {cores} threads)"},
            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 

@@ -146,6 +146,46 @@ typedef struct {
     const csa2_attn_args* attn;   /* HOST [L] */
 } csa2_stack_args;
 
+/*
+ * One decode step's cache update for B sequences ([CED] "Why Prefill Recomputes
+ * a Recent Segment", closing paragraph: after each output, the new token's
+ * global KV from the encoder output E is appended to the shared cache and each
+ * decoder layer updates its local state; [KVC]: the appended row is FP4).
+ *   pos        [B]        int32 position of the new token (its row), 0 <= pos < N
+ *   kv_new     [B, D]     fp32 global KV row of the new token, quantised into
+ *                         kv_fp4 [B,N,D/2] and kv_scale [B,N,D/16] at row pos[b]
+ *                         with exactly the bytes csa2_fp4_quantize writes
+ *   ki_new     [S, B, Di] int8 index key of the new token for each of S key sets,
+ *                         copied to ki[s] + (b * N + pos[b]) * Di
+ *   ki         HOST [S]   device pointers, each [B, N, Di]
+ *   kl_new, vl_new [L, B, D] bf16 local K and V of the new token for each layer
+ *   kl, vl     HOST [L]   device pointers, each [B, Lcap, D]: layer l's local
+ *                         buffers; row r holds position local_base[b] + r
+ *   local_base [B]        int32, read and updated
+ * The new local row goes to row pos - local_base. When that is Lcap (the buffer
+ * is full), the W - 1 rows before it first move to rows 0..W-2 in every layer and
+ * local_base becomes pos - (W - 1); attention over the buffers then sees the
+ * same window (positions [pos - W + 1, pos]). A position further past the end, or
+ * before local_base, is reported as CSA2_ERR_RANGE on the device.
+ * Limits: D % 16 == 0, 16 <= Di <= 128 with Di % 16 == 0, 0 <= S <= 32,
+ *         0 <= L <= 64, and when L > 0: W >= 1 and Lcap >= 2W - 1.
+ * No workspace; every write goes to the caller's buffers.
+ */
+typedef struct {
+    int32_t B, N, D, Di, S, L, W, Lcap;
+    const int32_t* pos;
+    const float* kv_new;
+    uint8_t* kv_fp4;
+    uint8_t* kv_scale;
+    const int8_t* ki_new;
+    int8_t* const* ki;          /* HOST [S] */
+    const uint16_t* kl_new;
+    const uint16_t* vl_new;
+    uint16_t* const* kl;        /* HOST [L] */
+    uint16_t* const* vl;        /* HOST [L] */
+    int32_t* local_base;
+} csa2_append_args;
+
 /* Workspace bytes a call with these arguments needs. which: 0 = csa2_index_topk
  * (args = csa2_index_args*), 1 = csa2_sparse_attn (csa2_attn_args*),
  * 2 = csa2_layer_stack (csa2_stack_args*). Returns 0 for invalid arguments.
@@ -203,6 +243,10 @@ csa2_status csa2_sparse_attn_noalloc(const csa2_attn_args* args, int32_t* d_stat
  * a timeout, zero the workspace before the next call.
  * Waits on a CTA's own copies and tensor-core operations keep the fixed budget. */
 csa2_status csa2_set_wait_controls(int64_t budget_cycles, int32_t skip_arrival);
+
+/* Append one token per sequence to the global cache, the index keys and every
+ * layer's local buffers (csa2_append_args above). */
+csa2_status csa2_cache_append(const csa2_append_args* args, int32_t* d_status, void* stream);
 
 /* Static text for a status code. */
 const char* csa2_status_string(csa2_status s);

@@ -45,12 +45,22 @@ class AttnArgs(Structure):
     ]
 
 
+class AppendArgs(Structure):
+    _fields_ = [
+        ("B", c_int32), ("N", c_int32), ("D", c_int32), ("Di", c_int32), ("S", c_int32), ("L", c_int32),
+        ("W", c_int32), ("Lcap", c_int32),
+        ("pos", c_void_p), ("kv_new", c_void_p), ("kv_fp4", c_void_p), ("kv_scale", c_void_p),
+        ("ki_new", c_void_p), ("ki", c_void_p), ("kl_new", c_void_p), ("vl_new", c_void_p),
+        ("kl", c_void_p), ("vl", c_void_p), ("local_base", c_void_p),
+    ]
+
+
 class StackArgs(Structure):
     _fields_ = [("L", c_int32), ("idx", POINTER(IndexArgs)), ("attn", POINTER(AttnArgs))]
 
 
 EXPORTED = ("csa2_workspace_bytes", "csa2_index_topk", "csa2_sparse_attn", "csa2_layer_stack",
-            "csa2_fp4_quantize", "csa2_status_string", "csa2_set_wait_controls", "csa2_sparse_attn_noalloc")
+            "csa2_fp4_quantize", "csa2_status_string", "csa2_set_wait_controls", "csa2_sparse_attn_noalloc", "csa2_cache_append")
 
 
 def library_path() -> str:
@@ -77,6 +87,8 @@ def lib():
                 f.restype = c_int
             L.csa2_fp4_quantize.argtypes = [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]
             L.csa2_fp4_quantize.restype = c_int
+            L.csa2_cache_append.argtypes = [POINTER(AppendArgs), c_void_p, c_void_p]
+            L.csa2_cache_append.restype = c_int
             L.csa2_set_wait_controls.argtypes = [c_int64, c_int32]
             L.csa2_set_wait_controls.restype = c_int
             L.csa2_status_string.argtypes = [c_int]
@@ -103,6 +115,10 @@ def csa2_layer_stack(args: StackArgs, workspace: int, ws_bytes: int, d_status: i
 
 def csa2_fp4_quantize(x: int, rows: int, D: int, fp4: int, scale: int, stream: int) -> int:
     return lib().csa2_fp4_quantize(x, rows, D, fp4, scale, stream)
+
+
+def csa2_cache_append(args: AppendArgs, d_status: int, stream: int) -> int:
+    return lib().csa2_cache_append(ctypes.byref(args), d_status, stream)
 
 
 def csa2_set_wait_controls(budget_cycles: int, skip_arrival: int) -> int:

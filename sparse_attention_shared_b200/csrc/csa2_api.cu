@@ -16,6 +16,7 @@
 // next call; after a reported error, zero it again.
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 
 #include "csa2_common.cuh"
@@ -35,7 +36,27 @@ csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* ticke
 bool attn_cluster_fits(const csa2_attn_args& a);
 csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
                                 cudaStream_t stream);
+int attn_slice_cluster(const csa2_attn_args& a);
+csa2_status launch_attn_slice(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
+                              cudaStream_t stream);
+
+// The attention kernel for a call: the slice kernel (one cluster of at most 8 CTAs per
+// query), else the 12-CTA cluster kernel, else one CTA per tile with a ticket merge.
+static csa2_status run_attn(const csa2_attn_args& a, const int32_t* topk, int list_ready, int* tickets,
+                            void* scratch, int32_t* d_status, cudaStream_t stream) {
+    static const int path = [] {
+        const char* e = getenv("CSA2_ATTN_PATH");
+        return e ? atoi(e) : 0;
+    }();
+    if (path == 0 && attn_slice_cluster(a) > 0) return launch_attn_slice(a, topk, list_ready, d_status, stream);
+    if (path <= 1 && attn_cluster_fits(a)) return launch_attn_cluster(a, topk, list_ready, d_status, stream);
+    return launch_attn(a, topk, tickets, scratch, d_status, stream);
+}
 void set_wait_controls(long long budget, int skip);
+// cache_append.cu
+csa2_status launch_cache_append(const csa2_append_args& a, int32_t* d_status, cudaStream_t stream);
+int append_max_sets();
+int append_max_layers();
 // fp4_quant.cu
 cudaError_t launch_fp4_quantize(const float* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales,
                                 cudaStream_t stream);
@@ -203,8 +224,7 @@ csa2_status csa2_sparse_attn(const csa2_attn_args* args, void* workspace, size_t
         a.local_base = a.q_pos;
         a.Lloc = 0;
     }
-    if (attn_cluster_fits(a)) return launch_attn_cluster(a, a.topk, 0, d_status, static_cast<cudaStream_t>(stream));
-    return launch_attn(a, a.topk, tickets, scratch, d_status, static_cast<cudaStream_t>(stream));
+    return run_attn(a, a.topk, 0, tickets, scratch, d_status, static_cast<cudaStream_t>(stream));
 }
 
 csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t ws_bytes, int32_t* d_status,
@@ -260,11 +280,37 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
         // kernel is the previous layer's attention), so its clusters may gather their
         // global rows before waiting for that kernel; not when a copy came between.
         const int list_ready = (ix.mode == CSA2_REUSE && !copied) ? 1 : 0;
-        st = attn_cluster_fits(a) ? launch_attn_cluster(a, cur, list_ready, d_status, strm)
-                                  : launch_attn(a, cur, tickets, scratch, d_status, strm);
+        st = run_attn(a, cur, list_ready, tickets, scratch, d_status, strm);
         if (st != CSA2_OK) return st;
     }
     return CSA2_OK;
+}
+
+csa2_status csa2_cache_append(const csa2_append_args* a, int32_t* d_status, void* stream) {
+    if (!a) return CSA2_ERR_NULL;
+    if (a->B < 1 || a->N < 1 || a->N >= (1 << 27) || a->D < 16 || a->D % 16) return CSA2_ERR_SHAPE;
+    if (a->S < 0 || a->S > append_max_sets() || a->L < 0 || a->L > append_max_layers()) return CSA2_ERR_SHAPE;
+    if (a->S > 0 && (a->Di < 16 || a->Di > 128 || a->Di % 16)) return CSA2_ERR_SHAPE;
+    if (a->L > 0 && (a->W < 1 || a->Lcap < std::max(1, 2 * a->W - 1))) return CSA2_ERR_SHAPE;
+    if (!a->pos || !a->kv_new || !a->kv_fp4 || !a->kv_scale) return CSA2_ERR_NULL;
+    if (!al16(a->pos) || !al16(a->kv_new) || !al16(a->kv_fp4) || !al16(a->kv_scale)) return CSA2_ERR_ALIGN;
+    if (a->S > 0) {
+        if (!a->ki_new || !a->ki) return CSA2_ERR_NULL;
+        if (!al16(a->ki_new)) return CSA2_ERR_ALIGN;
+        for (int s = 0; s < a->S; ++s) {
+            if (!a->ki[s]) return CSA2_ERR_NULL;
+            if (!al16(a->ki[s])) return CSA2_ERR_ALIGN;
+        }
+    }
+    if (a->L > 0) {
+        if (!a->kl_new || !a->vl_new || !a->kl || !a->vl || !a->local_base) return CSA2_ERR_NULL;
+        if (!al16(a->kl_new) || !al16(a->vl_new) || !al16(a->local_base)) return CSA2_ERR_ALIGN;
+        for (int l = 0; l < a->L; ++l) {
+            if (!a->kl[l] || !a->vl[l]) return CSA2_ERR_NULL;
+            if (!al16(a->kl[l]) || !al16(a->vl[l])) return CSA2_ERR_ALIGN;
+        }
+    }
+    return launch_cache_append(*a, d_status, static_cast<cudaStream_t>(stream));
 }
 
 csa2_status csa2_set_wait_controls(int64_t budget_cycles, int32_t skip_arrival) {

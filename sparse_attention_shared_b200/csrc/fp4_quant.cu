@@ -1,33 +1,10 @@
-// FP4 (E2M1) quantisation with one E4M3 scale per 16 values.
-//
-// Format: "DeepSeek-V4.1 Flash Pushes KV Cache Compression for Agent Workloads",
-// section "Ana Gelisme" (E2M1 values, E4M3 scale per 16 channels). Rounding
-// rules fixed by this library: scale = E4M3 nearest amax/6 (ties to even,
-// saturating at 448); code = E2M1 nearest x/scale (ties to even, saturating
-// at +-6); zero scale -> zero codes; no -0.
-//
-// One thread per 16-value group. The E2M1 decision compares |x| with the
-// seven midpoints times the scale; each product has at most 7 significant bits
-// and is exact in fp32, so the decision is the one the exact quotient gives.
-// Strict and non-strict comparisons alternate so that ties go to the even code.
+// FP4 (E2M1) quantisation with one E4M3 scale per 16 values ("DeepSeek-V4.1
+// Flash Pushes KV Cache Compression for Agent Workloads", section "Ana Gelisme");
+// the rounding rules are in fp4_codec.cuh. One thread per 16-value group.
 #include "csa2_common.cuh"
+#include "fp4_codec.cuh"
 
 namespace csa2 {
-
-__device__ __forceinline__ uint32_t e4m3_from_f32_rne_sat(float v) {
-    // Hardware conversion: round to nearest even, clamp to the largest finite
-    // value (448). The value is non-negative here.
-    uint16_t packed;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(packed) : "f"(0.0f), "f"(v));
-    return packed & 0xFFu;
-}
-
-__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
-    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
-    float v = (e == 0) ? (float)m * 0.001953125f                        // m * 2^-9
-                       : __uint_as_float(((e + 120u) << 23) | (m << 20)); // 2^(e-7) * (1 + m/8)
-    return (b & 0x80u) ? -v : v;
-}
 
 __global__ void __launch_bounds__(256) fp4_quantize_kernel(const float* __restrict__ x, int64_t groups,
                                                            uint8_t* __restrict__ codes,
@@ -41,24 +18,8 @@ __global__ void __launch_bounds__(256) fp4_quantize_kernel(const float* __restri
         float4 f = src[i];
         v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
     }
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    const uint32_t sc = e4m3_from_f32_rne_sat(__fdiv_rn(amax, 6.0f));
-    const float s = e4m3_to_f32(sc);
-    uint32_t packed[2] = {0u, 0u};
-    if (s > 0.f) {
-        const float t1 = 0.25f * s, t2 = 0.75f * s, t3 = 1.25f * s, t4 = 1.75f * s;
-        const float t5 = 2.5f * s, t6 = 3.5f * s, t7 = 5.0f * s;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float a = fabsf(v[i]);
-            uint32_t c = (uint32_t)(a > t1) + (uint32_t)(a >= t2) + (uint32_t)(a > t3) + (uint32_t)(a >= t4) +
-                         (uint32_t)(a > t5) + (uint32_t)(a >= t6) + (uint32_t)(a > t7);
-            if (v[i] < 0.f && c != 0u) c |= 8u;
-            packed[i >> 3] |= c << (4 * (i & 7));
-        }
-    }
+    uint32_t packed[2];
+    const uint32_t sc = fp4_quantize_group16(v, packed);
     reinterpret_cast<uint2*>(codes)[g] = make_uint2(packed[0], packed[1]);
     scales[g] = (uint8_t)sc;
 }

@@ -2,6 +2,7 @@
 marshalling only. Every step of the computation runs in libcsa2.so."""
 from __future__ import annotations
 
+import ctypes
 from typing import Dict, List, Optional, Sequence
 
 import numpy as np
@@ -137,6 +138,31 @@ def sparse_attn(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base, W: int, ws
     st = status.ptr if status is not None else 0
     check(capi.csa2_sparse_attn(a, _ptr(buf), buf.numel(), st, _stream(stream)), "csa2_sparse_attn")
     return out, lse
+
+
+def cache_append(pos, kv_new, kv_fp4, kv_scale, ki_new=None, ki_sets=(), kl_new=None, vl_new=None, kl_layers=(),
+                 vl_layers=(), local_base=None, W: int = 0, status: Status = None, stream=None):
+    """Append one token per sequence (csa2_cache_append): its global row (fp32 [B, D])
+    into the FP4 cache at row pos[b], its index key ([S, B, Di]) into each key set,
+    and each layer's local K/V ([L, B, D] bf16) into that layer's buffers
+    ([B, Lcap, D]); local_base is updated in place."""
+    _need_cuda(pos, kv_new, kv_fp4, kv_scale, ki_new, kl_new, vl_new, local_base, *ki_sets, *kl_layers, *vl_layers)
+    a = capi.AppendArgs()
+    B, D = kv_new.shape
+    a.B, a.N, a.D = B, kv_fp4.shape[1], D
+    a.S, a.L, a.W = len(ki_sets), len(kl_layers), W
+    a.Di = int(ki_sets[0].shape[-1]) if ki_sets else 0
+    a.Lcap = int(kl_layers[0].shape[1]) if kl_layers else 0
+    ki_arr = (ctypes.c_void_p * max(1, a.S))(*[_ptr(t) for t in ki_sets])
+    kl_arr = (ctypes.c_void_p * max(1, a.L))(*[_ptr(t) for t in kl_layers])
+    vl_arr = (ctypes.c_void_p * max(1, a.L))(*[_ptr(t) for t in vl_layers])
+    a.pos, a.kv_new, a.kv_fp4, a.kv_scale = _ptr(pos), _ptr(kv_new), _ptr(kv_fp4), _ptr(kv_scale)
+    a.ki_new, a.ki = _ptr(ki_new), ctypes.cast(ki_arr, ctypes.c_void_p)
+    a.kl_new, a.vl_new = _ptr(kl_new), _ptr(vl_new)
+    a.kl, a.vl = ctypes.cast(kl_arr, ctypes.c_void_p), ctypes.cast(vl_arr, ctypes.c_void_p)
+    a.local_base = _ptr(local_base)
+    st = status.ptr if status is not None else 0
+    check(capi.csa2_cache_append(a, st, _stream(stream)), "csa2_cache_append")
 
 
 def packed_views(specs, device, align: int = 256):

@@ -288,7 +288,10 @@ def test_attention_tiny(ws, status):
     (2, 4096, 1, 16, 128, 1, 0),         # single global entry, no window
     (2, 4096, 1, 16, 128, 2048, 0),      # no local branch
     (1, 300, 1, 16, 128, 512, 64),       # fewer positions than k: -1 padding
-    (2, 8192, 1, 16, 128, 4096, 1024),   # 16 + 8 tiles: more than one cluster holds, ticket merge
+    (2, 8192, 1, 16, 128, 4096, 1024),   # 8 CTAs of 4 blocks and a window tile each: the largest cluster
+    (2, 8192, 1, 16, 128, 4096, 2048),   # 16 window tiles: more than one cluster holds, ticket merge
+    (3, 5000, 1, 32, 64, 700, 300),      # 32 heads at D = 64, ragged blocks
+    (2, 4096, 1, 16, 128, 1, 512),       # one global entry, four window tiles: CTAs with no global block
 ])
 def test_attention_shapes(B, N, Tq, Hq, D, k, W, ws, status):
     _attn_case(B, N, Tq, Hq, D, k, W, seed=B * 7 + N, ws=ws, status=status)
@@ -364,25 +367,57 @@ def test_layer_stack_rejects_bad_mode_order(ws):
         ops.LayerStack([layers[3]], dw.q_pos, dw.kv_fp4, dw.kv_scale, dw.local_base)                # REINDEX first
 
 
-# ---------------------------------------------------------------- full-size workloads, sampled
-def test_decode_full_sampled(ws, status):
-    wl = synth.make_workload("decode_full")
-    _check_stack(wl, [(0, 0), (17, 0), (31, 0)], ws, status, keep_reuse=False)
+# ---------------------------------------------------------------- full-size workloads, every unit
+def _check_stack_every_unit(wl, ws, status):
+    """The whole workload through the CUDA stack; every query's pool and top-k list of
+    every layer compared bit for bit with the C++ oracle (threads over units), every
+    list checked for the causal layout, and every query's output and lse at every
+    layer compared within the tolerances."""
+    from oracle import cpp as C
+    s = wl.spec
+    dw = DeviceWorkload(wl)
+    st = ops.LayerStack(dw.layer_dicts(), dw.q_pos, dw.kv_fp4, dw.kv_scale, dw.local_base, keep_reuse_lists=False)
+    st.run(ws, status)
+    torch.cuda.synchronize()
+    status.check("stack")
+    q_pos = wl.q_pos()
+    lists = C.stack_lists(wl)
+    for li, e in enumerate(lists):
+        if st.topks[li] is not None:
+            assert_list_invariants(st.topks[li].cpu().numpy(), q_pos, f"layer {li} topk")
+            assert_lists_equal(st.topks[li], e["topk"], f"layer {li} ({e['mode']}) topk, every unit")
+        if st.pools[li] is not None:
+            assert_list_invariants(st.pools[li].cpu().numpy(), q_pos, f"layer {li} pool")
+            assert_lists_equal(st.pools[li], e["pool"], f"layer {li} pool, every unit")
+    codes, scales = C.fp4_quantize(wl.kv_f32())
+    assert_lists_equal(dw.kv_fp4, codes, "FP4 codes of the cache")
+    assert_lists_equal(dw.kv_scale, scales, "E4M3 scales of the cache")
+    outs = C.stack_outputs(wl, codes, scales, lists, range(s.B))
+    worst = 0.0
+    for li in range(s.L):
+        worst = max(worst, assert_attn_close(st.outs[li], st.lses[li], outs[li]["out"], outs[li]["lse"],
+                                             f"layer {li}, every unit"))
+    return worst
 
 
-def test_prefill_chunk_sampled(ws, status):
-    # 4096 queries of one sequence (one CTA per query, scores spilled), 32 heads
-    wl = synth.make_workload("prefill_chunk")
-    _check_stack(wl, [(0, 0), (0, 1777), (0, 4095)], ws, status, keep_reuse=False)
+def test_decode_full_every_unit(ws, status):
+    _check_stack_every_unit(synth.make_workload("decode_full"), ws, status)
 
 
-def test_long_1m_sampled(ws, status):
-    # one sequence of 2^20 positions, 64 queries: the Full scan spills its scores (two
-    # CTAs per query), nine Reindex layers select from the pool by the group's single select
-    wl = synth.make_workload("long_1m")
-    _check_stack(wl, [(0, 0), (0, 63)], ws, status, keep_reuse=False)
+def test_prefill_chunk_every_unit(ws, status):
+    # 4096 queries of one sequence, 32 heads; the multi-query scoring kernel, then the select-only pass
+    _check_stack_every_unit(synth.make_workload("prefill_chunk"), ws, status)
 
 
-def test_stack20_128k_sampled(ws, status):
-    wl = synth.make_workload("stack20_128k")
-    _check_stack(wl, [(0, 0), (15, 0)], ws, status, keep_reuse=False)
+def test_long_1m_every_unit(ws, status):
+    # one sequence of 2^20 positions, 64 queries: the Full layer's scores spill (two CTAs per query),
+    # nine Reindex layers select from the pool by the group's single select
+    _check_stack_every_unit(synth.make_workload("long_1m"), ws, status)
+
+
+def test_stack20_128k_every_unit(ws, status):
+    _check_stack_every_unit(synth.make_workload("stack20_128k"), ws, status)
+
+
+def test_tiny_every_unit(ws, status):
+    _check_stack_every_unit(synth.make_workload("tiny"), ws, status)
