@@ -37,6 +37,7 @@
 #include <algorithm>
 #include <atomic>
 #include <climits>
+#include <cstdlib>
 #include <cstring>
 
 #include "csa2_common.cuh"
@@ -2206,9 +2207,21 @@ static cudaError_t launch_mq(const MqParams& mp, const CUtensorMap& map, int gri
     return cudaLaunchKernelEx(&cfg, kern, mp, map);
 }
 
+int reindex_cluster_size(const csa2_index_args& a, int P_in);
+csa2_status launch_reindex_cl(const csa2_index_args& a, const int32_t* pool_in, int P_in, int pool_ready,
+                              const csa2_attn_args* pf, int32_t* d_status, cudaStream_t stream);
+
 // Launch one indexer call. `ws` holds plan_index(a).ws_bytes bytes (zero at first use).
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
                          int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready) {
+    static const int rx_path = [] {
+        const char* e = getenv("CSA2_REINDEX_PATH");
+        return e ? atoi(e) : 0;
+    }();
+    // Reindex over a pool of at most a few thousand entries per CTA: the clustered kernel
+    // (reindex.cu); its pool was written two or more kernels back when keys_ready is set
+    if (a.mode == CSA2_REINDEX && rx_path == 0 && reindex_cluster_size(a, P_in) > 0)
+        return launch_reindex_cl(a, pool_in, P_in, keys_ready, pf, d_status, stream);
     const int sms = num_sms();
     csa2_index_args aa = a;
     aa.P_in = P_in;

@@ -47,6 +47,7 @@ class WorkloadSpec:
     W: int
     layers: tuple
     description: str = ""
+    replay: bool = False  # bounded replay: local KV exists only for the Tq replayed positions
 
     @property
     def L(self) -> int:
@@ -54,6 +55,8 @@ class WorkloadSpec:
 
     @property
     def local_base(self) -> int:
+        if self.replay:
+            return self.N - self.Tq
         return max(0, self.N - self.Tq - self.W + 1)
 
     @property
@@ -117,6 +120,12 @@ CONFIGS: Dict[str, WorkloadSpec] = {
         description="1 seq x 1048576 positions, 64 decode queries, layer 1 Full "
                     "(pool 8192, top-2048), layers 2-20 alternate Reindex (top-1024) and Reuse, "
                     "one shared key set, SWA 1024"),
+    "replay_prefill": WorkloadSpec(
+        "replay_prefill", B=4, N=131072, Tq=512, Hq=16, D=128, Hi=8, Di=64, W=512,
+        layers=_stack20_layers(), replay=True,
+        description="bounded-replay prefill: the last 512 of 131072 prompt positions of 4 seqs replayed "
+                    "through 20 layers [Full,Reuse,Reuse,Reindex]x5 (pool 8192, top-2048), window 512 "
+                    "with references before the replayed segment cut"),
     "paper_schedule": WorkloadSpec(
         "paper_schedule", B=16, N=131072, Tq=1, Hq=16, D=128, Hi=8, Di=64, W=128,
         layers=_paper_layers(),

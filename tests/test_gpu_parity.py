@@ -421,3 +421,11 @@ def test_stack20_128k_every_unit(ws, status):
 
 def test_tiny_every_unit(ws, status):
     _check_stack_every_unit(synth.make_workload("tiny"), ws, status)
+
+
+def test_replay_prefill_every_unit(ws, status):
+    # bounded replay: the last 256 of 16384 prompt positions through [F,U,U,RI]x5, window references cut at
+    # the segment (local_base = N - 256); the Full layers score the 256 queries in blocks that share key tiles
+    wl = synth.make_workload("replay_prefill", B=2, N=16384, Tq=256, W=256)
+    assert wl.spec.local_base == 16384 - 256
+    _check_stack_every_unit(wl, ws, status)

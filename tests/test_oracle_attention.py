@@ -109,3 +109,29 @@ def test_window_bounds():
 def test_empty_union():
     out, lse = O.attend(np.ones((2, 8)), np.zeros((0, 8)), np.zeros((0, 8)), 1.0)
     assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def test_bounded_replay_truncates_window_at_the_segment():
+    """Bounded replay ("CED: Continuing Context with a Causal Encoder and Decoder",
+    "Why Prefill Recomputes a Recent Segment", Fig. 6): only the last R prompt
+    positions pass through the decoder again, and window references before the
+    replayed segment are cut. With local_base = N - R the first replayed position
+    reads only its own local row, and the last position (R = W) reads the same W
+    rows as a full execution, so its output equals the untruncated one while the
+    first position's does not."""
+    wl = synth.make_workload("replay_prefill", B=1, N=3000, Tq=8, W=8, layers=synth.workloads._stack20_layers(64, 256)[:2])
+    s = wl.spec
+    assert s.local_base == s.N - s.Tq and s.Lloc == s.Tq
+    assert O.window_positions(s.N - s.Tq, s.W, s.local_base).tolist() == [s.N - s.Tq]
+    assert O.window_positions(s.N - 1, s.W, s.local_base).tolist() == list(range(s.N - s.W, s.N))
+    codes, scales = O.fp4_quantize(wl.kv_f32()[0])
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((s.Hq, s.D))
+    kl = rng.standard_normal((s.N, s.D))       # local rows of every position (a full execution's)
+    vl = rng.standard_normal((s.N, s.D))
+    topk = np.sort(rng.choice(s.N - s.Tq, 64, replace=False)).astype(np.int32)
+    seg = slice(s.local_base, s.N)
+    for t, same in ((s.N - 1, True), (s.N - s.Tq, False)):
+        trunc = O.attention_unit(q, codes, scales, topk, kl[seg], vl[seg], s.local_base, t, s.W)
+        full = O.attention_unit(q, codes, scales, topk, kl, vl, 0, t, s.W)
+        assert np.allclose(trunc[0], full[0], rtol=0, atol=1e-12) == same
