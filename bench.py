@@ -52,12 +52,12 @@ def unit_bytes(spec):
     once per kernel call): index keys scanned or gathered, pool/list indices, FP4
     rows gathered (D/2 + D/16 bytes), local K+V rows, queries and outputs."""
     D, Di, Hi, Hq = spec.D, spec.Di, spec.Hi, spec.Hq
-    t = spec.N - 1
+    t = spec.n_pos - 1
     total = 0
     k_cur, pool_P = 0, 0
     for L in spec.layers:
         if L.mode == "FULL":
-            total += (t + 1) * Di + Hi * Di + (L.P + L.k) * 4
+            total += entries_read(spec, t) * Di + Hi * Di + (L.P + L.k) * 4
             k_cur = L.k
             pool_P = L.P or pool_P
         elif L.mode == "REINDEX":
@@ -67,11 +67,16 @@ def unit_bytes(spec):
     return total
 
 
+def entries_read(spec, t):
+    """Global entries the query at position t reads (compression rate m: complete groups)."""
+    return (t + 1) // spec.m if spec.m > 1 else t + 1
+
+
 def full_launch_bytes(spec, q_pos):
     """Algorithmic bytes of the first layer's Full indexer call: every sequence's keys
     up to its last query position once, then per query its index query and lists."""
     L = spec.layers[0]
-    keys = sum(int(q_pos[b].max()) + 1 for b in range(spec.B)) * spec.Di
+    keys = sum(entries_read(spec, int(q_pos[b].max())) for b in range(spec.B)) * spec.Di
     return keys + spec.B * spec.Tq * (spec.Hi * spec.Di + (L.P + L.k) * 4)
 
 
@@ -102,7 +107,7 @@ def list_bytes(spec, q_pos, local_base, pools, topks):
     total, cur, pool, P_in = 0, None, None, 0
     for li, L in enumerate(spec.layers):
         if L.mode == "FULL":
-            total += sum(int(q_pos[b].max()) + 1 for b in range(B)) * Di
+            total += sum(entries_read(spec, int(q_pos[b].max())) for b in range(B)) * Di
             total += B * Tq * (Hi * Di + (L.P + L.k) * 4)
             cur = topks[li]
             if L.P:
@@ -240,7 +245,7 @@ def build_device_stack(wl, torch, ops, np):
 
     q_pos, base = dev(wl.q_pos()), dev(wl.local_base_arr())
     kv = dev(wl.kv_f32())
-    codes, scales = ops.fp4_quantize(kv.view(-1, s.D))
+    codes, scales = ops.fp4_compress(kv.view(-1, s.D), s.m) if s.m > 1 else ops.fp4_quantize(kv.view(-1, s.D))
     del kv
     wl.drop("kv")
     codes, scales = codes.view(s.B, s.N, -1), scales.view(s.B, s.N, -1)
@@ -256,7 +261,7 @@ def build_device_stack(wl, torch, ops, np):
                 wl.drop(("ki", L.key_set))
             d.update(qi=dev(wl.qi(li)), w=wl.w(li), ki=keys[L.key_set], k=L.k, P=L.P)
         layers.append(d)
-    stack = ops.LayerStack(layers, q_pos, codes, scales, base)
+    stack = ops.LayerStack(layers, q_pos, codes, scales, base, m=s.m)
     return stack, layers, q_pos, codes, scales, base
 
 
@@ -468,7 +473,7 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
     pool_t = torch.empty((s.B, s.Tq, max(Lf.P, 1)), dtype=torch.int32, device="cuda")
     topk_t = torch.empty((s.B, s.Tq, Lf.k), dtype=torch.int32, device="cuda")
     ia = ops.make_index_args(capi.CSA2_FULL, q_pos, d0["qi"], w_host, d0["ki"], Lf.k, Lf.P, None,
-                             pool_t if Lf.P else None, topk_t)
+                             pool_t if Lf.P else None, topk_t, s.m)
     buf = ws.get(capi.csa2_workspace_bytes(0, ia))
     fcall = lambda sp: capi.csa2_index_topk(ia, int(buf.data_ptr()), buf.numel(), st.ptr, sp)
     ms = time_alone(args, torch, fcall, flush, stream, n)
@@ -484,7 +489,7 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
         d = layers[li]
         o = torch.empty_like(d["q"])
         lse = torch.empty(d["q"].shape[:-1], dtype=torch.float32, device="cuda")
-        aa = ops.make_attn_args(q_pos, d["q"], codes, scales, topk_dev, d["kl"], d["vl"], base, s.W, o, lse)
+        aa = ops.make_attn_args(q_pos, d["q"], codes, scales, topk_dev, d["kl"], d["vl"], base, s.W, o, lse, s.m)
         abuf = ws.get(capi.csa2_workspace_bytes(1, aa))
         acall = lambda sp: capi.csa2_sparse_attn(aa, int(abuf.data_ptr()), abuf.numel(), st.ptr, sp)
         t = time_alone(args, torch, acall, flush, stream, n)
@@ -501,7 +506,7 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
         Lr = s.layers[li_r]
         wr = np.ascontiguousarray(np.asarray(d["w"], dtype=np.int32))
         topk_r = torch.empty((s.B, s.Tq, Lr.k), dtype=torch.int32, device="cuda")
-        ra = ops.make_index_args(capi.CSA2_REINDEX, q_pos, d["qi"], wr, d["ki"], Lr.k, 0, pool_t, None, topk_r)
+        ra = ops.make_index_args(capi.CSA2_REINDEX, q_pos, d["qi"], wr, d["ki"], Lr.k, 0, pool_t, None, topk_r, s.m)
         rbuf = ws.get(capi.csa2_workspace_bytes(0, ra))
         rcall = lambda sp: capi.csa2_index_topk(ra, int(rbuf.data_ptr()), rbuf.numel(), st.ptr, sp)
         ms = time_alone(args, torch, rcall, flush, stream, n)
@@ -534,7 +539,7 @@ def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, 
     for d in layers2:
         if d["mode"] != "REUSE":
             d["qi"] = next(it)
-    stack2 = ops.LayerStack(layers2, views[0], codes, scales, base, packed_outputs=True)
+    stack2 = ops.LayerStack(layers2, views[0], codes, scales, base, packed_outputs=True, m=s.m)
     host_in = din.cpu().pin_memory()
     host_out = torch.empty_like(stack2.out_buf, device="cpu").pin_memory()
     h2d = din.numel()                 # bytes of the one input copy (tensors + alignment gaps)
@@ -585,7 +590,7 @@ def cpu_baseline(workload: str, seconds: float):
     wl = synth.make_workload(workload)
     s = wl.spec
     threads = C.host_threads()
-    codes, scales = C.fp4_quantize(wl.kv_f32())     # quantising the cache is setup, not a decode step
+    codes, scales = C.fp4_quantize(wl.kv_f32() if s.m <= 1 else C.compress_entries(wl.kv_f32(), s.m))     # quantising the cache is setup, not a decode step
     wl.drop("kv")
     for li in range(s.L):                             # draw every input before the clock starts
         wl.q(li), wl.kl(li), wl.vl(li)
@@ -633,7 +638,7 @@ def run_reference(args, rank, world):
     wl = synth.make_workload(args.workload)
     s = wl.spec
     threads = C.host_threads()
-    codes, scales = C.fp4_quantize(wl.kv_f32())
+    codes, scales = C.fp4_quantize(wl.kv_f32() if s.m <= 1 else C.compress_entries(wl.kv_f32(), s.m))
     wl.drop("kv")
     state = {"st": C.StackState(wl)}
 

@@ -93,9 +93,18 @@ typedef struct {
     int32_t P_in;               /* Reindex only */
     int32_t* pool_out;          /* Full with P > 0 */
     int32_t* topk_out;
+    int32_t m;                  /* sequence compression rate of ki (see below); 0 or 1: one entry per position */
 } csa2_index_args;
 
 /*
+ * Sequence compression rate m ([CED] "What Does the Sequence Compression Rate
+ * Reduce?"): with m >= 2 (the encoder's CSA2 uses m = 2) row j of the global
+ * cache and of the index keys is one entry that combines positions m*j ..
+ * m*j + m - 1, N counts entries, and a query at position t reads entry j only
+ * once the whole group is causal: j <= (t + 1) / m - 1. Lists then hold entry
+ * indices; the local window stays on positions. csa2_fp4_compress builds such a
+ * cache. 0 <= m <= 8.
+ *
  * One attention call for B sequences x Tq queries.
  *   q        [B,Tq,Hq,D]   bf16 main queries
  *   kv_fp4   [B,N,D/2]     FP4 E2M1 codes, element 2j in the low nibble
@@ -124,6 +133,7 @@ typedef struct {
     const int32_t* local_base;
     uint16_t* out;
     float* lse;
+    int32_t m;                  /* sequence compression rate of the global cache; 0 or 1: one row per position */
 } csa2_attn_args;
 
 /*
@@ -213,6 +223,15 @@ csa2_status csa2_layer_stack(const csa2_stack_args* args, void* workspace, size_
  *   x [rows, D] fp32, D % 16 == 0 -> fp4 [rows, D/2], scale [rows, D/16]. */
 csa2_status csa2_fp4_quantize(const float* x, int64_t rows, int32_t D, uint8_t* fp4,
                               uint8_t* scale, void* stream);
+
+/* Global entries of compression rate m from per-position rows, FP4-quantised:
+ * entry g of x [groups * m, D] fp32 combines rows g*m .. g*m + m - 1. The pages do
+ * not give the combining rule; this library takes their mean, summed left to right
+ * in fp32 and scaled by 1/m (exact for m in {1, 2, 4, 8}), and quantises it like
+ * csa2_fp4_quantize -> fp4 [groups, D/2], scale [groups, D/16]. m = 1 is
+ * csa2_fp4_quantize. */
+csa2_status csa2_fp4_compress(const float* x, int64_t groups, int32_t m, int32_t D, uint8_t* fp4, uint8_t* scale,
+                              void* stream);
 
 /* Attention without a caller workspace, for callers that cannot allocate device
  * memory: code running inside a host framework that owns every device allocation

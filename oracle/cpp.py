@@ -54,6 +54,10 @@ def lib():
             L.orc_e4m3_round.argtypes = [dbl]
             L.orc_e4m3_round.restype = i32
             L.orc_fp4_quantize.argtypes = [vp, i64, i32, vp, vp, i32]
+            L.orc_compress_entries.argtypes = [vp, i64, i32, i32, vp]
+            L.orc_compress_entries.restype = None
+            L.orc_last_entry.argtypes = [i32, i32]
+            L.orc_last_entry.restype = i32
             L.orc_fp4_value.argtypes = [vp, vp, i32]
             L.orc_fp4_value.restype = dbl
             L.orc_index_full.argtypes = [vp, vp, i32, i32, vp, i32, i32, i32, i32, vp, vp]
@@ -87,6 +91,23 @@ def fp4_quantize(x: np.ndarray, threads: int = 0):
     scales = np.empty(x.shape[:-1] + (D // 16,), np.uint8)
     lib().orc_fp4_quantize(_p(x), rows, D, _p(codes), _p(scales), threads or host_threads())
     return codes, scales
+
+
+def compress_entries(x: np.ndarray, m: int) -> np.ndarray:
+    """Entries of compression rate m from per-position rows [..., n, D]: [..., n / m, D]."""
+    x = _c(x, np.float32)
+    D = x.shape[-1]
+    groups = x.size // D // m
+    out = np.empty(x.shape[:-2] + (x.shape[-2] // m, D), np.float32)
+    lib().orc_compress_entries(_p(x), groups, m, D, _p(out))
+    return out
+
+
+def last_entries(q_pos, m: int) -> np.ndarray:
+    """The last global entry each query position may read."""
+    q = np.asarray(q_pos, dtype=np.int32)
+    L = lib()
+    return np.vectorize(lambda t: L.orc_last_entry(int(t), m), otypes=[np.int32])(q) if q.size else q
 
 
 def index_full(qi, w, keys, t: int, k: int, P: int = 0):
@@ -186,7 +207,8 @@ def run_layer(st: StackState, li: int, codes=None, scales=None, threads: int = 0
     q_pos = st.pick(wl.q_pos())
     e = {"mode": L.mode, "pool": None}
     if L.mode == "FULL":
-        p, st.cur = index_full_batch(q_pos, st.pick(wl.qi(li)), wl.w(li), st.pick(wl.ki(L.key_set)), L.k, L.P, threads)
+        q_ent = q_pos if s.m <= 1 else last_entries(q_pos, s.m)   # the bound on global entries
+        p, st.cur = index_full_batch(q_ent, st.pick(wl.qi(li)), wl.w(li), st.pick(wl.ki(L.key_set)), L.k, L.P, threads)
         if p is not None:
             st.pool = p
         e["pool"] = p

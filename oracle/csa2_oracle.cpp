@@ -165,6 +165,24 @@ void orc_fp4_quantize(const float* x, int64_t rows, int D, uint8_t* codes, uint8
     });
 }
 
+// Global entries of sequence compression rate m ([CED] "What Does the Sequence
+// Compression Rate Reduce?": at m = 2 two positions become one entry). The pages
+// give no combining rule; this reading takes the mean: entry g of x [groups*m][D]
+// is (x[g*m] + ... + x[g*m + m - 1]) summed left to right in fp32, times 1/m.
+void orc_compress_entries(const float* x, int64_t groups, int m, int D, float* out) {
+    for (int64_t g = 0; g < groups; ++g)
+        for (int d = 0; d < D; ++d) {
+            float acc = x[(g * m) * D + d];
+            for (int r = 1; r < m; ++r) acc = acc + x[(g * m + r) * D + d];
+            out[g * D + d] = acc * (1.0f / (float)m);
+        }
+}
+
+// The last global entry a query at position t may read: entries are positions at
+// m <= 1; at m >= 2 entry j covers positions m*j .. m*j + m - 1 and is read once
+// the whole group is causal.
+int orc_last_entry(int t, int m) { return m <= 1 ? t : (t + 1) / m - 1; }
+
 // Value of element d of an FP4 row: e2m1(code) * e4m3(scale of its 16-group).
 double orc_fp4_value(const uint8_t* codes_row, const uint8_t* scales_row, int d) {
     const int byte = codes_row[d / 2];

@@ -183,20 +183,45 @@ def pad_list(pos: np.ndarray, length: int) -> np.ndarray:
     return out
 
 
-def valid_positions(t: int, N: int) -> np.ndarray:
-    """Causal candidates of the query at position t: 0 <= s <= t and s < N
-    ([CED] "One Token Sequence and Causal Access", Fig. 2)."""
-    return np.arange(0, min(t, N - 1) + 1, dtype=np.int64)
+def last_entry(t: int, m: int = 1) -> int:
+    """The last global entry the query at position t may read. With sequence
+    compression rate m >= 2, entry j combines positions m*j .. m*j + m - 1 ([CED]
+    "What Does the Sequence Compression Rate Reduce?": two positions become one
+    entry at m = 2; the teaching example counts only complete groups), so it is
+    readable once position m*j + m - 1 <= t. With m = 1 entries are positions."""
+    if m <= 1:
+        return t
+    return (t + 1) // m - 1
 
 
-def index_full(qi, w, keys_seq, t: int, k: int, P: int = 0):
+def valid_positions(t: int, N: int, m: int = 1) -> np.ndarray:
+    """Causal candidates of the query at position t: entries 0 <= s <= last_entry(t)
+    and s < N ([CED] "One Token Sequence and Causal Access", Fig. 2)."""
+    return np.arange(0, min(last_entry(t, m), N - 1) + 1, dtype=np.int64)
+
+
+def compress_entries(x: np.ndarray, m: int) -> np.ndarray:
+    """Global entries of compression rate m from per-position rows x [n, D] (n a
+    multiple of m): entry g combines rows g*m .. g*m + m - 1. The pages give no
+    combining rule (PARITY UNPINNED for the rule itself); this reading takes the
+    mean, summed left to right in fp32 and scaled by 1/m, which is exact for m a
+    power of two."""
+    x = np.asarray(x, dtype=np.float32)
+    g = x.reshape(x.shape[:-2] + (x.shape[-2] // m, m, x.shape[-1]))
+    acc = g[..., 0, :].copy()
+    for r in range(1, m):
+        acc = (acc + g[..., r, :]).astype(np.float32)
+    return (acc * np.float32(1.0 / m)).astype(np.float32)
+
+
+def index_full(qi, w, keys_seq, t: int, k: int, P: int = 0, m: int = 1):
     """Full mode: score every causal position, keep the top-P pool and the top-k list.
 
     keys_seq [N, Di] int8 of the query's sequence. Returns (pool or None, topk),
     each padded with -1 to its length. topk is the top-k of the same scores, so it
     is a subset of the pool ([CED] Fig. 5, "Hierarchical Sparse Indexer").
     """
-    cand = valid_positions(t, keys_seq.shape[0])
+    cand = valid_positions(t, keys_seq.shape[0], m)
     sc = index_scores(qi, w, keys_seq[cand])
     topk = pad_list(select_best(sc, cand, k), k)
     pool = pad_list(select_best(sc, cand, P), P) if P > 0 else None
@@ -280,7 +305,7 @@ FULL, REINDEX, REUSE = "FULL", "REINDEX", "REUSE"
 
 
 def layer_stack_unit(layers: Sequence[dict], t: int, kv_codes_seq, kv_scales_seq,
-                     local_base: int, with_attention: bool = True) -> List[Dict]:
+                     local_base: int, with_attention: bool = True, m: int = 1) -> List[Dict]:
     """Run the decoder layers for one query at position t.
 
     Each entry of `layers` is a dict with
@@ -299,7 +324,7 @@ def layer_stack_unit(layers: Sequence[dict], t: int, kv_codes_seq, kv_scales_seq
         mode = L["mode"]
         entry = {"mode": mode, "pool": None}
         if mode == FULL:
-            pool_l, cur = index_full(L["qi"], L["w"], L["keys"], t, L["k"], L.get("P", 0))
+            pool_l, cur = index_full(L["qi"], L["w"], L["keys"], t, L["k"], L.get("P", 0), m)
             if pool_l is not None:
                 pool = pool_l
             entry["pool"] = pool_l

@@ -21,7 +21,9 @@ class OracleCache:
 
     def seq(self, b: int):
         if b not in self._seq:
-            self._seq[b] = O.fp4_quantize(self.wl.kv_f32()[b])
+            m = self.wl.spec.m
+            x = self.wl.kv_f32()[b]
+            self._seq[b] = O.fp4_quantize(O.compress_entries(x, m) if m > 1 else x)
         return self._seq[b]
 
 
@@ -49,5 +51,5 @@ def run_units(wl, units: Iterable[Tuple[int, int]], cache: OracleCache = None,
         t = int(wl.q_pos()[b, j])
         codes, scales = cache.seq(b) if with_attention else (None, None)
         res[(b, j)] = O.layer_stack_unit(layer_inputs(wl, b, j, with_attention), t, codes, scales,
-                                         int(wl.local_base_arr()[b]), with_attention)
+                                         int(wl.local_base_arr()[b]), with_attention, wl.spec.m)
     return res

@@ -31,7 +31,7 @@ class IndexArgs(Structure):
         ("k", c_int32), ("P", c_int32), ("mode", c_int32),
         ("q_pos", c_void_p), ("qi", c_void_p), ("w", c_void_p), ("ki", c_void_p),
         ("ki_seq_stride", c_int64), ("pool_in", c_void_p), ("P_in", c_int32),
-        ("pool_out", c_void_p), ("topk_out", c_void_p),
+        ("pool_out", c_void_p), ("topk_out", c_void_p), ("m", c_int32),
     ]
 
 
@@ -41,7 +41,7 @@ class AttnArgs(Structure):
         ("k", c_int32), ("W", c_int32), ("Lloc", c_int32),
         ("q_pos", c_void_p), ("q", c_void_p), ("kv_fp4", c_void_p), ("kv_scale", c_void_p),
         ("topk", c_void_p), ("kl", c_void_p), ("vl", c_void_p), ("local_base", c_void_p),
-        ("out", c_void_p), ("lse", c_void_p),
+        ("out", c_void_p), ("lse", c_void_p), ("m", c_int32),
     ]
 
 
@@ -60,7 +60,8 @@ class StackArgs(Structure):
 
 
 EXPORTED = ("csa2_workspace_bytes", "csa2_index_topk", "csa2_sparse_attn", "csa2_layer_stack",
-            "csa2_fp4_quantize", "csa2_status_string", "csa2_set_wait_controls", "csa2_sparse_attn_noalloc", "csa2_cache_append")
+            "csa2_fp4_quantize", "csa2_status_string", "csa2_set_wait_controls", "csa2_sparse_attn_noalloc", "csa2_cache_append",
+            "csa2_fp4_compress")
 
 
 def library_path() -> str:
@@ -87,6 +88,8 @@ def lib():
                 f.restype = c_int
             L.csa2_fp4_quantize.argtypes = [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]
             L.csa2_fp4_quantize.restype = c_int
+            L.csa2_fp4_compress.argtypes = [c_void_p, c_int64, c_int32, c_int32, c_void_p, c_void_p, c_void_p]
+            L.csa2_fp4_compress.restype = c_int
             L.csa2_cache_append.argtypes = [POINTER(AppendArgs), c_void_p, c_void_p]
             L.csa2_cache_append.restype = c_int
             L.csa2_set_wait_controls.argtypes = [c_int64, c_int32]
@@ -123,6 +126,10 @@ def csa2_cache_append(args: AppendArgs, d_status: int, stream: int) -> int:
 
 def csa2_set_wait_controls(budget_cycles: int, skip_arrival: int) -> int:
     return lib().csa2_set_wait_controls(budget_cycles, skip_arrival)
+
+
+def csa2_fp4_compress(x: int, groups: int, m: int, D: int, fp4: int, scale: int, stream: int) -> int:
+    return lib().csa2_fp4_compress(x, groups, m, D, fp4, scale, stream)
 
 
 def csa2_status_string(code: int) -> str:

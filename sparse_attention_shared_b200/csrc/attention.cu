@@ -52,6 +52,7 @@ struct AttnParams {
     int* tickets;   // [units]
     int32_t* status;
     int list_ready; // the list and the cache were complete before the previous kernel began
+    int m;          // sequence compression rate of the global entries
 };
 
 template <int HQP>
@@ -152,9 +153,11 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
         S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
 
     int t = p.q_pos[u];
-    if (t < 0 || t >= p.N) {
+    int tg = last_entry(t, p.m);   // the last global entry the query reads
+    if (t < 0 || tg >= p.N) {
         if (tid == 0 && tau == 0) report(p.status, CSA2_ERR_RANGE, u);
         t = -1;
+        tg = -1;
     }
     const int base = p.local_base[b];
 
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
     if (global_tile) {
         const int j = tau * kTileKeys + r;
         int s = (j < p.k) ? p.topk[(size_t)u * p.k + j] : -1;
-        if (s >= 0 && (s > t || s >= p.N)) {
+        if (s >= 0 && (s > tg || s >= p.N)) {
             report(p.status, CSA2_ERR_RANGE, u);
             s = -1;
         }
@@ -563,9 +566,11 @@ __global__ void __launch_bounds__(kClThreads, 2)
         const int j0 = rank * 2 * kTileKeys + tid;
         s0 = (j0 < p.k) ? __ldcg(p.topk + (size_t)u * p.k + j0) : -1;
     }
-    if (t < 0 || t >= p.N) {
+    int tg = last_entry(t, p.m);   // the last global entry the query reads
+    if (t < 0 || tg >= p.N) {
         if (tid == 0 && rank == 0) report(p.status, CSA2_ERR_RANGE, u);
         t = -1;
+        tg = -1;
     }
     const int lo_w = max(max(base, t - p.W + 1), 0);
 
@@ -574,7 +579,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
     uint4 c0[D / 32];
     uint32_t sc0[D / 64];
     if (glob) {
-        if (s0 >= 0 && (s0 > t || s0 >= p.N)) { report(p.status, CSA2_ERR_RANGE, u); s0 = -1; }
+        if (s0 >= 0 && (s0 > tg || s0 >= p.N)) { report(p.status, CSA2_ERR_RANGE, u); s0 = -1; }
         v0 = s0 >= 0;
         if (v0) {
             const size_t row = (size_t)b * p.N + s0;
@@ -925,10 +930,12 @@ __global__ void __launch_bounds__(kSlThreads, 1)
     __syncthreads();   // the barriers (initialised by thread 0) and the TMEM address are set
 
     int t = p.q_pos[u];
-    const bool t_ok = t >= 0 && t < p.N;
+    int tg = last_entry(t, p.m);   // the last global entry the query reads
+    const bool t_ok = t >= 0 && tg < p.N;
     if (!t_ok) {
         if (tid == 0 && rank == 0) report(p.status, CSA2_ERR_RANGE, u);
         t = -1;
+        tg = -1;
     }
     const int base = p.local_base[b];
     const int lo_w = max(max(base, t - p.W + 1), 0);
@@ -957,7 +964,7 @@ __global__ void __launch_bounds__(kSlThreads, 1)
             const int lb = j >> 7;
             const int e = (rank + lb * CS) * kTileKeys + (j & 127);
             int s = (lb < nb && e < p.k) ? __ldcg(p.topk + (size_t)u * p.k + e) : -1;
-            if (s >= 0 && (s > t || s >= p.N)) {
+            if (s >= 0 && (s > tg || s >= p.N)) {
                 report(p.status, CSA2_ERR_RANGE, u);
                 s = -1;
             }
@@ -1311,6 +1318,7 @@ csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* ticke
     p.tickets = tickets;
     p.part = static_cast<float*>(scratch);
     p.status = d_status;
+    p.m = a.m;
     cudaError_t e;
     if (pl.HQP == 16 && a.D == 128) e = launch_attn_variant<16, 128>(p, pl.units, stream);
     else if (pl.HQP == 16 && a.D == 64) e = launch_attn_variant<16, 64>(p, pl.units, stream);
@@ -1418,6 +1426,7 @@ csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, in
     p.tickets = nullptr;
     p.status = d_status;
     p.list_ready = list_ready;
+    p.m = a.m;
     CUtensorMap km, vm;
     memset(&km, 0, sizeof(km));
     memset(&vm, 0, sizeof(vm));
@@ -1489,6 +1498,7 @@ csa2_status launch_attn_slice(const csa2_attn_args& a, const int32_t* topk, int 
     p.tickets = nullptr;
     p.status = d_status;
     p.list_ready = list_ready;
+    p.m = a.m;
     CUtensorMap km, vm;
     memset(&km, 0, sizeof(km));
     memset(&vm, 0, sizeof(vm));

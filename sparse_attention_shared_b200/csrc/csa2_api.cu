@@ -60,6 +60,8 @@ int append_max_layers();
 // fp4_quant.cu
 cudaError_t launch_fp4_quantize(const float* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales,
                                 cudaStream_t stream);
+cudaError_t launch_fp4_compress(const float* x, int64_t groups, int m, int D, uint8_t* codes, uint8_t* scales,
+                                cudaStream_t stream);
 
 static size_t a256(size_t x) { return (x + 255) / 256 * 256; }
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -70,6 +72,7 @@ static csa2_status check_index(const csa2_index_args* a, bool in_stack) {
     if (a->B < 1 || a->Tq < 1 || a->N < 1 || a->N >= (1 << 27)) return CSA2_ERR_SHAPE;
     if ((int64_t)a->B * a->Tq > (1 << 26)) return CSA2_ERR_SHAPE;
     if (a->Hi < 1 || a->Hi > 16 || a->Di < 16 || a->Di > 128 || a->Di % 16) return CSA2_ERR_SHAPE;
+    if (a->m < 0 || a->m > 8) return CSA2_ERR_SHAPE;
     if (a->k < 1 || a->P < 0) return CSA2_ERR_SHAPE;
     if (a->mode == CSA2_FULL && a->P > 0 && a->k > a->P) return CSA2_ERR_SHAPE;
     if (!a->q_pos || !a->qi || !a->w || !a->ki || !a->topk_out) return CSA2_ERR_NULL;
@@ -94,6 +97,7 @@ static csa2_status check_attn(const csa2_attn_args* a, bool in_stack) {
     if ((int64_t)a->B * a->Tq > 65535) return CSA2_ERR_UNSUPPORTED;
     if (a->Hq < 1 || a->Hq > 32) return CSA2_ERR_UNSUPPORTED;
     if (a->D != 64 && a->D != 128) return CSA2_ERR_UNSUPPORTED;
+    if (a->m < 0 || a->m > 8) return CSA2_ERR_SHAPE;
     if ((!in_stack && a->k < 1) || a->W < 0 || a->Lloc < 0) return CSA2_ERR_SHAPE;
     if ((int64_t)a->k + a->W > 16384) return CSA2_ERR_UNSUPPORTED;   // the merge keeps <= 128 tile weights
     if (!a->q_pos || !a->q || !a->kv_fp4 || !a->kv_scale || !a->out) return CSA2_ERR_NULL;
@@ -125,7 +129,7 @@ static csa2_status check_stack(const csa2_stack_args* s) {
             if (ix.mode == CSA2_REINDEX && !have_pool) return CSA2_ERR_MODE;
             csa2_status st = check_index(&ix, true);
             if (st != CSA2_OK) return st;
-            if (ix.B != a0.B || ix.Tq != a0.Tq || ix.N != a0.N) return CSA2_ERR_SHAPE;
+            if (ix.B != a0.B || ix.Tq != a0.Tq || ix.N != a0.N || ix.m != a0.m) return CSA2_ERR_SHAPE;
             have_list = true;
             if (ix.mode == CSA2_FULL && ix.P > 0) have_pool = true;
         }
@@ -284,6 +288,16 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
         if (st != CSA2_OK) return st;
     }
     return CSA2_OK;
+}
+
+csa2_status csa2_fp4_compress(const float* x, int64_t groups, int32_t m, int32_t D, uint8_t* fp4, uint8_t* scale,
+                              void* stream) {
+    if (!x || !fp4 || !scale) return CSA2_ERR_NULL;
+    if (groups < 0 || D < 16 || D % 16 || (m != 1 && m != 2 && m != 4 && m != 8)) return CSA2_ERR_SHAPE;
+    if (!al16(x) || !al16(fp4) || !al16(scale)) return CSA2_ERR_ALIGN;
+    return launch_fp4_compress(x, groups, m, D, fp4, scale, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? CSA2_OK
+               : CSA2_ERR_CUDA;
 }
 
 csa2_status csa2_cache_append(const csa2_append_args* a, int32_t* d_status, void* stream) {

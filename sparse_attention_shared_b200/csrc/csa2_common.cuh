@@ -25,6 +25,13 @@ __device__ __forceinline__ void report(int32_t* st, int code, int detail) {
     }
 }
 
+// Last global entry a query at position t may read ("CED: Continuing Context with a
+// Causal Encoder and Decoder", "What Does the Sequence Compression Rate Reduce?"):
+// with compression rate m >= 2, entry j combines positions m j .. m j + m - 1 and
+// is read once all of them are <= t (complete groups); with m <= 1 entries are
+// positions. Negative for a query that can read no entry yet.
+__host__ __device__ __forceinline__ int last_entry(int t, int m) { return m >= 2 ? (t + 1) / m - 1 : t; }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -85,6 +85,7 @@ struct IdxParams {
     const uint8_t* pf_fp4;
     const uint8_t* pf_scale;
     int pf_N, pf_code_bytes, pf_scale_bytes;
+    int m;                   // sequence compression rate of the global entries (<= 1: one per position)
     long long wait_budget;   // SM cycles a CTA waits at a group barrier before it reports a timeout
     int skip_arrival;        // fault injection: the last CTA of a group never arrives at its first barrier
     int* ctrl;           // [slots][kCtrlInts]
@@ -1547,11 +1548,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int u = group; u < p.units; u += p.groups, ++j) {
         const int b = u / p.Tq;
         int t = p.q_pos[u];
-        if (t < 0 || t >= p.N) {
+        int tg = last_entry(t, p.m);   // the last global entry the query reads
+        if (t < 0 || tg >= p.N) {
             if (tid == 0 && cta == 0) report(p.status, CSA2_ERR_RANGE, u);
             t = -1;
+            tg = -1;
         }
-        const int n_all = t + 1;
+        const int n_all = tg + 1;
         const int lo = min(cta * p.chunk, n_all);
         const int my_n = min(lo + p.chunk, n_all) - lo;
         const int nst = p.pre ? 0 : (my_n + kRows - 1) / kRows;   // select only: no key tiles
@@ -1730,6 +1733,7 @@ constexpr int kMqMinN = 8192;                             // ... on a key set of
 
 struct MqParams {
     int B, Tq, N, Hi, nblk, splits;
+    int m;               // sequence compression rate of the global entries
     int32_t w[8];
     const int32_t* q_pos;
     const int8_t* qi;
@@ -1788,7 +1792,8 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         int t = -1;
         if (tid < nq) {
             t = p.q_pos[(size_t)b * p.Tq + j0 + tid];
-            if (t < 0 || t >= p.N) t = -1;   // no scores; the select kernel reports the position
+            const int tg = last_entry(t, p.m);
+            t = (t < 0 || tg >= p.N) ? -1 : tg;   // no scores past the last entry; the select kernel reports a bad position
         }
         S.tq[tid] = t;
     }
@@ -1931,12 +1936,14 @@ __global__ void __launch_bounds__(kSel, 1)
         const int nq = p.Hi * p.Di / 16;   // int4 chunks of the index query (<= 128)
         const int4 qv = tid < nq ? reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * p.Di)[tid] : make_int4(0, 0, 0, 0);
         int t = p.q_pos[u];
-        const bool bad_t = (t < 0 || t >= p.N);
+        int tg = last_entry(t, p.m);   // the last global entry the query reads
+        const bool bad_t = (t < 0 || tg >= p.N);
         if (bad_t) {
             if (tid == 0 && cta == 0) report(p.status, CSA2_ERR_RANGE, u);
             t = -1;
+            tg = -1;
         }
-        const int n_all = full ? (t + 1) : (bad_t ? 0 : p.P_in);
+        const int n_all = full ? (tg + 1) : (bad_t ? 0 : p.P_in);
         const int lo = min(cta * p.chunk, n_all);
         const int hi = min(lo + p.chunk, n_all);
 
@@ -1999,7 +2006,7 @@ __global__ void __launch_bounds__(kSel, 1)
                 for (int q2 = 0; q2 < RB; ++q2) {
                     const int e = e0 + q2 * kSel + tid;
                     sidx[q2] = (e0 == 0) ? sidx0[q2] : ((e < my_n) ? __ldg(pool + lo + e) : -1);
-                    okr[q2] = e < my_n && sidx[q2] >= 0 && sidx[q2] <= t;
+                    okr[q2] = e < my_n && sidx[q2] >= 0 && sidx[q2] <= tg;
                     if (e < my_n && !okr[q2]) first_bad = min(first_bad, e);
                     if (okr[q2]) {
                         const int4* row = reinterpret_cast<const int4*>(kb + (size_t)sidx[q2] * p.Di);
@@ -2259,6 +2266,7 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
         p.pf_scale_bytes = pf->D / 16;
     }
     p.keys_ready = keys_ready;
+    p.m = a.m;
     p.status = d_status;
     p.wait_budget = group_wait_budget();
     p.skip_arrival = group_skip_arrival();
@@ -2309,6 +2317,7 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
         mp.splits = std::max(1, std::min(sms / std::max(items, 1), (a.N / kMqRows + 7) / 8));
         for (int h = 0; h < 8; ++h) mp.w[h] = h < a.Hi ? a.w[h] : 0;
         mp.q_pos = a.q_pos; mp.qi = a.qi;
+        mp.m = a.m;
         mp.scores = static_cast<int32_t*>(scratch);
         mp.sstride = pl.pstride;
         mp.status = d_status;

@@ -56,6 +56,7 @@ struct RxParams {
     const int32_t* pool;
     int32_t* topk_out;
     int pool_ready;      // the pool and the keys were complete before the previous kernel began
+    int m;               // sequence compression rate of the global entries
     const uint8_t* pf_fp4;
     const uint8_t* pf_scale;
     int pf_N, pf_code_bytes, pf_scale_bytes;
@@ -196,8 +197,8 @@ __global__ void __launch_bounds__(kRxThreads, 1) index_reindex_cl_kernel(const _
     const int b = u / p.Tq;
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");   // waited on before the first push
 
-    int t = p.q_pos[u];
-    const bool t_ok = t >= 0 && t < p.N;
+    int t = last_entry(p.q_pos[u], p.m);   // the last global entry the query reads
+    const bool t_ok = p.q_pos[u] >= 0 && t < p.N;
     if (!t_ok) {
         if (tid == 0 && rank == 0) report(p.status, CSA2_ERR_RANGE, u);
         t = -1;
@@ -415,6 +416,7 @@ csa2_status launch_reindex_cl(const csa2_index_args& a, const int32_t* pool_in, 
     p.pool = pool_in;
     p.topk_out = a.topk_out;
     p.pool_ready = pool_ready;
+    p.m = a.m;
     if (pf != nullptr && pf->kv_fp4 != nullptr && pf->kv_scale != nullptr && pf->B == a.B) {
         p.pf_fp4 = pf->kv_fp4;
         p.pf_scale = pf->kv_scale;

@@ -69,6 +69,19 @@ class Status:
             raise capi.Csa2Error(code, f"{where} (detail {detail})")
 
 
+def fp4_compress(x: torch.Tensor, m: int, stream=None):
+    """fp32 [groups * m, D] -> FP4 entries of compression rate m (the mean of m rows):
+    (codes uint8 [groups, D/2], scales uint8 [groups, D/16])."""
+    _need_cuda(x)
+    x = x.contiguous()
+    D = x.shape[-1]
+    groups = x.numel() // D // m
+    codes = torch.empty((groups, D // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((groups, D // 16), dtype=torch.uint8, device=x.device)
+    check(capi.csa2_fp4_compress(_ptr(x), groups, m, D, _ptr(codes), _ptr(scales), _stream(stream)), "csa2_fp4_compress")
+    return codes, scales
+
+
 def fp4_quantize(x: torch.Tensor, stream=None):
     """fp32 [rows, D] -> (codes uint8 [rows, D/2], scales uint8 [rows, D/16])."""
     _need_cuda(x)
@@ -82,7 +95,7 @@ def fp4_quantize(x: torch.Tensor, stream=None):
 
 
 def make_index_args(mode: int, q_pos, qi, w_host: np.ndarray, ki, k: int, P: int = 0, pool_in=None,
-                    pool_out=None, topk_out=None) -> IndexArgs:
+                    pool_out=None, topk_out=None, m: int = 0) -> IndexArgs:
     B, Tq, Hi, Di = qi.shape
     a = IndexArgs()
     a.B, a.Tq, a.N, a.Hi, a.Di, a.k, a.P, a.mode = B, Tq, ki.shape[1], Hi, Di, k, P, mode
@@ -91,19 +104,21 @@ def make_index_args(mode: int, q_pos, qi, w_host: np.ndarray, ki, k: int, P: int
     a.pool_in = _ptr(pool_in)
     a.P_in = 0 if pool_in is None else int(pool_in.shape[-1])
     a.pool_out, a.topk_out = _ptr(pool_out), _ptr(topk_out)
+    a.m = m
     return a
 
 
 def index_topk(mode: str, q_pos, qi, w, ki, k: int, P: int = 0, pool_in=None, ws: Workspace = None,
-               status: Status = None, stream=None):
+               status: Status = None, stream=None, m: int = 0):
     """Full or Reindex top-k. Returns (pool or None, topk) as int32 tensors."""
     _need_cuda(q_pos, qi, ki, pool_in)
-    m = capi.MODES[mode]
+    mode_id = capi.MODES[mode]
     B, Tq = qi.shape[:2]
     w_host = np.ascontiguousarray(np.asarray(w if not torch.is_tensor(w) else w.cpu().numpy(), dtype=np.int32))
     topk = torch.empty((B, Tq, k), dtype=torch.int32, device=qi.device)
-    pool = torch.empty((B, Tq, P), dtype=torch.int32, device=qi.device) if (m == capi.CSA2_FULL and P > 0) else None
-    a = make_index_args(m, q_pos, qi, w_host, ki, k, P if m == capi.CSA2_FULL else 0, pool_in, pool, topk)
+    pool = torch.empty((B, Tq, P), dtype=torch.int32, device=qi.device) if (mode_id == capi.CSA2_FULL and P > 0) else None
+    a = make_index_args(mode_id, q_pos, qi, w_host, ki, k, P if mode_id == capi.CSA2_FULL else 0, pool_in, pool,
+                        topk, m)
     ws = ws or Workspace(str(qi.device))
     nbytes = capi.csa2_workspace_bytes(0, a)
     buf = ws.get(nbytes)
@@ -112,7 +127,7 @@ def index_topk(mode: str, q_pos, qi, w, ki, k: int, P: int = 0, pool_in=None, ws
     return pool, topk
 
 
-def make_attn_args(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base, W: int, out, lse) -> AttnArgs:
+def make_attn_args(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base, W: int, out, lse, m: int = 0) -> AttnArgs:
     B, Tq, Hq, D = q.shape
     a = AttnArgs()
     a.B, a.Tq, a.N, a.Hq, a.D = B, Tq, kv_fp4.shape[1], Hq, D
@@ -122,17 +137,18 @@ def make_attn_args(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base, W: int,
     a.q_pos, a.q, a.kv_fp4, a.kv_scale = _ptr(q_pos), _ptr(q), _ptr(kv_fp4), _ptr(kv_scale)
     a.topk, a.kl, a.vl, a.local_base = _ptr(topk), _ptr(kl), _ptr(vl), _ptr(local_base)
     a.out, a.lse = _ptr(out), _ptr(lse)
+    a.m = m
     return a
 
 
 def sparse_attn(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base, W: int, ws: Workspace = None,
-                status: Status = None, stream=None):
+                status: Status = None, stream=None, m: int = 0):
     """Attention over the listed global FP4 rows plus the window. Returns (out bf16, lse fp32)."""
     _need_cuda(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base)
     B, Tq, Hq, D = q.shape
     out = torch.empty((B, Tq, Hq, D), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=q.device)
-    a = make_attn_args(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base, W, out, lse)
+    a = make_attn_args(q_pos, q, kv_fp4, kv_scale, topk, kl, vl, local_base, W, out, lse, m)
     ws = ws or Workspace(str(q.device))
     buf = ws.get(capi.csa2_workspace_bytes(1, a))
     st = status.ptr if status is not None else 0
@@ -193,7 +209,7 @@ class LayerStack:
     """
 
     def __init__(self, layers: Sequence[Dict], q_pos, kv_fp4, kv_scale, local_base,
-                 keep_reuse_lists: bool = False, with_lse: bool = True, packed_outputs: bool = False):
+                 keep_reuse_lists: bool = False, with_lse: bool = True, packed_outputs: bool = False, m: int = 0):
         dev = q_pos.device
         self.out_buf = None
         packed = None
@@ -228,7 +244,7 @@ class LayerStack:
                 topk = torch.empty((B, Tq, cur_k), dtype=torch.int32, device=dev)
                 if P > 0:
                     pool = torch.empty((B, Tq, P), dtype=torch.int32, device=dev)
-                idx_arr[l] = make_index_args(mode, q_pos, d["qi"], w_host, d["ki"], cur_k, P, None, pool, topk)
+                idx_arr[l] = make_index_args(mode, q_pos, d["qi"], w_host, d["ki"], cur_k, P, None, pool, topk, m)
             else:
                 if keep_reuse_lists:
                     topk = torch.empty((B, Tq, cur_k), dtype=torch.int32, device=dev)
@@ -243,7 +259,8 @@ class LayerStack:
                 out = torch.empty((B, Tq, Hq, D), dtype=torch.bfloat16, device=dev)
                 lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev) if with_lse else None
             kl, vl = d.get("kl"), d.get("vl")
-            attn_arr[l] = make_attn_args(q_pos, q, kv_fp4, kv_scale, None, kl, vl, local_base, int(d["W"]), out, lse)
+            attn_arr[l] = make_attn_args(q_pos, q, kv_fp4, kv_scale, None, kl, vl, local_base, int(d["W"]), out, lse,
+                                         m)
             self.keep.extend([d.get("qi"), d.get("ki"), q, kl, vl])
             self.pools.append(pool)
             self.topks.append(topk)

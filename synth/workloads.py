@@ -48,20 +48,25 @@ class WorkloadSpec:
     layers: tuple
     description: str = ""
     replay: bool = False  # bounded replay: local KV exists only for the Tq replayed positions
+    m: int = 1            # sequence compression rate: N global entries cover m * N positions
 
     @property
     def L(self) -> int:
         return len(self.layers)
 
     @property
+    def n_pos(self) -> int:
+        return self.m * self.N
+
+    @property
     def local_base(self) -> int:
         if self.replay:
-            return self.N - self.Tq
-        return max(0, self.N - self.Tq - self.W + 1)
+            return self.n_pos - self.Tq
+        return max(0, self.n_pos - self.Tq - self.W + 1)
 
     @property
     def Lloc(self) -> int:
-        return self.N - self.local_base
+        return self.n_pos - self.local_base
 
     @property
     def n_key_sets(self) -> int:
@@ -126,6 +131,12 @@ CONFIGS: Dict[str, WorkloadSpec] = {
         description="bounded-replay prefill: the last 512 of 131072 prompt positions of 4 seqs replayed "
                     "through 20 layers [Full,Reuse,Reuse,Reindex]x5 (pool 8192, top-2048), window 512 "
                     "with references before the replayed segment cut"),
+    "encoder_m2": WorkloadSpec(
+        "encoder_m2", B=16, N=65536, Tq=1, Hq=16, D=128, Hi=8, Di=64, W=512,
+        layers=_stack20_layers(), m=2,
+        description="encoder-side CSA2 at sequence compression rate 2: 16 seqs x 131072 positions in 65536 "
+                    "global entries (each the mean of two positions), 20 layers [Full,Reuse,Reuse,Reindex]x5, "
+                    "pool 8192, top-2048, SWA 512 over positions"),
     "paper_schedule": WorkloadSpec(
         "paper_schedule", B=16, N=131072, Tq=1, Hq=16, D=128, Hi=8, Di=64, W=128,
         layers=_paper_layers(),
@@ -160,16 +171,17 @@ class Workload:
     def q_pos(self) -> np.ndarray:
         s = self.spec
         return self._get("q_pos", lambda: np.broadcast_to(
-            np.arange(s.N - s.Tq, s.N, dtype=np.int32), (s.B, s.Tq)).copy())
+            np.arange(s.n_pos - s.Tq, s.n_pos, dtype=np.int32), (s.B, s.Tq)).copy())
 
     def local_base_arr(self) -> np.ndarray:
         s = self.spec
         return self._get("local_base", lambda: np.full((s.B,), s.local_base, dtype=np.int32))
 
     def kv_f32(self) -> np.ndarray:
-        """Global KV before quantisation: [B, N, D] fp32, N(0,1)."""
+        """Global KV before quantisation (and, at compression rate m > 1, before the
+        entries are formed): [B, m * N, D] fp32 per position, N(0,1)."""
         s = self.spec
-        return self._get("kv", lambda: normal_f32(self.seed, _TID_KV, (s.B, s.N, s.D)))
+        return self._get("kv", lambda: normal_f32(self.seed, _TID_KV, (s.B, s.n_pos, s.D)))
 
     def ki(self, key_set: int) -> np.ndarray:
         """int8 index keys [B, N, Di]."""

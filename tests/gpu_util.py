@@ -33,7 +33,10 @@ class DeviceWorkload:
         self.q_pos = dev(wl.q_pos())
         self.local_base = dev(wl.local_base_arr())
         kv = dev(wl.kv_f32())
-        self.kv_fp4, self.kv_scale = ops.fp4_quantize(kv.view(-1, s.D))
+        if s.m > 1:
+            self.kv_fp4, self.kv_scale = ops.fp4_compress(kv.view(-1, s.D), s.m)
+        else:
+            self.kv_fp4, self.kv_scale = ops.fp4_quantize(kv.view(-1, s.D))
         self.kv_fp4 = self.kv_fp4.view(s.B, s.N, s.D // 2)
         self.kv_scale = self.kv_scale.view(s.B, s.N, s.D // 16)
         del kv

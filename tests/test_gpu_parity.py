@@ -376,7 +376,8 @@ def _check_stack_every_unit(wl, ws, status):
     from oracle import cpp as C
     s = wl.spec
     dw = DeviceWorkload(wl)
-    st = ops.LayerStack(dw.layer_dicts(), dw.q_pos, dw.kv_fp4, dw.kv_scale, dw.local_base, keep_reuse_lists=False)
+    st = ops.LayerStack(dw.layer_dicts(), dw.q_pos, dw.kv_fp4, dw.kv_scale, dw.local_base, keep_reuse_lists=False,
+                        m=s.m)
     st.run(ws, status)
     torch.cuda.synchronize()
     status.check("stack")
@@ -389,7 +390,8 @@ def _check_stack_every_unit(wl, ws, status):
         if st.pools[li] is not None:
             assert_list_invariants(st.pools[li].cpu().numpy(), q_pos, f"layer {li} pool")
             assert_lists_equal(st.pools[li], e["pool"], f"layer {li} pool, every unit")
-    codes, scales = C.fp4_quantize(wl.kv_f32())
+    kv = wl.kv_f32() if s.m <= 1 else C.compress_entries(wl.kv_f32(), s.m)
+    codes, scales = C.fp4_quantize(kv)
     assert_lists_equal(dw.kv_fp4, codes, "FP4 codes of the cache")
     assert_lists_equal(dw.kv_scale, scales, "E4M3 scales of the cache")
     outs = C.stack_outputs(wl, codes, scales, lists, range(s.B))
@@ -429,3 +431,26 @@ def test_replay_prefill_every_unit(ws, status):
     wl = synth.make_workload("replay_prefill", B=2, N=16384, Tq=256, W=256)
     assert wl.spec.local_base == 16384 - 256
     _check_stack_every_unit(wl, ws, status)
+
+
+def test_encoder_m2_every_unit(ws, status):
+    # sequence compression rate 2: 4096 entries (each the mean of two positions) for 8192 positions; queries
+    # at an odd and an even position read only complete entries
+    wl = synth.make_workload("encoder_m2", B=3, N=4096, Tq=2)
+    assert wl.spec.n_pos == 8192
+    _check_stack_every_unit(wl, ws, status)
+
+
+def test_encoder_m2_early_positions(ws, status):
+    """Queries at positions 0..5 with m = 2 read entries 0..(t+1)/2-1: none at t = 0."""
+    B, Nent, m = 1, 64, 2
+    qi = synth.randint_i8(12, 1, (B, 6, 8, 64))
+    ki = synth.randint_i8(12, 2, (B, Nent, 64))
+    w = synth.randint_i32(12, 3, (8,), 1, 8)
+    q_pos = np.arange(6, dtype=np.int32)[None, :]
+    _, topk = ops.index_topk("FULL", dev(q_pos), dev(qi), w, dev(ki), 4, ws=ws, status=status, m=m)
+    got = topk.cpu().numpy()
+    for j in range(6):
+        _, ref = O.index_full(qi[0, j], w, ki[0], j, 4, 0, m)
+        assert np.array_equal(got[0, j], ref)
+        assert (got[0, j] >= 0).sum() == min(4, (j + 1) // 2)
