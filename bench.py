@@ -351,8 +351,10 @@ def run_ours(args, rank, world, local_rank):
     except Exception:  # noqa: BLE001
         pass
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    bf16_peak = float(peaks.get("bf16_tflops", 1590.0))
+    int8_peak = 2.0 * bf16_peak   # the nominal dense int8 : bf16 ratio (4.5 : 2.25 PFLOP/s) times the measured bf16
     kernels = kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales, base, qp_host, base_host,
-                               ws, st, flush, stream, hbm_peak)
+                               ws, st, flush, stream, hbm_peak, bf16_peak, int8_peak)
     traffic_db = {}
     try:
         traffic_db = json.load(open(os.path.join(ROOT, "profiles", "traffic.json"))).get(args.workload, {})
@@ -361,10 +363,18 @@ def run_ours(args, rank, world, local_rank):
     for kc in kernels:
         kc["traffic"] = traffic_db.get(kc["class"], {}).get("bytes_per_launch")
     top = max(kernels, key=lambda kc: kc["share"])
-    roofline = {"bound": "hbm", "achieved": top["gbs"], "peak": hbm_peak, "unit": "GB/s", "frac": top["frac"],
-                "traffic": top["traffic"], "kernel": top["kernel"], "class": top["class"],
-                "kernel_ms": top["ms"], "algorithmic_bytes": top["algorithmic_bytes"], "share": top["share"],
-                "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback 6650 GB/s"}
+    if top.get("tensor_frac", 0.0) > top["frac"]:   # the tensor pipe is the tighter bound
+        roofline = {"bound": "tensor", "achieved": top["tensor_tops"], "peak": top["tensor_peak_tops"],
+                    "unit": "TFLOP/s" if top["tensor_kind"] == "bf16" else "TOPS (int8)", "frac": top["tensor_frac"],
+                    "traffic": top["traffic"], "kernel": top["kernel"], "class": top["class"], "kernel_ms": top["ms"],
+                    "algorithmic_ops": top["tensor_ops"], "share": top["share"],
+                    "peak_source": ("MEASURED_PEAKS.json bf16_tflops (measured)" if peaks else "fallback 1590 TFLOP/s")
+                    + (" x 2 (nominal int8 : bf16 dense ratio)" if top["tensor_kind"] == "int8" else "")}
+    else:
+        roofline = {"bound": "hbm", "achieved": top["gbs"], "peak": hbm_peak, "unit": "GB/s", "frac": top["frac"],
+                    "traffic": top["traffic"], "kernel": top["kernel"], "class": top["class"],
+                    "kernel_ms": top["ms"], "algorithmic_bytes": top["algorithmic_bytes"], "share": top["share"],
+                    "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback 6650 GB/s"}
     # the lists of the last timed step (the same inputs every step)
     host = lambda ts: [t.cpu().numpy() if t is not None else None for t in ts]
     step_bytes = list_bytes(s, qp_host, base.cpu().numpy(), host(stack.pools), host(stack.topks))
@@ -451,7 +461,7 @@ def reindex_call_bytes(spec, pool, k):
 
 
 def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales, base, qp_host, base_host, ws, st,
-                     flush, stream, hbm_peak):
+                     flush, stream, hbm_peak, bf16_peak, int8_peak):
     """Each kernel class of one step, timed alone through the public calls on the
     step's own tensors: the Full-mode indexer, the Reindex indexer, and attention for
     a Full, a Reuse and a Reindex layer. Per class: ms per launch, launches per step,
@@ -464,10 +474,15 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
     n = args.kernel_launches
     out = []
 
-    def entry(cls, kernel, ms, count, nbytes):
+    def entry(cls, kernel, ms, count, nbytes, ops=0, ops_peak=None, ops_kind=None):
         gbs = nbytes / (ms * 1e-3) / 1e9
-        out.append({"class": cls, "kernel": kernel, "ms": round(ms, 5), "launches_per_step": count,
-                    "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)})
+        e = {"class": cls, "kernel": kernel, "ms": round(ms, 5), "launches_per_step": count,
+             "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)}
+        if ops and ops_peak:
+            tops = ops / (ms * 1e-3) / 1e12
+            e.update({"tensor_ops": int(ops), "tensor_kind": ops_kind, "tensor_tops": round(tops, 2),
+                      "tensor_peak_tops": round(ops_peak, 1), "tensor_frac": round(tops / ops_peak, 4)})
+        out.append(e)
 
     w_host = np.ascontiguousarray(np.asarray(d0["w"], dtype=np.int32))
     pool_t = torch.empty((s.B, s.Tq, max(Lf.P, 1)), dtype=torch.int32, device="cuda")
@@ -479,10 +494,12 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
     ms = time_alone(args, torch, fcall, flush, stream, n)
     st.check("Full indexer timing")
     mq = s.Tq >= 4 and s.N >= 8192 and s.Hi <= 8 and s.Di in (32, 64, 128)
-    kname = (f"index_full_tc_kernel<{s.Di}>" if s.Di in (32, 64, 128) else "index_dp4a_kernel<0,0>")
+    kname = (f"index_full_cl_kernel<{s.Di}>" if s.Di in (32, 64, 128) else "index_dp4a_kernel<0,0>")
     if mq:
-        kname = f"index_mq_score_kernel<{s.Di}> + {kname} (select only)"
-    entry("full_index", kname, ms, n_launch["FULL"], full_launch_bytes(s, qp_host))
+        kname = f"index_mq_score_kernel<{s.Di}> + index_full_tc_kernel<{s.Di}> (select only)"
+    # the contraction the scan performs, counted over the causal pairs only: 2 * Hi * Di per (query, key)
+    int8_ops = 2 * s.Hi * s.Di * sum(entries_read(s, int(t)) for t in qp_host.reshape(-1))
+    entry("full_index", kname, ms, n_launch["FULL"], full_launch_bytes(s, qp_host), int8_ops, int8_peak, "int8")
     topk_h = topk_t.cpu().numpy()
 
     def attn_entry(cls, li, topk_dev, topk_host, count):
@@ -495,7 +512,15 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
         t = time_alone(args, torch, acall, flush, stream, n)
         st.check(f"attention timing ({cls})")
         HQP = 16 if s.Hq <= 16 else 32
-        entry(cls, f"sparse_attn_cl_kernel<{HQP},{s.D}>", t, count, attn_call_bytes(s, qp_host, base_host, topk_host))
+        # S = K Q^T and O = P V over the query's union: 4 * Hq * D flops per (query, entry)
+        n_ent = int((topk_host >= 0).sum())
+        if s.W > 0:
+            t_all = qp_host.reshape(-1).astype(np.int64)
+            lo = np.maximum(np.maximum(t_all - s.W + 1, np.repeat(base_host.astype(np.int64), s.Tq)), 0)
+            n_ent += int(np.maximum(t_all - lo + 1, 0).sum())
+        flops = 4 * s.Hq * s.D * n_ent
+        entry(cls, f"sparse_attn_sl_kernel<{HQP},{s.D}>", t, count, attn_call_bytes(s, qp_host, base_host, topk_host),
+              flops, bf16_peak, "bf16")
 
     attn_entry("attn_full", li_f, topk_t, topk_h, n_launch["FULL"])
     if n_launch["REUSE"]:
@@ -511,8 +536,8 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
         rcall = lambda sp: capi.csa2_index_topk(ra, int(rbuf.data_ptr()), rbuf.numel(), st.ptr, sp)
         ms = time_alone(args, torch, rcall, flush, stream, n)
         st.check("Reindex timing")
-        rk = ("index_dp4a_kernel<8,64>" if (s.Hi <= 8 and s.Di == 64) else
-              "index_dp4a_kernel<4,32>" if (s.Hi <= 4 and s.Di == 32) else "index_dp4a_kernel<0,0>")
+        rk = (f"index_reindex_cl_kernel<{8 if s.Hi <= 8 else 16},{s.Di}>" if s.Di in (32, 64, 128)
+              else "index_dp4a_kernel<0,0>")
         entry("reindex_index", rk, ms, n_launch["REINDEX"], reindex_call_bytes(s, pool_t.cpu().numpy(), Lr.k))
         attn_entry("attn_reindex", li_r, topk_r, topk_r.cpu().numpy(), n_launch["REINDEX"])
     tot = sum(kc["ms"] * kc["launches_per_step"] for kc in out)
