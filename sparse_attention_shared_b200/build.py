@@ -24,8 +24,15 @@ def _stale(obj: str, src: str) -> bool:
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    objdir = os.path.join(HERE, "_build")
+LIB_CHECKED = os.path.join(HERE, "libcsa2_checked.so")
+
+
+def build(force: bool = False, verbose: bool = False, extra=None, checked: bool = False) -> str:
+    """Build libcsa2.so, or with checked=True the range-checked libcsa2_checked.so
+    (-DCSA2_CHECKED: computed indices are checked and reported instead of accessed)."""
+    lib = LIB_CHECKED if checked else LIB
+    extra = list(extra or []) + (["-DCSA2_CHECKED"] if checked else [])
+    objdir = os.path.join(HERE, "_build_checked" if checked else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs, changed = [], False
     for src in SOURCES:
@@ -33,20 +40,20 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
         o = os.path.join(objdir, src.replace(".cu", ".o"))
         objs.append(o)
         if force or _stale(o, s):
-            cmd = [NVCC, *FLAGS, *(extra or []), "-c", s, "-o", o]
+            cmd = [NVCC, *FLAGS, *extra, "-c", s, "-o", o]
             if verbose:
                 print(" ".join(cmd), flush=True)
             subprocess.check_call(cmd)
             changed = True
-    if changed or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if changed or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs, "-lcudart"]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
+    build(force="--force" in sys.argv, verbose=True, checked="--checked" in sys.argv)

@@ -64,8 +64,13 @@ EXPORTED = ("csa2_workspace_bytes", "csa2_index_topk", "csa2_sparse_attn", "csa2
             "csa2_fp4_compress")
 
 
+def checked_library() -> bool:
+    """CSA2_LIBRARY=checked selects the range-checked build (libcsa2_checked.so)."""
+    return os.environ.get("CSA2_LIBRARY", "") == "checked"
+
+
 def library_path() -> str:
-    return os.path.join(_HERE, "libcsa2.so")
+    return os.path.join(_HERE, "libcsa2_checked.so" if checked_library() else "libcsa2.so")
 
 
 def lib():
@@ -75,7 +80,7 @@ def lib():
         if _lib is None:
             from . import build as _build
             try:
-                path = _build.build()
+                path = _build.build(checked=checked_library())
             except Exception as e:  # noqa: BLE001
                 raise RuntimeError(f"cannot build the CSA2 CUDA library: {e}") from e
             L = ctypes.CDLL(path)

@@ -1011,7 +1011,9 @@ __global__ void __launch_bounds__(kSlThreads, 1)
                     o.z = f16x2_mul(d[2], s2x);
                     o.w = f16x2_mul(d[3], s2x);
                 }
-                *reinterpret_cast<uint4*>(S.gtile + (c >> 3) * G::kGPanel + sw128(j, c & 7)) = o;
+                const uint32_t off = (c >> 3) * G::kGPanel + sw128(j, c & 7);
+                if (CSA2_CHECK(off + 16u <= sizeof(S.gtile), p.status, 2101))
+                    *reinterpret_cast<uint4*>(S.gtile + off) = o;
             }
         }
     };
@@ -1051,8 +1053,10 @@ __global__ void __launch_bounds__(kSlThreads, 1)
         v16.z = bf16x2_to_f16x2(v.z, f);
         v16.w = bf16x2_to_f16x2(v.w, f);
         const uint32_t off = (c >> 3) * (HQP * 128) + sw128(h, c & 7);
-        *reinterpret_cast<uint4*>(S.qf16 + off) = v16;
-        *reinterpret_cast<uint4*>(S.qbf16 + off) = v;
+        if (CSA2_CHECK(off + 16u <= (uint32_t)G::kQBytes, p.status, 2102)) {
+            *reinterpret_cast<uint4*>(S.qf16 + off) = v16;
+            *reinterpret_cast<uint4*>(S.qbf16 + off) = v;
+        }
         if (c == 0) S.qmul[h] = p.scale_log2 * __uint_as_float((uint32_t)(127 - k2) << 23);
     }
 
@@ -1077,8 +1081,9 @@ __global__ void __launch_bounds__(kSlThreads, 1)
                 if (c < D / 8) {
                     const uint16_t* src = (lane < 16 ? p.kl : p.vl) + ((size_t)b * p.Lloc + (t - base)) * D;
                     const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + c);
-                    uint8_t* dst = (lane < 16 ? S.kwin : S.vwin) + (c >> 3) * kPanelBytes + sw128(r0, c & 7);
-                    *reinterpret_cast<uint4*>(dst) = v;
+                    const uint32_t off = (c >> 3) * kPanelBytes + sw128(r0, c & 7);
+                    uint8_t* dst = (lane < 16 ? S.kwin : S.vwin) + off;
+                    if (CSA2_CHECK(off + 16u <= sizeof(S.kwin), p.status, 2104)) *reinterpret_cast<uint4*>(dst) = v;
                 }
             }
         }
@@ -1177,8 +1182,10 @@ __global__ void __launch_bounds__(kSlThreads, 1)
             const float mh = S.mfin[h];
             const float pv = (a[i][h] != -INFINITY && mh != -INFINITY) ? exp2f(a[i][h] - mh) : 0.f;
             ls[h] += pv;
-            *reinterpret_cast<uint16_t*>(pb + sw128(h, (key & 63) >> 3)) =
-                is_win ? __bfloat16_as_ushort(__float2bfloat16_rn(pv)) : __half_as_ushort(__float2half_rn(pv));
+            uint8_t* dst = pb + sw128(h, (key & 63) >> 3);
+            if (CSA2_CHECK(dst >= S.kwin && dst + 2 <= S.kwin + sizeof(S.kwin), p.status, 2103))
+                *reinterpret_cast<uint16_t*>(dst) =
+                    is_win ? __bfloat16_as_ushort(__float2bfloat16_rn(pv)) : __half_as_ushort(__float2half_rn(pv));
         }
     }
     {
@@ -1241,7 +1248,8 @@ __global__ void __launch_bounds__(kSlThreads, 1)
 #pragma unroll
         for (int h = 0; h < HQP; ++h) {
             if (h >= p.Hq) break;
-            st_dsmem(dsmem_addr(&S.recv_o[(h / CS) * CS + rank][tid], h % CS), live ? ov[h] : 0.f);
+            if (CSA2_CHECK((h / CS) * CS + rank < HQP + kSlMaxCluster, p.status, 2105))
+                st_dsmem(dsmem_addr(&S.recv_o[(h / CS) * CS + rank][tid], h % CS), live ? ov[h] : 0.f);
         }
     }
     if (tid < p.Hq) {

@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kAppendThreads) cache_append_kernel(const __gr
     }
     const uint4* kn = reinterpret_cast<const uint4*>(p.kl_new + ((size_t)l * p.B + b) * p.D);
     const uint4* vn = reinterpret_cast<const uint4*>(p.vl_new + ((size_t)l * p.B + b) * p.D);
+    if (!CSA2_CHECK(row >= 0 && row < p.Lcap, p.status, 2401)) return;
     for (int c = tid; c < cpr; c += kAppendThreads) {
         kl[(size_t)row * cpr + c] = kn[c];
         vl[(size_t)row * cpr + c] = vn[c];

@@ -25,6 +25,22 @@ __device__ __forceinline__ void report(int32_t* st, int code, int detail) {
     }
 }
 
+// Range-checked build (compiled with -DCSA2_CHECKED, library libcsa2_checked.so): a
+// computed shared- or global-memory index is checked before the access it guards; a
+// violation is reported as CSA2_ERR_RANGE with `detail` naming the site, and the
+// access is skipped. In the normal build the check is the constant true.
+#ifdef CSA2_CHECKED
+#define CSA2_CHECK(cond, st, detail) (::csa2::checked_ok((cond), (st), (detail)))
+#else
+#define CSA2_CHECK(cond, st, detail) (true)
+#endif
+
+__device__ __forceinline__ bool checked_ok(bool cond, int32_t* st, int detail) {
+    if (!cond) report(st, CSA2_ERR_RANGE, detail);
+    return cond;
+}
+
+
 // Last global entry a query at position t may read ("CED: Continuing Context with a
 // Causal Encoder and Decoder", "What Does the Sequence Compression Rate Reduce?"):
 // with compression rate m >= 2, entry j combines positions m j .. m j + m - 1 and

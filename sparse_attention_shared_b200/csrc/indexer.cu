@@ -2404,7 +2404,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int i = tid; i < C; i += kSel) {
                     int c = 0;
                     while (X.goff[tr][c + 1] <= i) ++c;
-                    X.gc[tr][i] = ld_dsmem_i32(&X.lc[tr][i - X.goff[tr][c]], c);
+                    if (CSA2_CHECK(i < kCandCap && c < G && i - X.goff[tr][c] < kCandCap, p.status, 2301))
+                        X.gc[tr][i] = ld_dsmem_i32(&X.lc[tr][i - X.goff[tr][c]], c);
                 }
             }
             sel_sync();

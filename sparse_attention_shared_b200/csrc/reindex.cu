@@ -253,6 +253,7 @@ __global__ void __launch_bounds__(kRxThreads, 1) index_reindex_cl_kernel(const _
         const int e = lo + i * kRxThreads + tid;
         if (e >= min(lo + p.slice, p.P_in)) continue;
         const int x = spos[i] >= 0 ? rx_score<HI, DI>(rows[i], qs, p.w) : 0;
+        if (!CSA2_CHECK(e < Pc, p.status, 2201)) continue;
         st_dsmem_i32(sc0 + 4u * (uint32_t)e, x);
         st_dsmem_i32(ps0 + 4u * (uint32_t)e, spos[i]);
     }
@@ -264,6 +265,7 @@ __global__ void __launch_bounds__(kRxThreads, 1) index_reindex_cl_kernel(const _
     int32_t* out = p.topk_out + (size_t)u * p.k;
     const bool pf = p.pf_fp4 != nullptr;
     auto emit = [&](int idx, int s) {
+        if (!CSA2_CHECK(idx >= 0 && idx < p.k, p.status, 2203)) return;
         out[idx] = s;
         if (pf) {
             const size_t row = (size_t)b * p.pf_N + s;
@@ -291,7 +293,10 @@ __global__ void __launch_bounds__(kRxThreads, 1) index_reindex_cl_kernel(const _
         const int above0 = M.info[1];
         const int32_t blo = rx_d0_lo(B0);
         for (int i = tid; i < n; i += kRxThreads)
-            if (ps[i] >= 0 && rx_d0(sc[i]) == B0) c1[atomicAdd(&M.cnt[0], 1)] = (uint16_t)i;
+            if (ps[i] >= 0 && rx_d0(sc[i]) == B0) {
+                const int slot = atomicAdd(&M.cnt[0], 1);
+                if (CSA2_CHECK(slot < Pc, p.status, 2202)) c1[slot] = (uint16_t)i;
+            }
         for (int i = tid; i < kRxBins; i += kRxThreads) hist[i] = 0;
         __syncthreads();
         const int n1 = M.cnt[0];
@@ -303,7 +308,10 @@ __global__ void __launch_bounds__(kRxThreads, 1) index_reindex_cl_kernel(const _
         const int above1 = M.info[1];
         for (int j = tid; j < n1; j += kRxThreads) {
             const int i = c1[j];
-            if ((((uint32_t)(sc[i] - blo) >> 12) & 4095u) == B1) c2[atomicAdd(&M.cnt[1], 1)] = (uint16_t)i;
+            if ((((uint32_t)(sc[i] - blo) >> 12) & 4095u) == B1) {
+                const int slot = atomicAdd(&M.cnt[1], 1);
+                if (CSA2_CHECK(slot < Pc, p.status, 2202)) c2[slot] = (uint16_t)i;
+            }
         }
         for (int i = tid; i < kRxBins; i += kRxThreads) hist[i] = 0;
         __syncthreads();
