@@ -123,3 +123,38 @@ def test_index_workspace_holds_shared_key_scores():
         assert ws(Tq, N) - base == (Tq * N * 4 + 512 + 255) // 256 * 256
     assert ws(64, 4096) == base      # below 8192 keys
     assert ws(3, 8192) == base       # fewer than 4 queries
+
+
+def test_compress_validation():
+    fake = 1 << 20
+    assert capi.csa2_fp4_compress(fake, 4, 3, 128, fake, fake, 0) == 2     # m must be 1, 2, 4 or 8
+    assert capi.csa2_fp4_compress(fake, 4, 2, 24, fake, fake, 0) == 2      # D % 16
+    assert capi.csa2_fp4_compress(0, 4, 2, 128, fake, fake, 0) == 1
+    assert capi.csa2_fp4_compress(fake + 4, 4, 2, 128, fake, fake, 0) == 3
+
+
+def test_compression_rate_field_is_validated():
+    a, _w = _index_args(m=9)
+    assert capi.csa2_index_topk(a, 0, 0, 0, 0) == 2
+    a, _w = _index_args(m=2)
+    assert capi.csa2_workspace_bytes(0, a) > 0
+
+
+def test_append_validation():
+    fake = 1 << 20
+    arr = (ctypes.c_void_p * 2)(fake, fake)
+
+    def args(**kw):
+        a = capi.AppendArgs()
+        a.B, a.N, a.D, a.Di, a.S, a.L, a.W, a.Lcap = 2, 1024, 128, 64, 1, 2, 64, 127
+        a.pos = a.kv_new = a.kv_fp4 = a.kv_scale = a.ki_new = a.kl_new = a.vl_new = a.local_base = fake
+        a.ki = a.kl = a.vl = ctypes.cast(arr, ctypes.c_void_p).value
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return a
+    assert capi.csa2_cache_append(args(Lcap=126), 0, 0) == 2      # Lcap < 2W - 1
+    assert capi.csa2_cache_append(args(S=33), 0, 0) == 2
+    assert capi.csa2_cache_append(args(D=120), 0, 0) == 2
+    assert capi.csa2_cache_append(args(pos=0), 0, 0) == 1
+    assert capi.csa2_cache_append(args(kv_new=fake + 8), 0, 0) == 3
+    assert capi.csa2_cache_append(args(L=1, W=0), 0, 0) == 2
