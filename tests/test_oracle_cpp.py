@@ -231,6 +231,10 @@ def test_empty_union():
     ("long_1m", dict(N=6000, Tq=4), [(0, 0), (0, 3)]),
     ("paper_schedule", dict(B=2, N=3000), [(0, 0), (1, 0)]),
     ("tiny", {}, [(0, 0), (0, 15)]),
+    ("decode_full", dict(B=3, N=4000), [(0, 0), (2, 0)]),
+    ("prefill_chunk", dict(N=3000, Tq=40), [(0, 0), (0, 21), (0, 39)]),
+    ("replay_prefill", dict(B=2, N=3000, Tq=64, W=64), [(0, 0), (1, 63)]),
+    ("encoder_m2", dict(B=2, N=2000), [(0, 0), (1, 0)]),
 ])
 def test_stack_matches_numpy_oracle(name, kw, units):
     """Lists bit-exact and outputs within 1e-12 of the numpy oracle through whole
@@ -251,3 +255,43 @@ def test_stack_matches_numpy_oracle(name, kw, units):
                 assert np.array_equal(lists[li]["pool"][b, j], r["pool"])
             assert np.abs(outs[li]["out"][b, j] - r["out"]).max() < 1e-12
             assert np.abs(outs[li]["lse"][b, j] - r["lse"]).max() < 1e-12
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_small_calls_match_numpy_oracle(seed):
+    """Random small shapes (head counts, widths, k, P, positions, windows, compression rate)."""
+    rng = np.random.default_rng(1000 + seed)
+    N = int(rng.integers(1, 400))
+    Hi, Di = int(rng.integers(1, 17)), int(rng.choice([16, 32, 48, 64]))
+    m = int(rng.choice([1, 1, 2]))
+    keys = synth.randint_i8(seed, 1, (N, Di), -128, 127)
+    if seed % 3 == 0:
+        keys[:] = keys[0]                                   # all scores equal
+    qi = synth.randint_i8(seed, 2, (Hi, Di), -128, 127)
+    w = rng.integers(-5, 9, Hi).astype(np.int32)
+    t = int(rng.integers(0, m * N))
+    k = int(rng.integers(1, N + 3))
+    P = int(rng.choice([0, k, k + int(rng.integers(0, 50))]))
+    te = O.last_entry(t, m)
+    p1, t1 = C.index_full(qi, w, keys, te, k, P)
+    p2, t2 = O.index_full(qi, w, keys, t, k, P, m)
+    assert np.array_equal(t1, t2)
+    if P:
+        assert np.array_equal(p1, p2)
+        k2 = int(rng.integers(1, P + 1))
+        assert np.array_equal(C.index_reindex(qi[::-1].copy(), w, keys, p1, k2),
+                              O.index_reindex(qi[::-1].copy(), w, keys, p1, k2))
+    D, Hq = int(rng.choice([64, 128])), int(rng.integers(1, 33))
+    W = int(rng.integers(0, 40))
+    npos = m * N
+    base = max(0, t - W + 1 - int(rng.integers(0, 5)))
+    x = synth.normal_f32(seed, 3, (N, D))
+    codes, scales = C.fp4_quantize(x)
+    q = _bits(synth.normal_f32(seed, 4, (Hq, D)))
+    kl = _bits(synth.normal_f32(seed, 5, (max(1, npos - base), D)))
+    vl = _bits(synth.normal_f32(seed, 6, (max(1, npos - base), D)))
+    o1, l1 = C.attention_unit(q, codes, scales, t1, kl, vl, base, t, W)
+    o2, l2 = O.attention_unit(O.bf16_to_f64(q), codes, scales, t1, O.bf16_to_f64(kl), O.bf16_to_f64(vl), base, t, W)
+    fin = np.isfinite(l2)
+    assert np.array_equal(np.isfinite(l1), fin)
+    assert np.abs(o1 - o2).max() < 1e-12 and np.abs(l1[fin] - l2[fin]).max(initial=0) < 1e-12
