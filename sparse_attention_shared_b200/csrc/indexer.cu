@@ -2194,7 +2194,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int n_all = tg + 1;
         const int lo = min(rank * p.chunk, n_all);
         const int my_n = min(lo + p.chunk, n_all) - lo;
-        const int nst = (my_n + kRows - 1) / kRows;
+        const int nst = p.pre ? 0 : (my_n + kRows - 1) / kRows;   // select only: no key tiles
 
         // ---- the index query as the MMA's B operand; zero the histogram
         if (warp != kSel / 32) {
@@ -2290,6 +2290,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // so no CTA may leave them early. The flag is shared below and every CTA leaves
         // the loop together after this query.
         const int my_abort = S.abort;
+        if (p.pre) {
+            // select only: the unit's scores come from the multi-query scoring kernel (16-byte
+            // loads, four in flight per thread; the unit's row and the chunk start are
+            // multiples of 4 elements), and the level-0 histogram is built here
+            const int* src = p.pre + (size_t)u * p.pstride + lo;
+            const int nv = my_n >> 2;
+            const int4* src4 = reinterpret_cast<const int4*>(src);
+#pragma unroll 1
+            for (int v0 = tid; v0 < nv; v0 += 4 * kTcThreads) {
+                int4 x4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int v = v0 + q * kTcThreads;
+                    x4[q] = v < nv ? __ldcg(src4 + v) : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int v = v0 + q * kTcThreads;
+                    if (v >= nv) continue;
+                    reinterpret_cast<int4*>(S.sc)[v] = x4[q];
+                    atomicAdd(&S.hist0[bin0(x4[q].x)], 1);
+                    atomicAdd(&S.hist0[bin0(x4[q].y)], 1);
+                    atomicAdd(&S.hist0[bin0(x4[q].z)], 1);
+                    atomicAdd(&S.hist0[bin0(x4[q].w)], 1);
+                }
+            }
+            for (int e = 4 * nv + tid; e < my_n; e += kTcThreads) {
+                const int x = __ldcg(src + e);
+                S.sc[e] = x;
+                atomicAdd(&S.hist0[bin0(x)], 1);
+            }
+            __syncthreads();
+        }
 
         // ---- 1. level-0 totals and each track's threshold bin
         cl_hist_allreduce(S.hist0, X, G, rank);
@@ -2823,24 +2856,35 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
         const char* ev = getenv("CSA2_FULL_PATH");
         return ev ? atoi(ev) : 0;
     }();
-    if (a.mode == CSA2_FULL && !pl.mq && full_path == 0 && (a.Di == 32 || a.Di == 64 || a.Di == 128)) {
+    bool cl_done = false;
+    if (a.mode == CSA2_FULL && full_path == 0 && (a.Di == 32 || a.Di == 64 || a.Di == 128)) {
         const int units = a.B * a.Tq;
-        const int G = std::max(1, std::min(std::min(kClMaxG / 2, sms / std::max(1, std::min(units, sms))),
-                                           (a.N + 1023) / 1024));
-        const int chunk = (int)align_up((size_t)((a.N + G - 1) / G), 256);
-        if (chunk <= kSmemScores) {
+        // a scan: the widest cluster the SMs allow per unit (up to 8, at least 1024 keys a CTA);
+        // select only (after the multi-query scoring kernel): the narrowest whose chunks fit
+        // shared memory, so that more units are cut at once
+        int G = std::max(1, std::min(std::min(kClMaxG / 2, sms / std::max(1, std::min(units, sms))),
+                                     (a.N + 1023) / 1024));
+        if (pl.mq) G = std::max(1, (a.N + kSmemScores - 1) / kSmemScores);
+        int chunk = (int)align_up((size_t)((a.N + G - 1) / G), 256);
+        if (pl.mq && chunk > kSmemScores) {   // the rounding to 256 pushed a chunk past shared memory
+            ++G;
+            chunk = (int)align_up((size_t)((a.N + G - 1) / G), 256);
+        }
+        if (chunk <= kSmemScores && G <= kClMaxG / 2) {
             IdxParams q = p;
             q.G = G;
             q.groups = std::min(units, std::max(1, sms / G));
             q.chunk = chunk;
             q.spill = nullptr;
-            q.pre = nullptr;
+            q.pre = pl.mq ? static_cast<int32_t*>(scratch) : nullptr;
             const cudaError_t ce = a.Di == 64 ? launch_cl(index_full_cl_kernel<64>, q, map, stream)
                                    : a.Di == 32 ? launch_cl(index_full_cl_kernel<32>, q, map, stream)
                                                 : launch_cl(index_full_cl_kernel<128>, q, map, stream);
-            return ce == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+            if (ce != cudaSuccess) return CSA2_ERR_CUDA;
+            cl_done = true;
         }
     }
+    if (cl_done) return CSA2_OK;
     if (a.mode == CSA2_FULL && a.Di == 64) e = launch_coop(index_full_tc_kernel<64>, kTcThreads, p, map, grid, stream);
     else if (a.mode == CSA2_FULL && a.Di == 32) e = launch_coop(index_full_tc_kernel<32>, kTcThreads, p, map, grid, stream);
     else if (a.mode == CSA2_FULL && a.Di == 128) e = launch_coop(index_full_tc_kernel<128>, kTcThreads, p, map, grid, stream);
