@@ -53,7 +53,30 @@ struct AttnParams {
     int32_t* status;
     int list_ready; // the list and the cache were complete before the previous kernel began
     int m;          // sequence compression rate of the global entries
+    // L2 prefetch of another layer's index keys (pf_keys nullptr: off): bytes [pf_lo, pf_hi)
+    // of every sequence (sequence b at pf_keys + b * pf_seq_stride), split over the launch's CTAs
+    const uint8_t* pf_keys;
+    int64_t pf_seq_stride, pf_lo, pf_hi;
 };
+
+// Bulk prefetch of [p, p + bytes) into L2 (no shared memory, no completion to wait for).
+__device__ __forceinline__ void prefetch_l2_bulk(const uint8_t* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// This CTA's share of the key prefetch: CTA `part` of `parts` of its sequence. The range's
+// ends and the sequence stride are multiples of 16 bytes (the bulk prefetch needs that),
+// and every share starts at a multiple of 256 bytes from the range's start.
+__device__ __forceinline__ void prefetch_keys_share(const AttnParams& p, int b, int part, int parts) {
+    if (p.pf_keys == nullptr || threadIdx.x != 0) return;
+    if (((p.pf_lo | p.pf_hi | p.pf_seq_stride) & 15) != 0) return;
+    const int64_t span = p.pf_hi - p.pf_lo;
+    const int64_t per = ((span + parts - 1) / parts + 255) / 256 * 256;
+    const int64_t lo = p.pf_lo + (int64_t)part * per, hi = min(p.pf_hi, lo + per);
+    const uint8_t* base = p.pf_keys + (int64_t)b * p.pf_seq_stride;
+    constexpr int64_t kPiece = 64 * 1024;
+    for (int64_t o = lo; o < hi; o += kPiece) prefetch_l2_bulk(base + o, (uint32_t)min(kPiece, hi - o));
+}
 
 template <int HQP>
 struct __align__(1024) AttnSmem {
@@ -952,6 +975,8 @@ __global__ void __launch_bounds__(kSlThreads, 1)
         }
     };
     if (early_win) issue_window();
+    // another layer's index keys, which no layer writes, into L2 while this latency-bound layer runs
+    prefetch_keys_share(p, b, (u % p.Tq) * CS + rank, p.Tq * CS);
 
     // ---- 1. global rows: list entries, FP4 codes and scales, exact dequantisation to f16
     int srow[RPT];
@@ -1489,7 +1514,7 @@ static cudaError_t launch_sl_variant(const AttnParams& p, const CUtensorMap& km,
 }
 
 csa2_status launch_attn_slice(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, const KeyPrefetch* kp) {
     const int units = a.B * a.Tq;
     if (units == 0) return CSA2_OK;
     const int cs = attn_slice_cluster(a);
@@ -1507,6 +1532,12 @@ csa2_status launch_attn_slice(const csa2_attn_args& a, const int32_t* topk, int 
     p.status = d_status;
     p.list_ready = list_ready;
     p.m = a.m;
+    if (kp != nullptr && kp->keys != nullptr && kp->hi > kp->lo) {
+        p.pf_keys = kp->keys;
+        p.pf_seq_stride = kp->seq_stride;
+        p.pf_lo = kp->lo;
+        p.pf_hi = kp->hi;
+    }
     CUtensorMap km, vm;
     memset(&km, 0, sizeof(km));
     memset(&vm, 0, sizeof(vm));

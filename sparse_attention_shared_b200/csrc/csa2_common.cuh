@@ -265,6 +265,13 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
+// Bytes [lo, hi) of every sequence of an index-key set (sequence b at keys + b * seq_stride)
+// that a launch prefetches into L2 for a later layer.
+struct KeyPrefetch {
+    const uint8_t* keys;
+    int64_t seq_stride, lo, hi;
+};
+
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 inline cudaError_t set_smem_once(const void* kern, int bytes) {
     static std::mutex mu;
