@@ -78,9 +78,24 @@ def assert_lists_equal(gpu: torch.Tensor, ref: np.ndarray, what: str):
                              f"gpu {g[tuple(bad[0])]} oracle {ref[tuple(bad[0])]}")
 
 
-def assert_attn_close(out: torch.Tensor, lse, ref_out: np.ndarray, ref_lse: np.ndarray, what: str):
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |x|: the largest error of rounding x to bf16."""
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.ldexp(1.0, (e - 8).astype(np.int64)), 0.0)
+
+
+def assert_attn_close(out: torch.Tensor, lse, ref_out: np.ndarray, ref_lse: np.ndarray, what: str,
+                      output_rounding: bool = False):
+    """max |out - ref| <= 3e-3 (the bar for the five workloads). With output_rounding,
+    the bar applies to the error beyond the bf16 output's own rounding (half a bf16 ulp
+    of the reference): an output of magnitude >= 1 cannot be within 3e-3 of its fp64
+    value once stored as bf16 (half an ulp there is 3.9e-3)."""
     o = out.float().cpu().numpy().astype(np.float64)
-    err = np.abs(o - ref_out).max()
+    diff = np.abs(o - ref_out)
+    if output_rounding:
+        diff = np.maximum(diff - bf16_half_ulp(ref_out), 0.0)
+    err = diff.max()
     assert err <= OUT_TOL, f"{what}: max |out diff| {err:.3e} > {OUT_TOL}"
     if lse is not None:
         l = lse.cpu().numpy().astype(np.float64)

@@ -91,9 +91,12 @@ def test_ticket_attention_stays_inside_its_buffers():
     q = torch.from_numpy(synth.normal_bf16(3, 2, (B, 1, Hq, D)).view(np.int16)).cuda().view(torch.bfloat16)
     kl = torch.from_numpy(synth.normal_bf16(3, 3, (B, W, D)).view(np.int16)).cuda().view(torch.bfloat16)
     vl = torch.from_numpy(synth.normal_bf16(3, 4, (B, W, D)).view(np.int16)).cuda().view(torch.bfloat16)
-    a = ops.make_attn_args(torch.full((B, 1), N - 1, dtype=torch.int32, device="cuda"), q,
-                           codes.view(B, N, D // 2), scales.view(B, N, D // 16), torch.from_numpy(topk).cuda(), kl, vl,
-                           torch.full((B,), base, dtype=torch.int32, device="cuda"), W, out, lse)
+    # the argument structure holds raw pointers: keep every tensor alive until the call is done
+    d_pos = torch.full((B, 1), N - 1, dtype=torch.int32, device="cuda")
+    d_topk = torch.from_numpy(topk).cuda()
+    d_base = torch.full((B,), base, dtype=torch.int32, device="cuda")
+    a = ops.make_attn_args(d_pos, q, codes.view(B, N, D // 2), scales.view(B, N, D // 16), d_topk, kl, vl, d_base, W,
+                           out, lse)
     from sparse_attention_shared_b200 import capi
     ws, status = ops.Workspace(), ops.Status()
     buf = ws.get(capi.csa2_workspace_bytes(1, a))

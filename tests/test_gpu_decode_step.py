@@ -110,7 +110,10 @@ def test_append_then_stack_six_tokens():
                     cur = C.index_reindex(qi[l][b, 0], w[l], keys_hist[L["key_set"]][b, : p + 1], pool, L["k"])
                 assert_lists_equal(stack.topks[l][b, 0], cur, f"step {i} layer {l} seq {b}: list")
                 ro, rl = C.attention_unit(q[l][b, 0], rc[b], rs[b], cur, kl_hist[l][b], vl_hist[l][b], 0, p, W)
-                assert_attn_close(stack.outs[l][b, 0], stack.lses[l][b, 0], ro, rl, f"step {i} layer {l} seq {b}")
+                # window 64 and top-256 give outputs up to about 1.5 here: the bar applies beyond
+                # the bf16 output's own rounding
+                assert_attn_close(stack.outs[l][b, 0], stack.lses[l][b, 0], ro, rl, f"step {i} layer {l} seq {b}",
+                                  output_rounding=True)
 
 
 def test_append_rejects_bad_sizes():

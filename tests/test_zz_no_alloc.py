@@ -78,7 +78,9 @@ def test_noalloc_against_the_oracle_without_window():
         gc, gs = ops.fp4_quantize(dev(kv.reshape(-1, D)))
         out = torch.empty((B, Tq, Hq, D), dtype=torch.bfloat16, device="cuda")
         lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device="cuda")
-        a = ops.make_attn_args(dev(q_pos), bf16_dev(q), gc.view(B, N, D // 2), gs.view(B, N, D // 16), dev(topk),
+        # the argument structure holds raw pointers: keep every tensor alive until the call is done
+        d_pos, d_q, d_topk = dev(q_pos), bf16_dev(q), dev(topk)
+        a = ops.make_attn_args(d_pos, d_q, gc.view(B, N, D // 2), gs.view(B, N, D // 16), d_topk,
                                None, None, None, 0, out, lse)
         st = ops.Status()
         assert f(ctypes.byref(a), st.ptr, stream) == 0
