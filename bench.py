@@ -493,10 +493,7 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
     fcall = lambda sp: capi.csa2_index_topk(ia, int(buf.data_ptr()), buf.numel(), st.ptr, sp)
     ms = time_alone(args, torch, fcall, flush, stream, n)
     st.check("Full indexer timing")
-    mq = s.Tq >= 4 and s.N >= 8192 and s.Hi <= 8 and s.Di in (32, 64, 128)
-    kname = (f"index_full_cl_kernel<{s.Di}>" if s.Di in (32, 64, 128) else "index_dp4a_kernel<0,0>")
-    if mq:
-        kname = f"index_mq_score_kernel<{s.Di}> + index_full_tc_kernel<{s.Di}> (select only)"
+    kname = index_kernel_name(s, "FULL")
     # the contraction the scan performs, counted over the causal pairs only: 2 * Hi * Di per (query, key)
     int8_ops = 2 * s.Hi * s.Di * sum(entries_read(s, int(t)) for t in qp_host.reshape(-1))
     entry("full_index", kname, ms, n_launch["FULL"], full_launch_bytes(s, qp_host), int8_ops, int8_peak, "int8")
@@ -519,7 +516,7 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
             lo = np.maximum(np.maximum(t_all - s.W + 1, np.repeat(base_host.astype(np.int64), s.Tq)), 0)
             n_ent += int(np.maximum(t_all - lo + 1, 0).sum())
         flops = 4 * s.Hq * s.D * n_ent
-        entry(cls, f"sparse_attn_sl_kernel<{HQP},{s.D}>", t, count, attn_call_bytes(s, qp_host, base_host, topk_host),
+        entry(cls, attn_kernel_name(s, HQP, int(topk_dev.shape[-1])), t, count, attn_call_bytes(s, qp_host, base_host, topk_host),
               flops, bf16_peak, "bf16")
 
     attn_entry("attn_full", li_f, topk_t, topk_h, n_launch["FULL"])
@@ -536,14 +533,37 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
         rcall = lambda sp: capi.csa2_index_topk(ra, int(rbuf.data_ptr()), rbuf.numel(), st.ptr, sp)
         ms = time_alone(args, torch, rcall, flush, stream, n)
         st.check("Reindex timing")
-        rk = (f"index_reindex_cl_kernel<{8 if s.Hi <= 8 else 16},{s.Di}>" if s.Di in (32, 64, 128)
-              else "index_dp4a_kernel<0,0>")
-        entry("reindex_index", rk, ms, n_launch["REINDEX"], reindex_call_bytes(s, pool_t.cpu().numpy(), Lr.k))
+        entry("reindex_index", index_kernel_name(s, "REINDEX"), ms, n_launch["REINDEX"], reindex_call_bytes(s, pool_t.cpu().numpy(), Lr.k))
         attn_entry("attn_reindex", li_r, topk_r, topk_r.cpu().numpy(), n_launch["REINDEX"])
     tot = sum(kc["ms"] * kc["launches_per_step"] for kc in out)
     for kc in out:
         kc["share"] = round(kc["ms"] * kc["launches_per_step"] / tot, 4) if tot > 0 else 0.0
     return out
+
+
+def index_kernel_name(s, mode):
+    """The kernel(s) csa2_index_topk launches for this workload's shapes (the library's
+    dispatch rules, restated for the report)."""
+    if mode == "FULL":
+        if s.Tq >= 4 and s.N >= 8192 and s.Hi <= 8 and s.Di in (32, 64, 128):
+            return f"index_mq_score_kernel<{s.Di}> + index_full_tc_kernel<{s.Di}> (select only)"
+        if s.Di in (32, 64, 128):
+            return f"index_full_tc_kernel<{s.Di}>"
+    if s.Hi <= 8 and s.Di == 64:
+        return "index_dp4a_kernel<8,64>"
+    if s.Hi <= 4 and s.Di == 32:
+        return "index_dp4a_kernel<4,32>"
+    return "index_dp4a_kernel<0,0>"
+
+
+def attn_kernel_name(s, HQP, k):
+    """The kernel csa2_sparse_attn launches: the cluster kernel while its cluster (one CTA
+    per 256 list entries, one per 128 window rows) holds at most 16 CTAs, else the ticket
+    kernel."""
+    cs = -(-k // 256) + -(-s.W // 128)
+    if 1 <= cs <= 16 and s.B * s.Tq <= 65535:
+        return f"sparse_attn_cl_kernel<{HQP},{s.D}>"
+    return f"sparse_attn_kernel<{HQP},{s.D}>"
 
 
 def run_e2e(args, torch, np, ops, capi, stack, layers, q_pos, s, flush, stream, st, graph, cache):

@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libcsa2.so")
-SOURCES = ["csa2_api.cu", "indexer.cu", "attention.cu", "fp4_quant.cu", "cache_append.cu", "reindex.cu"]
+SOURCES = ["csa2_api.cu", "indexer.cu", "attention.cu", "fp4_quant.cu", "cache_append.cu"]
 HEADERS = ["csa2_common.cuh", "fp4_codec.cuh", os.path.join("..", "..", "include", "csa2.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

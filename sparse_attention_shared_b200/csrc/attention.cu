@@ -53,30 +53,7 @@ struct AttnParams {
     int32_t* status;
     int list_ready; // the list and the cache were complete before the previous kernel began
     int m;          // sequence compression rate of the global entries
-    // L2 prefetch of another layer's index keys (pf_keys nullptr: off): bytes [pf_lo, pf_hi)
-    // of every sequence (sequence b at pf_keys + b * pf_seq_stride), split over the launch's CTAs
-    const uint8_t* pf_keys;
-    int64_t pf_seq_stride, pf_lo, pf_hi;
 };
-
-// Bulk prefetch of [p, p + bytes) into L2 (no shared memory, no completion to wait for).
-__device__ __forceinline__ void prefetch_l2_bulk(const uint8_t* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// This CTA's share of the key prefetch: CTA `part` of `parts` of its sequence. The range's
-// ends and the sequence stride are multiples of 16 bytes (the bulk prefetch needs that),
-// and every share starts at a multiple of 256 bytes from the range's start.
-__device__ __forceinline__ void prefetch_keys_share(const AttnParams& p, int b, int part, int parts) {
-    if (p.pf_keys == nullptr || threadIdx.x != 0) return;
-    if (((p.pf_lo | p.pf_hi | p.pf_seq_stride) & 15) != 0) return;
-    const int64_t span = p.pf_hi - p.pf_lo;
-    const int64_t per = ((span + parts - 1) / parts + 255) / 256 * 256;
-    const int64_t lo = p.pf_lo + (int64_t)part * per, hi = min(p.pf_hi, lo + per);
-    const uint8_t* base = p.pf_keys + (int64_t)b * p.pf_seq_stride;
-    constexpr int64_t kPiece = 64 * 1024;
-    for (int64_t o = lo; o < hi; o += kPiece) prefetch_l2_bulk(base + o, (uint32_t)min(kPiece, hi - o));
-}
 
 template <int HQP>
 struct __align__(1024) AttnSmem {
@@ -418,11 +395,12 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
         __threadfence();
         const float* pu = p.part + (size_t)u * p.ntiles * (HQP * (D + 2));
         const size_t stride = HQP * (D + 2);
-        const int nt = p.ntiles;
+        // (k + W <= 16384 gives at most 129 tiles: up to 256 fit each buffer)
+        const int nt = CSA2_CHECK(p.ntiles * HQP * 4 <= (int)sizeof(S.kbuf), p.status, 2104) ? p.ntiles : 0;
         float* wgt = reinterpret_cast<float*>(S.kbuf);             // [nt][HQP]
-        float* Mh = reinterpret_cast<float*>(S.vbuf);              // [HQP]
-        float* Lh = Mh + HQP;                                      // [HQP]
-        float* lsum = reinterpret_cast<float*>(S.kbuf + kPanelBytes);   // [nt][HQP] tile sums
+        float* lsum = reinterpret_cast<float*>(S.vbuf);            // [nt][HQP] tile sums
+        float* Mh = S.red[0];                                      // [HQP]
+        float* Lh = S.red[1];                                      // [HQP]
         for (int i = tid; i < nt * HQP; i += kAttnThreads) {
             const int s2 = i / HQP, h = i % HQP;
             wgt[i] = __ldcg(pu + s2 * stride + HQP * D + h);
@@ -819,19 +797,23 @@ __global__ void __launch_bounds__(kClThreads, 2)
 #pragma unroll
         for (int h = 0; h < HQP; ++h) {
             if (h >= p.Hq) break;
+            if (!CSA2_CHECK((h / CS) * CS + rank < HQP + 16 && h % CS < CS, p.status, 2101)) break;
             st_dsmem(dsmem_addr(&S.recv_o[(h / CS) * CS + rank][tid], h % CS), ok ? ov[h] : 0.f);
         }
     }
     if (tid < p.Hq) {
         const int row = (tid / CS) * CS + rank, owner = tid % CS;
-        st_dsmem(dsmem_addr(&S.recv_m[row], owner), ok ? S.mfin[tid] : -INFINITY);
-        st_dsmem(dsmem_addr(&S.recv_l[row], owner), ok ? S.lfin[tid] : 0.f);
+        if (CSA2_CHECK(row < HQP + 16, p.status, 2102)) {
+            st_dsmem(dsmem_addr(&S.recv_m[row], owner), ok ? S.mfin[tid] : -INFINITY);
+            st_dsmem(dsmem_addr(&S.recv_l[row], owner), ok ? S.lfin[tid] : 0.f);
+        }
     }
     cluster_sync_all();   // after it no CTA touches another's shared memory
     constexpr int kSlots = kClThreads / D;
     const int slot = tid / D, dim = tid % D;
     for (int h = rank + slot * CS; h < p.Hq; h += kSlots * CS) {
         const int r0 = (h / CS) * CS;
+        if (!CSA2_CHECK(r0 + CS <= HQP + 16, p.status, 2103)) break;
         float M = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 16; ++c)
@@ -854,457 +836,6 @@ __global__ void __launch_bounds__(kClThreads, 2)
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kCols);
-}
-
-// ------------------------------------------------------------ slice variant
-// One thread-block cluster of CS <= 8 CTAs per query, one CTA per SM (256 threads).
-// CTA r takes the 128-entry blocks r, r + CS, r + 2 CS, ... of the query's list (at
-// most SlGeom<HQP>::GB of them) and the 128-row window tile r, and computes one
-// softmax partial over all of its rows: S = K Q^T per 128-row block on the tensor
-// cores (f16 for the dequantised global rows, bf16 for the window), P in shared
-// memory, O^T = V^T P accumulated over every block in one TMEM accumulator. The
-// cluster merges the CS partials through distributed shared memory.
-// A layer takes few CTAs (4 per query at top-2048 and a 512-row window), so the
-// next layer's CTAs find free SMs while this layer runs. Launched with programmatic
-// stream serialisation, they stage all that does not depend on the previous layer
-// before their dependency wait: a Reuse layer's rows (its list was written two or
-// more kernels earlier), and for one query per sequence the window rows, whose
-// newest row (the query's own position, this layer's projection of the current
-// token) is read again after the wait.
-constexpr int kSlThreads = 256;
-constexpr int kSlMaxCluster = 8;
-
-template <int HQP>
-struct SlGeom {
-    static constexpr int GB = HQP == 16 ? 4 : 2;          // 128-row global blocks per CTA
-    static constexpr int kGPanel = GB * kPanelBytes;      // one 64-dim panel of the global rows
-    static constexpr int kQBytes = 2 * HQP * 128;         // [2 panels][HQP rows][128 B]
-    static constexpr int kPGlob = GB * 2 * HQP * 128;     // P of the global rows: [GB * 2 key panels][HQP][128 B]
-    static constexpr uint32_t kCols = 128;                // TMEM: S of GB + 1 blocks, then O
-};
-
-template <int HQP>
-struct AttnSlSmem {   // placed at a 1024-byte-aligned address
-    uint8_t gtile[2 * SlGeom<HQP>::kGPanel];   // global rows in f16, [panel][GB * 128 rows][128 B], 128B swizzle
-    uint8_t kwin[2 * kPanelBytes];             // window K (bf16), [panel][128 rows][128 B]; once S is done: P
-    uint8_t vwin[2 * kPanelBytes];             // window V (bf16)
-    uint8_t qf16[SlGeom<HQP>::kQBytes];        // Q scaled per head by a power of two into f16
-    uint8_t qbf16[SlGeom<HQP>::kQBytes];       // Q as given
-    float recv_o[HQP + kSlMaxCluster][128];    // merge: head h from CTA c sits in row (h / CS) * CS + c
-    float recv_m[HQP + kSlMaxCluster], recv_l[HQP + kSlMaxCluster];
-    float qmul[HQP];                           // per head: softmax scale (log2 units) over the Q scaling
-    float red[kSlThreads / 32][HQP];
-    float mfin[HQP], lfin[HQP];
-    uint64_t bar_tma, bar_s, bar_o;
-    uint32_t tmem_base;
-};
-
-static_assert(sizeof(AttnSlSmem<16>) + 1024 <= 227 * 1024 && sizeof(AttnSlSmem<32>) + 1024 <= 227 * 1024,
-              "slice attention shared memory");
-static_assert(offsetof(AttnSlSmem<16>, kwin) % 1024 == 0 && offsetof(AttnSlSmem<16>, qf16) % 1024 == 0 &&
-                  offsetof(AttnSlSmem<16>, qbf16) % 1024 == 0 && offsetof(AttnSlSmem<32>, kwin) % 1024 == 0 &&
-                  offsetof(AttnSlSmem<32>, qf16) % 1024 == 0 && offsetof(AttnSlSmem<32>, qbf16) % 1024 == 0,
-              "operand alignment");
-static_assert(SlGeom<16>::kPGlob + 2 * 16 * 128 <= 2 * kPanelBytes && SlGeom<32>::kPGlob + 2 * 32 * 128 <= 2 * kPanelBytes,
-              "P fits where the window K was");
-
-template <int HQP, int D>
-__global__ void __launch_bounds__(kSlThreads, 1)
-    sparse_attn_sl_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap kl_map,
-                          const __grid_constant__ CUtensorMap vl_map) {
-    static_assert(HQP == 16 || HQP == 32, "head padding");
-    static_assert(D == 64 || D == 128, "head dim (held as 128 in shared memory, zero-padded)");
-    using G = SlGeom<HQP>;
-    constexpr int RPT = G::GB * kTileKeys / kSlThreads;   // global rows per thread (2 or 1)
-    constexpr int NSET = G::GB / 2 + 1;                   // row sets per thread in the softmax
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    AttnSlSmem<HQP>& S =
-        *reinterpret_cast<AttnSlSmem<HQP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int half = warp >> 2, qtr = warp & 3;
-    const int CS = gridDim.x;
-    const int rank = (int)cluster_ctarank();
-    const int u = blockIdx.y;
-    const int b = u / p.Tq;
-    const int kb = (p.k + kTileKeys - 1) / kTileKeys;
-    int nb = 0;                                            // this CTA's blocks: rank + i * CS < kb
-#pragma unroll
-    for (int i = 0; i < G::GB; ++i)
-        if (rank + i * CS < kb) nb = i + 1;
-    const bool win = rank < p.nlt;
-    const bool has_rows = nb > 0 || win;                   // CTA-uniform
-
-    // ---- 0. set-up that reads no input
-    if (warp == 0) tmem_alloc(&S.tmem_base, G::kCols);
-    if (tid == 0) {
-        mbar_init(&S.bar_tma, 1);
-        mbar_init(&S.bar_s, 1);
-        mbar_init(&S.bar_o, 1);
-        mbar_fence_init();
-    }
-    // every CTA of the cluster has started: waited on before the first push into a peer
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-    if (D == 64) {   // dims 64..127 of the window tiles stay zero
-        for (int i = tid; i < kPanelBytes / 16; i += kSlThreads) {
-            reinterpret_cast<uint4*>(S.kwin + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4*>(S.vwin + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
-        }
-    }
-    __syncthreads();   // the barriers (initialised by thread 0) and the TMEM address are set
-
-    int t = p.q_pos[u];
-    int tg = last_entry(t, p.m);   // the last global entry the query reads
-    const bool t_ok = t >= 0 && tg < p.N;
-    if (!t_ok) {
-        if (tid == 0 && rank == 0) report(p.status, CSA2_ERR_RANGE, u);
-        t = -1;
-        tg = -1;
-    }
-    const int base = p.local_base[b];
-    const int lo_w = max(max(base, t - p.W + 1), 0);
-    const int w0 = lo_w + rank * kTileKeys;                // position of the window tile's row 0
-    const bool early_win = win && p.Tq == 1;
-    auto issue_window = [&]() {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&S.bar_tma, 2u * (D / 64) * kPanelBytes);
-#pragma unroll
-            for (int pn = 0; pn < D / 64; ++pn) {
-                tma_load_3d(S.kwin + pn * kPanelBytes, &kl_map, pn * 64, w0 - base, b, &S.bar_tma);
-                tma_load_3d(S.vwin + pn * kPanelBytes, &vl_map, pn * 64, w0 - base, b, &S.bar_tma);
-            }
-        }
-    };
-    if (early_win) issue_window();
-    // another layer's index keys, which no layer writes, into L2 while this latency-bound layer runs
-    prefetch_keys_share(p, b, (u % p.Tq) * CS + rank, p.Tq * CS);
-
-    // ---- 1. global rows: list entries, FP4 codes and scales, exact dequantisation to f16
-    int srow[RPT];
-    uint4 cw[RPT][D / 32];
-    uint32_t scw[RPT][D / 64];
-    auto gather = [&]() {
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-            const int j = tid + i * kSlThreads;            // local row: block j / 128, row j % 128
-            const int lb = j >> 7;
-            const int e = (rank + lb * CS) * kTileKeys + (j & 127);
-            int s = (lb < nb && e < p.k) ? __ldcg(p.topk + (size_t)u * p.k + e) : -1;
-            if (s >= 0 && (s > tg || s >= p.N)) {
-                report(p.status, CSA2_ERR_RANGE, u);
-                s = -1;
-            }
-            srow[i] = s;
-        }
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-            if (srow[i] < 0) continue;
-            const size_t row = (size_t)b * p.N + srow[i];
-            const uint4* cp = reinterpret_cast<const uint4*>(p.kv_fp4 + row * (D / 2));
-#pragma unroll
-            for (int q = 0; q < D / 32; ++q) cw[i][q] = __ldg(cp + q);
-            if (D == 128) {
-                const uint2 s2 = __ldg(reinterpret_cast<const uint2*>(p.kv_scale + row * 8));
-                scw[i][0] = s2.x;
-                scw[i][(D / 64) - 1] = s2.y;
-            } else {
-                scw[i][0] = __ldg(reinterpret_cast<const uint32_t*>(p.kv_scale + row * 4));
-            }
-        }
-    };
-    auto dequant = [&]() {
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-            const int j = tid + i * kSlThreads;
-            if ((j >> 7) >= nb) continue;
-            const bool v = srow[i] >= 0;
-            uint32_t sp[D / 32];   // f16x2 scale pairs (groups 2i, 2i + 1)
-#pragma unroll
-            for (int q = 0; q < D / 32; ++q) sp[q] = v ? e4m3x2_f16(scw[i][q >> 1] >> (16 * (q & 1))) : 0u;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                uint4 o = make_uint4(0, 0, 0, 0);
-                if (v && c < D / 8) {
-                    const uint4 w4 = cw[i][c >> 2];
-                    const uint32_t w = (c & 3) == 0 ? w4.x : (c & 3) == 1 ? w4.y : (c & 3) == 2 ? w4.z : w4.w;
-                    const uint32_t g = c >> 1;
-                    const uint32_t pr = sp[g >> 1];
-                    const uint32_t s2x = (g & 1) ? ((pr >> 16) | (pr & 0xFFFF0000u)) : ((pr & 0xFFFFu) | (pr << 16));
-                    uint32_t d[4];
-                    e2m1x8_f16(w, d);
-                    o.x = f16x2_mul(d[0], s2x);
-                    o.y = f16x2_mul(d[1], s2x);
-                    o.z = f16x2_mul(d[2], s2x);
-                    o.w = f16x2_mul(d[3], s2x);
-                }
-                const uint32_t off = (c >> 3) * G::kGPanel + sw128(j, c & 7);
-                if (CSA2_CHECK(off + 16u <= sizeof(S.gtile), p.status, 2101))
-                    *reinterpret_cast<uint4*>(S.gtile + off) = o;
-            }
-        }
-    };
-    if (p.list_ready) {   // the list and the cache were complete before the previous kernel began
-        gather();
-        dequant();
-    }
-    pdl_wait();
-    pdl_launch_dependents();
-    if (!p.list_ready) gather();
-
-    // ---- 2. the query (it depends on the previous layer): f16 copy scaled per head by
-    // 2^k (its largest value into [2^14, 2^15)) for the global blocks, bf16 for the window
-    constexpr int kQv = HQP * 16 / kSlThreads;   // 16-byte chunks per thread (16 chunks per padded head)
-    uint4 qv[kQv];
-#pragma unroll
-    for (int q = 0; q < kQv; ++q) {
-        const int i = tid + q * kSlThreads;
-        const int h = i >> 4, c = i & 15;
-        qv[q] = make_uint4(0, 0, 0, 0);
-        if (h < p.Hq && c < D / 8) qv[q] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
-    }
-    if (!p.list_ready) dequant();
-#pragma unroll
-    for (int q = 0; q < kQv; ++q) {
-        const int i = tid + q * kSlThreads;
-        const int h = i >> 4, c = i & 15;
-        const uint4 v = qv[q];
-        uint32_t e = bf16x8_max_exp(v);
-#pragma unroll
-        for (int o = 1; o < 16; o <<= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
-        const int k2 = (e == 0u) ? 0 : min(141 - (int)e, 126);
-        const float f = __uint_as_float((uint32_t)(127 + k2) << 23);
-        uint4 v16;
-        v16.x = bf16x2_to_f16x2(v.x, f);
-        v16.y = bf16x2_to_f16x2(v.y, f);
-        v16.z = bf16x2_to_f16x2(v.z, f);
-        v16.w = bf16x2_to_f16x2(v.w, f);
-        const uint32_t off = (c >> 3) * (HQP * 128) + sw128(h, c & 7);
-        if (CSA2_CHECK(off + 16u <= (uint32_t)G::kQBytes, p.status, 2102)) {
-            *reinterpret_cast<uint4*>(S.qf16 + off) = v16;
-            *reinterpret_cast<uint4*>(S.qbf16 + off) = v;
-        }
-        if (c == 0) S.qmul[h] = p.scale_log2 * __uint_as_float((uint32_t)(127 - k2) << 23);
-    }
-
-    // ---- 3. the window tile
-    bool ok = true;
-    bool wvalid = false;
-    const int rr = qtr * 32 + lane;   // this thread's row within a 128-row block (its TMEM lane)
-    if (win) {
-        if (!early_win) issue_window();
-        const int pos = w0 + rr;
-        wvalid = half == 0 && t_ok && p.W > 0 && pos <= t;
-        if (wvalid && pos - base >= p.Lloc) {
-            report(p.status, CSA2_ERR_RANGE, u);
-            wvalid = false;
-        }
-        ok = mbar_wait(&S.bar_tma, 0, p.status, 12);
-        if (early_win && ok && warp == 0) {
-            // the query's own row, read after the dependency wait over the early copy
-            const int r0 = t - w0;
-            if (t_ok && r0 >= 0 && r0 < kTileKeys && t - base < p.Lloc) {
-                const int c = lane & 15;
-                if (c < D / 8) {
-                    const uint16_t* src = (lane < 16 ? p.kl : p.vl) + ((size_t)b * p.Lloc + (t - base)) * D;
-                    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + c);
-                    const uint32_t off = (c >> 3) * kPanelBytes + sw128(r0, c & 7);
-                    uint8_t* dst = (lane < 16 ? S.kwin : S.vwin) + off;
-                    if (CSA2_CHECK(off + 16u <= sizeof(S.kwin), p.status, 2104)) *reinterpret_cast<uint4*>(dst) = v;
-                }
-            }
-        }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = S.tmem_base;
-    const uint32_t tmem_o = tmem + (uint32_t)(G::GB + 1) * HQP;
-
-    // ---- 4. S = K Q^T per 128-row block (keys as M, heads as N)
-    if (tid == 0 && has_rows) {
-        const uint32_t ga = smem_u32(S.gtile), qa = smem_u32(S.qf16), kwa = smem_u32(S.kwin), qb = smem_u32(S.qbf16);
-        constexpr uint32_t id16 = idesc_f16(128, HQP, 0), idb = idesc_bf16(128, HQP, 0);
-        for (int lb = 0; lb < nb; ++lb) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = smem_desc(ga + (kk >> 2) * G::kGPanel + lb * kPanelBytes + (kk & 3) * 32, 16, 1024);
-                const uint64_t bd = smem_desc(qa + (kk >> 2) * (HQP * 128) + (kk & 3) * 32, 16, 1024);
-                mma_bf16(tmem + lb * HQP, ad, bd, id16, kk > 0 ? 1u : 0u);
-            }
-        }
-        if (win) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = smem_desc(kwa + (kk >> 2) * kPanelBytes + (kk & 3) * 32, 16, 1024);
-                const uint64_t bd = smem_desc(qb + (kk >> 2) * (HQP * 128) + (kk & 3) * 32, 16, 1024);
-                mma_bf16(tmem + G::GB * HQP, ad, bd, idb, kk > 0 ? 1u : 0u);
-            }
-        }
-        mma_commit(&S.bar_s);
-    }
-    if (has_rows) ok = mbar_wait(&S.bar_s, 0, p.status, 10) && ok;
-    tc_fence_after();
-
-    // ---- 5. softmax partial: set i < GB / 2 is global block 2 i + half (row rr), the
-    // last set the window tile (threads of half 0)
-    float a[NSET][HQP];
-#pragma unroll
-    for (int i = 0; i < NSET; ++i) {
-        const bool is_win = i == NSET - 1;
-        const int lb = 2 * i + half;
-        const bool present = has_rows && ok && (is_win ? (half == 0 && win) : lb < nb);   // warp-uniform
-        if (present) {
-            const uint32_t col = is_win ? (uint32_t)G::GB * HQP : (uint32_t)lb * HQP;
-            float tmp[16];
-#pragma unroll
-            for (int c0 = 0; c0 < HQP; c0 += 16) {
-                tmem_ld16(tmem + col + ((uint32_t)(qtr * 32) << 16) + c0, tmp);
-                tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < 16; ++x) a[i][c0 + x] = tmp[x];
-            }
-        }
-        const bool v = present && (is_win ? wvalid : srow[i < RPT ? i : 0] >= 0);
-#pragma unroll
-        for (int h = 0; h < HQP; ++h) a[i][h] = v ? a[i][h] * (is_win ? p.scale_log2 : S.qmul[h]) : -INFINITY;
-    }
-    const int hl = (HQP == 16) ? ((lane >> 1) & 15) : lane;   // the head this lane ends up holding
-    {
-        float v[HQP];
-#pragma unroll
-        for (int h = 0; h < HQP; ++h) {
-            float m = a[0][h];
-#pragma unroll
-            for (int i = 1; i < NSET; ++i) m = fmaxf(m, a[i][h]);
-            v[h] = m;
-        }
-        const float m = warp_transpose_reduce<HQP, true>(v);
-        if (HQP == 32 || (lane & 1) == 0) S.red[warp][hl] = m;
-    }
-    __syncthreads();
-    if (tid < HQP) {
-        float m = S.red[0][tid];
-#pragma unroll
-        for (int w = 1; w < kSlThreads / 32; ++w) m = fmaxf(m, S.red[w][tid]);
-        S.mfin[tid] = m;
-    }
-    __syncthreads();
-    uint8_t* Pg = S.kwin;                    // P of the global rows (f16), then of the window (bf16)
-    uint8_t* Pw = S.kwin + G::kPGlob;
-    float ls[HQP];
-#pragma unroll
-    for (int h = 0; h < HQP; ++h) ls[h] = 0.f;
-#pragma unroll
-    for (int i = 0; i < NSET; ++i) {
-        const bool is_win = i == NSET - 1;
-        const int lb = 2 * i + half;
-        const bool present = has_rows && (is_win ? (half == 0 && win) : lb < nb);
-        if (!present) continue;
-        const int key = is_win ? rr : lb * kTileKeys + rr;
-        uint8_t* pb = (is_win ? Pw : Pg) + (key >> 6) * (HQP * 128) + (key & 7) * 2;
-#pragma unroll
-        for (int h = 0; h < HQP; ++h) {
-            const float mh = S.mfin[h];
-            const float pv = (a[i][h] != -INFINITY && mh != -INFINITY) ? exp2f(a[i][h] - mh) : 0.f;
-            ls[h] += pv;
-            uint8_t* dst = pb + sw128(h, (key & 63) >> 3);
-            if (CSA2_CHECK(dst >= S.kwin && dst + 2 <= S.kwin + sizeof(S.kwin), p.status, 2103))
-                *reinterpret_cast<uint16_t*>(dst) =
-                    is_win ? __bfloat16_as_ushort(__float2bfloat16_rn(pv)) : __half_as_ushort(__float2half_rn(pv));
-        }
-    }
-    {
-        const float l = warp_transpose_reduce<HQP, false>(ls);
-        if (HQP == 32 || (lane & 1) == 0) S.red[warp][hl] = l;
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (tid < HQP) {
-        float l = 0.f;
-#pragma unroll
-        for (int w = 0; w < kSlThreads / 32; ++w) l += S.red[w][tid];
-        S.lfin[tid] = l;
-    }
-
-    // ---- 6. O^T = V^T P over every block of the CTA (head dim as M, keys as the reduction)
-    if (tid == 0 && has_rows) {
-        const uint32_t ga = smem_u32(S.gtile), va = smem_u32(S.vwin), pg = smem_u32(Pg), pw = smem_u32(Pw);
-        constexpr uint32_t id16 = idesc_f16(128, HQP, 1), idb = idesc_bf16(128, HQP, 1);
-        int n = 0;
-        for (int kk = 0; kk < nb * (kTileKeys / 16); ++kk, ++n) {
-            const uint64_t ad = smem_desc(ga + kk * 2048, G::kGPanel, 1024);
-            const uint64_t bd = smem_desc(pg + (kk >> 2) * (HQP * 128) + (kk & 3) * 32, 16, 1024);
-            mma_bf16(tmem_o, ad, bd, id16, n > 0 ? 1u : 0u);
-        }
-        if (win) {
-#pragma unroll
-            for (int kk = 0; kk < kTileKeys / 16; ++kk, ++n) {
-                const uint64_t ad = smem_desc(va + kk * 2048, kPanelBytes, 1024);
-                const uint64_t bd = smem_desc(pw + (kk >> 2) * (HQP * 128) + (kk & 3) * 32, 16, 1024);
-                mma_bf16(tmem_o, ad, bd, idb, n > 0 ? 1u : 0u);
-            }
-        }
-        mma_commit(&S.bar_o);
-    }
-    if (has_rows) ok = mbar_wait(&S.bar_o, 0, p.status, 11) && ok;
-    tc_fence_after();
-    float ov[HQP];
-#pragma unroll
-    for (int h = 0; h < HQP; ++h) ov[h] = 0.f;
-    if (warp < 4 && has_rows && ok) {   // O^T rows (the head dim) sit in TMEM lanes 0..127
-        float tmp[16];
-#pragma unroll
-        for (int c0 = 0; c0 < HQP; c0 += 16) {
-            tmem_ld16(tmem_o + ((uint32_t)(warp * 32) << 16) + c0, tmp);
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 16; ++x) ov[c0 + x] = tmp[x];
-        }
-    }
-    tc_fence_before();
-
-    // ---- 7. merge: every CTA pushes its partial of head h into the CTA that merges h
-    // (CTA h % CS); one cluster barrier publishes the pushes
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    const bool live = has_rows && ok;
-    if (tid < D) {
-#pragma unroll
-        for (int h = 0; h < HQP; ++h) {
-            if (h >= p.Hq) break;
-            if (CSA2_CHECK((h / CS) * CS + rank < HQP + kSlMaxCluster, p.status, 2105))
-                st_dsmem(dsmem_addr(&S.recv_o[(h / CS) * CS + rank][tid], h % CS), live ? ov[h] : 0.f);
-        }
-    }
-    if (tid < p.Hq) {
-        const int row = (tid / CS) * CS + rank, owner = tid % CS;
-        st_dsmem(dsmem_addr(&S.recv_m[row], owner), live ? S.mfin[tid] : -INFINITY);
-        st_dsmem(dsmem_addr(&S.recv_l[row], owner), live ? S.lfin[tid] : 0.f);
-    }
-    cluster_sync_all();   // after it no CTA touches another's shared memory
-    constexpr int kSlots = kSlThreads / D;
-    const int slot = tid / D, dim = tid % D;
-    for (int h = rank + slot * CS; h < p.Hq; h += kSlots * CS) {
-        const int r0 = (h / CS) * CS;
-        float M = -INFINITY;
-        for (int c = 0; c < CS; ++c) M = fmaxf(M, S.recv_m[r0 + c]);
-        float L = 0.f, acc = 0.f;
-        if (M != -INFINITY) {
-            for (int c = 0; c < CS; ++c) {
-                const float mc = S.recv_m[r0 + c];
-                const float wgt = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-                L += wgt * S.recv_l[r0 + c];
-                acc += wgt * S.recv_o[r0 + c][dim];
-            }
-        }
-        p.out[((size_t)u * p.Hq + h) * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(L > 0.f ? acc / L : 0.f));
-        if (dim == 0 && p.lse != nullptr)
-            p.lse[(size_t)u * p.Hq + h] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, G::kCols);
 }
 
 // ------------------------------------------------------------ host side
@@ -1477,81 +1008,5 @@ csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, in
     return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }
 
-
-// Slice attention: one cluster of at most kSlMaxCluster CTAs per query (0: does not fit).
-int attn_slice_cluster(const csa2_attn_args& a) {
-    const int HQP = a.Hq <= 16 ? 16 : 32;
-    const int GB = HQP == 16 ? SlGeom<16>::GB : SlGeom<32>::GB;
-    const int kb = (a.k + kTileKeys - 1) / kTileKeys, nlt = (a.W + kTileKeys - 1) / kTileKeys;
-    const int cs = std::max(std::max((kb + GB - 1) / GB, nlt), 1);
-    return (cs <= kSlMaxCluster && (int64_t)a.B * a.Tq <= 65535) ? cs : 0;
-}
-
-template <int HQP, int D>
-static cudaError_t launch_sl_variant(const AttnParams& p, const CUtensorMap& km, const CUtensorMap& vm, int cs,
-                                     int units, cudaStream_t stream) {
-    auto kern = sparse_attn_sl_kernel<HQP, D>;
-    const size_t smem = sizeof(AttnSlSmem<HQP>) + 1024;
-    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(cs, units);
-    cfg.blockDim = dim3(kSlThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    // set-up, the window rows before the query's own and (list_ready) the global rows are
-    // read before griddepcontrol.wait: none of them is written by the previous kernel
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, p, km, vm);
-}
-
-csa2_status launch_attn_slice(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
-                              cudaStream_t stream, const KeyPrefetch* kp) {
-    const int units = a.B * a.Tq;
-    if (units == 0) return CSA2_OK;
-    const int cs = attn_slice_cluster(a);
-    if (cs == 0) return CSA2_ERR_UNSUPPORTED;
-    AttnParams p{};
-    p.B = a.B; p.Tq = a.Tq; p.N = a.N; p.Hq = a.Hq; p.D = a.D; p.k = a.k; p.W = a.W; p.Lloc = a.Lloc;
-    p.nlt = (a.W + kTileKeys - 1) / kTileKeys;
-    p.ngt = (a.k + kTileKeys - 1) / kTileKeys;
-    p.ntiles = cs;
-    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)a.D));
-    p.q_pos = a.q_pos; p.q = a.q; p.kv_fp4 = a.kv_fp4; p.kv_scale = a.kv_scale; p.topk = topk;
-    p.kl = a.kl; p.vl = a.vl; p.local_base = a.local_base; p.out = a.out; p.lse = a.lse;
-    p.part = nullptr;
-    p.tickets = nullptr;
-    p.status = d_status;
-    p.list_ready = list_ready;
-    p.m = a.m;
-    if (kp != nullptr && kp->keys != nullptr && kp->hi > kp->lo) {
-        p.pf_keys = kp->keys;
-        p.pf_seq_stride = kp->seq_stride;
-        p.pf_lo = kp->lo;
-        p.pf_hi = kp->hi;
-    }
-    CUtensorMap km, vm;
-    memset(&km, 0, sizeof(km));
-    memset(&vm, 0, sizeof(vm));
-    if (a.W > 0) {
-        if (!encode_local_map(&km, a.kl, a.B, a.Lloc, a.D) || !encode_local_map(&vm, a.vl, a.B, a.Lloc, a.D))
-            return CSA2_ERR_CUDA;
-    }
-    const int HQP = a.Hq <= 16 ? 16 : 32;
-    cudaError_t e;
-    if (HQP == 16 && a.D == 128) e = launch_sl_variant<16, 128>(p, km, vm, cs, units, stream);
-    else if (HQP == 16 && a.D == 64) e = launch_sl_variant<16, 64>(p, km, vm, cs, units, stream);
-    else if (HQP == 32 && a.D == 128) e = launch_sl_variant<32, 128>(p, km, vm, cs, units, stream);
-    else e = launch_sl_variant<32, 64>(p, km, vm, cs, units, stream);
-    return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
-}
 
 }  // namespace csa2

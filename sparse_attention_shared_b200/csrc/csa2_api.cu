@@ -37,20 +37,13 @@ csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* ticke
 bool attn_cluster_fits(const csa2_attn_args& a);
 csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
                                 cudaStream_t stream);
-int attn_slice_cluster(const csa2_attn_args& a);
-csa2_status launch_attn_slice(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
-                              cudaStream_t stream, const KeyPrefetch* kp);
 
-// The attention kernel for a call: the slice kernel (one cluster of at most 8 CTAs per
-// query), else the 12-CTA cluster kernel, else one CTA per tile with a ticket merge.
+// The attention kernel for a call: the cluster kernel (one CTA per 256 list entries or
+// 128 window rows, the partials merged through distributed shared memory), else one CTA
+// per tile with a ticket merge.
 static csa2_status run_attn(const csa2_attn_args& a, const int32_t* topk, int list_ready, int* tickets,
-                            void* scratch, int32_t* d_status, cudaStream_t stream, const KeyPrefetch* kp = nullptr) {
-    static const int path = [] {
-        const char* e = getenv("CSA2_ATTN_PATH");
-        return e ? atoi(e) : 0;
-    }();
-    if (path == 0 && attn_slice_cluster(a) > 0) return launch_attn_slice(a, topk, list_ready, d_status, stream, kp);
-    if (path <= 1 && attn_cluster_fits(a)) return launch_attn_cluster(a, topk, list_ready, d_status, stream);
+                            void* scratch, int32_t* d_status, cudaStream_t stream) {
+    if (attn_cluster_fits(a)) return launch_attn_cluster(a, topk, list_ready, d_status, stream);
     return launch_attn(a, topk, tickets, scratch, d_status, stream);
 }
 void set_wait_controls(long long budget, int skip);
@@ -244,31 +237,6 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
     int* tickets = static_cast<int*>(ws_at(workspace, R));
     void* scratch = ws_at(workspace, R + tickets_bytes(units));
 
-    // The Full layers' key scans are bandwidth-bound and their keys depend on no layer; the
-    // latency-bound attention launches of the up to three layers before a Full layer each
-    // prefetch a third of its keys into L2 (CSA2_KEY_PREFETCH=0 turns this off).
-    static const int key_prefetch = [] {
-        const char* e = getenv("CSA2_KEY_PREFETCH");
-        return e ? atoi(e) : 1;
-    }();
-    std::vector<KeyPrefetch> kps(s->L, KeyPrefetch{nullptr, 0, 0, 0});
-    if (key_prefetch) {   // (N * Di and the sequence stride are multiples of 16 bytes)
-        for (int f = 1; f < s->L; ++f) {
-            const csa2_index_args& fx = s->idx[f];
-            if (fx.mode != CSA2_FULL) continue;
-            int first = f - 1;   // the launches between the previous Full layer and this one, at most three
-            while (first > 0 && f - first < 3 && s->idx[first].mode != CSA2_FULL) --first;
-            if (s->idx[first].mode == CSA2_FULL && first != f - 1) ++first;
-            const int parts = f - first;
-            const int64_t bytes = (int64_t)fx.N * fx.Di;
-            for (int l = first; l < f; ++l) {
-                // 256-byte pieces: every prefetch address and size stays a multiple of 16 bytes
-                const int64_t per = ((bytes + parts - 1) / parts + 255) / 256 * 256;
-                kps[l] = KeyPrefetch{reinterpret_cast<const uint8_t*>(fx.ki), fx.ki_seq_stride,
-                                     (l - first) * per, std::min(bytes, (l - first + 1) * per)};
-            }
-        }
-    }
     const int32_t* cur = nullptr;   // the current layer's list
     int cur_k = 0;
     const int32_t* pool = nullptr;  // the most recent Full layer's pool
@@ -310,7 +278,7 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
         // kernel is the previous layer's attention), so its clusters may gather their
         // global rows before waiting for that kernel; not when a copy came between.
         const int list_ready = (ix.mode == CSA2_REUSE && !copied) ? 1 : 0;
-        st = run_attn(a, cur, list_ready, tickets, scratch, d_status, strm, &kps[l]);
+        st = run_attn(a, cur, list_ready, tickets, scratch, d_status, strm);
         if (st != CSA2_OK) return st;
     }
     return CSA2_OK;

@@ -29,10 +29,14 @@ __device__ __forceinline__ void report(int32_t* st, int code, int detail) {
 // computed shared- or global-memory index is checked before the access it guards; a
 // violation is reported as CSA2_ERR_RANGE with `detail` naming the site, and the
 // access is skipped. In the normal build the check is the constant true.
+// CSA2_GUARD keeps its bound in both builds (an access the normal build skips quietly)
+// and reports a violation in the checked one.
 #ifdef CSA2_CHECKED
 #define CSA2_CHECK(cond, st, detail) (::csa2::checked_ok((cond), (st), (detail)))
+#define CSA2_GUARD(cond, st, detail) (::csa2::checked_ok((cond), (st), (detail)))
 #else
 #define CSA2_CHECK(cond, st, detail) (true)
+#define CSA2_GUARD(cond, st, detail) (cond)
 #endif
 
 __device__ __forceinline__ bool checked_ok(bool cond, int32_t* st, int detail) {
@@ -264,13 +268,6 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
-
-// Bytes [lo, hi) of every sequence of an index-key set (sequence b at keys + b * seq_stride)
-// that a launch prefetches into L2 for a later layer.
-struct KeyPrefetch {
-    const uint8_t* keys;
-    int64_t seq_stride, lo, hi;
-};
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 inline cudaError_t set_smem_once(const void* kern, int bytes) {

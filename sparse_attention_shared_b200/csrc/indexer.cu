@@ -876,7 +876,8 @@ __device__ __noinline__ int count_range(const int* sc, int n, int lo_t, int hi_t
 // The taken elements go to out[base ..] in position order.
 struct ListCut {
     int T, all, quota, base, r;
-    int32_t* out;   // nullptr: track off
+    int32_t* out;      // nullptr: track off
+    int32_t* status;   // status word (reports of the range-checked build)
 };
 
 // The global cache rows of one sequence that its top-k list selects are pulled into
@@ -956,8 +957,8 @@ __device__ __forceinline__ void write_lists(const int* sc, int n, int base, cons
         const bool t0 = g0 || (q0 && oq0 < c0.quota), t1 = g1 || (q1 && oq1 < c1.quota);
         if (t0 || t1) {
             const int pos = pool ? pool[base + e] : base + e;
-            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if ((unsigned)k < (unsigned)c0.r) c0.out[k] = pos; }
-            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if ((unsigned)k < (unsigned)c1.r) { c1.out[k] = pos; prefetch_row(pf, pos); } }
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) c0.out[k] = pos; }
+            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c1.r, c1.status, 2202)) { c1.out[k] = pos; prefetch_row(pf, pos); } }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
     }
@@ -1014,8 +1015,8 @@ __device__ __forceinline__ void write_from_lists(const int* sc, int base, const 
         if (t0 || t1) {
             const int e = base + (ent & 0x0FFFFFFF);
             const int pos = pool ? pool[e] : e;
-            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if ((unsigned)k < (unsigned)c0.r) c0.out[k] = pos; }
-            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if ((unsigned)k < (unsigned)c1.r) { c1.out[k] = pos; prefetch_row(pf, pos); } }
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) c0.out[k] = pos; }
+            if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c1.r, c1.status, 2202)) { c1.out[k] = pos; prefetch_row(pf, pos); } }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
     }
@@ -1253,6 +1254,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
             ListCut& lc = cut[tr];
             lc.r = p.r[tr];
             lc.out = lc.r > 0 ? p.out[tr] + (size_t)c.u * lc.r : nullptr;
+            lc.status = p.status;
             lc.all = st == TS_ALL;
             lc.T = T[tr];
             lc.quota = 0;
@@ -1351,8 +1353,8 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
     }
     sel_sync();
     const int r = p.r[1];
-    ListCut none{INT_MAX, 0, 0, 0, 0, nullptr};
-    ListCut cut{INT_MAX, 0, 0, 0, r, p.out[1] + (size_t)c.u * r};
+    ListCut none{INT_MAX, 0, 0, 0, 0, nullptr, p.status};
+    ListCut cut{INT_MAX, 0, 0, 0, r, p.out[1] + (size_t)c.u * r, p.status};
     bool lists = false;
     if (n <= r) {
         cut.all = 1;
@@ -2056,505 +2058,6 @@ __global__ void __launch_bounds__(kSel, 1)
     }
 }
 
-// ------------------------------------------------------------ Full mode in thread-block clusters
-// The G CTAs that score one query form a thread-block cluster (G <= 16, one CTA per
-// SM), so the exact select exchanges its histograms, candidates and counts through
-// distributed shared memory instead of global memory and spin barriers:
-//   1. the level-0 histograms (built by the scan's epilogue) are summed across the
-//      cluster: CTA r adds its slice of bins over every CTA, then every CTA reads
-//      every slice; each track (pool, top-k) finds the bin holding its r-th best
-//      score and the interval of scores that bin covers;
-//   2. while a track's interval holds more than kCandCap scores, two more 12-bit
-//      digits narrow it the same way (rare: long runs of equal scores);
-//   3. each CTA compacts its scores inside the intervals and publishes how many it
-//      has above them; every CTA reads every CTA's candidates, finds the exact
-//      threshold T and the number of ties at T to take, and, from the candidates'
-//      owners, its own output offset and tie quota;
-//   4. each CTA writes its selected positions in order with no further exchange.
-// The scan is the warp-specialised tensor-core scan of index_full_tc_kernel. The
-// kernel keeps no state in the workspace.
-constexpr int kClMaxG = 16;
-
-struct ClSel {   // select-phase buffers, over the key stages
-    int htot[kBins];            // the cluster's histogram totals (a copy in every CTA)
-    int hown[kBins];            // this CTA's slice of the totals (read by the others)
-    int hl[kBins];              // a local histogram
-    int lc[2][kCandCap];        // this CTA's scores inside each track's interval (read by the others)
-    int gc[2][kCandCap];        // every CTA's, in CTA order
-    int pub[2][4];              // per track: [0] own scores above the interval, [1] own scores in it
-    int goff[2][kClMaxG + 1];   // offsets of the CTAs' candidates in gc
-    int cnt_gt[2][kClMaxG], cnt_eq[2][kClMaxG];
-    int above_c[2][kClMaxG];    // every CTA's scores above the interval
-    int lcnt[2];
-    int abort_any;
-};
-static_assert(sizeof(ClSel) <= sizeof(((IdxSmem*)0)->stage), "select buffers over the key stages");
-
-__device__ __forceinline__ int ld_dsmem_i32(const void* p, uint32_t rank) {
-    int v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(dsmem_addr(p, rank)) : "memory");
-    return v;
-}
-
-// In a 4096-bin histogram in shared memory, the bin holding the r-th largest element
-// (1-based): out[0] = bin, out[1] = elements in higher bins, out[2] = elements in it.
-// Select threads only.
-__device__ void find_rank_bin_smem(const int* hist, int r, int* red, int* out) {
-    const int t = threadIdx.x;
-    int h[kBpt];
-    int s = 0;
-#pragma unroll
-    for (int i = 0; i < kBpt; ++i) {
-        h[i] = hist[kBpt * t + i];
-        s += h[i];
-    }
-    int total;
-    const int excl = sel_scan_excl(s, red, total);
-    int above = total - excl - s;   // elements in bins above this thread's range
-    if (above < r && r <= above + s) {
-#pragma unroll
-        for (int i = kBpt - 1; i >= 0; --i) {
-            if (above < r && r <= above + h[i]) {
-                out[0] = kBpt * t + i;
-                out[1] = above;
-                out[2] = h[i];
-            }
-            above += h[i];
-        }
-    }
-    sel_sync();
-}
-
-// Totals of the histogram `h` that every CTA of the cluster holds at the same shared
-// address, into X.htot of every CTA. Every thread of the CTA calls this (it contains
-// two cluster barriers); the select threads do the work.
-__device__ void cl_hist_allreduce(const int* h, ClSel& X, int G, int rank) {
-    cluster_sync_all();   // every CTA's h is complete
-    const int per = (kBins + G - 1) / G;
-    if (threadIdx.x < kSel) {
-        const int b0 = rank * per, b1 = min(kBins, b0 + per);
-        for (int i = b0 + (int)threadIdx.x; i < b1; i += kSel) {
-            int s = 0;
-            for (int c = 0; c < G; ++c) s += ld_dsmem_i32(h + i, c);
-            X.hown[i] = s;
-        }
-    }
-    cluster_sync_all();   // every slice is summed
-    if (threadIdx.x < kSel)
-        for (int i = threadIdx.x; i < kBins; i += kSel) X.htot[i] = ld_dsmem_i32(&X.hown[i], i / per);
-    __syncthreads();
-}
-
-struct ClTrack {
-    int r, rrem, lo, hi, level;
-    bool on, all;
-    uint64_t prefix;
-};
-
-template <int DI>
-__global__ void __launch_bounds__(kTcThreads, 1)
-    index_full_cl_kernel(const __grid_constant__ IdxParams p, const __grid_constant__ CUtensorMap kmap) {
-    static_assert(DI == 32 || DI == 64 || DI == 128, "tensor-core key widths");
-    IdxSmem& S = idx_smem();
-    ClSel& X = *reinterpret_cast<ClSel*>(&S.stage[0][0]);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int G = p.G;
-    const int rank = (int)cluster_ctarank();
-    const int cl = blockIdx.x / G;
-    constexpr int kRows = (kStageBytes / DI) < 256 ? (kStageBytes / DI) : 256;
-    constexpr int kBlocks = kRows / 128;
-    constexpr uint32_t kSwz = DI == 32 ? 6u : DI == 64 ? 4u : 2u;
-    constexpr uint32_t kSbo = 8 * DI;
-    constexpr uint32_t kIdesc = idesc_i8(128, 16);
-
-    if (warp == 0) tmem_alloc(&S.tmem_base, 32 * kTmemBufs);
-    if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) { mbar_init(&S.full_bar[i], 1); mbar_init(&S.empty_bar[i], 1); }
-        for (int i = 0; i < kTmemBufs; ++i) { mbar_init(&S.tfull_bar[i], 1); mbar_init(&S.tempty_bar[i], kSel / 64); }
-        S.abort = 0;
-        mbar_fence_init();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    pdl_launch_dependents();
-    const bool producer = warp == kSel / 32;
-    if (!(producer && p.keys_ready)) pdl_wait();
-    const uint32_t tmem = S.tmem_base;
-    uint32_t seq = 0;
-
-    for (int u = cl; u < p.units; u += p.groups) {
-        const int b = u / p.Tq;
-        int t = p.q_pos[u];
-        int tg = last_entry(t, p.m);
-        if (t < 0 || tg >= p.N) {
-            if (tid == 0 && rank == 0) report(p.status, CSA2_ERR_RANGE, u);
-            tg = -1;
-        }
-        const int n_all = tg + 1;
-        const int lo = min(rank * p.chunk, n_all);
-        const int my_n = min(lo + p.chunk, n_all) - lo;
-        const int nst = p.pre ? 0 : (my_n + kRows - 1) / kRows;   // select only: no key tiles
-
-        // ---- the index query as the MMA's B operand; zero the histogram
-        if (warp != kSel / 32) {
-            constexpr int kStg = kTcThreads - 32;
-            const int li = tid < kSel ? tid : tid - 32;
-            fence_proxy_async_smem();
-            for (int i = li; i < p.Hi * DI / 16; i += kStg)
-                reinterpret_cast<int4*>(S.q)[i] = reinterpret_cast<const int4*>(p.qi + (size_t)u * p.Hi * DI)[i];
-            for (int i = li; i < kBins; i += kStg) S.hist0[i] = 0;
-            asm volatile("bar.sync 2, %0;" ::"n"(kStg) : "memory");
-            for (int i = li; i < DI; i += kStg) {
-                const int h = i / (DI / 16), c2 = i % (DI / 16);
-                int4 v = make_int4(0, 0, 0, 0);
-                if (h < p.Hi) v = reinterpret_cast<const int4*>(S.q + h * DI)[c2];
-                *reinterpret_cast<int4*>(S.qtc + tile_off(h, c2, DI)) = v;
-            }
-            fence_proxy_async_smem();
-            asm volatile("bar.sync 2, %0;" ::"n"(kStg) : "memory");
-        }
-
-        // ---- the scan (TMA producer, MMA issuer, epilogue), as in index_full_tc_kernel
-        if (warp == kSel / 32) {
-            if (lane == 0) {
-                const uint64_t pol = l2_evict_first_policy();
-                for (int s2 = 0; s2 < nst; ++s2) {
-                    const uint32_t i = seq + s2, slot = i % kStages;
-                    if (i >= (uint32_t)kStages &&
-                        !mbar_wait(&S.empty_bar[slot], ((i / kStages) - 1) & 1u, p.status, 5)) { S.abort = 1; break; }
-                    mbar_arrive_expect_tx(&S.full_bar[slot], (uint32_t)(kRows * DI));
-                    tma_load_keys(S.stage[slot], &kmap, 0, lo + s2 * kRows, b, &S.full_bar[slot], pol);
-                }
-            }
-        } else if (warp == kSel / 32 + 1) {
-            if (lane == 0) {
-                const uint32_t b0 = smem_u32(S.qtc);
-                for (int s2 = 0; s2 < nst; ++s2) {
-                    const uint32_t i = seq + s2, slot = i % kStages, buf = i % kTmemBufs;
-                    if (!mbar_wait(&S.full_bar[slot], (i / kStages) & 1u, p.status, 3)) { S.abort = 1; break; }
-                    if (i >= (uint32_t)kTmemBufs &&
-                        !mbar_wait(&S.tempty_bar[buf], ((i / kTmemBufs) - 1) & 1u, p.status, 6)) { S.abort = 1; break; }
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(S.stage[slot]);
-                    const uint32_t d0 = tmem + buf * 32u;
-#pragma unroll
-                    for (int blk = 0; blk < kBlocks; ++blk) {
-#pragma unroll
-                        for (int kk = 0; kk < DI / 32; ++kk)
-                            mma_i8(d0 + blk * 16, smem_desc(a0 + blk * 128 * DI + kk * 32, 16, kSbo, kSwz),
-                                   smem_desc(b0 + kk * 32, 16, kSbo, kSwz), kIdesc, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&S.empty_bar[slot]);
-                    mma_commit(&S.tfull_bar[buf]);
-                }
-            }
-        } else {
-            const int egrp = warp >> 3, wl = warp & 7, tl = tid & 255;
-            const bool in_block = (wl >> 2) < kBlocks;
-            const uint32_t lane_base = tmem + (uint32_t)(wl >> 2) * 16u + ((uint32_t)(wl & 3) * 32u << 16);
-            for (int s2 = egrp; s2 < nst; s2 += 2) {
-                const uint32_t i = seq + s2, buf = i % kTmemBufs;
-                const bool got = mbar_wait(&S.tfull_bar[buf], (i / kTmemBufs) & 1u, p.status, 4);
-                if (!__all_sync(0xffffffffu, got)) { S.abort = 1; break; }
-                tc_fence_after();
-                int x = 0;
-                if (in_block) {
-                    int acc[8];
-                    const uint32_t ta = lane_base + buf * 32u;
-                    tmem_ld8(ta, acc);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) x += p.w[h] * max(acc[h], 0);
-                    if (p.Hi > 8) {
-                        tmem_ld8(ta + 8, acc);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int h = 0; h < 8; ++h) x += p.w[8 + h] * max(acc[h], 0);
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.tempty_bar[buf]);
-                const int e = s2 * kRows + tl;
-                if (in_block && e < my_n) {
-                    S.sc[e] = x;
-                    atomicAdd(&S.hist0[bin0(x)], 1);
-                }
-            }
-        }
-        seq += nst;
-        __syncthreads();
-        // A CTA whose wait ran out (S.abort) still takes part in every cluster barrier of
-        // this query, with whatever scores it has: the cluster's barriers are not bounded,
-        // so no CTA may leave them early. The flag is shared below and every CTA leaves
-        // the loop together after this query.
-        const int my_abort = S.abort;
-        if (p.pre) {
-            // select only: the unit's scores come from the multi-query scoring kernel (16-byte
-            // loads, four in flight per thread; the unit's row and the chunk start are
-            // multiples of 4 elements), and the level-0 histogram is built here
-            const int* src = p.pre + (size_t)u * p.pstride + lo;
-            const int nv = my_n >> 2;
-            const int4* src4 = reinterpret_cast<const int4*>(src);
-#pragma unroll 1
-            for (int v0 = tid; v0 < nv; v0 += 4 * kTcThreads) {
-                int4 x4[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int v = v0 + q * kTcThreads;
-                    x4[q] = v < nv ? __ldcg(src4 + v) : make_int4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int v = v0 + q * kTcThreads;
-                    if (v >= nv) continue;
-                    reinterpret_cast<int4*>(S.sc)[v] = x4[q];
-                    atomicAdd(&S.hist0[bin0(x4[q].x)], 1);
-                    atomicAdd(&S.hist0[bin0(x4[q].y)], 1);
-                    atomicAdd(&S.hist0[bin0(x4[q].z)], 1);
-                    atomicAdd(&S.hist0[bin0(x4[q].w)], 1);
-                }
-            }
-            for (int e = 4 * nv + tid; e < my_n; e += kTcThreads) {
-                const int x = __ldcg(src + e);
-                S.sc[e] = x;
-                atomicAdd(&S.hist0[bin0(x)], 1);
-            }
-            __syncthreads();
-        }
-
-        // ---- 1. level-0 totals and each track's threshold bin
-        cl_hist_allreduce(S.hist0, X, G, rank);
-        ClTrack tk[2];
-#pragma unroll
-        for (int tr = 0; tr < 2; ++tr) {
-            ClTrack& k = tk[tr];
-            k.r = p.r[tr];
-            k.on = k.r > 0;
-            k.all = k.on && n_all <= k.r;
-            k.level = 0;
-            k.rrem = 0;
-            k.lo = 1;
-            k.hi = 0;
-            k.prefix = 0;
-        }
-        int cbig[2] = {0, 0};   // scores in the interval, cluster-wide
-        if (tid < kSel) {
-#pragma unroll
-            for (int tr = 0; tr < 2; ++tr) {
-                ClTrack& k = tk[tr];
-                if (!k.on || k.all) continue;
-                find_rank_bin_smem(X.htot, k.r, S.red, S.info + 8 * tr);
-                const int d = S.info[8 * tr];
-                k.rrem = k.r - S.info[8 * tr + 1];
-                cbig[tr] = S.info[8 * tr + 2];
-                k.prefix = (uint64_t)d;
-                bin0_interval((uint32_t)d, k.lo, k.hi);
-            }
-        }
-        // ---- 2. narrow an interval that holds too many scores (the same decisions in every CTA)
-#pragma unroll 1
-        for (int tr = 0; tr < 2; ++tr) {
-            // every thread must take part in the cluster barriers: the decision is shared
-            // through shared memory
-            if (tid == 0) S.info[40 + tr] = (tk[tr].on && !tk[tr].all) ? cbig[tr] : 0;
-            __syncthreads();
-            int cb = S.info[40 + tr];
-#pragma unroll 1
-            for (int lv = 1; lv <= 2 && cb > kCandCap; ++lv) {
-                if (tid < kSel) {
-                    for (int i = tid; i < kBins; i += kSel) X.hl[i] = 0;
-                    sel_sync();
-                    radix_hist<false>(S.sc, my_n, tk[tr].lo, tk[tr].hi, lv, X.hl);
-                }
-                cl_hist_allreduce(X.hl, X, G, rank);
-                if (tid < kSel) {
-                    ClTrack& k = tk[tr];
-                    find_rank_bin_smem(X.htot, k.rrem, S.red, S.info + 8 * tr);
-                    const int d = S.info[8 * tr];
-                    k.rrem -= S.info[8 * tr + 1];
-                    k.prefix = (k.prefix << 12) | (uint64_t)d;
-                    k.level = lv;
-                    prefix_interval(lv, k.prefix, k.lo, k.hi);
-                    if (tid == 0) S.info[40 + tr] = S.info[8 * tr + 2];
-                }
-                __syncthreads();
-                cb = S.info[40 + tr];
-            }
-        }
-        // ---- 3. candidates: own scores inside each interval, and own scores above it
-        if (tid < kSel) {
-            if (tid < 2) X.lcnt[tid] = 0;
-            sel_sync();
-            int above[2] = {0, 0};
-            for (int e = tid; e < my_n; e += kSel) {
-                const int x = S.sc[e];
-#pragma unroll
-                for (int tr = 0; tr < 2; ++tr) {
-                    const ClTrack& k = tk[tr];
-                    if (!k.on || k.all) continue;
-                    if (x > k.hi) ++above[tr];
-                    else if (x >= k.lo && k.level < 2) {
-                        const int slot = atomicAdd(&X.lcnt[tr], 1);
-                        if (slot < kCandCap) X.lc[tr][slot] = x;
-                    }
-                }
-            }
-            const int a0 = sel_sum(above[0], S.red);
-            const int a1 = sel_sum(above[1], S.red);
-            if (tid == 0) {
-                X.pub[0][0] = a0; X.pub[1][0] = a1;
-                X.pub[0][1] = min(X.lcnt[0], kCandCap); X.pub[1][1] = min(X.lcnt[1], kCandCap);
-                X.pub[0][3] = my_abort;
-            }
-        }
-        cluster_sync_all();   // every CTA's candidates and counts are published
-        int T[2] = {INT_MAX, INT_MAX}, need[2] = {0, 0};
-        if (tid < kSel) {
-            // every CTA's counts; exact tracks (the interval is one score) need no candidates
-            if (tid < 2 * G) {
-                const int tr = tid / G, c = tid % G;
-                X.above_c[tr][c] = ld_dsmem_i32(&X.pub[tr][0], c);   // above the interval
-                X.cnt_gt[tr][c] = ld_dsmem_i32(&X.pub[tr][1], c);    // in it (for the offsets below)
-            }
-            if (tid == 64) {
-                int a = 0;
-                for (int c = 0; c < G; ++c) a |= ld_dsmem_i32(&X.pub[0][3], c);
-                X.abort_any = a;
-            }
-            sel_sync();
-            if (tid < 2) {
-                int o = 0;
-                for (int c = 0; c < G; ++c) { X.goff[tid][c] = o; o = min(o + X.cnt_gt[tid][c], kCandCap); }
-                X.goff[tid][G] = o;
-            }
-            sel_sync();
-#pragma unroll
-            for (int tr = 0; tr < 2; ++tr) {
-                if (!tk[tr].on || tk[tr].all || tk[tr].level == 2) continue;
-                const int C = X.goff[tr][G];
-                for (int i = tid; i < C; i += kSel) {
-                    int c = 0;
-                    while (X.goff[tr][c + 1] <= i) ++c;
-                    if (CSA2_CHECK(i < kCandCap && c < G && i - X.goff[tr][c] < kCandCap, p.status, 2301))
-                        X.gc[tr][i] = ld_dsmem_i32(&X.lc[tr][i - X.goff[tr][c]], c);
-                }
-            }
-            sel_sync();
-        }
-        // the exchange is done: no CTA reads another's shared memory for this query any more
-        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-        ListCut cut[2];
-        if (tid < kSel) {
-#pragma unroll
-            for (int tr = 0; tr < 2; ++tr) {
-                const ClTrack& k = tk[tr];
-                if (!k.on || k.all) continue;
-                if (k.level == 2) {   // the interval is the single score T
-                    T[tr] = k.lo;
-                    need[tr] = k.rrem;
-                    continue;
-                }
-                // the rrem-th best candidate: two 12-bit digits of its offset in the interval
-                const int C = X.goff[tr][G];
-                for (int i = tid; i < kBins; i += kSel) X.hl[i] = 0;
-                sel_sync();
-                for (int i = tid; i < C; i += kSel) atomicAdd(&X.hl[((uint32_t)(X.gc[tr][i] - k.lo) >> 12) & 4095u], 1);
-                sel_sync();
-                find_rank_bin_smem(X.hl, k.rrem, S.red, S.info + 24);
-                const uint32_t d1 = (uint32_t)S.info[24];
-                const int above1 = S.info[25];
-                for (int i = tid; i < kBins; i += kSel) X.hl[i] = 0;
-                sel_sync();
-                for (int i = tid; i < C; i += kSel) {
-                    const uint32_t off = (uint32_t)(X.gc[tr][i] - k.lo);
-                    if (((off >> 12) & 4095u) == d1) atomicAdd(&X.hl[off & 4095u], 1);
-                }
-                sel_sync();
-                find_rank_bin_smem(X.hl, k.rrem - above1, S.red, S.info + 24);
-                T[tr] = k.lo + (int)((d1 << 12) | (uint32_t)S.info[24]);
-                need[tr] = k.rrem - above1 - S.info[25];
-            }
-            // per-CTA counts above T and ties at T: from the candidates (their owner is
-            // known by offset) or, for an exact track, by a sweep of own scores published
-            // in the level-2 case below
-            if (tid < 2 * kClMaxG) { (&X.cnt_gt[0][0])[tid] = 0; (&X.cnt_eq[0][0])[tid] = 0; }   // reused as counts of candidates
-            sel_sync();
-#pragma unroll
-            for (int tr = 0; tr < 2; ++tr) {
-                if (!tk[tr].on || tk[tr].all || tk[tr].level == 2) continue;
-                const int C = X.goff[tr][G];
-                for (int i = tid; i < C; i += kSel) {
-                    int c = 0;
-                    while (X.goff[tr][c + 1] <= i) ++c;
-                    const int x = X.gc[tr][i];
-                    if (x > T[tr]) atomicAdd(&X.cnt_gt[tr][c], 1);
-                    else if (x == T[tr]) atomicAdd(&X.cnt_eq[tr][c], 1);
-                }
-            }
-            sel_sync();
-        }
-        // exact tracks: every CTA's ties at T (the interval) by a sweep, one more exchange
-        const bool exact = (tk[0].on && !tk[0].all && tk[0].level == 2) || (tk[1].on && !tk[1].all && tk[1].level == 2);
-        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-        if (__syncthreads_or(exact && tid < kSel)) {
-            if (tid < kSel) {
-                int eq[2] = {0, 0};
-                for (int e = tid; e < my_n; e += kSel) {
-                    const int x = S.sc[e];
-#pragma unroll
-                    for (int tr = 0; tr < 2; ++tr) eq[tr] += (tk[tr].level == 2 && x == tk[tr].lo);
-                }
-                const int e0 = sel_sum(eq[0], S.red), e1 = sel_sum(eq[1], S.red);
-                if (tid == 0) { X.pub[0][2] = e0; X.pub[1][2] = e1; }
-            }
-            cluster_sync_all();
-            if (tid < 2 * G) {
-                const int tr = tid / G, c = tid % G;
-                if (tk[tr].level == 2) X.cnt_eq[tr][c] = ld_dsmem_i32(&X.pub[tr][2], c);
-            }
-            cluster_sync_all();   // the reads are done
-        }
-        if (tid < kSel) {
-            // this CTA's output offset and tie quota, per track
-#pragma unroll
-            for (int tr = 0; tr < 2; ++tr) {
-                ListCut& lc = cut[tr];
-                const ClTrack& k = tk[tr];
-                lc.r = k.r;
-                lc.out = k.on ? p.out[tr] + (size_t)u * k.r : nullptr;
-                lc.all = k.all;
-                lc.T = T[tr];
-                lc.quota = 0;
-                lc.base = lo;
-                if (!k.on || k.all) continue;
-                int base = 0, eq_before = 0;
-                for (int c = 0; c < rank; ++c) {
-                    const int eqc = X.cnt_eq[tr][c];
-                    const int q = max(0, min(need[tr] - eq_before, eqc));
-                    base += X.above_c[tr][c] + X.cnt_gt[tr][c] + q;
-                    eq_before += eqc;
-                }
-                lc.quota = max(0, min(need[tr] - eq_before, X.cnt_eq[tr][rank]));
-                lc.base = base;
-            }
-            write_lists<false>(S.sc, my_n, lo, nullptr, cut[0], cut[1], S.wsum, row_prefetch(p, u));
-            if (rank == G - 1) {
-#pragma unroll
-                for (int tr = 0; tr < 2; ++tr)
-                    if (cut[tr].out)
-                        for (int i = min(cut[tr].r, n_all) + tid; i < cut[tr].r; i += kSel) cut[tr].out[i] = -1;
-            }
-        }
-        __syncthreads();
-        if (X.abort_any) break;   // the same decision in every CTA of the cluster
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 32 * kTmemBufs);
-}
-
 // ------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -2696,28 +2199,6 @@ static cudaError_t launch_coop(Kern kern, int threads, const IdxParams& p, const
 // Cluster launch of the Full kernel: clusters of q.G CTAs, q.groups clusters, programmatic
 // stream serialisation (the kernel reads nothing the previous kernel writes before
 // griddepcontrol.wait, except that a producer with keys_ready starts the key stream).
-template <typename Kern>
-static cudaError_t launch_cl(Kern kern, const IdxParams& q, const CUtensorMap& map, cudaStream_t stream) {
-    const size_t smem = index_smem_bytes();
-    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(q.G * q.groups);
-    cfg.blockDim = dim3(kTcThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = q.G;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, q, map);
-}
-
 template <int DI>
 static cudaError_t launch_mq(const MqParams& mp, const CUtensorMap& map, int grid, cudaStream_t stream) {
     auto kern = index_mq_score_kernel<DI>;
@@ -2738,21 +2219,9 @@ static cudaError_t launch_mq(const MqParams& mp, const CUtensorMap& map, int gri
     return cudaLaunchKernelEx(&cfg, kern, mp, map);
 }
 
-int reindex_cluster_size(const csa2_index_args& a, int P_in);
-csa2_status launch_reindex_cl(const csa2_index_args& a, const int32_t* pool_in, int P_in, int pool_ready,
-                              const csa2_attn_args* pf, int32_t* d_status, cudaStream_t stream);
-
 // Launch one indexer call. `ws` holds plan_index(a).ws_bytes bytes (zero at first use).
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
                          int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready) {
-    static const int rx_path = [] {
-        const char* e = getenv("CSA2_REINDEX_PATH");
-        return e ? atoi(e) : 0;
-    }();
-    // Reindex over a pool of at most a few thousand entries per CTA: the clustered kernel
-    // (reindex.cu); its pool was written two or more kernels back when keys_ready is set
-    if (a.mode == CSA2_REINDEX && rx_path == 0 && reindex_cluster_size(a, P_in) > 0)
-        return launch_reindex_cl(a, pool_in, P_in, keys_ready, pf, d_status, stream);
     const int sms = num_sms();
     csa2_index_args aa = a;
     aa.P_in = P_in;
@@ -2851,40 +2320,6 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
                          : launch_mq<128>(mp, mmap, mgrid, stream);
         if (e != cudaSuccess) return CSA2_ERR_CUDA;
     }
-    // Full mode whose query groups fit a cluster: the cluster kernel, no workspace state
-    static const int full_path = [] {
-        const char* ev = getenv("CSA2_FULL_PATH");
-        return ev ? atoi(ev) : 0;
-    }();
-    bool cl_done = false;
-    if (a.mode == CSA2_FULL && full_path == 0 && (a.Di == 32 || a.Di == 64 || a.Di == 128)) {
-        const int units = a.B * a.Tq;
-        // a scan: the widest cluster the SMs allow per unit (up to 8, at least 1024 keys a CTA);
-        // select only (after the multi-query scoring kernel): the narrowest whose chunks fit
-        // shared memory, so that more units are cut at once
-        int G = std::max(1, std::min(std::min(kClMaxG / 2, sms / std::max(1, std::min(units, sms))),
-                                     (a.N + 1023) / 1024));
-        if (pl.mq) G = std::max(1, (a.N + kSmemScores - 1) / kSmemScores);
-        int chunk = (int)align_up((size_t)((a.N + G - 1) / G), 256);
-        if (pl.mq && chunk > kSmemScores) {   // the rounding to 256 pushed a chunk past shared memory
-            ++G;
-            chunk = (int)align_up((size_t)((a.N + G - 1) / G), 256);
-        }
-        if (chunk <= kSmemScores && G <= kClMaxG / 2) {
-            IdxParams q = p;
-            q.G = G;
-            q.groups = std::min(units, std::max(1, sms / G));
-            q.chunk = chunk;
-            q.spill = nullptr;
-            q.pre = pl.mq ? static_cast<int32_t*>(scratch) : nullptr;
-            const cudaError_t ce = a.Di == 64 ? launch_cl(index_full_cl_kernel<64>, q, map, stream)
-                                   : a.Di == 32 ? launch_cl(index_full_cl_kernel<32>, q, map, stream)
-                                                : launch_cl(index_full_cl_kernel<128>, q, map, stream);
-            if (ce != cudaSuccess) return CSA2_ERR_CUDA;
-            cl_done = true;
-        }
-    }
-    if (cl_done) return CSA2_OK;
     if (a.mode == CSA2_FULL && a.Di == 64) e = launch_coop(index_full_tc_kernel<64>, kTcThreads, p, map, grid, stream);
     else if (a.mode == CSA2_FULL && a.Di == 32) e = launch_coop(index_full_tc_kernel<32>, kTcThreads, p, map, grid, stream);
     else if (a.mode == CSA2_FULL && a.Di == 128) e = launch_coop(index_full_tc_kernel<128>, kTcThreads, p, map, grid, stream);

@@ -4,8 +4,8 @@ Each output buffer (pool, top-k list, bf16 out, fp32 lse of every layer) is carv
 from a larger allocation whose bytes before and after it hold a known pattern.
 After the call the patterns must be intact: no kernel writes outside the buffers
 the caller passed. The workloads are small enough to run in seconds but cover the
-cluster Full kernel, the clustered Reindex, the slice attention, the ticket merge
-and the cooperative kernel with spilled scores."""
+Full and Reindex kernels (scores in shared memory and spilled), the multi-query
+scoring kernel, the cluster attention and the ticket merge."""
 import numpy as np
 import pytest
 import torch
@@ -64,7 +64,7 @@ def _guarded_stack(wl):
 
 
 @pytest.mark.parametrize("name,kw", [
-    ("stack20_128k", dict(B=3, N=20000)),                    # cluster Full, clustered Reindex, slice attention
+    ("stack20_128k", dict(B=3, N=20000)),                    # Full, Reindex, cluster attention
     ("paper_schedule", dict(B=2, N=9000)),
     ("long_1m", dict(N=40000, Tq=6)),                        # multi-query scoring + cooperative select
     ("decode_full", dict(B=150, N=20000)),                   # more units than SMs: one CTA per unit, spilled scores

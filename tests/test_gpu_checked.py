@@ -1,9 +1,9 @@
 """The range-checked build (libcsa2_checked.so, compiled with -DCSA2_CHECKED).
 
-In that build every computed shared- or global-memory index of the cluster kernels
-(slice attention, clustered Reindex, the Full kernel's candidate exchange, the cache
-append) is checked before its access and a violation goes to the status word as
-CSA2_ERR_RANGE. Here a set of parity tests runs in a child process against that
+In that build the computed indices that the kernels' bounds rest on (the ordered list
+writes of the select, the attention cluster's merge rows, the ticket merge's tile
+buffers, the cache append's local rows) are checked before their access and a
+violation goes to the status word as CSA2_ERR_RANGE. Here a set of parity tests runs in a child process against that
 library: they must pass, and no check may fire (every test checks the status word)."""
 import os
 import subprocess

@@ -45,9 +45,8 @@ def _timed_failing_call(fn):
 
 @pytest.mark.parametrize("mode", ["FULL", "REINDEX"])
 def test_group_wait_runs_out_and_the_next_call_is_exact(mode):
-    # Sizes that take the cooperative kernels, whose CTAs meet at spin barriers: a Full
-    # chunk beyond a cluster's shared memory (4 queries x 400000 keys), and a Reindex pool
-    # beyond the clustered kernel's 16384 entries (the group's distributed select).
+    # Groups of several CTAs per query, which meet at spin barriers: 4 queries x 400000
+    # keys in Full mode, and a Reindex pool of 20000 entries (the group's distributed select).
     B, N, k, P = 4, 400000, 1024, 20000
     qi, w, ki, q_pos = _inputs(11, B, N)
     ws, st = ops.Workspace(), ops.Status()

@@ -288,10 +288,11 @@ def test_attention_tiny(ws, status):
     (2, 4096, 1, 16, 128, 1, 0),         # single global entry, no window
     (2, 4096, 1, 16, 128, 2048, 0),      # no local branch
     (1, 300, 1, 16, 128, 512, 64),       # fewer positions than k: -1 padding
-    (2, 8192, 1, 16, 128, 4096, 1024),   # 8 CTAs of 4 blocks and a window tile each: the largest cluster
-    (2, 8192, 1, 16, 128, 4096, 2048),   # 16 window tiles: more than one cluster holds, ticket merge
+    (2, 8192, 1, 16, 128, 4096, 1024),   # 16 list CTAs + 8 window CTAs: past the cluster limit, ticket merge
+    (2, 8192, 1, 16, 128, 4096, 2048),   # 16 window tiles: ticket merge
     (3, 5000, 1, 32, 64, 700, 300),      # 32 heads at D = 64, ragged blocks
-    (2, 4096, 1, 16, 128, 1, 512),       # one global entry, four window tiles: CTAs with no global block
+    (2, 4096, 1, 16, 128, 1, 512),       # one global entry, four window tiles
+    (1, 20000, 1, 32, 128, 100, 16284),  # k + W = 16384 with both branches ragged: 129 tiles, 32 heads
 ])
 def test_attention_shapes(B, N, Tq, Hq, D, k, W, ws, status):
     _attn_case(B, N, Tq, Hq, D, k, W, seed=B * 7 + N, ws=ws, status=status)
