@@ -75,7 +75,7 @@ struct IdxParams {
     int P_in;
     int units, G, groups, chunk;
     int32_t* spill;      // [groups*G][chunk] scores when chunk > kSmemScores
-    int local_sel;       // Reindex: the group leader selects over all of the unit's scores
+    int local_sel;       // Reindex: every CTA of the group cuts over all of the unit's scores
     int keys_ready;      // keys and positions were complete before the previous kernel began
     const int32_t* pre;  // Full, select only: every unit's scores by position ([units][pstride]), else nullptr
     int64_t pstride;
@@ -85,6 +85,11 @@ struct IdxParams {
     const uint8_t* pf_fp4;
     const uint8_t* pf_scale;
     int pf_N, pf_code_bytes, pf_scale_bytes;
+    // L2 prefetch of the index-key rows of the pool entries, for the Reindex layer that
+    // rescores this pool (pk_keys nullptr: off)
+    const int8_t* pk_keys;
+    int64_t pk_seq_stride;
+    int pk_row_bytes;
     int m;                   // sequence compression rate of the global entries (<= 1: one per position)
     long long wait_budget;   // SM cycles a CTA waits at a group barrier before it reports a timeout
     int skip_arrival;        // fault injection: the last CTA of a group never arrives at its first barrier
@@ -410,16 +415,21 @@ __device__ __forceinline__ int2 sel_scan_excl2(int2 v, int* red, int2& total) {
 
 // The thresholds of both tracks at once. For track k (skipped when Ck = 0): the
 // rk-th largest value (1-based, with multiplicity) among the values xk[0..Ck) in
-// shared memory that lie in [lok, hik] (others are ignored), by radix passes of up
-// to 12 bits over x - lok (a pass of b bits uses max(kSel, 2^b) bins, thread t
-// owning bins [per*t, per*t + per)). The two tracks share every barrier.
-// Returns {T0, need0, T1, need1}: need = how many elements equal to T are ranked
-// within the first r.
+// shared memory that lie in [lok, hik] (others are ignored). Radix passes of up to 8
+// bits over x - lok, from the top: the select threads count the values that share the
+// digits fixed so far into a 256-bin histogram per track, then warp k alone finds the
+// bin holding rank rk (eight bins per lane and one suffix scan across the lanes). A
+// pass costs two barriers; the histograms are double-buffered so the next pass's
+// buffer is cleared during this one. A track whose chosen bin holds at most 32 values
+// with bits still to resolve ranks those values directly instead.
+// hist: 1088 ints ([2 buffers][2 tracks][256] and [2][32] values). The two tracks
+// share every barrier. Returns {T0, need0, T1, need1}: need = how many elements
+// equal to T are ranked within the first r.
+static_assert(kSel == 2 * 256, "local_select2: one histogram bin of one track per select thread");
 __device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo0, int hi0, const int* x1, int C1,
                                            int r1, int lo1, int hi1, int* hist, int* red, int* info) {
-    const int t = threadIdx.x;
-    int* h0 = hist;
-    int* h1 = hist + kBins;
+    (void)red;
+    const int t = threadIdx.x, lane = t & 31, wk = t >> 5;
     auto nbits = [](int lo, int hi) {
         const uint32_t w = (uint32_t)((long long)hi - (long long)lo);
         return w == 0u ? 0 : 32 - __clz(w);
@@ -428,22 +438,23 @@ __device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo
     uint32_t pf0 = 0, pf1 = 0;
     int T0 = 0, T1 = 0;
     bool fin0 = false, fin1 = false;   // threshold found by ranking the last few values directly
+    int* bv = hist + 1024;             // the last few values of each track
+    hist[t] = 0;                       // buffer 0 (kSel = 2 tracks x 256 bins)
+    sel_sync();
+    int buf = 0;
 #pragma unroll 1
     while (rem0 > 0 || rem1 > 0) {
-        const int tk0 = min(rem0, 12), sh0 = rem0 - tk0, per0 = rem0 > 0 ? max(kSel, 1 << tk0) / kSel : 0;
-        const int tk1 = min(rem1, 12), sh1 = rem1 - tk1, per1 = rem1 > 0 ? max(kSel, 1 << tk1) / kSel : 0;
-#pragma unroll 1
-        for (int i = t; i < kSel * per0; i += kSel) h0[i] = 0;
-#pragma unroll 1
-        for (int i = t; i < kSel * per1; i += kSel) h1[i] = 0;
-        sel_sync();
+        int* hb = hist + buf * 512;
+        const int tk0 = min(rem0, 8), sh0 = rem0 - tk0;
+        const int tk1 = min(rem1, 8), sh1 = rem1 - tk1;
+        hist[(buf ^ 1) * 512 + t] = 0;   // last read before the barrier that ended the previous pass
         if (rem0 > 0) {
 #pragma unroll 1
             for (int i = t; i < C0; i += kSel) {
                 const int x = x0[i];
                 const uint32_t v = (uint32_t)((long long)x - (long long)lo0);
                 if (x >= lo0 && x <= hi0 && (uint32_t)(((uint64_t)v) >> (sh0 + tk0)) == pf0)
-                    atomicAdd(&h0[(v >> sh0) & ((1u << tk0) - 1u)], 1);
+                    atomicAdd(&hb[(v >> sh0) & ((1u << tk0) - 1u)], 1);
             }
         }
         if (rem1 > 0) {
@@ -452,48 +463,51 @@ __device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo
                 const int x = x1[i];
                 const uint32_t v = (uint32_t)((long long)x - (long long)lo1);
                 if (x >= lo1 && x <= hi1 && (uint32_t)(((uint64_t)v) >> (sh1 + tk1)) == pf1)
-                    atomicAdd(&h1[(v >> sh1) & ((1u << tk1) - 1u)], 1);
+                    atomicAdd(&hb[256 + ((v >> sh1) & ((1u << tk1) - 1u))], 1);
             }
         }
         sel_sync();
-        int s0 = 0, s1 = 0;
-#pragma unroll 1
-        for (int i = 0; i < per0; ++i) s0 += h0[per0 * t + i];
-#pragma unroll 1
-        for (int i = 0; i < per1; ++i) s1 += h1[per1 * t + i];
-        int2 tot;
-        const int2 ex = sel_scan_excl2(make_int2(s0, s1), red, tot);
-        int ab0 = tot.x - ex.x - s0, ab1 = tot.y - ex.y - s1;   // elements in bins above this thread's range
-        if (rem0 > 0 && ab0 < r0 && r0 <= ab0 + s0) {
-#pragma unroll 1
-            for (int i = per0 - 1; i >= 0; --i) {
-                const int h = h0[per0 * t + i];
-                if (r0 <= ab0 + h) { info[0] = per0 * t + i; info[1] = ab0; info[4] = h; break; }
-                ab0 += h;
+        if (wk < 2 && (wk == 0 ? rem0 : rem1) > 0) {
+            // warp wk: lane l holds bins 8l .. 8l + 7; the bin with (count above) < r <= (count above) + its count
+            const int r = wk == 0 ? r0 : r1;
+            const int4* h4 = reinterpret_cast<const int4*>(hb + wk * 256 + 8 * lane);
+            const int4 ha = h4[0], hb4 = h4[1];
+            const int hv[8] = {ha.x, ha.y, ha.z, ha.w, hb4.x, hb4.y, hb4.z, hb4.w};
+            int sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum += hv[i];
+            int incl = sum;   // this lane's bins and every higher lane's
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_down_sync(0xffffffffu, incl, o);
+                if (lane + o < 32) incl += y;
             }
-        }
-        if (rem1 > 0 && ab1 < r1 && r1 <= ab1 + s1) {
-#pragma unroll 1
-            for (int i = per1 - 1; i >= 0; --i) {
-                const int h = h1[per1 * t + i];
-                if (r1 <= ab1 + h) { info[2] = per1 * t + i; info[3] = ab1; info[5] = h; break; }
-                ab1 += h;
+            int above = incl - sum;
+            if (above < r && r <= incl) {
+#pragma unroll
+                for (int i = 7; i >= 0; --i) {
+                    if (r <= above + hv[i]) {
+                        info[3 * wk] = 8 * lane + i;
+                        info[3 * wk + 1] = above;
+                        info[3 * wk + 2] = hv[i];
+                        break;
+                    }
+                    above += hv[i];
+                }
             }
         }
         if (t == 0) { info[6] = 0; info[7] = 0; }
         sel_sync();
         if (rem0 > 0) { r0 -= info[1]; pf0 = (pf0 << tk0) | (uint32_t)info[0]; rem0 = sh0; }
-        if (rem1 > 0) { r1 -= info[3]; pf1 = (pf1 << tk1) | (uint32_t)info[2]; rem1 = sh1; }
-        // a track whose chosen bin holds at most 32 values, with bits still to resolve,
-        // finishes by ranking those values directly instead of another radix pass
-        const bool bf0 = rem0 > 0 && info[4] <= 32, bf1 = rem1 > 0 && info[5] <= 32;
+        if (rem1 > 0) { r1 -= info[4]; pf1 = (pf1 << tk1) | (uint32_t)info[3]; rem1 = sh1; }
+        const bool bf0 = rem0 > 0 && info[2] <= 32, bf1 = rem1 > 0 && info[5] <= 32;
         if (bf0 || bf1) {
-            if (bf0) {   // this track's histogram is no longer needed: it holds the values
+            if (bf0) {
 #pragma unroll 1
                 for (int i = t; i < C0; i += kSel) {
                     const int x = x0[i];
                     const uint32_t v = (uint32_t)((long long)x - (long long)lo0);
-                    if (x >= lo0 && x <= hi0 && (uint32_t)(((uint64_t)v) >> rem0) == pf0) h0[atomicAdd(&info[6], 1) & 31] = x;
+                    if (x >= lo0 && x <= hi0 && (uint32_t)(((uint64_t)v) >> rem0) == pf0) bv[atomicAdd(&info[6], 1) & 31] = x;
                 }
             }
             if (bf1) {
@@ -501,17 +515,17 @@ __device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo
                 for (int i = t; i < C1; i += kSel) {
                     const int x = x1[i];
                     const uint32_t v = (uint32_t)((long long)x - (long long)lo1);
-                    if (x >= lo1 && x <= hi1 && (uint32_t)(((uint64_t)v) >> rem1) == pf1) h1[atomicAdd(&info[7], 1) & 31] = x;
+                    if (x >= lo1 && x <= hi1 && (uint32_t)(((uint64_t)v) >> rem1) == pf1)
+                        bv[32 + (atomicAdd(&info[7], 1) & 31)] = x;
                 }
             }
             sel_sync();
             // warp 0 ranks track 0's values, warp 1 track 1's: the value with
             // (#larger) < r <= (#larger or equal) is the threshold
-            const int wk = t >> 5, ln = t & 31;
             if ((wk == 0 && bf0) || (wk == 1 && bf1)) {
-                const int m = min(wk == 0 ? info[6] : info[7], 32);
+                const int m = min(info[6 + wk], 32);
                 const int r = wk == 0 ? r0 : r1;
-                const int vi = ln < m ? (wk == 0 ? h0[ln] : h1[ln]) : 0;
+                const int vi = lane < m ? bv[32 * wk + lane] : 0;
                 int gt = 0, ge = 0;
 #pragma unroll 1
                 for (int j = 0; j < m; ++j) {
@@ -519,12 +533,13 @@ __device__ __noinline__ int4 local_select2(const int* x0, int C0, int r0, int lo
                     gt += vj > vi;
                     ge += vj >= vi;
                 }
-                if (ln < m && gt < r && r <= ge) { info[8 + 2 * wk] = vi; info[9 + 2 * wk] = r - gt; }
+                if (lane < m && gt < r && r <= ge) { info[8 + 2 * wk] = vi; info[9 + 2 * wk] = r - gt; }
             }
             sel_sync();
             if (bf0) { T0 = info[8]; r0 = info[9]; fin0 = true; rem0 = 0; }
             if (bf1) { T1 = info[10]; r1 = info[11]; fin1 = true; rem1 = 0; }
         }
+        buf ^= 1;
     }
     return make_int4(fin0 ? T0 : (int)((long long)lo0 + (long long)pf0), r0,
                      fin1 ? T1 : (int)((long long)lo1 + (long long)pf1), r1);
@@ -887,10 +902,16 @@ struct RowPrefetch {
     const uint8_t* fp4;     // the sequence's codes [N][code_bytes]
     const uint8_t* scale;   // the sequence's scales [N][scale_bytes]
     int code_bytes, scale_bytes;
+    const int8_t* keys;     // the sequence's index keys of the Reindex layer that rescores the pool
+    int key_bytes;
 };
 
 __device__ __forceinline__ RowPrefetch row_prefetch(const IdxParams& p, int u) {
-    RowPrefetch f{nullptr, nullptr, 0, 0};
+    RowPrefetch f{nullptr, nullptr, 0, 0, nullptr, 0};
+    if (p.pk_keys != nullptr) {
+        f.keys = p.pk_keys + (size_t)(u / p.Tq) * p.pk_seq_stride;
+        f.key_bytes = p.pk_row_bytes;
+    }
     if (p.pf_fp4 != nullptr) {
         const size_t b = (size_t)(u / p.Tq);
         f.fp4 = p.pf_fp4 + b * p.pf_N * p.pf_code_bytes;
@@ -905,6 +926,11 @@ __device__ __forceinline__ void prefetch_row(const RowPrefetch& f, int pos) {
     if (f.fp4 == nullptr || pos < 0) return;
     asm volatile("prefetch.global.L2 [%0];" ::"l"(f.fp4 + (size_t)pos * f.code_bytes));
     asm volatile("prefetch.global.L2 [%0];" ::"l"(f.scale + (size_t)pos * f.scale_bytes));
+}
+
+__device__ __forceinline__ void prefetch_key(const RowPrefetch& f, int pos) {
+    if (f.keys == nullptr || pos < 0) return;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(f.keys + (size_t)pos * f.key_bytes));
 }
 
 __device__ __forceinline__ void take_flags(int x, bool ok, const ListCut& c, bool& g, bool& e) {
@@ -957,7 +983,7 @@ __device__ __forceinline__ void write_lists(const int* sc, int n, int base, cons
         const bool t0 = g0 || (q0 && oq0 < c0.quota), t1 = g1 || (q1 && oq1 < c1.quota);
         if (t0 || t1) {
             const int pos = pool ? pool[base + e] : base + e;
-            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) c0.out[k] = pos; }
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) { c0.out[k] = pos; prefetch_key(pf, pos); } }
             if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c1.r, c1.status, 2202)) { c1.out[k] = pos; prefetch_row(pf, pos); } }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
@@ -1015,7 +1041,7 @@ __device__ __forceinline__ void write_from_lists(const int* sc, int base, const 
         if (t0 || t1) {
             const int e = base + (ent & 0x0FFFFFFF);
             const int pos = pool ? pool[e] : e;
-            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) c0.out[k] = pos; }
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) { c0.out[k] = pos; prefetch_key(pf, pos); } }
             if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c1.r, c1.status, 2202)) { c1.out[k] = pos; prefetch_row(pf, pos); } }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
@@ -1293,14 +1319,15 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
 
 // ------------------------------------------------------------ Reindex: one select per group
 // A Reindex pool fits in one CTA's shared memory, so the group does not run the
-// distributed select: every CTA publishes its scores (element order) and its
-// element count and meets the group at one barrier; then the group's first CTA
-// loads all of the unit's scores and cuts top-k alone, with the same order key,
-// the same exact threshold search and the same tie rule, while the others go on
-// to their next unit.
+// distributed select: every CTA publishes its scores (element order) and its element
+// count and meets the group at one barrier. Then every CTA loads all of the unit's
+// scores and finds the same exact cut (the order key's level-0 bin of the k-th best
+// score, the bin's scores as candidates, the exact threshold T and the number of ties
+// at T to take), and writes its own chunk's selected entries at its offset in the
+// list (the entries taken before its chunk), in pool order, which is position order.
 __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c,
                                                    int& bar_target) {
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     int32_t* rs = p.rscore + (size_t)c.u * p.rstride;
     int* cnt = sl.g0 + ((c.epoch + c.j) % 3) * kG0Stride + kBins;
     int* cnt_next = sl.g0 + ((c.epoch + c.j + 1) % 3) * kG0Stride + kBins;
@@ -1317,19 +1344,19 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         for (int i = zlo + tid; i < zhi; i += kSel) g0nxt[i] = 0;
         if (tid == 0 && c.cta == 0) *cnt_next = 0;
     }
-    // every CTA waits: the leader's zeroing of the next unit's count (above) is then
+    // every CTA waits: the first CTA's zeroing of the next unit's count (above) is then
     // ordered before any CTA's add for that unit
     bar_target += p.G;
     if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status, p.wait_budget,
                        p.skip_arrival && c.cta == p.G - 1))
         return false;
-    if (c.cta != 0) return true;
 
-    // the leader: all scores of the unit (valid pool entries form a prefix), as int4
-    // vectors with every load of a thread in flight at once
+    // all scores of the unit (valid pool entries form a prefix), as int4 vectors with
+    // every load of a thread in flight at once, and their level-0 histogram
     const int n = min(max(__ldcg(cnt), 0), p.P_in);
 #pragma unroll 1
     for (int i = tid; i < kBins; i += kSel) S.hist0[i] = 0;
+    if (tid == 0) S.info[20] = 0;
     sel_sync();
     {
         const int nv = (n + 3) >> 2;   // rstride is a multiple of 4: whole vectors stay in the unit's row
@@ -1355,7 +1382,7 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
     const int r = p.r[1];
     ListCut none{INT_MAX, 0, 0, 0, 0, nullptr, p.status};
     ListCut cut{INT_MAX, 0, 0, 0, r, p.out[1] + (size_t)c.u * r, p.status};
-    bool lists = false;
+    int T = INT_MAX, need = 0;
     if (n <= r) {
         cut.all = 1;
     } else {
@@ -1373,35 +1400,56 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
                 above += h[i];
             }
         }
-        if (tid == 0) S.wlist_ovf = 0;
         sel_sync();
         int blo, bhi;
         bin0_interval((uint32_t)S.info[0], blo, bhi);
         const int rrem = r - S.info[1];
-        // one pass builds the warps' ordered lists (top-k is track 1); the threshold
-        // comes from a radix select over the scores inside the bin's interval
-        gather_lists2<false>(S.sc, n, 1, 0, blo, bhi, wlists(S), S.wlist_n, &S.wlist_ovf, nullptr);
-        sel_sync();
-        // the radix select runs over the bin's elements only (from the lists), or over
-        // all n scores when a list overflowed; the key stages are free in Reindex mode
-        const int* xs = S.sc;
-        int nx = n;
-        if (S.wlist_ovf == 0) {
-            int* cx = reinterpret_cast<int*>(&S.stage[0][0]);
-            nx = vals_from_lists(S.sc, wlists(S), S.wlist_n, 8u, cx, S.wsum);
-            xs = cx;
-        }
-        const int4 ls = local_select2(S.sc, 0, 0, 1, 0, xs, nx, rrem, blo, bhi, histl(S, 0), S.red, S.info);
-        cut.T = ls.z;
-        cut.quota = ls.w;   // the ties at T ranked within the first r, all in this CTA
-        lists = S.wlist_ovf == 0;
-    }
-    if (lists)
-        write_from_lists<false>(S.sc, 0, c.pool, wlists(S), S.wlist_n, none, cut, S.wsum, row_prefetch(p, c.u));
-    else
-        write_lists<false>(S.sc, n, 0, c.pool, none, cut, S.wsum, row_prefetch(p, c.u));
+        // the bin's scores (any order) are the candidates; one reservation per warp and step
+        int* cx = reinterpret_cast<int*>(&S.stage[0][0]);
+        const unsigned below = (1u << lane) - 1u;
 #pragma unroll 1
-    for (int i = min(r, n) + tid; i < r; i += kSel) cut.out[i] = -1;
+        for (int e0 = 0; e0 < n; e0 += kSel) {
+            const int e = e0 + tid;
+            const int x = e < n ? S.sc[e] : 0;
+            const bool in = e < n && x >= blo && x <= bhi;
+            const unsigned b = __ballot_sync(0xffffffffu, in);
+            if (b == 0u) continue;
+            int w = 0;
+            if (lane == 0) w = atomicAdd(&S.info[20], __popc(b));
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (in) cx[w + __popc(b & below)] = x;
+        }
+        sel_sync();
+        const int nx = S.info[20];
+        const int4 ls = local_select2(S.sc, 0, 0, 1, 0, cx, nx, rrem, blo, bhi, histl(S, 0), S.red, S.info);
+        T = ls.z;
+        need = ls.w;   // the ties at T ranked within the first r
+    }
+    // this CTA's offset: the entries taken before its chunk; its own share of the ties
+    {
+        int4 a = make_int4(0, 0, 0, 0), bb = make_int4(0, 0, 0, 0);
+        const int e_end = min(c.lo + c.my_n, n);
+#pragma unroll 4
+        for (int e = tid; e < e_end; e += kSel) {
+            const int x = S.sc[e];
+            if (e < c.lo) { a.x += x > T; a.y += x == T; }
+            else a.z += x == T;
+        }
+        sel_total8(a, bb, S.red);
+        if (cut.all) {
+            cut.base = c.lo;
+        } else {
+            cut.T = T;
+            cut.base = a.x + min(need, a.y);
+            cut.quota = max(0, min(need - a.y, a.z));
+        }
+    }
+    if (c.my_n > 0)
+        write_lists<false>(S.sc + c.lo, c.my_n, c.lo, c.pool, none, cut, S.wsum, row_prefetch(p, c.u));
+    if (c.cta == p.G - 1) {
+#pragma unroll 1
+        for (int i = min(r, n) + tid; i < r; i += kSel) cut.out[i] = -1;
+    }
     sel_sync();
     return true;
 }
@@ -2041,7 +2089,7 @@ __global__ void __launch_bounds__(kSel, 1)
             }
             if (my_n > 0 && lo > 0 && tid == 0 && __ldg(pool + lo - 1) < 0) report(p.status, CSA2_ERR_RANGE, u);
 #pragma unroll 1
-            for (int e = tid; e < my_n; e += kSel) atomicAdd(&S.hist0[bin0(spill ? spill[e] : S.sc[e])], 1);
+            for (int e = tid; e < my_n && !p.local_sel; e += kSel) atomicAdd(&S.hist0[bin0(spill ? spill[e] : S.sc[e])], 1);
         }
         __syncthreads();
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
@@ -2221,7 +2269,8 @@ static cudaError_t launch_mq(const MqParams& mp, const CUtensorMap& map, int gri
 
 // Launch one indexer call. `ws` holds plan_index(a).ws_bytes bytes (zero at first use).
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
-                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready) {
+                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready,
+                         const csa2_index_args* rx) {
     const int sms = num_sms();
     csa2_index_args aa = a;
     aa.P_in = P_in;
@@ -2259,6 +2308,11 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
         p.pf_scale_bytes = pf->D / 16;
     }
     p.keys_ready = keys_ready;
+    if (a.mode == CSA2_FULL && a.P > 0 && rx != nullptr && rx->ki != nullptr && rx->B == a.B) {
+        p.pk_keys = rx->ki;
+        p.pk_seq_stride = rx->ki_seq_stride;
+        p.pk_row_bytes = rx->Di;
+    }
     p.m = a.m;
     p.status = d_status;
     p.wait_budget = group_wait_budget();
