@@ -1319,9 +1319,9 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
 
 // ------------------------------------------------------------ Reindex: one select per group
 // A Reindex pool fits in one CTA's shared memory, so the group does not run the
-// distributed select: every CTA publishes its scores (element order) and its element
-// count and meets the group at one barrier. Then every CTA loads all of the unit's
-// scores and finds the same exact cut (the order key's level-0 bin of the k-th best
+// distributed select: every CTA publishes its scores (element order), its element
+// count and its level-0 histogram, and meets the group at one barrier. Then every CTA
+// loads all of the unit's scores and the group's histogram and finds the same exact cut (the order key's level-0 bin of the k-th best
 // score, the bin's scores as candidates, the exact threshold T and the number of ties
 // at T to take), and writes its own chunk's selected entries at its offset in the
 // list (the entries taken before its chunk), in pool order, which is position order.
@@ -1329,10 +1329,12 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
                                                    int& bar_target) {
     const int tid = threadIdx.x, lane = tid & 31;
     int32_t* rs = p.rscore + (size_t)c.u * p.rstride;
-    int* cnt = sl.g0 + ((c.epoch + c.j) % 3) * kG0Stride + kBins;
+    int* g0cur = sl.g0 + ((c.epoch + c.j) % 3) * kG0Stride;
+    int* cnt = g0cur + kBins;
     int* cnt_next = sl.g0 + ((c.epoch + c.j + 1) % 3) * kG0Stride + kBins;
 #pragma unroll 1
     for (int e = tid; e < c.my_n; e += kSel) rs[c.lo + e] = S.sc[e];
+    push_hist(S.hist0, g0cur);   // (built over this CTA's valid scores)
     if (tid == 0 && c.my_n > 0) atomicAdd(cnt, c.my_n);
     {
         // the next level-0 buffer (bins and count) must be zero when the next unit,
@@ -1344,6 +1346,7 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         for (int i = zlo + tid; i < zhi; i += kSel) g0nxt[i] = 0;
         if (tid == 0 && c.cta == 0) *cnt_next = 0;
     }
+    if (tid == 0) S.info[20] = 0;
     // every CTA waits: the first CTA's zeroing of the next unit's count (above) is then
     // ordered before any CTA's add for that unit
     bar_target += p.G;
@@ -1351,30 +1354,34 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
                        p.skip_arrival && c.cta == p.G - 1))
         return false;
 
-    // all scores of the unit (valid pool entries form a prefix), as int4 vectors with
-    // every load of a thread in flight at once, and their level-0 histogram
+    // the group's histogram (kBpt bins a thread) and all scores of the unit (valid pool
+    // entries form a prefix), as int4 vectors with every load of a thread in flight at
+    // once. The score loads cover the whole row (rstride >= P_in, a multiple of 4) and
+    // are issued with the count's, which decides which of them are used.
     const int n = min(max(__ldcg(cnt), 0), p.P_in);
-#pragma unroll 1
-    for (int i = tid; i < kBins; i += kSel) S.hist0[i] = 0;
-    if (tid == 0) S.info[20] = 0;
-    sel_sync();
+    int hg[kBpt];
     {
-        const int nv = (n + 3) >> 2;   // rstride is a multiple of 4: whole vectors stay in the unit's row
+        const int4* g4 = reinterpret_cast<const int4*>(g0cur + kBpt * tid);
+#pragma unroll
+        for (int i = 0; i < kBpt / 4; ++i) {
+            const int4 v = __ldcg(g4 + i);
+            hg[4 * i] = v.x; hg[4 * i + 1] = v.y; hg[4 * i + 2] = v.z; hg[4 * i + 3] = v.w;
+        }
+    }
+    {
+        const int nv = (n + 3) >> 2;
+        const int nv_cap = (p.P_in + 3) >> 2;
         const int4* rs4 = reinterpret_cast<const int4*>(rs);
 #pragma unroll 1
-        for (int v0 = tid; v0 < nv; v0 += 4 * kSel) {
+        for (int v0 = tid; v0 < nv_cap; v0 += 4 * kSel) {
             int4 x4[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) x4[q] = (v0 + q * kSel < nv) ? __ldcg(rs4 + v0 + q * kSel) : make_int4(0, 0, 0, 0);
+            for (int q = 0; q < 4; ++q) x4[q] = (v0 + q * kSel < nv_cap) ? __ldcg(rs4 + v0 + q * kSel) : make_int4(0, 0, 0, 0);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int v = v0 + q * kSel;
                 if (v >= nv) continue;
                 reinterpret_cast<int4*>(S.sc)[v] = x4[q];
-                const int xs[4] = {x4[q].x, x4[q].y, x4[q].z, x4[q].w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (4 * v + k < n) atomicAdd(&S.hist0[bin0(xs[k])], 1);
             }
         }
     }
@@ -1386,18 +1393,18 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
     if (n <= r) {
         cut.all = 1;
     } else {
-        // level-0 bin holding rank r, from the shared histogram (kBpt bins per thread)
-        int h[kBpt], sum = 0;
+        // level-0 bin holding rank r, from the group's histogram
+        int sum = 0;
 #pragma unroll
-        for (int i = 0; i < kBpt; ++i) { h[i] = S.hist0[kBpt * tid + i]; sum += h[i]; }
+        for (int i = 0; i < kBpt; ++i) sum += hg[i];
         int total;
         const int excl = sel_scan_excl(sum, S.red, total);
         int above = total - excl - sum;
         if (above < r && r <= above + sum) {
 #pragma unroll
             for (int i = kBpt - 1; i >= 0; --i) {
-                if (above < r && r <= above + h[i]) { S.info[0] = kBpt * tid + i; S.info[1] = above; }
-                above += h[i];
+                if (above < r && r <= above + hg[i]) { S.info[0] = kBpt * tid + i; S.info[1] = above; }
+                above += hg[i];
             }
         }
         sel_sync();
@@ -1407,7 +1414,7 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         // the bin's scores (any order) are the candidates; one reservation per warp and step
         int* cx = reinterpret_cast<int*>(&S.stage[0][0]);
         const unsigned below = (1u << lane) - 1u;
-#pragma unroll 1
+#pragma unroll 4
         for (int e0 = 0; e0 < n; e0 += kSel) {
             const int e = e0 + tid;
             const int x = e < n ? S.sc[e] : 0;
@@ -1974,12 +1981,16 @@ __global__ void __launch_bounds__(kSel, 1)
         // Reindex: this CTA's slice of the pool does not depend on the query position
         // (the position only validates the entries), so its first entries and the index
         // query are loaded before the position arrives
-        int sidx0[RB];
+        // 64-byte keys with at most 8 heads: four lanes per key row (the row's 16-byte
+        // chunks), 128 rows per round, kQuadRounds rounds in flight
+        constexpr bool kQuad = (HI == 8 && DI == 64);
+        constexpr int kQuadRounds = 8;
+        int sidx0[kQuad ? kQuadRounds : RB];
         if (!full) {
             const int lo_r = min(cta * p.chunk, p.P_in), hi_r = min(lo_r + p.chunk, p.P_in);
 #pragma unroll
-            for (int q2 = 0; q2 < RB; ++q2) {
-                const int e = q2 * kSel + tid;
+            for (int q2 = 0; q2 < (kQuad ? kQuadRounds : RB); ++q2) {
+                const int e = kQuad ? q2 * (kSel / 4) + (tid >> 2) : q2 * kSel + tid;
                 sidx0[q2] = (e < hi_r - lo_r) ? __ldg(pool + lo_r + e) : -1;
             }
         }
@@ -2047,6 +2058,68 @@ __global__ void __launch_bounds__(kSel, 1)
             const int8_t* kb = p.ki + (size_t)b * p.ki_seq_stride;
             constexpr int kCh = DI > 0 ? DI / 16 : 8;   // 16-byte chunks per key row
             int first_bad = my_n;
+            if constexpr (kQuad) {
+                // lane l of a quad holds chunk l % 4 of its row: one load instruction of a
+                // warp covers 8 rows (8 lines instead of 32). Each lane's partial dot products
+                // of the 8 heads are summed over the quad by two halving exchanges (each lane
+                // ends with two heads), then ReLU, weights and a quad sum give the score.
+                const int sub = tid & 3, rw = tid >> 2;
+                const int hb = ((sub >> 1) & 1) * 4 + (sub & 1) * 2;   // this lane's two heads
+                const int wa = hb == 0 ? p.w[0] : hb == 2 ? p.w[2] : hb == 4 ? p.w[4] : p.w[6];
+                const int wb = hb == 0 ? p.w[1] : hb == 2 ? p.w[3] : hb == 4 ? p.w[5] : p.w[7];
+                int4 qc[8];
+#pragma unroll
+                for (int h = 0; h < 8; ++h) qc[h] = reinterpret_cast<const int4*>(S.q + h * 64)[sub];
+#pragma unroll 1
+                for (int e0 = 0; e0 < my_n; e0 += kQuadRounds * (kSel / 4)) {
+                    int sidx[kQuadRounds];
+                    bool okr[kQuadRounds];
+                    int4 kv[kQuadRounds];
+#pragma unroll
+                    for (int rd = 0; rd < kQuadRounds; ++rd) {
+                        const int e = e0 + rd * (kSel / 4) + rw;
+                        sidx[rd] = (e0 == 0) ? sidx0[rd] : ((e < my_n) ? __ldg(pool + lo + e) : -1);
+                    }
+#pragma unroll
+                    for (int rd = 0; rd < kQuadRounds; ++rd) {
+                        const int e = e0 + rd * (kSel / 4) + rw;
+                        okr[rd] = e < my_n && sidx[rd] >= 0 && sidx[rd] <= tg;
+                        if (e < my_n && !okr[rd]) first_bad = min(first_bad, e);
+                        kv[rd] = okr[rd] ? __ldg(reinterpret_cast<const int4*>(kb + (size_t)sidx[rd] * 64) + sub)
+                                         : make_int4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int rd = 0; rd < kQuadRounds; ++rd) {
+                        if (e0 + rd * (kSel / 4) >= my_n) break;   // warp-uniform
+                        int acc[8];
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            int a2 = __dp4a(kv[rd].x, qc[h].x, 0);
+                            a2 = __dp4a(kv[rd].y, qc[h].y, a2);
+                            a2 = __dp4a(kv[rd].z, qc[h].z, a2);
+                            acc[h] = __dp4a(kv[rd].w, qc[h].w, a2);
+                        }
+                        const bool up2 = (sub & 2) != 0, up1 = (sub & 1) != 0;
+                        int v4[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const int send = up2 ? acc[h] : acc[h + 4], keep = up2 ? acc[h + 4] : acc[h];
+                            v4[h] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                        }
+                        int v2[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int send = up1 ? v4[h] : v4[h + 2], keep = up1 ? v4[h + 2] : v4[h];
+                            v2[h] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                        }
+                        int x = wa * max(v2[0], 0) + wb * max(v2[1], 0);
+                        x += __shfl_xor_sync(0xffffffffu, x, 1);
+                        x += __shfl_xor_sync(0xffffffffu, x, 2);
+                        const int e = e0 + rd * (kSel / 4) + rw;
+                        if (sub == 0 && okr[rd]) { if (spill) spill[e] = x; else S.sc[e] = x; }
+                    }
+                }
+            } else {
 #pragma unroll 1
             for (int e0 = 0; e0 < my_n; e0 += RB * kSel) {
                 int sidx[RB];
@@ -2080,6 +2153,7 @@ __global__ void __launch_bounds__(kSel, 1)
                     if (okr[q2 + 1]) { if (spill) spill[eb] = xb; else S.sc[eb] = xb; }
                 }
             }
+            }
             const int fb = sel_min(first_bad, S.red);
             if (fb < my_n) {
                 // an entry past the first invalid one must be padding, never a position
@@ -2089,7 +2163,7 @@ __global__ void __launch_bounds__(kSel, 1)
             }
             if (my_n > 0 && lo > 0 && tid == 0 && __ldg(pool + lo - 1) < 0) report(p.status, CSA2_ERR_RANGE, u);
 #pragma unroll 1
-            for (int e = tid; e < my_n && !p.local_sel; e += kSel) atomicAdd(&S.hist0[bin0(spill ? spill[e] : S.sc[e])], 1);
+            for (int e = tid; e < my_n; e += kSel) atomicAdd(&S.hist0[bin0(spill ? spill[e] : S.sc[e])], 1);
         }
         __syncthreads();
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
