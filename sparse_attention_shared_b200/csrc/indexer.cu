@@ -705,13 +705,15 @@ __device__ __forceinline__ void gather_lists2(const int* sc, int n, int lo0, int
     const int nstep = (n + 63) >> 6;
     const int spw = (nstep + kSelWarps - 1) / kSelWarps;
     const int s0 = min(nstep, wp * spw), s1 = min(nstep, s0 + spw);
-    // four steps' loads are issued before any of their list stores (which the compiler
-    // cannot tell apart from the scores, so it would not move a later load above them)
+    // kIn steps' loads are issued before any of their list stores (which the compiler
+    // cannot tell apart from the scores, so it would not move a later load above them);
+    // spilled scores come from L2, so more of them are in flight
+    constexpr int kIn = kSpill ? 16 : 4;
 #pragma unroll 1
-    for (int st0 = s0; st0 < s1; st0 += 4) {
-        int2 xv[4];
+    for (int st0 = s0; st0 < s1; st0 += kIn) {
+        int2 xv[kIn];
 #pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
+        for (int u4 = 0; u4 < kIn; ++u4) {
             const int e = (st0 + u4) * 64 + 2 * lane;
             xv[u4] = make_int2(0, 0);
             if (st0 + u4 < s1) {
@@ -720,7 +722,7 @@ __device__ __forceinline__ void gather_lists2(const int* sc, int n, int lo0, int
             }
         }
 #pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
+        for (int u4 = 0; u4 < kIn; ++u4) {
             if (st0 + u4 >= s1) break;   // warp-uniform
             const int e = (st0 + u4) * 64 + 2 * lane;
             unsigned f[2];
@@ -1719,21 +1721,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // chunk goes to shared memory when it fits, and its histogram is built here
         const int* src = p.pre ? p.pre + (size_t)u * p.pstride + lo : nullptr;
         if (src) {
-            // 16-byte loads, four in flight per thread (the unit's row and the chunk
-            // start are multiples of 4 elements)
+            // 16-byte loads, eight in flight per thread (the unit's row and the chunk
+            // start are multiples of 4 elements): each round is one L2 round trip
+            constexpr int kIn = 8;
             const bool to_smem = p.chunk <= kSmemScores;
             const int nv = my_n >> 2;
             const int4* src4 = reinterpret_cast<const int4*>(src);
 #pragma unroll 1
-            for (int v0 = tid; v0 < nv; v0 += 4 * kTcThreads) {
-                int4 x4[4];
+            for (int v0 = tid; v0 < nv; v0 += kIn * kTcThreads) {
+                int4 x4[kIn];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < kIn; ++q) {
                     const int v = v0 + q * kTcThreads;
                     x4[q] = v < nv ? __ldcg(src4 + v) : make_int4(0, 0, 0, 0);
                 }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < kIn; ++q) {
                     const int v = v0 + q * kTcThreads;
                     if (v >= nv) continue;
                     if (to_smem) reinterpret_cast<int4*>(S.sc)[v] = x4[q];
