@@ -43,9 +43,14 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--kernel-launches", type=int, default=50)
     ap.add_argument("--eager", action="store_true", help="launch directly instead of replaying a CUDA graph")
+    ap.add_argument("--phase-trace", action="store_true",
+                    help="load the phase-trace build and print per-phase CTA times and the step's launch timeline "
+                         "instead of the JSON line")
     ap.add_argument("--override", default="",
                     help="replace workload fields, e.g. Tq=1024,N=33792 (a smaller case of the same shape, for profiling)")
     args = ap.parse_args()
+    if args.phase_trace:
+        os.environ["CSA2_LIBRARY"] = "trace"   # before the library is loaded
     args.overrides = {}
     for kv in filter(None, args.override.split(",")):
         k, v = kv.split("=")
@@ -744,6 +749,145 @@ def run_reference(args, rank, world):
     print(json.dumps(res), flush=True)
 
 
+# ------------------------------------------------------------------ phase trace
+PHASES = {
+    "full_index": {1: "dependency wait", 2: "scan done", 3: "histograms exchanged", 4: "threshold bins",
+                   5: "ordered lists", 7: "candidates exchanged", 8: "finalise", 12: "candidates loaded",
+                   13: "thresholds, counts", 9: "write", 10: "lists written", 11: "end"},
+    "reindex_index": {1: "dependency wait", 2: "scores done", 3: "scores published", 4: "all scores loaded",
+                      5: "candidates", 6: "threshold", 7: "offsets", 11: "end"},
+    "attention": {1: "dependency wait", 2: "positions", 3: "rows staged", 4: "tile ready", 5: "S done",
+                  6: "softmax done", 7: "O done", 8: "partials exchanged", 9: "end"},
+}
+KINDS = {1: "index_full_tc_kernel", 2: "index_dp4a_kernel", 3: "sparse_attn_cl_kernel", 4: "sparse_attn_kernel",
+         5: "index_mq_score_kernel"}
+
+
+def run_phase_trace(args):
+    """The phase-trace build: per kernel class, one launch alone after an L2 flush with the
+    median and 90th percentile over CTAs of the SM-clock time from the CTA's start to each
+    phase boundary; then every launch of one CUDA-graph replay of the whole stack with its
+    first CTA start, last CTA end and the gap to the launch before (global timer)."""
+    import numpy as np
+    import torch
+
+    import synth
+    from sparse_attention_shared_b200 import capi, ops
+
+    assert capi.trace_library()
+    L = capi.lib()
+    wl = synth.make_workload(args.workload, **args.overrides)
+    s = wl.spec
+    stack, layers, q_pos, codes, scales, base = build_device_stack(wl, torch, ops, np)
+    ws, st = ops.Workspace(), ops.Status()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ncta, cap = 1 << 16, 1 << 17
+    slots = torch.zeros((ncta, 32), dtype=torch.int64, device="cuda")
+    tl = torch.zeros((cap, 4), dtype=torch.int64, device="cuda")
+    ctr = torch.zeros((4,), dtype=torch.int32, device="cuda")
+    sp = int(torch.cuda.current_stream().cuda_stream)
+    clock_ghz = 1.965   # SM clocks are converted at the B200's boost clock (the bench line records the clocks seen)
+
+    def set_all(on_slots, on_tl):
+        for f in (L.csa2_trace_set_idx, L.csa2_trace_set_attn):
+            capi.check(f(slots.data_ptr(), ncta, 1 if on_slots else 0, tl.data_ptr() if on_tl else None,
+                         ctr.data_ptr(), cap), "trace buffers")
+
+    modes = [x.mode for x in s.layers]
+    li_f = modes.index("FULL")
+    d0, Lf = layers[li_f], s.layers[li_f]
+    pool_t = torch.empty((s.B, s.Tq, max(Lf.P, 1)), dtype=torch.int32, device="cuda")
+    topk_t = torch.empty((s.B, s.Tq, Lf.k), dtype=torch.int32, device="cuda")
+    ia = ops.make_index_args(capi.CSA2_FULL, q_pos, d0["qi"], np.ascontiguousarray(np.asarray(d0["w"], np.int32)),
+                             d0["ki"], Lf.k, Lf.P, None, pool_t if Lf.P else None, topk_t, s.m)
+    ibuf = ws.get(capi.csa2_workspace_bytes(0, ia))
+    calls = [("full_index", lambda: capi.csa2_index_topk(ia, ibuf.data_ptr(), ibuf.numel(), st.ptr, sp))]
+    if "REINDEX" in modes:
+        li_r = modes.index("REINDEX")
+        dr, Lr = layers[li_r], s.layers[li_r]
+        topk_r = torch.empty((s.B, s.Tq, Lr.k), dtype=torch.int32, device="cuda")
+        ra = ops.make_index_args(capi.CSA2_REINDEX, q_pos, dr["qi"], np.ascontiguousarray(np.asarray(dr["w"], np.int32)),
+                                 dr["ki"], Lr.k, 0, pool_t, None, topk_r, s.m)
+        rbuf = ws.get(capi.csa2_workspace_bytes(0, ra))
+        calls.append(("reindex_index", lambda: capi.csa2_index_topk(ra, rbuf.data_ptr(), rbuf.numel(), st.ptr, sp)))
+    da = layers[modes.index("REUSE") if "REUSE" in modes else li_f]
+    o = torch.empty_like(da["q"])
+    lse = torch.empty(da["q"].shape[:-1], dtype=torch.float32, device="cuda")
+    aa = ops.make_attn_args(q_pos, da["q"], codes, scales, topk_t, da["kl"], da["vl"], base, s.W, o, lse, s.m)
+    abuf = ws.get(capi.csa2_workspace_bytes(1, aa))
+    calls.append(("attention", lambda: capi.csa2_sparse_attn(aa, abuf.data_ptr(), abuf.numel(), st.ptr, sp)))
+
+    print(f"phase trace, workload {s.name} (B={s.B}, N={s.N}, Tq={s.Tq}); times in us from each CTA's start")
+    for name, fn in calls:
+        for _ in range(3):
+            capi.check(fn(), name)
+        torch.cuda.synchronize()
+        slots.zero_()
+        ctr.zero_()
+        set_all(True, True)
+        flush.zero_()
+        torch.cuda.synchronize()
+        capi.check(fn(), name)
+        torch.cuda.synchronize()
+        set_all(False, False)
+        h = slots.cpu().numpy()
+        n = min(int(ctr[0].item()), cap)
+        t = tl[:n].cpu().numpy()
+        used = np.nonzero(h[:, 31])[0]
+        span = (t[:, 3].max() - t[:, 2].min()) / 1e3 if n else 0.0
+        print(f"{name}: {len(used)} CTAs traced, launch span {span:.1f} us")
+        for k, label in sorted(PHASES["full_index" if name == "full_index" else name].items(),
+                               key=lambda kv: np.median(h[used, kv[0]]) if len(used) else 0):
+            v = h[used, k]
+            v = v[v > 0]
+            if len(v):
+                print(f"  {label:22s} median {np.median(v) / clock_ghz / 1e3:8.2f}  p90 {np.percentile(v, 90) / clock_ghz / 1e3:8.2f}")
+        for k in (16, 17):
+            v = h[used, k]
+            v = v[v > 0]
+            if len(v):
+                print(f"  candidates (track {k - 16}) median {int(np.median(v))}")
+    st.check("phase trace")
+
+    wsb = ws.get(stack.ws_bytes)
+    g = capture_graph(torch, lambda sp2: stack.run_raw(int(wsb.data_ptr()), wsb.numel(), st.ptr, sp2))
+    for _ in range(5):
+        flush.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    ctr.zero_()
+    set_all(False, True)
+    flush.zero_()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    set_all(False, False)
+    n = min(int(ctr[0].item()), cap)
+    t = tl[:n].cpu().numpy()
+    t = t[np.argsort(t[:, 2], kind="stable")]
+    t0 = t[:, 2].min()
+    launches = []
+    for kind in np.unique(t[:, 0]):
+        cur, seen = [], set()
+        for r in t[t[:, 0] == kind]:   # a launch ends where a CTA index repeats
+            if int(r[1]) in seen:
+                launches.append(np.array(cur))
+                cur, seen = [], set()
+            cur.append(r)
+            seen.add(int(r[1]))
+        if cur:
+            launches.append(np.array(cur))
+    launches.sort(key=lambda a: a[:, 2].min())
+    print(f"step timeline (one graph replay, {len(launches)} launches)")
+    prev = None
+    for a in launches:
+        st0, en = (a[:, 2].min() - t0) / 1e3, (a[:, 3].max() - t0) / 1e3
+        gap = "" if prev is None else f"  end - previous end {en - prev:6.1f}"
+        print(f"  {KINDS.get(int(a[0, 0]), a[0, 0]):22s} CTAs {len(a):5d} start {st0:8.1f} end {en:8.1f}{gap}")
+        prev = en
+    st.check("phase trace timeline")
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -751,6 +895,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.phase_trace:
+        run_phase_trace(args)
         return
     run_ours(args, rank, world, local_rank)
 

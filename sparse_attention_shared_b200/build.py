@@ -25,14 +25,17 @@ def _stale(obj: str, src: str) -> bool:
 
 
 LIB_CHECKED = os.path.join(HERE, "libcsa2_checked.so")
+LIB_TRACE = os.path.join(HERE, "libcsa2_trace.so")
 
 
-def build(force: bool = False, verbose: bool = False, extra=None, checked: bool = False) -> str:
-    """Build libcsa2.so, or with checked=True the range-checked libcsa2_checked.so
-    (-DCSA2_CHECKED: computed indices are checked and reported instead of accessed)."""
-    lib = LIB_CHECKED if checked else LIB
-    extra = list(extra or []) + (["-DCSA2_CHECKED"] if checked else [])
-    objdir = os.path.join(HERE, "_build_checked" if checked else "_build")
+def build(force: bool = False, verbose: bool = False, extra=None, checked: bool = False, trace: bool = False) -> str:
+    """Build libcsa2.so; with checked=True the range-checked libcsa2_checked.so
+    (-DCSA2_CHECKED: computed indices are checked and reported instead of accessed); with
+    trace=True the phase-trace libcsa2_trace.so (-DCSA2_PHASE_TRACE: kernels record phase clocks
+    and per-CTA start and end times into host-registered buffers)."""
+    lib = LIB_CHECKED if checked else LIB_TRACE if trace else LIB
+    extra = list(extra or []) + (["-DCSA2_CHECKED"] if checked else []) + (["-DCSA2_PHASE_TRACE"] if trace else [])
+    objdir = os.path.join(HERE, "_build_checked" if checked else "_build_trace" if trace else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs, changed = [], False
     for src in SOURCES:
@@ -56,4 +59,4 @@ def build(force: bool = False, verbose: bool = False, extra=None, checked: bool 
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, checked="--checked" in sys.argv)
+    build(force="--force" in sys.argv, verbose=True, checked="--checked" in sys.argv, trace="--trace" in sys.argv)

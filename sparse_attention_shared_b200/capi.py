@@ -69,8 +69,14 @@ def checked_library() -> bool:
     return os.environ.get("CSA2_LIBRARY", "") == "checked"
 
 
+def trace_library() -> bool:
+    """CSA2_LIBRARY=trace selects the phase-trace build (libcsa2_trace.so)."""
+    return os.environ.get("CSA2_LIBRARY", "") == "trace"
+
+
 def library_path() -> str:
-    return os.path.join(_HERE, "libcsa2_checked.so" if checked_library() else "libcsa2.so")
+    name = "libcsa2_checked.so" if checked_library() else "libcsa2_trace.so" if trace_library() else "libcsa2.so"
+    return os.path.join(_HERE, name)
 
 
 def lib():
@@ -80,7 +86,7 @@ def lib():
         if _lib is None:
             from . import build as _build
             try:
-                path = _build.build(checked=checked_library())
+                path = _build.build(checked=checked_library(), trace=trace_library())
             except Exception as e:  # noqa: BLE001
                 raise RuntimeError(f"cannot build the CSA2 CUDA library: {e}") from e
             L = ctypes.CDLL(path)
@@ -101,6 +107,11 @@ def lib():
             L.csa2_set_wait_controls.restype = c_int
             L.csa2_status_string.argtypes = [c_int]
             L.csa2_status_string.restype = c_char_p
+            if trace_library():   # (slots, rows, on, timeline, counter, capacity)
+                for name in ("csa2_trace_set_idx", "csa2_trace_set_attn"):
+                    f = getattr(L, name)
+                    f.argtypes = [c_void_p, ctypes.c_uint, c_int, c_void_p, c_void_p, ctypes.c_uint]
+                    f.restype = c_int
             _lib = L
     return _lib
 

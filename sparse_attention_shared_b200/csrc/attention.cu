@@ -133,6 +133,7 @@ __device__ __forceinline__ uint32_t bf16x8_max_exp(const uint4& v) {
 
 template <int HQP, int D>
 __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_constant__ AttnParams p) {
+    CSA2_TRACE_INIT();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     AttnSmem<HQP>& S =
         *reinterpret_cast<AttnSmem<HQP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -450,6 +451,7 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
         if (tid == 0) p.tickets[u] = 0;
     }
 
+    CSA2_TRACE_END(4);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kCols);
@@ -526,6 +528,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
     const int CS = gridDim.x;
     const int rank = (int)cluster_ctarank();
     const int u = blockIdx.y;
+    CSA2_TRACE_INIT();
     const int b = u / p.Tq;
     const int ngt2 = (p.k + 2 * kTileKeys - 1) / (2 * kTileKeys);
     const bool glob = rank < ngt2;
@@ -558,6 +561,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         pdl_launch_dependents();
         load_q();   // in flight while the list and the rows are fetched
     }
+    CSA2_TRACE(1);
 
     // ---- 1. positions and list entries; row tid of the tile is this thread's
     int t = p.q_pos[u];
@@ -574,6 +578,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         tg = -1;
     }
     const int lo_w = max(max(base, t - p.W + 1), 0);
+    CSA2_TRACE(2);   // positions
 
     // ---- 2. the tile's rows
     bool v0 = false;
@@ -627,6 +632,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         load_q();
     }
     __syncthreads();   // the barriers (initialised by thread 0) and TMEM address are set
+    CSA2_TRACE(3);
     bool ok = true;
     if (glob) {
         // A global tile is dequantised to f16 (code times scale is exact in f16) and
@@ -680,6 +686,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         }
     }
     if (!glob) ok = mbar_wait(&S.bar_tma, 0, p.status, 12);
+    CSA2_TRACE(4);   // tile staged
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -703,6 +710,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         mma_commit(&S.bar_s);
     }
     ok = mbar_wait(&S.bar_s, 0, p.status, 10) && ok;
+    CSA2_TRACE(5);   // S done
     tc_fence_after();
 
     // ---- 4. softmax partial over the tile's rows: thread tid holds key tid, which
@@ -763,6 +771,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         S.lfin[tid] = l;
     }
 
+    CSA2_TRACE(6);   // softmax done
     // ---- 5. O^T = V^T P (keys as the reduction; the head dim as M)
     if (tid == 0) {
         const uint32_t va = smem_u32(glob ? S.tbuf : S.tbuf + 2 * kPanelBytes), pa = smem_u32(S.qpbuf);
@@ -776,6 +785,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         mma_commit(&S.bar_o);
     }
     ok = mbar_wait(&S.bar_o, 0, p.status, 11) && ok;
+    CSA2_TRACE(7);   // O done
     tc_fence_after();
     float ov[HQP];
     if (warp < 4) {   // O^T rows (the head dim) sit in TMEM lanes 0..127
@@ -809,6 +819,7 @@ __global__ void __launch_bounds__(kClThreads, 2)
         }
     }
     cluster_sync_all();   // after it no CTA touches another's shared memory
+    CSA2_TRACE(8);   // partials exchanged
     constexpr int kSlots = kClThreads / D;
     const int slot = tid / D, dim = tid % D;
     for (int h = rank + slot * CS; h < p.Hq; h += kSlots * CS) {
@@ -833,6 +844,8 @@ __global__ void __launch_bounds__(kClThreads, 2)
         if (dim == 0 && p.lse != nullptr)
             p.lse[(size_t)u * p.Hq + h] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
     }
+    CSA2_TRACE(9);
+    CSA2_TRACE_END(3);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kCols);
@@ -1010,3 +1023,5 @@ csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, in
 
 
 }  // namespace csa2
+
+CSA2_TRACE_SETTER(csa2_trace_set_attn)

@@ -25,6 +25,69 @@ __device__ __forceinline__ void report(int32_t* st, int code, int detail) {
     }
 }
 
+// Phase-trace build (compiled with -DCSA2_PHASE_TRACE, library libcsa2_trace.so): the
+// indexer and attention kernels record, per CTA, the SM clock at numbered phase
+// boundaries (CSA2_TRACE) and, per launch, every CTA's start and end on the global
+// timer (CSA2_TRACE_END), into buffers the host registers with the csa2_trace_set_*
+// entry points of that library. Every record is bounded by the buffer sizes given
+// there. In the normal build the macros are empty.
+#ifdef CSA2_PHASE_TRACE
+static __device__ unsigned long long* g_trace_buf = nullptr;   // [ctas][32]: slot 31 start time, 30 start clock
+static __device__ unsigned int g_trace_ncta = 0;               // rows of g_trace_buf
+static __device__ int g_trace_on = 0;                          // phase slots on
+static __device__ unsigned long long* g_tl_buf = nullptr;      // [cap][4]: kernel kind, CTA, start ns, end ns
+static __device__ unsigned int* g_tl_ctr = nullptr;            // records taken (may pass cap)
+static __device__ unsigned int g_tl_cap = 0;
+__device__ __forceinline__ unsigned long long trace_gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ unsigned trace_cta() { return (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x; }
+__device__ __forceinline__ bool trace_slot_ok() {
+    return threadIdx.x == 0 && g_trace_on && g_trace_buf != nullptr && trace_cta() < g_trace_ncta;
+}
+#define CSA2_TRACE_INIT()                                                                         \
+    const unsigned long long csa2_trace_t0 = ::csa2::trace_gtimer();                            \
+    if (::csa2::trace_slot_ok()) {                                                              \
+        ::csa2::g_trace_buf[(size_t)::csa2::trace_cta() * 32 + 31] = csa2_trace_t0;              \
+        ::csa2::g_trace_buf[(size_t)::csa2::trace_cta() * 32 + 30] = (unsigned long long)clock64(); \
+    }
+#define CSA2_TRACE(slot)                                                                          \
+    if (::csa2::trace_slot_ok())                                                                  \
+        ::csa2::g_trace_buf[(size_t)::csa2::trace_cta() * 32 + (slot)] =                          \
+            (unsigned long long)clock64() - ::csa2::g_trace_buf[(size_t)::csa2::trace_cta() * 32 + 30];
+#define CSA2_TRACE_VAL(slot, v)                                                                   \
+    if (::csa2::trace_slot_ok()) ::csa2::g_trace_buf[(size_t)::csa2::trace_cta() * 32 + (slot)] = (unsigned long long)(v);
+#define CSA2_TRACE_END(kind)                                                                      \
+    if (threadIdx.x == 0 && ::csa2::g_tl_buf != nullptr) {                                        \
+        const unsigned csa2_trace_i = atomicAdd(::csa2::g_tl_ctr, 1u);                            \
+        if (csa2_trace_i < ::csa2::g_tl_cap) {                                                    \
+            ::csa2::g_tl_buf[4 * csa2_trace_i] = (kind);                                          \
+            ::csa2::g_tl_buf[4 * csa2_trace_i + 1] = ::csa2::trace_cta();                         \
+            ::csa2::g_tl_buf[4 * csa2_trace_i + 2] = csa2_trace_t0;                               \
+            ::csa2::g_tl_buf[4 * csa2_trace_i + 3] = ::csa2::trace_gtimer();                      \
+        }                                                                                         \
+    }
+// the host side of one translation unit's trace buffers (each unit has its own copies)
+#define CSA2_TRACE_SETTER(name)                                                                   \
+    extern "C" int name(void* slots, unsigned ncta, int on, void* tl, void* ctr, unsigned cap) {  \
+        if (cudaMemcpyToSymbol(csa2::g_trace_buf, &slots, sizeof(slots)) != cudaSuccess) return 1; \
+        if (cudaMemcpyToSymbol(csa2::g_trace_ncta, &ncta, sizeof(ncta)) != cudaSuccess) return 2;  \
+        if (cudaMemcpyToSymbol(csa2::g_trace_on, &on, sizeof(on)) != cudaSuccess) return 3;        \
+        if (cudaMemcpyToSymbol(csa2::g_tl_buf, &tl, sizeof(tl)) != cudaSuccess) return 4;          \
+        if (cudaMemcpyToSymbol(csa2::g_tl_ctr, &ctr, sizeof(ctr)) != cudaSuccess) return 5;        \
+        if (cudaMemcpyToSymbol(csa2::g_tl_cap, &cap, sizeof(cap)) != cudaSuccess) return 6;        \
+        return 0;                                                                                 \
+    }
+#else
+#define CSA2_TRACE_INIT()
+#define CSA2_TRACE(slot)
+#define CSA2_TRACE_VAL(slot, v)
+#define CSA2_TRACE_END(kind)
+#define CSA2_TRACE_SETTER(name)
+#endif
+
 // Range-checked build (compiled with -DCSA2_CHECKED, library libcsa2_checked.so): a
 // computed shared- or global-memory index is checked before the access it guards; a
 // violation is reported as CSA2_ERR_RANGE with `detail` naming the site, and the

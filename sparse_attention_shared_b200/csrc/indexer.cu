@@ -1080,6 +1080,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
     if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status, p.wait_budget,
                        p.skip_arrival && c.cta == p.G - 1))
         return false;
+    CSA2_TRACE(3);   // histograms exchanged
 
     const int n_total = full ? c.n_all : min(max(__ldcg(g0cur + kBins), 0), p.P_in);
     Track tk[2];
@@ -1124,6 +1125,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         }
     }
 
+    CSA2_TRACE(4);   // threshold bins found
     int list_tracks = 0;   // tracks whose final intervals the ordered lists hold (bit per track)
     // ---- rounds until every track knows its cut (usually one)
 #pragma unroll 1
@@ -1143,6 +1145,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
                                   lvl0 ? S.info + 48 : nullptr);
             list_tracks = (g0on ? 1 : 0) | (g1on ? 2 : 0);   // a gather rebuilds the lists
             sel_sync();
+            CSA2_TRACE(5);   // ordered lists built
             if (S.wlist_ovf == 0) {
                 cands_from_lists<kSpill>(sc, lo, wlists(S), S.wlist_n, lbuf, lcnt, S.wsum);
             } else {   // a list overflowed: gather the candidates by reservation
@@ -1197,6 +1200,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         if (!any) break;
         bar_target += p.G;
         if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status, p.wait_budget)) return false;
+        CSA2_TRACE(7);   // candidates exchanged
         bool pending = false;
 #pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
@@ -1222,6 +1226,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         if (!pending) break;
     }
 
+    CSA2_TRACE(8);
     // ---- finalize both tracks: threshold T, tie quota and this CTA's output offset
     ListCut cut[2];
     {
@@ -1250,6 +1255,9 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         const int eqb[2] = {S.red[4] + S.red[5], S.red[6] + S.red[7]};
         int T[2] = {INT_MAX, INT_MAX}, need[2] = {0, 0};
         if (n0 > 0 || n1 > 0) {
+            CSA2_TRACE(12);   // candidates loaded
+            CSA2_TRACE_VAL(16, n0);
+            CSA2_TRACE_VAL(17, n1);
             const int4 ls = local_select2(cx0, n0, tk[0].rrem, tk[0].lo, tk[0].hi, cx0 + 2 * kCandCap, n1, tk[1].rrem,
                                           tk[1].lo, tk[1].hi, histl(S, 0), S.red, S.info);
             if (n0 > 0) { T[0] = ls.x; need[0] = ls.y; }
@@ -1275,6 +1283,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
             else         { ca.z += gtb; ca.w += eqb2; cb.y += mine; }
         }
         sel_total8(ca, cb, S.red);
+        CSA2_TRACE(13);   // thresholds and counts
         const int gtb[2] = {ca.x, ca.z}, eqc[2] = {ca.y, ca.w}, mye[2] = {cb.x, cb.y};
 #pragma unroll
         for (int tr = 0; tr < 2; ++tr) {
@@ -1297,6 +1306,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
         }
     }
 
+    CSA2_TRACE(9);
     // ---- ordered write of both tracks: from the ordered lists when every active
     // track was cut inside its last gathered interval, else over the whole chunk
     const bool from_lists = list_tracks != 0 && S.wlist_ovf == 0 &&
@@ -1307,6 +1317,7 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
                                  row_prefetch(p, c.u));
     else
         write_lists<kSpill>(sc, my_n, lo, full ? nullptr : c.pool, cut[0], cut[1], S.wsum, row_prefetch(p, c.u));
+    CSA2_TRACE(10);   // lists written
     // padding: entries [min(r, n_total), r) = -1
     if (c.cta == p.G - 1) {
 #pragma unroll
@@ -1355,6 +1366,7 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
     if (!group_barrier(sl.ctrl + CTRL_BAR, bar_target, p.status, p.wait_budget,
                        p.skip_arrival && c.cta == p.G - 1))
         return false;
+    CSA2_TRACE(3);   // scores published
 
     // the group's histogram (kBpt bins a thread) and all scores of the unit (valid pool
     // entries form a prefix), as int4 vectors with every load of a thread in flight at
@@ -1388,6 +1400,7 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         }
     }
     sel_sync();
+    CSA2_TRACE(4);   // all scores loaded
     const int r = p.r[1];
     ListCut none{INT_MAX, 0, 0, 0, 0, nullptr, p.status};
     ListCut cut{INT_MAX, 0, 0, 0, r, p.out[1] + (size_t)c.u * r, p.status};
@@ -1430,9 +1443,12 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         }
         sel_sync();
         const int nx = S.info[20];
+        CSA2_TRACE(5);   // candidates
+        CSA2_TRACE_VAL(16, nx);
         const int4 ls = local_select2(S.sc, 0, 0, 1, 0, cx, nx, rrem, blo, bhi, histl(S, 0), S.red, S.info);
         T = ls.z;
         need = ls.w;   // the ties at T ranked within the first r
+        CSA2_TRACE(6);   // threshold
     }
     // this CTA's offset: the entries taken before its chunk; its own share of the ties
     {
@@ -1453,6 +1469,7 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
             cut.quota = max(0, min(need - a.y, a.z));
         }
     }
+    CSA2_TRACE(7);   // offsets
     if (c.my_n > 0)
         write_lists<false>(S.sc + c.lo, c.my_n, c.lo, c.pool, none, cut, S.wsum, row_prefetch(p, c.u));
     if (c.cta == p.G - 1) {
@@ -1570,6 +1587,7 @@ template <int DI>
 __global__ void __launch_bounds__(kTcThreads, 1)
     index_full_tc_kernel(const __grid_constant__ IdxParams p, const __grid_constant__ CUtensorMap kmap) {
     static_assert(DI == 32 || DI == 64 || DI == 128, "tensor-core key widths");
+    CSA2_TRACE_INIT();
     IdxSmem& S = idx_smem();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int group = blockIdx.x / p.G;
@@ -1598,6 +1616,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // TMA producer starts the key stream at once and fills its stages meanwhile.
     const bool producer = warp == kSel / 32;
     if (!(producer && p.keys_ready)) pdl_wait();
+    CSA2_TRACE(1);
     const int epoch = producer ? 0 : __ldcg(sl.ctrl + CTRL_EPOCH);
     int bar_target = producer ? 0 : __ldcg(sl.ctrl + CTRL_BAR_BASE);
     const uint32_t tmem = S.tmem_base;
@@ -1715,6 +1734,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         seq += nst;
         __syncthreads();
+        CSA2_TRACE(2);   // scan done
         if (S.abort) break;
 
         // select only: the unit's scores come from the multi-query scoring kernel; the
@@ -1764,6 +1784,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncthreads();
         if (S.abort) break;
     }
+    CSA2_TRACE(11);
+    CSA2_TRACE_END(1);
     if (!S.abort && cta == 0 && tid == 0) {
         sl.ctrl[CTRL_EPOCH] = epoch + j;
         sl.ctrl[CTRL_BAR_BASE] = bar_target;
@@ -1823,6 +1845,7 @@ __device__ __forceinline__ void tmem_ld16i(uint32_t taddr, int (&v)[16]) {
 template <int DI>
 __global__ void __launch_bounds__(kMqThreads, 1)
     index_mq_score_kernel(const __grid_constant__ MqParams p, const __grid_constant__ CUtensorMap kmap) {
+    CSA2_TRACE_INIT();
     static_assert(DI == 32 || DI == 64 || DI == 128, "tensor-core key widths");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     MqSmem<DI>& S = *reinterpret_cast<MqSmem<DI>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -1948,6 +1971,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kMqBufs * kMqN);
+    CSA2_TRACE_END(5);
 }
 
 // ------------------------------------------------------------ Reindex, and Full for other key widths
@@ -1955,6 +1979,7 @@ template <int HI, int DI>
 __global__ void __launch_bounds__(kSel, 1)
     index_dp4a_kernel(const __grid_constant__ IdxParams p, const __grid_constant__ CUtensorMap kmap) {
     IdxSmem& S = idx_smem();
+    CSA2_TRACE_INIT();
     const int tid = threadIdx.x;
     const int group = blockIdx.x / p.G;
     const int cta = blockIdx.x % p.G;
@@ -1971,6 +1996,7 @@ __global__ void __launch_bounds__(kSel, 1)
     __syncthreads();
     pdl_launch_dependents();   // the next kernel may start its own set-up
     pdl_wait();                // the workspace, pool and index query may come from the previous kernel
+    CSA2_TRACE(1);
     const int epoch = __ldcg(sl.ctrl + CTRL_EPOCH);
     int bar_target = __ldcg(sl.ctrl + CTRL_BAR_BASE);
     uint32_t stage_seq = 0;   // key tiles issued by this CTA so far
@@ -2169,6 +2195,7 @@ __global__ void __launch_bounds__(kSel, 1)
             for (int e = tid; e < my_n; e += kSel) atomicAdd(&S.hist0[bin0(spill ? spill[e] : S.sc[e])], 1);
         }
         __syncthreads();
+        CSA2_TRACE(2);   // scores done
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
         if (!full && p.local_sel)
             alive = reindex_local_unit(p, S, sl, c, bar_target);
@@ -2177,6 +2204,8 @@ __global__ void __launch_bounds__(kSel, 1)
                           : select_unit<false>(p, S, sl, c, bar_target, S.sc);
         __syncthreads();
     }
+    CSA2_TRACE(11);
+    CSA2_TRACE_END(2);
     if (alive && cta == 0 && tid == 0) {
         sl.ctrl[CTRL_EPOCH] = epoch + j;
         sl.ctrl[CTRL_BAR_BASE] = bar_target;
@@ -2467,3 +2496,5 @@ size_t index_scratch_bytes(const csa2_index_args& a, int P_in) {
 }
 
 }  // namespace csa2
+
+CSA2_TRACE_SETTER(csa2_trace_set_idx)

@@ -32,6 +32,18 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, name), name
 
 
+def test_phase_trace_build_exports_its_buffers_entry_points():
+    """The phase-trace variant (-DCSA2_PHASE_TRACE) has every declared entry point plus
+    the two trace-buffer setters; the normal library has no trace code."""
+    import ctypes
+    from sparse_attention_shared_b200 import build
+    T = ctypes.CDLL(build.build(trace=True))
+    for name in _declared() | {"csa2_trace_set_idx", "csa2_trace_set_attn"}:
+        assert hasattr(T, name), name
+    L = capi.lib()
+    assert not hasattr(L, "csa2_trace_set_idx") and not hasattr(L, "csa2_trace_set_attn")
+
+
 def test_wait_controls_validation():
     assert capi.csa2_set_wait_controls(-1, 0) == 2      # CSA2_ERR_SHAPE
     assert capi.csa2_set_wait_controls(0, 0) == 0       # the default budget, no injection
