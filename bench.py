@@ -552,7 +552,9 @@ def kernel_breakdown(args, torch, np, ops, capi, s, layers, q_pos, codes, scales
             lo = np.maximum(np.maximum(t_all - s.W + 1, np.repeat(base_host.astype(np.int64), s.Tq)), 0)
             n_ent += int(np.maximum(t_all - lo + 1, 0).sum())
         flops = 4 * s.Hq * s.D * n_ent
-        entry(cls, attn_kernel_name(s, HQP, int(topk_dev.shape[-1])), t, count, attn_call_bytes(s, qp_host, base_host, topk_host),
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        entry(cls, attn_kernel_name(s, HQP, int(topk_dev.shape[-1]), sms), t, count,
+              attn_call_bytes(s, qp_host, base_host, topk_host),
               flops, bf16_peak, "bf16")
 
     attn_entry("attn_full", li_f, topk_t, topk_h, n_launch["FULL"])
@@ -592,12 +594,14 @@ def index_kernel_name(s, mode):
     return "index_dp4a_kernel<0,0>"
 
 
-def attn_kernel_name(s, HQP, k):
-    """The kernel csa2_sparse_attn launches: the cluster kernel while its cluster (one CTA
-    per 256 list entries, one per 128 window rows) holds at most 16 CTAs, else the ticket
-    kernel."""
+def attn_kernel_name(s, HQP, k, sms):
+    """The kernel csa2_sparse_attn launches (the library's dispatch rule, restated): the
+    cluster kernel while its cluster (one CTA per 256 list entries, one per 128 window rows)
+    holds at most 16 CTAs and, at 16 heads, the call's clusters hold at most 4 CTAs per SM;
+    else the ticket kernel."""
     cs = -(-k // 256) + -(-s.W // 128)
-    if 1 <= cs <= 16 and s.B * s.Tq <= 65535:
+    many = s.Hq <= 16 and s.B * s.Tq * cs > 4 * sms
+    if 1 <= cs <= 16 and s.B * s.Tq <= 65535 and not many:
         return f"sparse_attn_cl_kernel<{HQP},{s.D}>"
     return f"sparse_attn_kernel<{HQP},{s.D}>"
 

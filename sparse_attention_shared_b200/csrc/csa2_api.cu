@@ -8,7 +8,8 @@
 // Workspace layout (bytes, every region 256-byte aligned):
 //   [0, R)            indexer slots: per-SM barrier counters, epochs, histogram
 //                     and candidate buffers. Persistent between calls.
-//   [R, R + T)        attention merge tickets, one int per query. Zero at rest.
+//   [R, R + T)        attention merge tickets, one int per query (T fixed: room for
+//                     65535 queries, the most a call accepts). Zero at rest.
 //   [R + T, end)      scratch: attention partials or spilled indexer scores,
 //                     rewritten by every call.
 // The whole workspace must be zero-filled before its first use. Every call
@@ -40,11 +41,17 @@ csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, in
                                 cudaStream_t stream);
 
 // The attention kernel for a call: the cluster kernel (one CTA per 256 list entries or
-// 128 window rows, the partials merged through distributed shared memory), else one CTA
-// per tile with a ticket merge.
+// 128 window rows, the partials merged through distributed shared memory) while the call
+// is latency-bound, else one CTA per 128-row tile with a ticket merge. Measured on one
+// B200 at 16 heads: the cluster kernel wins while the call's clusters hold at most about
+// four CTAs per SM (decode: 16-32 queries x 12 CTAs), the ticket kernel beyond (64 queries
+// x 16 CTAs: 57 against 61 us; 2048 queries x 12 CTAs: 0.83 against 0.98 ms). At 32 heads
+// (a prefill chunk of 4096 queries) the two are within 2%; the cluster kernel stays.
 static csa2_status run_attn(const csa2_attn_args& a, const int32_t* topk, int list_ready, int* tickets,
                             void* scratch, int32_t* d_status, cudaStream_t stream) {
-    if (attn_cluster_fits(a)) return launch_attn_cluster(a, topk, list_ready, d_status, stream);
+    const int cs = (a.k + 255) / 256 + (a.W + 127) / 128;
+    const bool many = a.Hq <= 16 && (int64_t)a.B * a.Tq * cs > 4LL * num_sms();
+    if (attn_cluster_fits(a) && !many) return launch_attn_cluster(a, topk, list_ready, d_status, stream);
     return launch_attn(a, topk, tickets, scratch, d_status, stream);
 }
 void set_wait_controls(long long budget, int skip);
@@ -106,7 +113,10 @@ static csa2_status check_attn(const csa2_attn_args* a, bool in_stack) {
     return CSA2_OK;
 }
 
-static size_t tickets_bytes(int units) { return a256((size_t)units * 4); }
+// The ticket region has one size for every call (room for the most queries a call may
+// have), so that no call's scratch ever lies where another call keeps its tickets: a
+// workspace shared by calls of different sizes stays zero there between calls.
+static size_t tickets_bytes(int /*units*/) { return a256((size_t)65535 * 4); }
 
 static void* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
 

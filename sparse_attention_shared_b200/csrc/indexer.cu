@@ -1330,6 +1330,178 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
     return true;
 }
 
+// ------------------------------------------------------------ select only: sampled threshold
+// The select-only pass of one query by one CTA, its scores in global memory (more than
+// shared memory holds). A sample of at most 4096 scores (every s-th position) gives
+// each track a threshold estimate: the sample's value at 1.2 times the rank the track's
+// cut would have in the sample, plus 16. One ordered pass keeps every score at or above
+// the lower estimate as a candidate (position order, a list per warp over its range
+// of positions) and counts the scores at or above each track's estimate. When every
+// track has at least its rank r there, all of its r best scores are candidates, and
+// the exact threshold, the ties to take and the ordered write run over the candidates
+// alone. Otherwise (a list overflowed or an estimate was too high) nothing is written
+// and the caller runs the full select.
+constexpr int kSampleMax = 4096;
+constexpr int kCandPerWarp = (kStages * kStageBytes) / (8 * kSelWarps);   // int2 entries per warp list (1024)
+
+__device__ __noinline__ bool sampled_select(const IdxParams& p, IdxSmem& S, const Slot& sl, int u, int j, int epoch,
+                                            const int* src, int n) {
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    const unsigned below = (1u << lane) - 1u;
+    int r[2], act[2];
+#pragma unroll
+    for (int tr = 0; tr < 2; ++tr) {
+        r[tr] = p.r[tr];
+        act[tr] = r[tr] > 0 && r[tr] < n;
+        if (r[tr] > 0 && !act[tr]) return false;   // a track that takes every score: the full select
+    }
+    if (!act[0] && !act[1]) return false;
+
+    // ---- sample and estimates
+    const int s = (n + kSampleMax - 1) / kSampleMax, m = (n + s - 1) / s;
+#pragma unroll
+    for (int q = 0; q < kSampleMax / kSel; ++q) {
+        const int i = q * kSel + tid;
+        if (i < m) S.sc[i] = __ldcg(src + (size_t)i * s);
+    }
+    sel_sync();
+    int qr[2];
+#pragma unroll
+    for (int tr = 0; tr < 2; ++tr)
+        qr[tr] = act[tr] ? min(m, (int)((long long)r[tr] * m / n * 6 / 5) + 16) : 0;
+    const int4 est = local_select2(S.sc, act[0] ? m : 0, qr[0], INT_MIN, INT_MAX, S.sc, act[1] ? m : 0, qr[1],
+                                   INT_MIN, INT_MAX, S.hist0, S.red, S.info);
+    const int te0 = act[0] ? est.x : INT_MAX, te1 = act[1] ? est.z : INT_MAX;
+    const int tlo = min(te0, te1);
+
+    // ---- one ordered pass: candidates >= tlo, counts >= each estimate
+    int2* lists = reinterpret_cast<int2*>(&S.stage[0][0]);
+    int2* list = lists + wp * kCandPerWarp;
+    const int nstep = (n + 127) >> 7, spw = (nstep + kSelWarps - 1) / kSelWarps;
+    const int s0 = min(nstep, wp * spw), s1 = min(nstep, s0 + spw);
+    int ln = 0, c0 = 0, c1 = 0;
+    constexpr int kIn = 8;
+#pragma unroll 1
+    for (int st0 = s0; st0 < s1; st0 += kIn) {
+        int4 xv[kIn];
+#pragma unroll
+        for (int q = 0; q < kIn; ++q) {
+            const int e = (st0 + q) * 128 + 4 * lane;   // rows are padded to 4 elements
+            xv[q] = (st0 + q < s1 && e < n) ? __ldcg(reinterpret_cast<const int4*>(src + e)) : make_int4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int q = 0; q < kIn; ++q) {
+            if (st0 + q >= s1) break;   // warp-uniform
+            const int e0 = (st0 + q) * 128 + 4 * lane;
+            const int x[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
+            bool f[4];
+            unsigned b[4];
+            int pre = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const bool ok = e0 + k < n;
+                f[k] = ok && x[k] >= tlo;
+                c0 += ok && x[k] >= te0;
+                c1 += ok && x[k] >= te1;
+                b[k] = __ballot_sync(0xffffffffu, f[k]);
+                pre += __popc(b[k] & below);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (f[k] && ln + pre < kCandPerWarp) list[ln + pre] = make_int2(x[k], e0 + k);
+                pre += f[k] ? 1 : 0;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ln += __popc(b[k]);
+        }
+    }
+    if (tid == 0) S.info[24] = 0;
+    sel_sync();
+    if (lane == 0) {
+        S.wlist_n[wp] = min(ln, kCandPerWarp);
+        if (ln > kCandPerWarp) S.info[24] = 1;
+    }
+    int4 ca = make_int4(c0, c1, 0, 0), cb = make_int4(0, 0, 0, 0);
+    sel_total8(ca, cb, S.red);   // (its barriers also publish wlist_n and the overflow flag)
+    if (S.info[24] != 0 || (act[0] && ca.x < r[0]) || (act[1] && ca.y < r[1])) {
+        sel_sync();
+        return false;
+    }
+
+    // ---- the candidates' scores, contiguous, and the exact cut of each track
+    int base = 0, total = 0;
+#pragma unroll 1
+    for (int w = 0; w < kSelWarps; ++w) {
+        base += w < wp ? S.wlist_n[w] : 0;
+        total += S.wlist_n[w];
+    }
+    const int mine = S.wlist_n[wp];
+#pragma unroll 1
+    for (int i = lane; i < mine; i += 32) S.sc[base + i] = list[i].x;
+    sel_sync();
+    const int4 ls = local_select2(S.sc, act[0] ? total : 0, r[0], tlo, INT_MAX, S.sc, act[1] ? total : 0, r[1],
+                                  tlo, INT_MAX, S.hist0, S.red, S.info);
+    ListCut cut[2];
+#pragma unroll
+    for (int tr = 0; tr < 2; ++tr) {
+        cut[tr].T = tr == 0 ? ls.x : ls.z;
+        cut[tr].quota = tr == 0 ? ls.y : ls.w;   // the ties at T ranked within the first r
+        cut[tr].all = 0;
+        cut[tr].base = 0;
+        cut[tr].r = r[tr];
+        cut[tr].out = act[tr] ? p.out[tr] + (size_t)u * r[tr] : nullptr;
+        cut[tr].status = p.status;
+    }
+
+    // ---- ordered write from the lists: counts per warp, then ranks within 32-entry steps
+    const RowPrefetch pf = row_prefetch(p, u);
+    int4 cnt = make_int4(0, 0, 0, 0);   // gt0, eq0, gt1, eq1
+#pragma unroll 1
+    for (int i = lane; i < mine; i += 32) {
+        const int x = list[i].x;
+        cnt.x += cut[0].out && x > cut[0].T;
+        cnt.y += cut[0].out && x == cut[0].T;
+        cnt.z += cut[1].out && x > cut[1].T;
+        cnt.w += cut[1].out && x == cut[1].T;
+    }
+    cnt = warp_sum4(cnt);
+    int4* w4 = reinterpret_cast<int4*>(S.wsum);
+    if (lane == 0) w4[wp] = cnt;
+    sel_sync();
+    int rg0 = 0, re0 = 0, rg1 = 0, re1 = 0;
+#pragma unroll 1
+    for (int w = 0; w < wp; ++w) {
+        const int4 a = w4[w];
+        rg0 += a.x; re0 += a.y; rg1 += a.z; re1 += a.w;
+    }
+#pragma unroll 1
+    for (int i0 = 0; i0 < mine; i0 += 32) {
+        const int i = i0 + lane;
+        const int2 ent = i < mine ? list[i] : make_int2(0, 0);
+        const bool g0 = i < mine && cut[0].out && ent.x > cut[0].T, q0 = i < mine && cut[0].out && ent.x == cut[0].T;
+        const bool g1 = i < mine && cut[1].out && ent.x > cut[1].T, q1 = i < mine && cut[1].out && ent.x == cut[1].T;
+        const unsigned bg0 = __ballot_sync(0xffffffffu, g0), bq0 = __ballot_sync(0xffffffffu, q0);
+        const unsigned bg1 = __ballot_sync(0xffffffffu, g1), bq1 = __ballot_sync(0xffffffffu, q1);
+        const int og0 = rg0 + __popc(bg0 & below), oq0 = re0 + __popc(bq0 & below);
+        const int og1 = rg1 + __popc(bg1 & below), oq1 = re1 + __popc(bq1 & below);
+        if (g0 || (q0 && oq0 < cut[0].quota)) {
+            const int k = og0 + min(oq0, cut[0].quota);
+            if (CSA2_GUARD((unsigned)k < (unsigned)r[0], p.status, 2203)) { cut[0].out[k] = ent.y; prefetch_key(pf, ent.y); }
+        }
+        if (g1 || (q1 && oq1 < cut[1].quota)) {
+            const int k = og1 + min(oq1, cut[1].quota);
+            if (CSA2_GUARD((unsigned)k < (unsigned)r[1], p.status, 2204)) { cut[1].out[k] = ent.y; prefetch_row(pf, ent.y); }
+        }
+        rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
+    }
+    // the next unit's level-0 buffer (bins and count) must be zero when it starts
+    int* g0nxt = sl.g0 + ((epoch + j + 1) % 3) * kG0Stride;
+#pragma unroll 1
+    for (int i = tid; i <= kBins; i += kSel) g0nxt[i] = 0;
+    sel_sync();
+    return true;
+}
+
 // ------------------------------------------------------------ Reindex: one select per group
 // A Reindex pool fits in one CTA's shared memory, so the group does not run the
 // distributed select: every CTA publishes its scores (element order), its element
@@ -1740,6 +1912,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // select only: the unit's scores come from the multi-query scoring kernel; the
         // chunk goes to shared memory when it fits, and its histogram is built here
         const int* src = p.pre ? p.pre + (size_t)u * p.pstride + lo : nullptr;
+        if (src && p.G == 1 && p.chunk > kSmemScores) {
+            // one CTA per query, scores in global memory: the sampled select first
+            if (tid < kSel) {
+                const bool done = sampled_select(p, S, sl, u, j, epoch, src, my_n);
+                if (tid == 0) S.info[25] = done ? 1 : 0;
+            }
+            __syncthreads();
+            if (S.info[25]) {
+                __syncthreads();   // (S.info is reused by the next unit)
+                continue;
+            }
+            for (int i = tid; i < kBins; i += kTcThreads) S.hist0[i] = 0;   // it used the histogram as scratch
+            __syncthreads();
+        }
         if (src) {
             // 16-byte loads, eight in flight per thread (the unit's row and the chunk
             // start are multiples of 4 elements): each round is one L2 round trip

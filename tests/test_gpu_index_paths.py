@@ -150,3 +150,29 @@ def test_weights_past_the_bound_are_rejected(ws):
     assert capi.csa2_index_topk(a, buf.data_ptr(), buf.numel(), 0, 0) == 5   # CSA2_ERR_RANGE
     w[3] = max_weight(8, 64)
     assert capi.csa2_workspace_bytes(0, a) > 0
+
+
+@pytest.mark.parametrize("kind", ["random", "rising", "equal"])
+def test_select_only_one_cta_per_query(kind, ws, status):
+    """Queries that share keys, more of them than SMs: the multi-query scoring kernel,
+    then one CTA per query cuts that query's scores from global memory. Random scores
+    take the sampled select (a threshold estimate from every s-th score, one candidate
+    pass, the exact cut over the candidates); scores that rise with the position (the
+    best ones all in the last warp's range of positions) and all-equal scores overflow
+    its candidate lists and take the full select. Every list bit-exact."""
+    from oracle import cpp as C
+    B, Tq, N, Hi, Di, k, P = 1, 160, 40000, 8, 64, 512, 2048
+    qi, w, ki = inputs(31, B, Tq, N, Hi, Di, False)
+    if kind == "rising":
+        qi[:] = 1
+        ki[:] = (np.arange(N) * 127 // N).astype(np.int8)[None, :, None]
+    elif kind == "equal":
+        ki[:] = 0
+    q_pos = np.broadcast_to(np.arange(N - Tq, N, dtype=np.int32), (B, Tq)).copy()
+    pool, topk = ops.index_topk("FULL", dev(q_pos), dev(qi), w, dev(ki), k, P, ws=ws, status=status)
+    status.check(kind)
+    rpool, rtopk = C.index_full_batch(q_pos, qi, w, ki, k, P)
+    assert_list_invariants(topk.cpu().numpy(), q_pos, "topk")
+    assert_list_invariants(pool.cpu().numpy(), q_pos, "pool")
+    assert_lists_equal(topk, rtopk, f"{kind}: topk")
+    assert_lists_equal(pool, rpool, f"{kind}: pool")

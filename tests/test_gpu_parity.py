@@ -455,3 +455,19 @@ def test_encoder_m2_early_positions(ws, status):
         _, ref = O.index_full(qi[0, j], w, ki[0], j, 4, 0, m)
         assert np.array_equal(got[0, j], ref)
         assert (got[0, j] >= 0).sum() == min(4, (j + 1) // 2)
+
+
+def test_one_workspace_serves_calls_of_different_sizes(status):
+    """A workspace is zeroed once and then serves calls of any sizes in turn. A Full call
+    over 4 queries that share 2^20 keys leaves their scores in its scratch; an attention
+    call over 320 queries that then merges by tickets (one CTA per tile) must find its
+    tickets zero, so the ticket region may not move with the number of queries."""
+    ws = ops.Workspace()
+    N1 = 1 << 20
+    qi = synth.randint_i8(5, 1, (1, 4, 8, 64))
+    ki = synth.randint_i8(5, 2, (1, N1, 64))
+    w = synth.randint_i32(5, 3, (8,), 1, 8)
+    q_pos = np.arange(N1 - 4, N1, dtype=np.int32)[None, :]
+    ops.index_topk("FULL", dev(q_pos), dev(qi), w, dev(ki), 2048, 0, ws=ws, status=status)
+    status.check("Full call")
+    _attn_case(1, 4096, 320, 16, 128, 256, 128, seed=9, ws=ws, status=status)
