@@ -755,7 +755,9 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ phase trace
 PHASES = {
-    "full_index": {1: "dependency wait", 2: "scan done", 3: "histograms exchanged", 4: "threshold bins",
+    "full_index": {1: "dependency wait", 2: "scan done", 18: "sample (select only)", 19: "estimates (select only)",
+                   20: "candidate pass (select only)", 21: "exact cut (select only)",
+                   3: "histograms exchanged", 4: "threshold bins",
                    5: "ordered lists", 7: "candidates exchanged", 8: "finalise", 12: "candidates loaded",
                    13: "thresholds, counts", 9: "write", 10: "lists written", 11: "end"},
     "reindex_index": {1: "dependency wait", 2: "scores done", 3: "scores published", 4: "all scores loaded",

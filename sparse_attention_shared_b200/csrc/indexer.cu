@@ -1332,9 +1332,9 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
 
 // ------------------------------------------------------------ select only: sampled threshold
 // The select-only pass of one query by one CTA, its scores in global memory (more than
-// shared memory holds). A sample of at most 4096 scores (every s-th position) gives
-// each track a threshold estimate: the sample's value at 1.2 times the rank the track's
-// cut would have in the sample, plus 16. One ordered pass keeps every score at or above
+// shared memory holds). A sample of at most 4096 scores (runs of 4 positions, every s-th
+// run) gives each track a threshold estimate: the sample's value at 1.2 times the rank
+// the track's cut would have in the sample, plus 16. One ordered pass keeps every score at or above
 // the lower estimate as a candidate (position order, a list per warp over its range
 // of positions) and counts the scores at or above each track's estimate. When every
 // track has at least its rank r there, all of its r best scores are candidates, and
@@ -1357,29 +1357,47 @@ __device__ __noinline__ bool sampled_select(const IdxParams& p, IdxSmem& S, cons
     }
     if (!act[0] && !act[1]) return false;
 
-    // ---- sample and estimates
-    const int s = (n + kSampleMax - 1) / kSampleMax, m = (n + s - 1) / s;
+    // ---- sample (runs of 4 positions: one 16-byte load each) and estimates
+    const int nruns = n >> 2;   // whole runs (n > r >= 1; a shorter tail is not sampled)
+    const int s = max(1, (nruns + kSampleMax / 4 - 1) / (kSampleMax / 4)), mr = nruns / s, m = 4 * mr;
+    int smin = INT_MAX, smax = INT_MIN;
 #pragma unroll
-    for (int q = 0; q < kSampleMax / kSel; ++q) {
+    for (int q = 0; q < kSampleMax / 4 / kSel; ++q) {
         const int i = q * kSel + tid;
-        if (i < m) S.sc[i] = __ldcg(src + (size_t)i * s);
+        if (i < mr) {
+            const int4 v = __ldcg(reinterpret_cast<const int4*>(src) + (size_t)i * s);
+            reinterpret_cast<int4*>(S.sc)[i] = v;
+            smin = min(min(smin, min(v.x, v.y)), min(v.z, v.w));
+            smax = max(max(smax, max(v.x, v.y)), max(v.z, v.w));
+        }
     }
+    if (m == 0) return false;
+    // the sample's range, so that the radix passes below spread over it
+    smin = __reduce_min_sync(0xffffffffu, smin);
+    smax = __reduce_max_sync(0xffffffffu, smax);
+    if (tid == 0) { S.info[26] = INT_MAX; S.info[27] = INT_MIN; S.info[28] = INT_MIN; }
     sel_sync();
+    if (lane == 0) { atomicMin(&S.info[26], smin); atomicMax(&S.info[27], smax); }
+    sel_sync();
+    smin = S.info[26];
+    smax = S.info[27];
+    CSA2_TRACE(18);   // sampled select: sample loaded
     int qr[2];
 #pragma unroll
     for (int tr = 0; tr < 2; ++tr)
         qr[tr] = act[tr] ? min(m, (int)((long long)r[tr] * m / n * 6 / 5) + 16) : 0;
-    const int4 est = local_select2(S.sc, act[0] ? m : 0, qr[0], INT_MIN, INT_MAX, S.sc, act[1] ? m : 0, qr[1],
-                                   INT_MIN, INT_MAX, S.hist0, S.red, S.info);
+    const int4 est = local_select2(S.sc, act[0] ? m : 0, qr[0], smin, smax, S.sc, act[1] ? m : 0, qr[1],
+                                   smin, smax, S.hist0, S.red, S.info);
     const int te0 = act[0] ? est.x : INT_MAX, te1 = act[1] ? est.z : INT_MAX;
     const int tlo = min(te0, te1);
+    CSA2_TRACE(19);   // sampled select: estimates
 
     // ---- one ordered pass: candidates >= tlo, counts >= each estimate
     int2* lists = reinterpret_cast<int2*>(&S.stage[0][0]);
     int2* list = lists + wp * kCandPerWarp;
     const int nstep = (n + 127) >> 7, spw = (nstep + kSelWarps - 1) / kSelWarps;
     const int s0 = min(nstep, wp * spw), s1 = min(nstep, s0 + spw);
-    int ln = 0, c0 = 0, c1 = 0;
+    int ln = 0, c0 = 0, c1 = 0, cmax = INT_MIN;
     constexpr int kIn = 8;
 #pragma unroll 1
     for (int st0 = s0; st0 < s1; st0 += kIn) {
@@ -1401,6 +1419,7 @@ __device__ __noinline__ bool sampled_select(const IdxParams& p, IdxSmem& S, cons
             for (int k = 0; k < 4; ++k) {
                 const bool ok = e0 + k < n;
                 f[k] = ok && x[k] >= tlo;
+                if (f[k]) cmax = max(cmax, x[k]);
                 c0 += ok && x[k] >= te0;
                 c1 += ok && x[k] >= te1;
                 b[k] = __ballot_sync(0xffffffffu, f[k]);
@@ -1417,12 +1436,15 @@ __device__ __noinline__ bool sampled_select(const IdxParams& p, IdxSmem& S, cons
     }
     if (tid == 0) S.info[24] = 0;
     sel_sync();
+    cmax = __reduce_max_sync(0xffffffffu, cmax);
     if (lane == 0) {
         S.wlist_n[wp] = min(ln, kCandPerWarp);
         if (ln > kCandPerWarp) S.info[24] = 1;
+        atomicMax(&S.info[28], cmax);   // the candidates' largest score: the exact cut's range
     }
     int4 ca = make_int4(c0, c1, 0, 0), cb = make_int4(0, 0, 0, 0);
     sel_total8(ca, cb, S.red);   // (its barriers also publish wlist_n and the overflow flag)
+    CSA2_TRACE(20);   // sampled select: candidate pass
     if (S.info[24] != 0 || (act[0] && ca.x < r[0]) || (act[1] && ca.y < r[1])) {
         sel_sync();
         return false;
@@ -1439,8 +1461,10 @@ __device__ __noinline__ bool sampled_select(const IdxParams& p, IdxSmem& S, cons
 #pragma unroll 1
     for (int i = lane; i < mine; i += 32) S.sc[base + i] = list[i].x;
     sel_sync();
-    const int4 ls = local_select2(S.sc, act[0] ? total : 0, r[0], tlo, INT_MAX, S.sc, act[1] ? total : 0, r[1],
-                                  tlo, INT_MAX, S.hist0, S.red, S.info);
+    const int chi = S.info[28];
+    const int4 ls = local_select2(S.sc, act[0] ? total : 0, r[0], tlo, chi, S.sc, act[1] ? total : 0, r[1],
+                                  tlo, chi, S.hist0, S.red, S.info);
+    CSA2_TRACE(21);   // sampled select: exact cut
     ListCut cut[2];
 #pragma unroll
     for (int tr = 0; tr < 2; ++tr) {
