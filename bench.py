@@ -595,10 +595,13 @@ def index_kernel_name(s, mode):
 
 
 def attn_kernel_name(s, HQP, k, sms):
-    """The kernel csa2_sparse_attn launches (the library's dispatch rule, restated): the
+    """The kernel csa2_sparse_attn launches (the library's dispatch rule, restated): one CTA
+    per query over all of its tiles for calls of at least two queries per SM; else the
     cluster kernel while its cluster (one CTA per 256 list entries, one per 128 window rows)
     holds at most 16 CTAs and, at 16 heads, the call's clusters hold at most 4 CTAs per SM;
     else the ticket kernel."""
+    if s.B * s.Tq >= 2 * sms:
+        return f"sparse_attn_seq_kernel<{HQP},{s.D}>"
     cs = -(-k // 256) + -(-s.W // 128)
     many = s.Hq <= 16 and s.B * s.Tq * cs > 4 * sms
     if 1 <= cs <= 16 and s.B * s.Tq <= 65535 and not many:
@@ -764,9 +767,12 @@ PHASES = {
                       5: "candidates", 6: "threshold", 7: "offsets", 11: "end"},
     "attention": {1: "dependency wait", 2: "positions", 3: "rows staged", 4: "tile ready", 5: "S done",
                   6: "softmax done", 7: "O done", 8: "partials exchanged", 9: "end"},
+    "attention_seq": {1: "first tile staged", 2: "first S done", 3: "first softmax done", 4: "first O done",
+                      5: "first tile done", 6: "last tile staged", 7: "last S done", 8: "last softmax done",
+                      9: "last O done", 10: "last tile done", 11: "end"},
 }
 KINDS = {1: "index_full_tc_kernel", 2: "index_dp4a_kernel", 3: "sparse_attn_cl_kernel", 4: "sparse_attn_kernel",
-         5: "index_mq_score_kernel"}
+         5: "index_mq_score_kernel", 6: "sparse_attn_seq_kernel"}
 
 
 def run_phase_trace(args):
@@ -842,7 +848,10 @@ def run_phase_trace(args):
         used = np.nonzero(h[:, 31])[0]
         span = (t[:, 3].max() - t[:, 2].min()) / 1e3 if n else 0.0
         print(f"{name}: {len(used)} CTAs traced, launch span {span:.1f} us")
-        for k, label in sorted(PHASES["full_index" if name == "full_index" else name].items(),
+        table = PHASES[name]
+        if name == "attention" and s.B * s.Tq >= 2 * torch.cuda.get_device_properties(0).multi_processor_count:
+            table = PHASES["attention_seq"]
+        for k, label in sorted(table.items(),
                                key=lambda kv: np.median(h[used, kv[0]]) if len(used) else 0):
             v = h[used, k]
             v = v[v > 0]

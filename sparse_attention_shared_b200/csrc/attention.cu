@@ -851,6 +851,306 @@ __global__ void __launch_bounds__(kClThreads, 2)
     if (warp == 0) tmem_dealloc(tmem, kCols);
 }
 
+// ------------------------------------------------------------ one CTA per query
+// For calls with many queries (a prefill chunk, a bounded replay), where throughput
+// counts rather than one query's latency: one CTA (128 threads) takes every tile of its
+// query in turn, the global tiles of its list and then its window tiles, 128 rows each,
+// with an online softmax. Per tile: S = K Q^T into TMEM, the tile's maximum per head
+// updates the running maximum m, P = exp2(s - m) goes to shared memory, O_tile^T = V^T P
+// into a fresh TMEM accumulator, and each thread (one row of O^T, one head dimension)
+// rescales its running o[h] by exp2(m_old - m_new) and adds the tile's. The query's
+// output is o / l at the end: no partials leave the CTA and nothing is merged.
+// Global rows are dequantised to bf16 (code times scale has at most seven significant
+// bits, so bf16 holds it exactly) and Q is bf16 for both kinds of tile.
+template <int HQP>
+struct __align__(1024) AttnSeqSmem {
+    uint8_t kbuf[2 * kPanelBytes];      // key tile (also the value tile of a global tile)
+    uint8_t vbuf[2 * kPanelBytes];      // value tile of a window tile
+    uint8_t qbuf[2 * HQP * 128];        // queries, [HQP rows x D] in 64-element panels
+    uint8_t pbuf[2 * HQP * 128];        // probabilities, [HQP rows x 128 keys] in 64-key panels
+    uint32_t lut[256];                  // code byte -> two bf16 E2M1 values
+    float red_m[4][HQP], red_l[4][HQP];
+    float m_run[HQP], l_run[HQP];       // running maximum (log2 units) and sum per head
+    float cf[HQP];                      // the tile's rescale exp2(m_old - m_new) per head
+    uint64_t bar_s, bar_o;
+    uint32_t tmem_base;
+};
+
+template <int HQP, int D>
+__global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
+    sparse_attn_seq_kernel(const __grid_constant__ AttnParams p) {
+    CSA2_TRACE_INIT();
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    AttnSeqSmem<HQP>& S =
+        *reinterpret_cast<AttnSeqSmem<HQP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    constexpr uint32_t kCols = (2 * HQP < 32) ? 32 : 2 * HQP;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int u = blockIdx.x;
+    const int b = u / p.Tq;
+
+    if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
+    if (tid == 0) {
+        mbar_init(&S.bar_s, 1);
+        mbar_init(&S.bar_o, 1);
+        mbar_fence_init();
+    }
+    for (int i = tid; i < 256; i += kAttnThreads)
+        S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
+    pdl_wait();   // the list, the query and the window's newest rows may come from the previous kernel
+    pdl_launch_dependents();
+
+    int t = p.q_pos[u];
+    int tg = last_entry(t, p.m);   // the last global entry the query reads
+    if (t < 0 || tg >= p.N) {
+        if (tid == 0) report(p.status, CSA2_ERR_RANGE, u);
+        t = -1;
+        tg = -1;
+    }
+    const int base = p.local_base[b];
+    const int lo_w = max(max(base, t - p.W + 1), 0);
+
+    // ---- queries -> qbuf (rows >= Hq are zero); a D = 64 value operand's second half is zero
+    for (int i = tid; i < HQP * (D / 8); i += kAttnThreads) {
+        const int h = i / (D / 8), c = i % (D / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (h < p.Hq) v = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
+        *reinterpret_cast<uint4*>(S.qbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = v;
+    }
+    if (D == 64) {
+        for (int i = tid; i < kPanelBytes / 16; i += kAttnThreads) {
+            reinterpret_cast<uint4*>(S.kbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(S.vbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    float o[HQP];   // this thread's row of O^T (head dimension tid), one value per head
+#pragma unroll
+    for (int h = 0; h < HQP; ++h) o[h] = 0.f;
+    if (tid < HQP) { S.m_run[tid] = -INFINITY; S.l_run[tid] = 0.f; }
+    const int lane = tid & 31;
+    const int hl = (HQP == 16) ? ((lane >> 1) & 15) : lane;   // the head a lane holds after a transpose-reduce
+    const int r = tid;   // this thread's key row of a tile
+    bool ok = true;
+    const int ntiles = p.ngt + p.nlt;
+#pragma unroll 1
+    for (int tau = 0; tau < ntiles; ++tau) {
+        const bool global_tile = tau < p.ngt;
+        bool valid = false;
+        // ---- the tile's 128 rows
+        if (global_tile) {
+            const int jj = tau * kTileKeys + r;
+            int s = (jj < p.k) ? __ldcg(p.topk + (size_t)u * p.k + jj) : -1;
+            if (s >= 0 && (s > tg || s >= p.N)) {
+                report(p.status, CSA2_ERR_RANGE, u);
+                s = -1;
+            }
+            valid = s >= 0;
+            if (valid) {
+                const size_t row = (size_t)b * p.N + s;
+                const uint4* cp = reinterpret_cast<const uint4*>(p.kv_fp4 + row * (D / 2));
+                uint4 codes[D / 32];
+#pragma unroll
+                for (int i = 0; i < D / 32; ++i) codes[i] = __ldg(cp + i);
+                uint32_t sw[D / 64];
+                if (D == 128) {
+                    const uint2 s2 = __ldg(reinterpret_cast<const uint2*>(p.kv_scale + row * 8));
+                    sw[0] = s2.x;
+                    sw[1 % (D / 64)] = s2.y;
+                } else {
+                    sw[0] = __ldg(reinterpret_cast<const uint32_t*>(p.kv_scale + row * 4));
+                }
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {           // 8 elements (4 code bytes) per chunk
+                    const uint4 cw = codes[c >> 2];
+                    const uint32_t w = (c & 3) == 0 ? cw.x : (c & 3) == 1 ? cw.y : (c & 3) == 2 ? cw.z : cw.w;
+                    const uint32_t g = c >> 1;              // 16-element scale group
+                    const uint32_t sb = (sw[g >> 2] >> (8 * (g & 3))) & 0xFFu;
+                    const uint32_t s16 = e4m3_bf16_bits(sb);
+                    const uint32_t s2x = s16 | (s16 << 16);
+                    uint4 ov;
+                    ov.x = bf16x2_mul(S.lut[w & 0xFFu], s2x);
+                    ov.y = bf16x2_mul(S.lut[(w >> 8) & 0xFFu], s2x);
+                    ov.z = bf16x2_mul(S.lut[(w >> 16) & 0xFFu], s2x);
+                    ov.w = bf16x2_mul(S.lut[w >> 24], s2x);
+                    *reinterpret_cast<uint4*>(S.kbuf + (c >> 3) * kPanelBytes + sw128(r, c & 7)) = ov;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c)
+                    *reinterpret_cast<uint4*>(S.kbuf + (c >> 3) * kPanelBytes + sw128(r, c & 7)) = make_uint4(0, 0, 0, 0);
+            }
+        } else {
+            // window rows [lo_w, t], tile lt: coalesced 16-byte loads of K and V
+            const int p0 = lo_w + (tau - p.ngt) * kTileKeys;
+            {
+                const int pr = p0 + r;
+                valid = (t >= 0) && (p.W > 0) && (pr <= t);
+                if (valid && (pr - base < 0 || pr - base >= p.Lloc)) {
+                    report(p.status, CSA2_ERR_RANGE, u);
+                    valid = false;
+                }
+            }
+            const uint4* kls = reinterpret_cast<const uint4*>(p.kl);
+            const uint4* vls = reinterpret_cast<const uint4*>(p.vl);
+            constexpr int CPR = D / 8;                              // 16-byte chunks per row
+            constexpr int ITERS = kTileKeys * CPR / kAttnThreads;   // chunks per thread per tensor
+            constexpr int BATCH = ITERS < 8 ? ITERS : 8;            // loads in flight per tensor
+#pragma unroll
+            for (int i0 = 0; i0 < ITERS; i0 += BATCH) {
+                uint4 kv[BATCH], vv[BATCH];
+#pragma unroll
+                for (int jb = 0; jb < BATCH; ++jb) {
+                    const int i = tid + (i0 + jb) * kAttnThreads;
+                    const int rr = i / CPR, c = i % CPR;
+                    const int pr = p0 + rr;
+                    const int lrow = pr - base;
+                    const bool okr = (t >= 0) && (p.W > 0) && (pr <= t) && lrow >= 0 && lrow < p.Lloc;
+                    kv[jb] = make_uint4(0, 0, 0, 0);
+                    vv[jb] = make_uint4(0, 0, 0, 0);
+                    if (okr) {
+                        const size_t off = ((size_t)b * p.Lloc + lrow) * CPR + c;
+                        kv[jb] = __ldg(kls + off);
+                        vv[jb] = __ldg(vls + off);
+                    }
+                }
+#pragma unroll
+                for (int jb = 0; jb < BATCH; ++jb) {
+                    const int i = tid + (i0 + jb) * kAttnThreads;
+                    const int rr = i / CPR, c = i % CPR;
+                    const uint32_t dst = (c >> 3) * kPanelBytes + sw128(rr, c & 7);
+                    *reinterpret_cast<uint4*>(S.kbuf + dst) = kv[jb];
+                    *reinterpret_cast<uint4*>(S.vbuf + dst) = vv[jb];
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();   // the tile (and, at the first tile, Q, the barriers and TMEM) is in place
+        tc_fence_after();
+        const int tslot = tau == 0 ? 1 : tau == ntiles - 1 ? 6 : 0;   // phase-trace slots (first, last tile)
+        if (tslot) { CSA2_TRACE(tslot); }   // tile staged
+        const uint32_t tmem_s = S.tmem_base, tmem_o = S.tmem_base + HQP;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+
+        // ---- S = K Q^T  (M = 128 keys, N = HQP heads, K = D)
+        if (tid == 0 && ok) {
+            const uint32_t ka = smem_u32(S.kbuf), qa = smem_u32(S.qbuf);
+            constexpr uint32_t idesc = idesc_bf16(128, HQP, 0);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t ad = smem_desc(ka + (kk >> 2) * kPanelBytes + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = smem_desc(qa + (kk >> 2) * (HQP * 128) + (kk & 3) * 32, 16, 1024);
+                mma_bf16(tmem_s, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&S.bar_s);
+        }
+        ok = ok && mbar_wait(&S.bar_s, (uint32_t)(tau & 1), p.status, 13);
+        tc_fence_after();
+        if (tslot) { CSA2_TRACE(tslot + 1); }   // S done
+
+        // ---- online softmax: the tile's maximum per head, then P and the tile's sums
+        float sv[HQP];
+#pragma unroll
+        for (int h = 0; h < HQP; ++h) sv[h] = 0.f;
+        if (ok) {
+            float tmp[16];
+#pragma unroll
+            for (int c0 = 0; c0 < HQP; c0 += 16) {
+                tmem_ld16(tmem_s + lane_off + c0, tmp);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sv[c0 + i] = tmp[i];
+            }
+        }
+        const bool rv = valid && ok;
+        {
+            float v[HQP];
+#pragma unroll
+            for (int h = 0; h < HQP; ++h) {
+                sv[h] = rv ? sv[h] * p.scale_log2 : -INFINITY;
+                v[h] = sv[h];
+            }
+            const float mx = warp_transpose_reduce<HQP, true>(v);
+            if (HQP == 32 || (lane & 1) == 0) S.red_m[warp][hl] = mx;
+        }
+        __syncthreads();
+        if (tid < HQP) {   // one thread per head: the new running maximum and the rescale
+            const float mt = fmaxf(fmaxf(S.red_m[0][tid], S.red_m[1][tid]), fmaxf(S.red_m[2][tid], S.red_m[3][tid]));
+            const float mo = S.m_run[tid], mn = fmaxf(mo, mt);
+            S.cf[tid] = (mn == -INFINITY) ? 1.f : exp2f(mo - mn);
+            S.m_run[tid] = mn;
+        }
+        __syncthreads();
+        {
+            float pv[HQP];
+#pragma unroll
+            for (int h = 0; h < HQP; ++h) {
+                const float mn = S.m_run[h];
+                pv[h] = (rv && mn != -INFINITY) ? exp2f(sv[h] - mn) : 0.f;
+                *reinterpret_cast<__nv_bfloat16*>(S.pbuf + (r >> 6) * (HQP * 128) + sw128(h, (r & 63) >> 3) + (r & 7) * 2) =
+                    __float2bfloat16_rn(pv[h]);
+            }
+            const float l = warp_transpose_reduce<HQP, false>(pv);
+            if (HQP == 32 || (lane & 1) == 0) S.red_l[warp][hl] = l;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();   // P and the tile sums are in place
+        tc_fence_after();
+        if (tslot) { CSA2_TRACE(tslot + 2); }   // softmax done
+
+        // ---- O_tile^T = V^T P  (M = 128 = head dim (padded), N = HQP, K = 128 keys)
+        if (tid == 0 && ok) {
+            const uint32_t va = smem_u32(global_tile ? S.kbuf : S.vbuf), pa = smem_u32(S.pbuf);
+            constexpr uint32_t idesc = idesc_bf16(128, HQP, 1);
+#pragma unroll
+            for (int kk = 0; kk < kTileKeys / 16; ++kk) {
+                const uint64_t ad = smem_desc(va + kk * 2048, kPanelBytes, 1024);
+                const uint64_t bd = smem_desc(pa + (kk >> 2) * (HQP * 128) + (kk & 3) * 32, 16, 1024);
+                mma_bf16(tmem_o, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&S.bar_o);
+        }
+        if (tid < HQP)   // (the thread that owns head tid's running values)
+            S.l_run[tid] = S.l_run[tid] * S.cf[tid] + (S.red_l[0][tid] + S.red_l[1][tid]) + (S.red_l[2][tid] + S.red_l[3][tid]);
+        ok = ok && mbar_wait(&S.bar_o, (uint32_t)(tau & 1), p.status, 14);
+        tc_fence_after();
+        if (tslot) { CSA2_TRACE(tslot + 3); }   // O done
+        if (ok) {
+            float tmp[16];
+#pragma unroll
+            for (int c0 = 0; c0 < HQP; c0 += 16) {
+                tmem_ld16(tmem_o + lane_off + c0, tmp);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[c0 + i] = o[c0 + i] * S.cf[c0 + i] + tmp[i];
+            }
+        }
+        tc_fence_before();
+        __syncthreads();   // every read of this tile's buffers, TMEM and sums is done
+        if (tslot) { CSA2_TRACE(tslot + 4); }   // tile done
+    }
+
+    // ---- out = o / l (thread = head dimension), lse in natural-log units
+    if (tid < D) {
+#pragma unroll
+        for (int h = 0; h < HQP; ++h) {
+            if (h >= p.Hq) break;
+            const float L = S.l_run[h];
+            p.out[((size_t)u * p.Hq + h) * D + tid] =
+                __bfloat16_as_ushort(__float2bfloat16_rn((ok && L > 0.f) ? o[h] / L : 0.f));
+        }
+    }
+    if (tid < p.Hq && p.lse != nullptr) {
+        const float mv = S.m_run[tid], lv = S.l_run[tid];
+        p.lse[(size_t)u * p.Hq + tid] = (ok && lv > 0.f) ? (mv + log2f(lv)) * 0.69314718055994530942f : -INFINITY;
+    }
+    CSA2_TRACE(11);
+    CSA2_TRACE_END(6);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(S.tmem_base, kCols);
+}
+
 // ------------------------------------------------------------ host side
 struct AttnPlan {
     int units, ngt, nlt, ntiles, HQP;
@@ -905,6 +1205,46 @@ csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* ticke
 }
 
 size_t attn_scratch_bytes(const csa2_attn_args& a) { return plan_attn(a).part_bytes; }
+
+template <int HQP, int D>
+static cudaError_t launch_seq_variant(const AttnParams& p, int units, cudaStream_t stream) {
+    auto kern = sparse_attn_seq_kernel<HQP, D>;
+    const size_t smem = sizeof(AttnSeqSmem<HQP>) + 1024;
+    cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(units);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    // the kernel reads no input before pdl_wait(): it may start while the previous kernel runs
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// One CTA per query over all of its tiles (calls with many queries).
+csa2_status launch_attn_seq(const csa2_attn_args& a, const int32_t* topk, int32_t* d_status, cudaStream_t stream) {
+    AttnPlan pl = plan_attn(a);
+    if (pl.units == 0) return CSA2_OK;
+    AttnParams p{};
+    p.B = a.B; p.Tq = a.Tq; p.N = a.N; p.Hq = a.Hq; p.D = a.D; p.k = a.k; p.W = a.W; p.Lloc = a.Lloc;
+    p.ngt = pl.ngt; p.nlt = pl.nlt; p.ntiles = pl.ntiles;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)a.D));
+    p.q_pos = a.q_pos; p.q = a.q; p.kv_fp4 = a.kv_fp4; p.kv_scale = a.kv_scale; p.topk = topk;
+    p.kl = a.kl; p.vl = a.vl; p.local_base = a.local_base; p.out = a.out; p.lse = a.lse;
+    p.status = d_status;
+    p.m = a.m;
+    cudaError_t e;
+    if (pl.HQP == 16 && a.D == 128) e = launch_seq_variant<16, 128>(p, pl.units, stream);
+    else if (pl.HQP == 16 && a.D == 64) e = launch_seq_variant<16, 64>(p, pl.units, stream);
+    else if (pl.HQP == 32 && a.D == 128) e = launch_seq_variant<32, 128>(p, pl.units, stream);
+    else e = launch_seq_variant<32, 64>(p, pl.units, stream);
+    return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
 
 }  // namespace csa2
 

@@ -37,6 +37,7 @@ size_t attn_scratch_bytes(const csa2_attn_args& a);
 csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* tickets, void* scratch,
                         int32_t* d_status, cudaStream_t stream);
 bool attn_cluster_fits(const csa2_attn_args& a);
+csa2_status launch_attn_seq(const csa2_attn_args& a, const int32_t* topk, int32_t* d_status, cudaStream_t stream);
 csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
                                 cudaStream_t stream);
 
@@ -49,6 +50,11 @@ csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, in
 // (a prefill chunk of 4096 queries) the two are within 2%; the cluster kernel stays.
 static csa2_status run_attn(const csa2_attn_args& a, const int32_t* topk, int list_ready, int* tickets,
                             void* scratch, int32_t* d_status, cudaStream_t stream) {
+    static const int seq_min = [] {   // TEMPORARY A/B
+        const char* e = getenv("CSA2_SEQ_MIN_UNITS");
+        return e ? atoi(e) : 2 * num_sms();
+    }();
+    if ((int64_t)a.B * a.Tq >= seq_min) return launch_attn_seq(a, topk, d_status, stream);
     const int cs = (a.k + 255) / 256 + (a.W + 127) / 128;
     const bool many = a.Hq <= 16 && (int64_t)a.B * a.Tq * cs > 4LL * num_sms();
     if (attn_cluster_fits(a) && !many) return launch_attn_cluster(a, topk, list_ready, d_status, stream);

@@ -293,6 +293,9 @@ def test_attention_tiny(ws, status):
     (3, 5000, 1, 32, 64, 700, 300),      # 32 heads at D = 64, ragged blocks
     (2, 4096, 1, 16, 128, 1, 512),       # one global entry, four window tiles
     (1, 20000, 1, 32, 128, 100, 16284),  # k + W = 16384 with both branches ragged: 129 tiles, 32 heads
+    (1, 3000, 300, 32, 64, 700, 300),    # 300 queries: one CTA per query over all tiles, 32 heads, D = 64
+    (1, 3000, 300, 8, 64, 256, 128),     # the same at 16 (padded) heads
+    (2, 5000, 160, 16, 128, 1000, 200),  # 320 queries over two sequences, ragged tiles, D = 128
 ])
 def test_attention_shapes(B, N, Tq, Hq, D, k, W, ws, status):
     _attn_case(B, N, Tq, Hq, D, k, W, seed=B * 7 + N, ws=ws, status=status)
