@@ -931,6 +931,7 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
     const int r = tid;   // this thread's key row of a tile
     bool ok = true;
     const int ntiles = p.ngt + p.nlt;
+    int s_next = -1;     // the next global tile's list entry for this row, loaded during this tile
 #pragma unroll 1
     for (int tau = 0; tau < ntiles; ++tau) {
         const bool global_tile = tau < p.ngt;
@@ -938,7 +939,7 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         // ---- the tile's 128 rows
         if (global_tile) {
             const int jj = tau * kTileKeys + r;
-            int s = (jj < p.k) ? __ldcg(p.topk + (size_t)u * p.k + jj) : -1;
+            int s = tau == 0 ? ((jj < p.k) ? __ldcg(p.topk + (size_t)u * p.k + jj) : -1) : s_next;
             if (s >= 0 && (s > tg || s >= p.N)) {
                 report(p.status, CSA2_ERR_RANGE, u);
                 s = -1;
@@ -1028,6 +1029,10 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         tc_fence_after();
         const int tslot = tau == 0 ? 1 : tau == ntiles - 1 ? 6 : 0;   // phase-trace slots (first, last tile)
         if (tslot) { CSA2_TRACE(tslot); }   // tile staged
+        if (tau + 1 < p.ngt) {   // the next tile's list entry, in flight during this tile
+            const int jn = (tau + 1) * kTileKeys + r;
+            s_next = jn < p.k ? __ldcg(p.topk + (size_t)u * p.k + jn) : -1;
+        }
         const uint32_t tmem_s = S.tmem_base, tmem_o = S.tmem_base + HQP;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
@@ -1112,6 +1117,11 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         }
         if (tid < HQP)   // (the thread that owns head tid's running values)
             S.l_run[tid] = S.l_run[tid] * S.cf[tid] + (S.red_l[0][tid] + S.red_l[1][tid]) + (S.red_l[2][tid] + S.red_l[3][tid]);
+        if (tau + 1 < p.ngt && s_next >= 0 && s_next < p.N) {   // the next tile's row towards L1
+            const size_t row = (size_t)b * p.N + s_next;
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(p.kv_fp4 + row * (D / 2)));
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(p.kv_scale + row * (D / 16)));
+        }
         ok = ok && mbar_wait(&S.bar_o, (uint32_t)(tau & 1), p.status, 14);
         tc_fence_after();
         if (tslot) { CSA2_TRACE(tslot + 3); }   // O done

@@ -41,20 +41,19 @@ csa2_status launch_attn_seq(const csa2_attn_args& a, const int32_t* topk, int32_
 csa2_status launch_attn_cluster(const csa2_attn_args& a, const int32_t* topk, int list_ready, int32_t* d_status,
                                 cudaStream_t stream);
 
-// The attention kernel for a call: the cluster kernel (one CTA per 256 list entries or
-// 128 window rows, the partials merged through distributed shared memory) while the call
-// is latency-bound, else one CTA per 128-row tile with a ticket merge. Measured on one
+// The attention kernel for a call: with many queries, one CTA per query over all of its
+// tiles; else the cluster kernel (one CTA per 256 list entries or 128 window rows, the
+// partials merged through distributed shared memory) while the call is latency-bound,
+// else one CTA per 128-row tile with a ticket merge. Measured on one
 // B200 at 16 heads: the cluster kernel wins while the call's clusters hold at most about
 // four CTAs per SM (decode: 16-32 queries x 12 CTAs), the ticket kernel beyond (64 queries
 // x 16 CTAs: 57 against 61 us; 2048 queries x 12 CTAs: 0.83 against 0.98 ms). At 32 heads
 // (a prefill chunk of 4096 queries) the two are within 2%; the cluster kernel stays.
 static csa2_status run_attn(const csa2_attn_args& a, const int32_t* topk, int list_ready, int* tickets,
                             void* scratch, int32_t* d_status, cudaStream_t stream) {
-    static const int seq_min = [] {   // TEMPORARY A/B
-        const char* e = getenv("CSA2_SEQ_MIN_UNITS");
-        return e ? atoi(e) : 2 * num_sms();
-    }();
-    if ((int64_t)a.B * a.Tq >= seq_min) return launch_attn_seq(a, topk, d_status, stream);
+    // at least two queries per SM: one CTA per query over all of its tiles (a prefill chunk
+    // of 4096 queries: 1.63 ms against 2.86 ms for the cluster kernel)
+    if ((int64_t)a.B * a.Tq >= 2LL * num_sms()) return launch_attn_seq(a, topk, d_status, stream);
     const int cs = (a.k + 255) / 256 + (a.W + 127) / 128;
     const bool many = a.Hq <= 16 && (int64_t)a.B * a.Tq * cs > 4LL * num_sms();
     if (attn_cluster_fits(a) && !many) return launch_attn_cluster(a, topk, list_ready, d_status, stream);
