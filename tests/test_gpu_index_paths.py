@@ -176,3 +176,28 @@ def test_select_only_one_cta_per_query(kind, ws, status):
     assert_list_invariants(pool.cpu().numpy(), q_pos, "pool")
     assert_lists_equal(topk, rtopk, f"{kind}: topk")
     assert_lists_equal(pool, rpool, f"{kind}: pool")
+
+
+@pytest.mark.parametrize("kind", ["random", "rising", "equal"])
+def test_full_decode_skewed_scores(kind, ws, status):
+    """Decode queries in groups of 12 CTAs with ragged prefixes: random scores, scores that
+    rise with the position (every selected entry in the last CTAs' chunks, runs of equal
+    scores) and all-equal scores (the whole cut is ties, taken by position). Every list
+    bit-exact."""
+    from oracle import cpp as C
+    B, Tq, N, Hi, Di, k, P = 12, 1, 40000, 8, 64, 512, 2048
+    qi, w, ki = inputs(37, B, Tq, N, Hi, Di, False)
+    if kind == "rising":
+        qi[:] = 1
+        ki[:] = (np.arange(N) * 127 // N).astype(np.int8)[None, :, None]
+    elif kind == "equal":
+        ki[:] = 0
+    q_pos = np.full((B, Tq), N - 1, np.int32)
+    q_pos[:, 0] -= np.arange(B, dtype=np.int32) * 977   # ragged prefixes
+    pool, topk = ops.index_topk("FULL", dev(q_pos), dev(qi), w, dev(ki), k, P, ws=ws, status=status)
+    status.check(kind)
+    rpool, rtopk = C.index_full_batch(q_pos, qi, w, ki, k, P)
+    assert_list_invariants(topk.cpu().numpy(), q_pos, "topk")
+    assert_list_invariants(pool.cpu().numpy(), q_pos, "pool")
+    assert_lists_equal(topk, rtopk, f"{kind}: topk")
+    assert_lists_equal(pool, rpool, f"{kind}: pool")
