@@ -61,17 +61,37 @@ struct __align__(1024) AttnSmem {
     uint8_t vbuf[2 * kPanelBytes];      // value tile of a local tile
     uint8_t qbuf[2 * HQP * 128];        // queries, [HQP rows x D] in 64-element panels
     uint8_t pbuf[2 * HQP * 128];        // probabilities, [HQP rows x 128 keys] in 64-key panels
-    uint32_t lut[256];                  // code byte -> two bf16 E2M1 values
     float red[4][HQP];
     uint64_t bar_s, bar_o;
     uint32_t tmem_base;
     int is_last;
 };
 
-__device__ __forceinline__ uint32_t e2m1_bf16_bits(uint32_t c) {
-    const uint32_t mag = c & 7u;
-    uint32_t bits = (mag == 0u) ? 0u : (mag == 1u) ? 0x3F00u : ((((mag >> 1) + 126u) << 7) | ((mag & 1u) << 6));
-    return bits | ((c & 8u) << 12);
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Eight E2M1 codes (a 32-bit word, lowest nibble first) as four bf16x2 words, lower
+// element in the lower half, by byte permutes: the three magnitude bits of each of four
+// codes pick its value's high and low byte from two 8-entry byte tables (|v| = 0, 0.5,
+// 1, 1.5, 2, 3, 4, 6 as bf16), two permutes interleave the bytes into values, and one
+// more per pair of values moves the codes' sign bits to bit 15 of each. Registers only:
+// no table in shared memory and no bank conflicts.
+__device__ __forceinline__ uint4 e2m1x8_bf16(uint32_t w) {
+    constexpr uint32_t kHi03 = 0x3F3F3F00u, kHi47 = 0x40404040u;   // high bytes, magnitudes 0-3 and 4-7
+    constexpr uint32_t kLo03 = 0xC0800000u, kLo47 = 0xC0804000u;   // low bytes
+    const uint32_t m = w & 0x77777777u, mh = m >> 16, w4 = w << 4;
+    const uint32_t ha = prmt(kHi03, kHi47, m), la = prmt(kLo03, kLo47, m);
+    const uint32_t hb = prmt(kHi03, kHi47, mh), lb = prmt(kLo03, kLo47, mh);
+    uint4 r;
+    // sign of code 2i: bit 7 of byte i of w << 4; of code 2i + 1: bit 7 of byte i of w
+    r.x = prmt(la, ha, 0x5140u) | (prmt(w4, w, 0x4000u) & 0x80008000u);
+    r.y = prmt(la, ha, 0x7362u) | (prmt(w4, w, 0x5010u) & 0x80008000u);
+    r.z = prmt(lb, hb, 0x5140u) | (prmt(w4, w, 0x6020u) & 0x80008000u);
+    r.w = prmt(lb, hb, 0x7362u) | (prmt(w4, w, 0x7030u) & 0x80008000u);
+    return r;
 }
 
 __device__ __forceinline__ uint32_t e4m3_bf16_bits(uint32_t b) {
@@ -150,8 +170,6 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
         mbar_init(&S.bar_o, 1);
         mbar_fence_init();
     }
-    for (int i = tid; i < 256; i += kAttnThreads)
-        S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
 
     int t = p.q_pos[u];
     int tg = last_entry(t, p.m);   // the last global entry the query reads
@@ -209,11 +227,12 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
                 const uint32_t sb = (sw[g >> 2] >> (8 * (g & 3))) & 0xFFu;
                 const uint32_t s16 = e4m3_bf16_bits(sb);
                 const uint32_t s2x = s16 | (s16 << 16);
+                const uint4 e = e2m1x8_bf16(w);
                 uint4 o;
-                o.x = bf16x2_mul(S.lut[w & 0xFFu], s2x);
-                o.y = bf16x2_mul(S.lut[(w >> 8) & 0xFFu], s2x);
-                o.z = bf16x2_mul(S.lut[(w >> 16) & 0xFFu], s2x);
-                o.w = bf16x2_mul(S.lut[w >> 24], s2x);
+                o.x = bf16x2_mul(e.x, s2x);
+                o.y = bf16x2_mul(e.y, s2x);
+                o.z = bf16x2_mul(e.z, s2x);
+                o.w = bf16x2_mul(e.w, s2x);
                 *reinterpret_cast<uint4*>(S.kbuf + (c >> 3) * kPanelBytes + sw128(r, c & 7)) = o;
             }
         } else {
@@ -489,11 +508,13 @@ static_assert(offsetof(AttnClSmem<16>, qpbuf) % 1024 == 0 && offsetof(AttnClSmem
               "operand alignment");
 static_assert(sizeof(AttnClSmem<32>) + 1024 <= 113 * 1024, "two clustered-attention CTAs per SM");
 
-// Reduce V values per lane (V = 16 or 32, one per head) across the 32 lanes of a
+// Reduce V values per lane (V = 8, 16 or 32, one per head) across the 32 lanes of a
 // warp with halving exchanges: after the call, lane l holds in v[0] the result for
-// head (l >> 1) & 15 (V = 16) or l & 31 (V = 32). 31 or 16 shuffles instead of 5*V.
+// value (l / (32 / V)) % V: head l & 31 (V = 32), (l >> 1) & 15 (V = 16) or (l >> 2) & 7
+// (V = 8). V - 1 + log2(32 / V) shuffles instead of 5*V.
 template <int V, bool kMax>
 __device__ __forceinline__ float warp_transpose_reduce(float (&v)[V]) {
+    static_assert(V == 8 || V == 16 || V == 32, "values per lane");
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int half = V / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
@@ -506,8 +527,9 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[V]) {
             v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
         }
     }
-    if (V == 16) {   // lanes l and l ^ 1 still hold partials of the same head
-        const float recv = __shfl_xor_sync(0xffffffffu, v[0], 1);
+#pragma unroll
+    for (int bit = 16 / V; bit >= 1; bit >>= 1) {   // lanes that still hold partials of the same value
+        const float recv = __shfl_xor_sync(0xffffffffu, v[0], bit);
         v[0] = kMax ? fmaxf(v[0], recv) : v[0] + recv;
     }
     return v[0];
@@ -853,13 +875,17 @@ __global__ void __launch_bounds__(kClThreads, 2)
 
 // ------------------------------------------------------------ one CTA per query
 // For calls with many queries (a prefill chunk, a bounded replay), where throughput
-// counts rather than one query's latency: one CTA (128 threads) takes every tile of its
-// query in turn, the global tiles of its list and then its window tiles, 128 rows each,
-// with an online softmax. Per tile: S = K Q^T into TMEM, the tile's maximum per head
-// updates the running maximum m, P = exp2(s - m) goes to shared memory, O_tile^T = V^T P
-// into a fresh TMEM accumulator, and each thread (one row of O^T, one head dimension)
-// rescales its running o[h] by exp2(m_old - m_new) and adds the tile's. The query's
-// output is o / l at the end: no partials leave the CTA and nothing is merged.
+// counts rather than one query's latency: one CTA (NT = 128 or 256 threads) takes every
+// tile of its query in turn, the global tiles of its list and then its window tiles, 128
+// rows each, with an online softmax. Per tile: S = K Q^T into TMEM, the tile's maximum per
+// head updates the running maximum m, P = exp2(s - m) goes to shared memory, O_tile^T =
+// V^T P into a fresh TMEM accumulator, and each thread (one row of O^T, one head
+// dimension, its part of the heads) rescales its running o[h] by exp2(m_old - m_new) and
+// adds the tile's. The query's output is o / l at the end: no partials leave the CTA and
+// nothing is merged. NT / 128 threads stage each row of a tile (a part of the row each);
+// in the softmax and the O update, warp w reads TMEM lanes 32 (w % 4) .. + 31 and the
+// columns of head part w / 4. 16 padded heads run 128 threads at three CTAs per SM, 32
+// heads 256 threads at two (shared memory holds two of those).
 // Global rows are dequantised to bf16 (code times scale has at most seven significant
 // bits, so bf16 holds it exactly) and Q is bf16 for both kinds of tile.
 template <int HQP>
@@ -868,23 +894,42 @@ struct __align__(1024) AttnSeqSmem {
     uint8_t vbuf[2 * kPanelBytes];      // value tile of a window tile
     uint8_t qbuf[2 * HQP * 128];        // queries, [HQP rows x D] in 64-element panels
     uint8_t pbuf[2 * HQP * 128];        // probabilities, [HQP rows x 128 keys] in 64-key panels
-    uint32_t lut[256];                  // code byte -> two bf16 E2M1 values
     float red_m[4][HQP], red_l[4][HQP];
     float m_run[HQP], l_run[HQP];       // running maximum (log2 units) and sum per head
     float cf[HQP];                      // the tile's rescale exp2(m_old - m_new) per head
+    int rowok[kTileKeys];               // the tile's rows that hold an entry
     uint64_t bar_s, bar_o;
     uint32_t tmem_base;
 };
 
-template <int HQP, int D>
-__global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
+// HH consecutive TMEM columns of this warp's 32 lanes (HH = 8 or 16).
+template <int HH>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[HH]) {
+    if constexpr (HH == 16) {
+        tmem_ld16(taddr, v);
+    } else {
+        int t[8];
+        tmem_ld8(taddr, t);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __int_as_float(t[i]);
+    }
+}
+
+template <int HQP> constexpr int seq_threads() { return HQP == 16 ? 128 : 256; }
+
+template <int HQP, int D, int NT = seq_threads<HQP>()>
+__global__ void __launch_bounds__(NT, NT == 128 && HQP == 16 ? 3 : 2)
     sparse_attn_seq_kernel(const __grid_constant__ AttnParams p) {
     CSA2_TRACE_INIT();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     AttnSeqSmem<HQP>& S =
         *reinterpret_cast<AttnSeqSmem<HQP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     constexpr uint32_t kCols = (2 * HQP < 32) ? 32 : 2 * HQP;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    constexpr int TPR = NT / 128;          // threads per row of a tile
+    constexpr int HH = HQP / TPR;          // heads per warp in the softmax and the O update
+    constexpr int kLpv = 32 / HH;          // lanes that hold one head after a transpose-reduce
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, hh0 = (warp >> 2) * HH;   // TMEM lane quarter, first head of this warp
     const int u = blockIdx.x;
     const int b = u / p.Tq;
 
@@ -894,8 +939,6 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         mbar_init(&S.bar_o, 1);
         mbar_fence_init();
     }
-    for (int i = tid; i < 256; i += kAttnThreads)
-        S.lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);
     pdl_wait();   // the list, the query and the window's newest rows may come from the previous kernel
     pdl_launch_dependents();
 
@@ -910,97 +953,105 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
     const int lo_w = max(max(base, t - p.W + 1), 0);
 
     // ---- queries -> qbuf (rows >= Hq are zero); a D = 64 value operand's second half is zero
-    for (int i = tid; i < HQP * (D / 8); i += kAttnThreads) {
+    for (int i = tid; i < HQP * (D / 8); i += NT) {
         const int h = i / (D / 8), c = i % (D / 8);
         uint4 v = make_uint4(0, 0, 0, 0);
         if (h < p.Hq) v = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)u * p.Hq + h) * D) + c);
         *reinterpret_cast<uint4*>(S.qbuf + (c >> 3) * (HQP * 128) + sw128(h, c & 7)) = v;
     }
     if (D == 64) {
-        for (int i = tid; i < kPanelBytes / 16; i += kAttnThreads) {
+        for (int i = tid; i < kPanelBytes / 16; i += NT) {
             reinterpret_cast<uint4*>(S.kbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
             reinterpret_cast<uint4*>(S.vbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
         }
     }
-    float o[HQP];   // this thread's row of O^T (head dimension tid), one value per head
+    float o[HH];   // this thread's row of O^T (head dimension 32 * quarter + lane), heads hh0 ..
 #pragma unroll
-    for (int h = 0; h < HQP; ++h) o[h] = 0.f;
+    for (int h = 0; h < HH; ++h) o[h] = 0.f;
     if (tid < HQP) { S.m_run[tid] = -INFINITY; S.l_run[tid] = 0.f; }
-    const int lane = tid & 31;
-    const int hl = (HQP == 16) ? ((lane >> 1) & 15) : lane;   // the head a lane holds after a transpose-reduce
-    const int r = tid;   // this thread's key row of a tile
+    const int hl = hh0 + ((lane / kLpv) % HH);   // the head a lane holds after a transpose-reduce
+    const bool hl_writer = (lane % kLpv) == 0;
+    const int rs = tid / TPR, part = tid % TPR;  // staging: this thread's row of a tile and its part
+    const int rm = quarter * 32 + lane;          // softmax: this thread's key row (TMEM lane)
     bool ok = true;
     const int ntiles = p.ngt + p.nlt;
-    int s_next = -1;     // the next global tile's list entry for this row, loaded during this tile
+    int s_next = -1;     // the next global tile's list entry for row rs, loaded during this tile
 #pragma unroll 1
     for (int tau = 0; tau < ntiles; ++tau) {
         const bool global_tile = tau < p.ngt;
-        bool valid = false;
-        // ---- the tile's 128 rows
+        // ---- the tile's 128 rows, two threads a row
         if (global_tile) {
-            const int jj = tau * kTileKeys + r;
+            const int jj = tau * kTileKeys + rs;
             int s = tau == 0 ? ((jj < p.k) ? __ldcg(p.topk + (size_t)u * p.k + jj) : -1) : s_next;
             if (s >= 0 && (s > tg || s >= p.N)) {
-                report(p.status, CSA2_ERR_RANGE, u);
+                if (part == 0) report(p.status, CSA2_ERR_RANGE, u);
                 s = -1;
             }
-            valid = s >= 0;
-            if (valid) {
+            if (part == 0) S.rowok[rs] = s >= 0;
+            constexpr int CH = D / 8 / TPR;   // 8-element chunks in this thread's part of a row
+            constexpr int SB = D / 16 / TPR;  // its scale bytes, one per 16-element group
+            if (s >= 0) {
                 const size_t row = (size_t)b * p.N + s;
-                const uint4* cp = reinterpret_cast<const uint4*>(p.kv_fp4 + row * (D / 2));
-                uint4 codes[D / 32];
+                const uint4* cp = reinterpret_cast<const uint4*>(p.kv_fp4 + row * (D / 2) + part * (D / 2 / TPR));
+                uint4 codes[CH / 4];
 #pragma unroll
-                for (int i = 0; i < D / 32; ++i) codes[i] = __ldg(cp + i);
-                uint32_t sw[D / 64];
-                if (D == 128) {
-                    const uint2 s2 = __ldg(reinterpret_cast<const uint2*>(p.kv_scale + row * 8));
-                    sw[0] = s2.x;
-                    sw[1 % (D / 64)] = s2.y;
+                for (int i = 0; i < CH / 4; ++i) codes[i] = __ldg(cp + i);
+                const uint8_t* sp = p.kv_scale + row * (D / 16) + part * SB;
+                uint64_t sw;
+                if constexpr (SB == 8) {
+                    const uint2 s2 = __ldg(reinterpret_cast<const uint2*>(sp));
+                    sw = (uint64_t)s2.x | ((uint64_t)s2.y << 32);
+                } else if constexpr (SB == 4) {
+                    sw = __ldg(reinterpret_cast<const uint32_t*>(sp));
                 } else {
-                    sw[0] = __ldg(reinterpret_cast<const uint32_t*>(p.kv_scale + row * 4));
+                    sw = __ldg(reinterpret_cast<const uint16_t*>(sp));
                 }
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) {           // 8 elements (4 code bytes) per chunk
+                for (int c = 0; c < CH; ++c) {           // 8 elements (4 code bytes) per chunk
                     const uint4 cw = codes[c >> 2];
                     const uint32_t w = (c & 3) == 0 ? cw.x : (c & 3) == 1 ? cw.y : (c & 3) == 2 ? cw.z : cw.w;
-                    const uint32_t g = c >> 1;              // 16-element scale group
-                    const uint32_t sb = (sw[g >> 2] >> (8 * (g & 3))) & 0xFFu;
-                    const uint32_t s16 = e4m3_bf16_bits(sb);
+                    const uint32_t s16 = e4m3_bf16_bits((uint32_t)(sw >> (8 * (c >> 1))) & 0xFFu);
                     const uint32_t s2x = s16 | (s16 << 16);
+                    const uint4 e = e2m1x8_bf16(w);
                     uint4 ov;
-                    ov.x = bf16x2_mul(S.lut[w & 0xFFu], s2x);
-                    ov.y = bf16x2_mul(S.lut[(w >> 8) & 0xFFu], s2x);
-                    ov.z = bf16x2_mul(S.lut[(w >> 16) & 0xFFu], s2x);
-                    ov.w = bf16x2_mul(S.lut[w >> 24], s2x);
-                    *reinterpret_cast<uint4*>(S.kbuf + (c >> 3) * kPanelBytes + sw128(r, c & 7)) = ov;
+                    ov.x = bf16x2_mul(e.x, s2x);
+                    ov.y = bf16x2_mul(e.y, s2x);
+                    ov.z = bf16x2_mul(e.z, s2x);
+                    ov.w = bf16x2_mul(e.w, s2x);
+                    const int cg = part * CH + c;        // the chunk within the row
+                    *reinterpret_cast<uint4*>(S.kbuf + (cg >> 3) * kPanelBytes + sw128(rs, cg & 7)) = ov;
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c)
-                    *reinterpret_cast<uint4*>(S.kbuf + (c >> 3) * kPanelBytes + sw128(r, c & 7)) = make_uint4(0, 0, 0, 0);
+                for (int c = 0; c < CH; ++c) {
+                    const int cg = part * CH + c;
+                    *reinterpret_cast<uint4*>(S.kbuf + (cg >> 3) * kPanelBytes + sw128(rs, cg & 7)) =
+                        make_uint4(0, 0, 0, 0);
+                }
             }
         } else {
             // window rows [lo_w, t], tile lt: coalesced 16-byte loads of K and V
             const int p0 = lo_w + (tau - p.ngt) * kTileKeys;
-            {
-                const int pr = p0 + r;
-                valid = (t >= 0) && (p.W > 0) && (pr <= t);
+            if (tid < kTileKeys) {
+                const int pr = p0 + tid;
+                bool valid = (t >= 0) && (p.W > 0) && (pr <= t);
                 if (valid && (pr - base < 0 || pr - base >= p.Lloc)) {
                     report(p.status, CSA2_ERR_RANGE, u);
                     valid = false;
                 }
+                S.rowok[tid] = valid;
             }
             const uint4* kls = reinterpret_cast<const uint4*>(p.kl);
             const uint4* vls = reinterpret_cast<const uint4*>(p.vl);
             constexpr int CPR = D / 8;                              // 16-byte chunks per row
-            constexpr int ITERS = kTileKeys * CPR / kAttnThreads;   // chunks per thread per tensor
+            constexpr int ITERS = kTileKeys * CPR / NT;    // chunks per thread per tensor
             constexpr int BATCH = ITERS < 8 ? ITERS : 8;            // loads in flight per tensor
 #pragma unroll
             for (int i0 = 0; i0 < ITERS; i0 += BATCH) {
                 uint4 kv[BATCH], vv[BATCH];
 #pragma unroll
                 for (int jb = 0; jb < BATCH; ++jb) {
-                    const int i = tid + (i0 + jb) * kAttnThreads;
+                    const int i = tid + (i0 + jb) * NT;
                     const int rr = i / CPR, c = i % CPR;
                     const int pr = p0 + rr;
                     const int lrow = pr - base;
@@ -1015,7 +1066,7 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
                 }
 #pragma unroll
                 for (int jb = 0; jb < BATCH; ++jb) {
-                    const int i = tid + (i0 + jb) * kAttnThreads;
+                    const int i = tid + (i0 + jb) * NT;
                     const int rr = i / CPR, c = i % CPR;
                     const uint32_t dst = (c >> 3) * kPanelBytes + sw128(rr, c & 7);
                     *reinterpret_cast<uint4*>(S.kbuf + dst) = kv[jb];
@@ -1030,11 +1081,11 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         const int tslot = tau == 0 ? 1 : tau == ntiles - 1 ? 6 : 0;   // phase-trace slots (first, last tile)
         if (tslot) { CSA2_TRACE(tslot); }   // tile staged
         if (tau + 1 < p.ngt) {   // the next tile's list entry, in flight during this tile
-            const int jn = (tau + 1) * kTileKeys + r;
+            const int jn = (tau + 1) * kTileKeys + rs;
             s_next = jn < p.k ? __ldcg(p.topk + (size_t)u * p.k + jn) : -1;
         }
         const uint32_t tmem_s = S.tmem_base, tmem_o = S.tmem_base + HQP;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
 
         // ---- S = K Q^T  (M = 128 keys, N = HQP heads, K = D)
         if (tid == 0 && ok) {
@@ -1053,29 +1104,23 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         if (tslot) { CSA2_TRACE(tslot + 1); }   // S done
 
         // ---- online softmax: the tile's maximum per head, then P and the tile's sums
-        float sv[HQP];
+        float sv[HH];
 #pragma unroll
-        for (int h = 0; h < HQP; ++h) sv[h] = 0.f;
+        for (int h = 0; h < HH; ++h) sv[h] = 0.f;
         if (ok) {
-            float tmp[16];
-#pragma unroll
-            for (int c0 = 0; c0 < HQP; c0 += 16) {
-                tmem_ld16(tmem_s + lane_off + c0, tmp);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) sv[c0 + i] = tmp[i];
-            }
+            tmem_ld_cols<HH>(tmem_s + lane_off + hh0, sv);
+            tmem_ld_wait();
         }
-        const bool rv = valid && ok;
+        const bool rv = ok && S.rowok[rm] != 0;
         {
-            float v[HQP];
+            float v[HH];
 #pragma unroll
-            for (int h = 0; h < HQP; ++h) {
+            for (int h = 0; h < HH; ++h) {
                 sv[h] = rv ? sv[h] * p.scale_log2 : -INFINITY;
                 v[h] = sv[h];
             }
-            const float mx = warp_transpose_reduce<HQP, true>(v);
-            if (HQP == 32 || (lane & 1) == 0) S.red_m[warp][hl] = mx;
+            const float mx = warp_transpose_reduce<HH, true>(v);
+            if (hl_writer) S.red_m[quarter][hl] = mx;
         }
         __syncthreads();
         if (tid < HQP) {   // one thread per head: the new running maximum and the rescale
@@ -1086,16 +1131,16 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         }
         __syncthreads();
         {
-            float pv[HQP];
+            float pv[HH];
 #pragma unroll
-            for (int h = 0; h < HQP; ++h) {
-                const float mn = S.m_run[h];
+            for (int h = 0; h < HH; ++h) {
+                const float mn = S.m_run[hh0 + h];
                 pv[h] = (rv && mn != -INFINITY) ? exp2f(sv[h] - mn) : 0.f;
-                *reinterpret_cast<__nv_bfloat16*>(S.pbuf + (r >> 6) * (HQP * 128) + sw128(h, (r & 63) >> 3) + (r & 7) * 2) =
-                    __float2bfloat16_rn(pv[h]);
+                *reinterpret_cast<__nv_bfloat16*>(S.pbuf + (rm >> 6) * (HQP * 128) + sw128(hh0 + h, (rm & 63) >> 3) +
+                                                  (rm & 7) * 2) = __float2bfloat16_rn(pv[h]);
             }
-            const float l = warp_transpose_reduce<HQP, false>(pv);
-            if (HQP == 32 || (lane & 1) == 0) S.red_l[warp][hl] = l;
+            const float l = warp_transpose_reduce<HH, false>(pv);
+            if (hl_writer) S.red_l[quarter][hl] = l;
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1117,7 +1162,7 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         }
         if (tid < HQP)   // (the thread that owns head tid's running values)
             S.l_run[tid] = S.l_run[tid] * S.cf[tid] + (S.red_l[0][tid] + S.red_l[1][tid]) + (S.red_l[2][tid] + S.red_l[3][tid]);
-        if (tau + 1 < p.ngt && s_next >= 0 && s_next < p.N) {   // the next tile's row towards L1
+        if (tau + 1 < p.ngt && part == 0 && s_next >= 0 && s_next < p.N) {   // the next tile's row towards L1
             const size_t row = (size_t)b * p.N + s_next;
             asm volatile("prefetch.global.L1 [%0];" ::"l"(p.kv_fp4 + row * (D / 2)));
             asm volatile("prefetch.global.L1 [%0];" ::"l"(p.kv_scale + row * (D / 16)));
@@ -1126,28 +1171,29 @@ __global__ void __launch_bounds__(kAttnThreads, HQP == 16 ? 3 : 2)
         tc_fence_after();
         if (tslot) { CSA2_TRACE(tslot + 3); }   // O done
         if (ok) {
-            float tmp[16];
+            float tmp[HH];
+            tmem_ld_cols<HH>(tmem_o + lane_off + hh0, tmp);
+            tmem_ld_wait();
 #pragma unroll
-            for (int c0 = 0; c0 < HQP; c0 += 16) {
-                tmem_ld16(tmem_o + lane_off + c0, tmp);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) o[c0 + i] = o[c0 + i] * S.cf[c0 + i] + tmp[i];
-            }
+            for (int h = 0; h < HH; ++h) o[h] = o[h] * S.cf[hh0 + h] + tmp[h];
         }
         tc_fence_before();
         __syncthreads();   // every read of this tile's buffers, TMEM and sums is done
         if (tslot) { CSA2_TRACE(tslot + 4); }   // tile done
     }
 
-    // ---- out = o / l (thread = head dimension), lse in natural-log units
-    if (tid < D) {
+    // ---- out = o / l (thread = head dimension, its part of the heads), lse in natural-log units
+    {
+        const int dim = quarter * 32 + lane;
+        if (dim < D) {
 #pragma unroll
-        for (int h = 0; h < HQP; ++h) {
-            if (h >= p.Hq) break;
-            const float L = S.l_run[h];
-            p.out[((size_t)u * p.Hq + h) * D + tid] =
-                __bfloat16_as_ushort(__float2bfloat16_rn((ok && L > 0.f) ? o[h] / L : 0.f));
+            for (int h = 0; h < HH; ++h) {
+                const int hg = hh0 + h;
+                if (hg >= p.Hq) break;
+                const float L = S.l_run[hg];
+                p.out[((size_t)u * p.Hq + hg) * D + dim] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn((ok && L > 0.f) ? o[h] / L : 0.f));
+            }
         }
     }
     if (tid < p.Hq && p.lse != nullptr) {
@@ -1218,13 +1264,14 @@ size_t attn_scratch_bytes(const csa2_attn_args& a) { return plan_attn(a).part_by
 
 template <int HQP, int D>
 static cudaError_t launch_seq_variant(const AttnParams& p, int units, cudaStream_t stream) {
-    auto kern = sparse_attn_seq_kernel<HQP, D>;
+    constexpr int NT = seq_threads<HQP>();
+    auto kern = sparse_attn_seq_kernel<HQP, D, NT>;
     const size_t smem = sizeof(AttnSeqSmem<HQP>) + 1024;
     cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(units);
-    cfg.blockDim = dim3(kAttnThreads);
+    cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

@@ -1676,6 +1676,72 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
     return true;
 }
 
+// Reindex with one CTA per query (more queries than SMs): the pool's scores and their
+// level-0 histogram are already in this CTA's shared memory, so the cut runs on them
+// directly (no publishing, no barrier): the bin of the k-th best score, that bin's scores
+// as candidates, the exact threshold and ties, and one ordered write of the pool.
+__device__ __forceinline__ bool reindex_single_unit(const IdxParams& p, IdxSmem& S, const Slot& sl, const UnitCtx& c) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int n = c.my_n;   // valid pool entries (a prefix), all in this CTA
+    const int r = p.r[1];
+    ListCut none{INT_MAX, 0, 0, 0, 0, nullptr, p.status};
+    ListCut cut{INT_MAX, 0, 0, 0, r, p.out[1] + (size_t)c.u * r, p.status};
+    if (tid == 0) S.info[20] = 0;
+    if (n <= r) {
+        cut.all = 1;
+        sel_sync();
+    } else {
+        int h[kBpt], sum = 0;
+#pragma unroll
+        for (int i = 0; i < kBpt; ++i) { h[i] = S.hist0[kBpt * tid + i]; sum += h[i]; }
+        int total;
+        const int excl = sel_scan_excl(sum, S.red, total);
+        int above = total - excl - sum;
+        if (above < r && r <= above + sum) {
+#pragma unroll
+            for (int i = kBpt - 1; i >= 0; --i) {
+                if (above < r && r <= above + h[i]) { S.info[0] = kBpt * tid + i; S.info[1] = above; }
+                above += h[i];
+            }
+        }
+        sel_sync();
+        int blo, bhi;
+        bin0_interval((uint32_t)S.info[0], blo, bhi);
+        const int rrem = r - S.info[1];
+        int* cx = reinterpret_cast<int*>(&S.stage[0][0]);
+        const unsigned below = (1u << lane) - 1u;
+#pragma unroll 4
+        for (int e0 = 0; e0 < n; e0 += kSel) {
+            const int e = e0 + tid;
+            const int x = e < n ? S.sc[e] : 0;
+            const bool in = e < n && x >= blo && x <= bhi;
+            const unsigned b = __ballot_sync(0xffffffffu, in);
+            if (b == 0u) continue;
+            int w = 0;
+            if (lane == 0) w = atomicAdd(&S.info[20], __popc(b));
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (in) cx[w + __popc(b & below)] = x;
+        }
+        sel_sync();
+        const int nx = S.info[20];
+        const int4 ls = local_select2(S.sc, 0, 0, 1, 0, cx, nx, rrem, blo, bhi, histl(S, 0), S.red, S.info);
+        cut.T = ls.z;
+        cut.quota = ls.w;   // the ties at T ranked within the first r
+    }
+    CSA2_TRACE(4);   // threshold found
+    if (n > 0) write_lists<false>(S.sc, n, 0, c.pool, none, cut, S.wsum, row_prefetch(p, c.u));
+    CSA2_TRACE(10);   // list written
+#pragma unroll 1
+    for (int i = min(r, n) + tid; i < r; i += kSel) cut.out[i] = -1;
+    {   // the next level-0 buffer (bins and count) must be zero when the next unit starts
+        int* g0nxt = sl.g0 + ((c.epoch + c.j + 1) % 3) * kG0Stride;
+#pragma unroll 1
+        for (int i = tid; i <= kBins; i += kSel) g0nxt[i] = 0;
+    }
+    sel_sync();
+    return true;
+}
+
 // ------------------------------------------------------------ scoring helpers
 // Score of one key row (DI/16 int4 chunks) against the index query held in
 // shared memory (HI heads of DI bytes, read as broadcasts). Heads at or past
@@ -2409,6 +2475,8 @@ __global__ void __launch_bounds__(kSel, 1)
         UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, pool};
         if (!full && p.local_sel)
             alive = reindex_local_unit(p, S, sl, c, bar_target);
+        else if (!full && p.G == 1 && !spill)
+            alive = reindex_single_unit(p, S, sl, c);
         else
             alive = spill ? select_unit<true>(p, S, sl, c, bar_target, spill)
                           : select_unit<false>(p, S, sl, c, bar_target, S.sc);

@@ -201,3 +201,42 @@ def test_full_decode_skewed_scores(kind, ws, status):
     assert_list_invariants(pool.cpu().numpy(), q_pos, "pool")
     assert_lists_equal(topk, rtopk, f"{kind}: topk")
     assert_lists_equal(pool, rpool, f"{kind}: pool")
+
+
+@pytest.mark.parametrize("kind", ["random", "rising", "equal", "ragged"])
+def test_reindex_one_cta_per_query(kind, ws, status):
+    """Reindex with more queries than SMs: one CTA per query cuts the rescored pool in
+    its own shared memory. Random scores; scores that rise with the position; all-equal
+    scores (the cut is all ties, taken by position); and ragged pools padded with -1,
+    some of them holding fewer entries than k (the whole pool is the list). Every list
+    bit-exact, and every entry taken from the query's pool."""
+    from oracle import cpp as C
+    if kind == "ragged":
+        B, Tq, N, Hi, Di, k, P = 2, 80, 3000, 8, 64, 1024, 4096
+    else:
+        B, Tq, N, Hi, Di, k, P = 1, 160, 40000, 8, 64, 2048, 8192
+    qi, w, ki = inputs(41, B, Tq, N, Hi, Di, False)
+    qi2, w2, ki2 = inputs(43, B, Tq, N, Hi, Di, False)
+    if kind == "rising":
+        qi2[:] = 1
+        ki2[:] = (np.arange(N) * 127 // N).astype(np.int8)[None, :, None]
+    elif kind == "equal":
+        ki2[:] = 0
+    if kind == "ragged":
+        q_pos = np.broadcast_to(np.linspace(200, N - 1, Tq).astype(np.int32), (B, Tq)).copy()
+    else:
+        q_pos = np.broadcast_to(np.arange(N - Tq, N, dtype=np.int32), (B, Tq)).copy()
+    pool, _ = ops.index_topk("FULL", dev(q_pos), dev(qi), w, dev(ki), min(k, P), P, ws=ws, status=status)
+    status.check("full")
+    _, topk = ops.index_topk("REINDEX", dev(q_pos), dev(qi2), w2, dev(ki2), k, pool_in=pool, ws=ws, status=status)
+    status.check(kind)
+    rp = pool.cpu().numpy()
+    ref = C.index_reindex_batch(qi2, w2, ki2, rp, k)
+    got = topk.cpu().numpy()
+    assert_list_invariants(got, q_pos, "reindex topk")
+    assert_lists_equal(topk, ref, f"{kind}: reindex topk")
+    if kind == "ragged":
+        assert (got[..., :3] >= 0).all() and (got[..., -1] == -1).any(), "short pools not reached"
+    for b in range(B):
+        for j in range(Tq):
+            assert set(got[b, j].tolist()) - {-1} <= set(rp[b, j].tolist()), "Reindex list outside the pool"
