@@ -584,7 +584,8 @@ def index_kernel_name(s, mode):
     dispatch rules, restated for the report)."""
     if mode == "FULL":
         if s.Tq >= 4 and s.N >= 8192 and s.Hi <= 8 and s.Di in (32, 64, 128):
-            return f"index_mq_score_kernel<{s.Di}> + index_full_tc_kernel<{s.Di}> (select only)"
+            return (f"index_mq_score_kernel<{s.Di}> (sample, mark) + index_mq_estimate_kernel + "
+                    f"index_mq_select_kernel<{s.Di}> + index_full_tc_kernel<{s.Di}> (queries left over)")
         if s.Di in (32, 64, 128):
             return f"index_full_tc_kernel<{s.Di}>"
     if s.Hi <= 8 and s.Di == 64:
@@ -758,8 +759,9 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ phase trace
 PHASES = {
-    "full_index": {1: "dependency wait", 2: "scan done", 18: "sample (select only)", 19: "estimates (select only)",
-                   20: "candidate pass (select only)", 21: "exact cut (select only)",
+    "full_index": {1: "dependency wait", 2: "scan done", 22: "candidates listed (shared-key cut)",
+                   23: "candidates scored (shared-key cut)", 24: "threshold (shared-key cut)",
+                   25: "lists written (shared-key cut)",
                    3: "histograms exchanged", 4: "threshold bins",
                    5: "ordered lists", 7: "candidates exchanged", 8: "finalise", 12: "candidates loaded",
                    13: "thresholds, counts", 9: "write", 10: "lists written", 11: "end"},
@@ -772,7 +774,7 @@ PHASES = {
                       9: "last O done", 10: "last tile done", 11: "end"},
 }
 KINDS = {1: "index_full_tc_kernel", 2: "index_dp4a_kernel", 3: "sparse_attn_cl_kernel", 4: "sparse_attn_kernel",
-         5: "index_mq_score_kernel", 6: "sparse_attn_seq_kernel"}
+         5: "index_mq_score_kernel", 6: "sparse_attn_seq_kernel", 7: "index_mq_select_kernel"}
 
 
 def run_phase_trace(args):

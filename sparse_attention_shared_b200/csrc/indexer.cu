@@ -77,8 +77,18 @@ struct IdxParams {
     int32_t* spill;      // [groups*G][chunk] scores when chunk > kSmemScores
     int local_sel;       // Reindex: every CTA of the group cuts over all of the unit's scores
     int keys_ready;      // keys and positions were complete before the previous kernel began
-    const int32_t* pre;  // Full, select only: every unit's scores by position ([units][pstride]), else nullptr
-    int64_t pstride;
+    // Full with queries that share keys: the sampled tiles' scores, the estimates, the
+    // candidate words (one bit per position), the candidates one CTA of the cut holds,
+    // and the units it leaves to the Full kernel ([0] count, [1 ..] units)
+    const int32_t* mq_sample;
+    int64_t mq_sstride;
+    int mq_tstep;
+    int4* mq_est;
+    const int32_t* mq_words;
+    int64_t mq_wstride;
+    int mq_cap;
+    int32_t* fb_list;
+    const int32_t* unit_list;   // Full kernel: the units to take ([0] count, [1 ..] units), nullptr: all
     int rstride;         // per-unit stride of rscore
     int32_t* rscore;     // [units][rstride] published scores (local_sel)
     // L2 prefetch of the global cache rows each top-k list selects (pf_fp4 nullptr: off)
@@ -1330,202 +1340,6 @@ __device__ __forceinline__ bool select_unit(const IdxParams& p, IdxSmem& S, cons
     return true;
 }
 
-// ------------------------------------------------------------ select only: sampled threshold
-// The select-only pass of one query by one CTA, its scores in global memory (more than
-// shared memory holds). A sample of at most 4096 scores (runs of 4 positions, every s-th
-// run) gives each track a threshold estimate: the sample's value at 1.2 times the rank
-// the track's cut would have in the sample, plus 16. One ordered pass keeps every score at or above
-// the lower estimate as a candidate (position order, a list per warp over its range
-// of positions) and counts the scores at or above each track's estimate. When every
-// track has at least its rank r there, all of its r best scores are candidates, and
-// the exact threshold, the ties to take and the ordered write run over the candidates
-// alone. Otherwise (a list overflowed or an estimate was too high) nothing is written
-// and the caller runs the full select.
-constexpr int kSampleMax = 4096;
-constexpr int kCandPerWarp = (kStages * kStageBytes) / (8 * kSelWarps);   // int2 entries per warp list (1024)
-
-__device__ __noinline__ bool sampled_select(const IdxParams& p, IdxSmem& S, const Slot& sl, int u, int j, int epoch,
-                                            const int* src, int n) {
-    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
-    const unsigned below = (1u << lane) - 1u;
-    int r[2], act[2];
-#pragma unroll
-    for (int tr = 0; tr < 2; ++tr) {
-        r[tr] = p.r[tr];
-        act[tr] = r[tr] > 0 && r[tr] < n;
-        if (r[tr] > 0 && !act[tr]) return false;   // a track that takes every score: the full select
-    }
-    if (!act[0] && !act[1]) return false;
-
-    // ---- sample (runs of 4 positions: one 16-byte load each) and estimates
-    const int nruns = n >> 2;   // whole runs (n > r >= 1; a shorter tail is not sampled)
-    const int s = max(1, (nruns + kSampleMax / 4 - 1) / (kSampleMax / 4)), mr = nruns / s, m = 4 * mr;
-    int smin = INT_MAX, smax = INT_MIN;
-#pragma unroll
-    for (int q = 0; q < kSampleMax / 4 / kSel; ++q) {
-        const int i = q * kSel + tid;
-        if (i < mr) {
-            const int4 v = __ldcg(reinterpret_cast<const int4*>(src) + (size_t)i * s);
-            reinterpret_cast<int4*>(S.sc)[i] = v;
-            smin = min(min(smin, min(v.x, v.y)), min(v.z, v.w));
-            smax = max(max(smax, max(v.x, v.y)), max(v.z, v.w));
-        }
-    }
-    if (m == 0) return false;
-    // the sample's range, so that the radix passes below spread over it
-    smin = __reduce_min_sync(0xffffffffu, smin);
-    smax = __reduce_max_sync(0xffffffffu, smax);
-    if (tid == 0) { S.info[26] = INT_MAX; S.info[27] = INT_MIN; S.info[28] = INT_MIN; }
-    sel_sync();
-    if (lane == 0) { atomicMin(&S.info[26], smin); atomicMax(&S.info[27], smax); }
-    sel_sync();
-    smin = S.info[26];
-    smax = S.info[27];
-    CSA2_TRACE(18);   // sampled select: sample loaded
-    int qr[2];
-#pragma unroll
-    for (int tr = 0; tr < 2; ++tr)
-        qr[tr] = act[tr] ? min(m, (int)((long long)r[tr] * m / n * 6 / 5) + 16) : 0;
-    const int4 est = local_select2(S.sc, act[0] ? m : 0, qr[0], smin, smax, S.sc, act[1] ? m : 0, qr[1],
-                                   smin, smax, S.hist0, S.red, S.info);
-    const int te0 = act[0] ? est.x : INT_MAX, te1 = act[1] ? est.z : INT_MAX;
-    const int tlo = min(te0, te1);
-    CSA2_TRACE(19);   // sampled select: estimates
-
-    // ---- one ordered pass: candidates >= tlo, counts >= each estimate
-    int2* lists = reinterpret_cast<int2*>(&S.stage[0][0]);
-    int2* list = lists + wp * kCandPerWarp;
-    const int nstep = (n + 127) >> 7, spw = (nstep + kSelWarps - 1) / kSelWarps;
-    const int s0 = min(nstep, wp * spw), s1 = min(nstep, s0 + spw);
-    int ln = 0, c0 = 0, c1 = 0, cmax = INT_MIN;
-    constexpr int kIn = 8;
-#pragma unroll 1
-    for (int st0 = s0; st0 < s1; st0 += kIn) {
-        int4 xv[kIn];
-#pragma unroll
-        for (int q = 0; q < kIn; ++q) {
-            const int e = (st0 + q) * 128 + 4 * lane;   // rows are padded to 4 elements
-            xv[q] = (st0 + q < s1 && e < n) ? __ldcg(reinterpret_cast<const int4*>(src + e)) : make_int4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int q = 0; q < kIn; ++q) {
-            if (st0 + q >= s1) break;   // warp-uniform
-            const int e0 = (st0 + q) * 128 + 4 * lane;
-            const int x[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
-            bool f[4];
-            unsigned b[4];
-            int pre = 0;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const bool ok = e0 + k < n;
-                f[k] = ok && x[k] >= tlo;
-                if (f[k]) cmax = max(cmax, x[k]);
-                c0 += ok && x[k] >= te0;
-                c1 += ok && x[k] >= te1;
-                b[k] = __ballot_sync(0xffffffffu, f[k]);
-                pre += __popc(b[k] & below);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                if (f[k] && ln + pre < kCandPerWarp) list[ln + pre] = make_int2(x[k], e0 + k);
-                pre += f[k] ? 1 : 0;
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) ln += __popc(b[k]);
-        }
-    }
-    if (tid == 0) S.info[24] = 0;
-    sel_sync();
-    cmax = __reduce_max_sync(0xffffffffu, cmax);
-    if (lane == 0) {
-        S.wlist_n[wp] = min(ln, kCandPerWarp);
-        if (ln > kCandPerWarp) S.info[24] = 1;
-        atomicMax(&S.info[28], cmax);   // the candidates' largest score: the exact cut's range
-    }
-    int4 ca = make_int4(c0, c1, 0, 0), cb = make_int4(0, 0, 0, 0);
-    sel_total8(ca, cb, S.red);   // (its barriers also publish wlist_n and the overflow flag)
-    CSA2_TRACE(20);   // sampled select: candidate pass
-    if (S.info[24] != 0 || (act[0] && ca.x < r[0]) || (act[1] && ca.y < r[1])) {
-        sel_sync();
-        return false;
-    }
-
-    // ---- the candidates' scores, contiguous, and the exact cut of each track
-    int base = 0, total = 0;
-#pragma unroll 1
-    for (int w = 0; w < kSelWarps; ++w) {
-        base += w < wp ? S.wlist_n[w] : 0;
-        total += S.wlist_n[w];
-    }
-    const int mine = S.wlist_n[wp];
-#pragma unroll 1
-    for (int i = lane; i < mine; i += 32) S.sc[base + i] = list[i].x;
-    sel_sync();
-    const int chi = S.info[28];
-    const int4 ls = local_select2(S.sc, act[0] ? total : 0, r[0], tlo, chi, S.sc, act[1] ? total : 0, r[1],
-                                  tlo, chi, S.hist0, S.red, S.info);
-    CSA2_TRACE(21);   // sampled select: exact cut
-    ListCut cut[2];
-#pragma unroll
-    for (int tr = 0; tr < 2; ++tr) {
-        cut[tr].T = tr == 0 ? ls.x : ls.z;
-        cut[tr].quota = tr == 0 ? ls.y : ls.w;   // the ties at T ranked within the first r
-        cut[tr].all = 0;
-        cut[tr].base = 0;
-        cut[tr].r = r[tr];
-        cut[tr].out = act[tr] ? p.out[tr] + (size_t)u * r[tr] : nullptr;
-        cut[tr].status = p.status;
-    }
-
-    // ---- ordered write from the lists: counts per warp, then ranks within 32-entry steps
-    const RowPrefetch pf = row_prefetch(p, u);
-    int4 cnt = make_int4(0, 0, 0, 0);   // gt0, eq0, gt1, eq1
-#pragma unroll 1
-    for (int i = lane; i < mine; i += 32) {
-        const int x = list[i].x;
-        cnt.x += cut[0].out && x > cut[0].T;
-        cnt.y += cut[0].out && x == cut[0].T;
-        cnt.z += cut[1].out && x > cut[1].T;
-        cnt.w += cut[1].out && x == cut[1].T;
-    }
-    cnt = warp_sum4(cnt);
-    int4* w4 = reinterpret_cast<int4*>(S.wsum);
-    if (lane == 0) w4[wp] = cnt;
-    sel_sync();
-    int rg0 = 0, re0 = 0, rg1 = 0, re1 = 0;
-#pragma unroll 1
-    for (int w = 0; w < wp; ++w) {
-        const int4 a = w4[w];
-        rg0 += a.x; re0 += a.y; rg1 += a.z; re1 += a.w;
-    }
-#pragma unroll 1
-    for (int i0 = 0; i0 < mine; i0 += 32) {
-        const int i = i0 + lane;
-        const int2 ent = i < mine ? list[i] : make_int2(0, 0);
-        const bool g0 = i < mine && cut[0].out && ent.x > cut[0].T, q0 = i < mine && cut[0].out && ent.x == cut[0].T;
-        const bool g1 = i < mine && cut[1].out && ent.x > cut[1].T, q1 = i < mine && cut[1].out && ent.x == cut[1].T;
-        const unsigned bg0 = __ballot_sync(0xffffffffu, g0), bq0 = __ballot_sync(0xffffffffu, q0);
-        const unsigned bg1 = __ballot_sync(0xffffffffu, g1), bq1 = __ballot_sync(0xffffffffu, q1);
-        const int og0 = rg0 + __popc(bg0 & below), oq0 = re0 + __popc(bq0 & below);
-        const int og1 = rg1 + __popc(bg1 & below), oq1 = re1 + __popc(bq1 & below);
-        if (g0 || (q0 && oq0 < cut[0].quota)) {
-            const int k = og0 + min(oq0, cut[0].quota);
-            if (CSA2_GUARD((unsigned)k < (unsigned)r[0], p.status, 2203)) { cut[0].out[k] = ent.y; prefetch_key(pf, ent.y); }
-        }
-        if (g1 || (q1 && oq1 < cut[1].quota)) {
-            const int k = og1 + min(oq1, cut[1].quota);
-            if (CSA2_GUARD((unsigned)k < (unsigned)r[1], p.status, 2204)) { cut[1].out[k] = ent.y; prefetch_row(pf, ent.y); }
-        }
-        rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
-    }
-    // the next unit's level-0 buffer (bins and count) must be zero when it starts
-    int* g0nxt = sl.g0 + ((epoch + j + 1) % 3) * kG0Stride;
-#pragma unroll 1
-    for (int i = tid; i <= kBins; i += kSel) g0nxt[i] = 0;
-    sel_sync();
-    return true;
-}
-
 // ------------------------------------------------------------ Reindex: one select per group
 // A Reindex pool fits in one CTA's shared memory, so the group does not run the
 // distributed select: every CTA publishes its scores (element order), its element
@@ -1855,7 +1669,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int group = blockIdx.x / p.G;
     const int cta = blockIdx.x % p.G;
     const Slot sl = slot_of(p, group);
-    int* spill = (p.chunk > kSmemScores && p.pre == nullptr) ? p.spill + (size_t)blockIdx.x * p.chunk : nullptr;
+    int* spill = (p.chunk > kSmemScores) ? p.spill + (size_t)blockIdx.x * p.chunk : nullptr;
     constexpr int kRows = (kStageBytes / DI) < 256 ? (kStageBytes / DI) : 256;   // rows per tile
     constexpr int kBlocks = kRows / 128;                                          // MMA row blocks per tile
     constexpr uint32_t kSwz = DI == 32 ? 6u : DI == 64 ? 4u : 2u;
@@ -1884,8 +1698,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tmem = S.tmem_base;
     uint32_t seq = 0;   // tiles processed by this CTA so far (same count in every role)
 
+    // every unit, or the ones a list names (the queries the shared-key cut left over)
+    const int nlist = p.unit_list ? __ldcg(p.unit_list) : p.units;
     int j = 0;
-    for (int u = group; u < p.units; u += p.groups, ++j) {
+    for (int i = group; i < nlist; i += p.groups, ++j) {
+        const int u = p.unit_list ? __ldcg(p.unit_list + 1 + i) : i;
         const int b = u / p.Tq;
         int t = p.q_pos[u];
         int tg = last_entry(t, p.m);   // the last global entry the query reads
@@ -1897,7 +1714,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int n_all = tg + 1;
         const int lo = min(cta * p.chunk, n_all);
         const int my_n = min(lo + p.chunk, n_all) - lo;
-        const int nst = p.pre ? 0 : (my_n + kRows - 1) / kRows;   // select only: no key tiles
+        const int nst = (my_n + kRows - 1) / kRows;
 
         // index query -> B operand (16 rows: heads, zero past Hi); zero the histogram. The
         // TMA warp takes no part: it starts streaming keys at once, and the others meet on
@@ -1999,62 +1816,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         CSA2_TRACE(2);   // scan done
         if (S.abort) break;
 
-        // select only: the unit's scores come from the multi-query scoring kernel; the
-        // chunk goes to shared memory when it fits, and its histogram is built here
-        const int* src = p.pre ? p.pre + (size_t)u * p.pstride + lo : nullptr;
-        if (src && p.G == 1 && p.chunk > kSmemScores) {
-            // one CTA per query, scores in global memory: the sampled select first
-            if (tid < kSel) {
-                const bool done = sampled_select(p, S, sl, u, j, epoch, src, my_n);
-                if (tid == 0) S.info[25] = done ? 1 : 0;
-            }
-            __syncthreads();
-            if (S.info[25]) {
-                __syncthreads();   // (S.info is reused by the next unit)
-                continue;
-            }
-            for (int i = tid; i < kBins; i += kTcThreads) S.hist0[i] = 0;   // it used the histogram as scratch
-            __syncthreads();
-        }
-        if (src) {
-            // 16-byte loads, eight in flight per thread (the unit's row and the chunk
-            // start are multiples of 4 elements): each round is one L2 round trip
-            constexpr int kIn = 8;
-            const bool to_smem = p.chunk <= kSmemScores;
-            const int nv = my_n >> 2;
-            const int4* src4 = reinterpret_cast<const int4*>(src);
-#pragma unroll 1
-            for (int v0 = tid; v0 < nv; v0 += kIn * kTcThreads) {
-                int4 x4[kIn];
-#pragma unroll
-                for (int q = 0; q < kIn; ++q) {
-                    const int v = v0 + q * kTcThreads;
-                    x4[q] = v < nv ? __ldcg(src4 + v) : make_int4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int q = 0; q < kIn; ++q) {
-                    const int v = v0 + q * kTcThreads;
-                    if (v >= nv) continue;
-                    if (to_smem) reinterpret_cast<int4*>(S.sc)[v] = x4[q];
-                    atomicAdd(&S.hist0[bin0(x4[q].x)], 1);
-                    atomicAdd(&S.hist0[bin0(x4[q].y)], 1);
-                    atomicAdd(&S.hist0[bin0(x4[q].z)], 1);
-                    atomicAdd(&S.hist0[bin0(x4[q].w)], 1);
-                }
-            }
-            for (int e = 4 * nv + tid; e < my_n; e += kTcThreads) {
-                const int x = __ldcg(src + e);
-                if (to_smem) S.sc[e] = x;
-                atomicAdd(&S.hist0[bin0(x)], 1);
-            }
-            __syncthreads();
-        }
-        const int* sel_src = src ? (p.chunk > kSmemScores ? src : nullptr) : spill;
-
         if (tid < kSel) {
             UnitCtx c{u, t, lo, my_n, n_all, cta, j, epoch, nullptr};
-            const bool ok = sel_src ? select_unit<true>(p, S, sl, c, bar_target, sel_src)
-                                    : select_unit<false>(p, S, sl, c, bar_target, S.sc);
+            const bool ok = spill ? select_unit<true>(p, S, sl, c, bar_target, spill)
+                                  : select_unit<false>(p, S, sl, c, bar_target, S.sc);
             if (!ok && tid == 0) S.abort = 1;
         }
         __syncthreads();
@@ -2076,9 +1841,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // block of up to kMqQ queries of a sequence and a range of 128-row key tiles. One
 // kind::i8 MMA per 32-byte K step scores a tile against all of the block's queries:
 // B row 8q + h holds query q's head h (zero past Hi or past the block), so N = 8 kMqQ,
-// and each key tile is read once per block instead of once per query. The epilogue
-// writes each query's scores, for the positions up to its own, to a per-unit array
-// that the Full kernel then cuts in its select-only mode.
+// and each key tile is read once per block instead of once per query. No query's
+// scores are kept in full. The call runs in four steps:
+//   1. sample (this kernel, kMqSample): every tstep-th tile only; each query's scores
+//      there, up to its own position, go to a compact per-unit sample;
+//   2. estimate (index_mq_estimate_kernel): per query and track, a threshold estimate
+//      from the sample, the sample's value at 1.2 times the rank the track's cut would
+//      have in it, plus 16; tlo is the lower of the two;
+//   3. mark (this kernel, kMqMark): every tile; per query, a bit per position for the
+//      scores at or above tlo (the candidates), one 32-bit word per 32 positions;
+//   4. cut (index_mq_select_kernel): per query, the candidates' positions in order,
+//      their scores recomputed from the keys, a check that each track has at least r
+//      candidates at or above its estimate (then its r best scores and every tie at
+//      its threshold are candidates), the exact cut and the ordered write. A query
+//      that fails the check, or has more candidates than shared memory holds, is
+//      listed for the cooperative Full kernel, which scans and cuts it in full.
 constexpr int kMqQ = 16;                                  // queries per block
 constexpr int kMqN = kMqQ * 8;                            // MMA N
 constexpr int kMqRows = 128;                              // key rows per tile (one M = 128 block)
@@ -2089,14 +1866,18 @@ constexpr int kMqThreads = (kMqGroups * 4 + 2) * 32;      // + the TMA and MMA w
 constexpr int kMqMin = 4;                                 // Tq from which a Full call takes this path
 constexpr int kMqMinN = 8192;                             // ... on a key set of at least this many positions
 
+enum { kMqSample = 0, kMqMark = 1 };
+
 struct MqParams {
     int B, Tq, N, Hi, nblk, splits;
     int m;               // sequence compression rate of the global entries
     int32_t w[8];
     const int32_t* q_pos;
     const int8_t* qi;
-    int32_t* scores;     // [B*Tq][sstride]
-    int64_t sstride;
+    int32_t* out;        // sample: [B*Tq][ostride] scores; mark: [B*Tq][ostride] candidate words
+    int64_t ostride;
+    int tstep;           // sample: every tstep-th key tile (mark: 1)
+    const int4* est;     // mark: per unit {tlo, te0, te1, tracks}
     int32_t* status;
 };
 
@@ -2106,6 +1887,7 @@ struct __align__(1024) MqSmem {
     uint8_t qb[kMqN * DI];               // the block's index queries as the B operand
     uint64_t full_bar[kMqStages], empty_bar[kMqStages], tfull_bar[kMqBufs], tempty_bar[kMqBufs];
     int tq[kMqQ];
+    int tlo[kMqQ];
     int tile_lo, tile_hi;
     uint32_t tmem_base;
 };
@@ -2118,7 +1900,7 @@ __device__ __forceinline__ void tmem_ld16i(uint32_t taddr, int (&v)[16]) {
         : "r"(taddr));
 }
 
-template <int DI>
+template <int DI, int MODE>
 __global__ void __launch_bounds__(kMqThreads, 1)
     index_mq_score_kernel(const __grid_constant__ MqParams p, const __grid_constant__ CUtensorMap kmap) {
     CSA2_TRACE_INIT();
@@ -2152,9 +1934,10 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         if (tid < nq) {
             t = p.q_pos[(size_t)b * p.Tq + j0 + tid];
             const int tg = last_entry(t, p.m);
-            t = (t < 0 || tg >= p.N) ? -1 : tg;   // no scores past the last entry; the select kernel reports a bad position
+            t = (t < 0 || tg >= p.N) ? -1 : tg;   // no scores past the last entry; the cut reports a bad position
         }
         S.tq[tid] = t;
+        if (MODE == kMqMark) S.tlo[tid] = tid < nq ? p.est[(size_t)b * p.Tq + j0 + tid].x : INT_MAX;
     }
     fence_proxy_async_smem();
     for (int i = tid; i < kMqN * (DI / 16); i += kMqThreads) {
@@ -2170,7 +1953,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
     if (tid == 0) {   // this split's share of the tiles that cover [0, the block's last position]
         int tmax = -1;
         for (int q = 0; q < kMqQ; ++q) tmax = max(tmax, S.tq[q]);
-        const int ntile = (tmax + kMqRows) / kMqRows;
+        const int ntile = ((tmax + kMqRows) / kMqRows + p.tstep - 1) / p.tstep;   // (sample: the sampled tiles)
         S.tile_lo = (int)((long long)ntile * split / p.splits);
         S.tile_hi = (int)((long long)ntile * (split + 1) / p.splits);
     }
@@ -2185,7 +1968,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                 const int slot = i % kMqStages;
                 if (i >= kMqStages && !mbar_wait(&S.empty_bar[slot], ((i / kMqStages) - 1) & 1u, p.status, 21)) break;
                 mbar_arrive_expect_tx(&S.full_bar[slot], (uint32_t)(kMqRows * DI));
-                tma_load_keys(S.stage[slot], &kmap, 0, (tile_lo + i) * kMqRows, b, &S.full_bar[slot], pol);
+                tma_load_keys(S.stage[slot], &kmap, 0, (tile_lo + i) * p.tstep * kMqRows, b, &S.full_bar[slot], pol);
             }
         }
     } else if (warp == kEpiWarps + 1) {
@@ -2238,16 +2021,302 @@ __global__ void __launch_bounds__(kMqThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.tempty_bar[buf]);
-            const int s = (tile_lo + i) * kMqRows + wl * 32 + lane;
+            const int kt = (tile_lo + i) * p.tstep;            // the key tile
+            const int s = kt * kMqRows + wl * 32 + lane;       // this lane's position
+            if (MODE == kMqSample) {
+                // sample entry (tile ordinal) * 128 + row, for the positions up to the query's own
+                const int e = (tile_lo + i) * kMqRows + wl * 32 + lane;
 #pragma unroll
-            for (int q = 0; q < kMqQ; ++q)
-                if (s <= tq[q]) p.scores[((size_t)b * p.Tq + j0 + q) * p.sstride + s] = x[q];
+                for (int q = 0; q < kMqQ; ++q)
+                    if (s <= tq[q]) p.out[((size_t)b * p.Tq + j0 + q) * p.ostride + e] = x[q];
+            } else {
+                // candidate word of each query for these 32 positions; lane q stores query q's
+                unsigned mine = 0u;
+#pragma unroll
+                for (int q = 0; q < kMqQ; ++q) {
+                    const unsigned m = __ballot_sync(0xffffffffu, s <= tq[q] && x[q] >= S.tlo[q]);
+                    if (lane == q) mine = m;
+                }
+                if (lane < nq)
+                    p.out[((size_t)b * p.Tq + j0 + lane) * p.ostride + kt * 4 + wl] = (int32_t)mine;
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kMqBufs * kMqN);
     CSA2_TRACE_END(5);
+}
+
+// ------------------------------------------------------------ shared keys: estimates and the cut
+constexpr int kMqSampleMax = 16384;  // sample entries per query (at most 128 sampled tiles)
+constexpr int kMqCap = 16384;        // candidates per query that the cut holds
+
+size_t mq_estimate_smem_bytes(int sstride) { return (size_t)(sstride + 1088 + 8 * kSelWarps + 64) * 4; }
+
+// Step 2: one CTA per query. The sampled tiles' entries up to the query's position form a
+// prefix of its sample (a sampled tile is whole or the last one); the estimate of each
+// track with 0 < r < n is the sample's value at rank min(m, r m / n * 1.2 + 16).
+__global__ void __launch_bounds__(kSel, 2) index_mq_estimate_kernel(const __grid_constant__ IdxParams p) {
+    extern __shared__ __align__(16) int sme[];
+    struct {
+        int* sc;     // [sstride] the sample
+        int* hist;   // [1088]
+        int* red;    // [8 * kSelWarps]
+        int* info;   // [64]
+    } S{sme, sme + p.mq_sstride, sme + p.mq_sstride + 1088, sme + p.mq_sstride + 1088 + 8 * kSelWarps};
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int u = blockIdx.x;
+    pdl_launch_dependents();
+    pdl_wait();
+    if (u == 0 && tid == 0) p.fb_list[0] = 0;   // the call's fallback list starts empty
+    const int t = p.q_pos[u], tg = last_entry(t, p.m);
+    const int n = (t < 0 || tg >= p.N) ? 0 : tg + 1;
+    int act[2];
+#pragma unroll
+    for (int tr = 0; tr < 2; ++tr) act[tr] = p.r[tr] > 0 && p.r[tr] < n;
+    int4 e = make_int4(INT_MAX, INT_MAX, INT_MAX, 0);
+    if (act[0] || act[1]) {
+        const int span = p.mq_tstep * kMqRows;
+        int m = 0;
+        for (int j = 0; j * span <= tg && j * kMqRows < p.mq_sstride; ++j) m += min(kMqRows, tg - j * span + 1);
+        const int32_t* src = p.mq_sample + (size_t)u * p.mq_sstride;
+        int smin = INT_MAX, smax = INT_MIN;
+        for (int i = tid; i < m; i += kSel) {
+            const int x = __ldcg(src + i);
+            S.sc[i] = x;
+            smin = min(smin, x);
+            smax = max(smax, x);
+        }
+        smin = __reduce_min_sync(0xffffffffu, smin);
+        smax = __reduce_max_sync(0xffffffffu, smax);
+        if (tid == 0) { S.info[26] = INT_MAX; S.info[27] = INT_MIN; }
+        sel_sync();
+        if (lane == 0) { atomicMin(&S.info[26], smin); atomicMax(&S.info[27], smax); }
+        sel_sync();
+        smin = S.info[26];
+        smax = S.info[27];
+        int qr[2];
+#pragma unroll
+        for (int tr = 0; tr < 2; ++tr)
+            qr[tr] = act[tr] ? min(m, (int)((long long)p.r[tr] * m / n * 6 / 5) + 16) : 0;
+        const int4 est = local_select2(S.sc, act[0] ? m : 0, qr[0], smin, smax, S.sc, act[1] ? m : 0, qr[1], smin,
+                                       smax, S.hist, S.red, S.info);
+        const int te0 = act[0] ? est.x : INT_MAX, te1 = act[1] ? est.z : INT_MAX;
+        e = make_int4(min(te0, te1), te0, te1, act[0] | (act[1] << 1));
+    }
+    if (tid == 0) p.mq_est[u] = e;
+}
+
+// Step 4: one CTA per query. Shared memory (1024-aligned): kMqRB row blocks of gathered
+// key rows and the index query as tensor-core operands, [cap] positions and [cap] scores
+// (cap from the launch), the histogram, reduction and count scratch, the barrier and
+// the TMEM address.
+template <int DI> constexpr int mq_rb() { return DI == 128 ? 4 : 8; }   // 128-row blocks per batch
+
+template <int DI>
+__global__ void __launch_bounds__(kSel, 1) index_mq_select_kernel(const __grid_constant__ IdxParams p) {
+    extern __shared__ __align__(1024) uint8_t smq_raw[];
+    uint8_t* sbase = smq_raw + ((1024u - (smem_u32(smq_raw) & 1023u)) & 1023u);
+    constexpr int kRB = mq_rb<DI>();
+    const int cap = p.mq_cap;
+    uint8_t* stage = sbase;                                   // [kRB][128 rows][DI], TMA-tile layout
+    uint8_t* qtc = stage + kRB * 128 * DI;                    // [16 rows][DI]: heads, zero past Hi
+    int* cpos = reinterpret_cast<int*>(qtc + (16 * DI > 1024 ? 16 * DI : 1024));
+    int* csc = cpos + cap;
+    int* hist = csc + cap;
+    int* red = hist + 1088;
+    int* info = red + 8 * kSelWarps;
+    int* wsum = info + 64;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(wsum + 4 * kSelWarps);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int u = blockIdx.x, b = u / p.Tq;
+    CSA2_TRACE_INIT();
+    pdl_launch_dependents();
+    pdl_wait();
+    const int t = p.q_pos[u], tg = last_entry(t, p.m);
+    const bool bad = t < 0 || tg >= p.N;
+    if (bad && tid == 0) report(p.status, CSA2_ERR_RANGE, u);
+    const int n = bad ? 0 : tg + 1;
+    // a track with r >= n takes every entry in order (none at a bad position), then -1
+#pragma unroll
+    for (int tr = 0; tr < 2; ++tr) {
+        const int r = p.r[tr];
+        if (r > 0 && r >= n) {
+            int32_t* out = p.out[tr] + (size_t)u * r;
+            for (int i = tid; i < r; i += kSel) out[i] = i < n ? i : -1;
+        }
+    }
+    const int4 e = p.mq_est[u];
+    const bool act0 = (e.w & 1) != 0, act1 = (e.w & 2) != 0;
+    if (!act0 && !act1) { CSA2_TRACE_END(7); return; }
+
+    // ---- the candidates' positions in order: warp w takes the words [w W, (w + 1) W), its
+    // lanes read 32 consecutive words at a time; counted, scanned over the warps, expanded
+    const int nw = (n + 31) >> 5;
+    const int wpw = (nw + kSelWarps * 32 - 1) / (kSelWarps * 32) * 32;   // words per warp
+    const int ww0 = min(nw, (tid >> 5) * wpw), ww1 = min(nw, ww0 + wpw);
+    const int32_t* words = p.mq_words + (size_t)u * p.mq_wstride;
+    auto word_at = [&](int w) -> unsigned {
+        if (w >= ww1) return 0u;
+        unsigned m = (unsigned)__ldcg(words + w);
+        const int valid = n - 32 * w;   // positions of this word up to the query's own
+        return valid >= 32 ? m : (m & ((1u << valid) - 1u));
+    };
+    int cnt = 0;
+#pragma unroll 4
+    for (int w = ww0 + lane; w < ww1; w += 32) cnt += __popc(word_at(w));
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    int total;
+    int off = sel_scan_excl(lane == 0 ? cnt : 0, red, total);   // the warp's first slot
+    off = __shfl_sync(0xffffffffu, off, 0);
+    CSA2_TRACE(22);   // candidates counted
+    bool fail = total > cap;
+    if (!fail) {
+        for (int w0 = ww0; w0 < ww1; w0 += 32) {
+            unsigned m = word_at(w0 + lane);
+            const int c = __popc(m);
+            int incl = c;   // inclusive scan of the counts over the lanes
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int k = off + incl - c;
+            while (m) {
+                const int bit = __ffs(m) - 1;
+                m &= m - 1u;
+                cpos[k++] = 32 * (w0 + lane) + bit;
+            }
+            off += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        // the index query as the B operand (16 rows: heads, zero past Hi), the barrier, TMEM
+        for (int i = tid; i < 16 * DI / 16; i += kSel) {
+            const int h = i / (DI / 16), c2 = i % (DI / 16);
+            int4 v = make_int4(0, 0, 0, 0);
+            if (h < p.Hi) v = reinterpret_cast<const int4*>(p.qi + ((size_t)u * p.Hi + h) * DI)[c2];
+            *reinterpret_cast<int4*>(qtc + tile_off(h, c2, DI)) = v;
+        }
+        if (tid == 0) {
+            mbar_init(bar, 1);
+            mbar_fence_init();
+        }
+        if (warp == 0) tmem_alloc(tmem_slot, 16 * kRB);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        sel_sync();
+        tc_fence_after();
+        const uint32_t tmem = *tmem_slot;
+        // ---- the candidates' scores on the tensor cores, kRB blocks of 128 rows a batch:
+        // the rows are gathered into operand tiles (DI / 16 threads per row, 16 bytes each),
+        // one kind::i8 MMA per block and 32-byte K step (N = 16), then warp w reads TMEM lane
+        // quarter w % 4 of blocks w / 4 and w / 4 + 4
+        constexpr uint32_t kSwz = DI == 32 ? 6u : DI == 64 ? 4u : 2u;
+        constexpr uint32_t kSbo = 8 * DI;
+        constexpr uint32_t kIdesc = idesc_i8(128, 16);
+        constexpr int CPR = DI / 16, CPT = kRB * 128 * CPR / kSel;   // chunks per row, per thread
+        const int8_t* kb = p.ki + (size_t)b * p.ki_seq_stride;
+        int c0 = 0, c1 = 0, cmax = INT_MIN;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int base = 0; base < total && ok; base += kRB * 128) {
+            const int nblk = min(kRB, (total - base + 127) / 128);
+            int4 v[CPT];
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) {
+                const int ci = tid + k * kSel, r = ci / CPR, g = base + r;
+                v[k] = g < total ? __ldg(reinterpret_cast<const int4*>(kb + (size_t)cpos[g] * DI) + ci % CPR)
+                                 : make_int4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) {
+                const int ci = tid + k * kSel, r = ci / CPR;
+                *reinterpret_cast<int4*>(stage + (r >> 7) * 128 * DI + tile_off(r & 127, ci % CPR, DI)) = v[k];
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            sel_sync();
+            tc_fence_after();
+            if (tid == 0) {
+                const uint32_t a0 = smem_u32(stage), b0 = smem_u32(qtc);
+                for (int blk = 0; blk < nblk; ++blk)
+#pragma unroll
+                    for (int kk = 0; kk < DI / 32; ++kk)
+                        mma_i8(tmem + blk * 16, smem_desc(a0 + blk * 128 * DI + kk * 32, 16, kSbo, kSwz),
+                               smem_desc(b0 + kk * 32, 16, kSbo, kSwz), kIdesc, kk > 0 ? 1u : 0u);
+                mma_commit(bar);
+            }
+            ok = sel_and(mbar_wait(bar, phase, p.status, 31) ? 1 : 0) != 0;   // (the same in every thread)
+            phase ^= 1u;
+            tc_fence_after();
+#pragma unroll
+            for (int bb = 0; bb < kRB; bb += 4) {
+                const int blk = warp / 4 + bb;
+                if (blk < nblk && ok) {   // (warp-uniform)
+                    int acc[8];
+                    tmem_ld8(tmem + blk * 16 + ((uint32_t)(warp & 3) * 32u << 16), acc);
+                    tmem_ld_wait();
+                    int x = 0;
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) x += p.w[h] * max(acc[h], 0);
+                    const int g = base + blk * 128 + (warp & 3) * 32 + lane;
+                    if (g < total) {
+                        csc[g] = x;
+                        c0 += x >= e.y;
+                        c1 += x >= e.z;
+                        cmax = max(cmax, x);
+                    }
+                }
+            }
+            tc_fence_before();
+            sel_sync();   // the tiles and TMEM are free for the next batch
+        }
+        tc_fence_after();
+        if (warp == 0) tmem_dealloc(tmem, 16 * kRB);
+        fail = !ok;
+        cmax = __reduce_max_sync(0xffffffffu, cmax);
+        if (tid == 0) info[28] = INT_MIN;
+        int4 ca = make_int4(c0, c1, 0, 0), cb = make_int4(0, 0, 0, 0);
+        sel_total8(ca, cb, red);   // (its first barrier also orders info[28] before the maxima below)
+        if (lane == 0) atomicMax(&info[28], cmax);
+        sel_sync();
+        cmax = info[28];
+        CSA2_TRACE(23);   // candidates scored
+        // every track needs r candidates at or above its estimate: then its r best scores
+        // and all ties at its threshold are candidates
+        fail = fail || (act0 && ca.x < p.r[0]) || (act1 && ca.y < p.r[1]);
+        if (!fail) {
+            const int4 ls = local_select2(csc, act0 ? total : 0, p.r[0], e.x, cmax, csc, act1 ? total : 0, p.r[1],
+                                          e.x, cmax, hist, red, info);
+            CSA2_TRACE(24);   // threshold
+            ListCut cut[2];
+#pragma unroll
+            for (int tr = 0; tr < 2; ++tr) {
+                const bool on = tr == 0 ? act0 : act1;
+                cut[tr].T = tr == 0 ? ls.x : ls.z;
+                cut[tr].quota = tr == 0 ? ls.y : ls.w;   // the ties at T ranked within the first r
+                cut[tr].all = 0;
+                cut[tr].base = 0;
+                cut[tr].r = p.r[tr];
+                cut[tr].out = on ? p.out[tr] + (size_t)u * p.r[tr] : nullptr;
+                cut[tr].status = p.status;
+            }
+            write_lists<false>(csc, total, 0, cpos, cut[0], cut[1], wsum, row_prefetch(p, u));
+            CSA2_TRACE(25);   // lists written
+        }
+    }
+    if (fail && tid == 0) {   // the Full kernel scans and cuts this query in full
+        const int i = atomicAdd(p.fb_list, 1);
+        p.fb_list[1 + i] = u;
+    }
+    CSA2_TRACE_END(7);
+}
+
+size_t mq_select_smem_bytes(int cap, int di) {
+    const int rb = di == 128 ? mq_rb<128>() : mq_rb<64>();
+    return 1024 + (size_t)rb * 128 * di + (size_t)std::max(1024, 16 * di) +
+           (size_t)(2 * cap + 1088 + 8 * kSelWarps + 64 + 4 * kSelWarps) * 4 + 16;
 }
 
 // ------------------------------------------------------------ Reindex, and Full for other key widths
@@ -2522,8 +2591,11 @@ void set_wait_controls(long long budget, int skip) {
 struct IdxPlan {
     int units, G, groups, chunk;
     int local_sel, rstride;
-    int mq;              // Full with queries sharing keys: multi-query scoring, then select only
-    int64_t pstride;     // per-unit stride of the scores it writes
+    int mq;              // Full with queries sharing keys: sample, estimate, mark, cut (+ Full for the rest)
+    int mq_tstep, mq_cap;
+    int64_t mq_sstride, mq_wstride;
+    int fb_groups, fb_G, fb_chunk;   // the Full kernel for the queries the cut leaves
+    size_t off_sample, off_words, off_est, off_fb;   // scratch offsets (the fallback's spill at 0)
     size_t spill_bytes;
 };
 
@@ -2586,9 +2658,28 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
     // (below kMqMinN keys the second launch costs more than the shared tiles save)
     pl.mq = (a.mode == CSA2_FULL && a.Tq >= kMqMin && a.N >= kMqMinN && a.Hi <= 8 &&
              (a.Di == 32 || a.Di == 64 || a.Di == 128)) ? 1 : 0;
-    pl.pstride = (int64_t)align_up((size_t)a.N, 4);
-    // (replaces the spill; the select's 64-element steps may read up to 63 elements past a unit's last score)
-    if (pl.mq) pl.spill_bytes = align_up((size_t)pl.units * (size_t)pl.pstride * 4 + 512, 256);
+    if (pl.mq) {
+        // (replaces the plan above) 32 to 128 sampled tiles, at least one in 64 (the estimate
+        // then ranks about r / 64 samples or more); a candidate word per 32 positions
+        const int ntile = (a.N + kMqRows - 1) / kMqRows;
+        const int want = std::min(128, std::max(32, (ntile + 63) / 64));
+        pl.mq_tstep = std::max(1, (ntile + want - 1) / want);
+        pl.mq_sstride = (int64_t)((ntile + pl.mq_tstep - 1) / pl.mq_tstep) * kMqRows;
+        pl.mq_wstride = (int64_t)ntile * 4;
+        pl.mq_cap = kMqCap;
+        // the fallback: groups of fb_G CTAs per query over the SMs, its scores spilled (at most 64 MB)
+        const size_t all = align_up((size_t)a.N, 256) * 4;
+        pl.fb_groups = (int)std::max<size_t>(1, std::min<size_t>({(size_t)sms, (size_t)pl.units, ((size_t)64 << 20) / all}));
+        pl.fb_G = std::max(1, std::min({kMaxG, sms / pl.fb_groups, (a.N + 1023) / 1024}));
+        pl.fb_chunk = (int)align_up((size_t)((a.N + pl.fb_G - 1) / pl.fb_G), 256);
+        const size_t per = (size_t)pl.fb_chunk * 4;
+        size_t off = pl.fb_chunk > kSmemScores ? align_up((size_t)pl.fb_groups * pl.fb_G * per + 512, 256) : 0;
+        pl.off_sample = off;  off += align_up((size_t)pl.units * pl.mq_sstride * 4, 256);
+        pl.off_words = off;   off += align_up((size_t)pl.units * pl.mq_wstride * 4, 256);
+        pl.off_est = off;     off += align_up((size_t)pl.units * 16, 256);
+        pl.off_fb = off;      off += align_up((size_t)(pl.units + 1) * 4, 256);
+        pl.spill_bytes = off;
+    }
     return pl;
 }
 
@@ -2631,9 +2722,9 @@ static cudaError_t launch_coop(Kern kern, int threads, const IdxParams& p, const
 // Cluster launch of the Full kernel: clusters of q.G CTAs, q.groups clusters, programmatic
 // stream serialisation (the kernel reads nothing the previous kernel writes before
 // griddepcontrol.wait, except that a producer with keys_ready starts the key stream).
-template <int DI>
+template <int DI, int MODE>
 static cudaError_t launch_mq(const MqParams& mp, const CUtensorMap& map, int grid, cudaStream_t stream) {
-    auto kern = index_mq_score_kernel<DI>;
+    auto kern = index_mq_score_kernel<DI, MODE>;
     // at least 116 KB, so that one CTA (and its 512 TMEM columns) holds an SM
     const size_t smem = std::max(sizeof(MqSmem<DI>) + 1024, (size_t)116 * 1024);
     cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem);
@@ -2649,6 +2740,85 @@ static cudaError_t launch_mq(const MqParams& mp, const CUtensorMap& map, int gri
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, mp, map);
+}
+
+// One CTA per query, programmatic dependent launch (nothing is read before griddepcontrol.wait).
+// smem_max: the kernel's largest dynamic shared memory over all calls (its attribute is set once).
+template <typename Kern>
+static cudaError_t launch_per_query(Kern kern, const IdxParams& p, size_t smem, size_t smem_max, cudaStream_t stream) {
+    if (smem_max > 48 * 1024) {
+        cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), (int)smem_max);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.units);
+    cfg.blockDim = dim3(kSel);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// The shared-key steps (sample, estimate, mark, cut) and the Full kernel for the
+// queries the cut leaves over.
+template <int DI>
+static cudaError_t launch_mq_steps(const csa2_index_args& a, const IdxPlan& pl, const IdxParams& p0,
+                                   const CUtensorMap& map, const CUtensorMap& mmap, uint8_t* scratch, int sms,
+                                   cudaStream_t stream) {
+    IdxParams p = p0;
+    p.mq_sample = reinterpret_cast<int32_t*>(scratch + pl.off_sample);
+    p.mq_sstride = pl.mq_sstride;
+    p.mq_tstep = pl.mq_tstep;
+    p.mq_est = reinterpret_cast<int4*>(scratch + pl.off_est);
+    p.mq_words = reinterpret_cast<int32_t*>(scratch + pl.off_words);
+    p.mq_wstride = pl.mq_wstride;
+    p.mq_cap = pl.mq_cap;
+    p.fb_list = reinterpret_cast<int32_t*>(scratch + pl.off_fb);
+    MqParams mp{};
+    mp.B = a.B; mp.Tq = a.Tq; mp.N = a.N; mp.Hi = a.Hi;
+    mp.nblk = (a.Tq + kMqQ - 1) / kMqQ;
+    const int items = a.B * mp.nblk;
+    for (int h = 0; h < 8; ++h) mp.w[h] = h < a.Hi ? a.w[h] : 0;
+    mp.q_pos = a.q_pos; mp.qi = a.qi;
+    mp.m = a.m;
+    mp.status = p.status;
+    // 1. the sampled tiles
+    mp.splits = std::max(1, std::min(sms / std::max(items, 1), (int)(pl.mq_sstride / kMqRows) / 8));
+    mp.tstep = pl.mq_tstep;
+    mp.out = const_cast<int32_t*>(p.mq_sample);
+    mp.ostride = pl.mq_sstride;
+    cudaError_t e = launch_mq<DI, kMqSample>(mp, mmap, items * mp.splits, stream);
+    if (e != cudaSuccess) return e;
+    // 2. the estimates
+    e = launch_per_query(index_mq_estimate_kernel, p, mq_estimate_smem_bytes((int)pl.mq_sstride),
+                         mq_estimate_smem_bytes(kMqSampleMax), stream);
+    if (e != cudaSuccess) return e;
+    // 3. the candidate words: each block's tiles split so that the grid covers the SMs, at least 8 tiles a split
+    mp.splits = std::max(1, std::min(sms / std::max(items, 1), (a.N / kMqRows + 7) / 8));
+    mp.tstep = 1;
+    mp.out = const_cast<int32_t*>(p.mq_words);
+    mp.ostride = pl.mq_wstride;
+    mp.est = p.mq_est;
+    e = launch_mq<DI, kMqMark>(mp, mmap, items * mp.splits, stream);
+    if (e != cudaSuccess) return e;
+    // 4. the cut
+    e = launch_per_query(index_mq_select_kernel<DI>, p, mq_select_smem_bytes(pl.mq_cap, DI),
+                         mq_select_smem_bytes(kMqCap, DI), stream);
+    if (e != cudaSuccess) return e;
+    // 5. the queries it left: the Full kernel over the list
+    IdxParams f = p0;
+    f.G = pl.fb_G;
+    f.groups = pl.fb_groups;
+    f.chunk = pl.fb_chunk;
+    f.spill = reinterpret_cast<int32_t*>(scratch);
+    f.unit_list = p.fb_list;
+    f.keys_ready = 0;
+    f.local_sel = 0;
+    return launch_coop(index_full_tc_kernel<DI>, kTcThreads, f, map, pl.fb_groups * pl.fb_G, stream);
 }
 
 // Launch one indexer call. `ws` holds plan_index(a).ws_bytes bytes (zero at first use).
@@ -2679,8 +2849,6 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
     p.cand = reinterpret_cast<int2*>(base + rg.off_cand);
     p.pub = reinterpret_cast<int*>(base + rg.off_pub);
     p.spill = (pl.chunk > kSmemScores && !pl.mq) ? static_cast<int32_t*>(scratch) : nullptr;
-    p.pre = pl.mq ? static_cast<int32_t*>(scratch) : nullptr;
-    p.pstride = pl.pstride;
     p.local_sel = pl.local_sel;
     p.rstride = pl.rstride;
     p.rscore = pl.local_sel ? static_cast<int32_t*>(scratch) : nullptr;
@@ -2724,7 +2892,7 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
     const int grid = pl.groups * pl.G;
     cudaError_t e;
     if (pl.mq) {
-        // scores of every query first (key tiles shared by blocks of kMqQ queries)
+        // key tiles shared by blocks of kMqQ queries
         EncodeTiledFn enc = get_encode_fn();
         if (!enc) return CSA2_ERR_CUDA;
         CUtensorMap mmap;
@@ -2740,23 +2908,11 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return CSA2_ERR_CUDA;
-        MqParams mp{};
-        mp.B = a.B; mp.Tq = a.Tq; mp.N = a.N; mp.Hi = a.Hi;
-        mp.nblk = (a.Tq + kMqQ - 1) / kMqQ;
-        const int items = a.B * mp.nblk;
-        // split each block's tiles so that the grid covers the SMs, at least 8 tiles a split
-        mp.splits = std::max(1, std::min(sms / std::max(items, 1), (a.N / kMqRows + 7) / 8));
-        for (int h = 0; h < 8; ++h) mp.w[h] = h < a.Hi ? a.w[h] : 0;
-        mp.q_pos = a.q_pos; mp.qi = a.qi;
-        mp.m = a.m;
-        mp.scores = static_cast<int32_t*>(scratch);
-        mp.sstride = pl.pstride;
-        mp.status = d_status;
-        const int mgrid = items * mp.splits;
-        e = a.Di == 64 ? launch_mq<64>(mp, mmap, mgrid, stream)
-            : a.Di == 32 ? launch_mq<32>(mp, mmap, mgrid, stream)
-                         : launch_mq<128>(mp, mmap, mgrid, stream);
-        if (e != cudaSuccess) return CSA2_ERR_CUDA;
+        uint8_t* sc = static_cast<uint8_t*>(scratch);
+        e = a.Di == 64   ? launch_mq_steps<64>(a, pl, p, map, mmap, sc, sms, stream)
+            : a.Di == 32 ? launch_mq_steps<32>(a, pl, p, map, mmap, sc, sms, stream)
+                         : launch_mq_steps<128>(a, pl, p, map, mmap, sc, sms, stream);
+        return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
     }
     if (a.mode == CSA2_FULL && a.Di == 64) e = launch_coop(index_full_tc_kernel<64>, kTcThreads, p, map, grid, stream);
     else if (a.mode == CSA2_FULL && a.Di == 32) e = launch_coop(index_full_tc_kernel<32>, kTcThreads, p, map, grid, stream);

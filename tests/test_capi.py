@@ -122,17 +122,37 @@ def test_stack_mode_order():
     assert capi.csa2_layer_stack(capi.StackArgs(2, idx, att), 0, 0, 0, 0) == 4
 
 
-def test_index_workspace_holds_shared_key_scores():
+def _shared_key_scratch(units, N, sms=148):
+    """The shared-key path's scratch, restated: the fallback's spill (groups of G CTAs per
+    query over the SMs, at most 64 MB), the sampled tiles' scores (32 to 128 tiles of 128
+    positions a query, at least one tile in 64), one candidate word per 32 positions a
+    query, the estimates and the fallback list; each part rounded up to 256 bytes."""
+    a256 = lambda x: (x + 255) // 256 * 256
+    ntile = -(-N // 128)
+    want = min(128, max(32, -(-ntile // 64)))
+    tstep = max(1, -(-ntile // want))
+    sstride = -(-ntile // tstep) * 128
+    groups = max(1, min(sms, units, (64 << 20) // (a256(N) * 4)))
+    G = max(1, min(64, sms // groups, (N + 1023) // 1024))
+    chunk = a256(-(-N // G))
+    spill = a256(groups * G * chunk * 4 + 512) if chunk > 16384 else 0
+    return spill + a256(units * sstride * 4) + a256(units * ntile * 4 * 4) + a256(units * 16) + a256((units + 1) * 4)
+
+
+def test_index_workspace_of_the_shared_key_path():
     """A Full call with at least 4 queries per sequence on a key set of at least 8192
-    positions scores its queries in blocks first, so its workspace also holds every
-    query's scores (B*Tq*N int32, plus slack, rounded to 256 bytes); smaller calls
-    score one query per unit and need none."""
+    positions scores its queries in blocks and keeps no query's scores in full: its
+    workspace holds a sample, candidate words, estimates and the fallback's spill, well
+    below B*Tq*N int32 scores; smaller calls score one query per unit and need none."""
     def ws(Tq, N):
         a, _w = _index_args(Tq=Tq, N=N, ki_seq_stride=N * 64)
         return capi.csa2_workspace_bytes(0, a)
     base = ws(1, 8192)
-    for Tq, N in [(64, 1 << 20), (64, 8192), (4, 8192)]:
-        assert ws(Tq, N) - base == (Tq * N * 4 + 512 + 255) // 256 * 256
+    for Tq, N in [(64, 1 << 20), (64, 8192), (4, 8192), (4096, 69632)]:
+        extra = ws(Tq, N) - base
+        assert extra == _shared_key_scratch(Tq, N), (Tq, N)
+        if N >= 69632:
+            assert extra < Tq * N * 4 // 2, (Tq, N)
     assert ws(64, 4096) == base      # below 8192 keys
     assert ws(3, 8192) == base       # fewer than 4 queries
 

@@ -153,13 +153,13 @@ def test_weights_past_the_bound_are_rejected(ws):
 
 
 @pytest.mark.parametrize("kind", ["random", "rising", "equal"])
-def test_select_only_one_cta_per_query(kind, ws, status):
-    """Queries that share keys, more of them than SMs: the multi-query scoring kernel,
-    then one CTA per query cuts that query's scores from global memory. Random scores
-    take the sampled select (a threshold estimate from every s-th score, one candidate
-    pass, the exact cut over the candidates); scores that rise with the position (the
-    best ones all in the last warp's range of positions) and all-equal scores overflow
-    its candidate lists and take the full select. Every list bit-exact."""
+def test_shared_keys_cut(kind, ws, status):
+    """Queries that share keys, more of them than SMs: the sampled tiles give each query
+    a threshold estimate, the marking pass records its candidates (one bit per
+    position), and one CTA per query rescores and cuts them. Random scores and scores
+    that rise with the position (runs of equal scores) take the cut; all-equal scores
+    make every position a candidate, more than the cut holds, and go to the Full
+    kernel's scan and select. Every list bit-exact."""
     from oracle import cpp as C
     B, Tq, N, Hi, Di, k, P = 1, 160, 40000, 8, 64, 512, 2048
     qi, w, ki = inputs(31, B, Tq, N, Hi, Di, False)

@@ -100,8 +100,9 @@ def test_index_full_shapes(B, N, Tq, k, P, ws, status):
     (1, 12000, 16, 4, 32, 256, 512),     # 32-byte keys, 4 heads
 ])
 def test_index_full_shared_keys(B, N, Tq, Hi, Di, k, P, ws, status):
-    """Tq >= 4 queries per sequence: the multi-query scoring kernel scores blocks of
-    queries against shared key tiles, and the Full kernel cuts in its select-only mode."""
+    """Tq >= 4 queries per sequence: blocks of queries share key tiles; sampled tiles give
+    each query a threshold estimate, the marking pass records its candidates, and one CTA
+    per query rescores and cuts them (a query with fewer positions than k takes them all)."""
     qi = synth.randint_i8(3, 10 + Tq, (B, Tq, Hi, Di))
     ki = synth.randint_i8(3, 20 + N, (B, N, Di))
     w = synth.randint_i32(3, 30, (Hi,), 1, 8)
@@ -110,6 +111,29 @@ def test_index_full_shared_keys(B, N, Tq, Hi, Di, k, P, ws, status):
     q_pos[:, -1] = N - 1
     q_pos[0, 0] = min(q_pos[0, 0], 5)        # a query with fewer positions than k
     _check_full(qi, w, ki, q_pos, k, P, ws, status)
+
+
+def test_index_shared_keys_bad_positions(ws):
+    """A shared-key call with positions outside [0, N): the status word says
+    CSA2_ERR_RANGE, those queries' lists are all -1, and every other query's lists are
+    exact."""
+    B, N, Tq, Hi, Di, k, P = 1, 9000, 20, 8, 64, 300, 1000
+    qi = synth.randint_i8(5, 1, (B, Tq, Hi, Di))
+    ki = synth.randint_i8(5, 2, (B, N, Di))
+    w = synth.randint_i32(5, 3, (Hi,), 1, 8)
+    q_pos = np.sort(np.random.default_rng(7).integers(N // 2, N, size=(B, Tq)), axis=1).astype(np.int32)
+    bad = [3, 11]
+    q_pos[0, 3], q_pos[0, 11] = -1, N
+    st = ops.Status()
+    pool, topk = ops.index_topk("FULL", dev(q_pos), dev(qi), w, dev(ki), k, P, ws=ws, status=st)
+    code, _ = st.read()
+    assert code == 5   # CSA2_ERR_RANGE
+    good = [j for j in range(Tq) if j not in bad]
+    rpool, rtopk = _oracle_full(qi[:, good], w, ki, q_pos[:, good], k, P)
+    got_t, got_p = topk.cpu().numpy(), pool.cpu().numpy()
+    assert_lists_equal(torch.from_numpy(np.ascontiguousarray(got_t[:, good])), rtopk, "topk")
+    assert_lists_equal(torch.from_numpy(np.ascontiguousarray(got_p[:, good])), rpool, "pool")
+    assert (got_t[:, bad] == -1).all() and (got_p[:, bad] == -1).all()
 
 
 def test_index_full_early_positions_and_padding(ws, status):
