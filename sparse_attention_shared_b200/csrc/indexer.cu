@@ -78,15 +78,14 @@ struct IdxParams {
     int local_sel;       // Reindex: every CTA of the group cuts over all of the unit's scores
     int keys_ready;      // keys and positions were complete before the previous kernel began
     // Full with queries that share keys: the sampled tiles' scores, the estimates, the
-    // candidate words (one bit per position), the candidates one CTA of the cut holds,
-    // and the units it leaves to the Full kernel ([0] count, [1 ..] units)
+    // candidate words (one bit per position) and the units the cut leaves to the Full
+    // kernel ([0] count, [1 ..] units)
     const int32_t* mq_sample;
     int64_t mq_sstride;
     int mq_tstep;
     int4* mq_est;
     const int32_t* mq_words;
     int64_t mq_wstride;
-    int mq_cap;
     int32_t* fb_list;
     const int32_t* unit_list;   // Full kernel: the units to take ([0] count, [1 ..] units), nullptr: all
     int rstride;         // per-unit stride of rscore
@@ -2051,6 +2050,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
 // ------------------------------------------------------------ shared keys: estimates and the cut
 constexpr int kMqSampleMax = 16384;  // sample entries per query (at most 128 sampled tiles)
 constexpr int kMqCap = 16384;        // candidates per query that the cut holds
+constexpr int kMqCapSmall = 8192;    // ... in its two-CTAs-per-SM form
 
 size_t mq_estimate_smem_bytes(int sstride) { return (size_t)(sstride + 1088 + 8 * kSelWarps + 64) * 4; }
 
@@ -2112,14 +2112,15 @@ __global__ void __launch_bounds__(kSel, 2) index_mq_estimate_kernel(const __grid
 // key rows and the index query as tensor-core operands, [cap] positions and [cap] scores
 // (cap from the launch), the histogram, reduction and count scratch, the barrier and
 // the TMEM address.
-template <int DI> constexpr int mq_rb() { return DI == 128 ? 4 : 8; }   // 128-row blocks per batch
+// 128-row blocks per batch; the small form (cap kMqCapSmall, two CTAs per SM) gathers 4
+template <int DI, bool SMALL> constexpr int mq_rb() { return (SMALL || DI == 128) ? 4 : 8; }
 
-template <int DI>
-__global__ void __launch_bounds__(kSel, 1) index_mq_select_kernel(const __grid_constant__ IdxParams p) {
+template <int DI, bool SMALL>
+__global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(const __grid_constant__ IdxParams p) {
     extern __shared__ __align__(1024) uint8_t smq_raw[];
     uint8_t* sbase = smq_raw + ((1024u - (smem_u32(smq_raw) & 1023u)) & 1023u);
-    constexpr int kRB = mq_rb<DI>();
-    const int cap = p.mq_cap;
+    constexpr int kRB = mq_rb<DI, SMALL>();
+    const int cap = SMALL ? kMqCapSmall : kMqCap;
     uint8_t* stage = sbase;                                   // [kRB][128 rows][DI], TMA-tile layout
     uint8_t* qtc = stage + kRB * 128 * DI;                    // [16 rows][DI]: heads, zero past Hi
     int* cpos = reinterpret_cast<int*>(qtc + (16 * DI > 1024 ? 16 * DI : 1024));
@@ -2313,8 +2314,9 @@ __global__ void __launch_bounds__(kSel, 1) index_mq_select_kernel(const __grid_c
     CSA2_TRACE_END(7);
 }
 
-size_t mq_select_smem_bytes(int cap, int di) {
-    const int rb = di == 128 ? mq_rb<128>() : mq_rb<64>();
+size_t mq_select_smem_bytes(bool small, int di) {
+    const int cap = small ? kMqCapSmall : kMqCap;
+    const int rb = (small || di == 128) ? 4 : 8;
     return 1024 + (size_t)rb * 128 * di + (size_t)std::max(1024, 16 * di) +
            (size_t)(2 * cap + 1088 + 8 * kSelWarps + 64 + 4 * kSelWarps) * 4 + 16;
 }
@@ -2666,7 +2668,12 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
         pl.mq_tstep = std::max(1, (ntile + want - 1) / want);
         pl.mq_sstride = (int64_t)((ntile + pl.mq_tstep - 1) / pl.mq_tstep) * kMqRows;
         pl.mq_wstride = (int64_t)ntile * 4;
-        pl.mq_cap = kMqCap;
+        // candidates expected: about 1.2 r + 16 n / m a track (r the larger track); the two-CTAs-per-SM
+        // cut when half its room covers that
+        const int m_s = (int)std::min<int64_t>(pl.mq_sstride, (int64_t)a.N);
+        const int r_max = std::max(a.P, a.k);
+        const long long expect = (long long)r_max * 6 / 5 + 16LL * a.N / std::max(m_s, 1);
+        pl.mq_cap = (2 * expect <= kMqCapSmall && a.Di <= 64) ? kMqCapSmall : kMqCap;
         // the fallback: groups of fb_G CTAs per query over the SMs, its scores spilled (at most 64 MB)
         const size_t all = align_up((size_t)a.N, 256) * 4;
         pl.fb_groups = (int)std::max<size_t>(1, std::min<size_t>({(size_t)sms, (size_t)pl.units, ((size_t)64 << 20) / all}));
@@ -2776,7 +2783,6 @@ static cudaError_t launch_mq_steps(const csa2_index_args& a, const IdxPlan& pl, 
     p.mq_est = reinterpret_cast<int4*>(scratch + pl.off_est);
     p.mq_words = reinterpret_cast<int32_t*>(scratch + pl.off_words);
     p.mq_wstride = pl.mq_wstride;
-    p.mq_cap = pl.mq_cap;
     p.fb_list = reinterpret_cast<int32_t*>(scratch + pl.off_fb);
     MqParams mp{};
     mp.B = a.B; mp.Tq = a.Tq; mp.N = a.N; mp.Hi = a.Hi;
@@ -2806,8 +2812,10 @@ static cudaError_t launch_mq_steps(const csa2_index_args& a, const IdxPlan& pl, 
     e = launch_mq<DI, kMqMark>(mp, mmap, items * mp.splits, stream);
     if (e != cudaSuccess) return e;
     // 4. the cut
-    e = launch_per_query(index_mq_select_kernel<DI>, p, mq_select_smem_bytes(pl.mq_cap, DI),
-                         mq_select_smem_bytes(kMqCap, DI), stream);
+    const bool small = pl.mq_cap == kMqCapSmall;
+    const size_t ssm = mq_select_smem_bytes(small, DI);
+    e = small ? launch_per_query(index_mq_select_kernel<DI, true>, p, ssm, ssm, stream)
+              : launch_per_query(index_mq_select_kernel<DI, false>, p, ssm, ssm, stream);
     if (e != cudaSuccess) return e;
     // 5. the queries it left: the Full kernel over the list
     IdxParams f = p0;
