@@ -2139,26 +2139,42 @@ __global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(co
     const int t = p.q_pos[u], tg = last_entry(t, p.m);
     const bool bad = t < 0 || tg >= p.N;
     if (bad && tid == 0) report(p.status, CSA2_ERR_RANGE, u);
-    const int n = bad ? 0 : tg + 1;
+    // Reindex with one CTA per query: the candidates are the unit's pool, whose valid
+    // entries (0 <= s <= the query's last entry) form a prefix, -1 padding after
+    const int32_t* pool = p.pool_in ? p.pool_in + (size_t)u * p.P_in : nullptr;
+    int n = bad ? 0 : tg + 1;
+    if (pool) {
+        int fb = p.P_in;
+        for (int i = tid; i < p.P_in; i += kSel) {
+            const int s = __ldg(pool + i);
+            if (!(s >= 0 && s <= tg)) fb = min(fb, i);
+        }
+        fb = sel_min(fb, red);
+        for (int i = fb + tid; i < p.P_in; i += kSel)   // past the first invalid entry: padding only
+            if (__ldg(pool + i) >= 0) report(p.status, CSA2_ERR_RANGE, u);
+        n = fb;
+    }
     // a track with r >= n takes every entry in order (none at a bad position), then -1
 #pragma unroll
     for (int tr = 0; tr < 2; ++tr) {
         const int r = p.r[tr];
         if (r > 0 && r >= n) {
             int32_t* out = p.out[tr] + (size_t)u * r;
-            for (int i = tid; i < r; i += kSel) out[i] = i < n ? i : -1;
+            for (int i = tid; i < r; i += kSel) out[i] = i < n ? (pool ? __ldg(pool + i) : i) : -1;
         }
     }
-    const int4 e = p.mq_est[u];
+    // the tracks to cut and their estimates (a pool: every entry is a candidate)
+    const bool pk = pool && p.r[1] > 0 && p.r[1] < n;
+    const int4 e = pool ? make_int4(INT_MIN, INT_MIN, INT_MIN, pk ? 2 : 0) : p.mq_est[u];
     const bool act0 = (e.w & 1) != 0, act1 = (e.w & 2) != 0;
     if (!act0 && !act1) { CSA2_TRACE_END(7); return; }
 
     // ---- the candidates' positions in order: warp w takes the words [w W, (w + 1) W), its
     // lanes read 32 consecutive words at a time; counted, scanned over the warps, expanded
-    const int nw = (n + 31) >> 5;
+    const int nw = pool ? 0 : (n + 31) >> 5;
     const int wpw = (nw + kSelWarps * 32 - 1) / (kSelWarps * 32) * 32;   // words per warp
     const int ww0 = min(nw, (tid >> 5) * wpw), ww1 = min(nw, ww0 + wpw);
-    const int32_t* words = p.mq_words + (size_t)u * p.mq_wstride;
+    const int32_t* words = pool ? nullptr : p.mq_words + (size_t)u * p.mq_wstride;
     auto word_at = [&](int w) -> unsigned {
         if (w >= ww1) return 0u;
         unsigned m = (unsigned)__ldcg(words + w);
@@ -2172,9 +2188,12 @@ __global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(co
     int total;
     int off = sel_scan_excl(lane == 0 ? cnt : 0, red, total);   // the warp's first slot
     off = __shfl_sync(0xffffffffu, off, 0);
+    if (pool) total = n;
     CSA2_TRACE(22);   // candidates counted
     bool fail = total > cap;
     if (!fail) {
+        if (pool)
+            for (int i = tid; i < n; i += kSel) cpos[i] = __ldg(pool + i);
         for (int w0 = ww0; w0 < ww1; w0 += 32) {
             unsigned m = word_at(w0 + lane);
             const int c = __popc(m);
@@ -2218,7 +2237,7 @@ __global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(co
         constexpr uint32_t kIdesc = idesc_i8(128, 16);
         constexpr int CPR = DI / 16, CPT = kRB * 128 * CPR / kSel;   // chunks per row, per thread
         const int8_t* kb = p.ki + (size_t)b * p.ki_seq_stride;
-        int c0 = 0, c1 = 0, cmax = INT_MIN;
+        int c0 = 0, c1 = 0, cmax = INT_MIN, cmin = INT_MAX;
         uint32_t phase = 0;
         bool ok = true;
         for (int base = 0; base < total && ok; base += kRB * 128) {
@@ -2267,6 +2286,7 @@ __global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(co
                         c0 += x >= e.y;
                         c1 += x >= e.z;
                         cmax = max(cmax, x);
+                        cmin = min(cmin, x);
                     }
                 }
             }
@@ -2277,19 +2297,22 @@ __global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(co
         if (warp == 0) tmem_dealloc(tmem, 16 * kRB);
         fail = !ok;
         cmax = __reduce_max_sync(0xffffffffu, cmax);
-        if (tid == 0) info[28] = INT_MIN;
+        cmin = __reduce_min_sync(0xffffffffu, cmin);
+        if (tid == 0) { info[28] = INT_MIN; info[29] = INT_MAX; }
         int4 ca = make_int4(c0, c1, 0, 0), cb = make_int4(0, 0, 0, 0);
-        sel_total8(ca, cb, red);   // (its first barrier also orders info[28] before the maxima below)
-        if (lane == 0) atomicMax(&info[28], cmax);
+        sel_total8(ca, cb, red);   // (its first barrier also orders info[28..29] before the extremes below)
+        if (lane == 0) { atomicMax(&info[28], cmax); atomicMin(&info[29], cmin); }
         sel_sync();
         cmax = info[28];
+        // the radix passes' range: the candidates' own, from the lower estimate on
+        const int clo = max(e.x, info[29]);
         CSA2_TRACE(23);   // candidates scored
         // every track needs r candidates at or above its estimate: then its r best scores
         // and all ties at its threshold are candidates
         fail = fail || (act0 && ca.x < p.r[0]) || (act1 && ca.y < p.r[1]);
         if (!fail) {
-            const int4 ls = local_select2(csc, act0 ? total : 0, p.r[0], e.x, cmax, csc, act1 ? total : 0, p.r[1],
-                                          e.x, cmax, hist, red, info);
+            const int4 ls = local_select2(csc, act0 ? total : 0, p.r[0], clo, cmax, csc, act1 ? total : 0, p.r[1],
+                                          clo, cmax, hist, red, info);
             CSA2_TRACE(24);   // threshold
             ListCut cut[2];
 #pragma unroll
@@ -2307,7 +2330,7 @@ __global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(co
             CSA2_TRACE(25);   // lists written
         }
     }
-    if (fail && tid == 0) {   // the Full kernel scans and cuts this query in full
+    if (fail && tid == 0 && p.fb_list) {   // the Full kernel scans and cuts this query in full
         const int i = atomicAdd(p.fb_list, 1);
         p.fb_list[1 + i] = u;
     }
@@ -2674,9 +2697,10 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
         const int r_max = std::max(a.P, a.k);
         const long long expect = (long long)r_max * 6 / 5 + 16LL * a.N / std::max(m_s, 1);
         pl.mq_cap = (2 * expect <= kMqCapSmall && a.Di <= 64) ? kMqCapSmall : kMqCap;
-        // the fallback: groups of fb_G CTAs per query over the SMs, its scores spilled (at most 64 MB)
+        // the fallback (a few queries a call at most, as a rule): up to 16 queries at a time, groups of
+        // fb_G CTAs each over the SMs, their scores spilled where a chunk exceeds shared memory (at most 64 MB)
         const size_t all = align_up((size_t)a.N, 256) * 4;
-        pl.fb_groups = (int)std::max<size_t>(1, std::min<size_t>({(size_t)sms, (size_t)pl.units, ((size_t)64 << 20) / all}));
+        pl.fb_groups = (int)std::max<size_t>(1, std::min<size_t>({(size_t)16, (size_t)pl.units, ((size_t)64 << 20) / all}));
         pl.fb_G = std::max(1, std::min({kMaxG, sms / pl.fb_groups, (a.N + 1023) / 1024}));
         pl.fb_chunk = (int)align_up((size_t)((a.N + pl.fb_G - 1) / pl.fb_G), 256);
         const size_t per = (size_t)pl.fb_chunk * 4;
@@ -2770,6 +2794,14 @@ static cudaError_t launch_per_query(Kern kern, const IdxParams& p, size_t smem, 
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
+// The cut, in its two-CTAs-per-SM form (8192 candidates) or its one-CTA form (16384).
+template <int DI>
+static cudaError_t launch_cut(const IdxParams& p, bool small, cudaStream_t stream) {
+    const size_t ssm = mq_select_smem_bytes(small, DI);
+    return small ? launch_per_query(index_mq_select_kernel<DI, true>, p, ssm, ssm, stream)
+                 : launch_per_query(index_mq_select_kernel<DI, false>, p, ssm, ssm, stream);
+}
+
 // The shared-key steps (sample, estimate, mark, cut) and the Full kernel for the
 // queries the cut leaves over.
 template <int DI>
@@ -2812,10 +2844,7 @@ static cudaError_t launch_mq_steps(const csa2_index_args& a, const IdxPlan& pl, 
     e = launch_mq<DI, kMqMark>(mp, mmap, items * mp.splits, stream);
     if (e != cudaSuccess) return e;
     // 4. the cut
-    const bool small = pl.mq_cap == kMqCapSmall;
-    const size_t ssm = mq_select_smem_bytes(small, DI);
-    e = small ? launch_per_query(index_mq_select_kernel<DI, true>, p, ssm, ssm, stream)
-              : launch_per_query(index_mq_select_kernel<DI, false>, p, ssm, ssm, stream);
+    e = launch_cut<DI>(p, pl.mq_cap == kMqCapSmall, stream);
     if (e != cudaSuccess) return e;
     // 5. the queries it left: the Full kernel over the list
     IdxParams f = p0;
@@ -2920,6 +2949,14 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
         e = a.Di == 64   ? launch_mq_steps<64>(a, pl, p, map, mmap, sc, sms, stream)
             : a.Di == 32 ? launch_mq_steps<32>(a, pl, p, map, mmap, sc, sms, stream)
                          : launch_mq_steps<128>(a, pl, p, map, mmap, sc, sms, stream);
+        return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+    }
+    if (a.mode == CSA2_REINDEX && pl.units >= sms && P_in > 0 && P_in <= kMqCap && a.Hi <= 8 &&
+        (a.Di == 32 || a.Di == 64 || a.Di == 128)) {
+        // one CTA per query: the pool is the cut's candidate list, rescored on the tensor cores
+        const bool small = P_in <= kMqCapSmall && a.Di <= 64;
+        e = a.Di == 64 ? launch_cut<64>(p, small, stream) : a.Di == 32 ? launch_cut<32>(p, small, stream)
+                                                                       : launch_cut<128>(p, small, stream);
         return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
     }
     if (a.mode == CSA2_FULL && a.Di == 64) e = launch_coop(index_full_tc_kernel<64>, kTcThreads, p, map, grid, stream);

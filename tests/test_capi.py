@@ -123,8 +123,8 @@ def test_stack_mode_order():
 
 
 def _shared_key_scratch(units, N, sms=148):
-    """The shared-key path's scratch, restated: the fallback's spill (groups of G CTAs per
-    query over the SMs, at most 64 MB), the sampled tiles' scores (32 to 128 tiles of 128
+    """The shared-key path's scratch, restated: the fallback's spill (up to 16 queries at a
+    time, groups of G CTAs each over the SMs, at most 64 MB), the sampled tiles' scores (32 to 128 tiles of 128
     positions a query, at least one tile in 64), one candidate word per 32 positions a
     query, the estimates and the fallback list; each part rounded up to 256 bytes."""
     a256 = lambda x: (x + 255) // 256 * 256
@@ -132,7 +132,7 @@ def _shared_key_scratch(units, N, sms=148):
     want = min(128, max(32, -(-ntile // 64)))
     tstep = max(1, -(-ntile // want))
     sstride = -(-ntile // tstep) * 128
-    groups = max(1, min(sms, units, (64 << 20) // (a256(N) * 4)))
+    groups = max(1, min(16, units, (64 << 20) // (a256(N) * 4)))
     G = max(1, min(64, sms // groups, (N + 1023) // 1024))
     chunk = a256(-(-N // G))
     spill = a256(groups * G * chunk * 4 + 512) if chunk > 16384 else 0

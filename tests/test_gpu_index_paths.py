@@ -203,18 +203,22 @@ def test_full_decode_skewed_scores(kind, ws, status):
     assert_lists_equal(pool, rpool, f"{kind}: pool")
 
 
-@pytest.mark.parametrize("kind", ["random", "rising", "equal", "ragged"])
-def test_reindex_one_cta_per_query(kind, ws, status):
-    """Reindex with more queries than SMs: one CTA per query cuts the rescored pool in
-    its own shared memory. Random scores; scores that rise with the position; all-equal
-    scores (the cut is all ties, taken by position); and ragged pools padded with -1,
-    some of them holding fewer entries than k (the whole pool is the list). Every list
-    bit-exact, and every entry taken from the query's pool."""
+@pytest.mark.parametrize("kind,Hi,Di", [("random", 8, 64), ("rising", 8, 64), ("equal", 8, 64), ("ragged", 8, 64),
+                                        ("random", 4, 32), ("random", 6, 128)])
+def test_reindex_one_cta_per_query(kind, Hi, Di, ws, status):
+    """Reindex with more queries than SMs: one CTA per query takes its pool as the
+    candidate list, rescores the entries on the tensor cores and cuts them in its own
+    shared memory. Random scores; scores that rise with the position; all-equal scores
+    (the cut is all ties, taken by position); ragged pools padded with -1, some of them
+    holding fewer entries than k (the whole pool is the list); 32- and 128-byte keys.
+    Every list bit-exact, and every entry taken from the query's pool."""
     from oracle import cpp as C
     if kind == "ragged":
-        B, Tq, N, Hi, Di, k, P = 2, 80, 3000, 8, 64, 1024, 4096
+        B, Tq, N, k, P = 2, 80, 3000, 1024, 4096
+    elif Di == 64:
+        B, Tq, N, k, P = 1, 160, 40000, 2048, 8192
     else:
-        B, Tq, N, Hi, Di, k, P = 1, 160, 40000, 8, 64, 2048, 8192
+        B, Tq, N, k, P = 1, 150, 20000, 700, 3000
     qi, w, ki = inputs(41, B, Tq, N, Hi, Di, False)
     qi2, w2, ki2 = inputs(43, B, Tq, N, Hi, Di, False)
     if kind == "rising":
