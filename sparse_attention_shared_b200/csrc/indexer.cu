@@ -2240,15 +2240,20 @@ __global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(co
         int c0 = 0, c1 = 0, cmax = INT_MIN, cmin = INT_MAX;
         uint32_t phase = 0;
         bool ok = true;
-        for (int base = 0; base < total && ok; base += kRB * 128) {
-            const int nblk = min(kRB, (total - base + 127) / 128);
-            int4 v[CPT];
+        // this batch's chunks in registers; the next batch's loads are issued once this
+        // batch's MMAs are, so they are in flight during its wait and epilogue
+        int4 v[CPT];
+        auto load_batch = [&](int b0) {
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
-                const int ci = tid + k * kSel, r = ci / CPR, g = base + r;
+                const int ci = tid + k * kSel, r = ci / CPR, g = b0 + r;
                 v[k] = g < total ? __ldg(reinterpret_cast<const int4*>(kb + (size_t)cpos[g] * DI) + ci % CPR)
                                  : make_int4(0, 0, 0, 0);
             }
+        };
+        load_batch(0);
+        for (int base = 0; base < total && ok; base += kRB * 128) {
+            const int nblk = min(kRB, (total - base + 127) / 128);
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
                 const int ci = tid + k * kSel, r = ci / CPR;
@@ -2267,6 +2272,7 @@ __global__ void __launch_bounds__(kSel, SMALL ? 2 : 1) index_mq_select_kernel(co
                                smem_desc(b0 + kk * 32, 16, kSbo, kSwz), kIdesc, kk > 0 ? 1u : 0u);
                 mma_commit(bar);
             }
+            if (base + kRB * 128 < total) load_batch(base + kRB * 128);
             ok = sel_and(mbar_wait(bar, phase, p.status, 31) ? 1 : 0) != 0;   // (the same in every thread)
             phase ^= 1u;
             tc_fence_after();

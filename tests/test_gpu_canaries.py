@@ -66,8 +66,9 @@ def _guarded_stack(wl):
 @pytest.mark.parametrize("name,kw", [
     ("stack20_128k", dict(B=3, N=20000)),                    # Full, Reindex, cluster attention
     ("paper_schedule", dict(B=2, N=9000)),
-    ("long_1m", dict(N=40000, Tq=6)),                        # multi-query scoring + cooperative select
+    ("long_1m", dict(N=40000, Tq=6)),                        # shared-key sample, estimate, mark and cut
     ("decode_full", dict(B=150, N=20000)),                   # more units than SMs: one CTA per unit, spilled scores
+    ("replay_prefill", dict(B=1, N=9000, Tq=160, W=128)),    # shared-key cut and Reindex cut, one CTA per query
 ])
 def test_outputs_stay_inside_their_buffers(name, kw):
     wl = synth.make_workload(name, **kw)
