@@ -201,7 +201,10 @@ typedef struct {
  * 2 = csa2_layer_stack (csa2_stack_args*). Returns 0 for invalid arguments.
  * A Full call whose sequences carry Tq >= 4 queries over N >= 8192 positions
  * (Hi <= 8, Di in {32, 64, 128}) scores its queries in blocks that share key
- * tiles before it selects; its workspace then also holds B*Tq*N int32 scores.
+ * tiles and keeps no query's scores in full: its workspace then also holds a
+ * sample of each query's scores (at most 16384 int32), one 32-bit candidate word
+ * per 32 positions and query, per-query estimates, a list of the queries left
+ * to the cooperative kernel, and that kernel's score spill (at most 64 MB).
  * One workspace may serve calls of any sizes in turn (on one stream): zero it once
  * before its first use; a call that ends without a device-reported error leaves it
  * ready for the next. */
