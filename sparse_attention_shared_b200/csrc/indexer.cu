@@ -32,6 +32,12 @@
 // exact threshold score T among them with a local radix select; exact ties at
 // T are cut by position through per-CTA counts. Every CTA then writes its
 // selected positions at its offset, in ascending order, with no further sync.
+//
+// Calls with many queries take other kernels below: Full calls whose queries share
+// keys (index_mq_score_kernel, index_mq_estimate_kernel, index_mq_select_kernel:
+// sampled estimates, candidate bits, a tensor-core rescoring cut, the cooperative
+// kernel for the queries left over), and Reindex calls with more queries than SMs
+// (index_mq_select_kernel over the pool).
 #include <cuda.h>
 
 #include <algorithm>
