@@ -435,18 +435,25 @@ def test_decode_full_every_unit(ws, status):
 
 
 def test_prefill_chunk_every_unit(ws, status):
-    # 4096 queries of one sequence, 32 heads; the multi-query scoring kernel, then the select-only pass
+    # 4096 queries of one sequence, 32 heads: the shared-key Full path (sampled estimates, candidate bits, the
+    # tensor-core cut at two queries per SM) and the per-query attention
     _check_stack_every_unit(synth.make_workload("prefill_chunk"), ws, status)
 
 
 def test_long_1m_every_unit(ws, status):
-    # one sequence of 2^20 positions, 64 queries: the Full layer's scores spill (two CTAs per query),
-    # nine Reindex layers select from the pool by the group's single select
+    # one sequence of 2^20 positions, 64 queries: the shared-key Full path (128 sampled tiles a query, the
+    # one-CTA cut), nine Reindex layers select from the pool by the group's single select
     _check_stack_every_unit(synth.make_workload("long_1m"), ws, status)
 
 
 def test_stack20_128k_every_unit(ws, status):
     _check_stack_every_unit(synth.make_workload("stack20_128k"), ws, status)
+
+
+def test_encoder_m2_shared_keys_every_unit(ws, status):
+    # compression rate 2 with 8 queries a sequence: the shared-key Full path reads entries up to each
+    # query's last one ((t + 1) / 2 - 1), then Reuse and Reindex layers
+    _check_stack_every_unit(synth.make_workload("encoder_m2", B=2, N=20000, Tq=8), ws, status)
 
 
 def test_tiny_every_unit(ws, status):
@@ -455,7 +462,8 @@ def test_tiny_every_unit(ws, status):
 
 def test_replay_prefill_every_unit(ws, status):
     # bounded replay: the last 256 of 16384 prompt positions through [F,U,U,RI]x5, window references cut at
-    # the segment (local_base = N - 256); the Full layers score the 256 queries in blocks that share key tiles
+    # the segment (local_base = N - 256); the Full layers take the shared-key path, the Reindex layers the
+    # tensor-core cut over the pool (512 queries, more than SMs)
     wl = synth.make_workload("replay_prefill", B=2, N=16384, Tq=256, W=256)
     assert wl.spec.local_base == 16384 - 256
     _check_stack_every_unit(wl, ws, status)
