@@ -2114,11 +2114,12 @@ __global__ void __launch_bounds__(kSel, 2) index_mq_estimate_kernel(const __grid
     if (tid == 0) p.mq_est[u] = e;
 }
 
-// Step 4: one CTA per query. Shared memory (1024-aligned): kMqRB row blocks of gathered
-// key rows and the index query as tensor-core operands, [cap] positions and [cap] scores
-// (cap from the launch), the histogram, reduction and count scratch, the barrier and
+// Step 4 (and Reindex with more queries than SMs): one CTA per query. Shared memory
+// (1024-aligned): kRB 128-row blocks of gathered key rows and the index query as
+// tensor-core operands, [cap] positions and [cap] scores (cap = kMqCap, or kMqCapSmall in
+// the two-CTAs-per-SM form), the histogram, reduction and count scratch, the barrier and
 // the TMEM address.
-// 128-row blocks per batch; the small form (cap kMqCapSmall, two CTAs per SM) gathers 4
+// 128-row blocks per batch: 8, or 4 in the small form and for 128-byte keys
 template <int DI, bool SMALL> constexpr int mq_rb() { return (SMALL || DI == 128) ? 4 : 8; }
 
 template <int DI, bool SMALL>
