@@ -884,14 +884,17 @@ __global__ void __launch_bounds__(kClThreads, 2)
 // adds the tile's. The query's output is o / l at the end: no partials leave the CTA and
 // nothing is merged. NT / 128 threads stage each row of a tile (a part of the row each);
 // in the softmax and the O update, warp w reads TMEM lanes 32 (w % 4) .. + 31 and the
-// columns of head part w / 4. 16 padded heads run 128 threads at three CTAs per SM, 32
-// heads 256 threads at two (shared memory holds two of those).
+// columns of head part w / 4. 16 padded heads run 128 threads at four CTAs per SM (a
+// window tile's values then follow its keys through one buffer), 32 heads 256 threads at
+// two (shared memory holds two of those).
 // Global rows are dequantised to bf16 (code times scale has at most seven significant
 // bits, so bf16 holds it exactly) and Q is bf16 for both kinds of tile.
 template <int HQP>
 struct __align__(1024) AttnSeqSmem {
     uint8_t kbuf[2 * kPanelBytes];      // key tile (also the value tile of a global tile)
-    uint8_t vbuf[2 * kPanelBytes];      // value tile of a window tile
+    // value tile of a window tile; at 16 heads the key buffer takes it once S has read the
+    // keys (1 KB here keeps the operands below 1024-byte aligned)
+    uint8_t vbuf[HQP == 16 ? 1024 : 2 * kPanelBytes];
     uint8_t qbuf[2 * HQP * 128];        // queries, [HQP rows x D] in 64-element panels
     uint8_t pbuf[2 * HQP * 128];        // probabilities, [HQP rows x 128 keys] in 64-key panels
     float red_m[4][HQP], red_l[4][HQP];
@@ -915,10 +918,13 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[HH]) {
     }
 }
 
+static_assert(offsetof(AttnSeqSmem<16>, qbuf) % 1024 == 0 && offsetof(AttnSeqSmem<32>, qbuf) % 1024 == 0,
+              "operand alignment");
+
 template <int HQP> constexpr int seq_threads() { return HQP == 16 ? 128 : 256; }
 
 template <int HQP, int D, int NT = seq_threads<HQP>()>
-__global__ void __launch_bounds__(NT, NT == 128 && HQP == 16 ? 3 : 2)
+__global__ void __launch_bounds__(NT, NT == 128 && HQP == 16 ? 4 : 2)
     sparse_attn_seq_kernel(const __grid_constant__ AttnParams p) {
     CSA2_TRACE_INIT();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -962,7 +968,7 @@ __global__ void __launch_bounds__(NT, NT == 128 && HQP == 16 ? 3 : 2)
     if (D == 64) {
         for (int i = tid; i < kPanelBytes / 16; i += NT) {
             reinterpret_cast<uint4*>(S.kbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4*>(S.vbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
+            if constexpr (HQP != 16) reinterpret_cast<uint4*>(S.vbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
         }
     }
     float o[HH];   // this thread's row of O^T (head dimension 32 * quarter + lane), heads hh0 ..
@@ -1061,7 +1067,7 @@ __global__ void __launch_bounds__(NT, NT == 128 && HQP == 16 ? 3 : 2)
                     if (okr) {
                         const size_t off = ((size_t)b * p.Lloc + lrow) * CPR + c;
                         kv[jb] = __ldg(kls + off);
-                        vv[jb] = __ldg(vls + off);
+                        if constexpr (HQP != 16) vv[jb] = __ldg(vls + off);
                     }
                 }
 #pragma unroll
@@ -1070,7 +1076,7 @@ __global__ void __launch_bounds__(NT, NT == 128 && HQP == 16 ? 3 : 2)
                     const int rr = i / CPR, c = i % CPR;
                     const uint32_t dst = (c >> 3) * kPanelBytes + sw128(rr, c & 7);
                     *reinterpret_cast<uint4*>(S.kbuf + dst) = kv[jb];
-                    *reinterpret_cast<uint4*>(S.vbuf + dst) = vv[jb];
+                    if constexpr (HQP != 16) *reinterpret_cast<uint4*>(S.vbuf + dst) = vv[jb];
                 }
             }
         }
@@ -1101,6 +1107,31 @@ __global__ void __launch_bounds__(NT, NT == 128 && HQP == 16 ? 3 : 2)
         }
         ok = ok && mbar_wait(&S.bar_s, (uint32_t)(tau & 1), p.status, 13);
         tc_fence_after();
+        if constexpr (HQP == 16) {
+            if (!global_tile) {   // the window tile's values go into the key buffer, which S has read
+                const int p0 = lo_w + (tau - p.ngt) * kTileKeys;
+                const uint4* vls = reinterpret_cast<const uint4*>(p.vl);
+                constexpr int CPR = D / 8, ITERS = kTileKeys * CPR / NT, BATCH = ITERS < 8 ? ITERS : 8;
+#pragma unroll
+                for (int i0 = 0; i0 < ITERS; i0 += BATCH) {
+                    uint4 vv[BATCH];
+#pragma unroll
+                    for (int jb = 0; jb < BATCH; ++jb) {
+                        const int i = tid + (i0 + jb) * NT;
+                        const int rr = i / CPR, c = i % CPR;
+                        const int pr = p0 + rr, lrow = pr - base;
+                        const bool okr = (t >= 0) && (p.W > 0) && (pr <= t) && lrow >= 0 && lrow < p.Lloc;
+                        vv[jb] = okr ? __ldg(vls + ((size_t)b * p.Lloc + lrow) * CPR + c) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int jb = 0; jb < BATCH; ++jb) {
+                        const int i = tid + (i0 + jb) * NT;
+                        const int rr = i / CPR, c = i % CPR;
+                        *reinterpret_cast<uint4*>(S.kbuf + (c >> 3) * kPanelBytes + sw128(rr, c & 7)) = vv[jb];
+                    }
+                }
+            }
+        }
         if (tslot) { CSA2_TRACE(tslot + 1); }   // S done
 
         // ---- online softmax: the tile's maximum per head, then P and the tile's sums
@@ -1150,7 +1181,7 @@ __global__ void __launch_bounds__(NT, NT == 128 && HQP == 16 ? 3 : 2)
 
         // ---- O_tile^T = V^T P  (M = 128 = head dim (padded), N = HQP, K = 128 keys)
         if (tid == 0 && ok) {
-            const uint32_t va = smem_u32(global_tile ? S.kbuf : S.vbuf), pa = smem_u32(S.pbuf);
+            const uint32_t va = smem_u32((global_tile || HQP == 16) ? S.kbuf : S.vbuf), pa = smem_u32(S.pbuf);
             constexpr uint32_t idesc = idesc_bf16(128, HQP, 1);
 #pragma unroll
             for (int kk = 0; kk < kTileKeys / 16; ++kk) {
