@@ -58,7 +58,10 @@ struct AttnParams {
 template <int HQP>
 struct __align__(1024) AttnSmem {
     uint8_t kbuf[2 * kPanelBytes];      // key tile (also the value tile of a global tile)
-    uint8_t vbuf[2 * kPanelBytes];      // value tile of a local tile
+    // value tile of a local tile, and the merge's tile sums; at 16 heads the key buffer takes
+    // the values once S has read the keys, and 9 KB hold the sums of up to 144 tiles (a
+    // multiple of 1024 bytes keeps the operands below aligned)
+    uint8_t vbuf[HQP == 16 ? 9216 : 2 * kPanelBytes];
     uint8_t qbuf[2 * HQP * 128];        // queries, [HQP rows x D] in 64-element panels
     uint8_t pbuf[2 * HQP * 128];        // probabilities, [HQP rows x 128 keys] in 64-key panels
     float red[4][HQP];
@@ -66,6 +69,8 @@ struct __align__(1024) AttnSmem {
     uint32_t tmem_base;
     int is_last;
 };
+static_assert(offsetof(AttnSmem<16>, qbuf) % 1024 == 0 && offsetof(AttnSmem<32>, qbuf) % 1024 == 0,
+              "operand alignment");
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
@@ -190,7 +195,7 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
     if (D == 64) {   // second M-half of the value operand stays zero
         for (int i = tid; i < kPanelBytes / 16; i += kAttnThreads) {
             reinterpret_cast<uint4*>(S.kbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4*>(S.vbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
+            if constexpr (HQP != 16) reinterpret_cast<uint4*>(S.vbuf + kPanelBytes)[i] = make_uint4(0, 0, 0, 0);
         }
     }
     __syncthreads();
@@ -273,7 +278,7 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
                 if (ok) {
                     const size_t off = ((size_t)b * p.Lloc + lrow) * CPR + c;
                     kv[j] = __ldg(kls + off);
-                    vv[j] = __ldg(vls + off);
+                    if constexpr (HQP != 16) vv[j] = __ldg(vls + off);
                 }
             }
 #pragma unroll
@@ -282,7 +287,7 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
                 const int rr = i / CPR, c = i % CPR;
                 const uint32_t dst = (c >> 3) * kPanelBytes + sw128(rr, c & 7);
                 *reinterpret_cast<uint4*>(S.kbuf + dst) = kv[j];
-                *reinterpret_cast<uint4*>(S.vbuf + dst) = vv[j];
+                if constexpr (HQP != 16) *reinterpret_cast<uint4*>(S.vbuf + dst) = vv[j];
             }
         }
     }
@@ -308,6 +313,32 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
     }
     bool ok = mbar_wait(&S.bar_s, 0, p.status, 10);
     tc_fence_after();
+    if constexpr (HQP == 16) {
+        if (!global_tile) {   // the local tile's values go into the key buffer, which S has read
+            const int lo = max(max(base, t - p.W + 1), 0);
+            const int p0 = lo + (tau - p.ngt) * kTileKeys;
+            const uint4* vls = reinterpret_cast<const uint4*>(p.vl);
+            constexpr int CPR = D / 8, ITERS = kTileKeys * CPR / kAttnThreads, BATCH = ITERS < 8 ? ITERS : 8;
+#pragma unroll
+            for (int i0 = 0; i0 < ITERS; i0 += BATCH) {
+                uint4 vv[BATCH];
+#pragma unroll
+                for (int j = 0; j < BATCH; ++j) {
+                    const int i = tid + (i0 + j) * kAttnThreads;
+                    const int rr = i / CPR, c = i % CPR;
+                    const int pr = p0 + rr, lrow = pr - base;
+                    const bool okr = (t >= 0) && (p.W > 0) && (pr <= t) && lrow >= 0 && lrow < p.Lloc;
+                    vv[j] = okr ? __ldg(vls + ((size_t)b * p.Lloc + lrow) * CPR + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int j = 0; j < BATCH; ++j) {
+                    const int i = tid + (i0 + j) * kAttnThreads;
+                    const int rr = i / CPR, c = i % CPR;
+                    *reinterpret_cast<uint4*>(S.kbuf + (c >> 3) * kPanelBytes + sw128(rr, c & 7)) = vv[j];
+                }
+            }
+        }
+    }
 
     // ---- tile softmax partial
     float sv[HQP];
@@ -366,7 +397,7 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
 
     // ---- O^T = V^T P  (M = 128 = head dim (padded), N = HQP, K = 128 keys)
     if (tid == 0 && ok) {
-        const uint32_t va = smem_u32(global_tile ? S.kbuf : S.vbuf), pa = smem_u32(S.pbuf);
+        const uint32_t va = smem_u32((global_tile || HQP == 16) ? S.kbuf : S.vbuf), pa = smem_u32(S.pbuf);
         constexpr uint32_t idesc = idesc_bf16(128, HQP, 1);
 #pragma unroll
         for (int kk = 0; kk < kTileKeys / 16; ++kk) {
@@ -415,8 +446,8 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const __grid_
         __threadfence();
         const float* pu = p.part + (size_t)u * p.ntiles * (HQP * (D + 2));
         const size_t stride = HQP * (D + 2);
-        // (k + W <= 16384 gives at most 129 tiles: up to 256 fit each buffer)
-        const int nt = CSA2_CHECK(p.ntiles * HQP * 4 <= (int)sizeof(S.kbuf), p.status, 2104) ? p.ntiles : 0;
+        // (k + W <= 16384 gives at most 129 tiles: each buffer holds at least 144)
+        const int nt = CSA2_CHECK(p.ntiles * HQP * 4 <= (int)sizeof(S.vbuf), p.status, 2104) ? p.ntiles : 0;
         float* wgt = reinterpret_cast<float*>(S.kbuf);             // [nt][HQP]
         float* lsum = reinterpret_cast<float*>(S.vbuf);            // [nt][HQP] tile sums
         float* Mh = S.red[0];                                      // [HQP]
