@@ -30,8 +30,7 @@ size_t index_region_bytes();
 size_t index_scratch_bytes(const csa2_index_args& a, int P_in);
 size_t index_smem_bytes();
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
-                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready,
-                         const csa2_index_args* rx);
+                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready);
 // attention.cu
 size_t attn_scratch_bytes(const csa2_attn_args& a);
 csa2_status launch_attn(const csa2_attn_args& a, const int32_t* topk, int* tickets, void* scratch,
@@ -219,7 +218,7 @@ csa2_status csa2_index_topk(const csa2_index_args* args, void* workspace, size_t
     void* scratch = ws_at(workspace, R + tickets_bytes(args->B * args->Tq));
     const int P_in = args->mode == CSA2_REINDEX ? args->P_in : 0;
     return launch_index(*args, args->pool_in, P_in, workspace, scratch, d_status, static_cast<cudaStream_t>(stream),
-                        nullptr, 0, nullptr);
+                        nullptr, 0);
 }
 
 csa2_status csa2_sparse_attn(const csa2_attn_args* args, void* workspace, size_t ws_bytes, int32_t* d_status,
@@ -264,14 +263,7 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
         // attention, which writes no key, position or pool: those were complete when it began.
         const int keys_ready = l > 0 ? 1 : 0;
         if (ix.mode == CSA2_FULL) {
-            // the Reindex layer (if any) that rescores this layer's pool: its key rows of the
-            // pool entries are pulled into L2 as the pool is written
-            const csa2_index_args* rx = nullptr;
-            for (int l2 = l + 1; ix.P > 0 && l2 < s->L && rx == nullptr; ++l2) {
-                if (s->idx[l2].mode == CSA2_FULL && s->idx[l2].P > 0) break;
-                if (s->idx[l2].mode == CSA2_REINDEX) rx = &s->idx[l2];
-            }
-            st = launch_index(ix, nullptr, 0, workspace, scratch, d_status, strm, &s->attn[l], keys_ready, rx);
+            st = launch_index(ix, nullptr, 0, workspace, scratch, d_status, strm, &s->attn[l], keys_ready);
             if (st != CSA2_OK) return st;
             cur = ix.topk_out;
             cur_k = ix.k;
@@ -280,7 +272,7 @@ csa2_status csa2_layer_stack(const csa2_stack_args* s, void* workspace, size_t w
                 pool_P = ix.P;
             }
         } else if (ix.mode == CSA2_REINDEX) {
-            st = launch_index(ix, pool, pool_P, workspace, scratch, d_status, strm, &s->attn[l], keys_ready, nullptr);
+            st = launch_index(ix, pool, pool_P, workspace, scratch, d_status, strm, &s->attn[l], keys_ready);
             if (st != CSA2_OK) return st;
             cur = ix.topk_out;
             cur_k = ix.k;

@@ -100,11 +100,6 @@ struct IdxParams {
     const uint8_t* pf_fp4;
     const uint8_t* pf_scale;
     int pf_N, pf_code_bytes, pf_scale_bytes;
-    // L2 prefetch of the index-key rows of the pool entries, for the Reindex layer that
-    // rescores this pool (pk_keys nullptr: off)
-    const int8_t* pk_keys;
-    int64_t pk_seq_stride;
-    int pk_row_bytes;
     int m;                   // sequence compression rate of the global entries (<= 1: one per position)
     long long wait_budget;   // SM cycles a CTA waits at a group barrier before it reports a timeout
     int skip_arrival;        // fault injection: the last CTA of a group never arrives at its first barrier
@@ -919,16 +914,10 @@ struct RowPrefetch {
     const uint8_t* fp4;     // the sequence's codes [N][code_bytes]
     const uint8_t* scale;   // the sequence's scales [N][scale_bytes]
     int code_bytes, scale_bytes;
-    const int8_t* keys;     // the sequence's index keys of the Reindex layer that rescores the pool
-    int key_bytes;
 };
 
 __device__ __forceinline__ RowPrefetch row_prefetch(const IdxParams& p, int u) {
-    RowPrefetch f{nullptr, nullptr, 0, 0, nullptr, 0};
-    if (p.pk_keys != nullptr) {
-        f.keys = p.pk_keys + (size_t)(u / p.Tq) * p.pk_seq_stride;
-        f.key_bytes = p.pk_row_bytes;
-    }
+    RowPrefetch f{nullptr, nullptr, 0, 0};
     if (p.pf_fp4 != nullptr) {
         const size_t b = (size_t)(u / p.Tq);
         f.fp4 = p.pf_fp4 + b * p.pf_N * p.pf_code_bytes;
@@ -943,11 +932,6 @@ __device__ __forceinline__ void prefetch_row(const RowPrefetch& f, int pos) {
     if (f.fp4 == nullptr || pos < 0) return;
     asm volatile("prefetch.global.L2 [%0];" ::"l"(f.fp4 + (size_t)pos * f.code_bytes));
     asm volatile("prefetch.global.L2 [%0];" ::"l"(f.scale + (size_t)pos * f.scale_bytes));
-}
-
-__device__ __forceinline__ void prefetch_key(const RowPrefetch& f, int pos) {
-    if (f.keys == nullptr || pos < 0) return;
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(f.keys + (size_t)pos * f.key_bytes));
 }
 
 __device__ __forceinline__ void take_flags(int x, bool ok, const ListCut& c, bool& g, bool& e) {
@@ -1000,7 +984,7 @@ __device__ __forceinline__ void write_lists(const int* sc, int n, int base, cons
         const bool t0 = g0 || (q0 && oq0 < c0.quota), t1 = g1 || (q1 && oq1 < c1.quota);
         if (t0 || t1) {
             const int pos = pool ? pool[base + e] : base + e;
-            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) { c0.out[k] = pos; prefetch_key(pf, pos); } }
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) { c0.out[k] = pos; } }
             if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c1.r, c1.status, 2202)) { c1.out[k] = pos; prefetch_row(pf, pos); } }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
@@ -1058,7 +1042,7 @@ __device__ __forceinline__ void write_from_lists(const int* sc, int base, const 
         if (t0 || t1) {
             const int e = base + (ent & 0x0FFFFFFF);
             const int pos = pool ? pool[e] : e;
-            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) { c0.out[k] = pos; prefetch_key(pf, pos); } }
+            if (t0) { const int k = c0.base + og0 + min(oq0, c0.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c0.r, c0.status, 2201)) { c0.out[k] = pos; } }
             if (t1) { const int k = c1.base + og1 + min(oq1, c1.quota); if (CSA2_GUARD((unsigned)k < (unsigned)c1.r, c1.status, 2202)) { c1.out[k] = pos; prefetch_row(pf, pos); } }
         }
         rg0 += __popc(bg0); re0 += __popc(bq0); rg1 += __popc(bg1); re1 += __popc(bq1);
@@ -2873,8 +2857,7 @@ static cudaError_t launch_mq_steps(const csa2_index_args& a, const IdxPlan& pl, 
 
 // Launch one indexer call. `ws` holds plan_index(a).ws_bytes bytes (zero at first use).
 csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P_in, void* region, void* scratch,
-                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready,
-                         const csa2_index_args* rx) {
+                         int32_t* d_status, cudaStream_t stream, const csa2_attn_args* pf, int keys_ready) {
     const int sms = num_sms();
     csa2_index_args aa = a;
     aa.P_in = P_in;
@@ -2910,11 +2893,6 @@ csa2_status launch_index(const csa2_index_args& a, const int32_t* pool_in, int P
         p.pf_scale_bytes = pf->D / 16;
     }
     p.keys_ready = keys_ready;
-    if (a.mode == CSA2_FULL && a.P > 0 && rx != nullptr && rx->ki != nullptr && rx->B == a.B) {
-        p.pk_keys = rx->ki;
-        p.pk_seq_stride = rx->ki_seq_stride;
-        p.pk_row_bytes = rx->Di;
-    }
     p.m = a.m;
     p.status = d_status;
     p.wait_budget = group_wait_budget();
