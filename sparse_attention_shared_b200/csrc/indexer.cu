@@ -134,6 +134,8 @@ constexpr int kHistlOff = 2 * (int)sizeof(int2) * kCandCap;   // byte offset of 
 constexpr int kListOff = kHistlOff + 2 * kBins * 4;            // byte offset of the per-warp ordered lists
 constexpr int kListCap = 512;                                  // entries per warp
 static_assert(kListOff + kSelWarps * kListCap * 4 <= (int)sizeof(((IdxSmem*)0)->stage), "select buffers");
+// (a Reindex pool cut in one select per group has at most kSmemScores entries over G >= 2 CTAs)
+static_assert(kSelWarps * kListCap >= kSmemScores / 2, "a Reindex chunk's positions fit the list region");
 static_assert(kStages * kStageBytes % 1024 == 0, "tensor-core operand alignment");
 static_assert(sizeof(IdxSmem) + 1024 <= 232448, "shared memory per block");
 
@@ -1469,8 +1471,10 @@ __device__ __forceinline__ bool reindex_local_unit(const IdxParams& p, IdxSmem& 
         }
     }
     CSA2_TRACE(7);   // offsets
+    // the chunk's pool positions sit in the list region (stored as its rows were gathered;
+    // the candidates and the radix histogram above lie below it)
     if (c.my_n > 0)
-        write_lists<false>(S.sc + c.lo, c.my_n, c.lo, c.pool, none, cut, S.wsum, row_prefetch(p, c.u));
+        write_lists<false>(S.sc + c.lo, c.my_n, 0, wlists(S), none, cut, S.wsum, row_prefetch(p, c.u));
     if (c.cta == p.G - 1) {
 #pragma unroll 1
         for (int i = min(r, n) + tid; i < r; i += kSel) cut.out[i] = -1;
@@ -2454,6 +2458,7 @@ __global__ void __launch_bounds__(kSel, 1)
             const int8_t* kb = p.ki + (size_t)b * p.ki_seq_stride;
             constexpr int kCh = DI > 0 ? DI / 16 : 8;   // 16-byte chunks per key row
             int first_bad = my_n;
+            int* lpos = p.local_sel ? wlists(S) : nullptr;   // the chunk's positions, for the ordered write
             if constexpr (kQuad) {
                 // lane l of a quad holds chunk l % 4 of its row: one load instruction of a
                 // warp covers 8 rows (8 lines instead of 32). Each lane's partial dot products
@@ -2483,6 +2488,7 @@ __global__ void __launch_bounds__(kSel, 1)
                         if (e < my_n && !okr[rd]) first_bad = min(first_bad, e);
                         kv[rd] = okr[rd] ? __ldg(reinterpret_cast<const int4*>(kb + (size_t)sidx[rd] * 64) + sub)
                                          : make_int4(0, 0, 0, 0);
+                        if (lpos != nullptr && sub == 0 && okr[rd]) lpos[e] = sidx[rd];
                     }
 #pragma unroll
                     for (int rd = 0; rd < kQuadRounds; ++rd) {
@@ -2526,6 +2532,7 @@ __global__ void __launch_bounds__(kSel, 1)
                     const int e = e0 + q2 * kSel + tid;
                     sidx[q2] = (e0 == 0) ? sidx0[q2] : ((e < my_n) ? __ldg(pool + lo + e) : -1);
                     okr[q2] = e < my_n && sidx[q2] >= 0 && sidx[q2] <= tg;
+                    if (lpos != nullptr && okr[q2]) lpos[e] = sidx[q2];
                     if (e < my_n && !okr[q2]) first_bad = min(first_bad, e);
                     if (okr[q2]) {
                         const int4* row = reinterpret_cast<const int4*>(kb + (size_t)sidx[q2] * p.Di);
