@@ -134,6 +134,30 @@ def test_reindex_paths(B, N, Hi, Di, P, k, extreme, ws, status):
         assert set(got[b, 0].tolist()) - {-1} <= set(rp[b, 0].tolist()), "Reindex list outside the pool"
 
 
+@pytest.mark.parametrize("Hi,Di", [(8, 64), (4, 32), (12, 64)])
+def test_reindex_padded_pools(Hi, Di, ws, status):
+    """Queries early in their sequences: the Full pools hold fewer valid entries than P
+    (-1 after them), and the valid prefix ends inside a CTA's chunk (4 CTAs of 1024
+    entries a query), at a chunk's end, or inside the first chunk; one query's prefix is
+    shorter than k, so its list ends in -1. Each of the three Reindex scoring forms
+    (<8,64>, <4,32>, generic) writes its chunk's positions from its own staging."""
+    B, N, P, k = 4, 12000, 4096, 1024
+    qi, w, ki = inputs(31 * Hi + Di, B, 1, N, Hi, Di, True)
+    q_pos = np.array([[N - 1], [2500], [3071], [700]], np.int32)   # valid pool entries: 4096, 2501, 3072, 701
+    pool, _ = check_full(qi, w, ki, q_pos, k, P, ws, status)
+    rp = pool.cpu().numpy()
+    for b, n_valid in enumerate([4096, 2501, 3072, 701]):
+        assert (rp[b, 0, :n_valid] >= 0).all() and (rp[b, 0, n_valid:] == -1).all()
+    qi2, w2, ki2 = inputs(31 * Hi + Di + 1, B, 1, N, Hi, Di, True)
+    _, topk = ops.index_topk("REINDEX", dev(q_pos), dev(qi2), w2, dev(ki2), k, pool_in=pool, ws=ws, status=status)
+    status.check("reindex, padded pools")
+    ref = np.stack([[O.index_reindex(qi2[b, 0], w2, ki2[b], rp[b, 0], k)] for b in range(B)])
+    got = topk.cpu().numpy()
+    assert_list_invariants(got, q_pos, "reindex topk")
+    assert_lists_equal(topk, ref, "reindex topk, padded pools")
+    assert (got[3, 0, 701:] == -1).all() and (got[3, 0, :701] >= 0).all()
+
+
 def test_weights_past_the_bound_are_rejected(ws):
     """One weight above the header's bound: the size query returns 0 and the call
     returns CSA2_ERR_RANGE before launching anything."""
