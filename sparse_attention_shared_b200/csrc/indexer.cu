@@ -2666,16 +2666,20 @@ IdxPlan plan_index(const csa2_index_args& a, int sms) {
     IdxPlan pl{};
     pl.units = a.B * a.Tq;
     const int n_max = (a.mode == CSA2_FULL) ? a.N : a.P_in;
+    // A Reindex pool that one CTA's shared memory holds is cut without the distributed select,
+    // whose 64-element steps want 256-aligned chunks: its groups take chunks down to 512 entries.
+    const bool rx_small = a.mode == CSA2_REINDEX && a.P_in <= kSmemScores;
+    const int min_chunk = rx_small ? 512 : 1024;
     if (pl.units >= sms) {
         pl.G = 1;
         pl.groups = sms;
     } else {
         pl.groups = pl.units;
         pl.G = std::max(1, std::min(kMaxG, sms / pl.units));
-        pl.G = std::max(1, std::min(pl.G, (n_max + 1023) / 1024));
+        pl.G = std::max(1, std::min(pl.G, (n_max + min_chunk - 1) / min_chunk));
     }
     int chunk = (n_max + pl.G - 1) / pl.G;
-    chunk = (int)align_up((size_t)std::max(chunk, 1), 256);
+    chunk = (int)align_up((size_t)std::max(chunk, 1), rx_small ? 64 : 256);
     pl.chunk = chunk;
     pl.spill_bytes = 0;
     // (+ 512 bytes: the select's 64-element steps may read up to 63 elements past a chunk's end)
