@@ -113,6 +113,8 @@ REINDEX_CASES = [
     (2, 9000, 12, 64, 2048, 500, True),         # generic (Hi > 8)
     (2, 6000, 5, 96, 1500, 200, True),          # generic (Di = 96)
     (2, 40000, 8, 64, 20000, 2048, True),       # pool larger than one CTA's shared memory: distributed select
+    (2, 20000, 8, 64, 5000, 1500, True),        # <8,64>, ten CTAs a query of 512 entries, the last one ragged (392)
+    (1, 9000, 4, 32, 3000, 700, False),         # <4,32>, six CTAs, the last one 440 entries
 ]
 
 
