@@ -450,6 +450,12 @@ def test_stack20_128k_every_unit(ws, status):
     _check_stack_every_unit(synth.make_workload("stack20_128k"), ws, status)
 
 
+def test_paper_schedule_every_unit(ws, status):
+    # the pages' own schedule at full size: [Full + 3 Reuse] + 4 x [Reindex + 3 Reuse] on one shared key set,
+    # pool 2048 and top-512 (the Reindex groups take four CTAs of 512 pool entries a query), SWA 128
+    _check_stack_every_unit(synth.make_workload("paper_schedule"), ws, status)
+
+
 def test_encoder_m2_shared_keys_every_unit(ws, status):
     # compression rate 2 with 8 queries a sequence: the shared-key Full path reads entries up to each
     # query's last one ((t + 1) / 2 - 1), then Reuse and Reindex layers
